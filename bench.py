@@ -1,0 +1,435 @@
+"""Benchmark of the QSA hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl qsa|reference] [--no-decode] [--no-e2e]
+
+One step = the whole hot path over one batch of synthetic input:
+  prefill (the headline, 131072 tokens, 16 q / 2 KV heads, D 128, 4x64 indexer, k 512 + own block):
+    pool indexer keys -> score + top-k (chunked scores in a workspace) -> gather-sparse attention;
+  decode (second leg, 32 sequences x 262144-token caches, k 512): pool the newest block ->
+    score + top-k over the pooled-key cache -> split-KV sparse attention + merge.
+Inputs are resident in HBM when the timed region starts and are larger than L2 (126 MB), so no L2
+flush is done between steps.  Times are CUDA events on the launching stream, max over ranks.
+With N > 1 every rank runs its own workload (different seed; no data-path collective), so the
+scaling is weak.  ``--impl reference`` times the CPU oracle on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from hybrid_sparse_attention_qsa_b200 import inputs as I  # noqa: E402
+
+METRIC = "QSA prefill tokens/s @128K and decode tokens/s @256K ctx; % of roofline"
+PREFILL = "prefill_128k"
+DECODE = "decode_256k"
+
+
+# ------------------------------------------------------------------------------------------- helpers
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm_gbs=p["hbm_gbs"], bf16_tflops=p["bf16_tflops"],
+                    bf16_tflops_sustained=p.get("bf16_tflops_sustained", p["bf16_tflops"]), source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+def tokens_attended(T: int, k: int, blk: int = 4) -> np.ndarray:
+    """|S(t)| = blk * min(t // blk, k) + t % blk + 1 for t = 0 .. T-1."""
+    t = np.arange(T, dtype=np.int64)
+    return blk * np.minimum(t // blk, k) + t % blk + 1
+
+
+def prefill_work(w) -> dict:
+    """Algorithmic work of one prefill step (per batch element times B)."""
+    S = tokens_attended(w.T, w.k, w.blk)
+    gathered = int(S.sum()) * w.Hkv * w.D * 2 * 2            # K and V bytes gathered
+    qo = w.T * w.Hq * w.D * 2 * 2                             # q read + o written
+    attn_bytes = (gathered + qo) * w.B
+    attn_flops = int(S.sum()) * w.Hq * 4 * w.D * w.B
+    pairs = int((np.arange(w.T) // w.blk).sum())             # causally visible (t, block) pairs
+    idx_flops = pairs * 2 * w.Hi * w.Di * w.B
+    return dict(attn_bytes=attn_bytes, attn_flops=attn_flops, index_flops=idx_flops, pairs=pairs * w.B)
+
+
+def decode_work(w) -> dict:
+    nb = (w.T - 1) // w.blk
+    S = w.blk * min(nb, w.k) + (w.T - 1) % w.blk + 1
+    kp_bytes = nb * w.Di * 2
+    gathered = S * w.Hkv * w.D * 2 * 2
+    qo = w.Hq * w.D * 2 * 2 + w.Hi * w.Di * 2
+    return dict(bytes=(kp_bytes + gathered + qo) * w.B, kp_bytes=kp_bytes * w.B, gathered=gathered * w.B)
+
+
+class Clocks:
+    """nvidia-smi sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200", "-f", self.path],
+                                         stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return None
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+# ------------------------------------------------------------------------------------------- CPU oracle
+def oracle_sample(w, n_rows: int, host: dict | None = None, seed: int = 0):
+    """Time the oracle (as it stands) on n_rows query rows spread over the workload.  Returns
+    (seconds, rows, threads)."""
+    import oracle as O
+    if host is None:
+        x = I.make_prefill(w, "cpu")
+        host = {n: I.bits(x[n]) for n in x}
+    t0 = time.perf_counter()
+    kp = O.pool_block_keys(host["ki"], blk=w.blk)
+    rows = np.unique(np.linspace(0, w.T - 1, n_rows).astype(np.int64))
+    O.prefill_rows(host["q"], host["k"], host["v"], host["qi"], kp, [(0, int(t)) for t in rows], topk=w.k, blk=w.blk)
+    dt = time.perf_counter() - t0
+    return dt, len(rows), O.hardware_threads()
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = I.WORKLOADS[PREFILL]
+    x = I.make_prefill(w, "cpu")
+    host = {n: I.bits(x[n]) for n in x}
+    del x
+    n_rows = args.ref_rows
+    for _ in range(args.warmup):
+        oracle_sample(w, n_rows, host)
+    times = []
+    for _ in range(args.steps):
+        dt, rows, cores = oracle_sample(w, n_rows, host)
+        times.append(dt)
+    total = sum(times)
+    value = rows * args.steps / total
+    sample = f"{rows} query rows spread evenly over the {w.T}-token prefill (pooling of all keys included)"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * total / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": PREFILL, "B": w.B, "T": w.T, "Hq": w.Hq, "Hkv": w.Hkv,
+                                              "D": w.D, "Hi": w.Hi, "Di": w.Di, "blk": w.blk, "k": w.k},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------------------------------- GPU arm
+def select_launches(w, ws_bytes: int) -> int:
+    """Kernels qsa_select_topk launches for a prefill with a scores workspace of ws_bytes."""
+    nbk = w.T // w.blk
+    R = max(1, ws_bytes // (nbk * 4))
+    n = 0
+    for r0 in range(0, w.T, R):
+        rows = min(R, w.T - r0)
+        if min(nbk, (r0 + rows - 1) // w.blk) > 0:
+            n += 1          # score kernel
+        n += 1              # top-k kernel
+    return n * w.B
+
+
+def run_qsa(args):
+    import hybrid_sparse_attention_qsa_b200 as Q
+
+    world, rank, local = dist_setup()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    pk = peaks()
+    stream = torch.cuda.current_stream(dev)
+
+    # ---------------------------------------------------------------- prefill (headline)
+    w = I.WORKLOADS[args.workload].with_(seed=I.WORKLOADS[args.workload].seed + 1000 * rank)
+    x = I.make_prefill(w, dev)
+    nbk = w.T // w.blk
+    ws_bytes = Q.qsa_workspace_size(Q.qsa.QSA_OP_SELECT_TOPK, w.B, w.T, nbk, w.k, w.Hq, w.D)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    kp = torch.empty(w.B, nbk, w.Di, dtype=torch.bfloat16, device=dev)
+    idx = torch.empty(w.B, w.T, w.k, dtype=torch.int32, device=dev)
+    out = torch.empty_like(x["q"])
+    lse = torch.empty(w.B, w.T, w.Hq, dtype=torch.float32, device=dev)
+
+    def step(ev=None):
+        Q.qsa_pool_block_keys(x["ki"], kp)
+        if ev:
+            ev[0].record(stream)
+        Q.qsa_select_topk(w.k, qi=x["qi"], kp=kp, idx=idx, workspace=ws)
+        if ev:
+            ev[1].record(stream)
+        Q.qsa_sparse_attn_prefill(x["q"], x["k"], x["v"], idx, out=out, lse=lse)
+        if ev:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert Q.qsa_get_device_status() == 0
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with Clocks(local) as clk:
+        t0.record(stream)
+        for s in range(args.steps):
+            step(evs[s])
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    clocks = clk.summary()
+    ms_total = max_over_ranks(t0.elapsed_time(t1), world, dev)
+    ms_step = ms_total / args.steps
+    ms_select = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    ms_attn = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    value = world * w.B * w.T / (ms_step / 1000)
+    work = prefill_work(w)
+    attn_gbs = work["attn_bytes"] / (ms_attn / 1000) / 1e9
+    launches = (1 + select_launches(w, ws_bytes) + 1) * args.steps
+
+    # indexer alone (scores for all rows materialised once; untimed in the step above)
+    idx_ms = None
+    try:
+        if args.no_indexer:
+            raise torch.OutOfMemoryError("skipped")
+        scores = torch.empty(w.B, w.T, nbk, dtype=torch.float32, device=dev)
+        Q.qsa_index_score(x["qi"], kp, scores=scores)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 3
+        e0.record(stream)
+        for _ in range(reps):
+            Q.qsa_index_score(x["qi"], kp, scores=scores)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        idx_ms = e0.elapsed_time(e1) / reps
+        del scores
+    except torch.OutOfMemoryError:
+        pass
+
+    # end to end through the public API from pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        host = {n: torch.empty_like(x[n], device="cpu").pin_memory() for n in ("q", "k", "v", "qi", "ki")}
+        for n in host:
+            host[n].copy_(x[n])
+        hout = torch.empty_like(out, device="cpu").pin_memory()
+        dx = {n: torch.empty_like(x[n]) for n in host}
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = hout.numel() * hout.element_size()
+
+        def e2e_step():
+            for n in host:
+                dx[n].copy_(host[n], non_blocking=True)
+            r = Q.prefill(dx["q"], dx["k"], dx["v"], dx["qi"], dx["ki"], topk=w.k, workspace=ws)
+            hout.copy_(r["out"], non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        a0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        a1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(a0.elapsed_time(a1), world, dev) / args.e2e_steps
+        e2e = {"value": world * w.B * w.T / (e2e_ms / 1000), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+        del host, hout, dx
+    del x, ws, idx, out, lse, kp
+    torch.cuda.empty_cache()
+
+    # ---------------------------------------------------------------- decode leg
+    decode = None
+    if not args.no_decode:
+        wd = I.WORKLOADS[DECODE].with_(seed=I.WORKLOADS[DECODE].seed + 1000 * rank)
+        xd = I.make_decode(wd, dev)
+        nbd = wd.T // wd.blk
+        kpd = Q.qsa_pool_block_keys(xd["ki"])
+        wsd = torch.empty(Q.qsa_workspace_size(Q.qsa.QSA_OP_SELECT_TOPK, wd.B, 1, nbd, wd.k, wd.Hq, wd.D),
+                          dtype=torch.uint8, device=dev)
+        splits = Q.qsa.lib().qsa_decode_default_splits(wd.B, wd.k)
+        wsa = torch.empty(max(16, Q.qsa_workspace_size(Q.qsa.QSA_OP_SPARSE_ATTN_DECODE, wd.B, 1, 0, wd.k, wd.Hq, wd.D,
+                                                       splits)), dtype=torch.uint8, device=dev)
+        idxd = torch.empty(wd.B, wd.k, dtype=torch.int32, device=dev)
+        outd = torch.empty_like(xd["q"])
+        lsed = torch.empty(wd.B, wd.Hq, dtype=torch.float32, device=dev)
+        j = (wd.T - 1) // wd.blk          # the block holding the newest token
+        ki_last = xd["ki"][:, j * wd.blk:(j + 1) * wd.blk]
+        kp_last = kpd[:, j:j + 1]
+
+        def dstep():
+            if (wd.T % wd.blk) == 0:       # the new token completed block j: pool that row of every sequence
+                Q.qsa_pool_block_keys(ki_last, kp_last, pos0=j * wd.blk)
+            Q.qsa_select_topk(wd.k, qi=xd["qi"], kp=kpd, seqlens=xd["seqlens"], idx=idxd, workspace=wsd)
+            Q.qsa_sparse_attn_decode(xd["q"], xd["k"], xd["v"], xd["seqlens"], idxd, num_splits=splits, out=outd,
+                                     lse=lsed, workspace=wsa)
+
+        for _ in range(max(args.warmup, 3)):
+            dstep()
+        torch.cuda.synchronize()
+        assert Q.qsa_get_device_status() == 0
+        dsteps = args.decode_steps
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        d0.record(stream)
+        for _ in range(dsteps):
+            dstep()
+        d1.record(stream)
+        torch.cuda.synchronize()
+        dms = max_over_ranks(d0.elapsed_time(d1), world, dev) / dsteps
+        dw = decode_work(wd)
+        dgbs = dw["bytes"] / (dms / 1000) / 1e9
+        decode = {"workload": DECODE, "value": world * wd.B / (dms / 1000), "unit": "tokens/s", "ms_per_step": dms,
+                  "steps": dsteps, "num_splits": splits,
+                  "gpu_launches_per_step": 1 + 2 + 1 + (1 if splits > 1 else 0),
+                  "roofline": {"bound": "hbm", "achieved": dgbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                               "frac": dgbs / pk["hbm_gbs"], "bytes_per_step": dw["bytes"],
+                               "basis": "pooled-key cache read + gathered K/V of the selected tokens + q/o"}}
+        del xd, kpd, wsd, wsa, idxd, outd, lsed
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": args.workload, "B": w.B, "T": w.T, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "Hi": w.Hi,
+                       "Di": w.Di, "blk": w.blk, "k": w.k, "boost": f"{w.boost_frac:g} of keys x{w.boost:g}",
+                       "l2": "inputs larger than L2, no flush", "parallelism": f"independent replicas x{world}"},
+            "roofline": {"bound": "hbm", "kernel": "sparse_attn_kernel<2>", "achieved": attn_gbs,
+                         "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": attn_gbs / pk["hbm_gbs"],
+                         "traffic": None, "peak_source": pk["source"],
+                         "basis": "gathered K/V bytes of every selected token + q read + o write",
+                         "bytes_per_launch": work["attn_bytes"], "ms_per_launch": ms_attn},
+            "step_breakdown_ms": {"pool": None, "score_topk": ms_select, "attention": ms_attn},
+            "indexer": None if idx_ms is None else {
+                "ms": idx_ms, "flops": work["index_flops"], "tflops": work["index_flops"] / idx_ms / 1e9,
+                "frac_of_bf16_peak": work["index_flops"] / idx_ms / 1e9 / pk["bf16_tflops"],
+                "note": "scores for every row materialised in HBM (fp32), timed alone"},
+            "gpu_launches": launches,
+            "clocks": clocks,
+            "e2e": e2e,
+            "decode": decode,
+        }
+        if not args.no_cpu_baseline and world == 1:
+            dt, rows, cores = oracle_sample(I.WORKLOADS[args.workload], args.ref_rows)
+            line["cpu_baseline"] = {"value": rows / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                    "sample": f"{rows} query rows spread evenly over the {w.T}-token prefill, "
+                                              f"pooling of all keys included"}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="qsa", choices=["qsa", "reference"])
+    ap.add_argument("--decode-steps", type=int, default=50)
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--ref-rows", type=int, default=96)
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-indexer", action="store_true", help="skip the stand-alone indexer timing (17 GB of scores)")
+    ap.add_argument("--workload", default=PREFILL, choices=[n for n, w in I.WORKLOADS.items() if w.kind == "prefill"],
+                    help="prefill workload of the headline leg (default: the 128K configuration)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_qsa(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

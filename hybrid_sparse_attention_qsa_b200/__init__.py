@@ -1,1 +1,11 @@
-"""B200-native Qwen Sparse Attention (QSA) hot path: the C-ABI library and its Python binding."""
+"""B200-native Qwen Sparse Attention (QSA) hot path.
+
+``qsa`` is the ctypes binding of the C-ABI library ``libqsa_b200.so`` (declared in include/qsa.h);
+``inputs`` draws the seeded synthetic workloads.  The library is loaded on first use and there is
+no CPU fallback.
+"""
+from . import qsa  # noqa: F401
+from .qsa import (QSAError, decode, prefill, qsa_abi_version, qsa_get_device_status,  # noqa: F401
+                  qsa_index_score, qsa_pool_block_keys, qsa_rope_index_queries, qsa_select_topk,
+                  qsa_set_wait_timeout_ns, qsa_sparse_attn_decode, qsa_sparse_attn_prefill,
+                  qsa_wait_timeout_selftest, qsa_workspace_size)

@@ -1,0 +1,270 @@
+// The C ABI (include/qsa.h): argument checks on the host, then launches on the caller's stream.
+#include <algorithm>
+#include <atomic>
+#include <cstdint>
+#include <mutex>
+
+#include "launch.h"
+#include "qsa.h"
+
+namespace qsa {
+
+__device__ unsigned int g_status_word;   // one per device that loads the library
+
+namespace {
+constexpr int kMaxDevices = 64;
+constexpr unsigned long long kDefaultWaitNs = 2000000000ull;
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+bool g_dev_ok[kMaxDevices];
+std::atomic<unsigned long long> g_wait_ns{kDefaultWaitNs};
+
+__global__ void wait_selftest_kernel(KernelCtl ctl) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, ctl);   // nothing ever arrives: the wait must give up
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool ok_ptr(const void* p) { return p != nullptr && aligned16(p); }
+cudaStream_t S(void* s) { return static_cast<cudaStream_t>(s); }
+qsa_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? QSA_OK : QSA_ERR_CUDA; }
+bool hi_supported(int Hi) { return Hi == 1 || Hi == 2 || Hi == 4 || Hi == 8; }
+}  // namespace
+
+const DeviceInfo* device_info() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_dev_ok[dev]) {
+    int sms = 0;
+    void* p = nullptr;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return nullptr;
+    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
+    g_dev[dev] = DeviceInfo{dev, sms, static_cast<unsigned*>(p)};
+    g_dev_ok[dev] = true;
+  }
+  return &g_dev[dev];
+}
+
+KernelCtl kernel_ctl(const DeviceInfo* di) { return KernelCtl{di->status, g_wait_ns.load()}; }
+
+}  // namespace qsa
+
+using namespace qsa;
+
+extern "C" {
+
+const char* qsa_status_string(qsa_status_t status) {
+  switch (status) {
+    case QSA_OK: return "QSA_OK";
+    case QSA_ERR_INVALID_ARGUMENT: return "QSA_ERR_INVALID_ARGUMENT";
+    case QSA_ERR_UNSUPPORTED: return "QSA_ERR_UNSUPPORTED";
+    case QSA_ERR_WORKSPACE_TOO_SMALL: return "QSA_ERR_WORKSPACE_TOO_SMALL";
+    case QSA_ERR_CUDA: return "QSA_ERR_CUDA";
+    case QSA_ERR_TIMEOUT: return "QSA_ERR_TIMEOUT";
+  }
+  return "QSA_ERR_UNKNOWN";
+}
+
+int qsa_abi_version(void) { return QSA_ABI_VERSION; }
+
+void qsa_set_wait_timeout_ns(uint64_t ns) { g_wait_ns.store(ns ? ns : kDefaultWaitNs); }
+
+qsa_status_t qsa_pool_block_keys(const void* ki, void* kp, int B, int L, int Di, int blk, float rope_theta,
+                                 int64_t pos0, int64_t ki_batch_stride, int64_t kp_batch_stride, void* stream) {
+  if (B < 0 || L < 0 || Di < 2 || Di > 256 || (Di & 1) || pos0 < 0) return QSA_ERR_INVALID_ARGUMENT;
+  if (ki_batch_stride < 0 || kp_batch_stride < 0) return QSA_ERR_INVALID_ARGUMENT;
+  const long long kis = ki_batch_stride ? ki_batch_stride : static_cast<long long>(L) * Di;
+  const long long kps = kp_batch_stride ? kp_batch_stride : static_cast<long long>(L / 4) * Di;
+  if (kis < static_cast<long long>(L) * Di || kps < static_cast<long long>(L / 4) * Di) return QSA_ERR_INVALID_ARGUMENT;
+  if (blk != 4) return QSA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * (L / blk) == 0) return QSA_OK;
+  if (!ok_ptr(ki) || !ok_ptr(kp)) return QSA_ERR_INVALID_ARGUMENT;
+  if (!device_info()) return QSA_ERR_CUDA;
+  return cuda_status(launch_pool(ki, kp, B, L, Di, blk, rope_theta > 0.f ? static_cast<double>(rope_theta) : 0.0,
+                                 pos0, kis, kps, S(stream)));
+}
+
+qsa_status_t qsa_rope_index_queries(const void* qi, void* qi_out, int B, int Tq, int Hi, int Di, int64_t q_pos0,
+                                    const int32_t* seqlens, float rope_theta, void* stream) {
+  if (B < 0 || Tq < 0 || Hi < 1 || Di < 2 || Di > 256 || (Di & 1) || q_pos0 < 0 || !(rope_theta > 0.f))
+    return QSA_ERR_INVALID_ARGUMENT;
+  if (seqlens && Tq != 1) return QSA_ERR_INVALID_ARGUMENT;
+  if (static_cast<long long>(B) * Tq == 0) return QSA_OK;
+  if (!ok_ptr(qi) || !ok_ptr(qi_out)) return QSA_ERR_INVALID_ARGUMENT;
+  if (!device_info()) return QSA_ERR_CUDA;
+  return cuda_status(launch_rope_queries(qi, qi_out, B, Tq, Hi, Di, q_pos0, seqlens, rope_theta, S(stream)));
+}
+
+static qsa_status_t check_score_args(const void* qi, const void* kp, const int32_t* seqlens, int B, int Tq, int NBk,
+                                     int Hi, int Di, int blk, int64_t q_pos0, int mode) {
+  if (B < 0 || Tq < 0 || NBk < 0 || q_pos0 < 0 || (mode != 0 && mode != 1)) return QSA_ERR_INVALID_ARGUMENT;
+  if (Di != 64 || !hi_supported(Hi) || blk != 4) return QSA_ERR_UNSUPPORTED;
+  if (seqlens) {
+    if (Tq != 1) return QSA_ERR_INVALID_ARGUMENT;
+  } else if (Tq > 0 && (q_pos0 + Tq - 1) / blk > NBk) {
+    return QSA_ERR_INVALID_ARGUMENT;   // the pooled keys do not cover the queries' candidates
+  }
+  if (static_cast<long long>(B) * Tq > 0 && NBk > 0 && (!ok_ptr(qi) || !ok_ptr(kp))) return QSA_ERR_INVALID_ARGUMENT;
+  return QSA_OK;
+}
+
+qsa_status_t qsa_index_score(const void* qi, const void* kp, const float* head_w, const int32_t* seqlens, int B,
+                             int Tq, int NBk, int Hi, int Di, int blk, int64_t q_pos0, qsa_score_mode_t mode,
+                             float* scores, int64_t ld_scores, void* stream) {
+  qsa_status_t st = check_score_args(qi, kp, seqlens, B, Tq, NBk, Hi, Di, blk, q_pos0, mode);
+  if (st != QSA_OK) return st;
+  if (ld_scores < std::max(NBk, 1)) return QSA_ERR_INVALID_ARGUMENT;
+  if (static_cast<long long>(B) * Tq == 0 || NBk == 0) return QSA_OK;
+  if (scores == nullptr) return QSA_ERR_INVALID_ARGUMENT;
+  const DeviceInfo* di = device_info();
+  if (!di) return QSA_ERR_CUDA;
+  if (seqlens)
+    return cuda_status(launch_score_decode(di, qi, kp, head_w, seqlens, B, NBk, Hi, Di, blk, mode, scores, ld_scores,
+                                           S(stream)));
+  return cuda_status(launch_score_prefill(di, qi, kp, head_w, B, Tq, NBk, Hi, Di, blk, q_pos0, mode, 0, B, 0, Tq,
+                                          scores, ld_scores, static_cast<long long>(Tq) * ld_scores, S(stream)));
+}
+
+qsa_status_t qsa_select_topk(const float* scores, int64_t ld_scores, const void* qi, const void* kp,
+                             const float* head_w, const int32_t* seqlens, int B, int Tq, int NBk, int Hi, int Di,
+                             int blk, int64_t q_pos0, qsa_score_mode_t mode, int k, int32_t* idx, void* workspace,
+                             size_t ws_bytes, void* stream) {
+  if (k < 1 || B < 0 || Tq < 0 || NBk < 0 || q_pos0 < 0) return QSA_ERR_INVALID_ARGUMENT;
+  if (blk != 4) return QSA_ERR_UNSUPPORTED;
+  if (seqlens && Tq != 1) return QSA_ERR_INVALID_ARGUMENT;
+  if (!seqlens && Tq > 0 && (q_pos0 + Tq - 1) / blk > NBk) return QSA_ERR_INVALID_ARGUMENT;
+  if (static_cast<long long>(B) * Tq == 0) return QSA_OK;
+  if (idx == nullptr) return QSA_ERR_INVALID_ARGUMENT;
+  cudaStream_t s = S(stream);
+  if (scores) {
+    if (ld_scores < std::max(NBk, 1)) return QSA_ERR_INVALID_ARGUMENT;
+    const DeviceInfo* di = device_info();
+    if (!di) return QSA_ERR_CUDA;
+    return cuda_status(launch_topk(di, scores, ld_scores, static_cast<long long>(Tq) * ld_scores, seqlens, Tq, NBk, blk,
+                                   q_pos0, 0, B, 0, Tq, k, idx, s));
+  }
+  qsa_status_t st = check_score_args(qi, kp, seqlens, B, Tq, NBk, Hi, Di, blk, q_pos0, mode);
+  if (st != QSA_OK) return st;
+  float* ws = static_cast<float*>(workspace);
+  const long long row_bytes = static_cast<long long>(std::max(NBk, 1)) * 4;
+  if (NBk > 0 && seqlens && (ws == nullptr || static_cast<long long>(ws_bytes) < row_bytes * B))
+    return QSA_ERR_WORKSPACE_TOO_SMALL;
+  const long long R = ws ? static_cast<long long>(ws_bytes) / row_bytes : 0;
+  if (NBk > 0 && !seqlens && R < 1) return QSA_ERR_WORKSPACE_TOO_SMALL;
+  const DeviceInfo* di = device_info();
+  if (!di) return QSA_ERR_CUDA;
+  if (NBk == 0) {   // no candidates anywhere: the lists are all -1
+    return cuda_status(launch_topk(di, nullptr, 1, 0, seqlens, Tq, 0, blk, q_pos0, 0, B, 0, Tq, k, idx, s));
+  }
+  if (seqlens) {
+    cudaError_t e = launch_score_decode(di, qi, kp, head_w, seqlens, B, NBk, Hi, Di, blk, mode, ws, NBk, s);
+    if (e == cudaSuccess) e = launch_topk(di, ws, NBk, NBk, seqlens, 1, NBk, blk, 0, 0, B, 0, 1, k, idx, s);
+    return cuda_status(e);
+  }
+  for (int b = 0; b < B; ++b) {
+    for (int r0 = 0; r0 < Tq; r0 += static_cast<int>(std::min<long long>(R, Tq))) {
+      const int rows = static_cast<int>(std::min<long long>(R, Tq - r0));
+      cudaError_t e = launch_score_prefill(di, qi, kp, head_w, B, Tq, NBk, Hi, Di, blk, q_pos0, mode, b, 1, r0, rows,
+                                           ws, NBk, 0, s);
+      if (e == cudaSuccess) e = launch_topk(di, ws, NBk, 0, nullptr, Tq, NBk, blk, q_pos0, b, 1, r0, rows, k, idx, s);
+      if (e != cudaSuccess) return QSA_ERR_CUDA;
+    }
+  }
+  return QSA_OK;
+}
+
+static qsa_status_t check_attn_shape(int Hq, int Hkv, int D, int blk, int k_blocks) {
+  if (Hq < 1 || Hkv < 1 || k_blocks < 0) return QSA_ERR_INVALID_ARGUMENT;
+  if (Hq % Hkv) return QSA_ERR_INVALID_ARGUMENT;
+  if (D != 128 || blk != 4 || Hkv > 2 || Hq / Hkv > 8) return QSA_ERR_UNSUPPORTED;
+  return QSA_OK;
+}
+
+qsa_status_t qsa_sparse_attn_prefill(const void* q, const void* k, const void* v, const int32_t* idx, int B, int Tq,
+                                     int Tk, int Hq, int Hkv, int D, int k_blocks, int blk, int64_t q_pos0,
+                                     float scale, void* out, float* lse, void* stream) {
+  qsa_status_t st = check_attn_shape(Hq, Hkv, D, blk, k_blocks);
+  if (st != QSA_OK) return st;
+  if (B < 0 || Tq < 0 || Tk < 0 || q_pos0 < 0 || q_pos0 + Tq > Tk) return QSA_ERR_INVALID_ARGUMENT;
+  if (static_cast<long long>(B) * Tq == 0) return QSA_OK;
+  if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(out) || (k_blocks > 0 && idx == nullptr))
+    return QSA_ERR_INVALID_ARGUMENT;
+  if (static_cast<long long>(B) * Tq > 0x7fffffffLL) return QSA_ERR_UNSUPPORTED;
+  const DeviceInfo* di = device_info();
+  if (!di) return QSA_ERR_CUDA;
+  return cuda_status(
+      launch_attn_prefill(di, q, k, v, idx, B, Tq, Tk, Hq, Hkv, k_blocks, q_pos0, scale, out, lse, S(stream)));
+}
+
+int qsa_decode_default_splits(int B, int k_blocks) {
+  const DeviceInfo* di = device_info();
+  if (!di || B < 1) return 1;
+  return decode_default_splits(di, B, std::max(k_blocks, 1));
+}
+
+qsa_status_t qsa_sparse_attn_decode(const void* q, const void* kcache, const void* vcache, const int32_t* seqlens,
+                                    const int32_t* idx, int B, int Lmax, int Hq, int Hkv, int D, int k_blocks, int blk,
+                                    float scale, int num_splits, void* out, float* lse, void* workspace,
+                                    size_t ws_bytes, void* stream) {
+  qsa_status_t st = check_attn_shape(Hq, Hkv, D, blk, k_blocks);
+  if (st != QSA_OK) return st;
+  if (B < 0 || Lmax < 1 || num_splits < 0) return QSA_ERR_INVALID_ARGUMENT;
+  if (B == 0) return QSA_OK;
+  if (!ok_ptr(q) || !ok_ptr(kcache) || !ok_ptr(vcache) || !ok_ptr(out) || seqlens == nullptr ||
+      (k_blocks > 0 && idx == nullptr))
+    return QSA_ERR_INVALID_ARGUMENT;
+  const DeviceInfo* di = device_info();
+  if (!di) return QSA_ERR_CUDA;
+  int splits = num_splits == 0 ? decode_default_splits(di, B, std::max(k_blocks, 1)) : num_splits;
+  splits = std::max(1, std::min(splits, std::max(k_blocks, 1)));
+  float* part = nullptr;
+  if (splits > 1) {
+    const size_t need = static_cast<size_t>(B) * splits * Hq * (D + 2) * sizeof(float);
+    if (workspace == nullptr || ws_bytes < need) return QSA_ERR_WORKSPACE_TOO_SMALL;
+    part = static_cast<float*>(workspace);
+  }
+  return cuda_status(launch_attn_decode(di, q, kcache, vcache, seqlens, idx, B, Lmax, Hq, Hkv, k_blocks, scale, splits,
+                                        out, lse, part, S(stream)));
+}
+
+size_t qsa_workspace_size(qsa_op_t op, int B, int Tq, int NBk, int k, int Hq, int D, int num_splits) {
+  if (op == QSA_OP_SELECT_TOPK) {
+    if (B < 0 || Tq < 0 || NBk < 0) return 0;
+    const long long row = static_cast<long long>(std::max(NBk, 1)) * 4;
+    if (Tq <= 1) return static_cast<size_t>(row * std::max(B, 1));
+    const long long cap = 512ll << 20;   // chunk of score rows kept at or below 512 MiB
+    const long long rows = std::max(1ll, std::min<long long>(Tq, cap / row));
+    return static_cast<size_t>(rows * row);
+  }
+  if (op == QSA_OP_SPARSE_ATTN_DECODE) {
+    if (B < 1 || Hq < 1 || D < 1) return 0;
+    int splits = num_splits > 0 ? num_splits : qsa_decode_default_splits(B, k);
+    splits = std::max(1, std::min(splits, std::max(k, 1)));
+    return static_cast<size_t>(B) * splits * Hq * (D + 2) * sizeof(float);
+  }
+  return 0;
+}
+
+qsa_status_t qsa_get_device_status(void* stream) {
+  if (cudaStreamSynchronize(S(stream)) != cudaSuccess) return QSA_ERR_CUDA;
+  unsigned v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status_word, sizeof v) != cudaSuccess) return QSA_ERR_CUDA;
+  if (v != 0 && cudaMemcpyToSymbol(g_status_word, &zero, sizeof zero) != cudaSuccess) return QSA_ERR_CUDA;
+  return static_cast<qsa_status_t>(v);
+}
+
+qsa_status_t qsa_wait_timeout_selftest(uint64_t timeout_ns, void* stream) {
+  const DeviceInfo* di = device_info();
+  if (!di) return QSA_ERR_CUDA;
+  KernelCtl ctl{di->status, timeout_ns ? timeout_ns : 1000000ull};
+  wait_selftest_kernel<<<1, 32, 0, S(stream)>>>(ctl);
+  return cuda_status(cudaPeekAtLastError());
+}
+
+}  // extern "C"

@@ -1,0 +1,375 @@
+// Indexer block scoring.
+//
+// "Qwen3.8-Flash-Next architecture" (flozi.net), "Der Weg eines Tokens durch das Modell", item 2:
+// the micro-block keys are scored with four indexer query heads that share one key head; the
+// page notes that the 4x pooling cuts the indexer's prefill work but leaves it dependent on the
+// context length.  Score (reading fixed in qsa.h): s(t,b) = sum_h w_h * max(0, qi[t,h] . kp[b]).
+//
+// Prefill: a dense contraction, run on the 5th-generation tensor cores.
+//   D[kp row m][qi row n] = sum_d kp[m][d] * qi[n][d]  with M = 128 pooled keys, N = 256 indexer
+//   rows (256/Hi queries x Hi heads), K = Di = 64 (four K=16 steps of tcgen05.mma kind::f16).
+//   The pooled keys sit in the M (TMEM lane) dimension, so one thread of the epilogue owns one
+//   pooled key and finds the Hi heads of a query in Hi adjacent TMEM columns: the ReLU-sum over
+//   heads needs no cross-thread traffic, and 32 lanes write 32 consecutive scores of a query row
+//   (one 128-byte store).  Both operands are K-major 128-byte-swizzled TMA boxes.
+//   Warp roles: warp 0 = TMA producer (qi tile once, then a 4-stage ring of kp tiles), warp 1 =
+//   TMEM allocator + single-thread MMA issuer, warps 2..9 = epilogue (two per TMEM lane quadrant,
+//   each taking half of the 256 columns).  Two 256-column fp32 accumulators in TMEM let the
+//   epilogue of tile i overlap the MMAs of tile i+1.  The causal bound is per CTA (tiles up to the
+//   last query row's visible blocks); the store mask is per query.
+// Decode: one query per sequence, so the contraction degenerates to a GEMV over the pooled-key
+//   cache; it is HBM-bound and runs on CUDA cores with 16-byte loads (8 lanes per pooled key).
+#include <mutex>
+
+#include "launch.h"
+
+namespace qsa {
+namespace {
+
+constexpr int kM = 128;          // pooled keys per tile (UMMA M, TMEM lanes)
+constexpr int kN = 256;          // indexer rows per tile (UMMA N)
+constexpr int kDi = 64;          // contraction depth (one 128-byte swizzle row)
+constexpr int kStages = 4;       // kp ring depth
+constexpr int kTilesPerCta = 16; // kp tiles handled by one CTA (split of long rows)
+constexpr int kScoreThreads = 320;
+constexpr int kQiBytes = kN * kDi * 2;   // 32768
+constexpr int kKpBytes = kM * kDi * 2;   // 16384
+constexpr int kScoreSmem = 1024 + kQiBytes + kStages * kKpBytes + 256 + 16384;  // last term: keep 1 CTA/SM
+
+struct ScoreArgs {
+  const float* head_w;
+  float* scores;
+  long long ld, batch_stride, q_pos0;
+  int NBk, blk, mode, b0, row0, rows;
+  KernelCtl ctl;
+};
+
+template <int HI>
+__global__ void __launch_bounds__(kScoreThreads, 1)
+    score_prefill_kernel(const __grid_constant__ CUtensorMap qi_map, const __grid_constant__ CUtensorMap kp_map,
+                         ScoreArgs a) {
+  constexpr int QPT = kN / HI;   // queries per tile
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* qi_s = smem;
+  uint8_t* kp_s = smem + kQiBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(kp_s + kStages * kKpBytes);
+  uint64_t* qi_full = bars;
+  uint64_t* kp_full = bars + 1;
+  uint64_t* kp_empty = kp_full + kStages;
+  uint64_t* tm_full = kp_empty + kStages;
+  uint64_t* tm_empty = tm_full + 2;
+  uint64_t* mma_done = tm_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bz = blockIdx.z;
+  const int b = a.b0 + bz;
+  const int r_first = a.row0 + static_cast<int>(blockIdx.x) * QPT;
+  const int r_last = min(r_first + QPT, a.row0 + a.rows) - 1;
+  const long long pos_last = a.q_pos0 + r_last;
+  const int nb_last = static_cast<int>(min(static_cast<long long>(a.NBk), pos_last / a.blk));
+  const int ntiles = (nb_last + kM - 1) / kM;
+  const int t_begin = static_cast<int>(blockIdx.y) * kTilesPerCta;
+  const int t_end = min(ntiles, t_begin + kTilesPerCta);
+  if (t_begin >= t_end) return;   // uniform over the CTA, before any barrier or TMEM use
+  const int nt = t_end - t_begin;
+
+  if (threadIdx.x == 0) {
+    mbar_init(qi_full, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&kp_full[s], 1);
+      mbar_init(&kp_empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tm_full[i], 1);
+      mbar_init(&tm_empty[i], 8);
+    }
+    mbar_init(mma_done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tensormap(&qi_map);
+      prefetch_tensormap(&kp_map);
+      mbar_arrive_expect_tx(qi_full, kQiBytes);
+      tma_load_3d(qi_s, &qi_map, qi_full, 0, r_first * HI, b);
+      int issued = 0;
+      for (int i = 0; i < nt; ++i) {
+        const int s = i % kStages;
+        const unsigned ph = (i / kStages) & 1u;
+        if (!mbar_wait(&kp_empty[s], ph ^ 1u, a.ctl)) break;
+        mbar_arrive_expect_tx(&kp_full[s], kKpBytes);
+        tma_load_3d(kp_s + s * kKpBytes, &kp_map, &kp_full[s], 0, (t_begin + i) * kM, b);
+        issued = i + 1;
+      }
+      // Never leave with a copy in flight: wait for the last fill of every stage and the qi tile.
+      mbar_wait(qi_full, 0, a.ctl);
+      for (int s = 0; s < kStages && s < issued; ++s) {
+        const int last = s + ((issued - 1 - s) / kStages) * kStages;
+        mbar_wait(&kp_full[s], (last / kStages) & 1u, a.ctl);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = umma_idesc_bf16_f32(kM, kN);
+      const uint64_t bdesc = sw128_kmajor_desc(smem_u32(qi_s));
+      bool ok = mbar_wait(qi_full, 0, a.ctl);
+      for (int i = 0; ok && i < nt; ++i) {
+        const int s = i % kStages;
+        const unsigned ph = (i / kStages) & 1u;
+        const int acc = i & 1;
+        const unsigned aph = (i >> 1) & 1u;
+        if (!mbar_wait(&kp_full[s], ph, a.ctl)) break;
+        if (!mbar_wait(&tm_empty[acc], aph ^ 1u, a.ctl)) break;
+        tc_fence_after();
+        const uint64_t adesc = sw128_kmajor_desc(smem_u32(kp_s + s * kKpBytes));
+#pragma unroll
+        for (int kk = 0; kk < kDi / 16; ++kk) {
+          // +32 bytes of K per step: +2 in the (>> 4) start-address field
+          umma_bf16(tmem + acc * kN, adesc + 2 * kk, bdesc + 2 * kk, idesc, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&kp_empty[s]);
+        umma_commit(&tm_full[acc]);
+      }
+      umma_commit(mma_done);
+      mbar_wait(mma_done, 0, a.ctl);
+    }
+    __syncwarp();
+  } else {
+    const int ew = warp - 2;                 // 0..7
+    const int quad = warp & 3;               // TMEM lane quadrant this warp may read
+    const int colbase = (ew >> 2) * (kN / 2);
+    const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
+    float w[HI];
+#pragma unroll
+    for (int h = 0; h < HI; ++h) w[h] = a.head_w ? a.head_w[h] : 1.0f;
+    float* srow_base = a.scores + static_cast<long long>(bz) * a.batch_stride;
+    for (int i = 0; i < nt; ++i) {
+      const int acc = i & 1;
+      const unsigned aph = (i >> 1) & 1u;
+      if (!mbar_wait(&tm_full[acc], aph, a.ctl)) break;
+      tc_fence_after();
+      const int kb = (t_begin + i) * kM + quad * 32 + lane;   // pooled key owned by this thread
+#pragma unroll 1
+      for (int c = 0; c < kN / 2; c += 32) {
+        uint32_t r[32];
+        tmem_ld_32x32(tmem + lane_addr + acc * kN + colbase + c, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int qq = 0; qq < 32 / HI; ++qq) {
+          const int row = r_first + (colbase + c) / HI + qq;
+          float sc = 0.0f;
+#pragma unroll
+          for (int h = 0; h < HI; ++h) {
+            float x = __uint_as_float(r[qq * HI + h]);
+            if (a.mode == 0) x = fmaxf(x, 0.0f);
+            sc = fmaf(w[h], x, sc);
+          }
+          if (row <= r_last) {
+            const int nbq = static_cast<int>(min(static_cast<long long>(a.NBk), (a.q_pos0 + row) / a.blk));
+            if (kb < nbq) srow_base[static_cast<long long>(row - a.row0) * a.ld + kb] = sc;
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tm_empty[acc]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------------------ decode GEMV
+template <int HI>
+__global__ void __launch_bounds__(256) score_decode_kernel(const uint16_t* __restrict__ qi,
+                                                           const uint16_t* __restrict__ kp,
+                                                           const float* __restrict__ head_w,
+                                                           const int32_t* __restrict__ seqlens, int NBk, int blk,
+                                                           int mode, float* __restrict__ scores, long long ld,
+                                                           KernelCtl ctl) {
+  const int b = blockIdx.y;
+  const int L = seqlens[b];
+  if (L < 1) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) record_status(ctl, kStBadArg);
+    return;
+  }
+  int nb = (L - 1) / blk;
+  if (nb > NBk) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) record_status(ctl, kStBadArg);
+    nb = NBk;
+  }
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int seg = lane & 7;      // 8-element segment of Di = 64
+  const int sub = lane >> 3;     // which of the 4 keys a warp instruction covers
+  float q[HI][8];
+#pragma unroll
+  for (int h = 0; h < HI; ++h) {
+    const uint4 raw = *reinterpret_cast<const uint4*>(qi + (static_cast<long long>(b) * HI + h) * kDi + seg * 8);
+    const uint32_t u[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      q[h][2 * e] = __uint_as_float(u[e] << 16);
+      q[h][2 * e + 1] = __uint_as_float(u[e] & 0xFFFF0000u);
+    }
+  }
+  float w[HI];
+#pragma unroll
+  for (int h = 0; h < HI; ++h) w[h] = head_w ? head_w[h] : 1.0f;
+  const uint16_t* kpb = kp + static_cast<long long>(b) * NBk * kDi;
+  float* srow = scores + static_cast<long long>(b) * ld;
+  constexpr int kU = 4;   // loads in flight per lane
+  const long long stride = static_cast<long long>(gridDim.x) * 8 * 4 * kU;
+  for (long long base = (static_cast<long long>(blockIdx.x) * 8 + warp) * 4 * kU; base < nb; base += stride) {
+    uint4 raw[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const long long row = base + u * 4 + sub;
+      raw[u] = row < nb ? __ldg(reinterpret_cast<const uint4*>(kpb + row * kDi + seg * 8)) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const uint32_t v[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
+      float kv[8];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        kv[2 * e] = __uint_as_float(v[e] << 16);
+        kv[2 * e + 1] = __uint_as_float(v[e] & 0xFFFF0000u);
+      }
+      float dot[HI];
+#pragma unroll
+      for (int h = 0; h < HI; ++h) {
+        float d = 0.0f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) d = fmaf(q[h][e], kv[e], d);
+        d += __shfl_xor_sync(0xffffffffu, d, 1);
+        d += __shfl_xor_sync(0xffffffffu, d, 2);
+        d += __shfl_xor_sync(0xffffffffu, d, 4);
+        dot[h] = d;
+      }
+      const long long row = base + u * 4 + sub;
+      if (seg == 0 && row < nb) {
+        float sc = 0.0f;
+#pragma unroll
+        for (int h = 0; h < HI; ++h) sc = fmaf(w[h], mode == 0 ? fmaxf(dot[h], 0.0f) : dot[h], sc);
+        srow[row] = sc;
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------ host helpers
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 3-D bf16 map over [d2][d1][64] with a 128-byte-swizzled box of {64, box_rows, 1}.
+bool make_map(CUtensorMap* m, const void* base, unsigned long long d1, unsigned long long d2, unsigned box_rows) {
+  EncodeTiledFn fn = encode_tiled();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(kDi), d1, d2};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(kDi) * 2, d1 * kDi * 2};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(kDi), box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int HI>
+cudaError_t launch_prefill_hi(const void* qi, const void* kp, const float* head_w, int Tq, int NBk, int blk,
+                              long long q_pos0, int mode, int b0, int nb, int row0, int rows, float* scores,
+                              long long ld, long long batch_stride, const KernelCtl& ctl, cudaStream_t s) {
+  static std::once_flag attr_once[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::call_once(attr_once[dev & 63], [] {
+    cudaFuncSetAttribute(score_prefill_kernel<HI>, cudaFuncAttributeMaxDynamicSharedMemorySize, kScoreSmem);
+  });
+  CUtensorMap qmap, kmap;
+  // Maps span all batches so the batch index is a TMA coordinate.
+  const int Btot = b0 + nb;
+  if (!make_map(&qmap, qi, static_cast<unsigned long long>(Tq) * HI, static_cast<unsigned long long>(Btot), kN) ||
+      !make_map(&kmap, kp, static_cast<unsigned long long>(NBk), static_cast<unsigned long long>(Btot), kM))
+    return cudaErrorInvalidValue;
+  constexpr int QPT = kN / HI;
+  const long long pos_last = q_pos0 + row0 + rows - 1;
+  const int nb_last = static_cast<int>(std::min<long long>(NBk, pos_last / blk));
+  const int ntiles = (nb_last + kM - 1) / kM;
+  if (ntiles == 0) return cudaSuccess;
+  dim3 grid((rows + QPT - 1) / QPT, (ntiles + kTilesPerCta - 1) / kTilesPerCta, nb);
+  ScoreArgs a{head_w, scores, ld, batch_stride, q_pos0, NBk, blk, mode, b0, row0, rows, ctl};
+  score_prefill_kernel<HI><<<grid, kScoreThreads, kScoreSmem, s>>>(qmap, kmap, a);
+  return cudaPeekAtLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_score_prefill(const DeviceInfo* di, const void* qi, const void* kp, const float* head_w, int B,
+                                 int Tq, int NBk, int Hi, int Di, int blk, long long q_pos0, int mode, int b0, int nb,
+                                 int row0, int rows, float* scores, long long ld, long long batch_stride,
+                                 cudaStream_t s) {
+  (void)B;
+  (void)Di;
+  if (rows <= 0 || nb <= 0) return cudaSuccess;
+  const KernelCtl ctl = kernel_ctl(di);
+  switch (Hi) {
+    case 1: return launch_prefill_hi<1>(qi, kp, head_w, Tq, NBk, blk, q_pos0, mode, b0, nb, row0, rows, scores, ld, batch_stride, ctl, s);
+    case 2: return launch_prefill_hi<2>(qi, kp, head_w, Tq, NBk, blk, q_pos0, mode, b0, nb, row0, rows, scores, ld, batch_stride, ctl, s);
+    case 4: return launch_prefill_hi<4>(qi, kp, head_w, Tq, NBk, blk, q_pos0, mode, b0, nb, row0, rows, scores, ld, batch_stride, ctl, s);
+    case 8: return launch_prefill_hi<8>(qi, kp, head_w, Tq, NBk, blk, q_pos0, mode, b0, nb, row0, rows, scores, ld, batch_stride, ctl, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_score_decode(const DeviceInfo* di, const void* qi, const void* kp, const float* head_w,
+                                const int32_t* seqlens, int B, int NBk, int Hi, int Di, int blk, int mode,
+                                float* scores, long long ld, cudaStream_t s) {
+  (void)Di;
+  if (B <= 0 || NBk <= 0) return cudaSuccess;
+  const KernelCtl ctl = kernel_ctl(di);
+  const int per_seq = std::max(1, (di->num_sms * 4 + B - 1) / B);
+  const int need = (NBk + 127) / 128;
+  dim3 grid(std::min(per_seq, need), B);
+  const uint16_t* q = static_cast<const uint16_t*>(qi);
+  const uint16_t* k = static_cast<const uint16_t*>(kp);
+  switch (Hi) {
+    case 1: score_decode_kernel<1><<<grid, 256, 0, s>>>(q, k, head_w, seqlens, NBk, blk, mode, scores, ld, ctl); break;
+    case 2: score_decode_kernel<2><<<grid, 256, 0, s>>>(q, k, head_w, seqlens, NBk, blk, mode, scores, ld, ctl); break;
+    case 4: score_decode_kernel<4><<<grid, 256, 0, s>>>(q, k, head_w, seqlens, NBk, blk, mode, scores, ld, ctl); break;
+    case 8: score_decode_kernel<8><<<grid, 256, 0, s>>>(q, k, head_w, seqlens, NBk, blk, mode, scores, ld, ctl); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaPeekAtLastError();
+}
+
+}  // namespace qsa

@@ -1,0 +1,54 @@
+// Internal launchers behind the C ABI (one per kernel family).  Arguments are validated by the
+// ABI layer before any of these is called.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace qsa {
+
+struct DeviceInfo {
+  int device;
+  int num_sms;
+  unsigned* status;   // device address of the status word
+};
+// Per-device cached attributes of the current device (nullptr on a runtime error).
+const DeviceInfo* device_info();
+KernelCtl kernel_ctl(const DeviceInfo* di);
+
+cudaError_t launch_pool(const void* ki, void* kp, int B, int L, int Di, int blk, double theta, long long pos0,
+                        long long ki_bs, long long kp_bs, cudaStream_t s);
+cudaError_t launch_rope_queries(const void* qi, void* qo, int B, int Tq, int Hi, int Di, long long q_pos0,
+                                const int32_t* seqlens, double theta, cudaStream_t s);
+
+// Prefill scores for query rows [row0, row0 + rows) of batches [b0, b0 + nb) into
+// scores + (b - b0) * batch_stride + (t - row0) * ld.
+cudaError_t launch_score_prefill(const DeviceInfo* di, const void* qi, const void* kp, const float* head_w, int B,
+                                 int Tq, int NBk, int Hi, int Di, int blk, long long q_pos0, int mode, int b0, int nb,
+                                 int row0, int rows, float* scores, long long ld, long long batch_stride,
+                                 cudaStream_t s);
+cudaError_t launch_score_decode(const DeviceInfo* di, const void* qi, const void* kp, const float* head_w,
+                                const int32_t* seqlens, int B, int NBk, int Hi, int Di, int blk, int mode,
+                                float* scores, long long ld, cudaStream_t s);
+
+// Top-k over score rows: row r of batch b (b0 <= b < b0 + nb, row0 <= r < row0 + rows) reads
+// scores + (b - b0) * batch_stride + (r - row0) * ld and writes idx + (b * Tq + r) * k.
+cudaError_t launch_topk(const DeviceInfo* di, const float* scores, long long ld, long long batch_stride,
+                        const int32_t* seqlens, int Tq, int NBk, int blk, long long q_pos0, int b0, int nb, int row0,
+                        int rows, int k, int32_t* idx, cudaStream_t s);
+
+cudaError_t launch_attn_prefill(const DeviceInfo* di, const void* q, const void* k, const void* v, const int32_t* idx,
+                                int B, int Tq, int Tk, int Hq, int Hkv, int k_blocks, long long q_pos0, float scale,
+                                void* out, float* lse, cudaStream_t s);
+cudaError_t launch_attn_decode(const DeviceInfo* di, const void* q, const void* kc, const void* vc,
+                               const int32_t* seqlens, const int32_t* idx, int B, int Lmax, int Hq, int Hkv,
+                               int k_blocks, float scale, int num_splits, void* out, float* lse, float* part,
+                               cudaStream_t s);
+int decode_default_splits(const DeviceInfo* di, int B, int k_blocks);
+
+cudaError_t launch_wait_selftest(const DeviceInfo* di, unsigned long long timeout_ns, cudaStream_t s);
+
+}  // namespace qsa

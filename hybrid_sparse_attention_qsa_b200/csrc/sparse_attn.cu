@@ -1,0 +1,541 @@
+// Gather-sparse attention over the selected micro-blocks (prefill and split-KV decode).
+//
+// "Qwen3.8-Flash-Next architecture" (flozi.net), "Der Weg eines Tokens durch das Modell", item 2:
+// after the selection, exact attention runs over only the selected tokens, with grouped query
+// heads sharing KV heads.  For query position p and head h (KV head g = h / (Hq/Hkv)):
+//   o = sum_{j in S} softmax_j(scale * q . k_j) v_j,  S = tokens of the listed blocks plus the own
+//   block's tokens blk*floor(p/blk) .. p.
+//
+// Design (B200, HBM/L2-bound: ~8 flop per gathered byte):
+//   * One work item = one query row (prefill) or one range of a sequence's index list (decode
+//     split).  Persistent CTAs walk the items; a producer warp streams the selected blocks of
+//     successive items through a 3-stage shared-memory ring without draining between items.
+//   * A block of 4 tokens is one contiguous 4*Hkv*D*2-byte run of K (and of V) in the [T][Hkv][D]
+//     layout, so each block is one 1-D bulk copy (cp.async.bulk, TMA engine) for K and one for V.
+//     A stage holds 16 blocks.  The smem pitch of a block slot is its size + 16 bytes, so the same
+//     token row of 8 consecutive slots falls in 8 different 16-byte bank groups: ldmatrix on
+//     "token j of slots 0..7" is conflict-free.
+//   * Consumer warp (g, j) owns KV head g and token j of every block: its 16 rows per stage are
+//     token j of the 16 slots.  Scores are computed transposed, S^T[token][head] = K_g Q_g^T, with
+//     mma.m16n8k16 (M = 16 tokens, N = 8 query heads of the group, K = D), so the 8 heads of a GQA
+//     group fill N exactly.  The fp32 online softmax runs per head column (exp2 form); P^T is
+//     transposed in registers (movmatrix) into the B operand of O^T[d][head] += V^T P^T.
+//   * The 4 warps of a KV head hold partial softmax states over disjoint token sets; they are
+//     merged through shared memory at the end of an item (log-sum-exp merge), then the output row
+//     is staged in shared memory and written with 16-byte stores.
+//   * Decode: each (sequence, split) is an item writing an unnormalised partial (o, m, l); a
+//     small kernel merges the splits.  With one split the item writes the final row directly.
+// Entries -1 and the own block in an index list are skipped; other entries outside [0, own) are
+// skipped and recorded in the device status word.  Every mbarrier wait is bounded.
+#include <algorithm>
+#include <cfloat>
+#include <mutex>
+
+#include "launch.h"
+
+namespace qsa {
+namespace {
+
+constexpr int kSlots = 16;
+constexpr int kStages = 3;
+constexpr int kD = 128;
+constexpr int kBlk = 4;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+template <int HKV>
+struct Cfg {
+  static constexpr int kBlockBytes = kBlk * HKV * kD * 2;     // one block of K (or of V)
+  static constexpr int kPitch = kBlockBytes + 16;
+  static constexpr int kStageBytes = 2 * kSlots * kPitch;     // K slots, then V slots
+  static constexpr int kConsumerWarps = kBlk * HKV;
+  static constexpr int kThreads = (kConsumerWarps + 1) * 32;
+  static constexpr int kMergeSlot = 32 * 32 * 4 + 32 * 4 * 4; // o fragments + (m0, m1, l0, l1) per lane
+  static constexpr int kMergeBytes = 3 * HKV * kMergeSlot;
+  static constexpr int kInfoBytes = kStages * 32;
+  static constexpr int kBarBytes = (2 * kStages + 2 * HKV) * 8;
+  static constexpr int kPendBytes = 64 * 4;
+  static constexpr int kSmem = 128 + kStages * kStageBytes + kMergeBytes + kInfoBytes + kBarBytes + kPendBytes;
+};
+
+struct StageInfo {
+  int nslots;
+  int last;
+  int pad[2];
+  uint8_t ntok[kSlots];
+};
+
+struct AttnArgs {
+  const uint16_t* q;
+  const uint16_t* k;
+  const uint16_t* v;
+  const int32_t* idx;
+  const int32_t* seqlens;   // decode when non-null
+  uint16_t* out;
+  float* lse;
+  float* part;              // decode partials [items][Hq][D + 2]
+  long long q_pos0;
+  int B, Tq, Tk, Hq, kblocks, splits, num_items;
+  float scale_log2;
+  KernelCtl ctl;
+};
+
+struct Item {
+  const uint16_t* kbase;
+  const uint16_t* vbase;
+  const int32_t* idx_row;
+  long long pos;
+  long long qrow;      // row of q ([B*Tq] or [B])
+  long long orow;      // row of out / lse / part
+  int lo, hi;
+  bool diag, ok, partial;
+};
+
+template <int HKV>
+__device__ __forceinline__ Item make_item(const AttnArgs& a, int i) {
+  Item it;
+  if (a.seqlens == nullptr) {
+    const int t = a.Tq - 1 - i / a.B;   // longest rows first
+    const int b = i % a.B;
+    it.qrow = static_cast<long long>(b) * a.Tq + t;
+    it.orow = it.qrow;
+    it.pos = a.q_pos0 + t;
+    it.kbase = a.k + static_cast<long long>(b) * a.Tk * HKV * kD;
+    it.vbase = a.v + static_cast<long long>(b) * a.Tk * HKV * kD;
+    it.idx_row = a.idx + it.qrow * a.kblocks;
+    it.lo = 0;
+    it.hi = a.kblocks;
+    it.diag = true;
+    it.ok = true;
+    it.partial = false;
+  } else {
+    const int b = i / a.splits, sp = i % a.splits;
+    const int L = a.seqlens[b];
+    it.ok = L >= 1 && L <= a.Tk;
+    it.pos = static_cast<long long>(L) - 1;
+    it.qrow = b;
+    it.orow = a.splits > 1 ? i : b;
+    it.kbase = a.k + static_cast<long long>(b) * a.Tk * HKV * kD;
+    it.vbase = a.v + static_cast<long long>(b) * a.Tk * HKV * kD;
+    it.idx_row = a.idx + static_cast<long long>(b) * a.kblocks;
+    const int chunk = (a.kblocks + a.splits - 1) / a.splits;
+    it.lo = min(a.kblocks, sp * chunk);
+    it.hi = min(a.kblocks, it.lo + chunk);
+    it.diag = sp == 0;
+    it.partial = a.splits > 1;
+  }
+  return it;
+}
+
+template <int HKV>
+__global__ void __launch_bounds__(Cfg<HKV>::kThreads, 1) sparse_attn_kernel(AttnArgs a) {
+  using C = Cfg<HKV>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  uint8_t* ring = smem;
+  uint8_t* merge = ring + kStages * C::kStageBytes;
+  StageInfo* info = reinterpret_cast<StageInfo*>(merge + C::kMergeBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(info) + C::kInfoBytes);
+  uint64_t* empty = full + kStages;
+  uint64_t* mfull = empty + kStages;    // per KV head: the 3 partner warps have written their state
+  uint64_t* mempty = mfull + HKV;       // per KV head: warp j=0 has consumed the merge slots
+  int* pend = reinterpret_cast<int*>(mempty + HKV);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int group = a.Hq / HKV;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], C::kConsumerWarps);
+    }
+    for (int g = 0; g < HKV; ++g) {
+      mbar_init(&mfull[g], kBlk - 1);
+      mbar_init(&mempty[g], 1);
+    }
+    fence_mbar_init();
+  }
+  // Zero the ring once so that unused slot rows are finite (they are masked, but 0 * NaN = NaN).
+  for (int i = threadIdx.x; i < kStages * C::kStageBytes / 16; i += blockDim.x)
+    reinterpret_cast<uint4*>(ring)[i] = make_uint4(0, 0, 0, 0);
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // order these writes before the bulk copies
+  __syncthreads();
+
+  if (warp == C::kConsumerWarps) {
+    // ------------------------------------------------------------------ producer warp
+    int st = 0;
+    unsigned ph = 0;
+    int fills = 0;
+    bool alive = true;
+    const uint32_t tok_bytes = HKV * kD * 2;
+    auto flush = [&](int n, bool last, const Item& it) -> bool {
+      if (!mbar_wait(&empty[st], ph ^ 1u, a.ctl)) return false;
+      int packed = lane < n ? pend[lane] : 0;
+      const int ntok = packed & 7;
+      const long long tok0 = packed >> 3;
+      if (lane < kSlots) info[st].ntok[lane] = static_cast<uint8_t>(lane < n ? ntok : 0);
+      if (lane == 0) {
+        info[st].nslots = n;
+        info[st].last = last ? 1 : 0;
+      }
+      const uint32_t mine = lane < n ? 2u * ntok * tok_bytes : 0u;
+      const uint32_t total = __reduce_add_sync(0xffffffffu, mine);
+      __syncwarp();
+      if (lane == 0) mbar_arrive_expect_tx(&full[st], total);
+      __syncwarp();
+      if (lane < n) {
+        uint8_t* kd = ring + st * C::kStageBytes + lane * C::kPitch;
+        uint8_t* vd = kd + kSlots * C::kPitch;
+        bulk_g2s(kd, it.kbase + tok0 * HKV * kD, ntok * tok_bytes, &full[st]);
+        bulk_g2s(vd, it.vbase + tok0 * HKV * kD, ntok * tok_bytes, &full[st]);
+      }
+      // drop the flushed entries from the pending list
+      int rest0 = n + lane < 64 ? pend[n + lane] : 0;
+      int rest1 = n + lane + 32 < 64 ? pend[n + lane + 32] : 0;
+      __syncwarp();
+      pend[lane] = rest0;
+      if (lane + 32 < 64) pend[lane + 32] = rest1;
+      __syncwarp();
+      ++fills;
+      if (++st == kStages) {
+        st = 0;
+        ph ^= 1u;
+      }
+      return true;
+    };
+    for (int item = blockIdx.x; alive && item < a.num_items; item += gridDim.x) {
+      const Item it = make_item<HKV>(a, item);
+      const long long own = it.pos >= 0 ? it.pos / kBlk : 0;
+      int npend = 0;
+      if (it.ok) {
+        for (int c = it.lo; alive && c < it.hi; c += 32) {
+          const int e = c + lane < it.hi ? it.idx_row[c + lane] : -1;
+          const bool valid = e >= 0 && e < own;
+          if (!valid && e != -1 && e != own) record_status(a.ctl, kStBadArg);
+          const unsigned m = __ballot_sync(0xffffffffu, valid);
+          if (valid) pend[npend + __popc(m & ((1u << lane) - 1u))] = (e * kBlk) << 3 | kBlk;
+          npend += __popc(m);
+          __syncwarp();
+          while (alive && npend > kSlots) {
+            alive = flush(kSlots, false, it);
+            npend -= kSlots;
+          }
+        }
+        if (it.diag) {
+          if (lane == 0) pend[npend] = static_cast<int>((own * kBlk) << 3) | static_cast<int>(it.pos - own * kBlk + 1);
+          ++npend;
+          __syncwarp();
+        }
+      } else if (lane == 0) {
+        record_status(a.ctl, kStBadArg);
+      }
+      while (alive && npend > kSlots) {
+        alive = flush(kSlots, false, it);
+        npend -= kSlots;
+      }
+      if (alive) alive = flush(npend, true, it);
+    }
+    // Never leave with a copy in flight: wait for the last fill of every stage.
+    for (int s = 0; s < kStages && s < fills; ++s) {
+      const int last = s + ((fills - 1 - s) / kStages) * kStages;
+      mbar_wait(&full[s], (last / kStages) & 1u, a.ctl);
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------------- consumer warps
+  const int g = warp / kBlk;       // KV head
+  const int j = warp % kBlk;       // token within each block
+  const int n_head = lane >> 2;    // head column this lane feeds in the B operand
+  const int cpair = 2 * (lane & 3);   // head columns of this lane's accumulators
+  const uint32_t ring_u32 = smem_u32(ring);
+  const int mi = lane >> 3;
+  const uint32_t k_off = static_cast<uint32_t>(((lane & 7) + (mi & 1) * 8) * C::kPitch + (j * HKV + g) * kD * 2 +
+                                               (mi >> 1) * 16);
+  const uint32_t v_off = static_cast<uint32_t>(((lane & 7) + (mi >> 1) * 8) * C::kPitch + (j * HKV + g) * kD * 2 +
+                                               (mi & 1) * 16);
+  float* mslot_base = reinterpret_cast<float*>(merge);
+  int st = 0;
+  unsigned ph = 0;
+  unsigned mph = 0;   // parity of the merge barriers (one phase per item)
+
+  for (int item = blockIdx.x; item < a.num_items; item += gridDim.x) {
+    const Item it = make_item<HKV>(a, item);
+    uint32_t qf[8][2];
+    {
+      const int hq = g * group + n_head;
+      const bool hv = n_head < group;
+      const uint16_t* qrow = a.q + (it.qrow * a.Hq + (hv ? hq : 0)) * kD;
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const int d0 = 16 * kk + cpair;
+        qf[kk][0] = hv ? *reinterpret_cast<const uint32_t*>(qrow + d0) : 0u;
+        qf[kk][1] = hv ? *reinterpret_cast<const uint32_t*>(qrow + d0 + 8) : 0u;
+      }
+    }
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+    float o[8][4];
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+
+    for (;;) {
+      if (!mbar_wait(&full[st], ph, a.ctl)) return;
+      const int ns = info[st].nslots;
+      const bool last = info[st].last != 0;
+      if (ns > 0) {
+        const uint32_t kst = ring_u32 + st * C::kStageBytes;
+        const uint32_t vst = kst + kSlots * C::kPitch;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4(kst + k_off + kk * 32, a0, a1, a2, a3);
+          mma_bf16_16816(acc, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
+        }
+        const int r0 = lane >> 2, r1 = r0 + 8;
+        const bool v0 = r0 < ns && j < info[st].ntok[r0];
+        const bool v1 = r1 < ns && j < info[st].ntok[r1];
+        const float x0 = v0 ? acc[0] * a.scale_log2 : -INFINITY;
+        const float x1 = v0 ? acc[1] * a.scale_log2 : -INFINITY;
+        const float x2 = v1 ? acc[2] * a.scale_log2 : -INFINITY;
+        const float x3 = v1 ? acc[3] * a.scale_log2 : -INFINITY;
+        float t0 = fmaxf(x0, x2), t1 = fmaxf(x1, x3);
+#pragma unroll
+        for (int o2 = 4; o2 < 32; o2 <<= 1) {
+          t0 = fmaxf(t0, __shfl_xor_sync(0xffffffffu, t0, o2));
+          t1 = fmaxf(t1, __shfl_xor_sync(0xffffffffu, t1, o2));
+        }
+        const float mn0 = fmaxf(m0, t0), mn1 = fmaxf(m1, t1);
+        const float ref0 = mn0 == -INFINITY ? 0.f : mn0;
+        const float ref1 = mn1 == -INFINITY ? 0.f : mn1;
+        const float al0 = exp2f(m0 - ref0), al1 = exp2f(m1 - ref1);
+        const float p0 = exp2f(x0 - ref0), p1 = exp2f(x1 - ref1);
+        const float p2 = exp2f(x2 - ref0), p3 = exp2f(x3 - ref1);
+        l0 = l0 * al0 + (p0 + p2);
+        l1 = l1 * al1 + (p1 + p3);
+        m0 = mn0;
+        m1 = mn1;
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+          o[mt][0] *= al0;
+          o[mt][1] *= al1;
+          o[mt][2] *= al0;
+          o[mt][3] *= al1;
+        }
+        const uint32_t b0 = movmatrix_t(pack_bf16x2(p0, p1));
+        const uint32_t b1 = movmatrix_t(pack_bf16x2(p2, p3));
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4_t(vst + v_off + mt * 32, a0, a1, a2, a3);
+          mma_bf16_16816(o[mt], a0, a1, a2, a3, b0, b1);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st]);
+      if (++st == kStages) {
+        st = 0;
+        ph ^= 1u;
+      }
+      if (last) break;
+    }
+
+    // ---- item epilogue: full row sums, merge the 4 token-warps of this KV head, write
+#pragma unroll
+    for (int o2 = 4; o2 < 32; o2 <<= 1) {
+      l0 += __shfl_xor_sync(0xffffffffu, l0, o2);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, o2);
+    }
+    float* my_slot = mslot_base + (g * 3 + (j > 0 ? j - 1 : 0)) * (C::kMergeSlot / 4);
+    if (j > 0) {
+      if (!mbar_wait(&mempty[g], mph ^ 1u, a.ctl)) return;
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) my_slot[(mt * 4 + e) * 32 + lane] = o[mt][e];
+      float* ml = my_slot + 1024;
+      ml[lane] = m0;
+      ml[32 + lane] = m1;
+      ml[64 + lane] = l0;
+      ml[96 + lane] = l1;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&mfull[g]);
+    } else {
+      if (!mbar_wait(&mfull[g], mph, a.ctl)) return;
+    }
+    if (j == 0) {
+#pragma unroll 1
+      for (int jj = 0; jj < kBlk - 1; ++jj) {
+        const float* sl = mslot_base + (g * 3 + jj) * (C::kMergeSlot / 4);
+        const float* ml = sl + 1024;
+        const float om0 = ml[lane], om1 = ml[32 + lane], ol0 = ml[64 + lane], ol1 = ml[96 + lane];
+        const float M0 = fmaxf(m0, om0), M1 = fmaxf(m1, om1);
+        const float R0 = M0 == -INFINITY ? 0.f : M0, R1 = M1 == -INFINITY ? 0.f : M1;
+        const float fs0 = exp2f(m0 - R0), fo0 = exp2f(om0 - R0);
+        const float fs1 = exp2f(m1 - R1), fo1 = exp2f(om1 - R1);
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+          o[mt][0] = o[mt][0] * fs0 + sl[(mt * 4 + 0) * 32 + lane] * fo0;
+          o[mt][1] = o[mt][1] * fs1 + sl[(mt * 4 + 1) * 32 + lane] * fo1;
+          o[mt][2] = o[mt][2] * fs0 + sl[(mt * 4 + 2) * 32 + lane] * fo0;
+          o[mt][3] = o[mt][3] * fs1 + sl[(mt * 4 + 3) * 32 + lane] * fo1;
+        }
+        l0 = l0 * fs0 + ol0 * fo0;
+        l1 = l1 * fs1 + ol1 * fo1;
+        m0 = M0;
+        m1 = M1;
+      }
+      if (!it.partial) {
+        // stage the normalised rows [head][d] as bf16, then 16-byte stores
+        // staged in merge slot (g, 0), which this warp has finished reading
+        uint16_t* stg = reinterpret_cast<uint16_t*>(mslot_base + (g * 3) * (C::kMergeSlot / 4));
+        const float inv0 = l0 > 0.f ? 1.f / l0 : 0.f, inv1 = l1 > 0.f ? 1.f / l1 : 0.f;
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+          const int d = 16 * mt + (lane >> 2);
+          stg[(cpair)*kD + d] = __bfloat16_as_ushort(__float2bfloat16_rn(o[mt][0] * inv0));
+          stg[(cpair + 1) * kD + d] = __bfloat16_as_ushort(__float2bfloat16_rn(o[mt][1] * inv1));
+          stg[(cpair)*kD + d + 8] = __bfloat16_as_ushort(__float2bfloat16_rn(o[mt][2] * inv0));
+          stg[(cpair + 1) * kD + d + 8] = __bfloat16_as_ushort(__float2bfloat16_rn(o[mt][3] * inv1));
+        }
+        __syncwarp();
+        uint16_t* orow = a.out + (it.orow * a.Hq + g * group) * kD;
+        const int chunks = group * kD / 8;   // 16-byte chunks of this KV head's output heads
+        for (int c = lane; c < chunks; c += 32)
+          reinterpret_cast<uint4*>(orow)[c] = reinterpret_cast<const uint4*>(stg)[c];
+        if (a.lse && lane < 4) {
+          if (cpair < group)
+            a.lse[it.orow * a.Hq + g * group + cpair] = l0 > 0.f ? (m0 + __log2f(l0)) * kLn2 : -INFINITY;
+          if (cpair + 1 < group)
+            a.lse[it.orow * a.Hq + g * group + cpair + 1] = l1 > 0.f ? (m1 + __log2f(l1)) * kLn2 : -INFINITY;
+        }
+        __syncwarp();
+      } else {
+        // unnormalised partial: part[item][h][0..D) = o, part[item][h][D] = m (log2 units), [D+1] = l
+        float* prow = a.part + it.orow * a.Hq * (kD + 2);
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+          const int d = 16 * mt + (lane >> 2);
+          if (cpair < group) {
+            prow[(g * group + cpair) * (kD + 2) + d] = o[mt][0];
+            prow[(g * group + cpair) * (kD + 2) + d + 8] = o[mt][2];
+          }
+          if (cpair + 1 < group) {
+            prow[(g * group + cpair + 1) * (kD + 2) + d] = o[mt][1];
+            prow[(g * group + cpair + 1) * (kD + 2) + d + 8] = o[mt][3];
+          }
+        }
+        if (lane < 4) {
+          if (cpair < group) {
+            prow[(g * group + cpair) * (kD + 2) + kD] = m0;
+            prow[(g * group + cpair) * (kD + 2) + kD + 1] = l0;
+          }
+          if (cpair + 1 < group) {
+            prow[(g * group + cpair + 1) * (kD + 2) + kD] = m1;
+            prow[(g * group + cpair + 1) * (kD + 2) + kD + 1] = l1;
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&mempty[g]);
+    }
+    mph ^= 1u;
+  }
+}
+
+// Merge of decode splits: out[b][h] = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s.
+__global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ part, int splits, int Hq,
+                                                      uint16_t* __restrict__ out, float* __restrict__ lse) {
+  const int b = blockIdx.x, h = blockIdx.y, d = threadIdx.x;
+  const float* p = part + (static_cast<long long>(b) * splits * Hq + h) * (kD + 2);
+  const long long step = static_cast<long long>(Hq) * (kD + 2);
+  float M = -INFINITY;
+  for (int s = 0; s < splits; ++s) M = fmaxf(M, p[s * step + kD]);
+  const float R = M == -INFINITY ? 0.f : M;
+  float acc = 0.f, l = 0.f;
+  for (int s = 0; s < splits; ++s) {
+    const float f = exp2f(p[s * step + kD] - R);
+    acc += f * p[s * step + d];
+    l += f * p[s * step + kD + 1];
+  }
+  out[(static_cast<long long>(b) * Hq + h) * kD + d] = __bfloat16_as_ushort(__float2bfloat16_rn(l > 0.f ? acc / l : 0.f));
+  if (lse && d == 0) lse[static_cast<long long>(b) * Hq + h] = l > 0.f ? (M + __log2f(l)) * kLn2 : -INFINITY;
+}
+
+template <int HKV>
+cudaError_t launch_attn(const DeviceInfo* di, AttnArgs a, cudaStream_t s) {
+  using C = Cfg<HKV>;
+  static std::once_flag once[64];
+  std::call_once(once[di->device & 63], [] {
+    cudaFuncSetAttribute(sparse_attn_kernel<HKV>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  });
+  const int grid = std::min(a.num_items, di->num_sms);
+  if (grid <= 0) return cudaSuccess;
+  sparse_attn_kernel<HKV><<<grid, C::kThreads, C::kSmem, s>>>(a);
+  return cudaPeekAtLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attn_prefill(const DeviceInfo* di, const void* q, const void* k, const void* v, const int32_t* idx,
+                                int B, int Tq, int Tk, int Hq, int Hkv, int k_blocks, long long q_pos0, float scale,
+                                void* out, float* lse, cudaStream_t s) {
+  AttnArgs a{};
+  a.q = static_cast<const uint16_t*>(q);
+  a.k = static_cast<const uint16_t*>(k);
+  a.v = static_cast<const uint16_t*>(v);
+  a.idx = idx;
+  a.seqlens = nullptr;
+  a.out = static_cast<uint16_t*>(out);
+  a.lse = lse;
+  a.part = nullptr;
+  a.q_pos0 = q_pos0;
+  a.B = B;
+  a.Tq = Tq;
+  a.Tk = Tk;
+  a.Hq = Hq;
+  a.kblocks = k_blocks;
+  a.splits = 1;
+  a.num_items = B * Tq;
+  a.scale_log2 = scale * kLog2e;
+  a.ctl = kernel_ctl(di);
+  return Hkv == 1 ? launch_attn<1>(di, a, s) : launch_attn<2>(di, a, s);
+}
+
+int decode_default_splits(const DeviceInfo* di, int B, int k_blocks) {
+  // about two items per SM, and at least ~32 blocks per split
+  const int want = std::max(1, (2 * di->num_sms + B - 1) / std::max(B, 1));
+  const int cap = std::max(1, (k_blocks + 31) / 32);
+  return std::min(want, cap);
+}
+
+cudaError_t launch_attn_decode(const DeviceInfo* di, const void* q, const void* kc, const void* vc,
+                               const int32_t* seqlens, const int32_t* idx, int B, int Lmax, int Hq, int Hkv,
+                               int k_blocks, float scale, int num_splits, void* out, float* lse, float* part,
+                               cudaStream_t s) {
+  AttnArgs a{};
+  a.q = static_cast<const uint16_t*>(q);
+  a.k = static_cast<const uint16_t*>(kc);
+  a.v = static_cast<const uint16_t*>(vc);
+  a.idx = idx;
+  a.seqlens = seqlens;
+  a.out = static_cast<uint16_t*>(out);
+  a.lse = lse;
+  a.part = part;
+  a.q_pos0 = 0;
+  a.B = B;
+  a.Tq = 1;
+  a.Tk = Lmax;
+  a.Hq = Hq;
+  a.kblocks = k_blocks;
+  a.splits = num_splits;
+  a.num_items = B * num_splits;
+  a.scale_log2 = scale * kLog2e;
+  a.ctl = kernel_ctl(di);
+  cudaError_t e = Hkv == 1 ? launch_attn<1>(di, a, s) : launch_attn<2>(di, a, s);
+  if (e != cudaSuccess || num_splits <= 1) return e;
+  combine_kernel<<<dim3(B, Hq), kD, 0, s>>>(part, num_splits, Hq, static_cast<uint16_t*>(out), lse);
+  return cudaPeekAtLastError();
+}
+
+}  // namespace qsa

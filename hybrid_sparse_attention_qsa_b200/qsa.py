@@ -1,0 +1,293 @@
+"""ctypes binding of libqsa_b200.so (include/qsa.h).
+
+Argument marshalling only: every step of the path runs in the library's CUDA kernels.  PyTorch
+supplies device memory (``data_ptr()``) and the current CUDA stream.  There is no fallback: if the
+library is missing or the call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libqsa_b200.so")
+
+QSA_OK = 0
+QSA_ERR_INVALID_ARGUMENT = 1
+QSA_ERR_UNSUPPORTED = 2
+QSA_ERR_WORKSPACE_TOO_SMALL = 3
+QSA_ERR_CUDA = 4
+QSA_ERR_TIMEOUT = 5
+
+QSA_SCORE_RELU_SUM = 0
+QSA_SCORE_LINEAR = 1
+
+QSA_OP_SELECT_TOPK = 1
+QSA_OP_SPARSE_ATTN_DECODE = 2
+
+# name -> (restype, argtypes), in the order of include/qsa.h
+_P, _I, _I64, _F, _SZ, _U64 = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t,
+                               ctypes.c_uint64)
+SIGNATURES = {
+    "qsa_status_string": (ctypes.c_char_p, [_I]),
+    "qsa_abi_version": (_I, []),
+    "qsa_pool_block_keys": (_I, [_P, _P, _I, _I, _I, _I, _F, _I64, _I64, _I64, _P]),
+    "qsa_rope_index_queries": (_I, [_P, _P, _I, _I, _I, _I, _I64, _P, _F, _P]),
+    "qsa_index_score": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I64, _I, _P, _I64, _P]),
+    "qsa_select_topk": (_I, [_P, _I64, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I64, _I, _I, _P, _P, _SZ, _P]),
+    "qsa_sparse_attn_prefill": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I64, _F, _P, _P, _P]),
+    "qsa_sparse_attn_decode": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P, _P, _P, _SZ, _P]),
+    "qsa_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I, _I]),
+    "qsa_decode_default_splits": (_I, [_I, _I]),
+    "qsa_get_device_status": (_I, [_P]),
+    "qsa_set_wait_timeout_ns": (None, [_U64]),
+    "qsa_wait_timeout_selftest": (_I, [_U64, _P]),
+}
+
+_lib = None
+
+
+class QSAError(RuntimeError):
+    def __init__(self, status: int, call: str):
+        self.status = status
+        super().__init__(f"{call} failed: {status_string(status)} ({status})")
+
+
+def lib():
+    """Load the library once.  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m hybrid_sparse_attention_qsa_b200.build`"
+                               " (or __graft_entry__.build()); there is no fallback path")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().qsa_status_string(status).decode()
+
+
+def _check(status: int, call: str):
+    if status != QSA_OK:
+        raise QSAError(status, call)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _need(t: torch.Tensor, dtype, name: str):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+# ---------------------------------------------------------------------------------------- ABI calls
+def qsa_abi_version() -> int:
+    return lib().qsa_abi_version()
+
+
+def _batch_view_ok(t: torch.Tensor) -> bool:
+    """[B, rows, Di] whose rows are packed inside each batch element (batch stride free)."""
+    return t.dim() == 3 and t.stride(2) == 1 and t.stride(1) == t.shape[2]
+
+
+def qsa_pool_block_keys(ki: torch.Tensor, kp: torch.Tensor | None = None, *, blk: int = 4, rope_theta: float = 0.0,
+                        pos0: int = 0) -> torch.Tensor:
+    """ki [B, L, Di] bf16 -> kp [B, L // blk, Di] bf16.  ki and kp may be batch-strided views (for
+    example the newest block of every sequence of a decode cache: ki[:, 4j:4j+4], kp[:, j:j+1])."""
+    if not ki.is_cuda or ki.dtype != torch.bfloat16 or not _batch_view_ok(ki):
+        raise ValueError("ki must be a CUDA bf16 [B, L, Di] tensor with packed rows")
+    B, L, Di = ki.shape
+    if kp is None:
+        kp = torch.empty(B, L // blk, Di, dtype=torch.bfloat16, device=ki.device)
+    if kp.dtype != torch.bfloat16 or not _batch_view_ok(kp) or tuple(kp.shape) != (B, L // blk, Di):
+        raise ValueError("kp must be a bf16 [B, L // blk, Di] tensor with packed rows")
+    _check(lib().qsa_pool_block_keys(_ptr(ki), _ptr(kp), B, L, Di, blk, rope_theta, pos0, ki.stride(0), kp.stride(0),
+                                     _stream(ki.device)), "qsa_pool_block_keys")
+    return kp
+
+
+def qsa_rope_index_queries(qi: torch.Tensor, qi_out: torch.Tensor | None = None, *, rope_theta: float, q_pos0: int = 0,
+                           seqlens: torch.Tensor | None = None) -> torch.Tensor:
+    """qi [B, Tq, Hi, Di] (or [B, Hi, Di] with seqlens) rotated at its positions."""
+    _need(qi, torch.bfloat16, "qi")
+    if seqlens is not None:
+        _need(seqlens, torch.int32, "seqlens")
+        B, Hi, Di = qi.shape
+        Tq = 1
+    else:
+        B, Tq, Hi, Di = qi.shape
+    if qi_out is None:
+        qi_out = torch.empty_like(qi)
+    _check(lib().qsa_rope_index_queries(_ptr(qi), _ptr(qi_out), B, Tq, Hi, Di, q_pos0, _ptr(seqlens), rope_theta,
+                                        _stream(qi.device)), "qsa_rope_index_queries")
+    return qi_out
+
+
+def qsa_index_score(qi: torch.Tensor, kp: torch.Tensor, *, head_w: torch.Tensor | None = None,
+                    seqlens: torch.Tensor | None = None, q_pos0: int = 0, mode: int = QSA_SCORE_RELU_SUM,
+                    scores: torch.Tensor | None = None, blk: int = 4) -> torch.Tensor:
+    """Prefill: qi [B, Tq, Hi, Di]; decode: qi [B, Hi, Di] with seqlens [B].  kp [B, NBk, Di].
+    Returns scores [B, Tq, NBk] fp32 (entries beyond each query's candidates are left as they were)."""
+    _need(qi, torch.bfloat16, "qi")
+    _need(kp, torch.bfloat16, "kp")
+    if seqlens is not None:
+        _need(seqlens, torch.int32, "seqlens")
+        B, Hi, Di = qi.shape
+        Tq = 1
+    else:
+        B, Tq, Hi, Di = qi.shape
+    NBk = kp.shape[1]
+    if scores is None:
+        scores = torch.full((B, Tq, max(NBk, 1)), float("nan"), dtype=torch.float32, device=qi.device)
+    _need(scores, torch.float32, "scores")
+    if head_w is not None:
+        _need(head_w, torch.float32, "head_w")
+    _check(lib().qsa_index_score(_ptr(qi), _ptr(kp), _ptr(head_w), _ptr(seqlens), B, Tq, NBk, Hi, Di, blk, q_pos0,
+                                 mode, _ptr(scores), scores.shape[-1], _stream(qi.device)), "qsa_index_score")
+    return scores
+
+
+def qsa_workspace_size(op: int, B: int, Tq: int, NBk: int, k: int, Hq: int, D: int, num_splits: int = 0) -> int:
+    return int(lib().qsa_workspace_size(op, B, Tq, NBk, k, Hq, D, num_splits))
+
+
+def qsa_select_topk(k: int, *, scores: torch.Tensor | None = None, qi: torch.Tensor | None = None,
+                    kp: torch.Tensor | None = None, head_w: torch.Tensor | None = None,
+                    seqlens: torch.Tensor | None = None, q_pos0: int = 0, mode: int = QSA_SCORE_RELU_SUM,
+                    NBk: int | None = None, idx: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                    blk: int = 4) -> torch.Tensor:
+    """Top-k block lists idx [B, Tq, k] int32 (decode: [B, k]).
+
+    From materialised ``scores`` [B, Tq, ld] (then NBk must be given or defaults to ld), or from
+    ``qi``/``kp`` with the scores computed chunk-wise in ``workspace`` (allocated if omitted)."""
+    ref = scores if scores is not None else qi
+    dev = ref.device
+    if scores is not None:
+        _need(scores, torch.float32, "scores")
+        B, Tq, ld = scores.shape
+        NBk = ld if NBk is None else NBk
+        Hi = Di = 0
+    else:
+        _need(qi, torch.bfloat16, "qi")
+        _need(kp, torch.bfloat16, "kp")
+        if seqlens is not None:
+            B, Hi, Di = qi.shape
+            Tq = 1
+        else:
+            B, Tq, Hi, Di = qi.shape
+        NBk = kp.shape[1]
+        ld = 0
+        if workspace is None:
+            nbytes = qsa_workspace_size(QSA_OP_SELECT_TOPK, B, Tq, NBk, k, 0, 0)
+            workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    if seqlens is not None:
+        _need(seqlens, torch.int32, "seqlens")
+    if idx is None:
+        idx = torch.empty((B, k) if seqlens is not None else (B, Tq, k), dtype=torch.int32, device=dev)
+    _need(idx, torch.int32, "idx")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().qsa_select_topk(_ptr(scores), ld, _ptr(qi), _ptr(kp), _ptr(head_w), _ptr(seqlens), B, Tq, NBk, Hi,
+                                 Di, blk, q_pos0, mode, k, _ptr(idx), _ptr(workspace), ws_bytes, _stream(dev)),
+           "qsa_select_topk")
+    return idx
+
+
+def qsa_sparse_attn_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, idx: torch.Tensor, *, q_pos0: int = 0,
+                            scale: float | None = None, out: torch.Tensor | None = None,
+                            lse: torch.Tensor | None = None, want_lse: bool = True, blk: int = 4):
+    """q [B, Tq, Hq, D], k/v [B, Tk, Hkv, D], idx [B, Tq, kb] -> (out [B, Tq, Hq, D], lse [B, Tq, Hq])."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, torch.bfloat16, n)
+    _need(idx, torch.int32, "idx")
+    B, Tq, Hq, D = q.shape
+    Tk, Hkv = k.shape[1], k.shape[2]
+    kb = idx.shape[-1]
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty(B, Tq, Hq, dtype=torch.float32, device=q.device)
+    _check(lib().qsa_sparse_attn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(idx), B, Tq, Tk, Hq, Hkv, D, kb, blk, q_pos0,
+                                         scale, _ptr(out), _ptr(lse), _stream(q.device)), "qsa_sparse_attn_prefill")
+    return out, lse
+
+
+def qsa_sparse_attn_decode(q: torch.Tensor, kcache: torch.Tensor, vcache: torch.Tensor, seqlens: torch.Tensor,
+                           idx: torch.Tensor, *, scale: float | None = None, num_splits: int = 0,
+                           out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+                           workspace: torch.Tensor | None = None, want_lse: bool = True, blk: int = 4):
+    """q [B, Hq, D], caches [B, Lmax, Hkv, D], seqlens [B], idx [B, kb] -> (out [B, Hq, D], lse [B, Hq])."""
+    for t, n in ((q, "q"), (kcache, "kcache"), (vcache, "vcache")):
+        _need(t, torch.bfloat16, n)
+    _need(seqlens, torch.int32, "seqlens")
+    _need(idx, torch.int32, "idx")
+    B, Hq, D = q.shape
+    Lmax, Hkv = kcache.shape[1], kcache.shape[2]
+    kb = idx.shape[-1]
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty(B, Hq, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        nbytes = qsa_workspace_size(QSA_OP_SPARSE_ATTN_DECODE, B, 1, 0, kb, Hq, D, num_splits)
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib().qsa_sparse_attn_decode(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(seqlens), _ptr(idx), B, Lmax, Hq, Hkv,
+                                        D, kb, blk, scale, num_splits, _ptr(out), _ptr(lse), _ptr(workspace), ws_bytes,
+                                        _stream(q.device)), "qsa_sparse_attn_decode")
+    return out, lse
+
+
+def qsa_get_device_status(device=None) -> int:
+    """Synchronise the current stream and read + clear the device status word."""
+    return int(lib().qsa_get_device_status(_stream(device)))
+
+
+def qsa_set_wait_timeout_ns(ns: int) -> None:
+    lib().qsa_set_wait_timeout_ns(ns)
+
+
+def qsa_wait_timeout_selftest(timeout_ns: int, device=None) -> None:
+    _check(lib().qsa_wait_timeout_selftest(timeout_ns, _stream(device)), "qsa_wait_timeout_selftest")
+
+
+# ---------------------------------------------------------------------------------------- whole path
+def prefill(q, k, v, qi, ki, *, topk: int, q_pos0: int = 0, rope_theta: float = 0.0, head_w=None,
+            mode: int = QSA_SCORE_RELU_SUM, scale: float | None = None, workspace=None, kp=None):
+    """The QSA layer for a prefill: pool (+RoPE) -> [RoPE queries] -> score + top-k -> sparse attention.
+    Returns dict(out, lse, idx, kp)."""
+    if kp is None:
+        kp = qsa_pool_block_keys(ki, rope_theta=rope_theta)
+    qr = qsa_rope_index_queries(qi, rope_theta=rope_theta, q_pos0=q_pos0) if rope_theta > 0 else qi
+    idx = qsa_select_topk(topk, qi=qr, kp=kp, head_w=head_w, q_pos0=q_pos0, mode=mode, workspace=workspace)
+    out, lse = qsa_sparse_attn_prefill(q, k, v, idx, q_pos0=q_pos0, scale=scale)
+    return dict(out=out, lse=lse, idx=idx, kp=kp)
+
+
+def decode(q, kcache, vcache, qi, kp, seqlens, *, topk: int, rope_theta: float = 0.0, head_w=None,
+           mode: int = QSA_SCORE_RELU_SUM, scale: float | None = None, num_splits: int = 0, workspace=None):
+    """One decode step on a pooled indexer-key cache kp [B, NBk, Di]: [RoPE query] -> score + top-k
+    -> split-KV sparse attention.  Returns dict(out, lse, idx)."""
+    qr = qsa_rope_index_queries(qi, rope_theta=rope_theta, seqlens=seqlens) if rope_theta > 0 else qi
+    idx = qsa_select_topk(topk, qi=qr, kp=kp, head_w=head_w, seqlens=seqlens, mode=mode, workspace=workspace)
+    out, lse = qsa_sparse_attn_decode(q, kcache, vcache, seqlens, idx, scale=scale, num_splits=num_splits)
+    return dict(out=out, lse=lse, idx=idx)

@@ -1,0 +1,218 @@
+/*
+ * qsa.h -- C ABI of the B200 (sm_100a) Qwen Sparse Attention (QSA) hot path.
+ *
+ * The method (from "Qwen3.8-Flash-Next architecture", flozi.net, section "Der Weg eines Tokens
+ * durch das Modell", item 2 "Die zwei Stufen von QSA"; and "Qwen3.8-Flash-Next", studioglobal.ai,
+ * section "Hybride Aufmerksamkeit fuer sehr lange Kontexte"):
+ *   1. an indexer maps tokens to light keys; groups of `blk` (= 4) consecutive keys are averaged
+ *      into one micro-block key, and RoPE is applied after the averaging;
+ *   2. every query is scored against its causally visible micro-blocks with Hi (= 4) indexer
+ *      query heads sharing one key head;
+ *   3. each query keeps its top-k blocks (k = 512 blocks = 2048 tokens) plus its own, possibly
+ *      incomplete, block;
+ *   4. exact softmax attention (GQA) runs over only the tokens of the kept blocks.
+ * Readings where the pages leave a step open (all fixed here, and in the CPU oracle):
+ *   - score s(t,b) = sum_h w_h * max(0, qi[t,h] . kp[b])  (QSA_SCORE_LINEAR drops the max);
+ *   - the candidates of the query at position p are the complete blocks b < floor(p/blk); the own
+ *     block (tokens blk*floor(p/blk) .. p) is always attended and never scored;
+ *   - top-k is taken on the fp32 scores; equal scores go to the lower block index; the list is
+ *     ascending and padded with -1 when fewer than k candidates exist;
+ *   - one index list per query, shared by all attention heads (one shared key head);
+ *   - pooled keys and rotated indexer queries are stored as bf16 (round to nearest even);
+ *   - RoPE is the half-split rotation of pairs (i, i + Di/2) by pos * theta^(-2i/Di); a pooled key
+ *     sits at the position of its block's first token.
+ *
+ * Conventions for every call:
+ *   - All tensor pointers are caller-owned, contiguous, 16-byte-aligned DEVICE memory; bf16
+ *     tensors are passed as `const void*` / `void*` (bf16 bit patterns).  Layouts are given per
+ *     call, outermost dimension first.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Work is enqueued on it
+ *     asynchronously; no call synchronises except qsa_get_device_status.  No call allocates
+ *     device memory; scratch memory comes from the caller's `workspace`.
+ *   - Arguments are checked on the host before any launch.  On a non-QSA_OK return nothing was
+ *     launched and no output was touched (QSA_ERR_CUDA: a launch was rejected by the runtime).
+ *   - Faults found on the device (an index list entry outside its query's causal range, a
+ *     sequence length outside the cache, a wait that ran out of time) are skipped by the kernel
+ *     and recorded in a per-device status word that qsa_get_device_status reads and clears.
+ *   - Supported shapes: blk = 4; Di = 64 for scoring (any even Di <= 256 for pooling/RoPE);
+ *     Hi in {1, 2, 4, 8}; attention D = 128, Hkv in {1, 2}, Hq/Hkv <= 8.  Other shapes return
+ *     QSA_ERR_UNSUPPORTED.
+ *   - Calls are thread-safe.  The library keeps only per-device caches (device attributes, the
+ *     status word) and no other mutable global state.
+ */
+#ifndef QSA_H
+#define QSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define QSA_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define QSA_API __attribute__((visibility("default")))
+#else
+#define QSA_API
+#endif
+
+typedef enum {
+  QSA_OK = 0,
+  QSA_ERR_INVALID_ARGUMENT = 1,    /* null pointer, negative size, misaligned pointer, bad index */
+  QSA_ERR_UNSUPPORTED = 2,         /* a shape outside the supported set above */
+  QSA_ERR_WORKSPACE_TOO_SMALL = 3, /* ws_bytes below what the call needs */
+  QSA_ERR_CUDA = 4,                /* the CUDA runtime rejected a launch or query */
+  QSA_ERR_TIMEOUT = 5              /* a device-side wait ran out of time (device status only) */
+} qsa_status_t;
+
+typedef enum {
+  QSA_SCORE_RELU_SUM = 0, /* s = sum_h w_h * max(0, qi_h . kp)   (the QSA indexer) */
+  QSA_SCORE_LINEAR = 1    /* s = sum_h w_h * (qi_h . kp)          (test mode: one GEMM) */
+} qsa_score_mode_t;
+
+typedef enum {
+  QSA_OP_SELECT_TOPK = 1,       /* qsa_select_topk with scores == NULL */
+  QSA_OP_SPARSE_ATTN_DECODE = 2 /* qsa_sparse_attn_decode with num_splits > 1 */
+} qsa_op_t;
+
+/* Human-readable name of a status code (static string, never NULL). */
+QSA_API const char* qsa_status_string(qsa_status_t status);
+
+/* QSA_ABI_VERSION of the loaded library. */
+QSA_API int qsa_abi_version(void);
+
+/*
+ * Micro-block key pooling (step 1: mean of each group of four keys, then RoPE).
+ *   ki [B][L][Di] bf16  ->  kp [B][floor(L/blk)][Di] bf16
+ *   kp[b][j] = bf16( rope( (1/blk) * sum_{i<blk} ki[b][blk*j + i], pos0 + blk*j ) )
+ * The mean is formed exactly (double) and rounded once to bf16.  rope_theta <= 0 disables RoPE.
+ * A trailing partial group (L mod blk tokens) is not pooled.  Batch strides are in elements
+ * (0 = packed: L*Di for ki, floor(L/blk)*Di for kp), so a decode step can pool the newest block
+ * j of every sequence of a [B][Lmax][Di] cache in one call: ki = &ki[0][blk*j][0], L = blk,
+ * ki_batch_stride = Lmax*Di, kp = &kp[0][j][0], kp_batch_stride = NBk*Di, pos0 = blk*j.
+ * Errors: INVALID_ARGUMENT (null, B/L < 0, Di odd or > 256), UNSUPPORTED (blk != 4).
+ */
+QSA_API qsa_status_t qsa_pool_block_keys(const void* ki, void* kp, int B, int L, int Di, int blk,
+                                         float rope_theta, int64_t pos0, int64_t ki_batch_stride,
+                                         int64_t kp_batch_stride, void* stream);
+
+/*
+ * RoPE of the indexer queries at their own positions (the query side of the rotation that the
+ * keys receive after pooling).
+ *   qi [B][Tq][Hi][Di] bf16 -> qi_out (same layout; may alias qi)
+ *   row t of batch b sits at position q_pos0 + t, or at seqlens[b] - 1 when seqlens != NULL
+ *   (decode: Tq must be 1).  Call it before qsa_index_score / qsa_select_topk when RoPE is on.
+ * Errors: INVALID_ARGUMENT (null, sizes, Di odd or > 256, rope_theta <= 0).
+ */
+QSA_API qsa_status_t qsa_rope_index_queries(const void* qi, void* qi_out, int B, int Tq, int Hi, int Di,
+                                    int64_t q_pos0, const int32_t* seqlens, float rope_theta,
+                                    void* stream);
+
+/*
+ * Indexer block scores (step 2: four indexer query heads against one shared key head).
+ *   qi [B][Tq][Hi][Di] bf16 (already rotated if RoPE is used), kp [B][NBk][Di] bf16,
+ *   head_w [Hi] fp32 or NULL (all ones)  ->  scores [B][Tq][ld_scores] fp32:
+ *   scores[b][t][j] = s(t, j) for j < NB(p) = floor(p/blk), p = q_pos0 + t (or seqlens[b]-1 with
+ *   seqlens != NULL, Tq == 1).  Entries j >= NB(p) are not written.
+ * Prefill runs on tcgen05 tensor cores (TMEM accumulators, TMA-fed); decode (seqlens != NULL)
+ * is a bandwidth-bound CUDA-core pass over the pooled-key cache.
+ * Requires floor((q_pos0 + Tq - 1)/blk) <= NBk (prefill) and ld_scores >= NBk.
+ * Errors: INVALID_ARGUMENT, UNSUPPORTED (Di != 64, Hi not in {1,2,4,8}, blk != 4).
+ */
+QSA_API qsa_status_t qsa_index_score(const void* qi, const void* kp, const float* head_w,
+                             const int32_t* seqlens, int B, int Tq, int NBk, int Hi, int Di,
+                             int blk, int64_t q_pos0, qsa_score_mode_t mode, float* scores,
+                             int64_t ld_scores, void* stream);
+
+/*
+ * Per-query top-k block selection (step 3: a budget of 512 whole blocks, i.e. 2048 tokens).
+ *   -> idx [B][Tq][k] int32: the k candidates with the largest fp32 score (equal scores: lower
+ *   index first), in ascending block order, -1 padded when NB(p) < k.  The own block is never
+ *   listed (it is implicit).
+ * scores != NULL: select from scores [B][Tq][ld_scores] (as written by qsa_index_score); qi, kp,
+ *   head_w, mode and workspace are ignored.
+ * scores == NULL: the scores are computed here, chunk by chunk, into `workspace` (at least one
+ *   score row of NBk floats; qsa_workspace_size(QSA_OP_SELECT_TOPK, ...) gives the size that lets
+ *   the whole call run in few chunks).  Arguments as for qsa_index_score.
+ * Errors: INVALID_ARGUMENT (k < 1, ...), UNSUPPORTED, WORKSPACE_TOO_SMALL.
+ */
+QSA_API qsa_status_t qsa_select_topk(const float* scores, int64_t ld_scores, const void* qi,
+                             const void* kp, const float* head_w, const int32_t* seqlens, int B,
+                             int Tq, int NBk, int Hi, int Di, int blk, int64_t q_pos0,
+                             qsa_score_mode_t mode, int k, int32_t* idx, void* workspace,
+                             size_t ws_bytes, void* stream);
+
+/*
+ * Gather-sparse attention, prefill (step 4: exact attention over the selected tokens, GQA).
+ *   q [B][Tq][Hq][D] bf16 for positions q_pos0 .. q_pos0+Tq-1 (q_pos0 + Tq <= Tk),
+ *   k, v [B][Tk][Hkv][D] bf16, idx [B][Tq][k_blocks] int32 (from qsa_select_topk; entries -1
+ *   and entries equal to the own block are skipped; other entries outside [0, own) are skipped
+ *   and flagged in the device status)  ->  out [B][Tq][Hq][D] bf16,
+ *   lse [B][Tq][Hq] fp32 (natural-log log-sum-exp of the scaled logits; may be NULL).
+ *   o(t,h) = sum_{j in S(t)} softmax_j(scale * q(t,h) . k(j,g)) v(j,g),  g = h / (Hq/Hkv),
+ *   S(t) = tokens of the listed blocks  U  { blk*floor(p/blk) .. p }.
+ * The softmax is kept in fp32 (online, exp2 form); products run on bf16 tensor cores.
+ * Errors: INVALID_ARGUMENT, UNSUPPORTED (D != 128, Hkv not in {1,2}, Hq/Hkv > 8, blk != 4).
+ */
+QSA_API qsa_status_t qsa_sparse_attn_prefill(const void* q, const void* k, const void* v,
+                                     const int32_t* idx, int B, int Tq, int Tk, int Hq, int Hkv,
+                                     int D, int k_blocks, int blk, int64_t q_pos0, float scale,
+                                     void* out, float* lse, void* stream);
+
+/*
+ * Gather-sparse attention, decode (split-KV).  One new token per sequence.
+ *   q [B][Hq][D] bf16; caches k, v [B][Lmax][Hkv][D] bf16 holding seqlens[b] tokens (the new
+ *   token included, so the query sits at position seqlens[b] - 1); idx [B][k_blocks] int32
+ *   -> out [B][Hq][D] bf16, lse [B][Hq] fp32 (may be NULL).
+ * The index list of each sequence is cut into num_splits ranges (0 = choose from the GPU size)
+ * that run in parallel; their partial softmax states are merged by log-sum-exp.  num_splits > 1
+ * needs workspace >= qsa_workspace_size(QSA_OP_SPARSE_ATTN_DECODE, B, 1, 0, k_blocks, Hq, D,
+ * num_splits) bytes.
+ * Errors: as for prefill, plus WORKSPACE_TOO_SMALL.
+ */
+QSA_API qsa_status_t qsa_sparse_attn_decode(const void* q, const void* kcache, const void* vcache,
+                                    const int32_t* seqlens, const int32_t* idx, int B, int Lmax,
+                                    int Hq, int Hkv, int D, int k_blocks, int blk, float scale,
+                                    int num_splits, void* out, float* lse, void* workspace,
+                                    size_t ws_bytes, void* stream);
+
+/*
+ * Workspace bytes for `op`.  QSA_OP_SELECT_TOPK: B, Tq, NBk (a chunk of score rows, capped);
+ * QSA_OP_SPARSE_ATTN_DECODE: B, Hq, D, num_splits (0 = the count the call would choose).
+ * Returns 0 for an unknown op or invalid sizes.
+ */
+QSA_API size_t qsa_workspace_size(qsa_op_t op, int B, int Tq, int NBk, int k, int Hq, int D,
+                          int num_splits);
+
+/* Split count qsa_sparse_attn_decode picks for num_splits == 0 on the current device. */
+QSA_API int qsa_decode_default_splits(int B, int k_blocks);
+
+/*
+ * Synchronises `stream`, then reads and clears the current device's status word:
+ * QSA_OK, QSA_ERR_INVALID_ARGUMENT (an index or sequence length was out of range and skipped),
+ * QSA_ERR_TIMEOUT (a device-side wait ran out of time and the kernel returned early), or
+ * QSA_ERR_CUDA (the synchronisation itself failed).
+ */
+QSA_API qsa_status_t qsa_get_device_status(void* stream);
+
+/*
+ * Device-side wait limit in nanoseconds for all later launches from this process (default
+ * 2e9 = 2 s; 0 restores the default).  Every spin on an mbarrier in the kernels gives up after
+ * this long, records QSA_ERR_TIMEOUT and returns.
+ */
+QSA_API void qsa_set_wait_timeout_ns(uint64_t ns);
+
+/*
+ * Self-test of the bounded waits: launches one CTA that waits on an mbarrier no thread ever
+ * completes, with a `timeout_ns` limit.  Afterwards qsa_get_device_status returns
+ * QSA_ERR_TIMEOUT and the context stays usable.
+ */
+QSA_API qsa_status_t qsa_wait_timeout_selftest(uint64_t timeout_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QSA_H */

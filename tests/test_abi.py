@@ -1,0 +1,109 @@
+"""The C-ABI library: it loads without a GPU, exports every symbol include/qsa.h declares, and
+rejects bad arguments on the host before any launch (no GPU needed for those paths)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from hybrid_sparse_attention_qsa_b200 import build as B
+from hybrid_sparse_attention_qsa_b200 import qsa as Q
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return Q.lib()
+
+
+def declared_symbols():
+    src = open(os.path.join(ROOT, "include", "qsa.h")).read()
+    return sorted(set(re.findall(r"QSA_API\s+[\w\s\*]+?\b(qsa_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_four_hot_path_calls():
+    names = declared_symbols()
+    for n in ("qsa_index_score", "qsa_select_topk", "qsa_sparse_attn_prefill", "qsa_sparse_attn_decode",
+              "qsa_pool_block_keys"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = declared_symbols()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(Q.SIGNATURES), "binding and header disagree"
+
+
+def test_abi_version_and_status_strings(lib):
+    assert Q.qsa_abi_version() == 1
+    assert Q.status_string(Q.QSA_ERR_WORKSPACE_TOO_SMALL) == "QSA_ERR_WORKSPACE_TOO_SMALL"
+    assert Q.status_string(99) == "QSA_ERR_UNKNOWN"
+
+
+P = ctypes.c_void_p
+FAKE = P(1 << 20)          # never dereferenced: every call below fails its host-side checks
+
+
+def test_pool_argument_checks(lib):
+    assert lib.qsa_pool_block_keys(None, None, 1, 8, 64, 4, 0.0, 0, 0, 0, None) == Q.QSA_ERR_INVALID_ARGUMENT
+    assert lib.qsa_pool_block_keys(FAKE, FAKE, 1, 8, 63, 4, 0.0, 0, 0, 0, None) == Q.QSA_ERR_INVALID_ARGUMENT
+    assert lib.qsa_pool_block_keys(FAKE, FAKE, 1, 8, 64, 3, 0.0, 0, 0, 0, None) == Q.QSA_ERR_UNSUPPORTED
+    assert lib.qsa_pool_block_keys(P(17), FAKE, 1, 8, 64, 4, 0.0, 0, 0, 0, None) == Q.QSA_ERR_INVALID_ARGUMENT
+    assert lib.qsa_pool_block_keys(None, None, 0, 8, 64, 4, 0.0, 0, 0, 0, None) == Q.QSA_OK      # empty: nothing to do
+    assert lib.qsa_pool_block_keys(None, None, 1, 3, 64, 4, 0.0, 0, 0, 0, None) == Q.QSA_OK      # no complete block
+
+
+def test_score_argument_checks(lib):
+    args = lambda **kw: dict(dict(qi=FAKE, kp=FAKE, w=None, sl=None, B=1, Tq=8, NBk=2, Hi=4, Di=64, blk=4, q0=0, mode=0,
+                                  s=FAKE, ld=2), **kw)
+
+    def call(**kw):
+        a = args(**kw)
+        return lib.qsa_index_score(a["qi"], a["kp"], a["w"], a["sl"], a["B"], a["Tq"], a["NBk"], a["Hi"], a["Di"],
+                                   a["blk"], a["q0"], a["mode"], a["s"], a["ld"], None)
+
+    assert call(Di=128) == Q.QSA_ERR_UNSUPPORTED
+    assert call(Hi=3) == Q.QSA_ERR_UNSUPPORTED
+    assert call(mode=2) == Q.QSA_ERR_INVALID_ARGUMENT
+    # row 11 has 2 candidates and kp holds NBk = 2 rows: valid; row 12 would need 3
+    assert call(Tq=13, NBk=2) == Q.QSA_ERR_INVALID_ARGUMENT   # ... row 12 needs 3 > NBk = 2
+    assert call(q0=5, Tq=8) == Q.QSA_ERR_INVALID_ARGUMENT      # row at position 12 again
+    assert call(ld=1) == Q.QSA_ERR_INVALID_ARGUMENT
+    assert call(sl=FAKE, Tq=2) == Q.QSA_ERR_INVALID_ARGUMENT
+    assert call(qi=P(8)) == Q.QSA_ERR_INVALID_ARGUMENT
+
+
+def test_select_and_attention_argument_checks(lib):
+    # k < 1
+    assert lib.qsa_select_topk(FAKE, 8, None, None, None, None, 1, 4, 8, 4, 64, 4, 0, 0, 0, FAKE, None, 0,
+                               None) == Q.QSA_ERR_INVALID_ARGUMENT
+    # scores == NULL needs a workspace
+    assert lib.qsa_select_topk(None, 0, FAKE, FAKE, None, None, 1, 40, 10, 4, 64, 4, 0, 0, 8, FAKE, None, 0,
+                               None) == Q.QSA_ERR_WORKSPACE_TOO_SMALL
+    # decode with too small a workspace
+    assert lib.qsa_select_topk(None, 0, FAKE, FAKE, None, FAKE, 2, 1, 10, 4, 64, 4, 0, 0, 8, FAKE, FAKE, 40,
+                               None) == Q.QSA_ERR_WORKSPACE_TOO_SMALL
+    pre = lambda D=128, Hq=16, Hkv=2, blk=4, Tq=8, Tk=8, q0=0: lib.qsa_sparse_attn_prefill(
+        FAKE, FAKE, FAKE, FAKE, 1, Tq, Tk, Hq, Hkv, D, 8, blk, q0, ctypes.c_float(0.1), FAKE, None, None)
+    assert pre(D=64) == Q.QSA_ERR_UNSUPPORTED
+    assert pre(Hkv=4, Hq=16) == Q.QSA_ERR_UNSUPPORTED
+    assert pre(Hq=24, Hkv=2) == Q.QSA_ERR_UNSUPPORTED        # group of 12: the d=256 / 24-head shape is not built
+    assert pre(Hq=15, Hkv=2) == Q.QSA_ERR_INVALID_ARGUMENT
+    assert pre(blk=8) == Q.QSA_ERR_UNSUPPORTED
+    assert pre(q0=4) == Q.QSA_ERR_INVALID_ARGUMENT           # q0 + Tq > Tk
+    dec = lambda ws, nbytes, splits: lib.qsa_sparse_attn_decode(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 100, 16, 2, 128, 64, 4,
+                                                                ctypes.c_float(0.1), splits, FAKE, None, ws, nbytes,
+                                                                None)
+    assert dec(None, 0, -1) == Q.QSA_ERR_INVALID_ARGUMENT
+
+
+def test_workspace_sizes(lib):
+    n = Q.qsa_workspace_size(Q.QSA_OP_SELECT_TOPK, 1, 131072, 32768, 512, 16, 128)
+    assert n >= 32768 * 4 and n <= 512 << 20 and n % (32768 * 4) == 0
+    assert Q.qsa_workspace_size(Q.QSA_OP_SELECT_TOPK, 32, 1, 65536, 512, 16, 128) == 32 * 65536 * 4
+    assert Q.qsa_workspace_size(Q.QSA_OP_SPARSE_ATTN_DECODE, 32, 1, 0, 512, 16, 128, 5) == 32 * 5 * 16 * 130 * 4
+    assert Q.qsa_workspace_size(99, 1, 1, 1, 1, 1, 1) == 0
