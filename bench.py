@@ -344,12 +344,18 @@ def run_qsa(args):
         ki_last = xd["ki"][:, j * wd.blk:(j + 1) * wd.blk]
         kp_last = kpd[:, j:j + 1]
 
-        def dstep():
+        def dstep(ev=None):
             if (wd.T % wd.blk) == 0:       # the new token completed block j: pool that row of every sequence
                 Q.qsa_pool_block_keys(ki_last, kp_last, pos0=j * wd.blk)
+            if ev:
+                ev[0].record(stream)
             Q.qsa_select_topk(wd.k, qi=xd["qi"], kp=kpd, seqlens=xd["seqlens"], idx=idxd, workspace=wsd)
+            if ev:
+                ev[1].record(stream)
             Q.qsa_sparse_attn_decode(xd["q"], xd["k"], xd["v"], xd["seqlens"], idxd, num_splits=splits, out=outd,
                                      lse=lsed, workspace=wsa)
+            if ev:
+                ev[2].record(stream)
 
         for _ in range(max(args.warmup, 3)):
             dstep()
@@ -364,10 +370,17 @@ def run_qsa(args):
         d1.record(stream)
         torch.cuda.synchronize()
         dms = max_over_ranks(d0.elapsed_time(d1), world, dev) / dsteps
+        devs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(5)]
+        for e in devs:
+            dstep(e)
+        torch.cuda.synchronize()
+        d_sel = statistics.mean(e[0].elapsed_time(e[1]) for e in devs)
+        d_att = statistics.mean(e[1].elapsed_time(e[2]) for e in devs)
         dw = decode_work(wd)
         dgbs = dw["bytes"] / (dms / 1000) / 1e9
         decode = {"workload": DECODE, "value": world * wd.B / (dms / 1000), "unit": "tokens/s", "ms_per_step": dms,
                   "steps": dsteps, "num_splits": splits,
+                  "step_breakdown_ms": {"score_topk": d_sel, "attention_and_merge": d_att},
                   "gpu_launches_per_step": 1 + 2 + 1 + (1 if splits > 1 else 0),
                   "roofline": {"bound": "hbm", "achieved": dgbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                                "frac": dgbs / pk["hbm_gbs"], "bytes_per_step": dw["bytes"],

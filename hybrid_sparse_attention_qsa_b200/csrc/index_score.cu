@@ -44,7 +44,7 @@ struct ScoreArgs {
   KernelCtl ctl;
 };
 
-template <int HI>
+template <int HI, int MODE>
 __global__ void __launch_bounds__(kScoreThreads, 1)
     score_prefill_kernel(const __grid_constant__ CUtensorMap qi_map, const __grid_constant__ CUtensorMap kp_map,
                          ScoreArgs a) {
@@ -154,32 +154,38 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     float w[HI];
 #pragma unroll
     for (int h = 0; h < HI; ++h) w[h] = a.head_w ? a.head_w[h] : 1.0f;
-    float* srow_base = a.scores + static_cast<long long>(bz) * a.batch_stride;
+    // Row tl of the tile sits at position pos_first + tl and has (pos_first + tl) >> 2 candidates
+    // (blk = 4).  Rows past r_last belong to the next window and are not written.
+    const long long pos_first = a.q_pos0 + r_first;
+    const int tl_last = r_last - r_first;
+    const int nbk = a.NBk;
+    float* srow = a.scores + static_cast<long long>(bz) * a.batch_stride + static_cast<long long>(r_first - a.row0) * a.ld;
+    const long long ld = a.ld;
     for (int i = 0; i < nt; ++i) {
       const int acc = i & 1;
       const unsigned aph = (i >> 1) & 1u;
       if (!mbar_wait(&tm_full[acc], aph, a.ctl)) break;
       tc_fence_after();
       const int kb = (t_begin + i) * kM + quad * 32 + lane;   // pooled key owned by this thread
+      float* col = srow + kb;
 #pragma unroll 1
       for (int c = 0; c < kN / 2; c += 32) {
         uint32_t r[32];
         tmem_ld_32x32(tmem + lane_addr + acc * kN + colbase + c, r);
         tmem_ld_wait();
+        const int q0 = (colbase + c) / HI;
 #pragma unroll
         for (int qq = 0; qq < 32 / HI; ++qq) {
-          const int row = r_first + (colbase + c) / HI + qq;
           float sc = 0.0f;
 #pragma unroll
           for (int h = 0; h < HI; ++h) {
             float x = __uint_as_float(r[qq * HI + h]);
-            if (a.mode == 0) x = fmaxf(x, 0.0f);
+            if (MODE == 0) x = fmaxf(x, 0.0f);
             sc = fmaf(w[h], x, sc);
           }
-          if (row <= r_last) {
-            const int nbq = static_cast<int>(min(static_cast<long long>(a.NBk), (a.q_pos0 + row) / a.blk));
-            if (kb < nbq) srow_base[static_cast<long long>(row - a.row0) * a.ld + kb] = sc;
-          }
+          const int tl = q0 + qq;
+          const int nbq = min(nbk, static_cast<int>((pos_first + tl) >> 2));
+          if (tl <= tl_last && kb < nbq) col[tl * ld] = sc;
         }
       }
       tc_fence_before();
@@ -313,7 +319,8 @@ cudaError_t launch_prefill_hi(const void* qi, const void* kp, const float* head_
   int dev = 0;
   cudaGetDevice(&dev);
   std::call_once(attr_once[dev & 63], [] {
-    cudaFuncSetAttribute(score_prefill_kernel<HI>, cudaFuncAttributeMaxDynamicSharedMemorySize, kScoreSmem);
+    cudaFuncSetAttribute(score_prefill_kernel<HI, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, kScoreSmem);
+    cudaFuncSetAttribute(score_prefill_kernel<HI, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kScoreSmem);
   });
   CUtensorMap qmap, kmap;
   // Maps span all batches so the batch index is a TMA coordinate.
@@ -328,7 +335,10 @@ cudaError_t launch_prefill_hi(const void* qi, const void* kp, const float* head_
   if (ntiles == 0) return cudaSuccess;
   dim3 grid((rows + QPT - 1) / QPT, (ntiles + kTilesPerCta - 1) / kTilesPerCta, nb);
   ScoreArgs a{head_w, scores, ld, batch_stride, q_pos0, NBk, blk, mode, b0, row0, rows, ctl};
-  score_prefill_kernel<HI><<<grid, kScoreThreads, kScoreSmem, s>>>(qmap, kmap, a);
+  if (mode == 0)
+    score_prefill_kernel<HI, 0><<<grid, kScoreThreads, kScoreSmem, s>>>(qmap, kmap, a);
+  else
+    score_prefill_kernel<HI, 1><<<grid, kScoreThreads, kScoreSmem, s>>>(qmap, kmap, a);
   return cudaPeekAtLastError();
 }
 

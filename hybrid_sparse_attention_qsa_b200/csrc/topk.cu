@@ -5,12 +5,22 @@
 // possibly incomplete, block.  Reading fixed in qsa.h: the top-k of the fp32 scores over the
 // candidates b < floor(p/blk), equal scores to the lower index, ascending output, -1 padded.
 //
-// One CTA per score row.  The k-th largest score is found exactly by a radix select on the
-// order-preserving 32-bit keys of the fp32 scores (three passes of 11, 11 and 10 bits over the
-// row, shared-memory histograms; the lanes of a warp that hit the same bin are merged with
-// match.any so one atomic per distinct bin is issued).  A final pass in index order emits every
-// key above the threshold and the first (k - #above) keys equal to it, with a block-wide scan for
-// the output positions, so the list comes out ascending without a sort.
+// One CTA per score row; the row is read from memory once on the fast path:
+//   1. a 2048-point sample of the row gives a threshold tau a little below the k-th largest
+//      score (its rank among the samples is chosen so that ~2.5k scores are expected above it);
+//   2. one coalesced pass collects every (key, index) with key >= tau into shared memory;
+//   3. an exact radix select on the candidates' order-preserving 32-bit keys gives the k-th key K*
+//      and how many keys equal to K* are taken; if equal keys must be split, a second radix select
+//      on their indices finds the largest index I* that is kept (lower index wins);
+//   4. the kept set {key > K*} U {key == K*, index <= I*} is marked in a shared bitmap of the row
+//      and emitted in ascending order by a block-wide scan of the bitmap's word counts.
+// Rows with at most `kCap` candidates skip steps 1-2.  If the threshold leaves fewer than k or more
+// than kCap candidates (heavy ties), it is moved and the pass retried; after that, or when the row
+// is too long for the bitmap, an exact three-pass radix select over the row in memory is used.
+// Lanes of a warp that hit the same histogram bin are merged with match.any (one atomic per bin).
+#include <algorithm>
+#include <mutex>
+
 #include "launch.h"
 
 namespace qsa {
@@ -18,14 +28,18 @@ namespace {
 
 constexpr int kTopkThreads = 512;
 constexpr int kWarps = kTopkThreads / 32;
-constexpr int kMaxBins = 2048;
+constexpr int kBins = 2048;
+constexpr int kCap = 6144;          // candidate capacity of the fast path
+constexpr int kSamples = 2048;
+constexpr int kMaxBitmapWords = 24576;   // rows up to 786432 candidates use the fast path
+constexpr int kFixedSmem = kCap * 8 + kBins * 4 + kSamples * 4 + (kWarps + 8) * 4;
 
 __device__ __forceinline__ uint32_t key_of(float s) {
   return score_key(s + 0.0f);   // -0 -> +0, so the two zeros compare equal as in fp32
 }
 
-// Exclusive scan of one value per thread over the block; returns the exclusive prefix and writes
-// the block total to *total.  Uses `ws` (kWarps + 1 words); ends with the block synchronised.
+// Exclusive scan of one value per thread over the block; returns the exclusive prefix and the
+// block total.  Uses `ws` (kWarps + 1 words); ends with the block synchronised.
 __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* ws, uint32_t* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint32_t x = v;
@@ -54,14 +68,140 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* ws, ui
   return r;
 }
 
+// Adds one histogram hit per lane with hit == true; lanes with the same digit share one atomic.
+__device__ __forceinline__ void hist_add(uint32_t* hist, bool hit, uint32_t digit) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t peers = __match_any_sync(0xffffffffu, hit ? digit : 0xFFFFFFFFu);
+  if (hit && lane == __ffs(peers) - 1) atomicAdd(&hist[digit], static_cast<uint32_t>(__popc(peers)));
+}
+
+// After a histogram of the current digit: find the bin holding the krem-th largest hit.  Writes
+// (bin, hits above the bin) to sel[0], sel[1].  All threads call it; ends synchronised.
+__device__ __forceinline__ void find_bin(const uint32_t* hist, int nbins, uint32_t krem, uint32_t* ws, uint32_t* sel) {
+  const int tid = threadIdx.x;
+  const int bpt = nbins / kTopkThreads;
+  uint32_t local = 0;
+  for (int q = 0; q < bpt; ++q) local += hist[tid * bpt + q];
+  uint32_t total;
+  const uint32_t excl = block_excl_scan(local, ws, &total);
+  const uint32_t above = total - excl - local;   // hits in the bins above this thread's range
+  if (above < krem && above + local >= krem) {
+    uint32_t acc = above;
+    for (int q = bpt - 1; q >= 0; --q) {
+      const uint32_t h = hist[tid * bpt + q];
+      if (acc + h >= krem) {
+        sel[0] = static_cast<uint32_t>(tid * bpt + q);
+        sel[1] = acc;
+        break;
+      }
+      acc += h;
+    }
+  }
+  __syncthreads();
+}
+
+// Radix select over values in shared memory: the krem-th largest of vals[0..m).  `passes` of the
+// (11, 11, 10)-bit digits are resolved from the top; unresolved low bits are returned as zero.
+// *left = how many values equal to the result (after the resolved bits) are still to be taken.
+__device__ uint32_t smem_select(const uint32_t* vals, int m, uint32_t krem, int passes, uint32_t* hist, uint32_t* ws,
+                                uint32_t* sel, uint32_t* left) {
+  const int shifts[3] = {21, 10, 0};
+  const int widths[3] = {11, 11, 10};
+  uint32_t prefix = 0, pmask = 0;
+  for (int pass = 0; pass < passes; ++pass) {
+    const int shift = shifts[pass], nbins = 1 << widths[pass];
+    const uint32_t dmask = static_cast<uint32_t>(nbins - 1);
+    for (int i = threadIdx.x; i < nbins; i += kTopkThreads) hist[i] = 0;
+    __syncthreads();
+    for (int base = 0; base < m; base += kTopkThreads) {
+      const int i = base + threadIdx.x;
+      const uint32_t v = i < m ? vals[i] : 0u;
+      const bool hit = i < m && (v & pmask) == prefix;
+      hist_add(hist, hit, (v >> shift) & dmask);
+    }
+    __syncthreads();
+    find_bin(hist, nbins, krem, ws, sel);
+    prefix |= sel[0] << shift;
+    pmask |= dmask << shift;
+    krem -= sel[1];
+    __syncthreads();
+  }
+  *left = krem;
+  return prefix;
+}
+
+// Exact fallback: three radix passes over the row in global memory, then an ordered emission.
+__device__ void topk_global(const float* s, int n, int k, int32_t* out, uint32_t* hist, uint32_t* ws, uint32_t* sel) {
+  const int tid = threadIdx.x;
+  const int shifts[3] = {21, 10, 0};
+  const int widths[3] = {11, 11, 10};
+  uint32_t prefix = 0, pmask = 0, krem = static_cast<uint32_t>(k);
+  for (int pass = 0; pass < 3; ++pass) {
+    const int shift = shifts[pass], nbins = 1 << widths[pass];
+    const uint32_t dmask = static_cast<uint32_t>(nbins - 1);
+    for (int i = tid; i < nbins; i += kTopkThreads) hist[i] = 0;
+    __syncthreads();
+    for (int base = 0; base < n; base += kTopkThreads) {
+      const int i = base + tid;
+      const uint32_t key = i < n ? key_of(s[i]) : 0u;
+      const bool hit = i < n && (key & pmask) == prefix;
+      hist_add(hist, hit, (key >> shift) & dmask);
+    }
+    __syncthreads();
+    find_bin(hist, nbins, krem, ws, sel);
+    prefix |= sel[0] << shift;
+    pmask |= dmask << shift;
+    krem -= sel[1];
+    __syncthreads();
+  }
+  const uint32_t kth = prefix, need_eq = krem;
+  uint32_t gt_tot = 0, eq_tot = 0;
+  for (int base = 0; base < n; base += 4 * kTopkThreads) {
+    const int i0 = base + 4 * tid;
+    uint32_t gt_m = 0, eq_m = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (i0 + e < n) {
+        const uint32_t key = key_of(s[i0 + e]);
+        gt_m |= (key > kth ? 1u : 0u) << e;
+        eq_m |= (key == kth ? 1u : 0u) << e;
+      }
+    }
+    const uint32_t packed = (static_cast<uint32_t>(__popc(gt_m)) << 16) | static_cast<uint32_t>(__popc(eq_m));
+    uint32_t total;
+    const uint32_t ex = block_excl_scan(packed, ws, &total);
+    uint32_t gt_run = gt_tot + (ex >> 16), eq_run = eq_tot + (ex & 0xFFFFu);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (gt_m & (1u << e)) {
+        const uint32_t p = gt_run + min(eq_run, need_eq);
+        if (p < static_cast<uint32_t>(k)) out[p] = i0 + e;
+        ++gt_run;
+      } else if (eq_m & (1u << e)) {
+        const uint32_t p = gt_run + eq_run;
+        if (eq_run < need_eq && p < static_cast<uint32_t>(k)) out[p] = i0 + e;
+        ++eq_run;
+      }
+    }
+    gt_tot += total >> 16;
+    eq_tot += total & 0xFFFFu;
+  }
+}
+
 __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const float* __restrict__ scores, long long ld,
                                                             long long batch_stride, const int32_t* __restrict__ seqlens,
                                                             int Tq, int NBk, int blk, long long q_pos0, int b0,
                                                             int row0, int k, int32_t* __restrict__ idx,
-                                                            KernelCtl ctl) {
-  __shared__ uint32_t hist[kMaxBins];
-  __shared__ uint32_t scan_ws[kWarps + 1];
-  __shared__ uint32_t sel_bin, sel_above;
+                                                            int bitmap_words, KernelCtl ctl) {
+  extern __shared__ uint32_t sm[];
+  uint32_t* cand_key = sm;                       // kCap
+  uint32_t* cand_idx = cand_key + kCap;          // kCap
+  uint32_t* hist = cand_idx + kCap;              // kBins
+  uint32_t* samp = hist + kBins;                 // kSamples
+  uint32_t* ws = samp + kSamples;                // kWarps + 1
+  uint32_t* sel = ws + kWarps + 1;               // 2
+  uint32_t* misc = sel + 2;                      // counter
+  uint32_t* bitmap = misc + 5;                   // bitmap_words
 
   const int tid = threadIdx.x, lane = tid & 31;
   const int r = row0 + static_cast<int>(blockIdx.x);
@@ -82,94 +222,140 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const float* __restr
     for (int i = tid; i < k; i += kTopkThreads) out[i] = i < n ? i : -1;
     return;
   }
-
-  // ---- radix select of the k-th largest key
-  uint32_t prefix = 0, pmask = 0, krem = static_cast<uint32_t>(k);
-  const int shifts[3] = {21, 10, 0};
-  const int widths[3] = {11, 11, 10};
-#pragma unroll 1
-  for (int pass = 0; pass < 3; ++pass) {
-    const int shift = shifts[pass];
-    const int nbins = 1 << widths[pass];
-    const uint32_t dmask = static_cast<uint32_t>(nbins - 1);
-    for (int i = tid; i < nbins; i += kTopkThreads) hist[i] = 0;
-    __syncthreads();
-    for (int base = 0; base < n; base += kTopkThreads) {
-      const int i = base + tid;
-      bool hit = false;
-      uint32_t digit = 0xFFFFFFFFu;
-      if (i < n) {
-        const uint32_t key = key_of(s[i]);
-        if ((key & pmask) == prefix) {
-          hit = true;
-          digit = (key >> shift) & dmask;
-        }
-      }
-      const uint32_t peers = __match_any_sync(0xffffffffu, digit);
-      if (hit && lane == __ffs(peers) - 1) atomicAdd(&hist[digit], static_cast<uint32_t>(__popc(peers)));
-    }
-    __syncthreads();
-    // Bin of the krem-th largest among the hits: thread t owns bins [t*bpt, (t+1)*bpt).
-    const int bpt = nbins / kTopkThreads;
-    uint32_t local = 0;
-    for (int q = 0; q < bpt; ++q) local += hist[tid * bpt + q];
-    // count of hits in bins above this thread's range = total - inclusive prefix
-    uint32_t total;
-    const uint32_t excl = block_excl_scan(local, scan_ws, &total);
-    const uint32_t above = total - excl - local;
-    if (above < krem && above + local >= krem) {
-      uint32_t acc = above;
-      for (int q = bpt - 1; q >= 0; --q) {
-        const uint32_t h = hist[tid * bpt + q];
-        if (acc + h >= krem) {
-          sel_bin = static_cast<uint32_t>(tid * bpt + q);
-          sel_above = acc;
-          break;
-        }
-        acc += h;
-      }
-    }
-    __syncthreads();
-    prefix |= sel_bin << shift;
-    pmask |= dmask << shift;
-    krem -= sel_above;
-    __syncthreads();
+  const int words = (n + 31) >> 5;
+  if (k >= kCap || words > bitmap_words) {
+    topk_global(s, n, k, out, hist, ws, sel);
+    return;
   }
-  const uint32_t kth = prefix;      // the exact k-th largest key
-  const uint32_t need_eq = krem;    // how many keys equal to kth are taken (lowest indices)
 
-  // ---- ordered emission: 4 consecutive elements per thread per chunk
-  uint32_t gt_tot = 0, eq_tot = 0;
-  for (int base = 0; base < n; base += 4 * kTopkThreads) {
-    const int i0 = base + 4 * tid;
-    uint32_t gt_m = 0, eq_m = 0;
+  // ---- 1-2. candidates (key, index) with key >= tau
+  int m = 0;
+  if (n <= kCap) {
+    for (int i = tid; i < n; i += kTopkThreads) {
+      cand_key[i] = key_of(s[i]);
+      cand_idx[i] = static_cast<uint32_t>(i);
+    }
+    m = n;
+    __syncthreads();
+  } else {
+    for (int j = tid; j < kSamples; j += kTopkThreads)
+      samp[j] = key_of(s[static_cast<int>((static_cast<long long>(j) * n) / kSamples)]);
+    __syncthreads();
+    const long long target = min(static_cast<long long>(k) * 5 / 2 + 128, static_cast<long long>(k + kCap) / 2);
+    long long rank = (static_cast<long long>(kSamples) * target + n - 1) / n;
+    const bool vec = ((reinterpret_cast<uintptr_t>(s) & 15u) == 0);
+    bool ok = false;
+    for (int attempt = 0; attempt < 3 && !ok; ++attempt) {
+      rank = max(1ll, min(rank, static_cast<long long>(kSamples)));
+      uint32_t dummy;
+      const uint32_t tau = smem_select(samp, kSamples, static_cast<uint32_t>(rank), 2, hist, ws, sel, &dummy);
+      if (tid == 0) misc[0] = 0;
+      __syncthreads();
+      for (int base = 0; base < n; base += 4 * kTopkThreads) {
+        const int i0 = base + 4 * tid;
+        uint32_t key[4];
+        if (vec && i0 + 3 < n) {
+          const float4 f = *reinterpret_cast<const float4*>(s + i0);
+          key[0] = key_of(f.x);
+          key[1] = key_of(f.y);
+          key[2] = key_of(f.z);
+          key[3] = key_of(f.w);
+        } else {
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int i = i0 + e;
-      if (i < n) {
-        const uint32_t key = key_of(s[i]);
-        gt_m |= (key > kth ? 1u : 0u) << e;
-        eq_m |= (key == kth ? 1u : 0u) << e;
+          for (int e = 0; e < 4; ++e) key[e] = i0 + e < n ? key_of(s[i0 + e]) : 0u;
+        }
+        uint32_t hm = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) hm |= (i0 + e < n && key[e] >= tau ? 1u : 0u) << e;
+        const uint32_t nh = static_cast<uint32_t>(__popc(hm));
+        uint32_t incl = nh;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        uint32_t wbase = 0;
+        if (lane == 31 && incl) wbase = atomicAdd(&misc[0], incl);
+        wbase = __shfl_sync(0xffffffffu, wbase, 31);
+        uint32_t p = wbase + incl - nh;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if (hm & (1u << e)) {
+            if (p < static_cast<uint32_t>(kCap)) {
+              cand_key[p] = key[e];
+              cand_idx[p] = static_cast<uint32_t>(i0 + e);
+            }
+            ++p;
+          }
+        }
+      }
+      __syncthreads();
+      const uint32_t got = misc[0];
+      __syncthreads();
+      if (got >= static_cast<uint32_t>(k) && got <= static_cast<uint32_t>(kCap)) {
+        ok = true;
+        m = static_cast<int>(got);
+      } else if (got < static_cast<uint32_t>(k)) {
+        rank *= 4;          // threshold too high: take it lower
+      } else {
+        rank /= 4;          // too many candidates: take it higher
       }
     }
-    const uint32_t packed = (static_cast<uint32_t>(__popc(gt_m)) << 16) | static_cast<uint32_t>(__popc(eq_m));
-    uint32_t total;
-    const uint32_t ex = block_excl_scan(packed, scan_ws, &total);
-    uint32_t gt_run = gt_tot + (ex >> 16), eq_run = eq_tot + (ex & 0xFFFFu);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      if (gt_m & (1u << e)) {
-        const uint32_t p = gt_run + min(eq_run, need_eq);
-        if (p < static_cast<uint32_t>(k)) out[p] = i0 + e;
-        ++gt_run;
-      } else if (eq_m & (1u << e)) {
-        const uint32_t p = gt_run + eq_run;
-        if (eq_run < need_eq && p < static_cast<uint32_t>(k)) out[p] = i0 + e;
-        ++eq_run;
+    if (!ok) {
+      topk_global(s, n, k, out, hist, ws, sel);
+      return;
+    }
+  }
+
+  // ---- 3. exact k-th key among the candidates, then the index cutoff among equal keys
+  uint32_t need_eq;
+  const uint32_t kth = smem_select(cand_key, m, static_cast<uint32_t>(k), 3, hist, ws, sel, &need_eq);
+  const uint32_t n_eq = hist[kth & 0x3FFu];   // last pass: hits in the K* bin = keys equal to K*
+  uint32_t icut = 0xFFFFFFFFu;
+  if (need_eq < n_eq) {
+    // the need_eq smallest indices among the keys equal to K*: select on ~index among them
+    uint32_t* inv = samp;   // reuse: up to kSamples entries, else fall back to a full pass below
+    if (tid == 0) misc[1] = 0;
+    __syncthreads();
+    for (int i = tid; i < m; i += kTopkThreads) {
+      if (cand_key[i] == kth) {
+        const uint32_t p = atomicAdd(&misc[1], 1u);
+        if (p < static_cast<uint32_t>(kSamples)) inv[p] = ~cand_idx[i];
       }
     }
-    gt_tot += total >> 16;
-    eq_tot += total & 0xFFFFu;
+    __syncthreads();
+    const int ne = static_cast<int>(misc[1]);
+    __syncthreads();
+    if (ne > kSamples) {
+      topk_global(s, n, k, out, hist, ws, sel);
+      return;
+    }
+    uint32_t dummy;
+    icut = ~smem_select(inv, ne, need_eq, 3, hist, ws, sel, &dummy);
+  }
+
+  // ---- 4-5. bitmap of the kept set, emitted in ascending order
+  for (int wd = tid; wd < words; wd += kTopkThreads) bitmap[wd] = 0u;
+  __syncthreads();
+  for (int i = tid; i < m; i += kTopkThreads) {
+    const uint32_t key = cand_key[i], id = cand_idx[i];
+    if (key > kth || (key == kth && id <= icut)) atomicOr(&bitmap[id >> 5], 1u << (id & 31));
+  }
+  __syncthreads();
+  const int wpt = (words + kTopkThreads - 1) / kTopkThreads;
+  const int w0 = tid * wpt, w1 = min(words, w0 + wpt);
+  uint32_t cnt = 0;
+  for (int wd = w0; wd < w1; ++wd) cnt += static_cast<uint32_t>(__popc(bitmap[wd]));
+  uint32_t total;
+  uint32_t p = block_excl_scan(cnt, ws, &total);
+  for (int wd = w0; wd < w1; ++wd) {
+    uint32_t bits = bitmap[wd];
+    while (bits) {
+      const int bit = __ffs(bits) - 1;
+      bits &= bits - 1;
+      if (p < static_cast<uint32_t>(k)) out[p] = wd * 32 + bit;
+      ++p;
+    }
   }
 }
 
@@ -179,9 +365,16 @@ cudaError_t launch_topk(const DeviceInfo* di, const float* scores, long long ld,
                         const int32_t* seqlens, int Tq, int NBk, int blk, long long q_pos0, int b0, int nb, int row0,
                         int rows, int k, int32_t* idx, cudaStream_t s) {
   if (rows <= 0 || nb <= 0) return cudaSuccess;
+  static std::once_flag once[64];
+  std::call_once(once[di->device & 63], [] {
+    cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         kFixedSmem + 32 + kMaxBitmapWords * 4);
+  });
+  const int words = std::min(kMaxBitmapWords, (std::max(NBk, 1) + 31) / 32);
+  const int smem = kFixedSmem + 32 + words * 4;
   dim3 grid(rows, nb);
-  topk_kernel<<<grid, kTopkThreads, 0, s>>>(scores, ld, batch_stride, seqlens, Tq, NBk, blk, q_pos0, b0, row0, k, idx,
-                                            kernel_ctl(di));
+  topk_kernel<<<grid, kTopkThreads, smem, s>>>(scores, ld, batch_stride, seqlens, Tq, NBk, blk, q_pos0, b0, row0, k,
+                                               idx, words, kernel_ctl(di));
   return cudaPeekAtLastError();
 }
 
