@@ -40,6 +40,7 @@ SIGNATURES = {
     "qsa_select_topk": (_I, [_P, _I64, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I64, _I, _I, _P, _P, _SZ, _P]),
     "qsa_sparse_attn_prefill": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I64, _F, _P, _P, _P]),
     "qsa_sparse_attn_decode": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P, _P, _P, _SZ, _P]),
+    "qsa_sparse_attn_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P, _P, _P]),
     "qsa_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I, _I]),
     "qsa_decode_default_splits": (_I, [_I, _I]),
     "qsa_get_device_status": (_I, [_P]),
@@ -254,6 +255,29 @@ def qsa_sparse_attn_decode(q: torch.Tensor, kcache: torch.Tensor, vcache: torch.
     _check(lib().qsa_sparse_attn_decode(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(seqlens), _ptr(idx), B, Lmax, Hq, Hkv,
                                         D, kb, blk, scale, num_splits, _ptr(out), _ptr(lse), _ptr(workspace), ws_bytes,
                                         _stream(q.device)), "qsa_sparse_attn_decode")
+    return out, lse
+
+
+def qsa_sparse_attn_decode_noalloc(q: torch.Tensor, kcache: torch.Tensor, vcache: torch.Tensor,
+                                   seqlens: torch.Tensor, idx: torch.Tensor, *, scale: float | None = None,
+                                   num_splits: int = 0, out: torch.Tensor | None = None,
+                                   lse: torch.Tensor | None = None, blk: int = 4):
+    """qsa_sparse_attn_decode without a workspace: the split partials live in the library's own
+    per-GPU scratch array (for callers that cannot allocate).  Pass ``out``/``lse`` to allocate
+    nothing at all here either."""
+    for t, n in ((q, "q"), (kcache, "kcache"), (vcache, "vcache")):
+        _need(t, torch.bfloat16, n)
+    _need(seqlens, torch.int32, "seqlens")
+    _need(idx, torch.int32, "idx")
+    B, Hq, D = q.shape
+    Lmax, Hkv = kcache.shape[1], kcache.shape[2]
+    kb = idx.shape[-1]
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib().qsa_sparse_attn_decode_noalloc(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(seqlens), _ptr(idx), B,
+                                                Lmax, Hq, Hkv, D, kb, blk, scale, num_splits, _ptr(out), _ptr(lse),
+                                                _stream(q.device)), "qsa_sparse_attn_decode_noalloc")
     return out, lse
 
 

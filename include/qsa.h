@@ -179,6 +179,34 @@ QSA_API qsa_status_t qsa_sparse_attn_decode(const void* q, const void* kcache, c
                                     size_t ws_bytes, void* stream);
 
 /*
+ * Decode attention for callers that cannot allocate device memory.
+ * (No counterpart on the pages: this is a deployment variant of qsa_sparse_attn_decode.)
+ * Some callers have no way to hand the library a workspace: code that runs while a stream is
+ * being captured into a CUDA graph (cudaMalloc is not allowed there), plugins of inference
+ * engines whose memory planner owns the whole device heap, and embedded hosts with a fixed device
+ * budget.  This entry point takes the same inputs and outputs as qsa_sparse_attn_decode but keeps
+ * the per-split partial results in a scratch array that is part of the library image itself
+ * (QSA_NOALLOC_DECODE_SCRATCH_BYTES per GPU, held by every GPU that loads the library until the
+ * process exits).  It calls no allocator.
+ *   - num_splits == 0 picks the largest split count up to qsa_decode_default_splits that fits the
+ *     array; an explicit num_splits > 1 whose partials, B * num_splits * Hq * (D + 2) * 4 bytes,
+ *     exceed QSA_NOALLOC_DECODE_SCRATCH_BYTES returns QSA_ERR_WORKSPACE_TOO_SMALL.
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
+ *     that device current; make that first call before any stream capture that should contain it.
+ *   - Every call, on every stream, shares the one array per device: calls whose kernels overlap on
+ *     the GPU race and corrupt each other's partials.  Serialise them (one stream, or events).
+ *   - Each call overwrites every partial it later reads, so nothing has to be cleared between
+ *     calls even though the array keeps the previous call's contents.
+ */
+#define QSA_NOALLOC_DECODE_SCRATCH_BYTES (4u << 20)
+QSA_API qsa_status_t qsa_sparse_attn_decode_noalloc(const void* q, const void* kcache,
+                                                    const void* vcache, const int32_t* seqlens,
+                                                    const int32_t* idx, int B, int Lmax, int Hq,
+                                                    int Hkv, int D, int k_blocks, int blk,
+                                                    float scale, int num_splits, void* out,
+                                                    float* lse, void* stream);
+
+/*
  * Workspace bytes for `op`.  QSA_OP_SELECT_TOPK: B, Tq, NBk (a chunk of score rows, capped);
  * QSA_OP_SPARSE_ATTN_DECODE: B, Hq, D, num_splits (0 = the count the call would choose).
  * Returns 0 for an unknown op or invalid sizes.
