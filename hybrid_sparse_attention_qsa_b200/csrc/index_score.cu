@@ -174,18 +174,37 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         tmem_ld_32x32(tmem + lane_addr + acc * kN + colbase + c, r);
         tmem_ld_wait();
         const int q0 = (colbase + c) / HI;
+        float sc[32 / HI];
 #pragma unroll
         for (int qq = 0; qq < 32 / HI; ++qq) {
-          float sc = 0.0f;
+          float acc_s = 0.0f;
 #pragma unroll
           for (int h = 0; h < HI; ++h) {
             float x = __uint_as_float(r[qq * HI + h]);
             if (MODE == 0) x = fmaxf(x, 0.0f);
-            sc = fmaf(w[h], x, sc);
+            acc_s = fmaf(w[h], x, acc_s);
           }
-          const int tl = q0 + qq;
-          const int nbq = min(nbk, static_cast<int>((pos_first + tl) >> 2));
-          if (tl <= tl_last && kb < nbq) col[tl * ld] = sc;
+          sc[qq] = acc_s;
+        }
+        // Queries q0 .. q0 + 32/HI - 1 of the tile: when all of them exist and see every pooled key
+        // of this warp, the stores need no mask (all tiles below the diagonal band).
+        float* dst = col + static_cast<long long>(q0) * ld;
+        const bool full = q0 + 32 / HI - 1 <= tl_last &&
+                          (t_begin + i) * kM + quad * 32 + 31 < min(nbk, static_cast<int>((pos_first + q0) >> 2));
+        if (full) {
+#pragma unroll
+          for (int qq = 0; qq < 32 / HI; ++qq) {
+            *dst = sc[qq];
+            dst += ld;
+          }
+        } else {
+#pragma unroll
+          for (int qq = 0; qq < 32 / HI; ++qq) {
+            const int tl = q0 + qq;
+            const int nbq = min(nbk, static_cast<int>((pos_first + tl) >> 2));
+            if (tl <= tl_last && kb < nbq) *dst = sc[qq];
+            dst += ld;
+          }
         }
       }
       tc_fence_before();

@@ -38,6 +38,7 @@ namespace {
 
 constexpr int kSlots = 16;
 constexpr int kStages = 3;
+constexpr int kSeg = 512;          // index-list entries staged in shared memory per buffer
 constexpr int kD = 128;
 constexpr int kBlk = 4;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -55,7 +56,9 @@ struct Cfg {
   static constexpr int kInfoBytes = kStages * 32;
   static constexpr int kBarBytes = (2 * kStages + 2 * HKV) * 8;
   static constexpr int kPendBytes = 64 * 4;
-  static constexpr int kSmem = 128 + kStages * kStageBytes + kMergeBytes + kInfoBytes + kBarBytes + kPendBytes;
+  static constexpr int kIdxBytes = 2 * kSeg * 4;              // double-buffered index-list segments
+  static constexpr int kSmem =
+      128 + kStages * kStageBytes + kMergeBytes + kInfoBytes + kBarBytes + kPendBytes + kIdxBytes;
 };
 
 struct StageInfo {
@@ -140,6 +143,7 @@ __global__ void __launch_bounds__(Cfg<HKV>::kThreads, 1) sparse_attn_kernel(Attn
   uint64_t* mfull = empty + kStages;    // per KV head: the 3 partner warps have written their state
   uint64_t* mempty = mfull + HKV;       // per KV head: warp j=0 has consumed the merge slots
   int* pend = reinterpret_cast<int*>(mempty + HKV);
+  int* idxbuf = pend + 64;              // [2][kSeg]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int group = a.Hq / HKV;
@@ -203,24 +207,52 @@ __global__ void __launch_bounds__(Cfg<HKV>::kThreads, 1) sparse_attn_kernel(Attn
       }
       return true;
     };
+    // The index list of an item is staged in shared memory by asynchronous copies one segment
+    // ahead (the next segment of this item or the first of the next item), so the copy ring never
+    // waits on a global load of the list.
+    auto fetch = [&](int item, int seg, int buf) {
+      if (item < a.num_items) {
+        const Item f = make_item<HKV>(a, item);
+        const int base = f.lo + seg * kSeg;
+        const int len = max(0, min(kSeg, f.hi - base));
+        for (int e = lane; e < len; e += 32) cp_async4(&idxbuf[buf * kSeg + e], f.idx_row + base + e);
+      }
+      cp_async_commit();
+    };
+    int buf = 0;
+    fetch(blockIdx.x, 0, 0);
     for (int item = blockIdx.x; alive && item < a.num_items; item += gridDim.x) {
       const Item it = make_item<HKV>(a, item);
       const long long own = it.pos >= 0 ? it.pos / kBlk : 0;
       int npend = 0;
-      if (it.ok) {
-        for (int c = it.lo; alive && c < it.hi; c += 32) {
-          const int e = c + lane < it.hi ? it.idx_row[c + lane] : -1;
-          const bool valid = e >= 0 && e < own;
-          if (!valid && e != -1 && e != own) record_status(a.ctl, kStBadArg);
-          const unsigned m = __ballot_sync(0xffffffffu, valid);
-          if (valid) pend[npend + __popc(m & ((1u << lane) - 1u))] = (e * kBlk) << 3 | kBlk;
-          npend += __popc(m);
-          __syncwarp();
-          while (alive && npend > kSlots) {
-            alive = flush(kSlots, false, it);
-            npend -= kSlots;
+      const int nseg = max(1, (it.hi - it.lo + kSeg - 1) / kSeg);
+      for (int seg = 0; seg < nseg; ++seg) {
+        if (seg + 1 < nseg)
+          fetch(item, seg + 1, buf ^ 1);
+        else
+          fetch(item + gridDim.x, 0, buf ^ 1);
+        cp_async_wait<1>();
+        __syncwarp();
+        const int len = max(0, min(kSeg, it.hi - (it.lo + seg * kSeg)));
+        if (it.ok) {
+          for (int c = 0; alive && c < len; c += 32) {
+            const int e = c + lane < len ? idxbuf[buf * kSeg + c + lane] : -1;
+            const bool valid = e >= 0 && e < own;
+            if (!valid && e != -1 && e != own) record_status(a.ctl, kStBadArg);
+            const unsigned m = __ballot_sync(0xffffffffu, valid);
+            if (valid) pend[npend + __popc(m & ((1u << lane) - 1u))] = (e * kBlk) << 3 | kBlk;
+            npend += __popc(m);
+            __syncwarp();
+            while (alive && npend > kSlots) {
+              alive = flush(kSlots, false, it);
+              npend -= kSlots;
+            }
           }
         }
+        __syncwarp();
+        buf ^= 1;
+      }
+      if (it.ok) {
         if (it.diag) {
           if (lane == 0) pend[npend] = static_cast<int>((own * kBlk) << 3) | static_cast<int>(it.pos - own * kBlk + 1);
           ++npend;
@@ -235,6 +267,7 @@ __global__ void __launch_bounds__(Cfg<HKV>::kThreads, 1) sparse_attn_kernel(Attn
       }
       if (alive) alive = flush(npend, true, it);
     }
+    cp_async_wait<0>();
     // Never leave with a copy in flight: wait for the last fill of every stage.
     for (int s = 0; s < kStages && s < fills; ++s) {
       const int last = s + ((fills - 1 - s) / kStages) * kStages;
@@ -259,20 +292,28 @@ __global__ void __launch_bounds__(Cfg<HKV>::kThreads, 1) sparse_attn_kernel(Attn
   unsigned ph = 0;
   unsigned mph = 0;   // parity of the merge barriers (one phase per item)
 
+  // B-operand fragments of the query heads of this KV head; the next item's are loaded before the
+  // merge of the current one so that their latency overlaps it.
+  const int hq = g * group + n_head;
+  const bool hv = n_head < group;
+  auto load_q = [&](int item, uint32_t (&f)[8][2]) {
+    if (item >= a.num_items) return;
+    const long long qrow = a.seqlens == nullptr
+                               ? static_cast<long long>(item % a.B) * a.Tq + (a.Tq - 1 - item / a.B)
+                               : static_cast<long long>(item / a.splits);
+    const uint16_t* qp = a.q + (qrow * a.Hq + (hv ? hq : 0)) * kD;
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      const int d0 = 16 * kk + cpair;
+      f[kk][0] = hv ? *reinterpret_cast<const uint32_t*>(qp + d0) : 0u;
+      f[kk][1] = hv ? *reinterpret_cast<const uint32_t*>(qp + d0 + 8) : 0u;
+    }
+  };
+  uint32_t qf[8][2], qn[8][2];
+  load_q(blockIdx.x, qf);
+
   for (int item = blockIdx.x; item < a.num_items; item += gridDim.x) {
     const Item it = make_item<HKV>(a, item);
-    uint32_t qf[8][2];
-    {
-      const int hq = g * group + n_head;
-      const bool hv = n_head < group;
-      const uint16_t* qrow = a.q + (it.qrow * a.Hq + (hv ? hq : 0)) * kD;
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const int d0 = 16 * kk + cpair;
-        qf[kk][0] = hv ? *reinterpret_cast<const uint32_t*>(qrow + d0) : 0u;
-        qf[kk][1] = hv ? *reinterpret_cast<const uint32_t*>(qrow + d0 + 8) : 0u;
-      }
-    }
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
     float o[8][4];
 #pragma unroll
@@ -340,6 +381,7 @@ __global__ void __launch_bounds__(Cfg<HKV>::kThreads, 1) sparse_attn_kernel(Attn
       if (last) break;
     }
 
+    load_q(item + gridDim.x, qn);
     // ---- item epilogue: full row sums, merge the 4 token-warps of this KV head, write
 #pragma unroll
     for (int o2 = 4; o2 < 32; o2 <<= 1) {
@@ -440,6 +482,11 @@ __global__ void __launch_bounds__(Cfg<HKV>::kThreads, 1) sparse_attn_kernel(Attn
       if (lane == 0) mbar_arrive(&mempty[g]);
     }
     mph ^= 1u;
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      qf[kk][0] = qn[kk][0];
+      qf[kk][1] = qn[kk][1];
+    }
   }
 }
 

@@ -251,41 +251,52 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const float* __restr
       const uint32_t tau = smem_select(samp, kSamples, static_cast<uint32_t>(rank), 2, hist, ws, sel, &dummy);
       if (tid == 0) misc[0] = 0;
       __syncthreads();
-      for (int base = 0; base < n; base += 4 * kTopkThreads) {
-        const int i0 = base + 4 * tid;
-        uint32_t key[4];
-        if (vec && i0 + 3 < n) {
-          const float4 f = *reinterpret_cast<const float4*>(s + i0);
-          key[0] = key_of(f.x);
-          key[1] = key_of(f.y);
-          key[2] = key_of(f.z);
-          key[3] = key_of(f.w);
-        } else {
+      // kU independent 16-byte loads per thread are in flight before any of them is used.
+      constexpr int kU = 4;
+      for (int base = 0; base < n; base += 4 * kTopkThreads * kU) {
+        uint32_t key[kU][4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) key[e] = i0 + e < n ? key_of(s[i0 + e]) : 0u;
+        for (int u = 0; u < kU; ++u) {
+          const int i0 = base + 4 * (u * kTopkThreads + tid);
+          if (vec && i0 + 3 < n) {
+            const float4 f = __ldcs(reinterpret_cast<const float4*>(s + i0));
+            key[u][0] = key_of(f.x);
+            key[u][1] = key_of(f.y);
+            key[u][2] = key_of(f.z);
+            key[u][3] = key_of(f.w);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) key[u][e] = i0 + e < n ? key_of(s[i0 + e]) : 0u;
+          }
         }
-        uint32_t hm = 0;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) hm |= (i0 + e < n && key[e] >= tau ? 1u : 0u) << e;
-        const uint32_t nh = static_cast<uint32_t>(__popc(hm));
-        uint32_t incl = nh;
+        for (int u = 0; u < kU; ++u) {
+          const int i0 = base + 4 * (u * kTopkThreads + tid);
+          uint32_t hm = 0;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += y;
-        }
-        uint32_t wbase = 0;
-        if (lane == 31 && incl) wbase = atomicAdd(&misc[0], incl);
-        wbase = __shfl_sync(0xffffffffu, wbase, 31);
-        uint32_t p = wbase + incl - nh;
+          for (int e = 0; e < 4; ++e) hm |= (i0 + e < n && key[u][e] >= tau ? 1u : 0u) << e;
+          const uint32_t nh = static_cast<uint32_t>(__popc(hm));
+          const unsigned any = __ballot_sync(0xffffffffu, nh != 0);
+          if (any == 0u) continue;   // warp-uniform: nothing of this warp passes the threshold
+          uint32_t incl = nh;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          if (hm & (1u << e)) {
-            if (p < static_cast<uint32_t>(kCap)) {
-              cand_key[p] = key[e];
-              cand_idx[p] = static_cast<uint32_t>(i0 + e);
+          for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+          }
+          uint32_t wbase = 0;
+          if (lane == 31) wbase = atomicAdd(&misc[0], incl);
+          wbase = __shfl_sync(0xffffffffu, wbase, 31);
+          uint32_t p = wbase + incl - nh;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            if (hm & (1u << e)) {
+              if (p < static_cast<uint32_t>(kCap)) {
+                cand_key[p] = key[u][e];
+                cand_idx[p] = static_cast<uint32_t>(i0 + e);
+              }
+              ++p;
             }
-            ++p;
           }
         }
       }
