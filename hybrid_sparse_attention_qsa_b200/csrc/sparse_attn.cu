@@ -39,10 +39,22 @@ namespace {
 constexpr int kSlots = 16;
 constexpr int kStages = 3;
 constexpr int kSeg = 512;          // index-list entries staged in shared memory per buffer
+constexpr int kIssuers_ = 4;       // warps that issue the bulk copies of a stage
 constexpr int kD = 128;
 constexpr int kBlk = 4;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
+
+// Published by the leading producer warp for every stage it fills (and read by the helper
+// producer warps and the consumers).  nslots == -1 tells the helpers that no stage follows.
+struct StageInfo {
+  int nslots;
+  int last;
+  const uint16_t* kbase;
+  const uint16_t* vbase;
+  int tok0[kSlots];
+  uint8_t ntok[kSlots];
+};
 
 template <int HKV>
 struct Cfg {
@@ -50,23 +62,18 @@ struct Cfg {
   static constexpr int kPitch = kBlockBytes + 16;
   static constexpr int kStageBytes = 2 * kSlots * kPitch;     // K slots, then V slots
   static constexpr int kConsumerWarps = kBlk * HKV;
-  static constexpr int kThreads = (kConsumerWarps + 1) * 32;
+  static constexpr int kIssuers = kIssuers_;
+  static constexpr int kThreads = (kConsumerWarps + kIssuers) * 32;
   static constexpr int kMergeSlot = 32 * 32 * 4 + 32 * 4 * 4; // o fragments + (m0, m1, l0, l1) per lane
   static constexpr int kMergeBytes = 3 * HKV * kMergeSlot;
-  static constexpr int kInfoBytes = kStages * 32;
-  static constexpr int kBarBytes = (2 * kStages + 2 * HKV) * 8;
+  static constexpr int kInfoBytes = kStages * ((sizeof(StageInfo) + 15) / 16 * 16);
+  static constexpr int kBarBytes = (3 * kStages + 2 * HKV) * 8;
   static constexpr int kPendBytes = 64 * 4;
   static constexpr int kIdxBytes = 2 * kSeg * 4;              // double-buffered index-list segments
   static constexpr int kSmem =
       128 + kStages * kStageBytes + kMergeBytes + kInfoBytes + kBarBytes + kPendBytes + kIdxBytes;
 };
 
-struct StageInfo {
-  int nslots;
-  int last;
-  int pad[2];
-  uint8_t ntok[kSlots];
-};
 
 struct AttnArgs {
   const uint16_t* q;
@@ -138,9 +145,12 @@ __global__ void __launch_bounds__(Cfg<HKV>::kThreads, 1) sparse_attn_kernel(Attn
   uint8_t* ring = smem;
   uint8_t* merge = ring + kStages * C::kStageBytes;
   StageInfo* info = reinterpret_cast<StageInfo*>(merge + C::kMergeBytes);
+  constexpr int kInfoStride = (sizeof(StageInfo) + 15) / 16 * 16;
+  auto info_at = [&](int s) { return reinterpret_cast<StageInfo*>(reinterpret_cast<uint8_t*>(info) + s * kInfoStride); };
   uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(info) + C::kInfoBytes);
   uint64_t* empty = full + kStages;
-  uint64_t* mfull = empty + kStages;    // per KV head: the 3 partner warps have written their state
+  uint64_t* ready = empty + kStages;    // per stage: slot list published for the helper issuers
+  uint64_t* mfull = ready + kStages;    // per KV head: the 3 partner warps have written their state
   uint64_t* mempty = mfull + HKV;       // per KV head: warp j=0 has consumed the merge slots
   int* pend = reinterpret_cast<int*>(mempty + HKV);
   int* idxbuf = pend + 64;              // [2][kSeg]
@@ -152,6 +162,7 @@ __global__ void __launch_bounds__(Cfg<HKV>::kThreads, 1) sparse_attn_kernel(Attn
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], C::kConsumerWarps);
+      mbar_init(&ready[s], 1);
     }
     for (int g = 0; g < HKV; ++g) {
       mbar_init(&mfull[g], kBlk - 1);
@@ -165,8 +176,39 @@ __global__ void __launch_bounds__(Cfg<HKV>::kThreads, 1) sparse_attn_kernel(Attn
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // order these writes before the bulk copies
   __syncthreads();
 
+  if (warp > C::kConsumerWarps) {
+    // ------------------------------------------------------------------ helper issuer warps
+    // The per-SM rate of 1-D bulk copies grows with the number of warps issuing them, so the
+    // copies of a stage are spread over kIssuers warps: helper h issues slots h, h + kIssuers, ...
+    const int h = warp - C::kConsumerWarps;
+    int st = 0;
+    unsigned ph = 0;
+    const uint32_t tok_bytes = HKV * kD * 2;
+    for (;;) {
+      if (!mbar_wait(&ready[st], ph, a.ctl)) break;
+      const StageInfo* inf = info_at(st);
+      const int n = inf->nslots;
+      if (n < 0) break;
+      const int slot = h + kIssuers_ * lane;
+      if (lane < kSlots / kIssuers_ && slot < n) {
+        const int ntok = inf->ntok[slot];
+        const long long tok0 = inf->tok0[slot];
+        uint8_t* kd = ring + st * C::kStageBytes + slot * C::kPitch;
+        uint8_t* vd = kd + kSlots * C::kPitch;
+        bulk_g2s(kd, inf->kbase + tok0 * HKV * kD, ntok * tok_bytes, &full[st]);
+        bulk_g2s(vd, inf->vbase + tok0 * HKV * kD, ntok * tok_bytes, &full[st]);
+      }
+      __syncwarp();
+      if (++st == kStages) {
+        st = 0;
+        ph ^= 1u;
+      }
+    }
+    return;
+  }
+
   if (warp == C::kConsumerWarps) {
-    // ------------------------------------------------------------------ producer warp
+    // ------------------------------------------------------------------ leading producer warp
     int st = 0;
     unsigned ph = 0;
     int fills = 0;
@@ -177,17 +219,26 @@ __global__ void __launch_bounds__(Cfg<HKV>::kThreads, 1) sparse_attn_kernel(Attn
       int packed = lane < n ? pend[lane] : 0;
       const int ntok = packed & 7;
       const long long tok0 = packed >> 3;
-      if (lane < kSlots) info[st].ntok[lane] = static_cast<uint8_t>(lane < n ? ntok : 0);
+      StageInfo* inf = info_at(st);
+      if (lane < kSlots) {
+        inf->ntok[lane] = static_cast<uint8_t>(lane < n ? ntok : 0);
+        inf->tok0[lane] = static_cast<int>(tok0);
+      }
       if (lane == 0) {
-        info[st].nslots = n;
-        info[st].last = last ? 1 : 0;
+        inf->nslots = n;
+        inf->last = last ? 1 : 0;
+        inf->kbase = it.kbase;
+        inf->vbase = it.vbase;
       }
       const uint32_t mine = lane < n ? 2u * ntok * tok_bytes : 0u;
       const uint32_t total = __reduce_add_sync(0xffffffffu, mine);
       __syncwarp();
-      if (lane == 0) mbar_arrive_expect_tx(&full[st], total);
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&full[st], total);   // registered before any helper can issue a copy
+        mbar_arrive(&ready[st]);
+      }
       __syncwarp();
-      if (lane < n) {
+      if (lane < n && lane % kIssuers_ == 0) {
         uint8_t* kd = ring + st * C::kStageBytes + lane * C::kPitch;
         uint8_t* vd = kd + kSlots * C::kPitch;
         bulk_g2s(kd, it.kbase + tok0 * HKV * kD, ntok * tok_bytes, &full[st]);
@@ -268,6 +319,14 @@ __global__ void __launch_bounds__(Cfg<HKV>::kThreads, 1) sparse_attn_kernel(Attn
       if (alive) alive = flush(npend, true, it);
     }
     cp_async_wait<0>();
+    // Tell the helpers that no stage follows (the stage is free once every consumer released it).
+    if (alive && mbar_wait(&empty[st], ph ^ 1u, a.ctl)) {
+      if (lane == 0) {
+        info_at(st)->nslots = -1;
+        mbar_arrive(&ready[st]);
+      }
+      __syncwarp();
+    }
     // Never leave with a copy in flight: wait for the last fill of every stage.
     for (int s = 0; s < kStages && s < fills; ++s) {
       const int last = s + ((fills - 1 - s) / kStages) * kStages;
@@ -321,8 +380,8 @@ __global__ void __launch_bounds__(Cfg<HKV>::kThreads, 1) sparse_attn_kernel(Attn
 
     for (;;) {
       if (!mbar_wait(&full[st], ph, a.ctl)) return;
-      const int ns = info[st].nslots;
-      const bool last = info[st].last != 0;
+      const int ns = info_at(st)->nslots;
+      const bool last = info_at(st)->last != 0;
       if (ns > 0) {
         const uint32_t kst = ring_u32 + st * C::kStageBytes;
         const uint32_t vst = kst + kSlots * C::kPitch;
@@ -334,8 +393,8 @@ __global__ void __launch_bounds__(Cfg<HKV>::kThreads, 1) sparse_attn_kernel(Attn
           mma_bf16_16816(acc, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
         }
         const int r0 = lane >> 2, r1 = r0 + 8;
-        const bool v0 = r0 < ns && j < info[st].ntok[r0];
-        const bool v1 = r1 < ns && j < info[st].ntok[r1];
+        const bool v0 = r0 < ns && j < info_at(st)->ntok[r0];
+        const bool v1 = r1 < ns && j < info_at(st)->ntok[r1];
         const float x0 = v0 ? acc[0] * a.scale_log2 : -INFINITY;
         const float x1 = v0 ? acc[1] * a.scale_log2 : -INFINITY;
         const float x2 = v1 ? acc[2] * a.scale_log2 : -INFINITY;
