@@ -19,6 +19,29 @@ DeviceInfo g_dev[kMaxDevices];
 bool g_dev_ok[kMaxDevices];
 std::atomic<unsigned long long> g_wait_ns{kDefaultWaitNs};
 
+// Per-device side stream and events used by qsa_select_topk to overlap chunks (created on first
+// use with the device current; kept until the process exits).
+struct SideStream {
+  std::mutex mu;
+  cudaStream_t stream = nullptr;
+  cudaEvent_t begin = nullptr, end = nullptr, score_done[2] = {nullptr, nullptr}, topk_done[2] = {nullptr, nullptr};
+};
+SideStream g_side[kMaxDevices];
+std::once_flag g_side_once[kMaxDevices];
+bool g_side_ok[kMaxDevices];
+
+SideStream* side_stream(int dev) {
+  std::call_once(g_side_once[dev], [dev] {
+    SideStream& ss = g_side[dev];
+    bool ok = cudaStreamCreateWithFlags(&ss.stream, cudaStreamNonBlocking) == cudaSuccess;
+    cudaEvent_t* evs[] = {&ss.begin, &ss.end, &ss.score_done[0], &ss.score_done[1], &ss.topk_done[0],
+                          &ss.topk_done[1]};
+    for (cudaEvent_t* ev : evs) ok = ok && cudaEventCreateWithFlags(ev, cudaEventDisableTiming) == cudaSuccess;
+    g_side_ok[dev] = ok;
+  });
+  return g_side_ok[dev] ? &g_side[dev] : nullptr;
+}
+
 __global__ void wait_selftest_kernel(KernelCtl ctl) {
   __shared__ uint64_t bar;
   if (threadIdx.x == 0) {
@@ -167,16 +190,47 @@ qsa_status_t qsa_select_topk(const float* scores, int64_t ld_scores, const void*
     if (e == cudaSuccess) e = launch_topk(di, ws, NBk, NBk, seqlens, 1, NBk, blk, 0, 0, B, 0, 1, k, idx, s);
     return cuda_status(e);
   }
-  for (int b = 0; b < B; ++b) {
-    for (int r0 = 0; r0 < Tq; r0 += static_cast<int>(std::min<long long>(R, Tq))) {
-      const int rows = static_cast<int>(std::min<long long>(R, Tq - r0));
-      cudaError_t e = launch_score_prefill(di, qi, kp, head_w, B, Tq, NBk, Hi, Di, blk, q_pos0, mode, b, 1, r0, rows,
-                                           ws, NBk, 0, s);
-      if (e == cudaSuccess) e = launch_topk(di, ws, NBk, 0, nullptr, Tq, NBk, blk, q_pos0, b, 1, r0, rows, k, idx, s);
-      if (e != cudaSuccess) return QSA_ERR_CUDA;
+  const long long chunks = static_cast<long long>(B) * ((Tq + R - 1) / R);
+  SideStream* side = chunks > 1 && R >= 2 ? side_stream(di->device) : nullptr;
+  if (side == nullptr) {
+    for (int b = 0; b < B; ++b) {
+      for (int r0 = 0; r0 < Tq; r0 += static_cast<int>(std::min<long long>(R, Tq))) {
+        const int rows = static_cast<int>(std::min<long long>(R, Tq - r0));
+        cudaError_t e = launch_score_prefill(di, qi, kp, head_w, B, Tq, NBk, Hi, Di, blk, q_pos0, mode, b, 1, r0,
+                                             rows, ws, NBk, 0, s);
+        if (e == cudaSuccess) e = launch_topk(di, ws, NBk, 0, nullptr, Tq, NBk, blk, q_pos0, b, 1, r0, rows, k, idx, s);
+        if (e != cudaSuccess) return QSA_ERR_CUDA;
+      }
+    }
+    return QSA_OK;
+  }
+  // Two halves of the workspace: the scores of chunk i+1 are computed on the caller's stream while
+  // the top-k of chunk i runs on a side stream (the kernels fit on an SM together).  Events order
+  // every reuse of a half and join the side stream back into the caller's stream.
+  const long long R2 = R / 2;
+  std::lock_guard<std::mutex> lk(side->mu);
+  cudaError_t e = cudaEventRecord(side->begin, s);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(side->stream, side->begin, 0);
+  long long c = 0;
+  for (int b = 0; e == cudaSuccess && b < B; ++b) {
+    for (int r0 = 0; e == cudaSuccess && r0 < Tq; r0 += static_cast<int>(R2), ++c) {
+      const int rows = static_cast<int>(std::min<long long>(R2, Tq - r0));
+      const int buf = static_cast<int>(c & 1);
+      float* half = ws + buf * R2 * NBk;
+      if (c >= 2) e = cudaStreamWaitEvent(s, side->topk_done[buf], 0);
+      if (e == cudaSuccess)
+        e = launch_score_prefill(di, qi, kp, head_w, B, Tq, NBk, Hi, Di, blk, q_pos0, mode, b, 1, r0, rows, half, NBk,
+                                 0, s);
+      if (e == cudaSuccess) e = cudaEventRecord(side->score_done[buf], s);
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(side->stream, side->score_done[buf], 0);
+      if (e == cudaSuccess)
+        e = launch_topk(di, half, NBk, 0, nullptr, Tq, NBk, blk, q_pos0, b, 1, r0, rows, k, idx, side->stream);
+      if (e == cudaSuccess) e = cudaEventRecord(side->topk_done[buf], side->stream);
     }
   }
-  return QSA_OK;
+  if (e == cudaSuccess) e = cudaEventRecord(side->end, side->stream);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s, side->end, 0);
+  return cuda_status(e);
 }
 
 static qsa_status_t check_attn_shape(int Hq, int Hkv, int D, int blk, int k_blocks) {

@@ -18,7 +18,7 @@
 //   epilogue of tile i overlap the MMAs of tile i+1.  The causal bound is per CTA (tiles up to the
 //   last query row's visible blocks); the store mask is per query.
 // Decode: one query per sequence, so the contraction degenerates to a GEMV over the pooled-key
-//   cache; it is HBM-bound and runs on CUDA cores with 16-byte loads (8 lanes per pooled key).
+//   cache; it is HBM-bound and runs as mma.sync tiles with the query heads in the N dimension.
 #include <mutex>
 
 #include "launch.h"
@@ -220,14 +220,20 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
   }
 }
 
-// ------------------------------------------------------------------------------ decode GEMV
+// ------------------------------------------------------------------------------ decode
+// One query per sequence: s(b) for the pooled keys of the cache, a GEMV bound by reading 128 bytes
+// per block.  mma.m16n8k16 does the arithmetic: 16 pooled keys x 8 head columns per tile (the Hi
+// indexer heads fill N, zero past Hi), the query's B fragments stay in registers and the keys' A
+// fragments are loaded straight from global memory (every byte once; the two halves of a 32-byte
+// sector are read by consecutive loads and meet in L1).  The 4 lanes of a key row then add their
+// heads with two shuffles.
 template <int HI>
 __global__ void __launch_bounds__(256) score_decode_kernel(const uint16_t* __restrict__ qi,
                                                            const uint16_t* __restrict__ kp,
                                                            const float* __restrict__ head_w,
                                                            const int32_t* __restrict__ seqlens, int NBk, int blk,
                                                            int mode, float* __restrict__ scores, long long ld,
-                                                           KernelCtl ctl) {
+                                                           int part_len, KernelCtl ctl) {
   const int b = blockIdx.y;
   const int L = seqlens[b];
   if (L < 1) {
@@ -239,60 +245,70 @@ __global__ void __launch_bounds__(256) score_decode_kernel(const uint16_t* __res
     if (blockIdx.x == 0 && threadIdx.x == 0) record_status(ctl, kStBadArg);
     nb = NBk;
   }
+  const int lo = static_cast<int>(blockIdx.x) * part_len;
+  const int c = max(0, min(nb, lo + part_len) - lo);
+  if (c == 0) return;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int seg = lane & 7;      // 8-element segment of Di = 64
-  const int sub = lane >> 3;     // which of the 4 keys a warp instruction covers
-  float q[HI][8];
+  uint32_t bq[4][2];
+  {
+    const int n = lane >> 2;
+    const uint16_t* qrow = qi + (static_cast<long long>(b) * HI + (n < HI ? n : 0)) * kDi;
 #pragma unroll
-  for (int h = 0; h < HI; ++h) {
-    const uint4 raw = *reinterpret_cast<const uint4*>(qi + (static_cast<long long>(b) * HI + h) * kDi + seg * 8);
-    const uint32_t u[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      q[h][2 * e] = __uint_as_float(u[e] << 16);
-      q[h][2 * e + 1] = __uint_as_float(u[e] & 0xFFFF0000u);
+    for (int kk = 0; kk < 4; ++kk) {
+      const int d0 = 16 * kk + 2 * (lane & 3);
+      bq[kk][0] = n < HI ? __ldg(reinterpret_cast<const uint32_t*>(qrow + d0)) : 0u;
+      bq[kk][1] = n < HI ? __ldg(reinterpret_cast<const uint32_t*>(qrow + d0 + 8)) : 0u;
     }
   }
-  float w[HI];
+  const int h0 = 2 * (lane & 3);
+  const float w0 = (h0 < HI) ? (head_w ? head_w[h0] : 1.f) : 0.f;
+  const float w1 = (h0 + 1 < HI) ? (head_w ? head_w[h0 + 1] : 1.f) : 0.f;
+  const uint16_t* kpb = kp + (static_cast<long long>(b) * NBk + lo) * kDi;
+  float* srow = scores + static_cast<long long>(b) * ld + lo;
+  const int ntiles = (c + 15) / 16;
+  constexpr int kWarps = 8, kUnroll = 4;
+  for (int t0 = warp; t0 < ntiles; t0 += kWarps * kUnroll) {
+    uint32_t a[kUnroll][4][4];
 #pragma unroll
-  for (int h = 0; h < HI; ++h) w[h] = head_w ? head_w[h] : 1.0f;
-  const uint16_t* kpb = kp + static_cast<long long>(b) * NBk * kDi;
-  float* srow = scores + static_cast<long long>(b) * ld;
-  constexpr int kU = 4;   // loads in flight per lane
-  const long long stride = static_cast<long long>(gridDim.x) * 8 * 4 * kU;
-  for (long long base = (static_cast<long long>(blockIdx.x) * 8 + warp) * 4 * kU; base < nb; base += stride) {
-    uint4 raw[kU];
+    for (int u = 0; u < kUnroll; ++u) {
+      const int t = t0 + u * kWarps;
+      const int r0 = t * 16 + (lane >> 2), r1 = r0 + 8;
+      const bool ok0 = t < ntiles && r0 < c, ok1 = t < ntiles && r1 < c;
+      const uint16_t* p0 = kpb + static_cast<long long>(ok0 ? r0 : 0) * kDi + 2 * (lane & 3);
+      const uint16_t* p1 = kpb + static_cast<long long>(ok1 ? r1 : 0) * kDi + 2 * (lane & 3);
 #pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      const long long row = base + u * 4 + sub;
-      raw[u] = row < nb ? __ldg(reinterpret_cast<const uint4*>(kpb + row * kDi + seg * 8)) : make_uint4(0, 0, 0, 0);
+      for (int kk = 0; kk < 4; ++kk) {
+        a[u][kk][0] = ok0 ? __ldg(reinterpret_cast<const uint32_t*>(p0 + 16 * kk)) : 0u;
+        a[u][kk][1] = ok1 ? __ldg(reinterpret_cast<const uint32_t*>(p1 + 16 * kk)) : 0u;
+        a[u][kk][2] = ok0 ? __ldg(reinterpret_cast<const uint32_t*>(p0 + 16 * kk + 8)) : 0u;
+        a[u][kk][3] = ok1 ? __ldg(reinterpret_cast<const uint32_t*>(p1 + 16 * kk + 8)) : 0u;
+      }
     }
 #pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      const uint32_t v[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
-      float kv[8];
+    for (int u = 0; u < kUnroll; ++u) {
+      const int t = t0 + u * kWarps;
+      if (t >= ntiles) break;   // warp-uniform
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        kv[2 * e] = __uint_as_float(v[e] << 16);
-        kv[2 * e + 1] = __uint_as_float(v[e] & 0xFFFF0000u);
+      for (int kk = 0; kk < 4; ++kk)
+        mma_bf16_16816(acc, a[u][kk][0], a[u][kk][1], a[u][kk][2], a[u][kk][3], bq[kk][0], bq[kk][1]);
+      float x0 = acc[0], x1 = acc[1], x2 = acc[2], x3 = acc[3];
+      if (mode == 0) {
+        x0 = fmaxf(x0, 0.f);
+        x1 = fmaxf(x1, 0.f);
+        x2 = fmaxf(x2, 0.f);
+        x3 = fmaxf(x3, 0.f);
       }
-      float dot[HI];
-#pragma unroll
-      for (int h = 0; h < HI; ++h) {
-        float d = 0.0f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) d = fmaf(q[h][e], kv[e], d);
-        d += __shfl_xor_sync(0xffffffffu, d, 1);
-        d += __shfl_xor_sync(0xffffffffu, d, 2);
-        d += __shfl_xor_sync(0xffffffffu, d, 4);
-        dot[h] = d;
-      }
-      const long long row = base + u * 4 + sub;
-      if (seg == 0 && row < nb) {
-        float sc = 0.0f;
-#pragma unroll
-        for (int h = 0; h < HI; ++h) sc = fmaf(w[h], mode == 0 ? fmaxf(dot[h], 0.0f) : dot[h], sc);
-        srow[row] = sc;
+      float v0 = fmaf(w1, x1, w0 * x0);   // key row lane/4, this lane's two head columns
+      float v1 = fmaf(w1, x3, w0 * x2);   // key row lane/4 + 8
+      v0 += __shfl_xor_sync(0xffffffffu, v0, 1);
+      v1 += __shfl_xor_sync(0xffffffffu, v1, 1);
+      v0 += __shfl_xor_sync(0xffffffffu, v0, 2);
+      v1 += __shfl_xor_sync(0xffffffffu, v1, 2);
+      const int r0 = t * 16 + (lane >> 2), r1 = r0 + 8;
+      if ((lane & 3) == 0) {
+        if (r0 < c) srow[r0] = v0;
+        if (r1 < c) srow[r1] = v1;
       }
     }
   }
@@ -386,16 +402,17 @@ cudaError_t launch_score_decode(const DeviceInfo* di, const void* qi, const void
   (void)Di;
   if (B <= 0 || NBk <= 0) return cudaSuccess;
   const KernelCtl ctl = kernel_ctl(di);
-  const int per_seq = std::max(1, (di->num_sms * 4 + B - 1) / B);
-  const int need = (NBk + 127) / 128;
-  dim3 grid(std::min(per_seq, need), B);
+  // about four CTAs per SM in total, parts of at least 1024 pooled keys
+  const int parts = std::max(1, std::min((di->num_sms * 4 + B - 1) / B, (NBk + 1023) / 1024));
+  const int part_len = ((NBk + parts - 1) / parts + 15) / 16 * 16;
+  dim3 grid((NBk + part_len - 1) / part_len, B);
   const uint16_t* q = static_cast<const uint16_t*>(qi);
   const uint16_t* k = static_cast<const uint16_t*>(kp);
   switch (Hi) {
-    case 1: score_decode_kernel<1><<<grid, 256, 0, s>>>(q, k, head_w, seqlens, NBk, blk, mode, scores, ld, ctl); break;
-    case 2: score_decode_kernel<2><<<grid, 256, 0, s>>>(q, k, head_w, seqlens, NBk, blk, mode, scores, ld, ctl); break;
-    case 4: score_decode_kernel<4><<<grid, 256, 0, s>>>(q, k, head_w, seqlens, NBk, blk, mode, scores, ld, ctl); break;
-    case 8: score_decode_kernel<8><<<grid, 256, 0, s>>>(q, k, head_w, seqlens, NBk, blk, mode, scores, ld, ctl); break;
+    case 1: score_decode_kernel<1><<<grid, 256, 0, s>>>(q, k, head_w, seqlens, NBk, blk, mode, scores, ld, part_len, ctl); break;
+    case 2: score_decode_kernel<2><<<grid, 256, 0, s>>>(q, k, head_w, seqlens, NBk, blk, mode, scores, ld, part_len, ctl); break;
+    case 4: score_decode_kernel<4><<<grid, 256, 0, s>>>(q, k, head_w, seqlens, NBk, blk, mode, scores, ld, part_len, ctl); break;
+    case 8: score_decode_kernel<8><<<grid, 256, 0, s>>>(q, k, head_w, seqlens, NBk, blk, mode, scores, ld, part_len, ctl); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaPeekAtLastError();

@@ -26,11 +26,26 @@
 namespace qsa {
 namespace {
 
-constexpr int kTopkThreads = 512;
+// Tuning knobs (compile time): threads per row, samples for the threshold, loads in flight per
+// thread in the filter pass, and how a warp appends its candidates (0: warp scan + one shared
+// atomic per warp; 1: one shared atomic per thread that has candidates).
+#ifndef QSA_TOPK_THREADS
+#define QSA_TOPK_THREADS 512
+#endif
+#ifndef QSA_TOPK_SAMPLES
+#define QSA_TOPK_SAMPLES 2048
+#endif
+#ifndef QSA_TOPK_LOADS
+#define QSA_TOPK_LOADS 4
+#endif
+#ifndef QSA_TOPK_APPEND
+#define QSA_TOPK_APPEND 1
+#endif
+constexpr int kTopkThreads = QSA_TOPK_THREADS;
 constexpr int kWarps = kTopkThreads / 32;
 constexpr int kBins = 2048;
 constexpr int kCap = 6144;          // candidate capacity of the fast path
-constexpr int kSamples = 2048;
+constexpr int kSamples = QSA_TOPK_SAMPLES;
 constexpr int kMaxBitmapWords = 24576;   // rows up to 786432 candidates use the fast path
 constexpr int kFixedSmem = kCap * 8 + kBins * 4 + kSamples * 4 + (kWarps + 8) * 4;
 
@@ -100,31 +115,62 @@ __device__ __forceinline__ void find_bin(const uint32_t* hist, int nbins, uint32
   __syncthreads();
 }
 
-// Radix select over values in shared memory: the krem-th largest of vals[0..m).  `passes` of the
-// (11, 11, 10)-bit digits are resolved from the top; unresolved low bits are returned as zero.
-// *left = how many values equal to the result (after the resolved bits) are still to be taken.
+// As find_bin, but the bins are scanned by warp 0 alone (no block-wide scan): lane l owns bins
+// [l*nbins/32, (l+1)*nbins/32).  All threads call it; ends synchronised.
+__device__ __forceinline__ void find_bin_warp(const uint32_t* hist, int nbins, uint32_t krem, uint32_t* sel) {
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    const int bpl = nbins / 32;
+    const uint32_t* hp = hist + lane * bpl;
+    uint32_t local = 0;
+#pragma unroll 8
+    for (int q = 0; q < bpl; ++q) local += hp[q];
+    uint32_t incl = local;   // hits in this lane's bins and every higher lane's
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_down_sync(0xffffffffu, incl, o);
+      if (lane + o < 32) incl += y;
+    }
+    const uint32_t above = incl - local;
+    if (above < krem && above + local >= krem) {
+      uint32_t acc = above;
+      for (int q = bpl - 1; q >= 0; --q) {
+        const uint32_t h = hp[q];
+        if (acc + h >= krem) {
+          sel[0] = static_cast<uint32_t>(lane * bpl + q);
+          sel[1] = acc;
+          break;
+        }
+        acc += h;
+      }
+    }
+  }
+  __syncthreads();
+}
+
+// Radix select over values in shared memory: the krem-th largest of vals[0..m), resolving
+// `passes` 8-bit digits from the top (4 passes resolve the whole key; unresolved low bits are
+// returned as zero).  *left = how many values equal to the result (on the resolved bits) are still
+// to be taken.  After the last pass hist[] holds that pass's histogram.  Needs >= 256 threads.
 __device__ uint32_t smem_select(const uint32_t* vals, int m, uint32_t krem, int passes, uint32_t* hist, uint32_t* ws,
                                 uint32_t* sel, uint32_t* left) {
-  const int shifts[3] = {21, 10, 0};
-  const int widths[3] = {11, 11, 10};
+  (void)ws;
   uint32_t prefix = 0, pmask = 0;
   for (int pass = 0; pass < passes; ++pass) {
-    const int shift = shifts[pass], nbins = 1 << widths[pass];
-    const uint32_t dmask = static_cast<uint32_t>(nbins - 1);
-    for (int i = threadIdx.x; i < nbins; i += kTopkThreads) hist[i] = 0;
+    const int shift = 24 - 8 * pass;
+    if (threadIdx.x < 256) hist[threadIdx.x] = 0;
     __syncthreads();
     for (int base = 0; base < m; base += kTopkThreads) {
       const int i = base + threadIdx.x;
       const uint32_t v = i < m ? vals[i] : 0u;
       const bool hit = i < m && (v & pmask) == prefix;
-      hist_add(hist, hit, (v >> shift) & dmask);
+      hist_add(hist, hit, (v >> shift) & 0xFFu);
     }
     __syncthreads();
-    find_bin(hist, nbins, krem, ws, sel);
+    find_bin_warp(hist, 256, krem, sel);   // ends synchronised
     prefix |= sel[0] << shift;
-    pmask |= dmask << shift;
+    pmask |= 0xFFu << shift;
     krem -= sel[1];
-    __syncthreads();
   }
   *left = krem;
   return prefix;
@@ -188,7 +234,7 @@ __device__ void topk_global(const float* s, int n, int k, int32_t* out, uint32_t
   }
 }
 
-__global__ void __launch_bounds__(kTopkThreads) topk_kernel(const float* __restrict__ scores, long long ld,
+__global__ void __launch_bounds__(kTopkThreads, 3) topk_kernel(const float* __restrict__ scores, long long ld,
                                                             long long batch_stride, const int32_t* __restrict__ seqlens,
                                                             int Tq, int NBk, int blk, long long q_pos0, int b0,
                                                             int row0, int k, int32_t* __restrict__ idx,
@@ -238,8 +284,28 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const float* __restr
     m = n;
     __syncthreads();
   } else {
-    for (int j = tid; j < kSamples; j += kTopkThreads)
-      samp[j] = key_of(s[static_cast<int>((static_cast<long long>(j) * n) / kSamples)]);
+    // Samples: kSamples/128 evenly spaced runs of 128 consecutive scores (one 16-byte load per
+    // thread; coalesced per warp).
+    {
+      constexpr int kRuns = kSamples / 128;
+      for (int j = tid; j < kSamples / 4; j += kTopkThreads) {
+        const int run = j >> 5, off = (j & 31) * 4;
+        const int i0 = (static_cast<int>((static_cast<long long>(run) * n) / kRuns) & ~3) + off;
+        float4 f;
+        if ((reinterpret_cast<uintptr_t>(s) & 15u) == 0 && i0 + 3 < n) {
+          f = __ldcs(reinterpret_cast<const float4*>(s + i0));
+        } else {
+          f.x = s[min(i0, n - 1)];
+          f.y = s[min(i0 + 1, n - 1)];
+          f.z = s[min(i0 + 2, n - 1)];
+          f.w = s[min(i0 + 3, n - 1)];
+        }
+        samp[4 * j] = key_of(f.x);
+        samp[4 * j + 1] = key_of(f.y);
+        samp[4 * j + 2] = key_of(f.z);
+        samp[4 * j + 3] = key_of(f.w);
+      }
+    }
     __syncthreads();
     const long long target = min(static_cast<long long>(k) * 5 / 2 + 128, static_cast<long long>(k + kCap) / 2);
     long long rank = (static_cast<long long>(kSamples) * target + n - 1) / n;
@@ -251,51 +317,58 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const float* __restr
       const uint32_t tau = smem_select(samp, kSamples, static_cast<uint32_t>(rank), 2, hist, ws, sel, &dummy);
       if (tid == 0) misc[0] = 0;
       __syncthreads();
+      // tau back to the float it orders like (keys of finite floats are never 0x7FFFFFFF..0)
+      const float tau_f = __uint_as_float((tau & 0x80000000u) ? (tau & 0x7FFFFFFFu) : ~tau);
       // kU independent 16-byte loads per thread are in flight before any of them is used.
-      constexpr int kU = 4;
+      constexpr int kU = QSA_TOPK_LOADS;
       for (int base = 0; base < n; base += 4 * kTopkThreads * kU) {
-        uint32_t key[kU][4];
+        float v[kU][4];
 #pragma unroll
         for (int u = 0; u < kU; ++u) {
           const int i0 = base + 4 * (u * kTopkThreads + tid);
           if (vec && i0 + 3 < n) {
             const float4 f = __ldcs(reinterpret_cast<const float4*>(s + i0));
-            key[u][0] = key_of(f.x);
-            key[u][1] = key_of(f.y);
-            key[u][2] = key_of(f.z);
-            key[u][3] = key_of(f.w);
+            v[u][0] = f.x;
+            v[u][1] = f.y;
+            v[u][2] = f.z;
+            v[u][3] = f.w;
           } else {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) key[u][e] = i0 + e < n ? key_of(s[i0 + e]) : 0u;
+            for (int e = 0; e < 4; ++e) v[u][e] = i0 + e < n ? s[i0 + e] : -INFINITY;
           }
         }
 #pragma unroll
         for (int u = 0; u < kU; ++u) {
           const int i0 = base + 4 * (u * kTopkThreads + tid);
-          uint32_t hm = 0;
-#pragma unroll
-          for (int e = 0; e < 4; ++e) hm |= (i0 + e < n && key[u][e] >= tau ? 1u : 0u) << e;
+          const int nvalid = min(4, max(0, n - i0));
+          const uint32_t hm = ((v[u][0] >= tau_f ? 1u : 0u) | (v[u][1] >= tau_f ? 2u : 0u) |
+                               (v[u][2] >= tau_f ? 4u : 0u) | (v[u][3] >= tau_f ? 8u : 0u)) &
+                              ((1u << nvalid) - 1u);
+#if QSA_TOPK_APPEND == 1
+          if (hm) {   // a shared-memory atomic per thread that has candidates
+            uint32_t p = atomicAdd(&misc[0], static_cast<uint32_t>(__popc(hm)));
+#else
           const uint32_t nh = static_cast<uint32_t>(__popc(hm));
-          const unsigned any = __ballot_sync(0xffffffffu, nh != 0);
-          if (any == 0u) continue;   // warp-uniform: nothing of this warp passes the threshold
-          uint32_t incl = nh;
+          if (__ballot_sync(0xffffffffu, nh != 0) != 0u) {   // warp-uniform
+            uint32_t incl = nh;
 #pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += y;
-          }
-          uint32_t wbase = 0;
-          if (lane == 31) wbase = atomicAdd(&misc[0], incl);
-          wbase = __shfl_sync(0xffffffffu, wbase, 31);
-          uint32_t p = wbase + incl - nh;
+            for (int o = 1; o < 32; o <<= 1) {
+              const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+              if (lane >= o) incl += y;
+            }
+            uint32_t wbase = 0;
+            if (lane == 31) wbase = atomicAdd(&misc[0], incl);
+            uint32_t p = __shfl_sync(0xffffffffu, wbase, 31) + incl - nh;
+#endif
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            if (hm & (1u << e)) {
-              if (p < static_cast<uint32_t>(kCap)) {
-                cand_key[p] = key[u][e];
-                cand_idx[p] = static_cast<uint32_t>(i0 + e);
+            for (int e = 0; e < 4; ++e) {
+              if (hm & (1u << e)) {
+                if (p < static_cast<uint32_t>(kCap)) {
+                  cand_key[p] = key_of(v[u][e]);
+                  cand_idx[p] = static_cast<uint32_t>(i0 + e);
+                }
+                ++p;
               }
-              ++p;
             }
           }
         }
@@ -320,8 +393,8 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const float* __restr
 
   // ---- 3. exact k-th key among the candidates, then the index cutoff among equal keys
   uint32_t need_eq;
-  const uint32_t kth = smem_select(cand_key, m, static_cast<uint32_t>(k), 3, hist, ws, sel, &need_eq);
-  const uint32_t n_eq = hist[kth & 0x3FFu];   // last pass: hits in the K* bin = keys equal to K*
+  const uint32_t kth = smem_select(cand_key, m, static_cast<uint32_t>(k), 4, hist, ws, sel, &need_eq);
+  const uint32_t n_eq = hist[kth & 0xFFu];   // last pass: hits in the K* bin = keys equal to K*
   uint32_t icut = 0xFFFFFFFFu;
   if (need_eq < n_eq) {
     // the need_eq smallest indices among the keys equal to K*: select on ~index among them
@@ -342,7 +415,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const float* __restr
       return;
     }
     uint32_t dummy;
-    icut = ~smem_select(inv, ne, need_eq, 3, hist, ws, sel, &dummy);
+    icut = ~smem_select(inv, ne, need_eq, 4, hist, ws, sel, &dummy);
   }
 
   // ---- 4-5. bitmap of the kept set, emitted in ascending order

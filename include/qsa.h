@@ -135,7 +135,10 @@ QSA_API qsa_status_t qsa_index_score(const void* qi, const void* kp, const float
  *   head_w, mode and workspace are ignored.
  * scores == NULL: the scores are computed here, chunk by chunk, into `workspace` (at least one
  *   score row of NBk floats; qsa_workspace_size(QSA_OP_SELECT_TOPK, ...) gives the size that lets
- *   the whole call run in few chunks).  Arguments as for qsa_index_score.
+ *   the whole call run in few chunks).  Arguments as for qsa_index_score.  With more than one
+ *   chunk the workspace is split in two halves and the top-k of one chunk runs on a per-device
+ *   internal stream while the next chunk is scored on `stream`; the internal stream is joined back
+ *   into `stream` before the call returns, so the call keeps the usual stream-ordered semantics.
  * Errors: INVALID_ARGUMENT (k < 1, ...), UNSUPPORTED, WORKSPACE_TOO_SMALL.
  */
 QSA_API qsa_status_t qsa_select_topk(const float* scores, int64_t ld_scores, const void* qi,
