@@ -18,7 +18,7 @@
 //   epilogue of tile i overlap the MMAs of tile i+1.  The causal bound is per CTA (tiles up to the
 //   last query row's visible blocks); the store mask is per query.
 // Decode: one query per sequence, so the contraction degenerates to a GEMV over the pooled-key
-//   cache; it is HBM-bound and runs as mma.sync tiles with the query heads in the N dimension.
+//   cache; it is HBM-bound: TMA-fed mma.sync tiles with the query heads in the N dimension.
 #include <mutex>
 
 #include "launch.h"
@@ -222,33 +222,65 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
 
 // ------------------------------------------------------------------------------ decode
 // One query per sequence: s(b) for the pooled keys of the cache, a GEMV bound by reading 128 bytes
-// per block.  mma.m16n8k16 does the arithmetic: 16 pooled keys x 8 head columns per tile (the Hi
-// indexer heads fill N, zero past Hi), the query's B fragments stay in registers and the keys' A
-// fragments are loaded straight from global memory (every byte once; the two halves of a 32-byte
-// sector are read by consecutive loads and meet in L1).  The 4 lanes of a key row then add their
-// heads with two shuffles.
+// per block.  A producer warp streams tiles of 128 pooled keys (16 KB, 128-byte swizzle) into a
+// 4-stage ring with TMA; four consumer warps take 32 keys each and run mma.m16n8k16 (16 keys x 8
+// head columns; the Hi indexer heads fill N, zero past Hi) with the query's B fragments in
+// registers and the keys' A fragments from ldmatrix on the swizzled tile (conflict-free).  The four
+// lanes of a key row then add their heads with two shuffles.
+constexpr int kDecStages = 4;
+constexpr int kDecThreads = 160;
+constexpr int kDecSmem = 1024 + kDecStages * kKpBytes + 128;
+
 template <int HI>
-__global__ void __launch_bounds__(256) score_decode_kernel(const uint16_t* __restrict__ qi,
-                                                           const uint16_t* __restrict__ kp,
-                                                           const float* __restrict__ head_w,
-                                                           const int32_t* __restrict__ seqlens, int NBk, int blk,
-                                                           int mode, float* __restrict__ scores, long long ld,
-                                                           int part_len, KernelCtl ctl) {
+__global__ void __launch_bounds__(kDecThreads) score_decode_kernel(const __grid_constant__ CUtensorMap kp_map,
+                                                                   const uint16_t* __restrict__ qi,
+                                                                   const float* __restrict__ head_w,
+                                                                   const int32_t* __restrict__ seqlens, int NBk,
+                                                                   int blk, int mode, float* __restrict__ scores,
+                                                                   long long ld, int part_len, KernelCtl ctl) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(ring + kDecStages * kKpBytes);
+  uint64_t* empty = full + kDecStages;
   const int b = blockIdx.y;
   const int L = seqlens[b];
-  if (L < 1) {
+  int nb = L >= 1 ? (L - 1) / blk : 0;
+  if (L < 1 || nb > NBk) {
     if (blockIdx.x == 0 && threadIdx.x == 0) record_status(ctl, kStBadArg);
-    return;
-  }
-  int nb = (L - 1) / blk;
-  if (nb > NBk) {
-    if (blockIdx.x == 0 && threadIdx.x == 0) record_status(ctl, kStBadArg);
-    nb = NBk;
+    nb = min(max(nb, 0), NBk);
   }
   const int lo = static_cast<int>(blockIdx.x) * part_len;
   const int c = max(0, min(nb, lo + part_len) - lo);
-  if (c == 0) return;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (c == 0) return;   // uniform over the CTA
+  const int ntiles = (c + kM - 1) / kM;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < kDecStages; ++st) {
+      mbar_init(&full[st], 1);
+      mbar_init(&empty[st], 4);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tensormap(&kp_map);
+      int issued = 0;
+      for (int i = 0; i < ntiles; ++i) {
+        const int st = i % kDecStages;
+        if (!mbar_wait(&empty[st], ((i / kDecStages) & 1u) ^ 1u, ctl)) break;
+        mbar_arrive_expect_tx(&full[st], kKpBytes);
+        tma_load_3d(ring + st * kKpBytes, &kp_map, &full[st], 0, lo + i * kM, b);
+        issued = i + 1;
+      }
+      for (int st = 0; st < kDecStages && st < issued; ++st) {   // no copy left in flight
+        const int last = st + ((issued - 1 - st) / kDecStages) * kDecStages;
+        mbar_wait(&full[st], (last / kDecStages) & 1u, ctl);
+      }
+    }
+    return;
+  }
+  const int cw = warp - 1;   // consumer 0..3: rows 32 cw .. 32 cw + 31 of each tile
   uint32_t bq[4][2];
   {
     const int n = lane >> 2;
@@ -263,35 +295,26 @@ __global__ void __launch_bounds__(256) score_decode_kernel(const uint16_t* __res
   const int h0 = 2 * (lane & 3);
   const float w0 = (h0 < HI) ? (head_w ? head_w[h0] : 1.f) : 0.f;
   const float w1 = (h0 + 1 < HI) ? (head_w ? head_w[h0 + 1] : 1.f) : 0.f;
-  const uint16_t* kpb = kp + (static_cast<long long>(b) * NBk + lo) * kDi;
   float* srow = scores + static_cast<long long>(b) * ld + lo;
-  const int ntiles = (c + 15) / 16;
-  constexpr int kWarps = 8, kUnroll = 4;
-  for (int t0 = warp; t0 < ntiles; t0 += kWarps * kUnroll) {
-    uint32_t a[kUnroll][4][4];
+  // ldmatrix.x4 addressing in a 128-byte-swizzled tile: lane l reads row (l & 7) + 8 ((l >> 3) & 1)
+  // of a 16-row slab, 16-byte chunk 2 kk + (l >> 4), stored at chunk position (chunk ^ (row & 7)).
+  const int lrow = (lane & 7) + 8 * ((lane >> 3) & 1);
+  const int lchunk = lane >> 4;
+  for (int i = 0; i < ntiles; ++i) {
+    const int st = i % kDecStages;
+    if (!mbar_wait(&full[st], (i / kDecStages) & 1u, ctl)) return;
+    const uint32_t tile = smem_u32(ring + st * kKpBytes);
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int t = t0 + u * kWarps;
-      const int r0 = t * 16 + (lane >> 2), r1 = r0 + 8;
-      const bool ok0 = t < ntiles && r0 < c, ok1 = t < ntiles && r1 < c;
-      const uint16_t* p0 = kpb + static_cast<long long>(ok0 ? r0 : 0) * kDi + 2 * (lane & 3);
-      const uint16_t* p1 = kpb + static_cast<long long>(ok1 ? r1 : 0) * kDi + 2 * (lane & 3);
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        a[u][kk][0] = ok0 ? __ldg(reinterpret_cast<const uint32_t*>(p0 + 16 * kk)) : 0u;
-        a[u][kk][1] = ok1 ? __ldg(reinterpret_cast<const uint32_t*>(p1 + 16 * kk)) : 0u;
-        a[u][kk][2] = ok0 ? __ldg(reinterpret_cast<const uint32_t*>(p0 + 16 * kk + 8)) : 0u;
-        a[u][kk][3] = ok1 ? __ldg(reinterpret_cast<const uint32_t*>(p1 + 16 * kk + 8)) : 0u;
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int t = t0 + u * kWarps;
-      if (t >= ntiles) break;   // warp-uniform
+    for (int h = 0; h < 2; ++h) {   // two 16-row slabs per warp
+      const int row = 32 * cw + 16 * h + lrow;
       float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_bf16_16816(acc, a[u][kk][0], a[u][kk][1], a[u][kk][2], a[u][kk][3], bq[kk][0], bq[kk][1]);
+      for (int kk = 0; kk < 4; ++kk) {
+        const int chunk = 2 * kk + lchunk;
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4(tile + row * 128 + ((chunk ^ (row & 7)) << 4), a0, a1, a2, a3);
+        mma_bf16_16816(acc, a0, a1, a2, a3, bq[kk][0], bq[kk][1]);
+      }
       float x0 = acc[0], x1 = acc[1], x2 = acc[2], x3 = acc[3];
       if (mode == 0) {
         x0 = fmaxf(x0, 0.f);
@@ -299,18 +322,20 @@ __global__ void __launch_bounds__(256) score_decode_kernel(const uint16_t* __res
         x2 = fmaxf(x2, 0.f);
         x3 = fmaxf(x3, 0.f);
       }
-      float v0 = fmaf(w1, x1, w0 * x0);   // key row lane/4, this lane's two head columns
+      float v0 = fmaf(w1, x1, w0 * x0);   // key row lane/4 of the slab: this lane's two head columns
       float v1 = fmaf(w1, x3, w0 * x2);   // key row lane/4 + 8
       v0 += __shfl_xor_sync(0xffffffffu, v0, 1);
       v1 += __shfl_xor_sync(0xffffffffu, v1, 1);
       v0 += __shfl_xor_sync(0xffffffffu, v0, 2);
       v1 += __shfl_xor_sync(0xffffffffu, v1, 2);
-      const int r0 = t * 16 + (lane >> 2), r1 = r0 + 8;
+      const int r0 = i * kM + 32 * cw + 16 * h + (lane >> 2), r1 = r0 + 8;
       if ((lane & 3) == 0) {
         if (r0 < c) srow[r0] = v0;
         if (r1 < c) srow[r1] = v1;
       }
     }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[st]);
   }
 }
 
@@ -402,17 +427,28 @@ cudaError_t launch_score_decode(const DeviceInfo* di, const void* qi, const void
   (void)Di;
   if (B <= 0 || NBk <= 0) return cudaSuccess;
   const KernelCtl ctl = kernel_ctl(di);
-  // about four CTAs per SM in total, parts of at least 1024 pooled keys
-  const int parts = std::max(1, std::min((di->num_sms * 4 + B - 1) / B, (NBk + 1023) / 1024));
-  const int part_len = ((NBk + parts - 1) / parts + 15) / 16 * 16;
+  CUtensorMap kmap;
+  if (!make_map(&kmap, kp, static_cast<unsigned long long>(NBk), static_cast<unsigned long long>(B), kM))
+    return cudaErrorInvalidValue;
+  static std::once_flag once[64];
+  std::call_once(once[di->device & 63], [] {
+    cudaFuncSetAttribute(score_decode_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem);
+    cudaFuncSetAttribute(score_decode_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem);
+    cudaFuncSetAttribute(score_decode_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem);
+    cudaFuncSetAttribute(score_decode_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem);
+  });
+  // about three CTAs per SM in total; parts are whole 128-key tiles
+  const int want = std::max(1, (di->num_sms * 3 + B - 1) / B);
+  const int tiles = (NBk + kM - 1) / kM;
+  const int part_tiles = std::max(1, (tiles + want - 1) / want);
+  const int part_len = part_tiles * kM;
   dim3 grid((NBk + part_len - 1) / part_len, B);
   const uint16_t* q = static_cast<const uint16_t*>(qi);
-  const uint16_t* k = static_cast<const uint16_t*>(kp);
   switch (Hi) {
-    case 1: score_decode_kernel<1><<<grid, 256, 0, s>>>(q, k, head_w, seqlens, NBk, blk, mode, scores, ld, part_len, ctl); break;
-    case 2: score_decode_kernel<2><<<grid, 256, 0, s>>>(q, k, head_w, seqlens, NBk, blk, mode, scores, ld, part_len, ctl); break;
-    case 4: score_decode_kernel<4><<<grid, 256, 0, s>>>(q, k, head_w, seqlens, NBk, blk, mode, scores, ld, part_len, ctl); break;
-    case 8: score_decode_kernel<8><<<grid, 256, 0, s>>>(q, k, head_w, seqlens, NBk, blk, mode, scores, ld, part_len, ctl); break;
+    case 1: score_decode_kernel<1><<<grid, kDecThreads, kDecSmem, s>>>(kmap, q, head_w, seqlens, NBk, blk, mode, scores, ld, part_len, ctl); break;
+    case 2: score_decode_kernel<2><<<grid, kDecThreads, kDecSmem, s>>>(kmap, q, head_w, seqlens, NBk, blk, mode, scores, ld, part_len, ctl); break;
+    case 4: score_decode_kernel<4><<<grid, kDecThreads, kDecSmem, s>>>(kmap, q, head_w, seqlens, NBk, blk, mode, scores, ld, part_len, ctl); break;
+    case 8: score_decode_kernel<8><<<grid, kDecThreads, kDecSmem, s>>>(kmap, q, head_w, seqlens, NBk, blk, mode, scores, ld, part_len, ctl); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaPeekAtLastError();

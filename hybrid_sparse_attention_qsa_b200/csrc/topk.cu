@@ -443,6 +443,277 @@ __global__ void __launch_bounds__(kTopkThreads, 3) topk_kernel(const float* __re
   }
 }
 
+
+// ======================================================================================
+// Warp-per-row variant (used when there are many rows): one warp owns a row end to end, so no
+// phase needs a block-wide barrier, and the 16 warps of an SM work on 16 rows at once.
+//   1. 1024 samples (32 runs of 32 consecutive scores) give tau, a little below the k-th largest
+//      (about 2k + 128 scores expected above it; two 8-bit radix passes on the samples);
+//   2. one pass over the row (kWU 16-byte loads per lane in flight) appends every score >= tau to
+//      the warp's shared-memory list IN INDEX ORDER (ballot-based compaction);
+//   3. four 8-bit radix passes over the list give the k-th key K* and how many keys equal to K* are
+//      kept (the lowest indices, since the list is in index order);
+//   4. one ordered pass over the list emits the kept indices ascending.
+// A row whose list would overflow (or hold fewer than k) moves tau and retries; after three tries
+// the warp falls back to four radix passes over the whole row in memory.
+constexpr int kWarpRowsPerCta = 8;
+constexpr int kWU = 8;            // 16-byte loads in flight per lane in the filter pass
+constexpr int kWSamples = 1024;
+
+__device__ __forceinline__ uint32_t lanemask_lt() {
+  uint32_t m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+// Warp-level radix select: the krem-th largest of vals[0..m) resolving `passes` 8-bit digits from
+// the top.  hist = 256 words of this warp.  *left = how many values equal to the result remain.
+__device__ uint32_t warp_select(const uint32_t* vals, int m, uint32_t krem, int passes, uint32_t* hist,
+                                uint32_t* left) {
+  const int lane = threadIdx.x & 31;
+  uint32_t prefix = 0, pmask = 0;
+  for (int pass = 0; pass < passes; ++pass) {
+    const int shift = 24 - 8 * pass;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) hist[lane * 8 + q] = 0;
+    __syncwarp();
+    for (int base = 0; base < m; base += 32) {
+      const int i = base + lane;
+      const uint32_t v = i < m ? vals[i] : 0u;
+      const bool hit = i < m && (v & pmask) == prefix;
+      const uint32_t digit = (v >> shift) & 0xFFu;
+      const uint32_t peers = __match_any_sync(0xffffffffu, hit ? digit : 0xFFFFFFFFu);
+      if (hit && lane == __ffs(peers) - 1) hist[digit] += static_cast<uint32_t>(__popc(peers));
+      __syncwarp();
+    }
+    const uint32_t* hp = hist + lane * 8;
+    uint32_t local = 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) local += hp[q];
+    uint32_t incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_down_sync(0xffffffffu, incl, o);
+      if (lane + o < 32) incl += y;
+    }
+    const uint32_t above = incl - local;
+    uint32_t mybin = 0, myabove = 0;
+    const bool mine = above < krem && above + local >= krem;
+    if (mine) {
+      uint32_t acc = above;
+      for (int q = 7; q >= 0; --q) {
+        if (acc + hp[q] >= krem) {
+          mybin = static_cast<uint32_t>(lane * 8 + q);
+          myabove = acc;
+          break;
+        }
+        acc += hp[q];
+      }
+    }
+    const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
+    const uint32_t bin = __shfl_sync(0xffffffffu, mybin, src);
+    krem -= __shfl_sync(0xffffffffu, myabove, src);
+    prefix |= bin << shift;
+    pmask |= 0xFFu << shift;
+    __syncwarp();
+  }
+  *left = krem;
+  return prefix;
+}
+
+__global__ void __launch_bounds__(kWarpRowsPerCta * 32) topk_warp_kernel(
+    const float* __restrict__ scores, long long ld, long long batch_stride, int Tq, int NBk, long long q_pos0, int b0,
+    int row0, int rows, int k, int cap, int32_t* __restrict__ idx) {
+  extern __shared__ uint32_t smw[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint32_t* ckey = smw + warp * (2 * cap + 256);   // cap keys, then cap indices, then 256 hist words
+  uint32_t* cidx = ckey + cap;
+  uint32_t* hist = cidx + cap;
+  const int r = row0 + static_cast<int>(blockIdx.x) * kWarpRowsPerCta + warp;
+  if (r >= row0 + rows) return;
+  const int bz = blockIdx.y;
+  const int b = b0 + bz;
+  const long long pos = q_pos0 + r;
+  const int n = static_cast<int>(min(static_cast<long long>(NBk), pos / 4));
+  const float* s = scores + static_cast<long long>(bz) * batch_stride + static_cast<long long>(r - row0) * ld;
+  int32_t* out = idx + (static_cast<long long>(b) * Tq + r) * k;
+  if (n <= k) {
+    for (int i = lane; i < k; i += 32) out[i] = i < n ? i : -1;
+    return;
+  }
+  const bool vec = (reinterpret_cast<uintptr_t>(s) & 15u) == 0;
+  const uint32_t lt = lanemask_lt();
+
+  // ---- candidates in index order
+  float tau_f = -INFINITY;
+  int m = 0;
+  bool ok = false;
+  long long rank = 0;
+  if (n > cap) {
+    // samples: 32 runs of 32 consecutive scores (coalesced 128-byte loads)
+#pragma unroll 4
+    for (int run = 0; run < 32; ++run) {
+      const int i = static_cast<int>((static_cast<long long>(run) * (n - 32)) / 31) + lane;
+      ckey[run * 32 + lane] = key_of(s[i]);
+    }
+    __syncwarp();
+    const long long target = 2ll * k + 128;
+    rank = (static_cast<long long>(kWSamples) * target + n - 1) / n;
+  }
+  for (int attempt = 0; attempt < 3 && !ok; ++attempt) {
+    if (n > cap) {
+      rank = max(1ll, min(rank, static_cast<long long>(kWSamples)));
+      uint32_t dummy;
+      const uint32_t tau = warp_select(ckey, kWSamples, static_cast<uint32_t>(rank), 2, hist, &dummy);
+      tau_f = __uint_as_float((tau & 0x80000000u) ? (tau & 0x7FFFFFFFu) : ~tau);
+    }
+    uint32_t cnt = 0;
+    bool over = false;
+    for (int base = 0; base < n; base += 128 * kWU) {
+      float v[kWU][4];
+#pragma unroll
+      for (int u = 0; u < kWU; ++u) {
+        const int i0 = base + (u * 32 + lane) * 4;
+        if (vec && i0 + 3 < n) {
+          const float4 f = __ldcs(reinterpret_cast<const float4*>(s + i0));
+          v[u][0] = f.x;
+          v[u][1] = f.y;
+          v[u][2] = f.z;
+          v[u][3] = f.w;
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) v[u][e] = i0 + e < n ? s[i0 + e] : -INFINITY;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kWU; ++u) {
+        const int i0 = base + (u * 32 + lane) * 4;
+        uint32_t hm = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) hm |= (i0 + e < n && v[u][e] >= tau_f ? 1u : 0u) << e;
+        const uint32_t m0 = __ballot_sync(0xffffffffu, hm & 1u), m1 = __ballot_sync(0xffffffffu, hm & 2u);
+        const uint32_t m2 = __ballot_sync(0xffffffffu, hm & 4u), m3 = __ballot_sync(0xffffffffu, hm & 8u);
+        const uint32_t total = __popc(m0) + __popc(m1) + __popc(m2) + __popc(m3);
+        if (total == 0) continue;
+        uint32_t p = cnt + __popc(m0 & lt) + __popc(m1 & lt) + __popc(m2 & lt) + __popc(m3 & lt);
+        if (cnt + total <= static_cast<uint32_t>(cap)) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            if (hm & (1u << e)) {
+              ckey[p] = key_of(v[u][e]);
+              cidx[p] = static_cast<uint32_t>(i0 + e);
+              ++p;
+            }
+          }
+        } else {
+          over = true;
+        }
+        cnt += total;
+      }
+      if (__any_sync(0xffffffffu, over)) break;
+    }
+    __syncwarp();
+    if (!over && cnt >= static_cast<uint32_t>(k)) {
+      ok = true;
+      m = static_cast<int>(cnt);
+    } else if (n > cap) {
+      // re-draw the samples (the list overwrote them) and move the threshold
+#pragma unroll 4
+      for (int run = 0; run < 32; ++run) {
+        const int i = static_cast<int>((static_cast<long long>(run) * (n - 32)) / 31) + lane;
+        ckey[run * 32 + lane] = key_of(s[i]);
+      }
+      __syncwarp();
+      rank = over ? rank / 4 : rank * 4;
+    } else {
+      break;   // n <= cap always succeeds with tau = -inf; not reached
+    }
+  }
+
+  uint32_t kth, need_eq;
+  if (ok) {
+    kth = warp_select(ckey, m, static_cast<uint32_t>(k), 4, hist, &need_eq);
+  } else {
+    // fallback: four radix passes over the row in memory
+    uint32_t prefix = 0, pmask = 0, krem = static_cast<uint32_t>(k);
+    for (int pass = 0; pass < 4; ++pass) {
+      const int shift = 24 - 8 * pass;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) hist[lane * 8 + q] = 0;
+      __syncwarp();
+      for (int base = 0; base < n; base += 32) {
+        const int i = base + lane;
+        const uint32_t key = i < n ? key_of(s[i]) : 0u;
+        const bool hit = i < n && (key & pmask) == prefix;
+        const uint32_t digit = (key >> shift) & 0xFFu;
+        const uint32_t peers = __match_any_sync(0xffffffffu, hit ? digit : 0xFFFFFFFFu);
+        if (hit && lane == __ffs(peers) - 1) hist[digit] += static_cast<uint32_t>(__popc(peers));
+        __syncwarp();
+      }
+      const uint32_t* hp = hist + lane * 8;
+      uint32_t local = 0;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) local += hp[q];
+      uint32_t incl = local;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_down_sync(0xffffffffu, incl, o);
+        if (lane + o < 32) incl += y;
+      }
+      const uint32_t above = incl - local;
+      uint32_t mybin = 0, myabove = 0;
+      const bool mine = above < krem && above + local >= krem;
+      if (mine) {
+        uint32_t acc = above;
+        for (int q = 7; q >= 0; --q) {
+          if (acc + hp[q] >= krem) {
+            mybin = static_cast<uint32_t>(lane * 8 + q);
+            myabove = acc;
+            break;
+          }
+          acc += hp[q];
+        }
+      }
+      const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
+      prefix |= __shfl_sync(0xffffffffu, mybin, src) << shift;
+      krem -= __shfl_sync(0xffffffffu, myabove, src);
+      pmask |= 0xFFu << shift;
+      __syncwarp();
+    }
+    kth = prefix;
+    need_eq = krem;
+  }
+
+  // ---- ordered emission (the list, or the whole row on the fallback, is in index order)
+  uint32_t out_run = 0, eq_run = 0;
+  const int len = ok ? m : n;
+  for (int base = 0; base < len; base += 32) {
+    const int i = base + lane;
+    uint32_t key = 0, id = 0;
+    if (i < len) {
+      if (ok) {
+        key = ckey[i];
+        id = cidx[i];
+      } else {
+        key = key_of(s[i]);
+        id = static_cast<uint32_t>(i);
+      }
+    }
+    const bool gt = i < len && key > kth;
+    const bool eq = i < len && key == kth;
+    const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
+    const uint32_t eq_rank = eq_run + __popc(eqm & lt);
+    const bool keep = gt || (eq && eq_rank < need_eq);
+    const uint32_t km = __ballot_sync(0xffffffffu, keep);
+    if (keep) {
+      const uint32_t p = out_run + __popc(km & lt);
+      if (p < static_cast<uint32_t>(k)) out[p] = static_cast<int32_t>(id);
+    }
+    out_run += __popc(km);
+    eq_run += __popc(eqm);
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_topk(const DeviceInfo* di, const float* scores, long long ld, long long batch_stride,
@@ -454,6 +725,19 @@ cudaError_t launch_topk(const DeviceInfo* di, const float* scores, long long ld,
     cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          kFixedSmem + 32 + kMaxBitmapWords * 4);
   });
+  // Many rows (prefill chunks): one warp per row.  Few long rows (decode): one CTA per row.
+  const int cap = std::max(3 * k, kWSamples);
+  const int warp_smem = kWarpRowsPerCta * (2 * cap + 256) * 4;
+  if (seqlens == nullptr && static_cast<long long>(rows) * nb >= 8ll * di->num_sms && warp_smem <= 200 * 1024) {
+    static std::once_flag wonce[64];
+    std::call_once(wonce[di->device & 63], [] {
+      cudaFuncSetAttribute(topk_warp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    });
+    dim3 wgrid((rows + kWarpRowsPerCta - 1) / kWarpRowsPerCta, nb);
+    topk_warp_kernel<<<wgrid, kWarpRowsPerCta * 32, warp_smem, s>>>(scores, ld, batch_stride, Tq, NBk, q_pos0, b0,
+                                                                    row0, rows, k, cap, idx);
+    return cudaPeekAtLastError();
+  }
   const int words = std::min(kMaxBitmapWords, (std::max(NBk, 1) + 31) / 32);
   const int smem = kFixedSmem + 32 + words * 4;
   dim3 grid(rows, nb);

@@ -139,6 +139,21 @@ def test_topk_bit_exact_from_scores(n_rows, pos0, k, levels):
     _status_ok()
 
 
+@pytest.mark.parametrize("n_rows,pos0,k,levels", [(1600, 60000, 512, 0), (1300, 40000, 512, 3), (1300, 9000, 64, 2),
+                                                  (1200, 3000, 512, 0), (1200, 262000, 1024, 0)])
+def test_topk_many_rows_bit_exact(n_rows, pos0, k, levels):
+    """Enough rows for the warp-per-row kernel, including heavy ties (threshold retries and the
+    in-memory fallback) and rows shorter than k."""
+    s, nbk = _topk_case(n_rows, pos0, k, levels, n_rows * 7 + k)
+    st = torch.from_numpy(s).to(DEV)
+    idx = Q.qsa_select_topk(k, scores=st, NBk=nbk, q_pos0=pos0).cpu().numpy()
+    for r in list(range(0, n_rows, 37)) + [n_rows - 1]:
+        n = (pos0 + r) // 4
+        ref, _ = O.select_topk(s[0, r, :n], k)
+        assert np.array_equal(idx[0, r], ref), (r, n)
+    _status_ok()
+
+
 def test_topk_decode_rows_bit_exact():
     B, L, k = 6, 262144, 512
     nbk = L // 4
