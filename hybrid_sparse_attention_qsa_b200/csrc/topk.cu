@@ -448,17 +448,29 @@ __global__ void __launch_bounds__(kTopkThreads, 3) topk_kernel(const float* __re
 // Warp-per-row variant (used when there are many rows): one warp owns a row end to end, so no
 // phase needs a block-wide barrier, and the 16 warps of an SM work on 16 rows at once.
 //   1. 1024 samples (32 runs of 32 consecutive scores) give tau, a little below the k-th largest
-//      (about 2k + 128 scores expected above it; two 8-bit radix passes on the samples);
+//      (about 1.8k + 64 scores expected above it; two 8-bit radix passes on the samples);
 //   2. one pass over the row (kWU 16-byte loads per lane in flight) appends every score >= tau to
 //      the warp's shared-memory list IN INDEX ORDER (ballot-based compaction);
 //   3. four 8-bit radix passes over the list give the k-th key K* and how many keys equal to K* are
 //      kept (the lowest indices, since the list is in index order);
 //   4. one ordered pass over the list emits the kept indices ascending.
-// A row whose list would overflow (or hold fewer than k) moves tau and retries; after three tries
-// the warp falls back to four radix passes over the whole row in memory.
-constexpr int kWarpRowsPerCta = 8;
-constexpr int kWU = 8;            // 16-byte loads in flight per lane in the filter pass
+// A row whose list would overflow (or hold fewer than k) moves tau by bisection on its sample rank
+// and retries; if no rank works (heavy ties) the warp falls back to four radix passes over the
+// whole row in memory.
+#ifndef QSA_TOPK_WROWS
+#define QSA_TOPK_WROWS 8
+#endif
+constexpr int kWarpRowsPerCta = QSA_TOPK_WROWS;
+#ifndef QSA_TOPK_WLOAD
+#define QSA_TOPK_WLOAD 0
+#endif
+#ifndef QSA_TOPK_WU
+#define QSA_TOPK_WU 8
+#endif
+constexpr int kWU = QSA_TOPK_WU;   // 16-byte loads in flight per lane in the filter pass
 constexpr int kWSamples = 1024;
+// Rows longer than this go to the CTA-per-row kernel, whose filter pass streams faster.
+constexpr int kWarpRowMax = 8192;
 
 __device__ __forceinline__ uint32_t lanemask_lt() {
   uint32_t m;
@@ -466,56 +478,28 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
   return m;
 }
 
-// Warp-level radix select: the krem-th largest of vals[0..m) resolving `passes` 8-bit digits from
-// the top.  hist = 256 words of this warp.  *left = how many values equal to the result remain.
+// Warp-level select, one bit at a time from the top: the krem-th largest of vals[0..m), resolving
+// the top 8*passes bits (unresolved low bits returned as zero).  Each bit costs one ballot + popc
+// per 32 values (no histogram, no atomics).  *left = how many values equal to the result (on the
+// resolved bits) remain to be taken.
 __device__ uint32_t warp_select(const uint32_t* vals, int m, uint32_t krem, int passes, uint32_t* hist,
                                 uint32_t* left) {
+  (void)hist;
   const int lane = threadIdx.x & 31;
-  uint32_t prefix = 0, pmask = 0;
-  for (int pass = 0; pass < passes; ++pass) {
-    const int shift = 24 - 8 * pass;
-#pragma unroll
-    for (int q = 0; q < 8; ++q) hist[lane * 8 + q] = 0;
-    __syncwarp();
+  uint32_t prefix = 0;
+  const int lowest = 32 - 8 * passes;
+  for (int bit = 31; bit >= lowest; --bit) {
+    const uint32_t want = (prefix >> bit) | 1u;   // top bits of prefix with this bit set
+    uint32_t cnt = 0;
     for (int base = 0; base < m; base += 32) {
       const int i = base + lane;
-      const uint32_t v = i < m ? vals[i] : 0u;
-      const bool hit = i < m && (v & pmask) == prefix;
-      const uint32_t digit = (v >> shift) & 0xFFu;
-      const uint32_t peers = __match_any_sync(0xffffffffu, hit ? digit : 0xFFFFFFFFu);
-      if (hit && lane == __ffs(peers) - 1) hist[digit] += static_cast<uint32_t>(__popc(peers));
-      __syncwarp();
+      const bool hit = i < m && (vals[i] >> bit) == want;
+      cnt += __popc(__ballot_sync(0xffffffffu, hit));
     }
-    const uint32_t* hp = hist + lane * 8;
-    uint32_t local = 0;
-#pragma unroll
-    for (int q = 0; q < 8; ++q) local += hp[q];
-    uint32_t incl = local;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_down_sync(0xffffffffu, incl, o);
-      if (lane + o < 32) incl += y;
-    }
-    const uint32_t above = incl - local;
-    uint32_t mybin = 0, myabove = 0;
-    const bool mine = above < krem && above + local >= krem;
-    if (mine) {
-      uint32_t acc = above;
-      for (int q = 7; q >= 0; --q) {
-        if (acc + hp[q] >= krem) {
-          mybin = static_cast<uint32_t>(lane * 8 + q);
-          myabove = acc;
-          break;
-        }
-        acc += hp[q];
-      }
-    }
-    const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
-    const uint32_t bin = __shfl_sync(0xffffffffu, mybin, src);
-    krem -= __shfl_sync(0xffffffffu, myabove, src);
-    prefix |= bin << shift;
-    pmask |= 0xFFu << shift;
-    __syncwarp();
+    if (cnt >= krem)
+      prefix |= 1u << bit;
+    else
+      krem -= cnt;
   }
   *left = krem;
   return prefix;
@@ -548,21 +532,26 @@ __global__ void __launch_bounds__(kWarpRowsPerCta * 32) topk_warp_kernel(
   float tau_f = -INFINITY;
   int m = 0;
   bool ok = false;
-  long long rank = 0;
-  if (n > cap) {
-    // samples: 32 runs of 32 consecutive scores (coalesced 128-byte loads)
+  // rank of tau among the samples: a larger rank gives a lower tau and more candidates.  A failed
+  // pass narrows (rlo, rhi), the open interval that must hold a working rank.
+  long long rank = 0, rlo = 0, rhi = kWSamples + 1;
+  auto draw_samples = [&]() {
 #pragma unroll 4
     for (int run = 0; run < 32; ++run) {
       const int i = static_cast<int>((static_cast<long long>(run) * (n - 32)) / 31) + lane;
       ckey[run * 32 + lane] = key_of(s[i]);
     }
     __syncwarp();
-    const long long target = 2ll * k + 128;
+  };
+  if (n > cap) {
+    draw_samples();
+    const long long target = (9ll * k) / 5 + 64;
     rank = (static_cast<long long>(kWSamples) * target + n - 1) / n;
   }
-  for (int attempt = 0; attempt < 3 && !ok; ++attempt) {
+  for (int attempt = 0; attempt < 6 && !ok; ++attempt) {
     if (n > cap) {
-      rank = max(1ll, min(rank, static_cast<long long>(kWSamples)));
+      rank = max(rlo + 1, min(rank, rhi - 1));
+      if (rank <= rlo || rank >= rhi) break;   // no rank left to try
       uint32_t dummy;
       const uint32_t tau = warp_select(ckey, kWSamples, static_cast<uint32_t>(rank), 2, hist, &dummy);
       tau_f = __uint_as_float((tau & 0x80000000u) ? (tau & 0x7FFFFFFFu) : ~tau);
@@ -575,7 +564,11 @@ __global__ void __launch_bounds__(kWarpRowsPerCta * 32) topk_warp_kernel(
       for (int u = 0; u < kWU; ++u) {
         const int i0 = base + (u * 32 + lane) * 4;
         if (vec && i0 + 3 < n) {
+#if QSA_TOPK_WLOAD == 1
+          const float4 f = __ldg(reinterpret_cast<const float4*>(s + i0));
+#else
           const float4 f = __ldcs(reinterpret_cast<const float4*>(s + i0));
+#endif
           v[u][0] = f.x;
           v[u][1] = f.y;
           v[u][2] = f.z;
@@ -610,23 +603,23 @@ __global__ void __launch_bounds__(kWarpRowsPerCta * 32) topk_warp_kernel(
         }
         cnt += total;
       }
-      if (__any_sync(0xffffffffu, over)) break;
+      if (over) break;   // warp-uniform
     }
     __syncwarp();
     if (!over && cnt >= static_cast<uint32_t>(k)) {
       ok = true;
       m = static_cast<int>(cnt);
     } else if (n > cap) {
-      // re-draw the samples (the list overwrote them) and move the threshold
-#pragma unroll 4
-      for (int run = 0; run < 32; ++run) {
-        const int i = static_cast<int>((static_cast<long long>(run) * (n - 32)) / 31) + lane;
-        ckey[run * 32 + lane] = key_of(s[i]);
+      draw_samples();   // the list overwrote them
+      if (over) {
+        rhi = rank;
+        rank = (rlo + rank) / 2;
+      } else {
+        rlo = rank;
+        rank = rhi > kWSamples ? rank * 2 : (rank + rhi) / 2;
       }
-      __syncwarp();
-      rank = over ? rank / 4 : rank * 4;
     } else {
-      break;   // n <= cap always succeeds with tau = -inf; not reached
+      break;
     }
   }
 
@@ -725,10 +718,13 @@ cudaError_t launch_topk(const DeviceInfo* di, const float* scores, long long ld,
     cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          kFixedSmem + 32 + kMaxBitmapWords * 4);
   });
-  // Many rows (prefill chunks): one warp per row.  Few long rows (decode): one CTA per row.
+  // Many short rows (early prefill chunks): one warp per row.  Long rows or few rows (late chunks,
+  // decode): one CTA per row.
   const int cap = std::max(3 * k, kWSamples);
   const int warp_smem = kWarpRowsPerCta * (2 * cap + 256) * 4;
-  if (seqlens == nullptr && static_cast<long long>(rows) * nb >= 8ll * di->num_sms && warp_smem <= 200 * 1024) {
+  const long long n_max = std::min<long long>(NBk, (q_pos0 + row0 + rows - 1) / blk);
+  if (seqlens == nullptr && static_cast<long long>(rows) * nb >= 8ll * di->num_sms && warp_smem <= 200 * 1024 &&
+      n_max <= kWarpRowMax) {
     static std::once_flag wonce[64];
     std::call_once(wonce[di->device & 63], [] {
       cudaFuncSetAttribute(topk_warp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);

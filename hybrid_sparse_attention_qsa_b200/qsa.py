@@ -315,3 +315,65 @@ def decode(q, kcache, vcache, qi, kp, seqlens, *, topk: int, rope_theta: float =
     idx = qsa_select_topk(topk, qi=qr, kp=kp, head_w=head_w, seqlens=seqlens, mode=mode, workspace=workspace)
     out, lse = qsa_sparse_attn_decode(q, kcache, vcache, seqlens, idx, scale=scale, num_splits=num_splits)
     return dict(out=out, lse=lse, idx=idx)
+
+
+_copy_streams = {}
+
+
+def _copy_stream(device) -> "torch.cuda.Stream":
+    d = torch.device(device).index
+    if d not in _copy_streams:
+        _copy_streams[d] = torch.cuda.Stream(device=device)
+    return _copy_streams[d]
+
+
+def prefill_host(q, k, v, qi, ki, *, topk: int, device="cuda", out=None, q_pos0: int = 0, rope_theta: float = 0.0,
+                 head_w=None, mode: int = QSA_SCORE_RELU_SUM, scale: float | None = None, workspace=None,
+                 device_buffers: dict | None = None):
+    """The QSA layer for a prefill whose inputs live in (pinned) host memory; returns the output in
+    host memory.  Transfers overlap the kernels: ki and qi are copied first, pooling and block
+    selection run while q, k and v are copied on a second stream, and the attention runs in two
+    halves of the query rows so that the first half's output is copied back while the second half
+    is computed.  ``device_buffers`` (name -> device tensor) lets a caller reuse device memory.
+    Returns dict(out=host tensor, lse=device tensor, idx=device tensor)."""
+    dev = torch.device(device)
+    main = torch.cuda.current_stream(dev)
+    side = _copy_stream(dev)
+    bufs = device_buffers if device_buffers is not None else {}
+    for name, t in (("q", q), ("k", k), ("v", v), ("qi", qi), ("ki", ki)):
+        if name not in bufs:
+            bufs[name] = torch.empty(t.shape, dtype=t.dtype, device=dev)
+    B, Tq, Hq, D = q.shape
+    if out is None:
+        out = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+    if "out" not in bufs:
+        bufs["out"] = torch.empty(q.shape, dtype=q.dtype, device=dev)
+    if "lse" not in bufs:
+        bufs["lse"] = torch.empty(B, Tq, Hq, dtype=torch.float32, device=dev)
+    if "kp" not in bufs:
+        bufs["kp"] = torch.empty(ki.shape[0], ki.shape[1] // 4, ki.shape[2], dtype=ki.dtype, device=dev)
+    bufs["ki"].copy_(ki, non_blocking=True)
+    bufs["qi"].copy_(qi, non_blocking=True)
+    side.wait_stream(main)
+    with torch.cuda.stream(side):
+        for name, t in (("k", k), ("v", v), ("q", q)):
+            bufs[name].copy_(t, non_blocking=True)
+    kp = qsa_pool_block_keys(bufs["ki"], bufs["kp"], rope_theta=rope_theta)
+    qr = qsa_rope_index_queries(bufs["qi"], rope_theta=rope_theta, q_pos0=q_pos0) if rope_theta > 0 else bufs["qi"]
+    idx = qsa_select_topk(topk, qi=qr, kp=kp, head_w=head_w, q_pos0=q_pos0, mode=mode, workspace=workspace,
+                          idx=bufs.get("idx"))
+    bufs["idx"] = idx
+    main.wait_stream(side)
+    half = Tq // 2 if (Tq >= 2 and B == 1) else Tq
+    spans = [(0, half), (half, Tq)] if half < Tq else [(0, Tq)]
+    for lo, hi in spans:
+        qpart = bufs["q"][:, lo:hi]
+        opart = bufs["out"][:, lo:hi]
+        if B == 1 or (lo == 0 and hi == Tq):
+            qsa_sparse_attn_prefill(qpart, bufs["k"], bufs["v"], idx[:, lo:hi], q_pos0=q_pos0 + lo, scale=scale,
+                                    out=opart, lse=bufs["lse"][:, lo:hi])
+        side.wait_stream(main)
+        with torch.cuda.stream(side):
+            out[:, lo:hi].copy_(opart, non_blocking=True)
+    main.wait_stream(side)
+    return dict(out=out, lse=bufs["lse"], idx=idx)
