@@ -36,6 +36,10 @@ from hybrid_sparse_attention_qsa_b200 import inputs as I  # noqa: E402
 METRIC = "QSA prefill tokens/s @128K and decode tokens/s @256K ctx; % of roofline"
 PREFILL = "prefill_128k"
 DECODE = "decode_256k"
+# DRAM bytes read + written by one sparse_attn_kernel<2> launch, from the ncu capture summarised in
+# profiles/sparse_attn_prefill_128k.md (dram__bytes_read.sum + dram__bytes_write.sum); set to None
+# whenever the kernel changes until it is captured again
+ATTN_DRAM_TRAFFIC = {"prefill_128k": 1.521689e9 + 0.521716e9}
 
 
 # ------------------------------------------------------------------------------------------- helpers
@@ -292,6 +296,32 @@ def run_qsa(args):
     except torch.OutOfMemoryError:
         pass
 
+    # dense causal attention on the same q/k/v (library SDPA, GQA), the comparison the vendor's
+    # kernel-level speedups are stated against; QSA's step (selection included) over it
+    dense = None
+    if not args.no_dense:
+        try:
+            g = w.Hq // w.Hkv   # K/V expanded to every query head so the flash backend takes the call
+            qd = x["q"].transpose(1, 2)
+            kd = x["k"].repeat_interleave(g, dim=2).transpose(1, 2)
+            vd = x["v"].repeat_interleave(g, dim=2).transpose(1, 2)
+            sdpa = torch.nn.functional.scaled_dot_product_attention
+            with torch.cuda.stream(stream):
+                sdpa(qd, kd, vd, is_causal=True)
+                f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                f0.record(stream)
+                for _ in range(2):
+                    sdpa(qd, kd, vd, is_causal=True)
+                f1.record(stream)
+            torch.cuda.synchronize()
+            dense_ms = f0.elapsed_time(f1) / 2
+            del qd, kd, vd
+            dense = {"impl": "torch scaled_dot_product_attention (causal, bf16, K/V expanded to Hq)", "ms": dense_ms,
+                     "qsa_step_ms": ms_step, "qsa_attention_ms": ms_attn,
+                     "speedup_step": dense_ms / ms_step, "speedup_attention_only": dense_ms / ms_attn}
+        except Exception as exc:   # library without a kernel for this shape
+            dense = {"unavailable": f"{type(exc).__name__}: {exc}"[:200]}
+
     # end to end through the public API from pinned host buffers
     e2e = None
     if not args.no_e2e:
@@ -395,7 +425,7 @@ def run_qsa(args):
                        "l2": "inputs larger than L2, no flush", "parallelism": f"independent replicas x{world}"},
             "roofline": {"bound": "hbm", "kernel": "sparse_attn_kernel<2>", "achieved": attn_gbs,
                          "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": attn_gbs / pk["hbm_gbs"],
-                         "traffic": None, "peak_source": pk["source"],
+                         "traffic": ATTN_DRAM_TRAFFIC.get(args.workload), "peak_source": pk["source"],
                          "basis": "gathered K/V bytes of every selected token + q read + o write",
                          "bytes_per_launch": work["attn_bytes"], "ms_per_launch": ms_attn},
             "step_breakdown_ms": {"pool": None, "score_topk": ms_select, "attention": ms_attn},
@@ -407,6 +437,7 @@ def run_qsa(args):
             "clocks": clocks,
             "e2e": e2e,
             "decode": decode,
+            "dense_compare": dense,
         }
         if not args.no_cpu_baseline and world == 1:
             dt, rows, cores = oracle_sample(I.WORKLOADS[args.workload], args.ref_rows)
@@ -432,6 +463,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-indexer", action="store_true", help="skip the stand-alone indexer timing (17 GB of scores)")
+    ap.add_argument("--no-dense", action="store_true", help="skip timing dense causal attention on the same inputs")
     ap.add_argument("--workload", default=PREFILL, choices=[n for n, w in I.WORKLOADS.items() if w.kind == "prefill"],
                     help="prefill workload of the headline leg (default: the 128K configuration)")
     args = ap.parse_args()
