@@ -57,6 +57,38 @@ bool ok_ptr(const void* p) { return p != nullptr && aligned16(p); }
 cudaStream_t S(void* s) { return static_cast<cudaStream_t>(s); }
 qsa_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? QSA_OK : QSA_ERR_CUDA; }
 bool hi_supported(int Hi) { return Hi == 1 || Hi == 2 || Hi == 4 || Hi == 8; }
+
+// ---- filtered selection (prefill without materialised scores)
+std::atomic<int> g_select_path{0};    // 0 automatic, 1 materialised scores, 2 filtered
+std::atomic<int> g_sample_rank{0};    // 0: the default rank of the threshold among the samples
+constexpr int kSampleShift = 4;       // every 16th pooled block is sampled ...
+constexpr int kSampleOff = 8;         // ... starting at block 8
+constexpr int kFallbackCtas = 128;    // CTAs (and scratch rows) of the exact redo of failed rows
+constexpr long long kFusedTarget = 4ll << 30;   // workspace the size query plans the filtered path in
+constexpr int kFusedMinRows = 16384;  // automatic choice: rows per sequence from which it pays
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+struct FusedPlan {
+  int rank, cap, ns, ld_s;
+  long long per_row, fixed;
+};
+// rank r of the threshold among the row's samples (about 16 r scores expected above it, at least
+// 2.5 k so a short list is a many-sigma event) and the list capacity 32 r.
+FusedPlan fused_plan(int NBk, int k) {
+  FusedPlan p;
+  p.rank = std::max(64, (5 * k + 31) / 32);
+  p.cap = 32 * p.rank;
+  p.ns = NBk > kSampleOff ? ((NBk - kSampleOff - 1) >> kSampleShift) + 1 : 0;
+  p.ld_s = (std::max(p.ns, 1) + 3) & ~3;
+  p.per_row = static_cast<long long>(p.ld_s) * 4 + 12 + static_cast<long long>(p.cap) * 8;
+  p.fixed = 6 * 256 + 4 + static_cast<long long>(kFallbackCtas) * std::max(NBk, 1) * 4;
+  return p;
+}
+long long fused_rows_fit(const FusedPlan& p, size_t ws_bytes) {
+  const long long avail = static_cast<long long>(ws_bytes) - p.fixed;
+  return avail > 0 ? avail / p.per_row : 0;
+}
 }  // namespace
 
 const DeviceInfo* device_info() {
@@ -95,6 +127,13 @@ const char* qsa_status_string(qsa_status_t status) {
 }
 
 int qsa_abi_version(void) { return QSA_ABI_VERSION; }
+
+qsa_status_t qsa_set_select_options(int path, int sample_rank) {
+  if (path < 0 || path > 2 || sample_rank < 0) return QSA_ERR_INVALID_ARGUMENT;
+  g_select_path.store(path);
+  g_sample_rank.store(sample_rank);
+  return QSA_OK;
+}
 
 void qsa_set_wait_timeout_ns(uint64_t ns) { g_wait_ns.store(ns ? ns : kDefaultWaitNs); }
 
@@ -189,6 +228,56 @@ qsa_status_t qsa_select_topk(const float* scores, int64_t ld_scores, const void*
     cudaError_t e = launch_score_decode(di, qi, kp, head_w, seqlens, B, NBk, Hi, Di, blk, mode, ws, NBk, s);
     if (e == cudaSuccess) e = launch_topk(di, ws, NBk, NBk, seqlens, 1, NBk, blk, 0, 0, B, 0, 1, k, idx, s);
     return cuda_status(e);
+  }
+  // Filtered selection: sampled scores -> thresholds -> score + filter -> select over the lists
+  // -> exact redo of failed rows, per chunk of rows of one sequence.
+  {
+    const FusedPlan fp = fused_plan(NBk, k);
+    const long long fit = fused_rows_fit(fp, ws_bytes);
+    const int path = g_select_path.load();
+    const bool able = Hi == 4 || Hi == 8;
+    if (path == 2 && !able) return QSA_ERR_UNSUPPORTED;
+    if (path == 2 && fit < 1) return QSA_ERR_WORKSPACE_TOO_SMALL;
+    if (path == 2 || (path == 0 && able && Tq >= kFusedMinRows && fit >= std::min(Tq, 4096))) {
+      long long R = std::min<long long>(Tq, fit);
+      if (R < Tq && R >= 64) R &= ~63ll;
+      uint8_t* w8 = static_cast<uint8_t*>(workspace);
+      float* samp = reinterpret_cast<float*>(w8);
+      size_t off = align256(static_cast<size_t>(R) * fp.ld_s * 4);
+      float* tau = reinterpret_cast<float*>(w8 + off);
+      off += align256(static_cast<size_t>(R) * 4);
+      int* cnt = reinterpret_cast<int*>(w8 + off);
+      off += align256(static_cast<size_t>(R) * 4);
+      int* fail = reinterpret_cast<int*>(w8 + off);
+      off += align256(static_cast<size_t>(R + 1) * 4);
+      uint2* cand = reinterpret_cast<uint2*>(w8 + off);
+      off += align256(static_cast<size_t>(R) * fp.cap * 8);
+      float* scratch = reinterpret_cast<float*>(w8 + off);
+      const int rank = g_sample_rank.load() > 0 ? g_sample_rank.load() : fp.rank;
+      const size_t qi_b = static_cast<size_t>(Tq) * Hi * Di * 2, kp_b = static_cast<size_t>(NBk) * Di * 2;
+      cudaError_t e = cudaSuccess;
+      for (int b = 0; e == cudaSuccess && b < B; ++b) {
+        const uint8_t* qib = static_cast<const uint8_t*>(qi) + b * qi_b;
+        const uint8_t* kpb = static_cast<const uint8_t*>(kp) + b * kp_b;
+        for (int r0 = 0; e == cudaSuccess && r0 < Tq; r0 += static_cast<int>(R)) {
+          const int rows = static_cast<int>(std::min<long long>(R, Tq - r0));
+          e = launch_score_prefill(di, qib, kpb, head_w, 1, Tq, NBk, Hi, Di, blk, q_pos0, mode, 0, 1, r0, rows, samp,
+                                   fp.ld_s, 0, s, kSampleShift, kSampleOff);
+          if (e == cudaSuccess)
+            e = launch_select_tau(di, samp, fp.ld_s, NBk, q_pos0, r0, rows, fp.cap, rank, kSampleShift, kSampleOff,
+                                  tau, fail, s);
+          if (e == cudaSuccess)
+            e = launch_score_filter(di, qib, kpb, head_w, Tq, NBk, Hi, q_pos0, mode, 0, 1, r0, rows, tau, cand, cnt,
+                                    fp.cap, s);
+          if (e == cudaSuccess)
+            e = launch_select_candidates(di, cand, cnt, fp.cap, Tq, NBk, q_pos0, b, r0, rows, k, idx, fail, s);
+          if (e == cudaSuccess)
+            e = launch_topk_fallback(di, qi, kp, head_w, Hi, mode, Tq, NBk, q_pos0, b, fail, scratch, kFallbackCtas, k,
+                                     idx, s);
+        }
+      }
+      return cuda_status(e);
+    }
   }
   const long long chunks = static_cast<long long>(B) * ((Tq + R - 1) / R);
   SideStream* side = chunks > 1 && R >= 2 ? side_stream(di->device) : nullptr;
@@ -294,7 +383,13 @@ size_t qsa_workspace_size(qsa_op_t op, int B, int Tq, int NBk, int k, int Hq, in
     if (Tq <= 1) return static_cast<size_t>(row * std::max(B, 1));
     const long long cap = 512ll << 20;   // chunk of score rows kept at or below 512 MiB
     const long long rows = std::max(1ll, std::min<long long>(Tq, cap / row));
-    return static_cast<size_t>(rows * row);
+    long long bytes = rows * row;
+    if (k >= 1) {   // room for the filtered path: all rows of a sequence, or chunks within ~4 GiB
+      const FusedPlan fp = fused_plan(NBk, k);
+      const long long frows = std::max(64ll, std::min<long long>(Tq, (kFusedTarget - fp.fixed) / fp.per_row));
+      bytes = std::max(bytes, fp.fixed + frows * fp.per_row);
+    }
+    return static_cast<size_t>(bytes);
   }
   if (op == QSA_OP_SPARSE_ATTN_DECODE) {
     if (B < 1 || Hq < 1 || D < 1) return 0;

@@ -58,6 +58,32 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
       : "memory");
   return ok != 0;
 }
+// As mbar_try_wait, but a thread whose phase is still open may be suspended for up to `hint_ns`
+// (it resumes as soon as the phase completes), so waiting warps take fewer issue slots.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, unsigned parity, unsigned hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait with suspension between polls (the limit is checked every 16 polls).
+__device__ __forceinline__ bool mbar_wait_suspend(uint64_t* bar, unsigned parity, const KernelCtl& ctl,
+                                                  unsigned hint_ns = 1000) {
+  if (mbar_try_wait_suspend(bar, parity, hint_ns)) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  for (unsigned it = 1;; ++it) {
+    if (mbar_try_wait_suspend(bar, parity, hint_ns)) return true;
+    if ((it & 15u) == 0u && globaltimer_ns() - t0 > ctl.wait_ns) {
+      record_status(ctl, kStTimeout);
+      return false;
+    }
+  }
+}
 // Waits for the phase with the given parity to complete.  Gives up after ctl.wait_ns, records
 // kStTimeout and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity, const KernelCtl& ctl) {

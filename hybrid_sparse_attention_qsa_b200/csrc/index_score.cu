@@ -20,6 +20,7 @@
 // Decode: one query per sequence, so the contraction degenerates to a GEMV over the pooled-key
 //   cache; it is HBM-bound: TMA-fed mma.sync tiles with the query heads in the N dimension.
 #include <mutex>
+#include <type_traits>
 
 #include "launch.h"
 
@@ -41,8 +42,72 @@ struct ScoreArgs {
   float* scores;
   long long ld, batch_stride, q_pos0;
   int NBk, blk, mode, b0, row0, rows;
+  // Column c of the kp map is pooled block (c << kshift) + koff: 0/0 for the scores themselves, a
+  // stride for the sampled scores that set the selection thresholds.
+  int kshift, koff;
   KernelCtl ctl;
 };
+
+// Columns of a map with stride 1 << kshift and offset koff that lie below nb blocks.
+__host__ __device__ __forceinline__ int visible_cols(int nb, int kshift, int koff) {
+  return nb > koff ? ((nb - koff - 1) >> kshift) + 1 : 0;
+}
+
+// TMA producer (one thread): the qi tile once, then kp tiles t_begin .. t_begin + nt - 1 through the
+// ring.  Returns only when no copy it issued is still in flight.
+__device__ __forceinline__ void produce_kp_tiles(const CUtensorMap* qi_map, const CUtensorMap* kp_map, uint8_t* qi_s,
+                                                 uint8_t* kp_s, uint64_t* qi_full, uint64_t* kp_full,
+                                                 uint64_t* kp_empty, int qi_row, int b, int t_begin, int nt,
+                                                 const KernelCtl& ctl) {
+  prefetch_tensormap(qi_map);
+  prefetch_tensormap(kp_map);
+  mbar_arrive_expect_tx(qi_full, kQiBytes);
+  tma_load_3d(qi_s, qi_map, qi_full, 0, qi_row, b);
+  int issued = 0;
+  for (int i = 0; i < nt; ++i) {
+    const int s = i % kStages;
+    const unsigned ph = (i / kStages) & 1u;
+    if (!mbar_wait_suspend(&kp_empty[s], ph ^ 1u, ctl)) break;
+    mbar_arrive_expect_tx(&kp_full[s], kKpBytes);
+    tma_load_3d(kp_s + s * kKpBytes, kp_map, &kp_full[s], 0, (t_begin + i) * kM, b);
+    issued = i + 1;
+  }
+  // Never leave with a copy in flight: wait for the last fill of every stage and the qi tile.
+  mbar_wait_suspend(qi_full, 0, ctl);
+  for (int s = 0; s < kStages && s < issued; ++s) {
+    const int last = s + ((issued - 1 - s) / kStages) * kStages;
+    mbar_wait_suspend(&kp_full[s], (last / kStages) & 1u, ctl);
+  }
+}
+
+// MMA issuer (one thread): tile i accumulates D = kp_tile . qi_tile^T into TMEM columns
+// (i & 1) * kN .. + kN, then frees its kp stage and signals the epilogue.
+__device__ __forceinline__ void issue_tile_mmas(uint32_t tmem, uint8_t* qi_s, uint8_t* kp_s, uint64_t* qi_full,
+                                                uint64_t* kp_full, uint64_t* kp_empty, uint64_t* tm_full,
+                                                uint64_t* tm_empty, uint64_t* mma_done, int nt, const KernelCtl& ctl) {
+  const uint32_t idesc = umma_idesc_bf16_f32(kM, kN);
+  const uint64_t bdesc = sw128_kmajor_desc(smem_u32(qi_s));
+  bool ok = mbar_wait_suspend(qi_full, 0, ctl);
+  for (int i = 0; ok && i < nt; ++i) {
+    const int s = i % kStages;
+    const unsigned ph = (i / kStages) & 1u;
+    const int acc = i & 1;
+    const unsigned aph = (i >> 1) & 1u;
+    if (!mbar_wait_suspend(&kp_full[s], ph, ctl)) break;
+    if (!mbar_wait_suspend(&tm_empty[acc], aph ^ 1u, ctl)) break;
+    tc_fence_after();
+    const uint64_t adesc = sw128_kmajor_desc(smem_u32(kp_s + s * kKpBytes));
+#pragma unroll
+    for (int kk = 0; kk < kDi / 16; ++kk) {
+      // +32 bytes of K per step: +2 in the (>> 4) start-address field
+      umma_bf16(tmem + acc * kN, adesc + 2 * kk, bdesc + 2 * kk, idesc, kk > 0 ? 1u : 0u);
+    }
+    umma_commit(&kp_empty[s]);
+    umma_commit(&tm_full[acc]);
+  }
+  umma_commit(mma_done);
+  mbar_wait_suspend(mma_done, 0, ctl);
+}
 
 template <int HI, int MODE>
 __global__ void __launch_bounds__(kScoreThreads, 1)
@@ -68,7 +133,8 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
   const int r_first = a.row0 + static_cast<int>(blockIdx.x) * QPT;
   const int r_last = min(r_first + QPT, a.row0 + a.rows) - 1;
   const long long pos_last = a.q_pos0 + r_last;
-  const int nb_last = static_cast<int>(min(static_cast<long long>(a.NBk), pos_last / a.blk));
+  const int nb_last = visible_cols(static_cast<int>(min(static_cast<long long>(a.NBk), pos_last / a.blk)), a.kshift,
+                                   a.koff);
   const int ntiles = (nb_last + kM - 1) / kM;
   const int t_begin = static_cast<int>(blockIdx.y) * kTilesPerCta;
   const int t_end = min(ntiles, t_begin + kTilesPerCta);
@@ -98,53 +164,12 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    if (lane == 0) {
-      prefetch_tensormap(&qi_map);
-      prefetch_tensormap(&kp_map);
-      mbar_arrive_expect_tx(qi_full, kQiBytes);
-      tma_load_3d(qi_s, &qi_map, qi_full, 0, r_first * HI, b);
-      int issued = 0;
-      for (int i = 0; i < nt; ++i) {
-        const int s = i % kStages;
-        const unsigned ph = (i / kStages) & 1u;
-        if (!mbar_wait(&kp_empty[s], ph ^ 1u, a.ctl)) break;
-        mbar_arrive_expect_tx(&kp_full[s], kKpBytes);
-        tma_load_3d(kp_s + s * kKpBytes, &kp_map, &kp_full[s], 0, (t_begin + i) * kM, b);
-        issued = i + 1;
-      }
-      // Never leave with a copy in flight: wait for the last fill of every stage and the qi tile.
-      mbar_wait(qi_full, 0, a.ctl);
-      for (int s = 0; s < kStages && s < issued; ++s) {
-        const int last = s + ((issued - 1 - s) / kStages) * kStages;
-        mbar_wait(&kp_full[s], (last / kStages) & 1u, a.ctl);
-      }
-    }
+    if (lane == 0)
+      produce_kp_tiles(&qi_map, &kp_map, qi_s, kp_s, qi_full, kp_full, kp_empty, r_first * HI, b, t_begin, nt, a.ctl);
     __syncwarp();
   } else if (warp == 1) {
-    if (lane == 0) {
-      const uint32_t idesc = umma_idesc_bf16_f32(kM, kN);
-      const uint64_t bdesc = sw128_kmajor_desc(smem_u32(qi_s));
-      bool ok = mbar_wait(qi_full, 0, a.ctl);
-      for (int i = 0; ok && i < nt; ++i) {
-        const int s = i % kStages;
-        const unsigned ph = (i / kStages) & 1u;
-        const int acc = i & 1;
-        const unsigned aph = (i >> 1) & 1u;
-        if (!mbar_wait(&kp_full[s], ph, a.ctl)) break;
-        if (!mbar_wait(&tm_empty[acc], aph ^ 1u, a.ctl)) break;
-        tc_fence_after();
-        const uint64_t adesc = sw128_kmajor_desc(smem_u32(kp_s + s * kKpBytes));
-#pragma unroll
-        for (int kk = 0; kk < kDi / 16; ++kk) {
-          // +32 bytes of K per step: +2 in the (>> 4) start-address field
-          umma_bf16(tmem + acc * kN, adesc + 2 * kk, bdesc + 2 * kk, idesc, kk > 0 ? 1u : 0u);
-        }
-        umma_commit(&kp_empty[s]);
-        umma_commit(&tm_full[acc]);
-      }
-      umma_commit(mma_done);
-      mbar_wait(mma_done, 0, a.ctl);
-    }
+    if (lane == 0)
+      issue_tile_mmas(tmem, qi_s, kp_s, qi_full, kp_full, kp_empty, tm_full, tm_empty, mma_done, nt, a.ctl);
     __syncwarp();
   } else {
     const int ew = warp - 2;                 // 0..7
@@ -159,12 +184,13 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     const long long pos_first = a.q_pos0 + r_first;
     const int tl_last = r_last - r_first;
     const int nbk = a.NBk;
+    const int ksh = a.kshift, kof = a.koff;
     float* srow = a.scores + static_cast<long long>(bz) * a.batch_stride + static_cast<long long>(r_first - a.row0) * a.ld;
     const long long ld = a.ld;
     for (int i = 0; i < nt; ++i) {
       const int acc = i & 1;
       const unsigned aph = (i >> 1) & 1u;
-      if (!mbar_wait(&tm_full[acc], aph, a.ctl)) break;
+      if (!mbar_wait_suspend(&tm_full[acc], aph, a.ctl)) break;
       tc_fence_after();
       const int kb = (t_begin + i) * kM + quad * 32 + lane;   // pooled key owned by this thread
       float* col = srow + kb;
@@ -189,8 +215,9 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         // Queries q0 .. q0 + 32/HI - 1 of the tile: when all of them exist and see every pooled key
         // of this warp, the stores need no mask (all tiles below the diagonal band).
         float* dst = col + static_cast<long long>(q0) * ld;
-        const bool full = q0 + 32 / HI - 1 <= tl_last &&
-                          (t_begin + i) * kM + quad * 32 + 31 < min(nbk, static_cast<int>((pos_first + q0) >> 2));
+        const bool full =
+            q0 + 32 / HI - 1 <= tl_last &&
+            (t_begin + i) * kM + quad * 32 + 31 < visible_cols(min(nbk, static_cast<int>((pos_first + q0) >> 2)), ksh, kof);
         if (full) {
 #pragma unroll
           for (int qq = 0; qq < 32 / HI; ++qq) {
@@ -201,7 +228,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
 #pragma unroll
           for (int qq = 0; qq < 32 / HI; ++qq) {
             const int tl = q0 + qq;
-            const int nbq = min(nbk, static_cast<int>((pos_first + tl) >> 2));
+            const int nbq = visible_cols(min(nbk, static_cast<int>((pos_first + tl) >> 2)), ksh, kof);
             if (tl <= tl_last && kb < nbq) *dst = sc[qq];
             dst += ld;
           }
@@ -211,6 +238,216 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&tm_empty[acc]);
     }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------------------ score + filter
+// Selection without materialised scores.  The same tile pipeline as score_prefill_kernel, one CTA
+// per strip of kN/HI queries over ALL their visible pooled keys (strips taken longest first).  The
+// epilogue compares each score with its query's threshold tau (set beforehand from sampled scores,
+// -inf for rows short enough to keep everything) and appends the survivors (order-preserving key,
+// block index) to the query's candidate list IN INDEX ORDER: the four warps that read the four TMEM
+// lane quadrants of a column half exchange their per-query counts of a tile through shared memory,
+// so every position is known without atomics.  Only the first `cap` entries of a list are stored;
+// the full count is written, so the selection can tell an overflowing list.
+constexpr int kFiltEpiWarps = 16;                 // four per TMEM lane quadrant
+constexpr int kFiltGroups = kFiltEpiWarps / 4;      // column groups of kN / kFiltGroups columns
+constexpr int kFiltThreads = 64 + kFiltEpiWarps * 32;
+constexpr int kFiltStash = 17;   // floats per lane row of the score stash (queries of a warp + 1)
+constexpr int kFiltSmem = 1024 + kQiBytes + kStages * kKpBytes + 256 + kFiltEpiWarps * 32 * kFiltStash * 4 +
+                          kFiltEpiWarps * 32 * 4 * 2 + 2 * kFiltGroups * 4 * 32 * 4;
+
+struct FilterArgs {
+  const float* head_w;
+  const float* tau;     // [rows] threshold of row row0 + i
+  uint2* cand;          // [rows][cap] (key, block index)
+  int* cnt;             // [rows] number of scores >= tau (may exceed cap)
+  long long q_pos0;
+  int NBk, b0, row0, rows, cap;
+  KernelCtl ctl;
+};
+
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+template <int HI, int MODE>
+__global__ void __launch_bounds__(kFiltThreads, 1)
+    score_filter_kernel(const __grid_constant__ CUtensorMap qi_map, const __grid_constant__ CUtensorMap kp_map,
+                        FilterArgs a) {
+  constexpr int QPT = kN / HI;                 // queries per strip
+  constexpr int CW = kN / kFiltGroups;         // TMEM columns per epilogue warp
+  constexpr int QW = CW / HI;                  // queries per epilogue warp
+  constexpr int QC = 32 / HI;                  // queries per 32-column TMEM load
+  static_assert(QW < kFiltStash && QW <= 32, "stash row and one bit per query of a warp");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* qi_s = smem;
+  uint8_t* kp_s = smem + kQiBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(kp_s + kStages * kKpBytes);
+  uint64_t* qi_full = bars;
+  uint64_t* kp_full = bars + 1;
+  uint64_t* kp_empty = kp_full + kStages;
+  uint64_t* tm_full = kp_empty + kStages;
+  uint64_t* tm_empty = tm_full + 2;
+  uint64_t* mma_done = tm_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  float* stash = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 256);   // [warp][lane][kFiltStash]
+  uint32_t* xmask = reinterpret_cast<uint32_t*>(stash + kFiltEpiWarps * 32 * kFiltStash);   // [warp][32]
+  uint32_t* xoff = xmask + kFiltEpiWarps * 32;                                                // [warp][32]
+  uint32_t* xcnt = xoff + kFiltEpiWarps * 32;                         // [2 tiles][groups][4 quadrants][32]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bz = blockIdx.z;
+  const int b = a.b0 + bz;
+  const int strip = static_cast<int>(gridDim.x - 1 - blockIdx.x);   // longest strips first
+  const int r_first = a.row0 + strip * QPT;
+  const int r_last = min(r_first + QPT, a.row0 + a.rows) - 1;
+  const long long pos_first = a.q_pos0 + r_first;
+  const int nb_last = static_cast<int>(min(static_cast<long long>(a.NBk), (a.q_pos0 + r_last) >> 2));
+  const int nt = (nb_last + kM - 1) / kM;
+  const int tl_last = r_last - r_first;
+  const long long list0 = static_cast<long long>(bz) * a.rows + (r_first - a.row0);   // list of the strip's row 0
+  if (nt == 0) {   // uniform over the CTA: no visible block, every count is 0
+    if (threadIdx.x <= tl_last) a.cnt[list0 + threadIdx.x] = 0;
+    return;
+  }
+
+  if (threadIdx.x == 0) {
+    mbar_init(qi_full, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&kp_full[s], 1);
+      mbar_init(&kp_empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tm_full[i], 1);
+      mbar_init(&tm_empty[i], kFiltEpiWarps);
+    }
+    mbar_init(mma_done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0)
+      produce_kp_tiles(&qi_map, &kp_map, qi_s, kp_s, qi_full, kp_full, kp_empty, r_first * HI, b, 0, nt, a.ctl);
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0)
+      issue_tile_mmas(tmem, qi_s, kp_s, qi_full, kp_full, kp_empty, tm_full, tm_empty, mma_done, nt, a.ctl);
+    __syncwarp();
+  } else {
+    const int ew = warp - 2;          // 0 .. kFiltEpiWarps - 1
+    const int quad = warp & 3;        // TMEM lane quadrant this warp may read
+    const int grp = ew >> 2;          // column group: queries grp*QW .. grp*QW + QW - 1
+    const int qbase = grp * QW;
+    const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t lt = [] {
+      uint32_t m;
+      asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+      return m;
+    }();
+    float w[HI];
+#pragma unroll
+    for (int h = 0; h < HI; ++h) w[h] = a.head_w ? a.head_w[h] : 1.0f;
+    // Thresholds of this warp's queries; a query past the strip's last row never passes.
+    float tq[QW];
+#pragma unroll
+    for (int q = 0; q < QW; ++q) tq[q] = qbase + q <= tl_last ? a.tau[list0 + qbase + q] : INFINITY;
+    // Slices below the first query's visible blocks need no visibility test when every query exists.
+    const int nb_min_full =
+        qbase + QW - 1 <= tl_last ? static_cast<int>(min(static_cast<long long>(a.NBk), (pos_first + qbase) >> 2)) : 0;
+    float* my_stash = stash + (ew * 32 + lane) * kFiltStash;
+    uint32_t* my_mask = xmask + ew * 32;
+    uint32_t* my_off = xoff + ew * 32;
+    uint2* list_q0 = a.cand + (list0 + qbase) * a.cap;   // list of the warp's first query
+    uint32_t run = 0;   // lane q: entries of query qbase + q before the current tile
+    bool dead = false;  // a wait timed out: keep meeting the barriers, touch nothing
+    for (int i = 0; i < nt; ++i) {
+      const int acc = i & 1;
+      const unsigned aph = (i >> 1) & 1u;
+      if (!dead && !mbar_wait_suspend(&tm_full[acc], aph, a.ctl)) dead = true;
+      tc_fence_after();
+      const int kb = i * kM + quad * 32 + lane;   // pooled block owned by this thread
+      uint32_t bits = 0;
+      // One pass over the warp's scores of the tile; FULL: every query of the warp exists and sees
+      // every block of its slice (tiles below the diagonal band), so no visibility test.
+      auto filter_tile = [&](auto full_c) {
+        constexpr bool FULL = decltype(full_c)::value;
+#pragma unroll
+        for (int c = 0; c < CW / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld_32x32(tmem + lane_addr + acc * kN + grp * CW + c * 32, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int qq = 0; qq < QC; ++qq) {
+            const int q = c * QC + qq;
+            float sc = 0.0f;
+#pragma unroll
+            for (int h = 0; h < HI; ++h) {
+              float x = __uint_as_float(r[qq * HI + h]);
+              if (MODE == 0) x = fmaxf(x, 0.0f);
+              sc = fmaf(w[h], x, sc);
+            }
+            bool pass = sc >= tq[q];
+            if (!FULL)
+              pass = pass && qbase + q <= tl_last &&
+                     kb < static_cast<int>(min(static_cast<long long>(a.NBk), (pos_first + qbase + q) >> 2));
+            my_stash[q] = sc;
+            const uint32_t m = __ballot_sync(0xffffffffu, pass);
+            my_mask[q] = m;   // the same value from every lane
+            if (pass) bits |= 1u << q;
+          }
+        }
+      };
+      if (!dead) {
+        if (i * kM + quad * 32 + 31 < nb_min_full)
+          filter_tile(std::integral_constant<bool, true>());
+        else
+          filter_tile(std::integral_constant<bool, false>());
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tm_empty[acc]);
+      // counts of this tile per (quadrant, query) -> each lane's position in its query's list
+      uint32_t* xc = xcnt + ((i & 1) * kFiltGroups + grp) * 4 * 32;
+      if (lane < QW) xc[quad * 32 + lane] = dead ? 0u : static_cast<uint32_t>(__popc(my_mask[lane]));
+      named_bar_sync(1 + grp, 128);
+      if (lane < QW) {
+        uint32_t pre = 0, tot = 0;
+#pragma unroll
+        for (int o = 0; o < 4; ++o) {
+          const uint32_t c = xc[o * 32 + lane];
+          pre += o < quad ? c : 0u;
+          tot += c;
+        }
+        my_off[lane] = run + pre;
+        run += tot;
+      }
+      __syncwarp();
+      while (bits) {
+        const int q = __ffs(bits) - 1;
+        bits &= bits - 1;
+        const uint32_t p = my_off[q] + static_cast<uint32_t>(__popc(my_mask[q] & lt));
+        if (p < static_cast<uint32_t>(a.cap))
+          list_q0[static_cast<long long>(q) * a.cap + p] = make_uint2(score_key(my_stash[q] + 0.0f), static_cast<uint32_t>(kb));
+      }
+      __syncwarp();
+    }
+    if (quad == 0 && lane < QW && qbase + lane <= tl_last) a.cnt[list0 + qbase + lane] = static_cast<int>(run);
   }
   tc_fence_before();
   __syncthreads();
@@ -357,12 +594,14 @@ EncodeTiledFn encode_tiled() {
   return fn;
 }
 
-// 3-D bf16 map over [d2][d1][64] with a 128-byte-swizzled box of {64, box_rows, 1}.
-bool make_map(CUtensorMap* m, const void* base, unsigned long long d1, unsigned long long d2, unsigned box_rows) {
+// 3-D bf16 map over [d2][d1][64] rows of 128 bytes (row pitch and batch pitch in bytes) with a
+// 128-byte-swizzled box of {64, box_rows, 1}.
+bool make_map_pitched(CUtensorMap* m, const void* base, unsigned long long d1, unsigned long long row_pitch,
+                      unsigned long long d2, unsigned long long batch_pitch, unsigned box_rows) {
   EncodeTiledFn fn = encode_tiled();
   if (!fn) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(kDi), d1, d2};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(kDi) * 2, d1 * kDi * 2};
+  cuuint64_t strides[2] = {row_pitch, batch_pitch};
   cuuint32_t box[3] = {static_cast<cuuint32_t>(kDi), box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
@@ -370,11 +609,15 @@ bool make_map(CUtensorMap* m, const void* base, unsigned long long d1, unsigned 
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
+bool make_map(CUtensorMap* m, const void* base, unsigned long long d1, unsigned long long d2, unsigned box_rows) {
+  return make_map_pitched(m, base, d1, kDi * 2ull, d2, d1 * kDi * 2ull, box_rows);
+}
 
 template <int HI>
 cudaError_t launch_prefill_hi(const void* qi, const void* kp, const float* head_w, int Tq, int NBk, int blk,
                               long long q_pos0, int mode, int b0, int nb, int row0, int rows, float* scores,
-                              long long ld, long long batch_stride, const KernelCtl& ctl, cudaStream_t s) {
+                              long long ld, long long batch_stride, int kshift, int koff, const KernelCtl& ctl,
+                              cudaStream_t s) {
   static std::once_flag attr_once[64];
   int dev = 0;
   cudaGetDevice(&dev);
@@ -383,22 +626,57 @@ cudaError_t launch_prefill_hi(const void* qi, const void* kp, const float* head_
     cudaFuncSetAttribute(score_prefill_kernel<HI, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kScoreSmem);
   });
   CUtensorMap qmap, kmap;
-  // Maps span all batches so the batch index is a TMA coordinate.
+  // Maps span all batches so the batch index is a TMA coordinate.  With kshift > 0 the kp map
+  // walks every (1 << kshift)-th pooled key starting at koff.
+  const int Btot = b0 + nb;
+  const int ncols = visible_cols(NBk, kshift, koff);
+  if (ncols == 0) return cudaSuccess;
+  const uint8_t* kbase = static_cast<const uint8_t*>(kp) + static_cast<size_t>(koff) * kDi * 2;
+  if (!make_map(&qmap, qi, static_cast<unsigned long long>(Tq) * HI, static_cast<unsigned long long>(Btot), kN) ||
+      !make_map_pitched(&kmap, kbase, static_cast<unsigned long long>(ncols), (kDi * 2ull) << kshift,
+                        static_cast<unsigned long long>(Btot),
+                        Btot == 1 ? std::max<unsigned long long>(static_cast<unsigned long long>(NBk) * kDi * 2,
+                                                                 ((kDi * 2ull) << kshift) * ncols)
+                                  : static_cast<unsigned long long>(NBk) * kDi * 2,
+                        kM))
+    return cudaErrorInvalidValue;
+  constexpr int QPT = kN / HI;
+  const long long pos_last = q_pos0 + row0 + rows - 1;
+  const int nb_last = static_cast<int>(std::min<long long>(NBk, pos_last / blk));
+  const int ntiles = (visible_cols(nb_last, kshift, koff) + kM - 1) / kM;
+  if (ntiles == 0) return cudaSuccess;
+  dim3 grid((rows + QPT - 1) / QPT, (ntiles + kTilesPerCta - 1) / kTilesPerCta, nb);
+  ScoreArgs a{head_w, scores, ld, batch_stride, q_pos0, NBk, blk, mode, b0, row0, rows, kshift, koff, ctl};
+  if (mode == 0)
+    score_prefill_kernel<HI, 0><<<grid, kScoreThreads, kScoreSmem, s>>>(qmap, kmap, a);
+  else
+    score_prefill_kernel<HI, 1><<<grid, kScoreThreads, kScoreSmem, s>>>(qmap, kmap, a);
+  return cudaPeekAtLastError();
+}
+
+template <int HI>
+cudaError_t launch_filter_hi(const void* qi, const void* kp, const float* head_w, int Tq, int NBk, long long q_pos0,
+                             int mode, int b0, int nb, int row0, int rows, const float* tau, uint2* cand, int* cnt,
+                             int cap, const KernelCtl& ctl, cudaStream_t s) {
+  static std::once_flag attr_once[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::call_once(attr_once[dev & 63], [] {
+    cudaFuncSetAttribute(score_filter_kernel<HI, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, kFiltSmem);
+    cudaFuncSetAttribute(score_filter_kernel<HI, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kFiltSmem);
+  });
+  CUtensorMap qmap, kmap;
   const int Btot = b0 + nb;
   if (!make_map(&qmap, qi, static_cast<unsigned long long>(Tq) * HI, static_cast<unsigned long long>(Btot), kN) ||
       !make_map(&kmap, kp, static_cast<unsigned long long>(NBk), static_cast<unsigned long long>(Btot), kM))
     return cudaErrorInvalidValue;
   constexpr int QPT = kN / HI;
-  const long long pos_last = q_pos0 + row0 + rows - 1;
-  const int nb_last = static_cast<int>(std::min<long long>(NBk, pos_last / blk));
-  const int ntiles = (nb_last + kM - 1) / kM;
-  if (ntiles == 0) return cudaSuccess;
-  dim3 grid((rows + QPT - 1) / QPT, (ntiles + kTilesPerCta - 1) / kTilesPerCta, nb);
-  ScoreArgs a{head_w, scores, ld, batch_stride, q_pos0, NBk, blk, mode, b0, row0, rows, ctl};
+  dim3 grid((rows + QPT - 1) / QPT, 1, nb);
+  FilterArgs a{head_w, tau, cand, cnt, q_pos0, NBk, b0, row0, rows, cap, ctl};
   if (mode == 0)
-    score_prefill_kernel<HI, 0><<<grid, kScoreThreads, kScoreSmem, s>>>(qmap, kmap, a);
+    score_filter_kernel<HI, 0><<<grid, kFiltThreads, kFiltSmem, s>>>(qmap, kmap, a);
   else
-    score_prefill_kernel<HI, 1><<<grid, kScoreThreads, kScoreSmem, s>>>(qmap, kmap, a);
+    score_filter_kernel<HI, 1><<<grid, kFiltThreads, kFiltSmem, s>>>(qmap, kmap, a);
   return cudaPeekAtLastError();
 }
 
@@ -407,16 +685,28 @@ cudaError_t launch_prefill_hi(const void* qi, const void* kp, const float* head_
 cudaError_t launch_score_prefill(const DeviceInfo* di, const void* qi, const void* kp, const float* head_w, int B,
                                  int Tq, int NBk, int Hi, int Di, int blk, long long q_pos0, int mode, int b0, int nb,
                                  int row0, int rows, float* scores, long long ld, long long batch_stride,
-                                 cudaStream_t s) {
+                                 cudaStream_t s, int kshift, int koff) {
   (void)B;
   (void)Di;
   if (rows <= 0 || nb <= 0) return cudaSuccess;
   const KernelCtl ctl = kernel_ctl(di);
   switch (Hi) {
-    case 1: return launch_prefill_hi<1>(qi, kp, head_w, Tq, NBk, blk, q_pos0, mode, b0, nb, row0, rows, scores, ld, batch_stride, ctl, s);
-    case 2: return launch_prefill_hi<2>(qi, kp, head_w, Tq, NBk, blk, q_pos0, mode, b0, nb, row0, rows, scores, ld, batch_stride, ctl, s);
-    case 4: return launch_prefill_hi<4>(qi, kp, head_w, Tq, NBk, blk, q_pos0, mode, b0, nb, row0, rows, scores, ld, batch_stride, ctl, s);
-    case 8: return launch_prefill_hi<8>(qi, kp, head_w, Tq, NBk, blk, q_pos0, mode, b0, nb, row0, rows, scores, ld, batch_stride, ctl, s);
+    case 1: return launch_prefill_hi<1>(qi, kp, head_w, Tq, NBk, blk, q_pos0, mode, b0, nb, row0, rows, scores, ld, batch_stride, kshift, koff, ctl, s);
+    case 2: return launch_prefill_hi<2>(qi, kp, head_w, Tq, NBk, blk, q_pos0, mode, b0, nb, row0, rows, scores, ld, batch_stride, kshift, koff, ctl, s);
+    case 4: return launch_prefill_hi<4>(qi, kp, head_w, Tq, NBk, blk, q_pos0, mode, b0, nb, row0, rows, scores, ld, batch_stride, kshift, koff, ctl, s);
+    case 8: return launch_prefill_hi<8>(qi, kp, head_w, Tq, NBk, blk, q_pos0, mode, b0, nb, row0, rows, scores, ld, batch_stride, kshift, koff, ctl, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_score_filter(const DeviceInfo* di, const void* qi, const void* kp, const float* head_w, int Tq,
+                                int NBk, int Hi, long long q_pos0, int mode, int b0, int nb, int row0, int rows,
+                                const float* tau, uint2* cand, int* cnt, int cap, cudaStream_t s) {
+  if (rows <= 0 || nb <= 0) return cudaSuccess;
+  const KernelCtl ctl = kernel_ctl(di);
+  switch (Hi) {
+    case 4: return launch_filter_hi<4>(qi, kp, head_w, Tq, NBk, q_pos0, mode, b0, nb, row0, rows, tau, cand, cnt, cap, ctl, s);
+    case 8: return launch_filter_hi<8>(qi, kp, head_w, Tq, NBk, q_pos0, mode, b0, nb, row0, rows, tau, cand, cnt, cap, ctl, s);
     default: return cudaErrorInvalidValue;
   }
 }

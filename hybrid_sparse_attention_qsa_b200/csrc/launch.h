@@ -26,10 +26,18 @@ cudaError_t launch_rope_queries(const void* qi, void* qo, int B, int Tq, int Hi,
 
 // Prefill scores for query rows [row0, row0 + rows) of batches [b0, b0 + nb) into
 // scores + (b - b0) * batch_stride + (t - row0) * ld.
+// With kshift > 0, column c of a row is the score of pooled block (c << kshift) + koff (the sampled
+// scores behind the selection thresholds); columns past the row's visible blocks are not written.
 cudaError_t launch_score_prefill(const DeviceInfo* di, const void* qi, const void* kp, const float* head_w, int B,
                                  int Tq, int NBk, int Hi, int Di, int blk, long long q_pos0, int mode, int b0, int nb,
                                  int row0, int rows, float* scores, long long ld, long long batch_stride,
-                                 cudaStream_t s);
+                                 cudaStream_t s, int kshift = 0, int koff = 0);
+// Scores of rows [row0, row0 + rows) of batches [b0, b0 + nb) compared with tau[list] on the fly;
+// the survivors go to cand[list][0 .. cap) in block order and their number to cnt[list], where
+// list = (b - b0) * rows + (t - row0).  Hi must be 4 or 8.
+cudaError_t launch_score_filter(const DeviceInfo* di, const void* qi, const void* kp, const float* head_w, int Tq,
+                                int NBk, int Hi, long long q_pos0, int mode, int b0, int nb, int row0, int rows,
+                                const float* tau, uint2* cand, int* cnt, int cap, cudaStream_t s);
 cudaError_t launch_score_decode(const DeviceInfo* di, const void* qi, const void* kp, const float* head_w,
                                 const int32_t* seqlens, int B, int NBk, int Hi, int Di, int blk, int mode,
                                 float* scores, long long ld, cudaStream_t s);
@@ -39,6 +47,18 @@ cudaError_t launch_score_decode(const DeviceInfo* di, const void* qi, const void
 cudaError_t launch_topk(const DeviceInfo* di, const float* scores, long long ld, long long batch_stride,
                         const int32_t* seqlens, int Tq, int NBk, int blk, long long q_pos0, int b0, int nb, int row0,
                         int rows, int k, int32_t* idx, cudaStream_t s);
+
+// Filtered selection (prefill): thresholds from sampled scores, the exact select over each row's
+// candidate list, and the exact redo of the rows listed in fail[1 .. fail[0]].
+cudaError_t launch_select_tau(const DeviceInfo* di, const float* samp, long long ld, int NBk, long long q_pos0,
+                              int row0, int rows, int cap, int rank, int kshift, int koff, float* tau, int* fail,
+                              cudaStream_t s);
+cudaError_t launch_select_candidates(const DeviceInfo* di, const uint2* cand, const int* cnt, int cap, int Tq, int NBk,
+                                     long long q_pos0, int b, int row0, int rows, int k, int32_t* idx, int* fail,
+                                     cudaStream_t s);
+cudaError_t launch_topk_fallback(const DeviceInfo* di, const void* qi, const void* kp, const float* head_w, int Hi,
+                                 int mode, int Tq, int NBk, long long q_pos0, int b, const int* fail, float* scratch,
+                                 int nctas, int k, int32_t* idx, cudaStream_t s);
 
 cudaError_t launch_attn_prefill(const DeviceInfo* di, const void* q, const void* k, const void* v, const int32_t* idx,
                                 int B, int Tq, int Tk, int Hq, int Hkv, int k_blocks, long long q_pos0, float scale,

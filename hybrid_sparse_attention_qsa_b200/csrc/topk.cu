@@ -249,7 +249,7 @@ __global__ void __launch_bounds__(kTopkThreads, 3) topk_kernel(const float* __re
   uint32_t* misc = sel + 2;                      // counter
   uint32_t* bitmap = misc + 5;                   // bitmap_words
 
-  const int tid = threadIdx.x, lane = tid & 31;
+  const int tid = threadIdx.x;
   const int r = row0 + static_cast<int>(blockIdx.x);
   const int bz = blockIdx.y;
   const int b = b0 + bz;
@@ -707,6 +707,65 @@ __global__ void __launch_bounds__(kWarpRowsPerCta * 32) topk_warp_kernel(
   }
 }
 
+// ======================================================================================
+// Exact redo of the rows that the filtered selection could not settle (list shorter than k, or
+// overflowing): one CTA per failed row at a time, grid-striding over the failure list
+// fail[1 .. fail[0]].  The row's scores are recomputed on CUDA cores in fp32 into the CTA's
+// scratch row (same formula: ReLU or linear per head, weighted sum), then selected exactly by the
+// three-pass radix select over memory.  With no failure the kernel only reads fail[0].
+__global__ void __launch_bounds__(kTopkThreads) topk_fallback_kernel(
+    const uint16_t* __restrict__ qi, const uint16_t* __restrict__ kp, const float* __restrict__ head_w, int Hi,
+    int mode, int Tq, int NBk, long long q_pos0, int b, const int* __restrict__ fail, float* __restrict__ scratch,
+    int k, int32_t* __restrict__ idx) {
+  __shared__ float qf[8 * 64];
+  __shared__ uint32_t hist[kBins];
+  __shared__ uint32_t ws[kWarps + 1];
+  __shared__ uint32_t sel[2];
+  const int tid = threadIdx.x;
+  const int nf = fail[0];
+  float* s = scratch + static_cast<long long>(blockIdx.x) * NBk;
+  float w[8];
+#pragma unroll
+  for (int h = 0; h < 8; ++h) w[h] = h < Hi ? (head_w ? head_w[h] : 1.0f) : 0.0f;
+  for (int f = blockIdx.x; f < nf; f += gridDim.x) {
+    const int t = fail[1 + f];
+    const int n = static_cast<int>(min(static_cast<long long>(NBk), (q_pos0 + t) >> 2));
+    const uint16_t* qrow = qi + (static_cast<long long>(b) * Tq + t) * Hi * 64;
+    for (int i = tid; i < Hi * 64; i += kTopkThreads) qf[i] = __uint_as_float(static_cast<uint32_t>(qrow[i]) << 16);
+    __syncthreads();
+    for (int j = tid; j < n; j += kTopkThreads) {
+      const uint4* kr = reinterpret_cast<const uint4*>(kp + (static_cast<long long>(b) * NBk + j) * 64);
+      float acc[8];
+#pragma unroll
+      for (int h = 0; h < 8; ++h) acc[h] = 0.0f;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const uint4 v = __ldg(kr + c);
+        const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float x = __uint_as_float((e & 1) ? (wd[e >> 1] & 0xFFFF0000u) : (wd[e >> 1] << 16));
+#pragma unroll
+          for (int h = 0; h < 8; ++h)
+            if (h < Hi) acc[h] = fmaf(qf[h * 64 + c * 8 + e], x, acc[h]);
+        }
+      }
+      float sc = 0.0f;
+#pragma unroll
+      for (int h = 0; h < 8; ++h) {
+        if (h < Hi) {
+          const float x = mode == 0 ? fmaxf(acc[h], 0.0f) : acc[h];
+          sc = fmaf(w[h], x, sc);
+        }
+      }
+      s[j] = sc;
+    }
+    __syncthreads();
+    topk_global(s, n, k, idx + (static_cast<long long>(b) * Tq + t) * k, hist, ws, sel);
+    __syncthreads();
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_topk(const DeviceInfo* di, const float* scores, long long ld, long long batch_stride,
@@ -739,6 +798,17 @@ cudaError_t launch_topk(const DeviceInfo* di, const float* scores, long long ld,
   dim3 grid(rows, nb);
   topk_kernel<<<grid, kTopkThreads, smem, s>>>(scores, ld, batch_stride, seqlens, Tq, NBk, blk, q_pos0, b0, row0, k,
                                                idx, words, kernel_ctl(di));
+  return cudaPeekAtLastError();
+}
+
+cudaError_t launch_topk_fallback(const DeviceInfo* di, const void* qi, const void* kp, const float* head_w, int Hi,
+                                 int mode, int Tq, int NBk, long long q_pos0, int b, const int* fail, float* scratch,
+                                 int nctas, int k, int32_t* idx, cudaStream_t s) {
+  (void)di;
+  if (nctas <= 0) return cudaSuccess;
+  topk_fallback_kernel<<<nctas, kTopkThreads, 0, s>>>(static_cast<const uint16_t*>(qi),
+                                                      static_cast<const uint16_t*>(kp), head_w, Hi, mode, Tq, NBk,
+                                                      q_pos0, b, fail, scratch, k, idx);
   return cudaPeekAtLastError();
 }
 

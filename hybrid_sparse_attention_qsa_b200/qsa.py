@@ -44,6 +44,7 @@ SIGNATURES = {
     "qsa_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I, _I]),
     "qsa_decode_default_splits": (_I, [_I, _I]),
     "qsa_get_device_status": (_I, [_P]),
+    "qsa_set_select_options": (_I, [_I, _I]),
     "qsa_set_wait_timeout_ns": (None, [_U64]),
     "qsa_wait_timeout_selftest": (_I, [_U64, _P]),
 }
@@ -284,6 +285,14 @@ def qsa_sparse_attn_decode_noalloc(q: torch.Tensor, kcache: torch.Tensor, vcache
 def qsa_get_device_status(device=None) -> int:
     """Synchronise the current stream and read + clear the device status word."""
     return int(lib().qsa_get_device_status(_stream(device)))
+
+
+QSA_SELECT_AUTO, QSA_SELECT_MATERIALISED, QSA_SELECT_FILTERED = 0, 1, 2
+
+
+def qsa_set_select_options(path: int = QSA_SELECT_AUTO, sample_rank: int = 0) -> None:
+    """How qsa_select_topk computes a prefill selection without given scores (process-wide)."""
+    _check(lib().qsa_set_select_options(path, sample_rank), "qsa_set_select_options")
 
 
 def qsa_set_wait_timeout_ns(ns: int) -> None:

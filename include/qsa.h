@@ -133,12 +133,24 @@ QSA_API qsa_status_t qsa_index_score(const void* qi, const void* kp, const float
  *   listed (it is implicit).
  * scores != NULL: select from scores [B][Tq][ld_scores] (as written by qsa_index_score); qi, kp,
  *   head_w, mode and workspace are ignored.
- * scores == NULL: the scores are computed here, chunk by chunk, into `workspace` (at least one
- *   score row of NBk floats; qsa_workspace_size(QSA_OP_SELECT_TOPK, ...) gives the size that lets
- *   the whole call run in few chunks).  Arguments as for qsa_index_score.  With more than one
- *   chunk the workspace is split in two halves and the top-k of one chunk runs on a per-device
- *   internal stream while the next chunk is scored on `stream`; the internal stream is joined back
- *   into `stream` before the call returns, so the call keeps the usual stream-ordered semantics.
+ * scores == NULL: the scores are computed here.  Arguments as for qsa_index_score.  Two ways,
+ *   both giving the same index lists; qsa_set_select_options can force one:
+ *   - materialised (decode; Hi of 1 or 2; short prefills): the scores are computed chunk by chunk
+ *     into `workspace` (at least one score row of NBk floats).  With more than one chunk the
+ *     workspace is split in two halves and the top-k of one chunk runs on a per-device internal
+ *     stream while the next chunk is scored on `stream`; the internal stream is joined back into
+ *     `stream` before the call returns, so the call keeps the usual stream-ordered semantics.
+ *   - filtered (prefill with Hi of 4 or 8, chosen automatically from 16384 rows per sequence when
+ *     the workspace holds 4096 rows or all of them): the scores are never stored.  Every 16th
+ *     pooled block is scored first; per row, a threshold with about 2.5 k (at least 1024) of the
+ *     row's scores expected above it is read off these samples; the tensor-core score kernel then
+ *     keeps only the scores at or above the threshold, in block order, and the top-k is selected
+ *     from that list.  A row whose list is shorter than k or longer than its capacity is redone
+ *     exactly over all its scores, so the result never depends on the thresholds.  Workspace per
+ *     row of a chunk: about 4 * NBk / 16 + 256 * max(64, ceil(5 k / 32)) bytes, plus
+ *     128 * NBk * 4 bytes for the redo.
+ *   qsa_workspace_size(QSA_OP_SELECT_TOPK, ...) gives a size that fits either way in few chunks
+ *   (up to about 4 GiB).
  * Errors: INVALID_ARGUMENT (k < 1, ...), UNSUPPORTED, WORKSPACE_TOO_SMALL.
  */
 QSA_API qsa_status_t qsa_select_topk(const float* scores, int64_t ld_scores, const void* qi,
@@ -227,6 +239,16 @@ QSA_API int qsa_decode_default_splits(int B, int k_blocks);
  * QSA_ERR_CUDA (the synchronisation itself failed).
  */
 QSA_API qsa_status_t qsa_get_device_status(void* stream);
+
+/*
+ * Chooses how qsa_select_topk computes a prefill selection when it is not given scores, for all
+ * later calls from this process: path 0 = automatic (default), 1 = materialised scores,
+ * 2 = filtered (UNSUPPORTED unless Hi is 4 or 8).  sample_rank > 0 replaces the filtered path's
+ * rank of the threshold among a row's samples (a testing and tuning knob: a small rank makes
+ * short lists and a large one overflowing lists, both redone exactly); 0 restores the default.
+ * Errors: INVALID_ARGUMENT (path outside 0..2, sample_rank < 0).
+ */
+QSA_API qsa_status_t qsa_set_select_options(int path, int sample_rank);
 
 /*
  * Device-side wait limit in nanoseconds for all later launches from this process (default

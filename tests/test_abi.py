@@ -101,9 +101,34 @@ def test_select_and_attention_argument_checks(lib):
     assert dec(None, 0, -1) == Q.QSA_ERR_INVALID_ARGUMENT
 
 
+def filtered_bytes(rows, nbk, k):
+    # the filtered selection's workspace as include/qsa.h states it: per row the sampled scores
+    # (every 16th block, padded to 4), threshold, count and failure slot, and the candidate list
+    # of 32 * max(64, ceil(5k/32)) (key, block) pairs; plus 128 scratch rows and alignment
+    rank = max(64, (5 * k + 31) // 32)
+    ns = (nbk - 9) // 16 + 1 if nbk > 8 else 0
+    per_row = ((max(ns, 1) + 3) // 4 * 4) * 4 + 12 + 32 * rank * 8
+    return 6 * 256 + 4 + 128 * max(nbk, 1) * 4 + rows * per_row
+
+
 def test_workspace_sizes(lib):
+    # 128K prefill: every row fits the filtered path in one chunk (under 4 GiB)
     n = Q.qsa_workspace_size(Q.QSA_OP_SELECT_TOPK, 1, 131072, 32768, 512, 16, 128)
-    assert n >= 32768 * 4 and n <= 512 << 20 and n % (32768 * 4) == 0
+    assert n == filtered_bytes(131072, 32768, 512) and n <= 4 << 30
+    # 1M prefill: chunks of rows within 4 GiB, never less than a 512 MiB chunk of score rows
+    n = Q.qsa_workspace_size(Q.QSA_OP_SELECT_TOPK, 1, 1048576, 262144, 512, 16, 128)
+    assert (512 << 20) <= n <= 4 << 30
+    # short prefill: the materialised chunk of all rows can be the larger of the two
+    n = Q.qsa_workspace_size(Q.QSA_OP_SELECT_TOPK, 1, 2048, 512, 64, 1, 128)
+    assert n == max(2048 * 512 * 4, filtered_bytes(2048, 512, 64))
     assert Q.qsa_workspace_size(Q.QSA_OP_SELECT_TOPK, 32, 1, 65536, 512, 16, 128) == 32 * 65536 * 4
     assert Q.qsa_workspace_size(Q.QSA_OP_SPARSE_ATTN_DECODE, 32, 1, 0, 512, 16, 128, 5) == 32 * 5 * 16 * 130 * 4
     assert Q.qsa_workspace_size(99, 1, 1, 1, 1, 1, 1) == 0
+
+
+def test_select_options_checks(lib):
+    assert lib.qsa_set_select_options(3, 0) == Q.QSA_ERR_INVALID_ARGUMENT
+    assert lib.qsa_set_select_options(-1, 0) == Q.QSA_ERR_INVALID_ARGUMENT
+    assert lib.qsa_set_select_options(0, -5) == Q.QSA_ERR_INVALID_ARGUMENT
+    assert lib.qsa_set_select_options(2, 7) == Q.QSA_OK
+    assert lib.qsa_set_select_options(0, 0) == Q.QSA_OK

@@ -43,11 +43,20 @@ def test_decode_work():
 def test_select_launch_count():
     w = I.WORKLOADS["prefill_128k"]
     nbk = w.T // 4
-    # four chunks of rows -> 4 score + 4 top-k launches
-    assert bench.select_launches(w, nbk * 4 * (w.T // 4)) == 8
+    # a workspace too small for the filtered path (under 4096 rows of lists): 132 chunks of 1000
+    # score rows -> 132 score + 132 top-k launches
+    assert bench.select_launches(w, nbk * 4 * 1000) == 264
     # the first chunk of a 1-row workspace holds rows 0..0: no candidate, no score launch
     tiny = w.with_(T=12)
     assert bench.select_launches(tiny, 3 * 4) == 12 + 12 - 4
+    # the size the library asks for: the filtered path in one chunk, five launches
+    from hybrid_sparse_attention_qsa_b200 import qsa as Q
+    ws = Q.qsa_workspace_size(Q.QSA_OP_SELECT_TOPK, w.B, w.T, nbk, w.k, w.Hq, w.D)
+    assert bench.select_launches(w, ws) == 5
+    # short sequences stay on the materialised path
+    short = w.with_(T=8192)
+    ws = Q.qsa_workspace_size(Q.QSA_OP_SELECT_TOPK, 1, short.T, short.T // 4, short.k, 16, 128)
+    assert bench.select_launches(short, ws) == 2
 
 
 def _free_port():
