@@ -66,6 +66,7 @@ constexpr int kSampleOff = 8;         // ... starting at block 8
 constexpr int kFallbackCtas = 128;    // CTAs (and scratch rows) of the exact redo of failed rows
 constexpr long long kFusedTarget = 4ll << 30;   // workspace the size query plans the filtered path in
 constexpr int kFusedMinRows = 16384;  // automatic choice: rows per sequence from which it pays
+constexpr int kFusedMaxCap = 5120;    // longest candidate list the select kernel holds (k <= 1024)
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
@@ -235,7 +236,7 @@ qsa_status_t qsa_select_topk(const float* scores, int64_t ld_scores, const void*
     const FusedPlan fp = fused_plan(NBk, k);
     const long long fit = fused_rows_fit(fp, ws_bytes);
     const int path = g_select_path.load();
-    const bool able = Hi == 4 || Hi == 8;
+    const bool able = (Hi == 4 || Hi == 8) && fp.cap <= kFusedMaxCap;
     if (path == 2 && !able) return QSA_ERR_UNSUPPORTED;
     if (path == 2 && fit < 1) return QSA_ERR_WORKSPACE_TOO_SMALL;
     if (path == 2 || (path == 0 && able && Tq >= kFusedMinRows && fit >= std::min(Tq, 4096))) {

@@ -236,7 +236,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tm_empty[acc]);
+      if (lane == 0) mbar_arrive_relaxed(&tm_empty[acc]);   // the tile's TMEM loads are complete
     }
   }
   tc_fence_before();
@@ -251,22 +251,21 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
 // Selection without materialised scores.  The same tile pipeline as score_prefill_kernel, one CTA
 // per strip of kN/HI queries over ALL their visible pooled keys (strips taken longest first).  The
 // epilogue compares each score with its query's threshold tau (set beforehand from sampled scores,
-// -inf for rows short enough to keep everything) and appends the survivors (order-preserving key,
-// block index) to the query's candidate list IN INDEX ORDER: the four warps that read the four TMEM
+// -inf for rows short enough to keep everything) and appends the survivors (fp32 score bits, block
+// index) to the query's candidate list IN INDEX ORDER: the four warps that read the four TMEM
 // lane quadrants of a column half exchange their per-query counts of a tile through shared memory,
 // so every position is known without atomics.  Only the first `cap` entries of a list are stored;
 // the full count is written, so the selection can tell an overflowing list.
 constexpr int kFiltEpiWarps = 16;                 // four per TMEM lane quadrant
 constexpr int kFiltGroups = kFiltEpiWarps / 4;      // column groups of kN / kFiltGroups columns
 constexpr int kFiltThreads = 64 + kFiltEpiWarps * 32;
-constexpr int kFiltStash = 17;   // floats per lane row of the score stash (queries of a warp + 1)
-constexpr int kFiltSmem = 1024 + kQiBytes + kStages * kKpBytes + 256 + kFiltEpiWarps * 32 * kFiltStash * 4 +
-                          kFiltEpiWarps * 32 * 4 * 2 + 2 * kFiltGroups * 4 * 32 * 4;
+constexpr int kFiltSmem = 1024 + kQiBytes + kStages * kKpBytes + 256 + 2 * kFiltGroups * 4 * 32 * 4 +
+                          kFiltEpiWarps * 32 * 4;
 
 struct FilterArgs {
   const float* head_w;
   const float* tau;     // [rows] threshold of row row0 + i
-  uint2* cand;          // [rows][cap] (key, block index)
+  uint2* cand;          // [rows][cap] (fp32 score bits, block index)
   int* cnt;             // [rows] number of scores >= tau (may exceed cap)
   long long q_pos0;
   int NBk, b0, row0, rows, cap;
@@ -285,7 +284,7 @@ __global__ void __launch_bounds__(kFiltThreads, 1)
   constexpr int CW = kN / kFiltGroups;         // TMEM columns per epilogue warp
   constexpr int QW = CW / HI;                  // queries per epilogue warp
   constexpr int QC = 32 / HI;                  // queries per 32-column TMEM load
-  static_assert(QW < kFiltStash && QW <= 32, "stash row and one bit per query of a warp");
+  static_assert(QW <= 32, "one lane per query of a warp");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* qi_s = smem;
@@ -298,10 +297,8 @@ __global__ void __launch_bounds__(kFiltThreads, 1)
   uint64_t* tm_empty = tm_full + 2;
   uint64_t* mma_done = tm_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
-  float* stash = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 256);   // [warp][lane][kFiltStash]
-  uint32_t* xmask = reinterpret_cast<uint32_t*>(stash + kFiltEpiWarps * 32 * kFiltStash);   // [warp][32]
-  uint32_t* xoff = xmask + kFiltEpiWarps * 32;                                                // [warp][32]
-  uint32_t* xcnt = xoff + kFiltEpiWarps * 32;                         // [2 tiles][groups][4 quadrants][32]
+  uint32_t* xcnt = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(bars) + 256);  // [2][groups][4][32]
+  uint32_t* xoff = xcnt + 2 * kFiltGroups * 4 * 32;                                       // [warp][32]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bz = blockIdx.z;
@@ -370,10 +367,9 @@ __global__ void __launch_bounds__(kFiltThreads, 1)
     // Slices below the first query's visible blocks need no visibility test when every query exists.
     const int nb_min_full =
         qbase + QW - 1 <= tl_last ? static_cast<int>(min(static_cast<long long>(a.NBk), (pos_first + qbase) >> 2)) : 0;
-    float* my_stash = stash + (ew * 32 + lane) * kFiltStash;
-    uint32_t* my_mask = xmask + ew * 32;
-    uint32_t* my_off = xoff + ew * 32;
     uint2* list_q0 = a.cand + (list0 + qbase) * a.cap;   // list of the warp's first query
+    uint32_t* my_off = xoff + ew * 32;
+    const uint32_t lane_bit = 1u << lane;
     uint32_t run = 0;   // lane q: entries of query qbase + q before the current tile
     bool dead = false;  // a wait timed out: keep meeting the barriers, touch nothing
     for (int i = 0; i < nt; ++i) {
@@ -382,7 +378,8 @@ __global__ void __launch_bounds__(kFiltThreads, 1)
       if (!dead && !mbar_wait_suspend(&tm_full[acc], aph, a.ctl)) dead = true;
       tc_fence_after();
       const int kb = i * kM + quad * 32 + lane;   // pooled block owned by this thread
-      uint32_t bits = 0;
+      float sc[QW];      // this thread's scores of the warp's queries
+      uint32_t m[QW];    // per query: the lanes (blocks) whose score passes (warp-uniform)
       // One pass over the warp's scores of the tile; FULL: every query of the warp exists and sees
       // every block of its slice (tiles below the diagonal band), so no visibility test.
       auto filter_tile = [&](auto full_c) {
@@ -395,21 +392,19 @@ __global__ void __launch_bounds__(kFiltThreads, 1)
 #pragma unroll
           for (int qq = 0; qq < QC; ++qq) {
             const int q = c * QC + qq;
-            float sc = 0.0f;
+            float x0 = 0.0f;
 #pragma unroll
             for (int h = 0; h < HI; ++h) {
               float x = __uint_as_float(r[qq * HI + h]);
               if (MODE == 0) x = fmaxf(x, 0.0f);
-              sc = fmaf(w[h], x, sc);
+              x0 = fmaf(w[h], x, x0);
             }
-            bool pass = sc >= tq[q];
+            bool pass = x0 >= tq[q];
             if (!FULL)
               pass = pass && qbase + q <= tl_last &&
                      kb < static_cast<int>(min(static_cast<long long>(a.NBk), (pos_first + qbase + q) >> 2));
-            my_stash[q] = sc;
-            const uint32_t m = __ballot_sync(0xffffffffu, pass);
-            my_mask[q] = m;   // the same value from every lane
-            if (pass) bits |= 1u << q;
+            sc[q] = x0;
+            m[q] = __ballot_sync(0xffffffffu, pass);
           }
         }
       };
@@ -418,13 +413,22 @@ __global__ void __launch_bounds__(kFiltThreads, 1)
           filter_tile(std::integral_constant<bool, true>());
         else
           filter_tile(std::integral_constant<bool, false>());
+      } else {
+#pragma unroll
+        for (int q = 0; q < QW; ++q) {
+          sc[q] = 0.0f;
+          m[q] = 0u;
+        }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tm_empty[acc]);
-      // counts of this tile per (quadrant, query) -> each lane's position in its query's list
+      if (lane == 0) mbar_arrive_relaxed(&tm_empty[acc]);   // the tile's TMEM loads are complete
+      // counts of this tile per (quadrant, query) -> the offset of each query's entries
+      uint32_t mine = 0;   // lane q: this warp's count for query q
+#pragma unroll
+      for (int q = 0; q < QW; ++q) mine = lane == q ? static_cast<uint32_t>(__popc(m[q])) : mine;
       uint32_t* xc = xcnt + ((i & 1) * kFiltGroups + grp) * 4 * 32;
-      if (lane < QW) xc[quad * 32 + lane] = dead ? 0u : static_cast<uint32_t>(__popc(my_mask[lane]));
+      if (lane < QW) xc[quad * 32 + lane] = mine;
       named_bar_sync(1 + grp, 128);
       if (lane < QW) {
         uint32_t pre = 0, tot = 0;
@@ -434,18 +438,28 @@ __global__ void __launch_bounds__(kFiltThreads, 1)
           pre += o < quad ? c : 0u;
           tot += c;
         }
-        my_off[lane] = run + pre;
+        my_off[lane] = run + pre;   // position of this warp's first entry of query q = lane
         run += tot;
       }
       __syncwarp();
-      while (bits) {
-        const int q = __ffs(bits) - 1;
-        bits &= bits - 1;
-        const uint32_t p = my_off[q] + static_cast<uint32_t>(__popc(my_mask[q] & lt));
-        if (p < static_cast<uint32_t>(a.cap))
-          list_q0[static_cast<long long>(q) * a.cap + p] = make_uint2(score_key(my_stash[q] + 0.0f), static_cast<uint32_t>(kb));
+      uint32_t offs[QW];   // every lane: the positions of all the warp's queries (broadcast loads)
+#pragma unroll
+      for (int q = 0; q < QW; q += 4) {
+        const uint4 o4 = *reinterpret_cast<const uint4*>(my_off + q);
+        offs[q] = o4.x;
+        offs[q + 1] = o4.y;
+        offs[q + 2] = o4.z;
+        offs[q + 3] = o4.w;
       }
-      __syncwarp();
+      // each query's passing lanes store (raw score bits, block) to consecutive list positions;
+      // branch-free: a store with no passing lane is fully predicated off
+#pragma unroll
+      for (int q = 0; q < QW; ++q) {
+        const uint32_t p = offs[q] + static_cast<uint32_t>(__popc(m[q] & lt));
+        if ((m[q] & lane_bit) && p < static_cast<uint32_t>(a.cap))
+          list_q0[static_cast<long long>(q) * a.cap + p] = make_uint2(__float_as_uint(sc[q]), static_cast<uint32_t>(kb));
+      }
+      __syncwarp();   // my_off is rewritten by the next tile
     }
     if (quad == 0 && lane < QW && qbase + lane <= tl_last) a.cnt[list0 + qbase + lane] = static_cast<int>(run);
   }

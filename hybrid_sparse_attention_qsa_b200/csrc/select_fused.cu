@@ -24,195 +24,230 @@
 namespace qsa {
 namespace {
 
-constexpr int kTauWarps = 4;
-constexpr int kTauBins = 2048;    // bins over the bits where a row's sampled keys differ
-constexpr int kSelWarps = 4;
 constexpr int kSelBins = 2048;    // bins of the first select pass (11 bits)
-constexpr int kSelSmemMax = 200 * 1024;
-
-__device__ __forceinline__ uint32_t lane_lt() {
-  uint32_t m;
-  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
-  return m;
-}
 
 __device__ __forceinline__ float key_to_float(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
 
-// Finds, over bins numbered 0..nbins-1 (a larger bin holds larger keys), the bin holding the
-// rank-th largest entry; returns it and the number of entries in higher bins.  Lane l scans
-// bins [nbins - (l + 1) * per, nbins - l * per) with per = nbins / 32; all lanes get the result.
-__device__ __forceinline__ uint32_t warp_find_bin(const uint32_t* hist, int nbins, uint32_t rank, uint32_t* above_out) {
-  const int lane = threadIdx.x & 31;
-  const int per = nbins / 32;
-  const int lo = nbins - (lane + 1) * per;
-  uint32_t local = 0;
-  for (int q = 0; q < per; q += 4) {
-    const uint4 v = *reinterpret_cast<const uint4*>(hist + lo + q);
-    local += v.x + v.y + v.z + v.w;
-  }
-  uint32_t incl = local;   // entries in this lane's bins and every higher bin
+constexpr int kSelThreads = 128;
+constexpr int kSelWarpsPerRow = kSelThreads / 32;
+
+// Exclusive block scan of one value per thread; also returns the block total.  Ends synchronised.
+__device__ __forceinline__ uint32_t sel_block_scan(uint32_t v, uint32_t* ws, uint32_t* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t x = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
+    const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
   }
-  const uint32_t above = incl - local;
-  const uint32_t win = __ballot_sync(0xffffffffu, above < rank && incl >= rank);
-  const int wl = win ? __ffs(win) - 1 : 31;
-  uint32_t acc = __shfl_sync(0xffffffffu, above, wl);
-  // the winning lane's bins, one per lane from its top (per <= 128 handled in chunks of 32)
-  const int wlo = nbins - (wl + 1) * per;
-  for (int top = wlo + per - 1; top >= wlo; top -= 32) {
-    const int bin = top - lane;
-    const uint32_t h = bin >= wlo ? hist[bin] : 0u;
-    uint32_t inc = h;   // entries in bins top-lane .. top
+  if (lane == 31) ws[warp] = x;
+  __syncthreads();
+  uint32_t before = 0, all = 0;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
-      if (lane >= o) inc += y;
-    }
-    const uint32_t hit = __ballot_sync(0xffffffffu, acc + inc >= rank && bin >= wlo);
-    if (hit) {
-      const int src = __ffs(hit) - 1;
-      *above_out = acc + __shfl_sync(0xffffffffu, inc - h, src);
-      return static_cast<uint32_t>(top - src);
-    }
-    acc += __shfl_sync(0xffffffffu, inc, 31);
+  for (int w = 0; w < kSelWarpsPerRow; ++w) {
+    const uint32_t t = ws[w];
+    before += w < warp ? t : 0u;
+    all += t;
   }
-  *above_out = acc;   // unreachable when rank <= the total
-  return static_cast<uint32_t>(wlo);
+  __syncthreads();
+  *total = all;
+  return before + x - v;
+}
+
+// Finds, over kSelBins bins in shared memory (a larger bin holds larger keys), the bin holding the
+// rank-th largest entry with the whole CTA; returns (bin, entries in higher bins) in sel[0], sel[1].
+// Ends synchronised.
+__device__ __forceinline__ void block_find_bin(const uint32_t* hist, uint32_t rank, uint32_t* ws, uint32_t* sel) {
+  constexpr int per = kSelBins / kSelThreads;
+  const int tid = threadIdx.x;
+  const int lo = kSelBins - per * (tid + 1);   // thread 0 holds the top bins
+  uint32_t local = 0;
+#pragma unroll
+  for (int q = 0; q < per; q += 4) {
+    const uint4 h4 = *reinterpret_cast<const uint4*>(hist + lo + q);
+    local += h4.x + h4.y + h4.z + h4.w;
+  }
+  uint32_t total;
+  const uint32_t above = sel_block_scan(local, ws, &total);   // entries in bins above this range
+  if (above < rank && above + local >= rank) {
+    uint32_t acc = above;
+    for (int q = per - 1; q >= 0; --q) {
+      const uint32_t h = hist[lo + q];
+      if (acc + h >= rank) {
+        sel[0] = static_cast<uint32_t>(lo + q);
+        sel[1] = acc;
+        break;
+      }
+      acc += h;
+    }
+  }
+  __syncthreads();
+}
+
+// Block-wide min and max of one key per thread (ws: 2 * kSelWarpsPerRow words).  Ends synchronised.
+__device__ __forceinline__ void block_minmax(uint32_t& kmin, uint32_t& kmax, uint32_t* ws) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  if (lane == 0) {
+    ws[2 * warp] = kmin;
+    ws[2 * warp + 1] = kmax;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int w = 0; w < kSelWarpsPerRow; ++w) {
+    kmin = min(kmin, ws[2 * w]);
+    kmax = max(kmax, ws[2 * w + 1]);
+  }
+  __syncthreads();
 }
 
 // ---------------------------------------------------------------------------------------------
-// Step 2: one warp per row.  tau = the lowest key of the histogram bin that holds the rank-th
-// largest sampled score (so at least `rank` samples are >= tau); -inf for rows of at most `cap`
-// blocks, whose lists keep every block.  The 2048 bins span the bits where the row's sampled keys
-// differ, so the samples spread over the bins whatever the scale of the scores.
-template <typename F>
-__device__ __forceinline__ void for_each_sample(const float* s, int m, F&& f) {
-  const int lane = threadIdx.x & 31;
-  // rows start 16-byte aligned (ld is a multiple of 4): 16-byte loads, eight in flight per lane
-  for (int base = 0; base < m; base += 32 * 4 * 8) {
-    float4 v[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int i0 = base + (u * 32 + lane) * 4;
-      v[u] = i0 < m ? __ldcg(reinterpret_cast<const float4*>(s + i0)) : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int i0 = base + (u * 32 + lane) * 4;
-      const float e[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        if (i0 + j < m) f(score_key(e[j] + 0.0f));
-    }
-  }
-}
+// Step 2: one CTA of kSelThreads per row.  tau = the lowest key of the histogram bin that holds
+// the rank-th largest sampled score (so at least `rank` samples are >= tau); -inf for rows of at
+// most `cap` blocks, whose lists keep every block.  The kSelBins bins span the bits where the
+// row's sampled keys differ, so the samples spread over the bins whatever the scale of the scores.
+// Up to kTauRegs * kSelThreads samples are read once into registers; longer rows are read twice.
+constexpr int kTauRegs = 16;
 
-__global__ void __launch_bounds__(kTauWarps * 32) tau_kernel(const float* __restrict__ samp, long long ld, int NBk,
-                                                             long long q_pos0, int row0, int rows, int cap, int rank,
-                                                             int kshift, int koff, float* __restrict__ tau,
-                                                             int* __restrict__ fail) {
-  extern __shared__ uint32_t tsm[];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (blockIdx.x == 0 && threadIdx.x == 0) fail[0] = 0;   // the failure list of this chunk starts empty
-  const int L = static_cast<int>(blockIdx.x) * kTauWarps + warp;
-  if (L >= rows) return;
+__global__ void __launch_bounds__(kSelThreads) tau_kernel(const float* __restrict__ samp, long long ld, int NBk,
+                                                          long long q_pos0, int row0, int cap, int rank, int kshift,
+                                                          int koff, float* __restrict__ tau, int* __restrict__ fail) {
+  __shared__ __align__(16) uint32_t hist[kSelBins];
+  __shared__ uint32_t ws[2 * kSelWarpsPerRow];
+  __shared__ uint32_t sel[2];
+  const int tid = threadIdx.x;
+  const int L = static_cast<int>(blockIdx.x);
+  if (L == 0 && tid == 0) fail[0] = 0;   // the failure list of this chunk starts empty
   const int n = static_cast<int>(min(static_cast<long long>(NBk), (q_pos0 + row0 + L) >> 2));
   if (n <= cap) {
-    if (lane == 0) tau[L] = -INFINITY;
+    if (tid == 0) tau[L] = -INFINITY;
     return;
   }
   const int m = n > koff ? ((n - koff - 1) >> kshift) + 1 : 0;
-  const float* s = samp + static_cast<long long>(L) * ld;
+  const float* s = samp + static_cast<long long>(L) * ld;   // 16-byte aligned (ld is a multiple of 4)
+  const bool in_regs = m <= kTauRegs * kSelThreads;
+  uint32_t key[kTauRegs];
   uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
-  for_each_sample(s, m, [&](uint32_t key) {
-    kmin = min(kmin, key);
-    kmax = max(kmax, key);
-  });
-  kmin = __reduce_min_sync(0xffffffffu, kmin);
-  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  if (in_regs) {
+    float4 f[kTauRegs / 4];
+#pragma unroll
+    for (int u = 0; u < kTauRegs / 4; ++u) {
+      const int i0 = (tid + u * kSelThreads) * 4;
+      f[u] = i0 < m ? __ldcs(reinterpret_cast<const float4*>(s + i0)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < kTauRegs / 4; ++u) {
+      const int i0 = (tid + u * kSelThreads) * 4;
+      const float e[4] = {f[u].x, f[u].y, f[u].z, f[u].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        key[u * 4 + j] = score_key(e[j] + 0.0f);
+        if (i0 + j < m) {
+          kmin = min(kmin, key[u * 4 + j]);
+          kmax = max(kmax, key[u * 4 + j]);
+        }
+      }
+    }
+  } else {
+    for (int i = tid; i < m; i += kSelThreads) {
+      const uint32_t k1 = score_key(s[i] + 0.0f);
+      kmin = min(kmin, k1);
+      kmax = max(kmax, k1);
+    }
+  }
+  block_minmax(kmin, kmax, ws);
   if (kmin == kmax) {   // every sample equal
-    if (lane == 0) tau[L] = key_to_float(kmin);
+    if (tid == 0) tau[L] = key_to_float(kmin);
     return;
   }
   const int hb = 31 - __clz(kmin ^ kmax);
   const int sh = max(0, hb - 10);
-  uint32_t* h = tsm + warp * kTauBins;
-  for (int i = lane * 4; i < kTauBins; i += 128) *reinterpret_cast<uint4*>(h + i) = make_uint4(0, 0, 0, 0);
-  __syncwarp();
-  for_each_sample(s, m, [&](uint32_t key) { atomicAdd(&h[(key >> sh) & (kTauBins - 1)], 1u); });
-  __syncwarp();
-  uint32_t above;
-  const uint32_t r = static_cast<uint32_t>(min(rank, m));
-  const uint32_t bin = warp_find_bin(h, kTauBins, r, &above);
+  for (int i = tid * 4; i < kSelBins; i += kSelThreads * 4)
+    *reinterpret_cast<uint4*>(hist + i) = make_uint4(0u, 0u, 0u, 0u);
+  __syncthreads();
+  if (in_regs) {
+#pragma unroll
+    for (int u = 0; u < kTauRegs / 4; ++u) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if ((tid + u * kSelThreads) * 4 + j < m) atomicAdd(&hist[(key[u * 4 + j] >> sh) & (kSelBins - 1)], 1u);
+    }
+  } else {
+    for (int i = tid; i < m; i += kSelThreads) atomicAdd(&hist[(score_key(s[i] + 0.0f) >> sh) & (kSelBins - 1)], 1u);
+  }
+  __syncthreads();
+  block_find_bin(hist, static_cast<uint32_t>(min(rank, m)), ws, sel);
   const uint32_t hi_mask = (sh + 11 >= 32) ? 0u : (0xFFFFFFFFu << (sh + 11));
-  if (lane == 0) tau[L] = key_to_float((kmax & hi_mask) | (bin << sh));
+  if (tid == 0) tau[L] = key_to_float((kmax & hi_mask) | (sel[0] << sh));
 }
 
 // ---------------------------------------------------------------------------------------------
-// Step 4: one warp per row.  The list holds (key, block) pairs in block order.  An 11-bit radix
-// pass over the bits where the listed keys differ finds the bin of the k-th largest key; the keys
-// of that bin are gathered and their remaining low bits resolved one at a time with ballots.  The
-// kept set {key > K*} U {the lowest-block keys == K*} is then emitted in list (= block) order.
+// Step 4: one CTA of kSelThreads per row.  The list holds (fp32 score bits, block) pairs in block
+// order; it is read once into registers (thread t holds entries 2 (t + 128 u) and 2 (t + 128 u) + 1)
+// and the scores turned into order-preserving keys.  An
+// 11-bit histogram over the bits where the listed keys differ finds the bin of the k-th largest
+// key; the keys of that bin are gathered and their remaining low bits resolved one at a time with
+// ballots (warp 0).  The kept set {key > K*} U {the first need_eq keys == K*} is then emitted in
+// list (= block) order with block-wide scans.
 __device__ void fail_row(int* fail, int t) {
-  if ((threadIdx.x & 31) == 0) {
-    const int slot = atomicAdd(&fail[0], 1);
-    fail[1 + slot] = t;
-  }
+  const int slot = atomicAdd(&fail[0], 1);
+  fail[1 + slot] = t;
 }
 
-__global__ void __launch_bounds__(kSelWarps * 32) cand_select_kernel(const uint2* __restrict__ cand,
-                                                                     const int* __restrict__ cnt, int cap, int Tq,
-                                                                     int NBk, long long q_pos0, int b, int row0,
-                                                                     int rows, int k, int32_t* __restrict__ idx,
-                                                                     int* __restrict__ fail) {
-  extern __shared__ uint32_t csm[];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int L = static_cast<int>(blockIdx.x) * (blockDim.x >> 5) + warp;
-  if (L >= rows) return;
+template <int U>
+__global__ void __launch_bounds__(kSelThreads) cand_select_kernel(const uint2* __restrict__ cand,
+                                                                  const int* __restrict__ cnt, int cap, int Tq, int NBk,
+                                                                  long long q_pos0, int b, int row0, int k,
+                                                                  int32_t* __restrict__ idx, int* __restrict__ fail) {
+  __shared__ __align__(16) uint32_t hist[kSelBins];   // histogram, then the k-th bin's keys
+  __shared__ uint32_t ws[2 * kSelWarpsPerRow];
+  __shared__ uint32_t sel[4];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int L = static_cast<int>(blockIdx.x);
   const int t = row0 + L;
   const int n = static_cast<int>(min(static_cast<long long>(NBk), (q_pos0 + t) >> 2));
   int32_t* out = idx + (static_cast<long long>(b) * Tq + t) * k;
   if (n <= k) {
-    for (int i = lane; i < k; i += 32) out[i] = i < n ? i : -1;
+    for (int i = tid; i < k; i += kSelThreads) out[i] = i < n ? i : -1;
     return;
   }
   const int c = cnt[L];
-  if (c < k || c > cap) {
-    fail_row(fail, t);
+  if (c < k || c > cap || c > 2 * U * kSelThreads) {
+    if (tid == 0) fail_row(fail, t);
     return;
   }
-  const uint2* lst = cand + static_cast<long long>(L) * cap;
-  uint32_t* keys = csm + warp * (cap + kSelBins);   // the list's keys
-  uint32_t* hist = keys + cap;                       // 11-bit histogram, then the k-th bin's keys
-  const uint32_t lt = lane_lt();
-
-  // keys into shared memory (eight 8-byte loads in flight per lane), with their min and max
+  // the whole list into registers: U 16-byte loads in flight per thread (cap is even, so every
+  // list starts 16-byte aligned)
+  const uint4* src = reinterpret_cast<const uint4*>(cand + static_cast<long long>(L) * cap);
+  const int c2 = (c + 1) >> 1;
+  uint4 v[U];
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int j = tid + u * kSelThreads;
+    v[u] = j < c2 ? __ldcs(src + j) : make_uint4(0u, 0u, 0u, 0u);
+  }
+  // entry 2j is (v.x, v.y), entry 2j + 1 is (v.z, v.w): fp32 score bits, turned into
+  // order-preserving keys here; invalid entries get key 0 (below any score)
   uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
-  for (int base = 0; base < c; base += 32 * 8) {
-    uint32_t v[8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int i = base + u * 32 + lane;
-      v[u] = i < c ? __ldcs(&lst[i].x) : 0u;
+  for (int u = 0; u < U; ++u) {
+    const int j = tid + u * kSelThreads;
+    v[u].x = score_key(__uint_as_float(v[u].x) + 0.0f);
+    v[u].z = score_key(__uint_as_float(v[u].z) + 0.0f);
+    if (2 * j + 1 >= c) v[u].z = 0u;
+    if (2 * j < c) {
+      kmin = min(kmin, v[u].x);
+      kmax = max(kmax, v[u].x);
     }
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int i = base + u * 32 + lane;
-      if (i < c) {
-        keys[i] = v[u];
-        kmin = min(kmin, v[u]);
-        kmax = max(kmax, v[u]);
-      }
+    if (2 * j + 1 < c) {
+      kmin = min(kmin, v[u].z);
+      kmax = max(kmax, v[u].z);
     }
   }
-  kmin = __reduce_min_sync(0xffffffffu, kmin);
-  kmax = __reduce_max_sync(0xffffffffu, kmax);
-  __syncwarp();
+  block_minmax(kmin, kmax, ws);
 
   bool keep_all = false;
   uint32_t kth = 0, need_eq = 0;
@@ -224,109 +259,159 @@ __global__ void __launch_bounds__(kSelWarps * 32) cand_select_kernel(const uint2
   } else {
     const int hb = 31 - __clz(kmin ^ kmax);      // highest bit where listed keys differ
     const int sh = max(0, hb - 10);              // the 11-bit digit covers bits sh .. sh + 10
-    for (int i = lane * 4; i < kSelBins; i += 128) *reinterpret_cast<uint4*>(hist + i) = make_uint4(0, 0, 0, 0);
-    __syncwarp();
-    for (int i = lane; i < c; i += 32) atomicAdd(&hist[(keys[i] >> sh) & (kSelBins - 1)], 1u);
-    __syncwarp();
-    uint32_t above;
-    const uint32_t B = warp_find_bin(hist, kSelBins, static_cast<uint32_t>(k), &above);
-    uint32_t krem = static_cast<uint32_t>(k) - above;
-    // every listed key shares the bits above bit sh + 10 with kmax
+    for (int i = tid * 4; i < kSelBins; i += kSelThreads * 4)
+      *reinterpret_cast<uint4*>(hist + i) = make_uint4(0u, 0u, 0u, 0u);
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int j = tid + u * kSelThreads;
+      if (2 * j < c) atomicAdd(&hist[(v[u].x >> sh) & (kSelBins - 1)], 1u);
+      if (2 * j + 1 < c) atomicAdd(&hist[(v[u].z >> sh) & (kSelBins - 1)], 1u);
+    }
+    __syncthreads();
+    block_find_bin(hist, static_cast<uint32_t>(k), ws, sel);
+    const uint32_t B = sel[0];
+    uint32_t krem = static_cast<uint32_t>(k) - sel[1];
     const uint32_t hi_mask = (sh + 11 >= 32) ? 0u : (0xFFFFFFFFu << (sh + 11));
-    uint32_t prefix = (kmax & hi_mask) | (B << sh);
+    uint32_t prefix = (kmax & hi_mask) | (B << sh);   // listed keys share the bits above sh + 10
     if (sh > 0) {
-      const uint32_t inbin = hist[B];   // <= c <= cap; the histogram space holds kSelBins keys
-      __syncwarp();
+      const uint32_t inbin = hist[B];
+      if (tid == 0) sel[2] = 0;
+      __syncthreads();   // every thread has read hist[B]: the space now gathers the bin's keys
       if (inbin > static_cast<uint32_t>(kSelBins)) {
-        fail_row(fail, t);
+        if (tid == 0) fail_row(fail, t);
         return;
       }
       uint32_t* buf = hist;
-      uint32_t pos = 0;
-      for (int base = 0; base < c; base += 32) {
-        const int i = base + lane;
-        const uint32_t key = i < c ? keys[i] : 0u;
-        const bool in = i < c && ((key >> sh) & (kSelBins - 1)) == B;
-        const uint32_t bm = __ballot_sync(0xffffffffu, in);
-        if (in) buf[pos + __popc(bm & lt)] = key;
-        pos += __popc(bm);
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int j = tid + u * kSelThreads;
+        if (2 * j < c && ((v[u].x >> sh) & (kSelBins - 1)) == B) buf[atomicAdd(&sel[2], 1u)] = v[u].x;
+        if (2 * j + 1 < c && ((v[u].z >> sh) & (kSelBins - 1)) == B) buf[atomicAdd(&sel[2], 1u)] = v[u].z;
       }
-      __syncwarp();
-      const int mb = static_cast<int>(inbin);
-      for (int bit = sh - 1; bit >= 0; --bit) {
-        const uint32_t want = (prefix >> bit) | 1u;
-        uint32_t cntb = 0;
-        for (int base = 0; base < mb; base += 32) {
-          const int i = base + lane;
-          cntb += __popc(__ballot_sync(0xffffffffu, i < mb && (buf[i] >> bit) == want));
+      __syncthreads();
+      if (warp == 0) {
+        const int mb = static_cast<int>(inbin);
+        for (int bit = sh - 1; bit >= 0; --bit) {
+          const uint32_t want = (prefix >> bit) | 1u;
+          uint32_t cntb = 0;
+          for (int base = 0; base < mb; base += 32) {
+            const int i = base + lane;
+            cntb += __popc(__ballot_sync(0xffffffffu, i < mb && (buf[i] >> bit) == want));
+          }
+          if (cntb >= krem)
+            prefix |= 1u << bit;
+          else
+            krem -= cntb;
         }
-        if (cntb >= krem)
-          prefix |= 1u << bit;
-        else
-          krem -= cntb;
+        if (lane == 0) {
+          sel[0] = prefix;
+          sel[1] = krem;
+        }
       }
+      __syncthreads();
+      prefix = sel[0];
+      krem = sel[1];
     }
     kth = prefix;
     need_eq = krem;
   }
 
-  // ordered emission: keys from shared memory, block indices from the list (batched loads)
-  uint32_t out_run = 0, eq_run = 0;
-  for (int base = 0; base < c; base += 32 * 8) {
-    uint32_t id[8];
+  // ordered emission: round u covers entries [256 u, 256 u + 256), two consecutive per thread.
+  // One pass of warp scans over all rounds at once and one exchange of the warps' round totals
+  // give every entry its number of kept entries before it.
+  uint32_t pk[U];   // per round: (entries > K*) << 16 | (entries == K*) among this thread's two
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int i = base + u * 32 + lane;
-      id[u] = i < c ? __ldcs(&lst[i].y) : 0u;
-    }
+  for (int u = 0; u < U; ++u) {
+    const int j = tid + u * kSelThreads;
+    const bool ok0 = 2 * j < c, ok1 = 2 * j + 1 < c;
+    const bool gt0 = ok0 && (keep_all || v[u].x > kth), gt1 = ok1 && (keep_all || v[u].z > kth);
+    const bool eq0 = ok0 && !keep_all && v[u].x == kth, eq1 = ok1 && !keep_all && v[u].z == kth;
+    pk[u] = ((static_cast<uint32_t>(gt0) + gt1) << 16) | (static_cast<uint32_t>(eq0) + eq1);
+  }
+  const int rounds = (c + 2 * kSelThreads - 1) / (2 * kSelThreads);   // rounds holding entries
+  uint32_t incl[U];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int i = base + u * 32 + lane;
-      const uint32_t key = i < c ? keys[i] : 0u;
-      const bool gt = i < c && (keep_all || key > kth);
-      const bool eq = i < c && !keep_all && key == kth;
-      const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
-      const uint32_t eq_rank = eq_run + __popc(eqm & lt);
-      const bool keep = gt || (eq && eq_rank < need_eq);
-      const uint32_t km = __ballot_sync(0xffffffffu, keep);
-      if (keep) {
-        const uint32_t p = out_run + __popc(km & lt);
-        if (p < static_cast<uint32_t>(k)) out[p] = static_cast<int32_t>(id[u]);
-      }
-      out_run += __popc(km);
-      eq_run += __popc(eqm);
+  for (int u = 0; u < U; ++u) {
+    if (u >= rounds) {   // uniform
+      incl[u] = 0;
+      continue;
     }
+    uint32_t x = pk[u];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    incl[u] = x;
+  }
+  if (lane == 31) {
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      if (u < rounds) hist[u * kSelWarpsPerRow + warp] = incl[u];   // the histogram is no longer needed
+  }
+  __syncthreads();
+  uint32_t gt_tot = 0, eq_tot = 0;   // entries of earlier rounds
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    if (u >= rounds) break;   // uniform
+    uint32_t before = 0, all = 0;
+#pragma unroll
+    for (int w = 0; w < kSelWarpsPerRow; ++w) {
+      const uint32_t t = hist[u * kSelWarpsPerRow + w];
+      before += w < warp ? t : 0u;
+      all += t;
+    }
+    const uint32_t ex = before + incl[u] - pk[u];
+    uint32_t gt_run = gt_tot + (ex >> 16), eq_run = eq_tot + (ex & 0xFFFFu);
+    const int j = tid + u * kSelThreads;
+    const bool ok0 = 2 * j < c, ok1 = 2 * j + 1 < c;
+    const bool gt0 = ok0 && (keep_all || v[u].x > kth), gt1 = ok1 && (keep_all || v[u].z > kth);
+    const bool eq0 = ok0 && !keep_all && v[u].x == kth, eq1 = ok1 && !keep_all && v[u].z == kth;
+    if (gt0) {
+      const uint32_t p = gt_run + min(eq_run, need_eq);
+      if (p < static_cast<uint32_t>(k)) out[p] = static_cast<int32_t>(v[u].y);
+      ++gt_run;
+    } else if (eq0) {
+      if (eq_run < need_eq && gt_run + eq_run < static_cast<uint32_t>(k)) out[gt_run + eq_run] = static_cast<int32_t>(v[u].y);
+      ++eq_run;
+    }
+    if (gt1) {
+      const uint32_t p = gt_run + min(eq_run, need_eq);
+      if (p < static_cast<uint32_t>(k)) out[p] = static_cast<int32_t>(v[u].w);
+    } else if (eq1) {
+      if (eq_run < need_eq && gt_run + eq_run < static_cast<uint32_t>(k)) out[gt_run + eq_run] = static_cast<int32_t>(v[u].w);
+    }
+    gt_tot += all >> 16;
+    eq_tot += all & 0xFFFFu;
   }
 }
+
 
 }  // namespace
 
 cudaError_t launch_select_tau(const DeviceInfo* di, const float* samp, long long ld, int NBk, long long q_pos0,
                               int row0, int rows, int cap, int rank, int kshift, int koff, float* tau, int* fail,
                               cudaStream_t s) {
+  (void)di;
   if (rows <= 0) return cudaSuccess;
-  constexpr int smem = kTauWarps * kTauBins * 4;
-  static std::once_flag once[64];
-  std::call_once(once[di->device & 63],
-                 [] { cudaFuncSetAttribute(tau_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem); });
-  tau_kernel<<<(rows + kTauWarps - 1) / kTauWarps, kTauWarps * 32, smem, s>>>(samp, ld, NBk, q_pos0, row0, rows, cap,
-                                                                            rank, kshift, koff, tau, fail);
+  tau_kernel<<<rows, kSelThreads, 0, s>>>(samp, ld, NBk, q_pos0, row0, cap, rank, kshift, koff, tau, fail);
   return cudaPeekAtLastError();
 }
 
 cudaError_t launch_select_candidates(const DeviceInfo* di, const uint2* cand, const int* cnt, int cap, int Tq, int NBk,
                                      long long q_pos0, int b, int row0, int rows, int k, int32_t* idx, int* fail,
                                      cudaStream_t s) {
+  (void)di;
   if (rows <= 0) return cudaSuccess;
-  static std::once_flag once[64];
-  std::call_once(once[di->device & 63], [] {
-    cudaFuncSetAttribute(cand_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelSmemMax);
-  });
-  const int per_warp = (cap + kSelBins) * 4;
-  const int warps = std::max(1, std::min(kSelWarps, kSelSmemMax / per_warp));
-  if (per_warp > kSelSmemMax) return cudaErrorInvalidValue;
-  cand_select_kernel<<<(rows + warps - 1) / warps, warps * 32, warps * per_warp, s>>>(cand, cnt, cap, Tq, NBk, q_pos0,
-                                                                                    b, row0, rows, k, idx, fail);
+  // lists of up to 2 * U * kSelThreads entries fit the registers; longer ones are refused (the
+  // caller only plans caps that fit)
+  if (cap <= 2 * 10 * kSelThreads)
+    cand_select_kernel<10><<<rows, kSelThreads, 0, s>>>(cand, cnt, cap, Tq, NBk, q_pos0, b, row0, k, idx, fail);
+  else if (cap <= 2 * 20 * kSelThreads)
+    cand_select_kernel<20><<<rows, kSelThreads, 0, s>>>(cand, cnt, cap, Tq, NBk, q_pos0, b, row0, k, idx, fail);
+  else
+    return cudaErrorInvalidValue;
   return cudaPeekAtLastError();
 }
 

@@ -140,8 +140,8 @@ QSA_API qsa_status_t qsa_index_score(const void* qi, const void* kp, const float
  *     workspace is split in two halves and the top-k of one chunk runs on a per-device internal
  *     stream while the next chunk is scored on `stream`; the internal stream is joined back into
  *     `stream` before the call returns, so the call keeps the usual stream-ordered semantics.
- *   - filtered (prefill with Hi of 4 or 8, chosen automatically from 16384 rows per sequence when
- *     the workspace holds 4096 rows or all of them): the scores are never stored.  Every 16th
+ *   - filtered (prefill with Hi of 4 or 8 and k <= 1024, chosen automatically from 16384 rows per
+ *     sequence when the workspace holds 4096 rows or all of them): the scores are never stored.  Every 16th
  *     pooled block is scored first; per row, a threshold with about 2.5 k (at least 1024) of the
  *     row's scores expected above it is read off these samples; the tensor-core score kernel then
  *     keeps only the scores at or above the threshold, in block order, and the top-k is selected
@@ -243,7 +243,7 @@ QSA_API qsa_status_t qsa_get_device_status(void* stream);
 /*
  * Chooses how qsa_select_topk computes a prefill selection when it is not given scores, for all
  * later calls from this process: path 0 = automatic (default), 1 = materialised scores,
- * 2 = filtered (UNSUPPORTED unless Hi is 4 or 8).  sample_rank > 0 replaces the filtered path's
+ * 2 = filtered (UNSUPPORTED unless Hi is 4 or 8 and k <= 1024).  sample_rank > 0 replaces the filtered path's
  * rank of the threshold among a row's samples (a testing and tuning knob: a small rank makes
  * short lists and a large one overflowing lists, both redone exactly); 0 restores the default.
  * Errors: INVALID_ARGUMENT (path outside 0..2, sample_rank < 0).
