@@ -329,8 +329,9 @@ def decode(q, kcache, vcache, qi, kp, seqlens, *, topk: int, rope_theta: float =
 _copy_streams = {}
 
 
-def _copy_stream(device) -> "torch.cuda.Stream":
-    d = torch.device(device).index
+def _copy_stream(device, which: str = "in") -> "torch.cuda.Stream":
+    """Per-device copy streams: one for host->device, one for device->host (PCIe is full duplex)."""
+    d = (torch.device(device).index, which)
     if d not in _copy_streams:
         _copy_streams[d] = torch.cuda.Stream(device=device)
     return _copy_streams[d]
@@ -338,21 +339,24 @@ def _copy_stream(device) -> "torch.cuda.Stream":
 
 def prefill_host(q, k, v, qi, ki, *, topk: int, device="cuda", out=None, q_pos0: int = 0, rope_theta: float = 0.0,
                  head_w=None, mode: int = QSA_SCORE_RELU_SUM, scale: float | None = None, workspace=None,
-                 device_buffers: dict | None = None):
+                 device_buffers: dict | None = None, chunks: int = 8):
     """The QSA layer for a prefill whose inputs live in (pinned) host memory; returns the output in
-    host memory.  Transfers overlap the kernels: ki and qi are copied first, pooling and block
-    selection run while q, k and v are copied on a second stream, and the attention runs in two
-    halves of the query rows so that the first half's output is copied back while the second half
-    is computed.  ``device_buffers`` (name -> device tensor) lets a caller reuse device memory.
+    host memory.  Transfers overlap the kernels.  ki and qi are copied first and the pooling and
+    block selection of all rows run while q, k and v follow in ``chunks`` causal row chunks on a
+    copy stream: chunk c's attention needs only its own query rows and the keys and values of the
+    positions before its end, so it starts as soon as that chunk has arrived, and its output goes
+    back on a second copy stream while the next chunk is computed.  ``device_buffers`` (name ->
+    device tensor) lets a caller reuse device memory.
     Returns dict(out=host tensor, lse=device tensor, idx=device tensor)."""
     dev = torch.device(device)
     main = torch.cuda.current_stream(dev)
-    side = _copy_stream(dev)
+    cin, cout = _copy_stream(dev, "in"), _copy_stream(dev, "out")
     bufs = device_buffers if device_buffers is not None else {}
     for name, t in (("q", q), ("k", k), ("v", v), ("qi", qi), ("ki", ki)):
         if name not in bufs:
             bufs[name] = torch.empty(t.shape, dtype=t.dtype, device=dev)
     B, Tq, Hq, D = q.shape
+    Tk = k.shape[1]
     if out is None:
         out = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
     if "out" not in bufs:
@@ -361,28 +365,44 @@ def prefill_host(q, k, v, qi, ki, *, topk: int, device="cuda", out=None, q_pos0:
         bufs["lse"] = torch.empty(B, Tq, Hq, dtype=torch.float32, device=dev)
     if "kp" not in bufs:
         bufs["kp"] = torch.empty(ki.shape[0], ki.shape[1] // 4, ki.shape[2], dtype=ki.dtype, device=dev)
-    bufs["ki"].copy_(ki, non_blocking=True)
-    bufs["qi"].copy_(qi, non_blocking=True)
-    side.wait_stream(main)
-    with torch.cuda.stream(side):
-        for name, t in (("k", k), ("v", v), ("q", q)):
-            bufs[name].copy_(t, non_blocking=True)
+    # row chunks (one sequence only: the rows of a chunk are then contiguous in every tensor)
+    n = max(1, min(chunks, Tq)) if B == 1 else 1
+    bounds = [(Tq * c) // n for c in range(n + 1)]
+    cin.wait_stream(main)   # the device buffers may still be read by earlier work on `main`
+    with torch.cuda.stream(cin):
+        bufs["ki"].copy_(ki, non_blocking=True)
+        bufs["qi"].copy_(qi, non_blocking=True)
+        sel_ready = torch.cuda.Event()
+        sel_ready.record(cin)
+        arrived = []
+        kv_done = 0   # key/value positions already sent
+        for c in range(n):
+            lo, hi = bounds[c], bounds[c + 1]
+            kv_end = Tk if c == n - 1 else min(Tk, q_pos0 + hi)   # keys a query of the chunk can see
+            if kv_end > kv_done:
+                bufs["k"][:, kv_done:kv_end].copy_(k[:, kv_done:kv_end], non_blocking=True)
+                bufs["v"][:, kv_done:kv_end].copy_(v[:, kv_done:kv_end], non_blocking=True)
+                kv_done = kv_end
+            bufs["q"][:, lo:hi].copy_(q[:, lo:hi], non_blocking=True)
+            ev = torch.cuda.Event()
+            ev.record(cin)
+            arrived.append(ev)
+    main.wait_event(sel_ready)
     kp = qsa_pool_block_keys(bufs["ki"], bufs["kp"], rope_theta=rope_theta)
     qr = qsa_rope_index_queries(bufs["qi"], rope_theta=rope_theta, q_pos0=q_pos0) if rope_theta > 0 else bufs["qi"]
     idx = qsa_select_topk(topk, qi=qr, kp=kp, head_w=head_w, q_pos0=q_pos0, mode=mode, workspace=workspace,
                           idx=bufs.get("idx"))
     bufs["idx"] = idx
-    main.wait_stream(side)
-    half = Tq // 2 if (Tq >= 2 and B == 1) else Tq
-    spans = [(0, half), (half, Tq)] if half < Tq else [(0, Tq)]
-    for lo, hi in spans:
-        qpart = bufs["q"][:, lo:hi]
+    for c in range(n):
+        lo, hi = bounds[c], bounds[c + 1]
+        if hi <= lo:
+            continue
+        main.wait_event(arrived[c])
         opart = bufs["out"][:, lo:hi]
-        if B == 1 or (lo == 0 and hi == Tq):
-            qsa_sparse_attn_prefill(qpart, bufs["k"], bufs["v"], idx[:, lo:hi], q_pos0=q_pos0 + lo, scale=scale,
-                                    out=opart, lse=bufs["lse"][:, lo:hi])
-        side.wait_stream(main)
-        with torch.cuda.stream(side):
+        qsa_sparse_attn_prefill(bufs["q"][:, lo:hi], bufs["k"], bufs["v"], idx[:, lo:hi], q_pos0=q_pos0 + lo,
+                                scale=scale, out=opart, lse=bufs["lse"][:, lo:hi])
+        cout.wait_stream(main)
+        with torch.cuda.stream(cout):
             out[:, lo:hi].copy_(opart, non_blocking=True)
-    main.wait_stream(side)
+    main.wait_stream(cout)
     return dict(out=out, lse=bufs["lse"], idx=idx)
