@@ -429,6 +429,28 @@ def run_qsa(args):
                   "roofline": {"bound": "hbm", "achieved": dgbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                                "frac": dgbs / pk["hbm_gbs"], "bytes_per_step": dw["bytes"],
                                "basis": "pooled-key cache read + gathered K/V of the selected tokens + q/o"}}
+        # dense attention of the same new tokens over the whole caches (library SDPA, GQA): the
+        # decode side of the kernel-level comparison
+        if not args.no_dense:
+            try:
+                qd = xd["q"].view(wd.B, wd.Hq, 1, wd.D)
+                kd = xd["k"].transpose(1, 2)   # [B, Hkv, L, D] views of the caches
+                vd = xd["v"].transpose(1, 2)
+                sdpa = torch.nn.functional.scaled_dot_product_attention
+                with torch.cuda.stream(stream):
+                    sdpa(qd, kd, vd, enable_gqa=True)
+                    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    f0.record(stream)
+                    for _ in range(5):
+                        sdpa(qd, kd, vd, enable_gqa=True)
+                    f1.record(stream)
+                torch.cuda.synchronize()
+                dd_ms = f0.elapsed_time(f1) / 5
+                decode["dense_compare"] = {"impl": "torch scaled_dot_product_attention (all cache positions, GQA, bf16)",
+                                           "ms": dd_ms, "qsa_step_ms": dms, "qsa_attention_ms": d_att,
+                                           "speedup_step": dd_ms / dms, "speedup_attention_only": dd_ms / d_att}
+            except Exception as exc:   # library without a kernel for this shape
+                decode["dense_compare"] = {"unavailable": f"{type(exc).__name__}: {exc}"[:200]}
         del xd, kpd, wsd, wsa, idxd, outd, lsed
 
     if rank == 0:

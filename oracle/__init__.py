@@ -65,6 +65,8 @@ def _load():
         lib.qo_bf16_round_f64.argtypes = [P, P, I64]
         lib.qo_pool_block_keys.argtypes = [P, P, I64, I64, I64, I64, D, I64]
         lib.qo_rope_rows.argtypes = [P, P, I64, I64, I64, P, D]
+        lib.qo_pool_block_keys_yarn.argtypes = [P, P, I64, I64, I64, I64, D, I64, D, D, D, D, D]
+        lib.qo_rope_rows_yarn.argtypes = [P, P, I64, I64, I64, P, D, D, D, D, D, D]
         lib.qo_index_scores.argtypes = [P, P, P, I64, I64, I64, I32, P]
         lib.qo_select_topk.argtypes = [P, I64, I64, P, P]
         lib.qo_select_topk.restype = I64
@@ -107,22 +109,37 @@ def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------- the four steps
-def pool_block_keys(ki: np.ndarray, blk: int = 4, rope_theta: float = 0.0, pos0: int = 0) -> np.ndarray:
-    """ki [B, L, Di] bf16 bits -> kp [B, L // blk, Di]."""
+def _yarn_args(yarn):
+    """YaRN parameters (factor, orig_ctx, alpha, beta, mscale); None = plain RoPE."""
+    if not yarn:
+        return (1.0, 0.0, 1.0, 32.0, 0.0)
+    return (float(yarn["factor"]), float(yarn["orig_ctx"]), float(yarn.get("alpha", 1.0)),
+            float(yarn.get("beta", 32.0)), float(yarn.get("mscale", 0.0)))
+
+
+def pool_block_keys(ki: np.ndarray, blk: int = 4, rope_theta: float = 0.0, pos0: int = 0, yarn=None) -> np.ndarray:
+    """ki [B, L, Di] bf16 bits -> kp [B, L // blk, Di]; `yarn` = dict(factor, orig_ctx[, alpha, beta,
+    mscale]) scales the rotary frequencies when RoPE is on."""
     ki = _u16(ki)
     B, L, Di = ki.shape
     kp = np.empty((B, L // blk, Di), dtype=np.uint16)
-    _load().qo_pool_block_keys(_p(ki), _p(kp), B, L, Di, blk, float(rope_theta), pos0)
+    if yarn:
+        _load().qo_pool_block_keys_yarn(_p(ki), _p(kp), B, L, Di, blk, float(rope_theta), pos0, *_yarn_args(yarn))
+    else:
+        _load().qo_pool_block_keys(_p(ki), _p(kp), B, L, Di, blk, float(rope_theta), pos0)
     return kp
 
 
-def rope_rows(x: np.ndarray, pos: np.ndarray, theta: float) -> np.ndarray:
-    """x [rows, H, Di] bf16 bits rotated at pos [rows]."""
+def rope_rows(x: np.ndarray, pos: np.ndarray, theta: float, yarn=None) -> np.ndarray:
+    """x [rows, H, Di] bf16 bits rotated at pos [rows] (YaRN-scaled with `yarn`)."""
     x = _u16(x)
     rows, H, Di = x.shape
     pos = np.ascontiguousarray(pos, dtype=np.int64)
     y = np.empty_like(x)
-    _load().qo_rope_rows(_p(x), _p(y), rows, H, Di, _p(pos), float(theta))
+    if yarn:
+        _load().qo_rope_rows_yarn(_p(x), _p(y), rows, H, Di, _p(pos), float(theta), *_yarn_args(yarn))
+    else:
+        _load().qo_rope_rows(_p(x), _p(y), rows, H, Di, _p(pos), float(theta))
     return y
 
 

@@ -86,14 +86,45 @@ uint16_t bf16_from_double(double x) {
   return sign | static_cast<uint16_t>(bits >> 16);
 }
 
+// YaRN context extension of the rotary frequencies (B. Peng, J. Quesnelle, H. Fan, E. Shippole,
+// "YaRN: Efficient Context Window Extension of Large Language Models", 2023, sections 3.2 and 3.4;
+// the pages name YaRN for the 1M-token context but give no parameters, so they are the caller's).
+// For a pair with base frequency f (radians per position) the wavelength is 2 pi / f and
+// r = orig_ctx * f / (2 pi) is the number of rotations it makes over the original context.  With
+// the ramp g = clamp((r - alpha) / (beta - alpha), 0, 1) the frequency becomes
+//   f' = (1 - g) * f / factor + g * f
+// (pairs that rotate fewer than alpha times are interpolated by the factor, those that rotate more
+// than beta times keep their frequency), and the rotated pair is scaled by mscale (the paper's
+// attention temperature, 0.1 ln(factor) + 1 unless given).  factor <= 1 is plain RoPE.
+struct Yarn {
+  double factor = 1.0, orig_ctx = 0.0, alpha = 1.0, beta = 32.0, mscale = 0.0;
+};
+
+double yarn_freq(double f, const Yarn& y) {
+  if (y.factor <= 1.0) return f;
+  const double kTwoPi = 6.283185307179586476925286766559;
+  const double r = y.orig_ctx * f / kTwoPi;
+  double g = (r - y.alpha) / (y.beta - y.alpha);
+  g = std::min(1.0, std::max(0.0, g));
+  if (QO_MUTANT == 12) g = 1.0 - g;
+  return (1.0 - g) * f / y.factor + g * f;
+}
+
+double yarn_mscale(const Yarn& y) {
+  if (y.factor <= 1.0) return 1.0;
+  return y.mscale > 0.0 ? y.mscale : 0.1 * std::log(y.factor) + 1.0;
+}
+
 // Half-split rotation of one (x1, x2) pair at position pos with frequency index i of Di/2.
 void rope_pair(double x1, double x2, double pos, int64_t i, int64_t Di, double theta,
-               double* y1, double* y2) {
+               double* y1, double* y2, const Yarn& yarn = Yarn()) {
   double inv_freq = std::pow(theta, -2.0 * static_cast<double>(i) / static_cast<double>(Di));
+  inv_freq = yarn_freq(inv_freq, yarn);
   double ang = pos * inv_freq;
   double c = std::cos(ang), s = std::sin(ang);
-  *y1 = QO_MUTANT == 7 ? x1 * c + x2 * s : x1 * c - x2 * s;
-  *y2 = x2 * c + x1 * s;
+  const double m = yarn_mscale(yarn);
+  *y1 = m * (QO_MUTANT == 7 ? x1 * c + x2 * s : x1 * c - x2 * s);
+  *y2 = m * (x2 * c + x1 * s);
 }
 
 // One indexer score row: s[b] for b < nb, the candidates of the query whose (already rotated)
@@ -222,8 +253,16 @@ void qo_bf16_round_f64(const double* x, uint16_t* y, int64_t n) {
 
 // ki [B][L][Di] -> kp [B][floor(L/blk)][Di]: the mean of each group of blk consecutive keys, then
 // (theta > 0) the half-split rotation at position pos0 + blk*b, then bf16 rounding.
-void qo_pool_block_keys(const uint16_t* ki, uint16_t* kp, int64_t B, int64_t L, int64_t Di,
-                        int64_t blk, double rope_theta, int64_t pos0) {
+void qo_pool_block_keys_yarn(const uint16_t* ki, uint16_t* kp, int64_t B, int64_t L, int64_t Di,
+                             int64_t blk, double rope_theta, int64_t pos0, double yarn_factor,
+                             double yarn_orig_ctx, double yarn_alpha, double yarn_beta,
+                             double yarn_mscale) {
+  Yarn yarn;
+  yarn.factor = yarn_factor;
+  yarn.orig_ctx = yarn_orig_ctx;
+  yarn.alpha = yarn_alpha;
+  yarn.beta = yarn_beta;
+  yarn.mscale = yarn_mscale;
   const int64_t nb = L / blk;
   std::vector<double> m(static_cast<size_t>(Di));
   for (int64_t b = 0; b < B; ++b) {
@@ -238,7 +277,7 @@ void qo_pool_block_keys(const uint16_t* ki, uint16_t* kp, int64_t B, int64_t L, 
         const double pos = static_cast<double>(pos0 + j * blk + (QO_MUTANT == 10 ? blk - 1 : 0));
         for (int64_t i = 0; i < Di / 2; ++i) {
           double y1, y2;
-          rope_pair(m[i], m[i + Di / 2], pos, i, Di, rope_theta, &y1, &y2);
+          rope_pair(m[i], m[i + Di / 2], pos, i, Di, rope_theta, &y1, &y2, yarn);
           dst[i] = bf16_from_double(y1);
           dst[i + Di / 2] = bf16_from_double(y2);
         }
@@ -249,9 +288,22 @@ void qo_pool_block_keys(const uint16_t* ki, uint16_t* kp, int64_t B, int64_t L, 
   }
 }
 
-// Rotate rows of indexer queries x [rows][H][Di] at positions pos[rows]; bf16 out.
-void qo_rope_rows(const uint16_t* x, uint16_t* y, int64_t rows, int64_t H, int64_t Di,
-                  const int64_t* pos, double theta) {
+void qo_pool_block_keys(const uint16_t* ki, uint16_t* kp, int64_t B, int64_t L, int64_t Di,
+                        int64_t blk, double rope_theta, int64_t pos0) {
+  qo_pool_block_keys_yarn(ki, kp, B, L, Di, blk, rope_theta, pos0, 1.0, 0.0, 1.0, 32.0, 0.0);
+}
+
+// Rotate rows of indexer queries x [rows][H][Di] at positions pos[rows] (YaRN-scaled when
+// yarn_factor > 1); bf16 out.
+void qo_rope_rows_yarn(const uint16_t* x, uint16_t* y, int64_t rows, int64_t H, int64_t Di,
+                       const int64_t* pos, double theta, double yarn_factor, double yarn_orig_ctx,
+                       double yarn_alpha, double yarn_beta, double yarn_mscale) {
+  Yarn yarn;
+  yarn.factor = yarn_factor;
+  yarn.orig_ctx = yarn_orig_ctx;
+  yarn.alpha = yarn_alpha;
+  yarn.beta = yarn_beta;
+  yarn.mscale = yarn_mscale;
   for (int64_t r = 0; r < rows; ++r) {
     for (int64_t h = 0; h < H; ++h) {
       const uint16_t* src = x + (r * H + h) * Di;
@@ -259,12 +311,17 @@ void qo_rope_rows(const uint16_t* x, uint16_t* y, int64_t rows, int64_t H, int64
       for (int64_t i = 0; i < Di / 2; ++i) {
         double y1, y2;
         rope_pair(bf16_to_double(src[i]), bf16_to_double(src[i + Di / 2]),
-                  static_cast<double>(pos[r]), i, Di, theta, &y1, &y2);
+                  static_cast<double>(pos[r]), i, Di, theta, &y1, &y2, yarn);
         dst[i] = bf16_from_double(y1);
         dst[i + Di / 2] = bf16_from_double(y2);
       }
     }
   }
+}
+
+void qo_rope_rows(const uint16_t* x, uint16_t* y, int64_t rows, int64_t H, int64_t Di,
+                  const int64_t* pos, double theta) {
+  qo_rope_rows_yarn(x, y, rows, H, Di, pos, theta, 1.0, 0.0, 1.0, 32.0, 0.0);
 }
 
 void qo_index_scores(const uint16_t* qi_row, const uint16_t* kp, const float* head_w, int64_t Hi,

@@ -21,6 +21,7 @@ MUTANTS = {
     9: "indexer query operand transposed",
     10: "pooled key rotated at the block end",
     11: "bf16 rounding truncates",
+    12: "YaRN ramp reversed (fast pairs interpolated, slow pairs kept)",
 }
 
 

@@ -147,6 +147,101 @@ def test_rope_keys_rotate_at_block_start_complex_form():
     assert np.all(np.abs(kp - expect) <= ulp_bf16(expect) / 2 * (1 + 1e-9) + 1e-30)
 
 
+# ---- YaRN-scaled RoPE ("YaRN: Efficient Context Window Extension of Large Language Models",
+# Peng et al. 2023, sections 3.2 and 3.4).  Pinned by the properties that define it rather than by
+# its formula: pairs that turn many times over the original context keep their frequency, pairs
+# that turn less than once are position-interpolated by the factor, the ramp in between is
+# monotone, the magnitude factor scales norms, and relative-position dependence survives.
+YARN = dict(factor=8.0, orig_ctx=4096, alpha=1.0, beta=32.0, mscale=1.0)
+
+
+def _yarn_pair_classes(Di=64, theta=10000.0, orig_ctx=4096):
+    f = theta ** (-2.0 * np.arange(Di // 2) / Di)
+    turns = orig_ctx * f / (2 * math.pi)
+    return np.nonzero(turns > 32.0)[0], np.nonzero(turns < 1.0)[0]
+
+
+def test_yarn_factor_one_is_plain_rope():
+    rng = np.random.default_rng(31)
+    x = rand_bits(rng, (6, 2, 64))
+    pos = np.array([0, 3, 77, 4096, 100000, 1048575])
+    assert np.array_equal(O.rope_rows(x, pos, 10000.0, yarn=dict(factor=1.0, orig_ctx=4096)),
+                          O.rope_rows(x, pos, 10000.0))
+    ki = rand_bits(rng, (1, 64, 64), 1 / 8)
+    assert np.array_equal(O.pool_block_keys(ki, rope_theta=10000.0, pos0=40, yarn=dict(factor=1.0, orig_ctx=4096)),
+                          O.pool_block_keys(ki, rope_theta=10000.0, pos0=40))
+
+
+def test_yarn_keeps_fast_pairs_and_interpolates_slow_pairs():
+    """A fast pair rotates exactly as plain RoPE; a slow pair at position p rotates as plain RoPE at
+    position p / factor (position interpolation), bit for bit."""
+    rng = np.random.default_rng(32)
+    Di, theta = 64, 10000.0
+    fast, slow = _yarn_pair_classes(Di, theta, YARN["orig_ctx"])
+    assert len(fast) >= 8 and len(slow) >= 6
+    x = rand_bits(rng, (4, 3, Di))
+    pos = np.array([8, 4096, 65536, 1048568])          # multiples of the factor
+    y = O.rope_rows(x, pos, theta, yarn=YARN)
+    plain = O.rope_rows(x, pos, theta)
+    interp = O.rope_rows(x, pos // 8, theta)
+    for i in fast:
+        assert np.array_equal(y[..., i], plain[..., i]) and np.array_equal(y[..., i + Di // 2], plain[..., i + Di // 2])
+    for i in slow:
+        assert np.array_equal(y[..., i], interp[..., i]) and np.array_equal(y[..., i + Di // 2], interp[..., i + Di // 2])
+
+
+def test_yarn_ramp_is_monotone_between_interpolation_and_extrapolation():
+    """The angle per position of each pair, read off a rotated basis vector at a small position,
+    is squeezed between the interpolated and the plain frequency and their ratio rises with the
+    pair's frequency."""
+    Di, theta, p = 64, 10000.0, 1     # angles below pi: no wrap-around
+    f = theta ** (-2.0 * np.arange(Di // 2) / Di)
+    ratios = []
+    for i in range(Di // 2):
+        x = np.zeros((1, 1, Di), dtype=np.uint16)
+        x[0, 0, i] = 0x3F80
+        y = f64(O.rope_rows(x, np.array([p]), theta, yarn=YARN))[0, 0]
+        ang = math.atan2(y[i + Di // 2], y[i]) / p
+        ratios.append(ang / f[i])
+    ratios = np.array(ratios)
+    assert np.all(ratios >= 1 / 8 - 1e-2) and np.all(ratios <= 1 + 1e-2)
+    assert np.all(np.diff(ratios[::-1]) >= -1e-2)    # from the slowest pair up: non-decreasing
+    assert ratios[0] > 0.99 and ratios[-1] < 0.13
+
+
+def test_yarn_magnitude_factor_scales_norms_and_keeps_relative_positions():
+    rng = np.random.default_rng(33)
+    q = rand_bits(rng, (1, 1, 64))
+    k = rand_bits(rng, (1, 1, 64))
+    y = dict(YARN, mscale=1.5)
+    r = f64(O.rope_rows(q, np.array([12345]), 10000.0, yarn=y))
+    assert abs(np.linalg.norm(r) - 1.5 * np.linalg.norm(f64(q))) <= 1e-2 * np.linalg.norm(f64(q))
+    dots = []
+    for shift in [0, 96, 40000]:
+        a = f64(O.rope_rows(q, np.array([50 + shift]), 10000.0, yarn=YARN)).ravel()
+        b = f64(O.rope_rows(k, np.array([18 + shift]), 10000.0, yarn=YARN)).ravel()
+        dots.append(a @ b)
+    assert np.ptp(dots) <= 2e-2 * np.linalg.norm(f64(q)) * np.linalg.norm(f64(k))
+
+
+def test_yarn_pooled_keys_match_yarn_rotated_means():
+    """Pooling with YaRN is the YaRN rotation of the block means at the block start."""
+    rng = np.random.default_rng(34)
+    ki = rand_bits(rng, (1, 48, 64), 1 / 8)
+    kp = O.pool_block_keys(ki, rope_theta=10000.0, pos0=800, yarn=YARN)
+    means = O.pool_block_keys(ki)                          # the means, rounded once
+    # rotate the exact means: compare in value with one bf16 rounding of slack on each side
+    m = f64(ki).reshape(12, 4, 64).mean(axis=1)
+    rot = f64(O.rope_rows(O.bf16_round(m)[:, None, :], 800 + 4 * np.arange(12), 10000.0, yarn=YARN))[:, 0]
+    got = f64(kp)[0]
+    # two roundings on the right (the mean, then the rotated value) against one on the left: the
+    # mean's rounding error moves within its rotation pair, so bound by the pair's magnitude
+    norm = np.hypot(m[:, :32], m[:, 32:])
+    tol = np.concatenate([1.5 * ulp_bf16(norm)] * 2, axis=1)
+    assert np.all(np.abs(got - rot) <= tol + 1e-30)
+    assert means.shape == kp.shape
+
+
 def test_rope_preserves_norm_and_depends_on_relative_position():
     rng = np.random.default_rng(6)
     Di, theta = 64, 10000.0
