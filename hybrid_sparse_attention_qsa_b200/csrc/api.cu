@@ -1,5 +1,6 @@
 // The C ABI (include/qsa.h): argument checks on the host, then launches on the caller's stream.
 #include <algorithm>
+#include <cmath>
 #include <atomic>
 #include <cstdint>
 #include <mutex>
@@ -138,10 +139,31 @@ qsa_status_t qsa_set_select_options(int path, int sample_rank) {
 
 void qsa_set_wait_timeout_ns(uint64_t ns) { g_wait_ns.store(ns ? ns : kDefaultWaitNs); }
 
-qsa_status_t qsa_pool_block_keys(const void* ki, void* kp, int B, int L, int Di, int blk, float rope_theta,
-                                 int64_t pos0, int64_t ki_batch_stride, int64_t kp_batch_stride, void* stream) {
+// Checks and resolves the rotary parameters (NULL or theta <= 0: no rotation).
+static qsa_status_t resolve_rope(const qsa_rope_params_t* in, RopeParams* out) {
+  *out = RopeParams{0.0, 1.0, 0.0, 1.0, 32.0, 1.0};
+  if (in == nullptr || !(in->theta > 0.0)) return QSA_OK;
+  out->theta = in->theta;
+  if (in->yarn_factor > 1.0) {
+    if (!(in->yarn_orig_ctx > 0.0) || !(in->yarn_beta > in->yarn_alpha)) return QSA_ERR_INVALID_ARGUMENT;
+    out->factor = in->yarn_factor;
+    out->orig_ctx = in->yarn_orig_ctx;
+    out->alpha = in->yarn_alpha;
+    out->beta = in->yarn_beta;
+    out->mscale = in->yarn_mscale > 0.0 ? in->yarn_mscale : 0.1 * std::log(in->yarn_factor) + 1.0;
+  } else if (!(in->yarn_factor >= 0.0)) {
+    return QSA_ERR_INVALID_ARGUMENT;
+  }
+  return QSA_OK;
+}
+
+qsa_status_t qsa_pool_block_keys_rope(const void* ki, void* kp, int B, int L, int Di, int blk,
+                                      const qsa_rope_params_t* rope, int64_t pos0, int64_t ki_batch_stride,
+                                      int64_t kp_batch_stride, void* stream) {
   if (B < 0 || L < 0 || Di < 2 || Di > 256 || (Di & 1) || pos0 < 0) return QSA_ERR_INVALID_ARGUMENT;
   if (ki_batch_stride < 0 || kp_batch_stride < 0) return QSA_ERR_INVALID_ARGUMENT;
+  RopeParams rp;
+  if (resolve_rope(rope, &rp) != QSA_OK) return QSA_ERR_INVALID_ARGUMENT;
   const long long kis = ki_batch_stride ? ki_batch_stride : static_cast<long long>(L) * Di;
   const long long kps = kp_batch_stride ? kp_batch_stride : static_cast<long long>(L / 4) * Di;
   if (kis < static_cast<long long>(L) * Di || kps < static_cast<long long>(L / 4) * Di) return QSA_ERR_INVALID_ARGUMENT;
@@ -149,19 +171,32 @@ qsa_status_t qsa_pool_block_keys(const void* ki, void* kp, int B, int L, int Di,
   if (static_cast<long long>(B) * (L / blk) == 0) return QSA_OK;
   if (!ok_ptr(ki) || !ok_ptr(kp)) return QSA_ERR_INVALID_ARGUMENT;
   if (!device_info()) return QSA_ERR_CUDA;
-  return cuda_status(launch_pool(ki, kp, B, L, Di, blk, rope_theta > 0.f ? static_cast<double>(rope_theta) : 0.0,
-                                 pos0, kis, kps, S(stream)));
+  return cuda_status(launch_pool(ki, kp, B, L, Di, blk, rp, pos0, kis, kps, S(stream)));
 }
 
-qsa_status_t qsa_rope_index_queries(const void* qi, void* qi_out, int B, int Tq, int Hi, int Di, int64_t q_pos0,
-                                    const int32_t* seqlens, float rope_theta, void* stream) {
-  if (B < 0 || Tq < 0 || Hi < 1 || Di < 2 || Di > 256 || (Di & 1) || q_pos0 < 0 || !(rope_theta > 0.f))
-    return QSA_ERR_INVALID_ARGUMENT;
+qsa_status_t qsa_pool_block_keys(const void* ki, void* kp, int B, int L, int Di, int blk, float rope_theta,
+                                 int64_t pos0, int64_t ki_batch_stride, int64_t kp_batch_stride, void* stream) {
+  const qsa_rope_params_t rope{rope_theta > 0.f ? static_cast<double>(rope_theta) : 0.0, 1.0, 0.0, 1.0, 32.0, 0.0};
+  return qsa_pool_block_keys_rope(ki, kp, B, L, Di, blk, &rope, pos0, ki_batch_stride, kp_batch_stride, stream);
+}
+
+qsa_status_t qsa_rope_index_queries_rope(const void* qi, void* qi_out, int B, int Tq, int Hi, int Di, int64_t q_pos0,
+                                         const int32_t* seqlens, const qsa_rope_params_t* rope, void* stream) {
+  RopeParams rp;
+  if (B < 0 || Tq < 0 || Hi < 1 || Di < 2 || Di > 256 || (Di & 1) || q_pos0 < 0) return QSA_ERR_INVALID_ARGUMENT;
+  if (resolve_rope(rope, &rp) != QSA_OK || !(rp.theta > 0.0)) return QSA_ERR_INVALID_ARGUMENT;
   if (seqlens && Tq != 1) return QSA_ERR_INVALID_ARGUMENT;
   if (static_cast<long long>(B) * Tq == 0) return QSA_OK;
   if (!ok_ptr(qi) || !ok_ptr(qi_out)) return QSA_ERR_INVALID_ARGUMENT;
   if (!device_info()) return QSA_ERR_CUDA;
-  return cuda_status(launch_rope_queries(qi, qi_out, B, Tq, Hi, Di, q_pos0, seqlens, rope_theta, S(stream)));
+  return cuda_status(launch_rope_queries(qi, qi_out, B, Tq, Hi, Di, q_pos0, seqlens, rp, S(stream)));
+}
+
+qsa_status_t qsa_rope_index_queries(const void* qi, void* qi_out, int B, int Tq, int Hi, int Di, int64_t q_pos0,
+                                    const int32_t* seqlens, float rope_theta, void* stream) {
+  if (!(rope_theta > 0.f)) return QSA_ERR_INVALID_ARGUMENT;
+  const qsa_rope_params_t rope{static_cast<double>(rope_theta), 1.0, 0.0, 1.0, 32.0, 0.0};
+  return qsa_rope_index_queries_rope(qi, qi_out, B, Tq, Hi, Di, q_pos0, seqlens, &rope, stream);
 }
 
 static qsa_status_t check_score_args(const void* qi, const void* kp, const int32_t* seqlens, int B, int Tq, int NBk,

@@ -19,10 +19,16 @@ struct DeviceInfo {
 const DeviceInfo* device_info();
 KernelCtl kernel_ctl(const DeviceInfo* di);
 
-cudaError_t launch_pool(const void* ki, void* kp, int B, int L, int Di, int blk, double theta, long long pos0,
+// Rotary parameters of the indexer (theta <= 0: no rotation); factor > 1 turns on YaRN scaling
+// with the given original context, ramp bounds and magnitude factor (already resolved).
+struct RopeParams {
+  double theta, factor, orig_ctx, alpha, beta, mscale;
+};
+
+cudaError_t launch_pool(const void* ki, void* kp, int B, int L, int Di, int blk, const RopeParams& rp, long long pos0,
                         long long ki_bs, long long kp_bs, cudaStream_t s);
 cudaError_t launch_rope_queries(const void* qi, void* qo, int B, int Tq, int Hi, int Di, long long q_pos0,
-                                const int32_t* seqlens, double theta, cudaStream_t s);
+                                const int32_t* seqlens, const RopeParams& rp, cudaStream_t s);
 
 // Prefill scores for query rows [row0, row0 + rows) of batches [b0, b0 + nb) into
 // scores + (b - b0) * batch_stride + (t - row0) * ld.

@@ -3,7 +3,7 @@
 // "Qwen3.8-Flash-Next architecture" (flozi.net), "Der Weg eines Tokens durch das Modell", item 2:
 // groups of four indexer keys are averaged into one micro-block key, and the rotary embedding is
 // applied after the averaging so that keys of different positions are not mixed at different
-// rotation phases.
+// rotation phases.  For contexts beyond the trained one the frequencies can be YaRN-scaled.
 //
 // Bandwidth-bound and tiny next to the rest of the path (at 131072 tokens: 16.8 MB read, 4.2 MB
 // written).  One warp per output row; lane i owns the rotation pair (i, i + Di/2), so the pair
@@ -18,17 +18,29 @@ __device__ __forceinline__ double bf16_to_f64(uint16_t h) {
   return static_cast<double>(__uint_as_float(static_cast<uint32_t>(h) << 16));
 }
 
-__device__ __forceinline__ void rope_rotate(double x1, double x2, double pos, int i, int Di, double theta,
+// YaRN context extension of the rotary frequencies ("YaRN: Efficient Context Window Extension of
+// Large Language Models", Peng et al. 2023, sections 3.2 and 3.4): with r = orig_ctx * f / 2 pi
+// rotations of a pair over the original context and g = clamp((r - alpha) / (beta - alpha), 0, 1),
+// the frequency f becomes (1 - g) f / factor + g f, and the rotated pair is scaled by mscale.
+// factor <= 1 leaves plain RoPE.
+__device__ __forceinline__ void rope_rotate(double x1, double x2, double pos, int i, int Di, const RopeParams& rp,
                                             double* y1, double* y2) {
-  const double inv_freq = pow(theta, -2.0 * static_cast<double>(i) / static_cast<double>(Di));
+  double inv_freq = pow(rp.theta, -2.0 * static_cast<double>(i) / static_cast<double>(Di));
+  double m = 1.0;
+  if (rp.factor > 1.0) {
+    const double r = rp.orig_ctx * inv_freq / 6.283185307179586476925286766559;
+    const double g = fmin(1.0, fmax(0.0, (r - rp.alpha) / (rp.beta - rp.alpha)));
+    inv_freq = (1.0 - g) * inv_freq / rp.factor + g * inv_freq;
+    m = rp.mscale;
+  }
   double s, c;
   sincos(pos * inv_freq, &s, &c);
-  *y1 = x1 * c - x2 * s;
-  *y2 = x2 * c + x1 * s;
+  *y1 = m * (x1 * c - x2 * s);
+  *y2 = m * (x2 * c + x1 * s);
 }
 
 __global__ void __launch_bounds__(256) pool_kernel(const uint16_t* __restrict__ ki, uint16_t* __restrict__ kp,
-                                                   int B, int L, int Di, int blk, double theta, long long pos0,
+                                                   int B, int L, int Di, int blk, RopeParams rp, long long pos0,
                                                    long long ki_bs, long long kp_bs) {
   const int nb = L / blk;
   const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
@@ -46,9 +58,9 @@ __global__ void __launch_bounds__(256) pool_kernel(const uint16_t* __restrict__ 
     }
     m1 /= static_cast<double>(blk);
     m2 /= static_cast<double>(blk);
-    if (theta > 0.0) {
+    if (rp.theta > 0.0) {
       double y1, y2;
-      rope_rotate(m1, m2, static_cast<double>(pos0 + j * blk), i, Di, theta, &y1, &y2);
+      rope_rotate(m1, m2, static_cast<double>(pos0 + j * blk), i, Di, rp, &y1, &y2);
       m1 = y1;
       m2 = y2;
     }
@@ -59,7 +71,7 @@ __global__ void __launch_bounds__(256) pool_kernel(const uint16_t* __restrict__ 
 
 __global__ void __launch_bounds__(256) rope_q_kernel(const uint16_t* qi, uint16_t* qo,
                                                      int B, int Tq, int Hi, int Di, long long q_pos0,
-                                                     const int32_t* __restrict__ seqlens, double theta) {
+                                                     const int32_t* __restrict__ seqlens, RopeParams rp) {
   const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);   // (b, t, h)
   if (row >= static_cast<long long>(B) * Tq * Hi) return;
   const int lane = threadIdx.x & 31;
@@ -70,7 +82,7 @@ __global__ void __launch_bounds__(256) rope_q_kernel(const uint16_t* qi, uint16_
   // Each rotation pair is read and written by one thread only, so qo may alias qi.
   for (int i = lane; i < half; i += 32) {
     double y1, y2;
-    rope_rotate(bf16_to_f64(qi[row * Di + i]), bf16_to_f64(qi[row * Di + i + half]), pos, i, Di, theta, &y1, &y2);
+    rope_rotate(bf16_to_f64(qi[row * Di + i]), bf16_to_f64(qi[row * Di + i + half]), pos, i, Di, rp, &y1, &y2);
     qo[row * Di + i] = bf16_bits_rne_f64(y1);
     qo[row * Di + i + half] = bf16_bits_rne_f64(y2);
   }
@@ -78,23 +90,23 @@ __global__ void __launch_bounds__(256) rope_q_kernel(const uint16_t* qi, uint16_
 
 }  // namespace
 
-cudaError_t launch_pool(const void* ki, void* kp, int B, int L, int Di, int blk, double theta, long long pos0,
+cudaError_t launch_pool(const void* ki, void* kp, int B, int L, int Di, int blk, const RopeParams& rp, long long pos0,
                         long long ki_bs, long long kp_bs, cudaStream_t s) {
   const long long rows = static_cast<long long>(B) * (L / blk);
   if (rows == 0) return cudaSuccess;
   const unsigned grid = static_cast<unsigned>((rows + 7) / 8);
   pool_kernel<<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(ki), static_cast<uint16_t*>(kp), B, L, Di, blk,
-                                   theta, pos0, ki_bs, kp_bs);
+                                   rp, pos0, ki_bs, kp_bs);
   return cudaPeekAtLastError();
 }
 
 cudaError_t launch_rope_queries(const void* qi, void* qo, int B, int Tq, int Hi, int Di, long long q_pos0,
-                                const int32_t* seqlens, double theta, cudaStream_t s) {
+                                const int32_t* seqlens, const RopeParams& rp, cudaStream_t s) {
   const long long rows = static_cast<long long>(B) * Tq * Hi;
   if (rows == 0) return cudaSuccess;
   const unsigned grid = static_cast<unsigned>((rows + 7) / 8);
   rope_q_kernel<<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(qi), static_cast<uint16_t*>(qo), B, Tq, Hi, Di,
-                                     q_pos0, seqlens, theta);
+                                     q_pos0, seqlens, rp);
   return cudaPeekAtLastError();
 }
 

@@ -223,17 +223,19 @@ __global__ void __launch_bounds__(kSelThreads) cand_select_kernel(const uint2* _
   // list starts 16-byte aligned)
   const uint4* src = reinterpret_cast<const uint4*>(cand + static_cast<long long>(L) * cap);
   const int c2 = (c + 1) >> 1;
+  const int rounds = (c + 2 * kSelThreads - 1) / (2 * kSelThreads);   // rounds holding entries
   uint4 v[U];
 #pragma unroll
   for (int u = 0; u < U; ++u) {
     const int j = tid + u * kSelThreads;
-    v[u] = j < c2 ? __ldcs(src + j) : make_uint4(0u, 0u, 0u, 0u);
+    v[u] = (u < rounds && j < c2) ? __ldcs(src + j) : make_uint4(0u, 0u, 0u, 0u);
   }
   // entry 2j is (v.x, v.y), entry 2j + 1 is (v.z, v.w): fp32 score bits, turned into
   // order-preserving keys here; invalid entries get key 0 (below any score)
   uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
 #pragma unroll
   for (int u = 0; u < U; ++u) {
+    if (u >= rounds) break;   // uniform
     const int j = tid + u * kSelThreads;
     v[u].x = score_key(__uint_as_float(v[u].x) + 0.0f);
     v[u].z = score_key(__uint_as_float(v[u].z) + 0.0f);
@@ -264,6 +266,7 @@ __global__ void __launch_bounds__(kSelThreads) cand_select_kernel(const uint2* _
     __syncthreads();
 #pragma unroll
     for (int u = 0; u < U; ++u) {
+      if (u >= rounds) break;   // uniform
       const int j = tid + u * kSelThreads;
       if (2 * j < c) atomicAdd(&hist[(v[u].x >> sh) & (kSelBins - 1)], 1u);
       if (2 * j + 1 < c) atomicAdd(&hist[(v[u].z >> sh) & (kSelBins - 1)], 1u);
@@ -285,6 +288,7 @@ __global__ void __launch_bounds__(kSelThreads) cand_select_kernel(const uint2* _
       uint32_t* buf = hist;
 #pragma unroll
       for (int u = 0; u < U; ++u) {
+        if (u >= rounds) break;   // uniform
         const int j = tid + u * kSelThreads;
         if (2 * j < c && ((v[u].x >> sh) & (kSelBins - 1)) == B) buf[atomicAdd(&sel[2], 1u)] = v[u].x;
         if (2 * j + 1 < c && ((v[u].z >> sh) & (kSelBins - 1)) == B) buf[atomicAdd(&sel[2], 1u)] = v[u].z;
@@ -323,13 +327,14 @@ __global__ void __launch_bounds__(kSelThreads) cand_select_kernel(const uint2* _
   uint32_t pk[U];   // per round: (entries > K*) << 16 | (entries == K*) among this thread's two
 #pragma unroll
   for (int u = 0; u < U; ++u) {
+    pk[u] = 0;
+    if (u >= rounds) continue;   // uniform
     const int j = tid + u * kSelThreads;
     const bool ok0 = 2 * j < c, ok1 = 2 * j + 1 < c;
     const bool gt0 = ok0 && (keep_all || v[u].x > kth), gt1 = ok1 && (keep_all || v[u].z > kth);
     const bool eq0 = ok0 && !keep_all && v[u].x == kth, eq1 = ok1 && !keep_all && v[u].z == kth;
     pk[u] = ((static_cast<uint32_t>(gt0) + gt1) << 16) | (static_cast<uint32_t>(eq0) + eq1);
   }
-  const int rounds = (c + 2 * kSelThreads - 1) / (2 * kSelThreads);   // rounds holding entries
   uint32_t incl[U];
 #pragma unroll
   for (int u = 0; u < U; ++u) {

@@ -35,7 +35,9 @@ SIGNATURES = {
     "qsa_status_string": (ctypes.c_char_p, [_I]),
     "qsa_abi_version": (_I, []),
     "qsa_pool_block_keys": (_I, [_P, _P, _I, _I, _I, _I, _F, _I64, _I64, _I64, _P]),
+    "qsa_pool_block_keys_rope": (_I, [_P, _P, _I, _I, _I, _I, _P, _I64, _I64, _I64, _P]),
     "qsa_rope_index_queries": (_I, [_P, _P, _I, _I, _I, _I, _I64, _P, _F, _P]),
+    "qsa_rope_index_queries_rope": (_I, [_P, _P, _I, _I, _I, _I, _I64, _P, _P, _P]),
     "qsa_index_score": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I64, _I, _P, _I64, _P]),
     "qsa_select_topk": (_I, [_P, _I64, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I64, _I, _I, _P, _P, _SZ, _P]),
     "qsa_sparse_attn_prefill": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I64, _F, _P, _P, _P]),
@@ -110,10 +112,24 @@ def _batch_view_ok(t: torch.Tensor) -> bool:
     return t.dim() == 3 and t.stride(2) == 1 and t.stride(1) == t.shape[2]
 
 
+class RopeParams(ctypes.Structure):
+    """qsa_rope_params_t: the indexer's rotary base and optional YaRN scaling."""
+    _fields_ = [("theta", ctypes.c_double), ("yarn_factor", ctypes.c_double), ("yarn_orig_ctx", ctypes.c_double),
+                ("yarn_alpha", ctypes.c_double), ("yarn_beta", ctypes.c_double), ("yarn_mscale", ctypes.c_double)]
+
+
+def _rope_params(theta: float, yarn: dict | None) -> RopeParams:
+    """yarn = dict(factor, orig_ctx[, alpha=1, beta=32, mscale=0 (the paper's default)])."""
+    y = yarn or {}
+    return RopeParams(float(theta), float(y.get("factor", 1.0)), float(y.get("orig_ctx", 0.0)),
+                      float(y.get("alpha", 1.0)), float(y.get("beta", 32.0)), float(y.get("mscale", 0.0)))
+
+
 def qsa_pool_block_keys(ki: torch.Tensor, kp: torch.Tensor | None = None, *, blk: int = 4, rope_theta: float = 0.0,
-                        pos0: int = 0) -> torch.Tensor:
+                        pos0: int = 0, yarn: dict | None = None) -> torch.Tensor:
     """ki [B, L, Di] bf16 -> kp [B, L // blk, Di] bf16.  ki and kp may be batch-strided views (for
-    example the newest block of every sequence of a decode cache: ki[:, 4j:4j+4], kp[:, j:j+1])."""
+    example the newest block of every sequence of a decode cache: ki[:, 4j:4j+4], kp[:, j:j+1]).
+    ``yarn`` (dict(factor, orig_ctx[, alpha, beta, mscale])) scales the rotary frequencies."""
     if not ki.is_cuda or ki.dtype != torch.bfloat16 or not _batch_view_ok(ki):
         raise ValueError("ki must be a CUDA bf16 [B, L, Di] tensor with packed rows")
     B, L, Di = ki.shape
@@ -121,13 +137,18 @@ def qsa_pool_block_keys(ki: torch.Tensor, kp: torch.Tensor | None = None, *, blk
         kp = torch.empty(B, L // blk, Di, dtype=torch.bfloat16, device=ki.device)
     if kp.dtype != torch.bfloat16 or not _batch_view_ok(kp) or tuple(kp.shape) != (B, L // blk, Di):
         raise ValueError("kp must be a bf16 [B, L // blk, Di] tensor with packed rows")
+    if yarn:
+        rp = _rope_params(rope_theta, yarn)
+        _check(lib().qsa_pool_block_keys_rope(_ptr(ki), _ptr(kp), B, L, Di, blk, ctypes.byref(rp), pos0, ki.stride(0),
+                                              kp.stride(0), _stream(ki.device)), "qsa_pool_block_keys_rope")
+        return kp
     _check(lib().qsa_pool_block_keys(_ptr(ki), _ptr(kp), B, L, Di, blk, rope_theta, pos0, ki.stride(0), kp.stride(0),
                                      _stream(ki.device)), "qsa_pool_block_keys")
     return kp
 
 
 def qsa_rope_index_queries(qi: torch.Tensor, qi_out: torch.Tensor | None = None, *, rope_theta: float, q_pos0: int = 0,
-                           seqlens: torch.Tensor | None = None) -> torch.Tensor:
+                           seqlens: torch.Tensor | None = None, yarn: dict | None = None) -> torch.Tensor:
     """qi [B, Tq, Hi, Di] (or [B, Hi, Di] with seqlens) rotated at its positions."""
     _need(qi, torch.bfloat16, "qi")
     if seqlens is not None:
@@ -138,6 +159,11 @@ def qsa_rope_index_queries(qi: torch.Tensor, qi_out: torch.Tensor | None = None,
         B, Tq, Hi, Di = qi.shape
     if qi_out is None:
         qi_out = torch.empty_like(qi)
+    if yarn:
+        rp = _rope_params(rope_theta, yarn)
+        _check(lib().qsa_rope_index_queries_rope(_ptr(qi), _ptr(qi_out), B, Tq, Hi, Di, q_pos0, _ptr(seqlens),
+                                                 ctypes.byref(rp), _stream(qi.device)), "qsa_rope_index_queries_rope")
+        return qi_out
     _check(lib().qsa_rope_index_queries(_ptr(qi), _ptr(qi_out), B, Tq, Hi, Di, q_pos0, _ptr(seqlens), rope_theta,
                                         _stream(qi.device)), "qsa_rope_index_queries")
     return qi_out
@@ -305,22 +331,23 @@ def qsa_wait_timeout_selftest(timeout_ns: int, device=None) -> None:
 
 # ---------------------------------------------------------------------------------------- whole path
 def prefill(q, k, v, qi, ki, *, topk: int, q_pos0: int = 0, rope_theta: float = 0.0, head_w=None,
-            mode: int = QSA_SCORE_RELU_SUM, scale: float | None = None, workspace=None, kp=None):
+            mode: int = QSA_SCORE_RELU_SUM, scale: float | None = None, workspace=None, kp=None, yarn=None):
     """The QSA layer for a prefill: pool (+RoPE) -> [RoPE queries] -> score + top-k -> sparse attention.
     Returns dict(out, lse, idx, kp)."""
     if kp is None:
-        kp = qsa_pool_block_keys(ki, rope_theta=rope_theta)
-    qr = qsa_rope_index_queries(qi, rope_theta=rope_theta, q_pos0=q_pos0) if rope_theta > 0 else qi
+        kp = qsa_pool_block_keys(ki, rope_theta=rope_theta, yarn=yarn)
+    qr = qsa_rope_index_queries(qi, rope_theta=rope_theta, q_pos0=q_pos0, yarn=yarn) if rope_theta > 0 else qi
     idx = qsa_select_topk(topk, qi=qr, kp=kp, head_w=head_w, q_pos0=q_pos0, mode=mode, workspace=workspace)
     out, lse = qsa_sparse_attn_prefill(q, k, v, idx, q_pos0=q_pos0, scale=scale)
     return dict(out=out, lse=lse, idx=idx, kp=kp)
 
 
 def decode(q, kcache, vcache, qi, kp, seqlens, *, topk: int, rope_theta: float = 0.0, head_w=None,
-           mode: int = QSA_SCORE_RELU_SUM, scale: float | None = None, num_splits: int = 0, workspace=None):
+           mode: int = QSA_SCORE_RELU_SUM, scale: float | None = None, num_splits: int = 0, workspace=None,
+           yarn=None):
     """One decode step on a pooled indexer-key cache kp [B, NBk, Di]: [RoPE query] -> score + top-k
     -> split-KV sparse attention.  Returns dict(out, lse, idx)."""
-    qr = qsa_rope_index_queries(qi, rope_theta=rope_theta, seqlens=seqlens) if rope_theta > 0 else qi
+    qr = qsa_rope_index_queries(qi, rope_theta=rope_theta, seqlens=seqlens, yarn=yarn) if rope_theta > 0 else qi
     idx = qsa_select_topk(topk, qi=qr, kp=kp, head_w=head_w, seqlens=seqlens, mode=mode, workspace=workspace)
     out, lse = qsa_sparse_attn_decode(q, kcache, vcache, seqlens, idx, scale=scale, num_splits=num_splits)
     return dict(out=out, lse=lse, idx=idx)
@@ -339,7 +366,7 @@ def _copy_stream(device, which: str = "in") -> "torch.cuda.Stream":
 
 def prefill_host(q, k, v, qi, ki, *, topk: int, device="cuda", out=None, q_pos0: int = 0, rope_theta: float = 0.0,
                  head_w=None, mode: int = QSA_SCORE_RELU_SUM, scale: float | None = None, workspace=None,
-                 device_buffers: dict | None = None, chunks: int = 8):
+                 device_buffers: dict | None = None, chunks: int = 8, yarn=None):
     """The QSA layer for a prefill whose inputs live in (pinned) host memory; returns the output in
     host memory.  Transfers overlap the kernels.  ki and qi are copied first and the pooling and
     block selection of all rows run while q, k and v follow in ``chunks`` causal row chunks on a
@@ -388,8 +415,9 @@ def prefill_host(q, k, v, qi, ki, *, topk: int, device="cuda", out=None, q_pos0:
             ev.record(cin)
             arrived.append(ev)
     main.wait_event(sel_ready)
-    kp = qsa_pool_block_keys(bufs["ki"], bufs["kp"], rope_theta=rope_theta)
-    qr = qsa_rope_index_queries(bufs["qi"], rope_theta=rope_theta, q_pos0=q_pos0) if rope_theta > 0 else bufs["qi"]
+    kp = qsa_pool_block_keys(bufs["ki"], bufs["kp"], rope_theta=rope_theta, yarn=yarn)
+    qr = (qsa_rope_index_queries(bufs["qi"], rope_theta=rope_theta, q_pos0=q_pos0, yarn=yarn) if rope_theta > 0
+          else bufs["qi"])
     idx = qsa_select_topk(topk, qi=qr, kp=kp, head_w=head_w, q_pos0=q_pos0, mode=mode, workspace=workspace,
                           idx=bufs.get("idx"))
     bufs["idx"] = idx

@@ -99,6 +99,34 @@ QSA_API qsa_status_t qsa_pool_block_keys(const void* ki, void* kp, int B, int L,
                                          int64_t kp_batch_stride, void* stream);
 
 /*
+ * Rotary parameters of the indexer, for the _rope variants below.  theta <= 0: no rotation.
+ * yarn_factor > 1 scales the frequencies for contexts beyond yarn_orig_ctx positions with YaRN
+ * ("YaRN: Efficient Context Window Extension of Large Language Models", Peng et al. 2023, sections
+ * 3.2 and 3.4; the pages name YaRN for the 1M-token context but give no parameters).  For the pair
+ * with base frequency f = theta^(-2i/Di) and r = yarn_orig_ctx * f / (2 pi) rotations over the
+ * original context, g = clamp((r - yarn_alpha) / (yarn_beta - yarn_alpha), 0, 1) and the frequency
+ * becomes (1 - g) f / yarn_factor + g f; the rotated pair is multiplied by yarn_mscale (<= 0: the
+ * paper's 0.1 ln(yarn_factor) + 1).  Typical ramp: yarn_alpha = 1, yarn_beta = 32.
+ */
+typedef struct qsa_rope_params {
+  double theta;
+  double yarn_factor;    /* <= 1: plain RoPE */
+  double yarn_orig_ctx;  /* > 0 when yarn_factor > 1 */
+  double yarn_alpha;
+  double yarn_beta;      /* > yarn_alpha */
+  double yarn_mscale;
+} qsa_rope_params_t;
+
+/*
+ * qsa_pool_block_keys with rotary parameters (NULL: no rotation).  Errors as above, and
+ * INVALID_ARGUMENT for inconsistent YaRN parameters.
+ */
+QSA_API qsa_status_t qsa_pool_block_keys_rope(const void* ki, void* kp, int B, int L, int Di, int blk,
+                                              const qsa_rope_params_t* rope, int64_t pos0,
+                                              int64_t ki_batch_stride, int64_t kp_batch_stride,
+                                              void* stream);
+
+/*
  * RoPE of the indexer queries at their own positions (the query side of the rotation that the
  * keys receive after pooling).
  *   qi [B][Tq][Hi][Di] bf16 -> qi_out (same layout; may alias qi)
@@ -109,6 +137,14 @@ QSA_API qsa_status_t qsa_pool_block_keys(const void* ki, void* kp, int B, int L,
 QSA_API qsa_status_t qsa_rope_index_queries(const void* qi, void* qi_out, int B, int Tq, int Hi, int Di,
                                     int64_t q_pos0, const int32_t* seqlens, float rope_theta,
                                     void* stream);
+
+/*
+ * qsa_rope_index_queries with rotary parameters (theta must be > 0); use the same parameters as
+ * for the keys.  Errors as above.
+ */
+QSA_API qsa_status_t qsa_rope_index_queries_rope(const void* qi, void* qi_out, int B, int Tq, int Hi,
+                                                 int Di, int64_t q_pos0, const int32_t* seqlens,
+                                                 const qsa_rope_params_t* rope, void* stream);
 
 /*
  * Indexer block scores (step 2: four indexer query heads against one shared key head).

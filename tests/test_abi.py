@@ -132,3 +132,13 @@ def test_select_options_checks(lib):
     assert lib.qsa_set_select_options(0, -5) == Q.QSA_ERR_INVALID_ARGUMENT
     assert lib.qsa_set_select_options(2, 7) == Q.QSA_OK
     assert lib.qsa_set_select_options(0, 0) == Q.QSA_OK
+
+
+def test_rope_params_checks(lib):
+    rp = Q.RopeParams(10000.0, 4.0, 0.0, 1.0, 32.0, 0.0)      # YaRN without an original context
+    assert lib.qsa_pool_block_keys_rope(1, 1, 1, 8, 64, 4, ctypes.byref(rp), 0, 0, 0, None) == Q.QSA_ERR_INVALID_ARGUMENT
+    rp = Q.RopeParams(10000.0, 4.0, 4096.0, 32.0, 1.0, 0.0)   # ramp bounds reversed
+    assert lib.qsa_pool_block_keys_rope(1, 1, 1, 8, 64, 4, ctypes.byref(rp), 0, 0, 0, None) == Q.QSA_ERR_INVALID_ARGUMENT
+    rp = Q.RopeParams(0.0, 1.0, 0.0, 1.0, 32.0, 0.0)          # the query rotation needs a base
+    assert lib.qsa_rope_index_queries_rope(1, 1, 1, 4, 4, 64, 0, None, ctypes.byref(rp), None) == Q.QSA_ERR_INVALID_ARGUMENT
+    assert lib.qsa_rope_index_queries_rope(1, 1, 1, 4, 4, 64, 0, None, None, None) == Q.QSA_ERR_INVALID_ARGUMENT

@@ -221,6 +221,55 @@ def test_whole_layer_with_rope_and_batches():
         print("rope batch", b, st)
 
 
+YARN = dict(factor=4.0, orig_ctx=262144, alpha=1.0, beta=32.0)
+
+
+def test_pool_and_query_rope_with_yarn_match_oracle():
+    ki = _randn_bf16((2, 4000, 64), 0.125, 71)
+    for pos0 in (0, 700000):
+        kp = I.bits(Q.qsa_pool_block_keys(ki, rope_theta=10000.0, pos0=pos0, yarn=YARN))
+        ref = O.pool_block_keys(I.bits(ki), rope_theta=10000.0, pos0=pos0, yarn=YARN)
+        diff = np.abs(O.bf16_to_f64(kp) - O.bf16_to_f64(ref))
+        assert (kp != ref).mean() <= 1e-4
+        assert np.all(diff <= np.maximum(np.abs(O.bf16_to_f64(ref)), 1e-30) * 2 ** -7)
+    qi = _randn_bf16((2, 300, 4, 64), 0.125, 72)
+    out = Q.qsa_rope_index_queries(qi, rope_theta=10000.0, q_pos0=900000, yarn=YARN)
+    pos = np.tile(np.arange(300) + 900000, 2)
+    ref = O.rope_rows(I.bits(qi).reshape(-1, 4, 64), pos, 10000.0, yarn=YARN).reshape(2, 300, 4, 64)
+    assert (I.bits(out) != ref).mean() <= 1e-4
+    seqlens = torch.tensor([5, 1048576], dtype=torch.int32, device=DEV)
+    qd = _randn_bf16((2, 4, 64), 0.125, 73)
+    outd = Q.qsa_rope_index_queries(qd, rope_theta=10000.0, seqlens=seqlens, yarn=dict(YARN, mscale=1.25))
+    refd = O.rope_rows(I.bits(qd), np.array([4, 1048575]), 10000.0, yarn=dict(YARN, mscale=1.25))
+    assert (I.bits(outd) != refd).mean() <= 1e-3
+    _status_ok()
+
+
+def test_whole_layer_with_yarn_rope():
+    """Pooled keys and indexer queries rotated with YaRN-scaled frequencies at positions past the
+    original context; the oracle gets its own YaRN-rotated keys and queries."""
+    T, k, theta, q0 = 2600, 48, 10000.0, 300000
+    x = _small_prefill(T, 16, 2, 4, 107)
+    y = dict(factor=8.0, orig_ctx=65536)
+    qrows = {n: x[n][:, 1000:].contiguous() for n in ("q", "qi")}
+    # a window of rows 1000.. of a sequence whose first token sits at position q0
+    res_kp = Q.qsa_pool_block_keys(x["ki"], rope_theta=theta, pos0=q0, yarn=y)
+    qr = Q.qsa_rope_index_queries(qrows["qi"], rope_theta=theta, q_pos0=q0 + 1000, yarn=y)
+    idx = Q.qsa_select_topk(k, qi=qr, kp=res_kp, q_pos0=1000)
+    out, lse = Q.qsa_sparse_attn_prefill(qrows["q"], x["k"], x["v"], idx, q_pos0=1000)
+    torch.cuda.synchronize()
+    _status_ok()
+    h = {n: I.bits(t) for n, t in x.items()}
+    kp = O.pool_block_keys(h["ki"], rope_theta=theta, pos0=q0, yarn=y)
+    assert (I.bits(res_kp) != kp).mean() <= 1e-3
+    rows = [r for r in H.sample_rows(T, k, n_random=30, seed=5) if r >= 1000]
+    qi_rot = O.rope_rows(h["qi"][0][rows], np.array(rows) + q0, theta, yarn=y)
+    sel = [r - 1000 for r in rows]
+    st = H.compare_prefill(idx.cpu().numpy()[0][sel], I.bits(out)[0][sel], lse.cpu().numpy()[0][sel], h["q"][0][rows],
+                           qi_rot, h["k"][0], h["v"][0], kp[0], rows, topk=k)
+    print("yarn", st)
+
+
 def test_chunked_prefill_matches_full_prefill():
     T, k, q0 = 2500, 64, 1234
     x = _small_prefill(T, 16, 2, 4, 55)
