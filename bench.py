@@ -71,6 +71,14 @@ def prefill_work(w) -> dict:
     return dict(attn_bytes=attn_bytes, attn_flops=attn_flops, index_flops=idx_flops, pairs=pairs * w.B)
 
 
+def attn_kernel_name(w) -> str:
+    """The attention kernel the library launches for this shape."""
+    group = w.Hq // w.Hkv
+    if w.D == 128 and group <= 8:
+        return f"sparse_attn_kernel<{w.Hkv}>"
+    return f"sparse_attn_wide_kernel<{w.Hkv},{w.D},{1 if group <= 8 else 2}>"
+
+
 def decode_work(w) -> dict:
     nb = (w.T - 1) // w.blk
     S = w.blk * min(nb, w.k) + (w.T - 1) % w.blk + 1
@@ -461,7 +469,7 @@ def run_qsa(args):
             "config": {"workload": args.workload, "B": w.B, "T": w.T, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "Hi": w.Hi,
                        "Di": w.Di, "blk": w.blk, "k": w.k, "boost": f"{w.boost_frac:g} of keys x{w.boost:g}",
                        "l2": "inputs larger than L2, no flush", "parallelism": f"independent replicas x{world}"},
-            "roofline": {"bound": "hbm", "kernel": "sparse_attn_kernel<2>", "achieved": attn_gbs,
+            "roofline": {"bound": "hbm", "kernel": attn_kernel_name(w), "achieved": attn_gbs,
                          "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": attn_gbs / pk["hbm_gbs"],
                          "traffic": ATTN_DRAM_TRAFFIC.get(args.workload), "peak_source": pk["source"],
                          "basis": "gathered K/V bytes of every selected token + q read + o write",

@@ -361,7 +361,7 @@ qsa_status_t qsa_select_topk(const float* scores, int64_t ld_scores, const void*
 static qsa_status_t check_attn_shape(int Hq, int Hkv, int D, int blk, int k_blocks) {
   if (Hq < 1 || Hkv < 1 || k_blocks < 0) return QSA_ERR_INVALID_ARGUMENT;
   if (Hq % Hkv) return QSA_ERR_INVALID_ARGUMENT;
-  if (D != 128 || blk != 4 || Hkv > 2 || Hq / Hkv > 8) return QSA_ERR_UNSUPPORTED;
+  if ((D != 128 && D != 256) || blk != 4 || Hkv > 2 || Hq / Hkv > 16) return QSA_ERR_UNSUPPORTED;
   return QSA_OK;
 }
 
@@ -378,7 +378,7 @@ qsa_status_t qsa_sparse_attn_prefill(const void* q, const void* k, const void* v
   const DeviceInfo* di = device_info();
   if (!di) return QSA_ERR_CUDA;
   return cuda_status(
-      launch_attn_prefill(di, q, k, v, idx, B, Tq, Tk, Hq, Hkv, k_blocks, q_pos0, scale, out, lse, S(stream)));
+      launch_attn_prefill(di, q, k, v, idx, B, Tq, Tk, Hq, Hkv, D, k_blocks, q_pos0, scale, out, lse, S(stream)));
 }
 
 int qsa_decode_default_splits(int B, int k_blocks) {
@@ -408,8 +408,8 @@ qsa_status_t qsa_sparse_attn_decode(const void* q, const void* kcache, const voi
     if (workspace == nullptr || ws_bytes < need) return QSA_ERR_WORKSPACE_TOO_SMALL;
     part = static_cast<float*>(workspace);
   }
-  return cuda_status(launch_attn_decode(di, q, kcache, vcache, seqlens, idx, B, Lmax, Hq, Hkv, k_blocks, scale, splits,
-                                        out, lse, part, S(stream)));
+  return cuda_status(launch_attn_decode(di, q, kcache, vcache, seqlens, idx, B, Lmax, Hq, Hkv, D, k_blocks, scale,
+                                        splits, out, lse, part, S(stream)));
 }
 
 size_t qsa_workspace_size(qsa_op_t op, int B, int Tq, int NBk, int k, int Hq, int D, int num_splits) {

@@ -41,7 +41,7 @@ extern "C" qsa_status_t qsa_sparse_attn_decode_noalloc(const void* q, const void
                                                        int Hq, int Hkv, int D, int k_blocks, int blk, float scale,
                                                        int num_splits, void* out, float* lse, void* stream) {
   if (Hq < 1 || Hkv < 1 || k_blocks < 0 || Hq % Hkv) return QSA_ERR_INVALID_ARGUMENT;
-  if (D != 128 || blk != 4 || Hkv > 2 || Hq / Hkv > 8) return QSA_ERR_UNSUPPORTED;
+  if ((D != 128 && D != 256) || blk != 4 || Hkv > 2 || Hq / Hkv > 16) return QSA_ERR_UNSUPPORTED;
   if (B < 0 || Lmax < 1 || num_splits < 0) return QSA_ERR_INVALID_ARGUMENT;
   if (B == 0) return QSA_OK;
   if (!ok_ptr(q) || !ok_ptr(kcache) || !ok_ptr(vcache) || !ok_ptr(out) || seqlens == nullptr ||
@@ -61,7 +61,7 @@ extern "C" qsa_status_t qsa_sparse_attn_decode_noalloc(const void* q, const void
     part = scratch_for(di->device, &e);
     if (e != cudaSuccess || part == nullptr) return QSA_ERR_CUDA;
   }
-  cudaError_t e = launch_attn_decode(di, q, kcache, vcache, seqlens, idx, B, Lmax, Hq, Hkv, k_blocks, scale, splits,
+  cudaError_t e = launch_attn_decode(di, q, kcache, vcache, seqlens, idx, B, Lmax, Hq, Hkv, D, k_blocks, scale, splits,
                                      out, lse, part, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? QSA_OK : QSA_ERR_CUDA;
 }

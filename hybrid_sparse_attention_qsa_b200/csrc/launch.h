@@ -67,10 +67,10 @@ cudaError_t launch_topk_fallback(const DeviceInfo* di, const void* qi, const voi
                                  int nctas, int k, int32_t* idx, cudaStream_t s);
 
 cudaError_t launch_attn_prefill(const DeviceInfo* di, const void* q, const void* k, const void* v, const int32_t* idx,
-                                int B, int Tq, int Tk, int Hq, int Hkv, int k_blocks, long long q_pos0, float scale,
-                                void* out, float* lse, cudaStream_t s);
+                                int B, int Tq, int Tk, int Hq, int Hkv, int D, int k_blocks, long long q_pos0,
+                                float scale, void* out, float* lse, cudaStream_t s);
 cudaError_t launch_attn_decode(const DeviceInfo* di, const void* q, const void* kc, const void* vc,
-                               const int32_t* seqlens, const int32_t* idx, int B, int Lmax, int Hq, int Hkv,
+                               const int32_t* seqlens, const int32_t* idx, int B, int Lmax, int Hq, int Hkv, int D,
                                int k_blocks, float scale, int num_splits, void* out, float* lse, float* part,
                                cudaStream_t s);
 int decode_default_splits(const DeviceInfo* di, int B, int k_blocks);

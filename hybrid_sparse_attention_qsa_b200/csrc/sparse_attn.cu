@@ -56,6 +56,19 @@ struct StageInfo {
   uint8_t ntok[kSlots];
 };
 
+// Shared-memory ring of the copy pipeline: per stage SLOTS block slots of K, then SLOTS of V.  A
+// block of 4 tokens of all KV heads is one contiguous run of kBlockBytes in the [T][Hkv][D] layout.
+template <int HKV, int D, int SLOTS>
+struct Ring {
+  static_assert(SLOTS % kIssuers_ == 0 && SLOTS <= 16, "slots per issuer warp");
+  static constexpr int kSlots = SLOTS;
+  static constexpr int kTokBytes = HKV * D * 2;               // one token of K (or V), all KV heads
+  static constexpr int kBlockBytes = kBlk * kTokBytes;        // one block of K (or of V)
+  static constexpr int kPitch = kBlockBytes + 16;             // +16: conflict-free ldmatrix across slots
+  static constexpr int kStageBytes = 2 * SLOTS * kPitch;      // K slots, then V slots
+  static constexpr int kInfoStride = (sizeof(StageInfo) + 15) / 16 * 16;
+};
+
 template <int HKV>
 struct Cfg {
   static constexpr int kBlockBytes = kBlk * HKV * kD * 2;     // one block of K (or of V)
@@ -101,7 +114,7 @@ struct Item {
   bool diag, ok, partial;
 };
 
-template <int HKV>
+template <int HKV, int D = kD>
 __device__ __forceinline__ Item make_item(const AttnArgs& a, int i) {
   Item it;
   if (a.seqlens == nullptr) {
@@ -110,8 +123,8 @@ __device__ __forceinline__ Item make_item(const AttnArgs& a, int i) {
     it.qrow = static_cast<long long>(b) * a.Tq + t;
     it.orow = it.qrow;
     it.pos = a.q_pos0 + t;
-    it.kbase = a.k + static_cast<long long>(b) * a.Tk * HKV * kD;
-    it.vbase = a.v + static_cast<long long>(b) * a.Tk * HKV * kD;
+    it.kbase = a.k + static_cast<long long>(b) * a.Tk * HKV * D;
+    it.vbase = a.v + static_cast<long long>(b) * a.Tk * HKV * D;
     it.idx_row = a.idx + it.qrow * a.kblocks;
     it.lo = 0;
     it.hi = a.kblocks;
@@ -125,8 +138,8 @@ __device__ __forceinline__ Item make_item(const AttnArgs& a, int i) {
     it.pos = static_cast<long long>(L) - 1;
     it.qrow = b;
     it.orow = a.splits > 1 ? i : b;
-    it.kbase = a.k + static_cast<long long>(b) * a.Tk * HKV * kD;
-    it.vbase = a.v + static_cast<long long>(b) * a.Tk * HKV * kD;
+    it.kbase = a.k + static_cast<long long>(b) * a.Tk * HKV * D;
+    it.vbase = a.v + static_cast<long long>(b) * a.Tk * HKV * D;
     it.idx_row = a.idx + static_cast<long long>(b) * a.kblocks;
     const int chunk = (a.kblocks + a.splits - 1) / a.splits;
     it.lo = min(a.kblocks, sp * chunk);
@@ -135,6 +148,177 @@ __device__ __forceinline__ Item make_item(const AttnArgs& a, int i) {
     it.partial = a.splits > 1;
   }
   return it;
+}
+
+// Helper issuer warp h (1 .. kIssuers_ - 1): issues slots h, h + kIssuers_, ... of every stage the
+// leading producer publishes, until it publishes nslots == -1.
+template <int HKV, int D, int SLOTS>
+__device__ __forceinline__ void attn_helper(const AttnArgs& a, int h, uint8_t* ring, uint8_t* info, uint64_t* full,
+                                            uint64_t* ready) {
+  using R = Ring<HKV, D, SLOTS>;
+  const int lane = threadIdx.x & 31;
+  auto info_at = [&](int s) { return reinterpret_cast<const StageInfo*>(info + s * R::kInfoStride); };
+  // ------------------------------------------------------------------ helper issuer warps
+  // The per-SM rate of 1-D bulk copies grows with the number of warps issuing them, so the
+  // copies of a stage are spread over kIssuers warps: helper h issues slots h, h + kIssuers, ...
+  int st = 0;
+  unsigned ph = 0;
+  const uint32_t tok_bytes = R::kTokBytes;
+  for (;;) {
+    if (!mbar_wait(&ready[st], ph, a.ctl)) break;
+    const StageInfo* inf = info_at(st);
+    const int n = inf->nslots;
+    if (n < 0) break;
+    const int slot = h + kIssuers_ * lane;
+    if (lane < R::kSlots / kIssuers_ && slot < n) {
+      const int ntok = inf->ntok[slot];
+      const long long tok0 = inf->tok0[slot];
+      uint8_t* kd = ring + st * R::kStageBytes + slot * R::kPitch;
+      uint8_t* vd = kd + R::kSlots * R::kPitch;
+      bulk_g2s(kd, inf->kbase + tok0 * HKV * D, ntok * tok_bytes, &full[st]);
+      bulk_g2s(vd, inf->vbase + tok0 * HKV * D, ntok * tok_bytes, &full[st]);
+    }
+    __syncwarp();
+    if (++st == kStages) {
+      st = 0;
+      ph ^= 1u;
+    }
+  }
+}
+
+// Leading producer warp: walks the work items, turns each index list into block copies (the
+// query's own block last), publishes each stage's slot list for the helpers and issues its own
+// share of the copies.  Returns only when no copy it registered is still in flight.
+template <int HKV, int D, int SLOTS>
+__device__ __forceinline__ void attn_producer(const AttnArgs& a, uint8_t* ring, uint8_t* info, uint64_t* full,
+                                              uint64_t* empty, uint64_t* ready, int* pend, int* idxbuf) {
+  using R = Ring<HKV, D, SLOTS>;
+  const int lane = threadIdx.x & 31;
+  auto info_at = [&](int s) { return reinterpret_cast<StageInfo*>(info + s * R::kInfoStride); };
+  // ------------------------------------------------------------------ leading producer warp
+  int st = 0;
+  unsigned ph = 0;
+  int fills = 0;
+  bool alive = true;
+  const uint32_t tok_bytes = R::kTokBytes;
+  auto flush = [&](int n, bool last, const Item& it) -> bool {
+    if (!mbar_wait(&empty[st], ph ^ 1u, a.ctl)) return false;
+    int packed = lane < n ? pend[lane] : 0;
+    const int ntok = packed & 7;
+    const long long tok0 = packed >> 3;
+    StageInfo* inf = info_at(st);
+    if (lane < R::kSlots) {
+      inf->ntok[lane] = static_cast<uint8_t>(lane < n ? ntok : 0);
+      inf->tok0[lane] = static_cast<int>(tok0);
+    }
+    if (lane == 0) {
+      inf->nslots = n;
+      inf->last = last ? 1 : 0;
+      inf->kbase = it.kbase;
+      inf->vbase = it.vbase;
+    }
+    const uint32_t mine = lane < n ? 2u * ntok * tok_bytes : 0u;
+    const uint32_t total = __reduce_add_sync(0xffffffffu, mine);
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&full[st], total);   // registered before any helper can issue a copy
+      mbar_arrive(&ready[st]);
+    }
+    __syncwarp();
+    if (lane < n && lane % kIssuers_ == 0) {
+      uint8_t* kd = ring + st * R::kStageBytes + lane * R::kPitch;
+      uint8_t* vd = kd + R::kSlots * R::kPitch;
+      bulk_g2s(kd, it.kbase + tok0 * HKV * D, ntok * tok_bytes, &full[st]);
+      bulk_g2s(vd, it.vbase + tok0 * HKV * D, ntok * tok_bytes, &full[st]);
+    }
+    // drop the flushed entries from the pending list
+    int rest0 = n + lane < 64 ? pend[n + lane] : 0;
+    int rest1 = n + lane + 32 < 64 ? pend[n + lane + 32] : 0;
+    __syncwarp();
+    pend[lane] = rest0;
+    if (lane + 32 < 64) pend[lane + 32] = rest1;
+    __syncwarp();
+    ++fills;
+    if (++st == kStages) {
+      st = 0;
+      ph ^= 1u;
+    }
+    return true;
+  };
+  // The index list of an item is staged in shared memory by asynchronous copies one segment
+  // ahead (the next segment of this item or the first of the next item), so the copy ring never
+  // waits on a global load of the list.
+  auto fetch = [&](int item, int seg, int buf) {
+    if (item < a.num_items) {
+      const Item f = make_item<HKV, D>(a, item);
+      const int base = f.lo + seg * kSeg;
+      const int len = max(0, min(kSeg, f.hi - base));
+      for (int e = lane; e < len; e += 32) cp_async4(&idxbuf[buf * kSeg + e], f.idx_row + base + e);
+    }
+    cp_async_commit();
+  };
+  int buf = 0;
+  fetch(blockIdx.x, 0, 0);
+  for (int item = blockIdx.x; alive && item < a.num_items; item += gridDim.x) {
+    const Item it = make_item<HKV, D>(a, item);
+    const long long own = it.pos >= 0 ? it.pos / kBlk : 0;
+    int npend = 0;
+    const int nseg = max(1, (it.hi - it.lo + kSeg - 1) / kSeg);
+    for (int seg = 0; seg < nseg; ++seg) {
+      if (seg + 1 < nseg)
+        fetch(item, seg + 1, buf ^ 1);
+      else
+        fetch(item + gridDim.x, 0, buf ^ 1);
+      cp_async_wait<1>();
+      __syncwarp();
+      const int len = max(0, min(kSeg, it.hi - (it.lo + seg * kSeg)));
+      if (it.ok) {
+        for (int c = 0; alive && c < len; c += 32) {
+          const int e = c + lane < len ? idxbuf[buf * kSeg + c + lane] : -1;
+          const bool valid = e >= 0 && e < own;
+          if (!valid && e != -1 && e != own) record_status(a.ctl, kStBadArg);
+          const unsigned m = __ballot_sync(0xffffffffu, valid);
+          if (valid) pend[npend + __popc(m & ((1u << lane) - 1u))] = (e * kBlk) << 3 | kBlk;
+          npend += __popc(m);
+          __syncwarp();
+          while (alive && npend > R::kSlots) {
+            alive = flush(R::kSlots, false, it);
+            npend -= R::kSlots;
+          }
+        }
+      }
+      __syncwarp();
+      buf ^= 1;
+    }
+    if (it.ok) {
+      if (it.diag) {
+        if (lane == 0) pend[npend] = static_cast<int>((own * kBlk) << 3) | static_cast<int>(it.pos - own * kBlk + 1);
+        ++npend;
+        __syncwarp();
+      }
+    } else if (lane == 0) {
+      record_status(a.ctl, kStBadArg);
+    }
+    while (alive && npend > R::kSlots) {
+      alive = flush(R::kSlots, false, it);
+      npend -= R::kSlots;
+    }
+    if (alive) alive = flush(npend, true, it);
+  }
+  cp_async_wait<0>();
+  // Tell the helpers that no stage follows (the stage is free once every consumer released it).
+  if (alive && mbar_wait(&empty[st], ph ^ 1u, a.ctl)) {
+    if (lane == 0) {
+      info_at(st)->nslots = -1;
+      mbar_arrive(&ready[st]);
+    }
+    __syncwarp();
+  }
+  // Never leave with a copy in flight: wait for the last fill of every stage.
+  for (int s = 0; s < kStages && s < fills; ++s) {
+    const int last = s + ((fills - 1 - s) / kStages) * kStages;
+    mbar_wait(&full[s], (last / kStages) & 1u, a.ctl);
+  }
 }
 
 template <int HKV>
@@ -177,161 +361,11 @@ __global__ void __launch_bounds__(Cfg<HKV>::kThreads, 1) sparse_attn_kernel(Attn
   __syncthreads();
 
   if (warp > C::kConsumerWarps) {
-    // ------------------------------------------------------------------ helper issuer warps
-    // The per-SM rate of 1-D bulk copies grows with the number of warps issuing them, so the
-    // copies of a stage are spread over kIssuers warps: helper h issues slots h, h + kIssuers, ...
-    const int h = warp - C::kConsumerWarps;
-    int st = 0;
-    unsigned ph = 0;
-    const uint32_t tok_bytes = HKV * kD * 2;
-    for (;;) {
-      if (!mbar_wait(&ready[st], ph, a.ctl)) break;
-      const StageInfo* inf = info_at(st);
-      const int n = inf->nslots;
-      if (n < 0) break;
-      const int slot = h + kIssuers_ * lane;
-      if (lane < kSlots / kIssuers_ && slot < n) {
-        const int ntok = inf->ntok[slot];
-        const long long tok0 = inf->tok0[slot];
-        uint8_t* kd = ring + st * C::kStageBytes + slot * C::kPitch;
-        uint8_t* vd = kd + kSlots * C::kPitch;
-        bulk_g2s(kd, inf->kbase + tok0 * HKV * kD, ntok * tok_bytes, &full[st]);
-        bulk_g2s(vd, inf->vbase + tok0 * HKV * kD, ntok * tok_bytes, &full[st]);
-      }
-      __syncwarp();
-      if (++st == kStages) {
-        st = 0;
-        ph ^= 1u;
-      }
-    }
+    attn_helper<HKV, kD, kSlots>(a, warp - C::kConsumerWarps, ring, reinterpret_cast<uint8_t*>(info), full, ready);
     return;
   }
-
   if (warp == C::kConsumerWarps) {
-    // ------------------------------------------------------------------ leading producer warp
-    int st = 0;
-    unsigned ph = 0;
-    int fills = 0;
-    bool alive = true;
-    const uint32_t tok_bytes = HKV * kD * 2;
-    auto flush = [&](int n, bool last, const Item& it) -> bool {
-      if (!mbar_wait(&empty[st], ph ^ 1u, a.ctl)) return false;
-      int packed = lane < n ? pend[lane] : 0;
-      const int ntok = packed & 7;
-      const long long tok0 = packed >> 3;
-      StageInfo* inf = info_at(st);
-      if (lane < kSlots) {
-        inf->ntok[lane] = static_cast<uint8_t>(lane < n ? ntok : 0);
-        inf->tok0[lane] = static_cast<int>(tok0);
-      }
-      if (lane == 0) {
-        inf->nslots = n;
-        inf->last = last ? 1 : 0;
-        inf->kbase = it.kbase;
-        inf->vbase = it.vbase;
-      }
-      const uint32_t mine = lane < n ? 2u * ntok * tok_bytes : 0u;
-      const uint32_t total = __reduce_add_sync(0xffffffffu, mine);
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&full[st], total);   // registered before any helper can issue a copy
-        mbar_arrive(&ready[st]);
-      }
-      __syncwarp();
-      if (lane < n && lane % kIssuers_ == 0) {
-        uint8_t* kd = ring + st * C::kStageBytes + lane * C::kPitch;
-        uint8_t* vd = kd + kSlots * C::kPitch;
-        bulk_g2s(kd, it.kbase + tok0 * HKV * kD, ntok * tok_bytes, &full[st]);
-        bulk_g2s(vd, it.vbase + tok0 * HKV * kD, ntok * tok_bytes, &full[st]);
-      }
-      // drop the flushed entries from the pending list
-      int rest0 = n + lane < 64 ? pend[n + lane] : 0;
-      int rest1 = n + lane + 32 < 64 ? pend[n + lane + 32] : 0;
-      __syncwarp();
-      pend[lane] = rest0;
-      if (lane + 32 < 64) pend[lane + 32] = rest1;
-      __syncwarp();
-      ++fills;
-      if (++st == kStages) {
-        st = 0;
-        ph ^= 1u;
-      }
-      return true;
-    };
-    // The index list of an item is staged in shared memory by asynchronous copies one segment
-    // ahead (the next segment of this item or the first of the next item), so the copy ring never
-    // waits on a global load of the list.
-    auto fetch = [&](int item, int seg, int buf) {
-      if (item < a.num_items) {
-        const Item f = make_item<HKV>(a, item);
-        const int base = f.lo + seg * kSeg;
-        const int len = max(0, min(kSeg, f.hi - base));
-        for (int e = lane; e < len; e += 32) cp_async4(&idxbuf[buf * kSeg + e], f.idx_row + base + e);
-      }
-      cp_async_commit();
-    };
-    int buf = 0;
-    fetch(blockIdx.x, 0, 0);
-    for (int item = blockIdx.x; alive && item < a.num_items; item += gridDim.x) {
-      const Item it = make_item<HKV>(a, item);
-      const long long own = it.pos >= 0 ? it.pos / kBlk : 0;
-      int npend = 0;
-      const int nseg = max(1, (it.hi - it.lo + kSeg - 1) / kSeg);
-      for (int seg = 0; seg < nseg; ++seg) {
-        if (seg + 1 < nseg)
-          fetch(item, seg + 1, buf ^ 1);
-        else
-          fetch(item + gridDim.x, 0, buf ^ 1);
-        cp_async_wait<1>();
-        __syncwarp();
-        const int len = max(0, min(kSeg, it.hi - (it.lo + seg * kSeg)));
-        if (it.ok) {
-          for (int c = 0; alive && c < len; c += 32) {
-            const int e = c + lane < len ? idxbuf[buf * kSeg + c + lane] : -1;
-            const bool valid = e >= 0 && e < own;
-            if (!valid && e != -1 && e != own) record_status(a.ctl, kStBadArg);
-            const unsigned m = __ballot_sync(0xffffffffu, valid);
-            if (valid) pend[npend + __popc(m & ((1u << lane) - 1u))] = (e * kBlk) << 3 | kBlk;
-            npend += __popc(m);
-            __syncwarp();
-            while (alive && npend > kSlots) {
-              alive = flush(kSlots, false, it);
-              npend -= kSlots;
-            }
-          }
-        }
-        __syncwarp();
-        buf ^= 1;
-      }
-      if (it.ok) {
-        if (it.diag) {
-          if (lane == 0) pend[npend] = static_cast<int>((own * kBlk) << 3) | static_cast<int>(it.pos - own * kBlk + 1);
-          ++npend;
-          __syncwarp();
-        }
-      } else if (lane == 0) {
-        record_status(a.ctl, kStBadArg);
-      }
-      while (alive && npend > kSlots) {
-        alive = flush(kSlots, false, it);
-        npend -= kSlots;
-      }
-      if (alive) alive = flush(npend, true, it);
-    }
-    cp_async_wait<0>();
-    // Tell the helpers that no stage follows (the stage is free once every consumer released it).
-    if (alive && mbar_wait(&empty[st], ph ^ 1u, a.ctl)) {
-      if (lane == 0) {
-        info_at(st)->nslots = -1;
-        mbar_arrive(&ready[st]);
-      }
-      __syncwarp();
-    }
-    // Never leave with a copy in flight: wait for the last fill of every stage.
-    for (int s = 0; s < kStages && s < fills; ++s) {
-      const int last = s + ((fills - 1 - s) / kStages) * kStages;
-      mbar_wait(&full[s], (last / kStages) & 1u, a.ctl);
-    }
+    attn_producer<HKV, kD, kSlots>(a, ring, reinterpret_cast<uint8_t*>(info), full, empty, ready, pend, idxbuf);
     return;
   }
 
@@ -549,22 +583,272 @@ __global__ void __launch_bounds__(Cfg<HKV>::kThreads, 1) sparse_attn_kernel(Attn
   }
 }
 
-// Merge of decode splits: out[b][h] = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s.
-__global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ part, int splits, int Hq,
+// ======================================================================================
+// Wide variant: head dimension D (128 or 256) and GQA groups of up to 16 query heads (the model
+// shape of the pages: D = 256, 24 query heads over 2 KV heads, groups of 12).  A stage holds 8 block
+// slots (the ring of 3 stages stays within shared memory at D = 256).  Consumer warp (g, hs) owns KV
+// head g and the query heads hs*8 .. hs*8+7 of its group (N = 8 of mma.m16n8k16; heads past the group
+// are zero columns), and covers all 32 tokens of a stage as two m16 tiles, so no merge between
+// warps is needed: m-tile t holds tokens 2t and 2t+1 of the 8 slots (rows = slot + 8 * token
+// parity), which keeps ldmatrix on 8 different slots (conflict-free with the padded pitch).
+constexpr int kWideSlots = 8;
+
+template <int HKV, int D, int NSUB>
+struct WideCfg {
+  using R = Ring<HKV, D, kWideSlots>;
+  static constexpr int kConsumerWarps = HKV * NSUB;
+  static constexpr int kThreads = (kConsumerWarps + kIssuers_) * 32;
+  static constexpr int kStageBytes = R::kStageBytes;
+  static constexpr int kStgBytes = kConsumerWarps * 8 * D * 2;   // per-warp output staging [8 heads][D]
+  static constexpr int kInfoBytes = kStages * R::kInfoStride;
+  static constexpr int kBarBytes = 3 * kStages * 8;
+  static constexpr int kPendBytes = 64 * 4;
+  static constexpr int kIdxBytes = 2 * kSeg * 4;
+  static constexpr int kSmem = 128 + kStages * kStageBytes + kStgBytes + kInfoBytes + kBarBytes + kPendBytes + kIdxBytes;
+  static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
+};
+
+template <int HKV, int D, int NSUB>
+__global__ void __launch_bounds__(WideCfg<HKV, D, NSUB>::kThreads, 1) sparse_attn_wide_kernel(AttnArgs a) {
+  using C = WideCfg<HKV, D, NSUB>;
+  using R = typename C::R;
+  constexpr int KS = D / 16;   // k-steps of the score product, m-tiles of the output
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  uint8_t* ring = smem;
+  uint8_t* stg_all = ring + kStages * C::kStageBytes;
+  uint8_t* info = stg_all + C::kStgBytes;
+  auto info_at = [&](int s) { return reinterpret_cast<StageInfo*>(info + s * R::kInfoStride); };
+  uint64_t* full = reinterpret_cast<uint64_t*>(info + C::kInfoBytes);
+  uint64_t* empty = full + kStages;
+  uint64_t* ready = empty + kStages;
+  int* pend = reinterpret_cast<int*>(ready + kStages);
+  int* idxbuf = pend + 64;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int group = a.Hq / HKV;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], C::kConsumerWarps);
+      mbar_init(&ready[s], 1);
+    }
+    fence_mbar_init();
+  }
+  // Zero the ring once so that unused slot rows are finite (they are masked, but 0 * NaN = NaN).
+  for (int i = threadIdx.x; i < kStages * C::kStageBytes / 16; i += blockDim.x)
+    reinterpret_cast<uint4*>(ring)[i] = make_uint4(0, 0, 0, 0);
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // order these writes before the bulk copies
+  __syncthreads();
+
+  if (warp > C::kConsumerWarps) {
+    attn_helper<HKV, D, kWideSlots>(a, warp - C::kConsumerWarps, ring, info, full, ready);
+    return;
+  }
+  if (warp == C::kConsumerWarps) {
+    attn_producer<HKV, D, kWideSlots>(a, ring, info, full, empty, ready, pend, idxbuf);
+    return;
+  }
+
+  // -------------------------------------------------------------------- consumer warps
+  const int g = warp / NSUB;            // KV head
+  const int hs = warp % NSUB;           // head subgroup: heads hs*8 .. hs*8+7 of the group
+  const int nvalid = min(8, group - hs * 8);
+  const int hbase = g * group + hs * 8;
+  const int n_head = lane >> 2;         // head column this lane feeds in the B operand
+  const int cpair = 2 * (lane & 3);     // head columns of this lane's accumulators
+  const uint32_t ring_u32 = smem_u32(ring);
+  // ldmatrix rows: lane & 7 = slot; the other lane bits pick the token parity and the 8-column half
+  const int slot_l = lane & 7;
+  const uint32_t k_off = static_cast<uint32_t>(slot_l * R::kPitch + (((lane >> 3) & 1) * HKV + g) * D * 2 +
+                                               ((lane >> 4) & 1) * 16);
+  const uint32_t v_off = static_cast<uint32_t>(slot_l * R::kPitch + (((lane >> 4) & 1) * HKV + g) * D * 2 +
+                                               ((lane >> 3) & 1) * 16);
+  constexpr uint32_t kTokPair = 2 * HKV * D * 2;   // bytes from tokens {0,1} to tokens {2,3} of a slot
+  uint16_t* stg = reinterpret_cast<uint16_t*>(stg_all) + warp * 8 * D;
+  int st = 0;
+  unsigned ph = 0;
+
+  auto load_q = [&](int item, uint32_t (&f)[KS][2]) {
+    if (item >= a.num_items) return;
+    const long long qrow = a.seqlens == nullptr
+                               ? static_cast<long long>(item % a.B) * a.Tq + (a.Tq - 1 - item / a.B)
+                               : static_cast<long long>(item / a.splits);
+    const bool hv = n_head < nvalid;
+    const uint16_t* qp = a.q + (qrow * a.Hq + (hv ? hbase + n_head : 0)) * D;
+#pragma unroll
+    for (int kk = 0; kk < KS; ++kk) {
+      const int d0 = 16 * kk + cpair;
+      f[kk][0] = hv ? *reinterpret_cast<const uint32_t*>(qp + d0) : 0u;
+      f[kk][1] = hv ? *reinterpret_cast<const uint32_t*>(qp + d0 + 8) : 0u;
+    }
+  };
+  uint32_t qf[KS][2];
+  load_q(blockIdx.x, qf);
+
+  for (int item = blockIdx.x; item < a.num_items; item += gridDim.x) {
+    const Item it = make_item<HKV, D>(a, item);
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+    float o[KS][4];
+#pragma unroll
+    for (int mt = 0; mt < KS; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+
+    for (;;) {
+      if (!mbar_wait(&full[st], ph, a.ctl)) return;
+      const int ns = info_at(st)->nslots;
+      const bool last = info_at(st)->last != 0;
+      if (ns > 0) {
+        const uint32_t kst = ring_u32 + st * C::kStageBytes;
+        const uint32_t vst = kst + kWideSlots * R::kPitch;
+        float acc[2][4];
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+#pragma unroll
+          for (int kk = 0; kk < KS; ++kk) {
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4(kst + k_off + t * kTokPair + kk * 32, a0, a1, a2, a3);
+            mma_bf16_16816(acc[t], a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
+          }
+        }
+        // rows: r0 = slot lane>>2 at token 2t, r1 = the same slot at token 2t + 1
+        const int sr = lane >> 2;
+        const int ntk = sr < ns ? info_at(st)->ntok[sr] : 0;
+        float x[2][4];
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          const bool v0 = 2 * t < ntk, v1 = 2 * t + 1 < ntk;
+          x[t][0] = v0 ? acc[t][0] * a.scale_log2 : -INFINITY;
+          x[t][1] = v0 ? acc[t][1] * a.scale_log2 : -INFINITY;
+          x[t][2] = v1 ? acc[t][2] * a.scale_log2 : -INFINITY;
+          x[t][3] = v1 ? acc[t][3] * a.scale_log2 : -INFINITY;
+        }
+        float t0 = fmaxf(fmaxf(x[0][0], x[0][2]), fmaxf(x[1][0], x[1][2]));
+        float t1 = fmaxf(fmaxf(x[0][1], x[0][3]), fmaxf(x[1][1], x[1][3]));
+#pragma unroll
+        for (int o2 = 4; o2 < 32; o2 <<= 1) {
+          t0 = fmaxf(t0, __shfl_xor_sync(0xffffffffu, t0, o2));
+          t1 = fmaxf(t1, __shfl_xor_sync(0xffffffffu, t1, o2));
+        }
+        const float mn0 = fmaxf(m0, t0), mn1 = fmaxf(m1, t1);
+        const float ref0 = mn0 == -INFINITY ? 0.f : mn0;
+        const float ref1 = mn1 == -INFINITY ? 0.f : mn1;
+        const float al0 = exp2f(m0 - ref0), al1 = exp2f(m1 - ref1);
+        float p[2][4];
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          p[t][0] = exp2f(x[t][0] - ref0);
+          p[t][1] = exp2f(x[t][1] - ref1);
+          p[t][2] = exp2f(x[t][2] - ref0);
+          p[t][3] = exp2f(x[t][3] - ref1);
+        }
+        l0 = l0 * al0 + (p[0][0] + p[0][2] + p[1][0] + p[1][2]);
+        l1 = l1 * al1 + (p[0][1] + p[0][3] + p[1][1] + p[1][3]);
+        m0 = mn0;
+        m1 = mn1;
+#pragma unroll
+        for (int mt = 0; mt < KS; ++mt) {
+          o[mt][0] *= al0;
+          o[mt][1] *= al1;
+          o[mt][2] *= al0;
+          o[mt][3] *= al1;
+        }
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          const uint32_t b0 = movmatrix_t(pack_bf16x2(p[t][0], p[t][1]));
+          const uint32_t b1 = movmatrix_t(pack_bf16x2(p[t][2], p[t][3]));
+#pragma unroll
+          for (int mt = 0; mt < KS; ++mt) {
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4_t(vst + v_off + t * kTokPair + mt * 32, a0, a1, a2, a3);
+            mma_bf16_16816(o[mt], a0, a1, a2, a3, b0, b1);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st]);
+      if (++st == kStages) {
+        st = 0;
+        ph ^= 1u;
+      }
+      if (last) break;
+    }
+
+    load_q(item + gridDim.x, qf);   // the next item's query (its latency overlaps the epilogue)
+    // ---- item epilogue: full row sums, then the output of this warp's heads
+#pragma unroll
+    for (int o2 = 4; o2 < 32; o2 <<= 1) {
+      l0 += __shfl_xor_sync(0xffffffffu, l0, o2);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, o2);
+    }
+    if (!it.partial) {
+      const float inv0 = l0 > 0.f ? 1.f / l0 : 0.f, inv1 = l1 > 0.f ? 1.f / l1 : 0.f;
+#pragma unroll
+      for (int mt = 0; mt < KS; ++mt) {
+        const int d = 16 * mt + (lane >> 2);
+        stg[cpair * D + d] = __bfloat16_as_ushort(__float2bfloat16_rn(o[mt][0] * inv0));
+        stg[(cpair + 1) * D + d] = __bfloat16_as_ushort(__float2bfloat16_rn(o[mt][1] * inv1));
+        stg[cpair * D + d + 8] = __bfloat16_as_ushort(__float2bfloat16_rn(o[mt][2] * inv0));
+        stg[(cpair + 1) * D + d + 8] = __bfloat16_as_ushort(__float2bfloat16_rn(o[mt][3] * inv1));
+      }
+      __syncwarp();
+      uint16_t* orow = a.out + (it.orow * a.Hq + hbase) * D;
+      const int chunks = nvalid * D / 8;   // 16-byte chunks of this warp's output heads
+      for (int c = lane; c < chunks; c += 32)
+        reinterpret_cast<uint4*>(orow)[c] = reinterpret_cast<const uint4*>(stg)[c];
+      if (a.lse && lane < 4) {
+        if (cpair < nvalid) a.lse[it.orow * a.Hq + hbase + cpair] = l0 > 0.f ? (m0 + __log2f(l0)) * kLn2 : -INFINITY;
+        if (cpair + 1 < nvalid)
+          a.lse[it.orow * a.Hq + hbase + cpair + 1] = l1 > 0.f ? (m1 + __log2f(l1)) * kLn2 : -INFINITY;
+      }
+      __syncwarp();
+    } else {
+      // unnormalised partial: part[item][h][0..D) = o, part[item][h][D] = m (log2 units), [D+1] = l
+      float* prow = a.part + it.orow * a.Hq * (D + 2);
+#pragma unroll
+      for (int mt = 0; mt < KS; ++mt) {
+        const int d = 16 * mt + (lane >> 2);
+        if (cpair < nvalid) {
+          prow[(hbase + cpair) * (D + 2) + d] = o[mt][0];
+          prow[(hbase + cpair) * (D + 2) + d + 8] = o[mt][2];
+        }
+        if (cpair + 1 < nvalid) {
+          prow[(hbase + cpair + 1) * (D + 2) + d] = o[mt][1];
+          prow[(hbase + cpair + 1) * (D + 2) + d + 8] = o[mt][3];
+        }
+      }
+      if (lane < 4) {
+        if (cpair < nvalid) {
+          prow[(hbase + cpair) * (D + 2) + D] = m0;
+          prow[(hbase + cpair) * (D + 2) + D + 1] = l0;
+        }
+        if (cpair + 1 < nvalid) {
+          prow[(hbase + cpair + 1) * (D + 2) + D] = m1;
+          prow[(hbase + cpair + 1) * (D + 2) + D + 1] = l1;
+        }
+      }
+    }
+  }
+}
+
+// Merge of decode splits: out[b][h] = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s.  One thread per
+// element of the head dimension D (blockDim.x == D).
+__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ part, int splits, int Hq, int D,
                                                       uint16_t* __restrict__ out, float* __restrict__ lse) {
   const int b = blockIdx.x, h = blockIdx.y, d = threadIdx.x;
-  const float* p = part + (static_cast<long long>(b) * splits * Hq + h) * (kD + 2);
-  const long long step = static_cast<long long>(Hq) * (kD + 2);
+  const float* p = part + (static_cast<long long>(b) * splits * Hq + h) * (D + 2);
+  const long long step = static_cast<long long>(Hq) * (D + 2);
   float M = -INFINITY;
-  for (int s = 0; s < splits; ++s) M = fmaxf(M, p[s * step + kD]);
+  for (int s = 0; s < splits; ++s) M = fmaxf(M, p[s * step + D]);
   const float R = M == -INFINITY ? 0.f : M;
   float acc = 0.f, l = 0.f;
   for (int s = 0; s < splits; ++s) {
-    const float f = exp2f(p[s * step + kD] - R);
+    const float f = exp2f(p[s * step + D] - R);
     acc += f * p[s * step + d];
-    l += f * p[s * step + kD + 1];
+    l += f * p[s * step + D + 1];
   }
-  out[(static_cast<long long>(b) * Hq + h) * kD + d] = __bfloat16_as_ushort(__float2bfloat16_rn(l > 0.f ? acc / l : 0.f));
+  out[(static_cast<long long>(b) * Hq + h) * D + d] = __bfloat16_as_ushort(__float2bfloat16_rn(l > 0.f ? acc / l : 0.f));
   if (lse && d == 0) lse[static_cast<long long>(b) * Hq + h] = l > 0.f ? (M + __log2f(l)) * kLn2 : -INFINITY;
 }
 
@@ -581,11 +865,39 @@ cudaError_t launch_attn(const DeviceInfo* di, AttnArgs a, cudaStream_t s) {
   return cudaPeekAtLastError();
 }
 
+template <int HKV, int D, int NSUB>
+cudaError_t launch_attn_wide_cfg(const DeviceInfo* di, AttnArgs a, cudaStream_t s) {
+  using C = WideCfg<HKV, D, NSUB>;
+  static std::once_flag once[64];
+  std::call_once(once[di->device & 63], [] {
+    cudaFuncSetAttribute(sparse_attn_wide_kernel<HKV, D, NSUB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         C::kSmem);
+  });
+  const int grid = std::min(a.num_items, di->num_sms);
+  if (grid <= 0) return cudaSuccess;
+  sparse_attn_wide_kernel<HKV, D, NSUB><<<grid, C::kThreads, C::kSmem, s>>>(a);
+  return cudaPeekAtLastError();
+}
+
+// D = 128 with groups of up to 8 heads takes the 16-slot kernel; D = 256, or groups of 9 .. 16,
+// the wide one.
+cudaError_t launch_attn_any(const DeviceInfo* di, AttnArgs a, int Hkv, int D, cudaStream_t s) {
+  const int group = a.Hq / Hkv;
+  if (D == kD && group <= 8) return Hkv == 1 ? launch_attn<1>(di, a, s) : launch_attn<2>(di, a, s);
+  const int nsub = group <= 8 ? 1 : 2;
+  if (D == 128) {
+    if (Hkv == 1) return nsub == 1 ? launch_attn_wide_cfg<1, 128, 1>(di, a, s) : launch_attn_wide_cfg<1, 128, 2>(di, a, s);
+    return nsub == 1 ? launch_attn_wide_cfg<2, 128, 1>(di, a, s) : launch_attn_wide_cfg<2, 128, 2>(di, a, s);
+  }
+  if (Hkv == 1) return nsub == 1 ? launch_attn_wide_cfg<1, 256, 1>(di, a, s) : launch_attn_wide_cfg<1, 256, 2>(di, a, s);
+  return nsub == 1 ? launch_attn_wide_cfg<2, 256, 1>(di, a, s) : launch_attn_wide_cfg<2, 256, 2>(di, a, s);
+}
+
 }  // namespace
 
 cudaError_t launch_attn_prefill(const DeviceInfo* di, const void* q, const void* k, const void* v, const int32_t* idx,
-                                int B, int Tq, int Tk, int Hq, int Hkv, int k_blocks, long long q_pos0, float scale,
-                                void* out, float* lse, cudaStream_t s) {
+                                int B, int Tq, int Tk, int Hq, int Hkv, int D, int k_blocks, long long q_pos0,
+                                float scale, void* out, float* lse, cudaStream_t s) {
   AttnArgs a{};
   a.q = static_cast<const uint16_t*>(q);
   a.k = static_cast<const uint16_t*>(k);
@@ -605,7 +917,7 @@ cudaError_t launch_attn_prefill(const DeviceInfo* di, const void* q, const void*
   a.num_items = B * Tq;
   a.scale_log2 = scale * kLog2e;
   a.ctl = kernel_ctl(di);
-  return Hkv == 1 ? launch_attn<1>(di, a, s) : launch_attn<2>(di, a, s);
+  return launch_attn_any(di, a, Hkv, D, s);
 }
 
 int decode_default_splits(const DeviceInfo* di, int B, int k_blocks) {
@@ -616,7 +928,7 @@ int decode_default_splits(const DeviceInfo* di, int B, int k_blocks) {
 }
 
 cudaError_t launch_attn_decode(const DeviceInfo* di, const void* q, const void* kc, const void* vc,
-                               const int32_t* seqlens, const int32_t* idx, int B, int Lmax, int Hq, int Hkv,
+                               const int32_t* seqlens, const int32_t* idx, int B, int Lmax, int Hq, int Hkv, int D,
                                int k_blocks, float scale, int num_splits, void* out, float* lse, float* part,
                                cudaStream_t s) {
   AttnArgs a{};
@@ -638,9 +950,9 @@ cudaError_t launch_attn_decode(const DeviceInfo* di, const void* q, const void* 
   a.num_items = B * num_splits;
   a.scale_log2 = scale * kLog2e;
   a.ctl = kernel_ctl(di);
-  cudaError_t e = Hkv == 1 ? launch_attn<1>(di, a, s) : launch_attn<2>(di, a, s);
+  cudaError_t e = launch_attn_any(di, a, Hkv, D, s);
   if (e != cudaSuccess || num_splits <= 1) return e;
-  combine_kernel<<<dim3(B, Hq), kD, 0, s>>>(part, num_splits, Hq, static_cast<uint16_t*>(out), lse);
+  combine_kernel<<<dim3(B, Hq), D, 0, s>>>(part, num_splits, Hq, D, static_cast<uint16_t*>(out), lse);
   return cudaPeekAtLastError();
 }
 

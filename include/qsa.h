@@ -205,7 +205,11 @@ QSA_API qsa_status_t qsa_select_topk(const float* scores, int64_t ld_scores, con
  *   o(t,h) = sum_{j in S(t)} softmax_j(scale * q(t,h) . k(j,g)) v(j,g),  g = h / (Hq/Hkv),
  *   S(t) = tokens of the listed blocks  U  { blk*floor(p/blk) .. p }.
  * The softmax is kept in fp32 (online, exp2 form); products run on bf16 tensor cores.
- * Errors: INVALID_ARGUMENT, UNSUPPORTED (D != 128, Hkv not in {1,2}, Hq/Hkv > 8, blk != 4).
+ * Shapes: D = 128 or 256, Hkv = 1 or 2, Hq/Hkv up to 16 -- the benchmark shape (16 query heads
+ * over 2 KV heads, D = 128) and the model shape of "Qwen3.8-Flash-Next architecture" (flozi.net),
+ * "Der Weg eines Tokens durch das Modell" (24 query heads over 2 KV heads, D = 256).
+ * Errors: INVALID_ARGUMENT, UNSUPPORTED (D not in {128, 256}, Hkv not in {1,2}, Hq/Hkv > 16,
+ * blk != 4).
  */
 QSA_API qsa_status_t qsa_sparse_attn_prefill(const void* q, const void* k, const void* v,
                                      const int32_t* idx, int B, int Tq, int Tk, int Hq, int Hkv,

@@ -91,7 +91,10 @@ def test_select_and_attention_argument_checks(lib):
         FAKE, FAKE, FAKE, FAKE, 1, Tq, Tk, Hq, Hkv, D, 8, blk, q0, ctypes.c_float(0.1), FAKE, None, None)
     assert pre(D=64) == Q.QSA_ERR_UNSUPPORTED
     assert pre(Hkv=4, Hq=16) == Q.QSA_ERR_UNSUPPORTED
-    assert pre(Hq=24, Hkv=2) == Q.QSA_ERR_UNSUPPORTED        # group of 12: the d=256 / 24-head shape is not built
+    assert pre(Hq=34, Hkv=2) == Q.QSA_ERR_UNSUPPORTED        # groups of more than 16 query heads
+    assert pre(D=512) == Q.QSA_ERR_UNSUPPORTED
+    # the model shape (24 query heads over 2 KV heads at head dimension 256) passes the shape checks
+    assert pre(Hq=24, Hkv=2, D=256) not in (Q.QSA_ERR_UNSUPPORTED, Q.QSA_ERR_INVALID_ARGUMENT)
     assert pre(Hq=15, Hkv=2) == Q.QSA_ERR_INVALID_ARGUMENT
     assert pre(blk=8) == Q.QSA_ERR_UNSUPPORTED
     assert pre(q0=4) == Q.QSA_ERR_INVALID_ARGUMENT           # q0 + Tq > Tk
