@@ -380,7 +380,7 @@ def run_qsa(args):
     # ---------------------------------------------------------------- decode leg
     decode = None
     if not args.no_decode:
-        wd = I.WORKLOADS[DECODE].with_(seed=I.WORKLOADS[DECODE].seed + 1000 * rank)
+        wd = I.WORKLOADS[args.decode_workload].with_(seed=I.WORKLOADS[args.decode_workload].seed + 1000 * rank)
         xd = I.make_decode(wd, dev)
         nbd = wd.T // wd.blk
         kpd = Q.qsa_pool_block_keys(xd["ki"])
@@ -430,7 +430,8 @@ def run_qsa(args):
         d_att = statistics.mean(e[1].elapsed_time(e[2]) for e in devs)
         dw = decode_work(wd)
         dgbs = dw["bytes"] / (dms / 1000) / 1e9
-        decode = {"workload": DECODE, "value": world * wd.B / (dms / 1000), "unit": "tokens/s", "ms_per_step": dms,
+        decode = {"workload": args.decode_workload, "value": world * wd.B / (dms / 1000), "unit": "tokens/s",
+                  "ms_per_step": dms,
                   "steps": dsteps, "num_splits": splits,
                   "step_breakdown_ms": {"score_topk": d_sel, "attention_and_merge": d_att},
                   "gpu_launches_per_step": 1 + 2 + 1 + (1 if splits > 1 else 0),
@@ -516,6 +517,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-indexer", action="store_true", help="skip the stand-alone indexer timing (17 GB of scores)")
     ap.add_argument("--no-dense", action="store_true", help="skip timing dense causal attention on the same inputs")
+    ap.add_argument("--decode-workload", default=DECODE,
+                    choices=[n for n, w in I.WORKLOADS.items() if w.kind == "decode"],
+                    help="decode workload of the second leg (default: 32 sequences of 256K tokens)")
     ap.add_argument("--workload", default=PREFILL, choices=[n for n, w in I.WORKLOADS.items() if w.kind == "prefill"],
                     help="prefill workload of the headline leg (default: the 128K configuration)")
     args = ap.parse_args()
