@@ -272,6 +272,17 @@ struct FilterArgs {
   KernelCtl ctl;
 };
 
+// A predicated 8-byte store: no branch around it, so a warp's stores of a query issue as one
+// instruction whatever the lanes' predicates.
+__device__ __forceinline__ void st_global_v2_if(bool pred, uint2* addr, uint32_t x, uint32_t y) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %0, 0;\n\t"
+      "@p st.global.v2.u32 [%1], {%2, %3};\n\t}" ::"r"(static_cast<uint32_t>(pred)),
+      "l"(addr), "r"(x), "r"(y)
+      : "memory");
+}
+
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
@@ -456,8 +467,9 @@ __global__ void __launch_bounds__(kFiltThreads, 1)
 #pragma unroll
       for (int q = 0; q < QW; ++q) {
         const uint32_t p = offs[q] + static_cast<uint32_t>(__popc(m[q] & lt));
-        if ((m[q] & lane_bit) && p < static_cast<uint32_t>(a.cap))
-          list_q0[static_cast<long long>(q) * a.cap + p] = make_uint2(__float_as_uint(sc[q]), static_cast<uint32_t>(kb));
+        const uint32_t e = static_cast<uint32_t>(q) * static_cast<uint32_t>(a.cap) + p;   // < QW * cap
+        st_global_v2_if((m[q] & lane_bit) != 0u && p < static_cast<uint32_t>(a.cap), list_q0 + e,
+                        __float_as_uint(sc[q]), static_cast<uint32_t>(kb));
       }
       __syncwarp();   // my_off is rewritten by the next tile
     }
