@@ -32,7 +32,8 @@ constexpr int kN = 256;          // indexer rows per tile (UMMA N)
 constexpr int kDi = 64;          // contraction depth (one 128-byte swizzle row)
 constexpr int kStages = 4;       // kp ring depth
 constexpr int kTilesPerCta = 16; // kp tiles handled by one CTA (split of long rows)
-constexpr int kScoreThreads = 320;
+constexpr int kScoreEpiWarps = 16;   // epilogue warps: four per TMEM lane quadrant
+constexpr int kScoreThreads = 64 + kScoreEpiWarps * 32;
 constexpr int kQiBytes = kN * kDi * 2;   // 32768
 constexpr int kKpBytes = kM * kDi * 2;   // 16384
 constexpr int kScoreSmem = 1024 + kQiBytes + kStages * kKpBytes + 256 + 16384;  // last term: keep 1 CTA/SM
@@ -149,7 +150,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tm_full[i], 1);
-      mbar_init(&tm_empty[i], 8);
+      mbar_init(&tm_empty[i], kScoreEpiWarps);
     }
     mbar_init(mma_done, 1);
     fence_mbar_init();
@@ -172,9 +173,10 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
       issue_tile_mmas(tmem, qi_s, kp_s, qi_full, kp_full, kp_empty, tm_full, tm_empty, mma_done, nt, a.ctl);
     __syncwarp();
   } else {
-    const int ew = warp - 2;                 // 0..7
+    const int ew = warp - 2;                 // 0 .. kScoreEpiWarps - 1
     const int quad = warp & 3;               // TMEM lane quadrant this warp may read
-    const int colbase = (ew >> 2) * (kN / 2);
+    constexpr int CW = kN / (kScoreEpiWarps / 4);   // columns of this warp: one column group
+    const int colbase = (ew >> 2) * CW;
     const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
     float w[HI];
 #pragma unroll
@@ -194,13 +196,18 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
       tc_fence_after();
       const int kb = (t_begin + i) * kM + quad * 32 + lane;   // pooled key owned by this thread
       float* col = srow + kb;
-#pragma unroll 1
-      for (int c = 0; c < kN / 2; c += 32) {
+#pragma unroll
+      for (int c = 0; c < CW; c += 32) {
         uint32_t r[32];
         tmem_ld_32x32(tmem + lane_addr + acc * kN + colbase + c, r);
         tmem_ld_wait();
         const int q0 = (colbase + c) / HI;
-        float sc[32 / HI];
+        // Queries q0 .. q0 + 32/HI - 1 of the tile: when all of them exist and see every pooled key
+        // of this warp, the stores need no mask (all tiles below the diagonal band).
+        float* dst = col + static_cast<long long>(q0) * ld;
+        const bool full =
+            q0 + 32 / HI - 1 <= tl_last &&
+            (t_begin + i) * kM + quad * 32 + 31 < visible_cols(min(nbk, static_cast<int>((pos_first + q0) >> 2)), ksh, kof);
 #pragma unroll
         for (int qq = 0; qq < 32 / HI; ++qq) {
           float acc_s = 0.0f;
@@ -210,28 +217,13 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
             if (MODE == 0) x = fmaxf(x, 0.0f);
             acc_s = fmaf(w[h], x, acc_s);
           }
-          sc[qq] = acc_s;
-        }
-        // Queries q0 .. q0 + 32/HI - 1 of the tile: when all of them exist and see every pooled key
-        // of this warp, the stores need no mask (all tiles below the diagonal band).
-        float* dst = col + static_cast<long long>(q0) * ld;
-        const bool full =
-            q0 + 32 / HI - 1 <= tl_last &&
-            (t_begin + i) * kM + quad * 32 + 31 < visible_cols(min(nbk, static_cast<int>((pos_first + q0) >> 2)), ksh, kof);
-        if (full) {
-#pragma unroll
-          for (int qq = 0; qq < 32 / HI; ++qq) {
-            *dst = sc[qq];
-            dst += ld;
-          }
-        } else {
-#pragma unroll
-          for (int qq = 0; qq < 32 / HI; ++qq) {
+          bool ok = full;
+          if (!full) {   // warp-uniform
             const int tl = q0 + qq;
-            const int nbq = visible_cols(min(nbk, static_cast<int>((pos_first + tl) >> 2)), ksh, kof);
-            if (tl <= tl_last && kb < nbq) *dst = sc[qq];
-            dst += ld;
+            ok = tl <= tl_last && kb < visible_cols(min(nbk, static_cast<int>((pos_first + tl) >> 2)), ksh, kof);
           }
+          if (ok) *dst = acc_s;
+          dst += ld;
         }
       }
       tc_fence_before();
