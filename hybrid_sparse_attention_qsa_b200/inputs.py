@@ -62,6 +62,8 @@ WORKLOADS = {
     # dimension 256) with the 128K recipe otherwise
     "prefill_128k_model": Workload("prefill_128k_model", "prefill", B=1, T=131072, Hq=24, Hkv=2, D=256, Hi=4, Di=64,
                                    blk=4, k=512, seed=5, boost_frac=0.05, boost=4.0),
+    "prefill_32k_model": Workload("prefill_32k_model", "prefill", B=1, T=32768, Hq=24, Hkv=2, D=256, Hi=4, Di=64,
+                                  blk=4, k=512, seed=7, boost_frac=0.05, boost=4.0),
 }
 
 
