@@ -234,7 +234,11 @@ __device__ void topk_global(const float* s, int n, int k, int32_t* out, uint32_t
   }
 }
 
-__global__ void __launch_bounds__(kTopkThreads, 3) topk_kernel(const float* __restrict__ scores, long long ld,
+// KU: 16-byte loads per thread in flight in the filter pass.  Launches with fewer rows than SMs
+// (decode) take KU = 16 at one CTA per SM, so a long row is read in few round trips; many-row
+// launches keep KU small for three CTAs per SM.
+template <int KU, int MINB>
+__global__ void __launch_bounds__(kTopkThreads, MINB) topk_kernel(const float* __restrict__ scores, long long ld,
                                                             long long batch_stride, const int32_t* __restrict__ seqlens,
                                                             int Tq, int NBk, int blk, long long q_pos0, int b0,
                                                             int row0, int k, int32_t* __restrict__ idx,
@@ -320,7 +324,7 @@ __global__ void __launch_bounds__(kTopkThreads, 3) topk_kernel(const float* __re
       // tau back to the float it orders like (keys of finite floats are never 0x7FFFFFFF..0)
       const float tau_f = __uint_as_float((tau & 0x80000000u) ? (tau & 0x7FFFFFFFu) : ~tau);
       // kU independent 16-byte loads per thread are in flight before any of them is used.
-      constexpr int kU = QSA_TOPK_LOADS;
+      constexpr int kU = KU;
       for (int base = 0; base < n; base += 4 * kTopkThreads * kU) {
         float v[kU][4];
 #pragma unroll
@@ -774,7 +778,9 @@ cudaError_t launch_topk(const DeviceInfo* di, const float* scores, long long ld,
   if (rows <= 0 || nb <= 0) return cudaSuccess;
   static std::once_flag once[64];
   std::call_once(once[di->device & 63], [] {
-    cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaFuncSetAttribute(topk_kernel<QSA_TOPK_LOADS, 3>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         kFixedSmem + 32 + kMaxBitmapWords * 4);
+    cudaFuncSetAttribute(topk_kernel<16, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          kFixedSmem + 32 + kMaxBitmapWords * 4);
   });
   // Many short rows (early prefill chunks): one warp per row.  Long rows or few rows (late chunks,
@@ -796,8 +802,12 @@ cudaError_t launch_topk(const DeviceInfo* di, const float* scores, long long ld,
   const int words = std::min(kMaxBitmapWords, (std::max(NBk, 1) + 31) / 32);
   const int smem = kFixedSmem + 32 + words * 4;
   dim3 grid(rows, nb);
-  topk_kernel<<<grid, kTopkThreads, smem, s>>>(scores, ld, batch_stride, seqlens, Tq, NBk, blk, q_pos0, b0, row0, k,
-                                               idx, words, kernel_ctl(di));
+  if (static_cast<long long>(rows) * nb < di->num_sms)
+    topk_kernel<16, 1><<<grid, kTopkThreads, smem, s>>>(scores, ld, batch_stride, seqlens, Tq, NBk, blk, q_pos0, b0,
+                                                         row0, k, idx, words, kernel_ctl(di));
+  else
+    topk_kernel<QSA_TOPK_LOADS, 3><<<grid, kTopkThreads, smem, s>>>(scores, ld, batch_stride, seqlens, Tq, NBk, blk,
+                                                                     q_pos0, b0, row0, k, idx, words, kernel_ctl(di));
   return cudaPeekAtLastError();
 }
 
