@@ -84,7 +84,7 @@ FusedPlan fused_plan(int NBk, int k) {
   p.ns = NBk > kSampleOff ? ((NBk - kSampleOff - 1) >> kSampleShift) + 1 : 0;
   p.ld_s = (std::max(p.ns, 1) + 3) & ~3;
   p.per_row = static_cast<long long>(p.ld_s) * 4 + 12 + static_cast<long long>(p.cap) * 8;
-  p.fixed = 6 * 256 + 4 + static_cast<long long>(kFallbackCtas) * std::max(NBk, 1) * 4;
+  p.fixed = 12 * 256 + 4 + static_cast<long long>(kFallbackCtas) * std::max(NBk, 1) * 4;
   return p;
 }
 long long fused_rows_fit(const FusedPlan& p, size_t ws_bytes) {
@@ -306,7 +306,7 @@ qsa_status_t qsa_select_topk(const float* scores, int64_t ld_scores, const void*
             e = launch_score_filter(di, qib, kpb, head_w, Tq, NBk, Hi, q_pos0, mode, 0, 1, r0, rows, tau, cand, cnt,
                                     fp.cap, s);
           if (e == cudaSuccess)
-            e = launch_select_candidates(di, cand, cnt, fp.cap, Tq, NBk, q_pos0, b, r0, rows, k, idx, fail, s);
+            e = launch_select_candidates(di, cand, cnt, fp.cap, Tq, NBk, q_pos0, b, r0, rows, k, idx, fail, 0, s);
           if (e == cudaSuccess)
             e = launch_topk_fallback(di, qi, kp, head_w, Hi, mode, Tq, NBk, q_pos0, b, fail, scratch, kFallbackCtas, k,
                                      idx, s);

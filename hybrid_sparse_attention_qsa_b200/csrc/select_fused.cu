@@ -198,15 +198,11 @@ __device__ void fail_row(int* fail, int t) {
 }
 
 template <int U>
-__global__ void __launch_bounds__(kSelThreads) cand_select_kernel(const uint2* __restrict__ cand,
-                                                                  const int* __restrict__ cnt, int cap, int Tq, int NBk,
-                                                                  long long q_pos0, int b, int row0, int k,
-                                                                  int32_t* __restrict__ idx, int* __restrict__ fail) {
-  __shared__ __align__(16) uint32_t hist[kSelBins];   // histogram, then the k-th bin's keys
-  __shared__ uint32_t ws[2 * kSelWarpsPerRow];
-  __shared__ uint32_t sel[4];
+__device__ __forceinline__ void select_row(const uint2* __restrict__ cand, const int* __restrict__ cnt, int cap,
+                                           int Tq, int NBk, long long q_pos0, int b, int row0, int k,
+                                           int32_t* __restrict__ idx, int* __restrict__ fail, int L, uint32_t* hist,
+                                           uint32_t* ws, uint32_t* sel) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int L = static_cast<int>(blockIdx.x);
   const int t = row0 + L;
   const int n = static_cast<int>(min(static_cast<long long>(NBk), (q_pos0 + t) >> 2));
   int32_t* out = idx + (static_cast<long long>(b) * Tq + t) * k;
@@ -392,6 +388,21 @@ __global__ void __launch_bounds__(kSelThreads) cand_select_kernel(const uint2* _
   }
 }
 
+// One CTA per row, or a persistent grid of fewer CTAs that walks the rows (so that it can run beside
+// the next chunk's score + filter kernel, one CTA per SM).
+template <int U>
+__global__ void __launch_bounds__(kSelThreads) cand_select_kernel(const uint2* __restrict__ cand,
+                                                                  const int* __restrict__ cnt, int cap, int Tq, int NBk,
+                                                                  long long q_pos0, int b, int row0, int rows, int k,
+                                                                  int32_t* __restrict__ idx, int* __restrict__ fail) {
+  __shared__ __align__(16) uint32_t hist[kSelBins];   // histogram, then the k-th bin's keys
+  __shared__ uint32_t ws[2 * kSelWarpsPerRow];
+  __shared__ uint32_t sel[4];
+  for (int L = static_cast<int>(blockIdx.x); L < rows; L += static_cast<int>(gridDim.x)) {
+    select_row<U>(cand, cnt, cap, Tq, NBk, q_pos0, b, row0, k, idx, fail, L, hist, ws, sel);
+    __syncthreads();   // the next row reuses the shared memory
+  }
+}
 
 }  // namespace
 
@@ -406,15 +417,16 @@ cudaError_t launch_select_tau(const DeviceInfo* di, const float* samp, long long
 
 cudaError_t launch_select_candidates(const DeviceInfo* di, const uint2* cand, const int* cnt, int cap, int Tq, int NBk,
                                      long long q_pos0, int b, int row0, int rows, int k, int32_t* idx, int* fail,
-                                     cudaStream_t s) {
+                                     int max_ctas, cudaStream_t s) {
   (void)di;
   if (rows <= 0) return cudaSuccess;
   // lists of up to 2 * U * kSelThreads entries fit the registers; longer ones are refused (the
   // caller only plans caps that fit)
+  const int grid = max_ctas > 0 ? std::min(rows, max_ctas) : rows;
   if (cap <= 2 * 10 * kSelThreads)
-    cand_select_kernel<10><<<rows, kSelThreads, 0, s>>>(cand, cnt, cap, Tq, NBk, q_pos0, b, row0, k, idx, fail);
+    cand_select_kernel<10><<<grid, kSelThreads, 0, s>>>(cand, cnt, cap, Tq, NBk, q_pos0, b, row0, rows, k, idx, fail);
   else if (cap <= 2 * 20 * kSelThreads)
-    cand_select_kernel<20><<<rows, kSelThreads, 0, s>>>(cand, cnt, cap, Tq, NBk, q_pos0, b, row0, k, idx, fail);
+    cand_select_kernel<20><<<grid, kSelThreads, 0, s>>>(cand, cnt, cap, Tq, NBk, q_pos0, b, row0, rows, k, idx, fail);
   else
     return cudaErrorInvalidValue;
   return cudaPeekAtLastError();

@@ -111,7 +111,7 @@ def filtered_bytes(rows, nbk, k):
     rank = max(64, (5 * k + 31) // 32)
     ns = (nbk - 9) // 16 + 1 if nbk > 8 else 0
     per_row = ((max(ns, 1) + 3) // 4 * 4) * 4 + 12 + 32 * rank * 8
-    return 6 * 256 + 4 + 128 * max(nbk, 1) * 4 + rows * per_row
+    return 12 * 256 + 4 + 128 * max(nbk, 1) * 4 + rows * per_row
 
 
 def test_workspace_sizes(lib):

@@ -98,7 +98,7 @@ def test_filtered_in_chunks_with_offset():
     rank = max(64, (5 * k + 31) // 32)
     ns = (nbk - 9) // 16 + 1
     per_row = ((ns + 3) // 4 * 4) * 4 + 12 + 32 * rank * 8
-    ws = torch.empty(6 * 256 + 4 + 128 * nbk * 4 + 3000 * per_row, dtype=torch.uint8, device=DEV)
+    ws = torch.empty(12 * 256 + 4 + 128 * nbk * 4 + 3000 * per_row, dtype=torch.uint8, device=DEV)
     fil = _select(Q.QSA_SELECT_FILTERED, 0, qi, kp, k, q_pos0=pos0, workspace=ws)
     assert np.array_equal(mat, fil)
 
@@ -133,3 +133,4 @@ def test_unsupported_head_count_is_refused():
     Q.qsa_set_select_options(Q.QSA_SELECT_FILTERED, 0)
     with pytest.raises(Q.QSAError):
         Q.qsa_select_topk(64, qi=qi, kp=kp)
+
