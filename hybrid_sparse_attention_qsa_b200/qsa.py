@@ -366,7 +366,7 @@ def _copy_stream(device, which: str = "in") -> "torch.cuda.Stream":
 
 def prefill_host(q, k, v, qi, ki, *, topk: int, device="cuda", out=None, q_pos0: int = 0, rope_theta: float = 0.0,
                  head_w=None, mode: int = QSA_SCORE_RELU_SUM, scale: float | None = None, workspace=None,
-                 device_buffers: dict | None = None, chunks: int = 8, yarn=None):
+                 device_buffers: dict | None = None, chunks: int = 32, yarn=None):
     """The QSA layer for a prefill whose inputs live in (pinned) host memory; returns the output in
     host memory.  Transfers overlap the kernels.  ki and qi are copied first and the pooling and
     block selection of all rows run while q, k and v follow in ``chunks`` causal row chunks on a
