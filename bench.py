@@ -396,42 +396,61 @@ def run_qsa(args):
         ki_last = xd["ki"][:, j * wd.blk:(j + 1) * wd.blk]
         kp_last = kpd[:, j:j + 1]
 
-        def dstep(ev=None):
+        def dsel():
             if (wd.T % wd.blk) == 0:       # the new token completed block j: pool that row of every sequence
                 Q.qsa_pool_block_keys(ki_last, kp_last, pos0=j * wd.blk)
-            if ev:
-                ev[0].record(stream)
             Q.qsa_select_topk(wd.k, qi=xd["qi"], kp=kpd, seqlens=xd["seqlens"], idx=idxd, workspace=wsd)
-            if ev:
-                ev[1].record(stream)
+
+        def datt():
             Q.qsa_sparse_attn_decode(xd["q"], xd["k"], xd["v"], xd["seqlens"], idxd, num_splits=splits, out=outd,
                                      lse=lsed, workspace=wsa)
-            if ev:
-                ev[2].record(stream)
 
         for _ in range(max(args.warmup, 3)):
-            dstep()
+            dsel()
+            datt()
+        torch.cuda.synchronize()
+        assert Q.qsa_get_device_status() == 0
+        # A decode step is replayed from a CUDA graph (the launches of one step, captured once), as a
+        # serving loop does: the device time is then not bounded by the host's launch rate.
+        g_step, g_sel, g_att = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_step):
+            dsel()
+            datt()
+        with torch.cuda.graph(g_sel):
+            dsel()
+        with torch.cuda.graph(g_att):
+            datt()
+        for _ in range(3):
+            g_step.replay()
         torch.cuda.synchronize()
         assert Q.qsa_get_device_status() == 0
         dsteps = args.decode_steps
+        gs = torch.cuda.current_stream(dev)
         d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         barrier(world)
-        d0.record(stream)
+        d0.record(gs)
         for _ in range(dsteps):
-            dstep()
-        d1.record(stream)
+            g_step.replay()
+        d1.record(gs)
         torch.cuda.synchronize()
         dms = max_over_ranks(d0.elapsed_time(d1), world, dev) / dsteps
-        devs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(5)]
-        for e in devs:
-            dstep(e)
+        # breakdown: each part's graph replayed 10 times back to back between two events
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        ev[0].record(gs)
+        for _ in range(10):
+            g_sel.replay()
+        ev[1].record(gs)
+        for _ in range(10):
+            g_att.replay()
+        ev[2].record(gs)
         torch.cuda.synchronize()
-        d_sel = statistics.mean(e[0].elapsed_time(e[1]) for e in devs)
-        d_att = statistics.mean(e[1].elapsed_time(e[2]) for e in devs)
+        d_sel = ev[0].elapsed_time(ev[1]) / 10
+        d_att = ev[1].elapsed_time(ev[2]) / 10
+        del g_step, g_sel, g_att
         dw = decode_work(wd)
         dgbs = dw["bytes"] / (dms / 1000) / 1e9
         decode = {"workload": args.decode_workload, "value": world * wd.B / (dms / 1000), "unit": "tokens/s",
-                  "ms_per_step": dms,
+                  "ms_per_step": dms, "launch": "CUDA graph of one step, replayed",
                   "steps": dsteps, "num_splits": splits,
                   "step_breakdown_ms": {"score_topk": d_sel, "attention_and_merge": d_att},
                   "gpu_launches_per_step": 1 + 2 + 1 + (1 if splits > 1 else 0),

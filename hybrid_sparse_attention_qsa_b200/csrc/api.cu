@@ -261,8 +261,13 @@ qsa_status_t qsa_select_topk(const float* scores, int64_t ld_scores, const void*
     return cuda_status(launch_topk(di, nullptr, 1, 0, seqlens, Tq, 0, blk, q_pos0, 0, B, 0, Tq, k, idx, s));
   }
   if (seqlens) {
+    // Decode: the scores of every sequence, then the top-k with a cluster of CTAs per sequence
+    // (one CTA per sequence for many sequences or short caches).
+    const int parts = topk_cluster_parts(di, B, NBk, k);
     cudaError_t e = launch_score_decode(di, qi, kp, head_w, seqlens, B, NBk, Hi, Di, blk, mode, ws, NBk, s);
-    if (e == cudaSuccess) e = launch_topk(di, ws, NBk, NBk, seqlens, 1, NBk, blk, 0, 0, B, 0, 1, k, idx, s);
+    if (e == cudaSuccess)
+      e = parts > 0 ? launch_topk_cluster(di, ws, NBk, seqlens, B, NBk, blk, k, idx, parts, s)
+                    : launch_topk(di, ws, NBk, NBk, seqlens, 1, NBk, blk, 0, 0, B, 0, 1, k, idx, s);
     return cuda_status(e);
   }
   // Filtered selection: sampled scores -> thresholds -> score + filter -> select over the lists

@@ -53,6 +53,12 @@ cudaError_t launch_score_decode(const DeviceInfo* di, const void* qi, const void
 cudaError_t launch_topk(const DeviceInfo* di, const float* scores, long long ld, long long batch_stride,
                         const int32_t* seqlens, int Tq, int NBk, int blk, long long q_pos0, int b0, int nb, int row0,
                         int rows, int k, int32_t* idx, cudaStream_t s);
+// Decode top-k with a thread-block cluster of `parts` CTAs per sequence row (row b reads
+// scores + b * ld).  topk_cluster_parts gives the cluster size for this device and shape, or 0
+// when the one-CTA-per-row kernel is the better choice (many rows, short rows, k > 1024).
+int topk_cluster_parts(const DeviceInfo* di, int B, int NBk, int k);
+cudaError_t launch_topk_cluster(const DeviceInfo* di, const float* scores, long long ld, const int32_t* seqlens, int B,
+                                int NBk, int blk, int k, int32_t* idx, int parts, cudaStream_t s);
 
 // Filtered selection (prefill): thresholds from sampled scores, the exact select over each row's
 // candidate list, and the exact redo of the rows listed in fail[1 .. fail[0]].

@@ -921,8 +921,9 @@ cudaError_t launch_attn_prefill(const DeviceInfo* di, const void* q, const void*
 }
 
 int decode_default_splits(const DeviceInfo* di, int B, int k_blocks) {
-  // about two items per SM, and at least ~32 blocks per split
-  const int want = std::max(1, (2 * di->num_sms + B - 1) / std::max(B, 1));
+  // One wave: at most one item per SM (a second, partial wave of items costs more than the longer
+  // items it saves), at most 8 splits per sequence, and at least ~32 blocks per split.
+  const int want = std::max(1, std::min(8, di->num_sms / std::max(B, 1)));
   const int cap = std::max(1, (k_blocks + 31) / 32);
   return std::min(want, cap);
 }

@@ -234,9 +234,236 @@ __device__ void topk_global(const float* s, int n, int k, int32_t* out, uint32_t
   }
 }
 
+// Shared-memory layout of the CTA-per-row kernels.
+struct TopkSmem {
+  uint32_t* cand_key;   // kCap
+  uint32_t* cand_idx;   // kCap
+  uint32_t* hist;       // kBins
+  uint32_t* samp;       // kSamples
+  uint32_t* ws;         // kWarps + 1
+  uint32_t* sel;        // 2
+  uint32_t* misc;       // 5 counters / flags
+  uint32_t* bitmap;     // bitmap words of the row
+};
+
+__device__ __forceinline__ TopkSmem topk_smem(uint32_t* sm) {
+  TopkSmem t;
+  t.cand_key = sm;
+  t.cand_idx = t.cand_key + kCap;
+  t.hist = t.cand_idx + kCap;
+  t.samp = t.hist + kBins;
+  t.ws = t.samp + kSamples;
+  t.sel = t.ws + kWarps + 1;
+  t.misc = t.sel + 2;
+  t.bitmap = t.misc + 5;
+  return t;
+}
+
+// kSamples keys of the row: kSamples/128 evenly spaced runs of 128 consecutive scores (one 16-byte
+// load per thread; coalesced per warp).  Ends synchronised.
+__device__ __forceinline__ void load_samples(const float* s, int n, uint32_t* samp) {
+  constexpr int kRuns = kSamples / 128;
+  for (int j = threadIdx.x; j < kSamples / 4; j += kTopkThreads) {
+    const int run = j >> 5, off = (j & 31) * 4;
+    const int i0 = (static_cast<int>((static_cast<long long>(run) * n) / kRuns) & ~3) + off;
+    float4 f;
+    if ((reinterpret_cast<uintptr_t>(s) & 15u) == 0 && i0 + 3 < n) {
+      f = __ldcs(reinterpret_cast<const float4*>(s + i0));
+    } else {
+      f.x = s[min(i0, n - 1)];
+      f.y = s[min(i0 + 1, n - 1)];
+      f.z = s[min(i0 + 2, n - 1)];
+      f.w = s[min(i0 + 3, n - 1)];
+    }
+    samp[4 * j] = key_of(f.x);
+    samp[4 * j + 1] = key_of(f.y);
+    samp[4 * j + 2] = key_of(f.z);
+    samp[4 * j + 3] = key_of(f.w);
+  }
+  __syncthreads();
+}
+
+// Sample rank whose key is expected to have ~2.5k + 128 scores of the row at or above it.
+__device__ __forceinline__ long long initial_rank(int n, int k) {
+  const long long target = min(static_cast<long long>(k) * 5 / 2 + 128, static_cast<long long>(k + kCap) / 2);
+  return (static_cast<long long>(kSamples) * target + n - 1) / n;
+}
+
+// The float whose key is the rank-th largest sample's key, resolved on its top 16 bits (a little
+// below that sample, so the candidates it admits include it).  Ends synchronised.
+__device__ __forceinline__ float tau_of_rank(long long rank, const TopkSmem& t) {
+  uint32_t dummy;
+  const uint32_t tau = smem_select(t.samp, kSamples, static_cast<uint32_t>(rank), 2, t.hist, t.ws, t.sel, &dummy);
+  // keys of finite floats are never 0x7FFFFFFF..0, so this inverts key_of on the resolved bits
+  return __uint_as_float((tau & 0x80000000u) ? (tau & 0x7FFFFFFFu) : ~tau);
+}
+
+// Appends every (key, index) of s[lo, hi) with score >= tau_f to the candidate arrays (unordered;
+// t.misc[0] counts them, including any beyond kCap, which are dropped).  lo is a multiple of 4.
+// KU independent 16-byte loads per thread are in flight before any of them is used.
+template <int KU>
+__device__ __forceinline__ void collect(const float* s, int lo, int hi, bool vec, float tau_f, const TopkSmem& t) {
+  const int tid = threadIdx.x;
+  for (int base = lo; base < hi; base += 4 * kTopkThreads * KU) {
+    float v[KU][4];
+#pragma unroll
+    for (int u = 0; u < KU; ++u) {
+      const int i0 = base + 4 * (u * kTopkThreads + tid);
+      if (vec && i0 + 3 < hi) {
+        const float4 f = __ldcs(reinterpret_cast<const float4*>(s + i0));
+        v[u][0] = f.x;
+        v[u][1] = f.y;
+        v[u][2] = f.z;
+        v[u][3] = f.w;
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) v[u][e] = i0 + e < hi ? s[i0 + e] : -INFINITY;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < KU; ++u) {
+      const int i0 = base + 4 * (u * kTopkThreads + tid);
+      const int nvalid = min(4, max(0, hi - i0));
+      const uint32_t hm = ((v[u][0] >= tau_f ? 1u : 0u) | (v[u][1] >= tau_f ? 2u : 0u) |
+                           (v[u][2] >= tau_f ? 4u : 0u) | (v[u][3] >= tau_f ? 8u : 0u)) &
+                          ((1u << nvalid) - 1u);
+#if QSA_TOPK_APPEND == 1
+      if (hm) {   // a shared-memory atomic per thread that has candidates
+        uint32_t p = atomicAdd(&t.misc[0], static_cast<uint32_t>(__popc(hm)));
+#else
+      const int lane = tid & 31;
+      const uint32_t nh = static_cast<uint32_t>(__popc(hm));
+      if (__ballot_sync(0xffffffffu, nh != 0) != 0u) {   // warp-uniform
+        uint32_t incl = nh;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        uint32_t wbase = 0;
+        if (lane == 31) wbase = atomicAdd(&t.misc[0], incl);
+        uint32_t p = __shfl_sync(0xffffffffu, wbase, 31) + incl - nh;
+#endif
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if (hm & (1u << e)) {
+            if (p < static_cast<uint32_t>(kCap)) {
+              t.cand_key[p] = key_of(v[u][e]);
+              t.cand_idx[p] = static_cast<uint32_t>(i0 + e);
+            }
+            ++p;
+          }
+        }
+      }
+    }
+  }
+}
+
+// Steps 3-5 on m candidates (k <= m <= kCap) in t.cand_key / t.cand_idx: the exact k-th key, the
+// index cutoff among equal keys, the bitmap of the kept set and its ascending emission.  Returns
+// false (nothing written) when more than kSamples candidates equal the k-th key; the caller then
+// selects over the row in memory.  All threads call it; starts and ends synchronised.
+__device__ bool select_emit(int m, int k, int words, int32_t* out, const TopkSmem& t) {
+  const int tid = threadIdx.x;
+  uint32_t need_eq;
+  const uint32_t kth = smem_select(t.cand_key, m, static_cast<uint32_t>(k), 4, t.hist, t.ws, t.sel, &need_eq);
+  const uint32_t n_eq = t.hist[kth & 0xFFu];   // last pass: hits in the K* bin = keys equal to K*
+  uint32_t icut = 0xFFFFFFFFu;
+  if (need_eq < n_eq) {
+    // the need_eq smallest indices among the keys equal to K*: select on ~index among them
+    uint32_t* inv = t.samp;   // reuse: up to kSamples entries
+    if (tid == 0) t.misc[1] = 0;
+    __syncthreads();
+    for (int i = tid; i < m; i += kTopkThreads) {
+      if (t.cand_key[i] == kth) {
+        const uint32_t p = atomicAdd(&t.misc[1], 1u);
+        if (p < static_cast<uint32_t>(kSamples)) inv[p] = ~t.cand_idx[i];
+      }
+    }
+    __syncthreads();
+    const int ne = static_cast<int>(t.misc[1]);
+    __syncthreads();
+    if (ne > kSamples) return false;
+    uint32_t dummy;
+    icut = ~smem_select(inv, ne, need_eq, 4, t.hist, t.ws, t.sel, &dummy);
+  }
+  for (int wd = tid; wd < words; wd += kTopkThreads) t.bitmap[wd] = 0u;
+  __syncthreads();
+  for (int i = tid; i < m; i += kTopkThreads) {
+    const uint32_t key = t.cand_key[i], id = t.cand_idx[i];
+    if (key > kth || (key == kth && id <= icut)) atomicOr(&t.bitmap[id >> 5], 1u << (id & 31));
+  }
+  __syncthreads();
+  const int wpt = (words + kTopkThreads - 1) / kTopkThreads;
+  const int w0 = tid * wpt, w1 = min(words, w0 + wpt);
+  uint32_t cnt = 0;
+  for (int wd = w0; wd < w1; ++wd) cnt += static_cast<uint32_t>(__popc(t.bitmap[wd]));
+  uint32_t total;
+  uint32_t p = block_excl_scan(cnt, t.ws, &total);
+  for (int wd = w0; wd < w1; ++wd) {
+    uint32_t bits = t.bitmap[wd];
+    while (bits) {
+      const int bit = __ffs(bits) - 1;
+      bits &= bits - 1;
+      if (p < static_cast<uint32_t>(k)) out[p] = wd * 32 + bit;
+      ++p;
+    }
+  }
+  __syncthreads();
+  return true;
+}
+
+// The whole selection of one row with n > k by one CTA (steps 1-5, threshold retries, and the
+// radix select over memory as the last resort).
+template <int KU>
+__device__ void topk_row(const float* s, int n, int k, int words, int bitmap_words, int32_t* out, const TopkSmem& t) {
+  const int tid = threadIdx.x;
+  if (k >= kCap || words > bitmap_words) {
+    topk_global(s, n, k, out, t.hist, t.ws, t.sel);
+    return;
+  }
+  int m = 0;
+  if (n <= kCap) {
+    for (int i = tid; i < n; i += kTopkThreads) {
+      t.cand_key[i] = key_of(s[i]);
+      t.cand_idx[i] = static_cast<uint32_t>(i);
+    }
+    m = n;
+    __syncthreads();
+  } else {
+    load_samples(s, n, t.samp);
+    long long rank = initial_rank(n, k);
+    const bool vec = ((reinterpret_cast<uintptr_t>(s) & 15u) == 0);
+    bool ok = false;
+    for (int attempt = 0; attempt < 3 && !ok; ++attempt) {
+      rank = max(1ll, min(rank, static_cast<long long>(kSamples)));
+      const float tau_f = tau_of_rank(rank, t);
+      if (tid == 0) t.misc[0] = 0;
+      __syncthreads();
+      collect<KU>(s, 0, n, vec, tau_f, t);
+      __syncthreads();
+      const uint32_t got = t.misc[0];
+      __syncthreads();
+      if (got >= static_cast<uint32_t>(k) && got <= static_cast<uint32_t>(kCap)) {
+        ok = true;
+        m = static_cast<int>(got);
+      } else if (got < static_cast<uint32_t>(k)) {
+        rank *= 4;          // threshold too high: take it lower
+      } else {
+        rank /= 4;          // too many candidates: take it higher
+      }
+    }
+    if (!ok) {
+      topk_global(s, n, k, out, t.hist, t.ws, t.sel);
+      return;
+    }
+  }
+  if (!select_emit(m, k, words, out, t)) topk_global(s, n, k, out, t.hist, t.ws, t.sel);
+}
+
 // KU: 16-byte loads per thread in flight in the filter pass.  Launches with fewer rows than SMs
-// (decode) take KU = 16 at one CTA per SM, so a long row is read in few round trips; many-row
-// launches keep KU small for three CTAs per SM.
+// take KU = 16 at one CTA per SM, so a long row is read in few round trips; many-row launches keep
+// KU small for three CTAs per SM.
 template <int KU, int MINB>
 __global__ void __launch_bounds__(kTopkThreads, MINB) topk_kernel(const float* __restrict__ scores, long long ld,
                                                             long long batch_stride, const int32_t* __restrict__ seqlens,
@@ -244,15 +471,7 @@ __global__ void __launch_bounds__(kTopkThreads, MINB) topk_kernel(const float* _
                                                             int row0, int k, int32_t* __restrict__ idx,
                                                             int bitmap_words, KernelCtl ctl) {
   extern __shared__ uint32_t sm[];
-  uint32_t* cand_key = sm;                       // kCap
-  uint32_t* cand_idx = cand_key + kCap;          // kCap
-  uint32_t* hist = cand_idx + kCap;              // kBins
-  uint32_t* samp = hist + kBins;                 // kSamples
-  uint32_t* ws = samp + kSamples;                // kWarps + 1
-  uint32_t* sel = ws + kWarps + 1;               // 2
-  uint32_t* misc = sel + 2;                      // counter
-  uint32_t* bitmap = misc + 5;                   // bitmap_words
-
+  const TopkSmem t = topk_smem(sm);
   const int tid = threadIdx.x;
   const int r = row0 + static_cast<int>(blockIdx.x);
   const int bz = blockIdx.y;
@@ -267,186 +486,12 @@ __global__ void __launch_bounds__(kTopkThreads, MINB) topk_kernel(const float* _
   const int n = pos < 0 ? 0 : static_cast<int>(min(static_cast<long long>(NBk), pos / blk));
   const float* s = scores + static_cast<long long>(bz) * batch_stride + static_cast<long long>(r - row0) * ld;
   int32_t* out = idx + (static_cast<long long>(b) * Tq + r) * k;
-
   if (n <= k) {
     for (int i = tid; i < k; i += kTopkThreads) out[i] = i < n ? i : -1;
     return;
   }
-  const int words = (n + 31) >> 5;
-  if (k >= kCap || words > bitmap_words) {
-    topk_global(s, n, k, out, hist, ws, sel);
-    return;
-  }
-
-  // ---- 1-2. candidates (key, index) with key >= tau
-  int m = 0;
-  if (n <= kCap) {
-    for (int i = tid; i < n; i += kTopkThreads) {
-      cand_key[i] = key_of(s[i]);
-      cand_idx[i] = static_cast<uint32_t>(i);
-    }
-    m = n;
-    __syncthreads();
-  } else {
-    // Samples: kSamples/128 evenly spaced runs of 128 consecutive scores (one 16-byte load per
-    // thread; coalesced per warp).
-    {
-      constexpr int kRuns = kSamples / 128;
-      for (int j = tid; j < kSamples / 4; j += kTopkThreads) {
-        const int run = j >> 5, off = (j & 31) * 4;
-        const int i0 = (static_cast<int>((static_cast<long long>(run) * n) / kRuns) & ~3) + off;
-        float4 f;
-        if ((reinterpret_cast<uintptr_t>(s) & 15u) == 0 && i0 + 3 < n) {
-          f = __ldcs(reinterpret_cast<const float4*>(s + i0));
-        } else {
-          f.x = s[min(i0, n - 1)];
-          f.y = s[min(i0 + 1, n - 1)];
-          f.z = s[min(i0 + 2, n - 1)];
-          f.w = s[min(i0 + 3, n - 1)];
-        }
-        samp[4 * j] = key_of(f.x);
-        samp[4 * j + 1] = key_of(f.y);
-        samp[4 * j + 2] = key_of(f.z);
-        samp[4 * j + 3] = key_of(f.w);
-      }
-    }
-    __syncthreads();
-    const long long target = min(static_cast<long long>(k) * 5 / 2 + 128, static_cast<long long>(k + kCap) / 2);
-    long long rank = (static_cast<long long>(kSamples) * target + n - 1) / n;
-    const bool vec = ((reinterpret_cast<uintptr_t>(s) & 15u) == 0);
-    bool ok = false;
-    for (int attempt = 0; attempt < 3 && !ok; ++attempt) {
-      rank = max(1ll, min(rank, static_cast<long long>(kSamples)));
-      uint32_t dummy;
-      const uint32_t tau = smem_select(samp, kSamples, static_cast<uint32_t>(rank), 2, hist, ws, sel, &dummy);
-      if (tid == 0) misc[0] = 0;
-      __syncthreads();
-      // tau back to the float it orders like (keys of finite floats are never 0x7FFFFFFF..0)
-      const float tau_f = __uint_as_float((tau & 0x80000000u) ? (tau & 0x7FFFFFFFu) : ~tau);
-      // kU independent 16-byte loads per thread are in flight before any of them is used.
-      constexpr int kU = KU;
-      for (int base = 0; base < n; base += 4 * kTopkThreads * kU) {
-        float v[kU][4];
-#pragma unroll
-        for (int u = 0; u < kU; ++u) {
-          const int i0 = base + 4 * (u * kTopkThreads + tid);
-          if (vec && i0 + 3 < n) {
-            const float4 f = __ldcs(reinterpret_cast<const float4*>(s + i0));
-            v[u][0] = f.x;
-            v[u][1] = f.y;
-            v[u][2] = f.z;
-            v[u][3] = f.w;
-          } else {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) v[u][e] = i0 + e < n ? s[i0 + e] : -INFINITY;
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < kU; ++u) {
-          const int i0 = base + 4 * (u * kTopkThreads + tid);
-          const int nvalid = min(4, max(0, n - i0));
-          const uint32_t hm = ((v[u][0] >= tau_f ? 1u : 0u) | (v[u][1] >= tau_f ? 2u : 0u) |
-                               (v[u][2] >= tau_f ? 4u : 0u) | (v[u][3] >= tau_f ? 8u : 0u)) &
-                              ((1u << nvalid) - 1u);
-#if QSA_TOPK_APPEND == 1
-          if (hm) {   // a shared-memory atomic per thread that has candidates
-            uint32_t p = atomicAdd(&misc[0], static_cast<uint32_t>(__popc(hm)));
-#else
-          const uint32_t nh = static_cast<uint32_t>(__popc(hm));
-          if (__ballot_sync(0xffffffffu, nh != 0) != 0u) {   // warp-uniform
-            uint32_t incl = nh;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-              const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-              if (lane >= o) incl += y;
-            }
-            uint32_t wbase = 0;
-            if (lane == 31) wbase = atomicAdd(&misc[0], incl);
-            uint32_t p = __shfl_sync(0xffffffffu, wbase, 31) + incl - nh;
-#endif
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              if (hm & (1u << e)) {
-                if (p < static_cast<uint32_t>(kCap)) {
-                  cand_key[p] = key_of(v[u][e]);
-                  cand_idx[p] = static_cast<uint32_t>(i0 + e);
-                }
-                ++p;
-              }
-            }
-          }
-        }
-      }
-      __syncthreads();
-      const uint32_t got = misc[0];
-      __syncthreads();
-      if (got >= static_cast<uint32_t>(k) && got <= static_cast<uint32_t>(kCap)) {
-        ok = true;
-        m = static_cast<int>(got);
-      } else if (got < static_cast<uint32_t>(k)) {
-        rank *= 4;          // threshold too high: take it lower
-      } else {
-        rank /= 4;          // too many candidates: take it higher
-      }
-    }
-    if (!ok) {
-      topk_global(s, n, k, out, hist, ws, sel);
-      return;
-    }
-  }
-
-  // ---- 3. exact k-th key among the candidates, then the index cutoff among equal keys
-  uint32_t need_eq;
-  const uint32_t kth = smem_select(cand_key, m, static_cast<uint32_t>(k), 4, hist, ws, sel, &need_eq);
-  const uint32_t n_eq = hist[kth & 0xFFu];   // last pass: hits in the K* bin = keys equal to K*
-  uint32_t icut = 0xFFFFFFFFu;
-  if (need_eq < n_eq) {
-    // the need_eq smallest indices among the keys equal to K*: select on ~index among them
-    uint32_t* inv = samp;   // reuse: up to kSamples entries, else fall back to a full pass below
-    if (tid == 0) misc[1] = 0;
-    __syncthreads();
-    for (int i = tid; i < m; i += kTopkThreads) {
-      if (cand_key[i] == kth) {
-        const uint32_t p = atomicAdd(&misc[1], 1u);
-        if (p < static_cast<uint32_t>(kSamples)) inv[p] = ~cand_idx[i];
-      }
-    }
-    __syncthreads();
-    const int ne = static_cast<int>(misc[1]);
-    __syncthreads();
-    if (ne > kSamples) {
-      topk_global(s, n, k, out, hist, ws, sel);
-      return;
-    }
-    uint32_t dummy;
-    icut = ~smem_select(inv, ne, need_eq, 4, hist, ws, sel, &dummy);
-  }
-
-  // ---- 4-5. bitmap of the kept set, emitted in ascending order
-  for (int wd = tid; wd < words; wd += kTopkThreads) bitmap[wd] = 0u;
-  __syncthreads();
-  for (int i = tid; i < m; i += kTopkThreads) {
-    const uint32_t key = cand_key[i], id = cand_idx[i];
-    if (key > kth || (key == kth && id <= icut)) atomicOr(&bitmap[id >> 5], 1u << (id & 31));
-  }
-  __syncthreads();
-  const int wpt = (words + kTopkThreads - 1) / kTopkThreads;
-  const int w0 = tid * wpt, w1 = min(words, w0 + wpt);
-  uint32_t cnt = 0;
-  for (int wd = w0; wd < w1; ++wd) cnt += static_cast<uint32_t>(__popc(bitmap[wd]));
-  uint32_t total;
-  uint32_t p = block_excl_scan(cnt, ws, &total);
-  for (int wd = w0; wd < w1; ++wd) {
-    uint32_t bits = bitmap[wd];
-    while (bits) {
-      const int bit = __ffs(bits) - 1;
-      bits &= bits - 1;
-      if (p < static_cast<uint32_t>(k)) out[p] = wd * 32 + bit;
-      ++p;
-    }
-  }
+  topk_row<KU>(s, n, k, (n + 31) >> 5, bitmap_words, out, t);
 }
-
 
 // ======================================================================================
 // Warp-per-row variant (used when there are many rows): one warp owns a row end to end, so no
@@ -712,6 +757,363 @@ __global__ void __launch_bounds__(kWarpRowsPerCta * 32) topk_warp_kernel(
 }
 
 // ======================================================================================
+// Decode (few long rows): a thread-block cluster of P CTAs per sequence row (grid P x rows,
+// cluster P x 1).  Each CTA
+//   1. issues the loads of its slice of the row (a quarter, an eighth ...) and of 2048 samples of
+//      the whole row (16 runs of 128), so the slice is on its way while the threshold is found;
+//   2. finds the threshold from the samples as every CTA of the row does, with the same result:
+//      an 11-bit histogram over the bits where the sampled keys differ; tau = the lowest key of
+//      the bin holding the rank-th largest sample (~2.5 k + 128 of the row's scores expected above
+//      it); rows of at most kCCap blocks keep every block;
+//   3. appends the slice's (key, block) pairs with key >= tau to its shared-memory list IN BLOCK
+//      ORDER (ballot compaction, one CTA-wide scan of the warps' counts per round of loads).
+// After a cluster barrier, CTA 0 reads every slice's count and list through distributed shared
+// memory (the slices in order, so the merged list is in block order), a second cluster barrier
+// releases the other CTAs, and CTA 0 selects exactly over the merged list: an 11-bit histogram
+// over the bits where the listed keys differ finds the bin of the k-th largest key, the bin's keys
+// are resolved bit by bit (warp 0), and {key > K*} U {the first need_eq keys == K*} is emitted in
+// list order.  If the lists together hold fewer than k or more than kCCap entries (heavy ties),
+// CTA 0 selects over the row in memory instead (three radix passes), so the result never depends
+// on the threshold.
+constexpr int kCT = kTopkThreads;          // threads per CTA (512)
+constexpr int kCWarps = kCT / 32;
+constexpr int kCCap = 6144;                // list capacity of a slice, and of the merged list
+constexpr int kCU = kCCap / kCT;           // merged entries per thread of CTA 0 (12)
+constexpr int kCLoads = 8;                 // 16-byte loads per thread per round (16384 scores)
+constexpr int kCSmem = kBins * 4 + kCCap * 8 + (kCLoads * kCWarps + 2 * kCWarps + 2 + 4 + 4) * 4;
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Every thread of every CTA of the cluster: shared-memory writes before it are visible to the
+// cluster's reads after it.
+__device__ __forceinline__ void cluster_barrier() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// The address of `p` (this CTA's shared memory) in the shared memory of cluster CTA `rank`.
+__device__ __forceinline__ uint32_t cluster_addr(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(p))), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint2 ld_cluster_v2(uint32_t a) {
+  uint2 v;
+  asm volatile("ld.shared::cluster.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a) : "memory");
+  return v;
+}
+
+// Block-wide min and max (ws: 2 * kCWarps words).  Ends synchronised.
+__device__ __forceinline__ void block_minmax512(uint32_t& kmin, uint32_t& kmax, uint32_t* ws) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  if (lane == 0) {
+    ws[2 * warp] = kmin;
+    ws[2 * warp + 1] = kmax;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int w = 0; w < kCWarps; ++w) {
+    kmin = min(kmin, ws[2 * w]);
+    kmax = max(kmax, ws[2 * w + 1]);
+  }
+  __syncthreads();
+}
+
+// Round of slice loads: element i0 + e of load u, i0 = r0 + 4 (u kCT + tid); beyond hi: -inf.
+__device__ __forceinline__ void load_round(float4 (&v)[kCLoads], const float* s, int r0, int hi, bool vec) {
+#pragma unroll
+  for (int u = 0; u < kCLoads; ++u) {
+    const int i0 = r0 + 4 * (u * kCT + static_cast<int>(threadIdx.x));
+    if (vec && i0 + 3 < hi) {
+      v[u] = __ldcs(reinterpret_cast<const float4*>(s + i0));
+    } else {
+      v[u].x = i0 < hi ? s[i0] : -INFINITY;
+      v[u].y = i0 + 1 < hi ? s[i0 + 1] : -INFINITY;
+      v[u].z = i0 + 2 < hi ? s[i0 + 2] : -INFINITY;
+      v[u].w = i0 + 3 < hi ? s[i0 + 3] : -INFINITY;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kCT, 1) topk_cluster_kernel(const float* __restrict__ scores, long long ld,
+                                                            const int32_t* __restrict__ seqlens, int NBk, int blk,
+                                                            int k, int32_t* __restrict__ idx, KernelCtl ctl) {
+  extern __shared__ __align__(16) uint8_t csm[];
+  uint32_t* hist = reinterpret_cast<uint32_t*>(csm);                        // kBins
+  uint2* list = reinterpret_cast<uint2*>(csm + kBins * 4);                  // kCCap
+  uint32_t* wcnt = reinterpret_cast<uint32_t*>(csm + kBins * 4 + kCCap * 8);  // kCLoads x kCWarps
+  uint32_t* ws = wcnt + kCLoads * kCWarps;                                  // 2 kCWarps + 2
+  uint32_t* sel = ws + 2 * kCWarps + 2;                                     // 4
+  uint32_t* misc = sel + 4;                                                 // [0]: the slice's count
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t lt = lanemask_lt();
+  const uint32_t part = cluster_rank();
+  const int P = static_cast<int>(gridDim.x);
+  const int b = blockIdx.y;
+  const long long pos = static_cast<long long>(seqlens[b]) - 1;
+  if (pos < 0 && tid == 0 && part == 0) record_status(ctl, kStBadArg);
+  const int n = pos < 0 ? 0 : static_cast<int>(min(static_cast<long long>(NBk), pos / blk));
+  const float* s = scores + static_cast<long long>(b) * ld;
+  int32_t* out = idx + static_cast<long long>(b) * k;
+  if (n <= k) {   // uniform over the cluster: no cluster barrier is reached
+    if (part == 0)
+      for (int i = tid; i < k; i += kCT) out[i] = i < n ? i : -1;
+    return;
+  }
+  const bool vec = (reinterpret_cast<uintptr_t>(s) & 15u) == 0;
+  const bool keep_every = n <= kCCap;   // every block is a candidate
+  const int chunk = ((n + P - 1) / P + 3) & ~3;
+  const int lo = min(n, static_cast<int>(part) * chunk), hi = min(n, lo + chunk);
+
+  // ---- 1. the slice's first round and the samples in flight together
+  float4 v[kCLoads];
+  load_round(v, s, lo, hi, vec);
+  for (int i = tid * 4; i < kBins; i += kCT * 4) *reinterpret_cast<uint4*>(hist + i) = make_uint4(0u, 0u, 0u, 0u);
+
+  // ---- 2. threshold key
+  uint32_t tkey = 0u;   // every key is >= 0
+  if (!keep_every) {
+    const int run = tid >> 5, off = (tid & 31) * 4;
+    const int i0 = (static_cast<int>((static_cast<long long>(run) * n) / (kSamples / 128)) & ~3) + off;  // i0 + 3 < n
+    float4 f;
+    if (vec) {
+      f = __ldcs(reinterpret_cast<const float4*>(s + i0));
+    } else {
+      f.x = s[i0];
+      f.y = s[i0 + 1];
+      f.z = s[i0 + 2];
+      f.w = s[i0 + 3];
+    }
+    const uint32_t sk[4] = {key_of(f.x), key_of(f.y), key_of(f.z), key_of(f.w)};
+    uint32_t kmin = min(min(sk[0], sk[1]), min(sk[2], sk[3]));
+    uint32_t kmax = max(max(sk[0], sk[1]), max(sk[2], sk[3]));
+    block_minmax512(kmin, kmax, ws);   // also orders the histogram's clearing before its use
+    if (kmin == kmax) {
+      tkey = kmin;
+    } else {
+      const int hb = 31 - __clz(kmin ^ kmax);
+      const int sh = max(0, hb - 10);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) atomicAdd(&hist[(sk[e] >> sh) & (kBins - 1)], 1u);
+      __syncthreads();
+      const long long target = min(static_cast<long long>(k) * 5 / 2 + 128, static_cast<long long>(k + kCCap) / 2);
+      const long long rank = max(1ll, min(static_cast<long long>(kSamples), (kSamples * target + n - 1) / n));
+      find_bin(hist, kBins, static_cast<uint32_t>(rank), ws, sel);   // ends synchronised
+      const uint32_t hi_mask = (sh + 11 >= 32) ? 0u : (0xFFFFFFFFu << (sh + 11));
+      tkey = (kmax & hi_mask) | (sel[0] << sh);
+    }
+  }
+
+  // ---- 3. the slice's candidates, in block order, into this CTA's list
+  uint32_t count = 0;   // entries of the earlier rounds
+  for (int r0 = lo; r0 < hi; r0 += 4 * kCT * kCLoads) {
+    if (r0 != lo) load_round(v, s, r0, hi, vec);
+    uint32_t hm[kCLoads], lp[kCLoads];
+#pragma unroll
+    for (int u = 0; u < kCLoads; ++u) {
+      const float e4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+      const int i0 = r0 + 4 * (u * kCT + tid);
+      uint32_t m = 0, before = 0, wc = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const bool hit = i0 + e < hi && key_of(e4[e]) >= tkey;
+        m |= (hit ? 1u : 0u) << e;
+        const uint32_t bal = __ballot_sync(0xffffffffu, hit);
+        before += static_cast<uint32_t>(__popc(bal & lt));
+        wc += static_cast<uint32_t>(__popc(bal));
+      }
+      hm[u] = m;
+      lp[u] = before;   // hits of the lower lanes of this warp in this load
+      if (lane == 0) wcnt[u * kCWarps + warp] = wc;
+    }
+    __syncthreads();
+    if (warp == 0) {   // exclusive scan of the kCLoads x kCWarps counts, (load, warp) order
+      constexpr int kPer = kCLoads * kCWarps / 32;
+      uint32_t c[kPer], sum = 0;
+#pragma unroll
+      for (int q = 0; q < kPer; ++q) {
+        c[q] = wcnt[lane * kPer + q];
+        sum += c[q];
+      }
+      uint32_t incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      uint32_t run = incl - sum;
+#pragma unroll
+      for (int q = 0; q < kPer; ++q) {
+        wcnt[lane * kPer + q] = run;
+        run += c[q];
+      }
+      if (lane == 31) misc[1] = incl;   // the round's total
+    }
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < kCLoads; ++u) {
+      const float e4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+      const int i0 = r0 + 4 * (u * kCT + tid);
+      uint32_t p = count + wcnt[u * kCWarps + warp] + lp[u];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if (hm[u] & (1u << e)) {
+          if (p < static_cast<uint32_t>(kCCap)) list[p] = make_uint2(key_of(e4[e]), static_cast<uint32_t>(i0 + e));
+          ++p;
+        }
+      }
+    }
+    count += misc[1];
+    __syncthreads();   // wcnt and misc[1] are rewritten by the next round
+  }
+  if (tid == 0) misc[0] = count;
+
+  // ---- 4. merge in CTA 0
+  cluster_barrier();
+  if (part != 0) {
+    cluster_barrier();   // CTA 0 has read this CTA's list
+    return;
+  }
+  uint32_t cnt[8], base[8], total = 0;
+  bool fits = true;
+#pragma unroll
+  for (int p = 0; p < 8; ++p) {
+    cnt[p] = p < P ? ld_cluster_u32(cluster_addr(misc, p)) : 0u;
+    fits = fits && cnt[p] <= static_cast<uint32_t>(kCCap);
+    base[p] = total;
+    total += cnt[p];
+  }
+  const bool ok = fits && total >= static_cast<uint32_t>(k) && total <= static_cast<uint32_t>(kCCap);
+  // thread t holds merged entries [kCU t, kCU t + kCU): (key, block)
+  uint2 ent[kCU];
+  const int j0 = tid * kCU;
+#pragma unroll
+  for (int u = 0; u < kCU; ++u) {
+    const uint32_t j = static_cast<uint32_t>(j0 + u);
+    ent[u] = make_uint2(0u, 0u);
+    if (ok && j < total) {
+      uint32_t p = 0, rel = j;   // the slice holding merged entry j, and j's place in it
+#pragma unroll
+      for (int q = 1; q < 8; ++q) {
+        if (q < P && j >= base[q]) {
+          p = static_cast<uint32_t>(q);
+          rel = j - base[q];
+        }
+      }
+      ent[u] = ld_cluster_v2(cluster_addr(list + rel, p));
+    }
+  }
+  cluster_barrier();
+  if (!ok) {
+    topk_global(s, n, k, out, hist, ws, sel);
+    return;
+  }
+  const int c = static_cast<int>(total);
+  const int mine = max(0, min(kCU, c - j0));   // entries this thread holds
+  bool keep_all = false;
+  uint32_t kth = 0, need_eq = 0;
+  if (c == k) {
+    keep_all = true;
+  } else {
+    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+#pragma unroll
+    for (int u = 0; u < kCU; ++u) {
+      if (u < mine) {
+        kmin = min(kmin, ent[u].x);
+        kmax = max(kmax, ent[u].x);
+      }
+    }
+    block_minmax512(kmin, kmax, ws);
+    if (kmin == kmax) {
+      kth = kmin;
+      need_eq = static_cast<uint32_t>(k);
+    } else {
+      const int hb = 31 - __clz(kmin ^ kmax);
+      const int sh = max(0, hb - 10);
+      for (int i = tid * 4; i < kBins; i += kCT * 4) *reinterpret_cast<uint4*>(hist + i) = make_uint4(0u, 0u, 0u, 0u);
+      __syncthreads();
+#pragma unroll
+      for (int u = 0; u < kCU; ++u)
+        if (u < mine) atomicAdd(&hist[(ent[u].x >> sh) & (kBins - 1)], 1u);
+      __syncthreads();
+      find_bin(hist, kBins, static_cast<uint32_t>(k), ws, sel);
+      const uint32_t B = sel[0];
+      uint32_t krem = static_cast<uint32_t>(k) - sel[1];
+      const uint32_t hi_mask = (sh + 11 >= 32) ? 0u : (0xFFFFFFFFu << (sh + 11));
+      uint32_t prefix = (kmax & hi_mask) | (B << sh);   // listed keys share the bits above sh + 10
+      if (sh > 0) {
+        const uint32_t inbin = hist[B];   // <= c <= kCCap
+        if (tid == 0) sel[2] = 0;
+        __syncthreads();   // every thread has read hist[B]: the space now gathers the bin's keys
+        uint32_t* buf = hist;   // kBins + 2 kCCap words (the histogram and this CTA's list) >= kCCap
+#pragma unroll
+        for (int u = 0; u < kCU; ++u)
+          if (u < mine && ((ent[u].x >> sh) & (kBins - 1)) == B) buf[atomicAdd(&sel[2], 1u)] = ent[u].x;
+        __syncthreads();
+        if (warp == 0) {
+          const int mb = static_cast<int>(inbin);
+          for (int bit = sh - 1; bit >= 0; --bit) {
+            const uint32_t want = (prefix >> bit) | 1u;
+            uint32_t cntb = 0;
+            for (int i0 = 0; i0 < mb; i0 += 32) {
+              const int i = i0 + lane;
+              cntb += __popc(__ballot_sync(0xffffffffu, i < mb && (buf[i] >> bit) == want));
+            }
+            if (cntb >= krem)
+              prefix |= 1u << bit;
+            else
+              krem -= cntb;
+          }
+          if (lane == 0) {
+            sel[0] = prefix;
+            sel[1] = krem;
+          }
+        }
+        __syncthreads();
+        prefix = sel[0];
+        krem = sel[1];
+      }
+      kth = prefix;
+      need_eq = krem;
+    }
+  }
+  // ordered emission: one CTA-wide scan of (entries > K*, entries == K*) per thread
+  uint32_t gt_n = 0, eq_n = 0;
+#pragma unroll
+  for (int u = 0; u < kCU; ++u) {
+    if (u < mine) {
+      gt_n += (keep_all || ent[u].x > kth) ? 1u : 0u;
+      eq_n += (!keep_all && ent[u].x == kth) ? 1u : 0u;
+    }
+  }
+  uint32_t all;
+  const uint32_t ex = block_excl_scan((gt_n << 16) | eq_n, ws, &all);
+  uint32_t gt_run = ex >> 16, eq_run = ex & 0xFFFFu;
+#pragma unroll
+  for (int u = 0; u < kCU; ++u) {
+    if (u < mine) {
+      const bool gt = keep_all || ent[u].x > kth, eq = !keep_all && ent[u].x == kth;
+      if (gt) {
+        const uint32_t p = gt_run + min(eq_run, need_eq);
+        if (p < static_cast<uint32_t>(k)) out[p] = static_cast<int32_t>(ent[u].y);
+        ++gt_run;
+      } else if (eq) {
+        if (eq_run < need_eq && gt_run + eq_run < static_cast<uint32_t>(k)) out[gt_run + eq_run] = static_cast<int32_t>(ent[u].y);
+        ++eq_run;
+      }
+    }
+  }
+}
+
+// ======================================================================================
 // Exact redo of the rows that the filtered selection could not settle (list shorter than k, or
 // overflowing): one CTA per failed row at a time, grid-striding over the failure list
 // fail[1 .. fail[0]].  The row's scores are recomputed on CUDA cores in fp32 into the CTA's
@@ -809,6 +1211,35 @@ cudaError_t launch_topk(const DeviceInfo* di, const float* scores, long long ld,
     topk_kernel<QSA_TOPK_LOADS, 3><<<grid, kTopkThreads, smem, s>>>(scores, ld, batch_stride, seqlens, Tq, NBk, blk,
                                                                      q_pos0, b0, row0, k, idx, words, kernel_ctl(di));
   return cudaPeekAtLastError();
+}
+
+int topk_cluster_parts(const DeviceInfo* di, int B, int NBk, int k) {
+  if (B < 1 || k > 1024 || NBk <= kCCap) return 0;
+  const int p = std::min(8, di->num_sms / B);
+  return p >= 2 ? p : 0;
+}
+
+cudaError_t launch_topk_cluster(const DeviceInfo* di, const float* scores, long long ld, const int32_t* seqlens, int B,
+                                int NBk, int blk, int k, int32_t* idx, int parts, cudaStream_t s) {
+  if (B <= 0) return cudaSuccess;
+  if (parts < 1 || parts > 8) return cudaErrorInvalidValue;
+  static std::once_flag once[64];
+  std::call_once(once[di->device & 63], [] {
+    cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kCSmem);
+  });
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(parts), static_cast<unsigned>(B), 1);
+  cfg.blockDim = dim3(kCT, 1, 1);
+  cfg.dynamicSmemBytes = kCSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(parts);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, topk_cluster_kernel, scores, ld, seqlens, NBk, blk, k, idx, kernel_ctl(di));
 }
 
 cudaError_t launch_topk_fallback(const DeviceInfo* di, const void* qi, const void* kp, const float* head_w, int Hi,

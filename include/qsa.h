@@ -172,7 +172,11 @@ QSA_API qsa_status_t qsa_index_score(const void* qi, const void* kp, const float
  * scores == NULL: the scores are computed here.  Arguments as for qsa_index_score.  Two ways,
  *   both giving the same index lists; qsa_set_select_options can force one:
  *   - materialised (decode; Hi of 1 or 2; short prefills): the scores are computed chunk by chunk
- *     into `workspace` (at least one score row of NBk floats).  With more than one chunk the
+ *     into `workspace` (at least one score row of NBk floats; decode: B rows).  In decode, with
+ *     few sequences (2 or more SMs per sequence), k <= 1024 and more than 6144 blocks, each
+ *     sequence's top-k runs on a thread-block cluster of up to 8 CTAs, one slice of the scores
+ *     each, merged through distributed shared memory; the lists equal those of one CTA per
+ *     sequence.  With more than one chunk the
  *     workspace is split in two halves and the top-k of one chunk runs on a per-device internal
  *     stream while the next chunk is scored on `stream`; the internal stream is joined back into
  *     `stream` before the call returns, so the call keeps the usual stream-ordered semantics.

@@ -1,0 +1,125 @@
+"""GPU: the decode selection with a thread-block cluster of CTAs per sequence against the
+one-CTA-per-sequence top-k over the same scores, and against the oracle.
+
+Both decode selections take the top-k of the same fp32 scores written by the decode score kernel
+(qsa_index_score then qsa_select_topk from scores: one CTA per row; qsa_select_topk from qi/kp:
+the cluster kernel when there are 2 or more SMs per sequence), so their index lists must be
+identical; the oracle's lists agree under the tie rule."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from hybrid_sparse_attention_qsa_b200 import inputs as I
+from hybrid_sparse_attention_qsa_b200 import qsa as Q
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+def _case(B, nbk, seed, Hi=4):
+    g = torch.Generator(device=DEV)
+    g.manual_seed(seed)
+    qi = (torch.randn((B, Hi, 64), generator=g, device=DEV) * 0.125).to(torch.bfloat16)
+    kp = (torch.randn((B, nbk, 64), generator=g, device=DEV) * 0.125).to(torch.bfloat16)
+    return qi, kp
+
+
+def _select(qi, kp, seqlens, k, cluster, **kw):
+    """cluster=True: scores and top-k in one call (the cluster top-k for few sequences);
+    cluster=False: the same scores materialised, then the one-CTA-per-row top-k."""
+    if cluster:
+        idx = Q.qsa_select_topk(k, qi=qi, kp=kp, seqlens=seqlens, **kw)
+    else:
+        sc = Q.qsa_index_score(qi, kp, seqlens=seqlens, **kw)
+        idx = Q.qsa_select_topk(k, scores=sc, NBk=kp.shape[1], seqlens=seqlens)
+    torch.cuda.synchronize()
+    assert Q.qsa_get_device_status() == Q.QSA_OK
+    return idx.cpu().numpy()
+
+
+def _oracle_rows(idx, qi, kp, seqlens, k, rows, head_w=None, mode=0):
+    qh, kph = I.bits(qi), I.bits(kp)
+    wh = None if head_w is None else head_w.cpu().numpy()
+    ora, kth, srows, nb = [], [], {}, []
+    for i, b in enumerate(rows):
+        n = (int(seqlens[b]) - 1) // 4
+        s = O.index_scores(qh[b], kph[b], n, head_w=wh, mode=mode)
+        ri, rk = O.select_topk(s, k)
+        ora.append(ri)
+        kth.append(rk)
+        srows[i] = s
+        nb.append(n)
+    got = idx[rows]
+    assert P.check_index_rows(got, np.array(nb), k) == []
+    res = P.compare_selection(got, np.array(ora), np.array(kth), lambda i: srows[i])
+    assert res["bad"] == [], res["bad"][:3]
+
+
+def test_cluster_equals_one_cta_on_the_256k_shape():
+    """32 sequences of 262144 tokens (65536 blocks), k = 512: the bench's decode shape (clusters
+    of 4 CTAs on 148 SMs)."""
+    B, L, k = 32, 262144, 512
+    qi, kp = _case(B, L // 4, 3)
+    seqlens = torch.full((B,), L, dtype=torch.int32, device=DEV)
+    one = _select(qi, kp, seqlens, k, cluster=False)
+    two = _select(qi, kp, seqlens, k, cluster=True)
+    assert np.array_equal(one, two)
+    _oracle_rows(two, qi, kp, seqlens.cpu().numpy(), k, [0, 17, 31])
+
+
+@pytest.mark.parametrize("B,k", [(1, 512), (7, 512), (5, 1000), (12, 64), (40, 1024), (9, 1)])
+def test_cluster_equals_one_cta_with_ragged_lengths(B, k):
+    """Lengths below k blocks, at the keep-every-block limit (6144 blocks), just above it, and
+    long, with clusters of 8 (B <= 18), 3 (B = 40) and 2 CTAs; linear scores with head weights."""
+    nbk = 70000
+    qi, kp = _case(B, nbk, 100 + B)
+    lens = [4 * nbk, 1, 5, 4 * k + 1, 4 * 6144 + 1, 4 * 6145 + 3, 100003, 4 * 40000 + 2, 4 * nbk - 1]
+    seqlens = torch.tensor([lens[b % len(lens)] for b in range(B)], dtype=torch.int32, device=DEV)
+    w = torch.linspace(0.5, 1.5, 4, device=DEV)
+    one = _select(qi, kp, seqlens, k, cluster=False, head_w=w, mode=1)
+    two = _select(qi, kp, seqlens, k, cluster=True, head_w=w, mode=1)
+    assert np.array_equal(one, two)
+    _oracle_rows(two, qi, kp, seqlens.cpu().numpy(), k, list(range(min(B, 9))), head_w=w, mode=1)
+
+
+def test_long_rows_take_several_rounds_per_slice():
+    """1M-token caches (262144 blocks): two sequences, clusters of 8, slices of 32768 scores, i.e.
+    two rounds of loads per CTA; k = 1024 as in the 1M workload."""
+    B, nbk, k = 2, 262144, 1024
+    qi, kp = _case(B, nbk, 44)
+    seqlens = torch.tensor([4 * nbk, 4 * 150001 + 3], dtype=torch.int32, device=DEV)
+    one = _select(qi, kp, seqlens, k, cluster=False)
+    two = _select(qi, kp, seqlens, k, cluster=True)
+    assert np.array_equal(one, two)
+    _oracle_rows(two, qi, kp, seqlens.cpu().numpy(), k, [0, 1])
+
+
+def test_heavy_ties_go_to_the_lowest_blocks():
+    """A zero query scores every block 0: the slices' lists overflow (long row) or together exceed
+    the merged capacity (shorter row), and CTA 0 selects over the row in memory: blocks 0 .. k-1."""
+    B, nbk, k = 4, 65536, 512
+    qi, kp = _case(B, nbk, 21)
+    qi[1] = 0
+    qi[2] = 0
+    seqlens = torch.tensor([4 * nbk, 4 * nbk, 4 * 20000 + 1, 4 * nbk - 7], dtype=torch.int32, device=DEV)
+    one = _select(qi, kp, seqlens, k, cluster=False)
+    two = _select(qi, kp, seqlens, k, cluster=True)
+    assert np.array_equal(one, two)
+    assert np.array_equal(two[1], np.arange(k, dtype=np.int32))
+    assert np.array_equal(two[2], np.arange(k, dtype=np.int32))
+
+
+def test_coarse_scores_with_ties_at_the_kth():
+    """Scores on a coarse grid (the indexer keys quantised), so many blocks tie at the k-th score
+    and the lower block indices must win among them."""
+    B, nbk, k = 6, 65536, 512
+    qi, kp = _case(B, nbk, 8)
+    kp = (kp.float() * 8).round().div(8).to(torch.bfloat16)
+    qi = (qi.float() * 4).round().div(4).to(torch.bfloat16)
+    seqlens = torch.full((B,), 4 * nbk, dtype=torch.int32, device=DEV)
+    one = _select(qi, kp, seqlens, k, cluster=False)
+    two = _select(qi, kp, seqlens, k, cluster=True)
+    assert np.array_equal(one, two)
