@@ -482,7 +482,10 @@ __global__ void __launch_bounds__(kFiltThreads, 1)
 // head columns; the Hi indexer heads fill N, zero past Hi) with the query's B fragments in
 // registers and the keys' A fragments from ldmatrix on the swizzled tile (conflict-free).  The four
 // lanes of a key row then add their heads with two shuffles.
-constexpr int kDecStages = 4;
+#ifndef QSA_DEC_STAGES
+#define QSA_DEC_STAGES 3
+#endif
+constexpr int kDecStages = QSA_DEC_STAGES;
 constexpr int kDecThreads = 160;
 constexpr int kDecSmem = 1024 + kDecStages * kKpBytes + 128;
 
@@ -745,8 +748,20 @@ cudaError_t launch_score_decode(const DeviceInfo* di, const void* qi, const void
     cudaFuncSetAttribute(score_decode_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem);
     cudaFuncSetAttribute(score_decode_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem);
   });
-  // about three CTAs per SM in total; parts are whole 128-key tiles
-  const int want = std::max(1, (di->num_sms * 3 + B - 1) / B);
+  // One wave: as many CTAs as fit on the device at once (a few stragglers in a second wave cost
+  // more than the whole wave's tail), split evenly over the sequences; parts are whole tiles.
+  static int occ[64][4];
+  static std::once_flag occ_once[64];
+  std::call_once(occ_once[di->device & 63], [di] {
+    auto* o = occ[di->device & 63];
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o[0], score_decode_kernel<1>, kDecThreads, kDecSmem);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o[1], score_decode_kernel<2>, kDecThreads, kDecSmem);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o[2], score_decode_kernel<4>, kDecThreads, kDecSmem);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o[3], score_decode_kernel<8>, kDecThreads, kDecSmem);
+  });
+  const int hslot = Hi == 1 ? 0 : Hi == 2 ? 1 : Hi == 4 ? 2 : 3;
+  const int slots = std::max(1, occ[di->device & 63][hslot]) * di->num_sms;
+  const int want = std::max(1, slots / B);
   const int tiles = (NBk + kM - 1) / kM;
   const int part_tiles = std::max(1, (tiles + want - 1) / want);
   const int part_len = part_tiles * kM;
