@@ -36,10 +36,10 @@ from hybrid_sparse_attention_qsa_b200 import inputs as I  # noqa: E402
 METRIC = "QSA prefill tokens/s @128K and decode tokens/s @256K ctx; % of roofline"
 PREFILL = "prefill_128k"
 DECODE = "decode_256k"
-# DRAM bytes read + written by one sparse_attn_kernel<2> launch, from the ncu capture summarised in
-# profiles/sparse_attn_prefill_128k.md (dram__bytes_read.sum + dram__bytes_write.sum); set to None
-# whenever the kernel changes until it is captured again
-ATTN_DRAM_TRAFFIC = {"prefill_128k": 1.521689e9 + 0.521716e9}
+# DRAM bytes read + written by one sparse_attn_kernel<2> launch on the 128K prefill, from one ncu
+# capture (dram__bytes_read.sum + dram__bytes_write.sum); set to None whenever the kernel changes
+# until it is captured again
+ATTN_DRAM_TRAFFIC = {"prefill_128k": 1.52e9 + 0.51862e9}
 
 
 # ------------------------------------------------------------------------------------------- helpers
@@ -453,7 +453,8 @@ def run_qsa(args):
                   "ms_per_step": dms, "launch": "CUDA graph of one step, replayed",
                   "steps": dsteps, "num_splits": splits,
                   "step_breakdown_ms": {"score_topk": d_sel, "attention_and_merge": d_att},
-                  "gpu_launches_per_step": 1 + 2 + 1 + (1 if splits > 1 else 0),
+                  "gpu_launches_per_step": 1 + 2 + 1 + (1 if Q.qsa.lib().qsa_decode_split_merge(
+                      wd.B, wd.Hq, wd.Hkv, wd.D, splits) == 2 else 0),
                   "roofline": {"bound": "hbm", "achieved": dgbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                                "frac": dgbs / pk["hbm_gbs"], "bytes_per_step": dw["bytes"],
                                "basis": "pooled-key cache read + gathered K/V of the selected tokens + q/o"}}

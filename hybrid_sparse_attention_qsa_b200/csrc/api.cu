@@ -392,6 +392,14 @@ int qsa_decode_default_splits(int B, int k_blocks) {
   return decode_default_splits(di, B, std::max(k_blocks, 1));
 }
 
+int qsa_decode_split_merge(int B, int Hq, int Hkv, int D, int num_splits) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || D < 1 || num_splits < 1 || Hq % Hkv) return -1;
+  if (num_splits == 1) return 0;
+  const DeviceInfo* di = device_info();
+  if (!di) return -1;
+  return decode_cluster_ok(di, B, Hq, Hkv, D, num_splits) ? 1 : 2;
+}
+
 qsa_status_t qsa_sparse_attn_decode(const void* q, const void* kcache, const void* vcache, const int32_t* seqlens,
                                     const int32_t* idx, int B, int Lmax, int Hq, int Hkv, int D, int k_blocks, int blk,
                                     float scale, int num_splits, void* out, float* lse, void* workspace,

@@ -81,6 +81,8 @@ cudaError_t launch_attn_decode(const DeviceInfo* di, const void* q, const void* 
                                int k_blocks, float scale, int num_splits, void* out, float* lse, float* part,
                                cudaStream_t s);
 int decode_default_splits(const DeviceInfo* di, int B, int k_blocks);
+// Whether a decode launch with these sizes merges its splits inside thread-block clusters.
+bool decode_cluster_ok(const DeviceInfo* di, int B, int Hq, int Hkv, int D, int splits);
 
 cudaError_t launch_wait_selftest(const DeviceInfo* di, unsigned long long timeout_ns, cudaStream_t s);
 

@@ -99,9 +99,32 @@ struct AttnArgs {
   float* part;              // decode partials [items][Hq][D + 2]
   long long q_pos0;
   int B, Tq, Tk, Hq, kblocks, splits, num_items;
+  int cluster;              // decode: the splits of a sequence form a thread-block cluster (1 item per CTA)
   float scale_log2;
   KernelCtl ctl;
 };
+
+// Cluster-wide barrier (every thread of every CTA of the cluster): shared-memory writes before it
+// are visible to the cluster's reads after it.  Exited threads do not hold it up.
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// The address of `p` (this CTA's shared memory) in the shared memory of cluster CTA `rank`.
+__device__ __forceinline__ uint32_t cluster_addr(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(p))), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float4 ld_cluster_f4(uint32_t a) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a) : "memory");
+  return v;
+}
 
 struct Item {
   const uint16_t* kbase;
@@ -186,12 +209,28 @@ __device__ __forceinline__ void attn_helper(const AttnArgs& a, int h, uint8_t* r
   }
 }
 
+// Asynchronous copy of index-list segment `seg` of work item `item` into idxbuf[buf], one
+// committed cp.async group (issued by one warp; an empty group past the last item).
+template <int HKV, int D>
+__device__ __forceinline__ void attn_fetch_list(const AttnArgs& a, int item, int seg, int* idxbuf, int buf) {
+  const int lane = threadIdx.x & 31;
+  if (item < a.num_items) {
+    const Item f = make_item<HKV, D>(a, item);
+    const int base = f.lo + seg * kSeg;
+    const int len = max(0, min(kSeg, f.hi - base));
+    for (int e = lane; e < len; e += 32) cp_async4(&idxbuf[buf * kSeg + e], f.idx_row + base + e);
+  }
+  cp_async_commit();
+}
+
 // Leading producer warp: walks the work items, turns each index list into block copies (the
 // query's own block last), publishes each stage's slot list for the helpers and issues its own
-// share of the copies.  Returns only when no copy it registered is still in flight.
+// share of the copies.  Returns only when no copy it registered is still in flight.  With
+// `prefetched` the first segment of the CTA's first item is already on its way (attn_fetch_list).
 template <int HKV, int D, int SLOTS>
 __device__ __forceinline__ void attn_producer(const AttnArgs& a, uint8_t* ring, uint8_t* info, uint64_t* full,
-                                              uint64_t* empty, uint64_t* ready, int* pend, int* idxbuf) {
+                                              uint64_t* empty, uint64_t* ready, int* pend, int* idxbuf,
+                                              bool prefetched = false) {
   using R = Ring<HKV, D, SLOTS>;
   const int lane = threadIdx.x & 31;
   auto info_at = [&](int s) { return reinterpret_cast<StageInfo*>(info + s * R::kInfoStride); };
@@ -248,17 +287,9 @@ __device__ __forceinline__ void attn_producer(const AttnArgs& a, uint8_t* ring, 
   // The index list of an item is staged in shared memory by asynchronous copies one segment
   // ahead (the next segment of this item or the first of the next item), so the copy ring never
   // waits on a global load of the list.
-  auto fetch = [&](int item, int seg, int buf) {
-    if (item < a.num_items) {
-      const Item f = make_item<HKV, D>(a, item);
-      const int base = f.lo + seg * kSeg;
-      const int len = max(0, min(kSeg, f.hi - base));
-      for (int e = lane; e < len; e += 32) cp_async4(&idxbuf[buf * kSeg + e], f.idx_row + base + e);
-    }
-    cp_async_commit();
-  };
+  auto fetch = [&](int item, int seg, int buf) { attn_fetch_list<HKV, D>(a, item, seg, idxbuf, buf); };
   int buf = 0;
-  fetch(blockIdx.x, 0, 0);
+  if (!prefetched) fetch(blockIdx.x, 0, 0);
   for (int item = blockIdx.x; alive && item < a.num_items; item += gridDim.x) {
     const Item it = make_item<HKV, D>(a, item);
     const long long own = it.pos >= 0 ? it.pos / kBlk : 0;
@@ -321,7 +352,11 @@ __device__ __forceinline__ void attn_producer(const AttnArgs& a, uint8_t* ring, 
   }
 }
 
-template <int HKV>
+// CL: decode with the splits of a sequence merged inside its thread-block cluster (a separate
+// instantiation, so that the prefill and split-partials code is compiled without it; there the
+// label of the cluster tail has no jump to it).
+#pragma nv_diag_suppress 177
+template <int HKV, bool CL = false>
 __global__ void __launch_bounds__(Cfg<HKV>::kThreads, 1) sparse_attn_kernel(AttnArgs a) {
   using C = Cfg<HKV>;
   extern __shared__ uint8_t smem_raw[];
@@ -354,18 +389,35 @@ __global__ void __launch_bounds__(Cfg<HKV>::kThreads, 1) sparse_attn_kernel(Attn
     }
     fence_mbar_init();
   }
-  // Zero the ring once so that unused slot rows are finite (they are masked, but 0 * NaN = NaN).
-  for (int i = threadIdx.x; i < kStages * C::kStageBytes / 16; i += blockDim.x)
-    reinterpret_cast<uint4*>(ring)[i] = make_uint4(0, 0, 0, 0);
+  // The producer starts fetching its first index-list segment while the ring is zeroed.
+  if (warp == C::kConsumerWarps) attn_fetch_list<HKV, kD>(a, blockIdx.x, 0, idxbuf, 0);
+  // Zero the V slots once so that unused slot rows are finite (their probabilities are 0, but
+  // 0 * NaN = NaN).  Unused K rows need no zeroing: their scores are replaced by -inf (a select,
+  // no arithmetic on them).
+  constexpr int kVChunks = kSlots * C::kPitch / 16;   // 16-byte chunks of one stage's V slots
+  for (int i = threadIdx.x; i < kStages * kVChunks; i += blockDim.x) {
+    const int s = i / kVChunks, c = i - s * kVChunks;
+    reinterpret_cast<uint4*>(ring + s * C::kStageBytes + kSlots * C::kPitch)[c] = make_uint4(0, 0, 0, 0);
+  }
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // order these writes before the bulk copies
   __syncthreads();
 
+  // In cluster mode every warp of every CTA passes the two cluster barriers of the split merge
+  // exactly once (the consumer warps that merge inside their epilogue, the others here).
   if (warp > C::kConsumerWarps) {
     attn_helper<HKV, kD, kSlots>(a, warp - C::kConsumerWarps, ring, reinterpret_cast<uint8_t*>(info), full, ready);
+    if constexpr (CL) {
+      cluster_sync_all();
+      cluster_sync_all();
+    }
     return;
   }
   if (warp == C::kConsumerWarps) {
-    attn_producer<HKV, kD, kSlots>(a, ring, reinterpret_cast<uint8_t*>(info), full, empty, ready, pend, idxbuf);
+    attn_producer<HKV, kD, kSlots>(a, ring, reinterpret_cast<uint8_t*>(info), full, empty, ready, pend, idxbuf, true);
+    if constexpr (CL) {
+      cluster_sync_all();
+      cluster_sync_all();
+    }
     return;
   }
 
@@ -404,6 +456,7 @@ __global__ void __launch_bounds__(Cfg<HKV>::kThreads, 1) sparse_attn_kernel(Attn
   };
   uint32_t qf[8][2], qn[8][2];
   load_q(blockIdx.x, qf);
+  bool merged = false;   // CL: this warp has passed the two cluster barriers
 
   for (int item = blockIdx.x; item < a.num_items; item += gridDim.x) {
     const Item it = make_item<HKV>(a, item);
@@ -413,7 +466,10 @@ __global__ void __launch_bounds__(Cfg<HKV>::kThreads, 1) sparse_attn_kernel(Attn
     for (int mt = 0; mt < 8; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
 
     for (;;) {
-      if (!mbar_wait(&full[st], ph, a.ctl)) return;
+      if (!mbar_wait(&full[st], ph, a.ctl)) {
+        if constexpr (CL) goto consumer_tail;
+        return;
+      }
       const int ns = info_at(st)->nslots;
       const bool last = info_at(st)->last != 0;
       if (ns > 0) {
@@ -483,7 +539,10 @@ __global__ void __launch_bounds__(Cfg<HKV>::kThreads, 1) sparse_attn_kernel(Attn
     }
     float* my_slot = mslot_base + (g * 3 + (j > 0 ? j - 1 : 0)) * (C::kMergeSlot / 4);
     if (j > 0) {
-      if (!mbar_wait(&mempty[g], mph ^ 1u, a.ctl)) return;
+      if (!mbar_wait(&mempty[g], mph ^ 1u, a.ctl)) {
+        if constexpr (CL) goto consumer_tail;
+        return;
+      }
 #pragma unroll
       for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
@@ -496,7 +555,10 @@ __global__ void __launch_bounds__(Cfg<HKV>::kThreads, 1) sparse_attn_kernel(Attn
       __syncwarp();
       if (lane == 0) mbar_arrive(&mfull[g]);
     } else {
-      if (!mbar_wait(&mfull[g], mph, a.ctl)) return;
+      if (!mbar_wait(&mfull[g], mph, a.ctl)) {
+        if constexpr (CL) goto consumer_tail;
+        return;
+      }
     }
     if (j == 0) {
 #pragma unroll 1
@@ -520,7 +582,46 @@ __global__ void __launch_bounds__(Cfg<HKV>::kThreads, 1) sparse_attn_kernel(Attn
         m0 = M0;
         m1 = M1;
       }
-      if (!it.partial) {
+      if (CL && it.partial) {
+        // Split merge inside the cluster: this warp's unnormalised state (o, m, l) goes to merge
+        // slot (g, 0), which it has finished reading, in its register layout (36 floats a lane);
+        // after a cluster barrier, rank 0 folds the other ranks' states into its own (log-sum-exp
+        // merge, ranks in order) and writes the final row below; a second barrier keeps the
+        // other CTAs (and their shared memory) alive until rank 0 has read them.
+        float* cs = mslot_base + (g * 3) * (C::kMergeSlot / 4) + lane * 36;
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt)
+          *reinterpret_cast<float4*>(cs + 4 * mt) = make_float4(o[mt][0], o[mt][1], o[mt][2], o[mt][3]);
+        *reinterpret_cast<float4*>(cs + 32) = make_float4(m0, m1, l0, l1);
+        cluster_sync_all();
+        const uint32_t rank = cluster_rank();
+        if (rank == 0) {
+          for (int r = 1; r < a.splits; ++r) {
+            const uint32_t ra = cluster_addr(cs, static_cast<uint32_t>(r));
+            const float4 ml4 = ld_cluster_f4(ra + 128);
+            const float M0 = fmaxf(m0, ml4.x), M1 = fmaxf(m1, ml4.y);
+            const float R0 = M0 == -INFINITY ? 0.f : M0, R1 = M1 == -INFINITY ? 0.f : M1;
+            const float fs0 = exp2f(m0 - R0), fo0 = exp2f(ml4.x - R0);
+            const float fs1 = exp2f(m1 - R1), fo1 = exp2f(ml4.y - R1);
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) {
+              const float4 ro = ld_cluster_f4(ra + 16 * mt);
+              o[mt][0] = o[mt][0] * fs0 + ro.x * fo0;
+              o[mt][1] = o[mt][1] * fs1 + ro.y * fo1;
+              o[mt][2] = o[mt][2] * fs0 + ro.z * fo0;
+              o[mt][3] = o[mt][3] * fs1 + ro.w * fo1;
+            }
+            l0 = l0 * fs0 + ml4.z * fo0;
+            l1 = l1 * fs1 + ml4.w * fo1;
+            m0 = M0;
+            m1 = M1;
+          }
+        }
+        __syncwarp();
+        cluster_sync_all();
+        merged = true;
+      }
+      if (!it.partial || (CL && cluster_rank() == 0)) {
         // stage the normalised rows [head][d] as bf16, then 16-byte stores
         // staged in merge slot (g, 0), which this warp has finished reading
         uint16_t* stg = reinterpret_cast<uint16_t*>(mslot_base + (g * 3) * (C::kMergeSlot / 4));
@@ -534,18 +635,19 @@ __global__ void __launch_bounds__(Cfg<HKV>::kThreads, 1) sparse_attn_kernel(Attn
           stg[(cpair + 1) * kD + d + 8] = __bfloat16_as_ushort(__float2bfloat16_rn(o[mt][3] * inv1));
         }
         __syncwarp();
-        uint16_t* orow = a.out + (it.orow * a.Hq + g * group) * kD;
+        const long long frow = it.partial ? it.qrow : it.orow;   // cluster mode: the sequence's row
+        uint16_t* orow = a.out + (frow * a.Hq + g * group) * kD;
         const int chunks = group * kD / 8;   // 16-byte chunks of this KV head's output heads
         for (int c = lane; c < chunks; c += 32)
           reinterpret_cast<uint4*>(orow)[c] = reinterpret_cast<const uint4*>(stg)[c];
         if (a.lse && lane < 4) {
           if (cpair < group)
-            a.lse[it.orow * a.Hq + g * group + cpair] = l0 > 0.f ? (m0 + __log2f(l0)) * kLn2 : -INFINITY;
+            a.lse[frow * a.Hq + g * group + cpair] = l0 > 0.f ? (m0 + __log2f(l0)) * kLn2 : -INFINITY;
           if (cpair + 1 < group)
-            a.lse[it.orow * a.Hq + g * group + cpair + 1] = l1 > 0.f ? (m1 + __log2f(l1)) * kLn2 : -INFINITY;
+            a.lse[frow * a.Hq + g * group + cpair + 1] = l1 > 0.f ? (m1 + __log2f(l1)) * kLn2 : -INFINITY;
         }
         __syncwarp();
-      } else {
+      } else if (!CL) {
         // unnormalised partial: part[item][h][0..D) = o, part[item][h][D] = m (log2 units), [D+1] = l
         float* prow = a.part + it.orow * a.Hq * (kD + 2);
 #pragma unroll
@@ -581,7 +683,15 @@ __global__ void __launch_bounds__(Cfg<HKV>::kThreads, 1) sparse_attn_kernel(Attn
       qf[kk][1] = qn[kk][1];
     }
   }
+consumer_tail:
+  if constexpr (CL) {
+    if (!merged) {
+      cluster_sync_all();
+      cluster_sync_all();
+    }
+  }
 }
+#pragma nv_diag_default 177
 
 // ======================================================================================
 // Wide variant: head dimension D (128 or 256) and GQA groups of up to 16 query heads (the model
@@ -920,6 +1030,58 @@ cudaError_t launch_attn_prefill(const DeviceInfo* di, const void* q, const void*
   return launch_attn_any(di, a, Hkv, D, s);
 }
 
+// Split-KV decode as clusters: one CTA per item (B * splits <= SMs), a cluster of `splits` CTAs per
+// sequence, the D = 128 kernel (groups of up to 8 heads), and all clusters resident at once.
+bool decode_cluster_ok(const DeviceInfo* di, int B, int Hq, int Hkv, int D, int splits) {
+  if (splits < 2 || splits > 8 || D != kD || Hq / Hkv > 8 || (Hkv != 1 && Hkv != 2)) return false;
+  if (static_cast<long long>(B) * splits > di->num_sms) return false;
+  static int max_clusters[64][2][9];
+  static std::once_flag once[64];
+  std::call_once(once[di->device & 63], [] {
+    cudaFuncSetAttribute(sparse_attn_kernel<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<1>::kSmem);
+    cudaFuncSetAttribute(sparse_attn_kernel<2, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<2>::kSmem);
+  });
+  int& mc = max_clusters[di->device & 63][Hkv - 1][splits];
+  if (mc == 0) {   // cached per device, KV head count and cluster size (-1: query failed)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(splits * B));
+    cfg.blockDim = dim3(Hkv == 1 ? Cfg<1>::kThreads : Cfg<2>::kThreads);
+    cfg.dynamicSmemBytes = Hkv == 1 ? Cfg<1>::kSmem : Cfg<2>::kSmem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(splits);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    const cudaError_t e = Hkv == 1 ? cudaOccupancyMaxActiveClusters(&n, sparse_attn_kernel<1, true>, &cfg)
+                                   : cudaOccupancyMaxActiveClusters(&n, sparse_attn_kernel<2, true>, &cfg);
+    mc = (e == cudaSuccess && n > 0) ? n : -1;
+    if (e != cudaSuccess) cudaGetLastError();
+  }
+  return mc >= B;
+}
+
+template <int HKV>
+cudaError_t launch_attn_cluster(const DeviceInfo* di, AttnArgs a, cudaStream_t s) {
+  using C = Cfg<HKV>;
+  (void)di;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(a.num_items));   // one item per CTA
+  cfg.blockDim = dim3(C::kThreads);
+  cfg.dynamicSmemBytes = C::kSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(a.splits);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, sparse_attn_kernel<HKV, true>, a);
+}
+
 int decode_default_splits(const DeviceInfo* di, int B, int k_blocks) {
   // One wave: at most one item per SM (a second, partial wave of items costs more than the longer
   // items it saves), at most 8 splits per sequence, and at least ~32 blocks per split.
@@ -951,6 +1113,10 @@ cudaError_t launch_attn_decode(const DeviceInfo* di, const void* q, const void* 
   a.num_items = B * num_splits;
   a.scale_log2 = scale * kLog2e;
   a.ctl = kernel_ctl(di);
+  if (num_splits > 1 && decode_cluster_ok(di, B, Hq, Hkv, D, num_splits)) {
+    a.cluster = 1;   // the splits of a sequence merge inside their cluster: no partials, no merge kernel
+    return Hkv == 1 ? launch_attn_cluster<1>(di, a, s) : launch_attn_cluster<2>(di, a, s);
+  }
   cudaError_t e = launch_attn_any(di, a, Hkv, D, s);
   if (e != cudaSuccess || num_splits <= 1) return e;
   combine_kernel<<<dim3(B, Hq), D, 0, s>>>(part, num_splits, Hq, D, static_cast<uint16_t*>(out), lse);

@@ -45,6 +45,7 @@ SIGNATURES = {
     "qsa_sparse_attn_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P, _P, _P]),
     "qsa_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I, _I]),
     "qsa_decode_default_splits": (_I, [_I, _I]),
+    "qsa_decode_split_merge": (_I, [_I, _I, _I, _I, _I]),
     "qsa_get_device_status": (_I, [_P]),
     "qsa_set_select_options": (_I, [_I, _I]),
     "qsa_set_wait_timeout_ns": (None, [_U64]),

@@ -226,9 +226,13 @@ QSA_API qsa_status_t qsa_sparse_attn_prefill(const void* q, const void* k, const
  *   token included, so the query sits at position seqlens[b] - 1); idx [B][k_blocks] int32
  *   -> out [B][Hq][D] bf16, lse [B][Hq] fp32 (may be NULL).
  * The index list of each sequence is cut into num_splits ranges (0 = choose from the GPU size)
- * that run in parallel; their partial softmax states are merged by log-sum-exp.  num_splits > 1
- * needs workspace >= qsa_workspace_size(QSA_OP_SPARSE_ATTN_DECODE, B, 1, 0, k_blocks, Hq, D,
- * num_splits) bytes.
+ * that run in parallel; their partial softmax states are merged by log-sum-exp: inside the
+ * attention kernel when the splits of a sequence can run as one thread-block cluster (D = 128,
+ * groups of up to 8 heads, 2 .. 8 splits, B * num_splits <= SMs, every cluster resident at once;
+ * the partials meet in distributed shared memory), otherwise by a second kernel over partials in
+ * `workspace` (qsa_decode_split_merge tells which).  num_splits > 1 needs workspace >=
+ * qsa_workspace_size(QSA_OP_SPARSE_ATTN_DECODE, B, 1, 0, k_blocks, Hq, D, num_splits) bytes
+ * either way.
  * Errors: as for prefill, plus WORKSPACE_TOO_SMALL.
  */
 QSA_API qsa_status_t qsa_sparse_attn_decode(const void* q, const void* kcache, const void* vcache,
@@ -275,6 +279,14 @@ QSA_API size_t qsa_workspace_size(qsa_op_t op, int B, int Tq, int NBk, int k, in
 
 /* Split count qsa_sparse_attn_decode picks for num_splits == 0 on the current device. */
 QSA_API int qsa_decode_default_splits(int B, int k_blocks);
+
+/*
+ * How qsa_sparse_attn_decode merges num_splits (>= 1, as passed after the default is resolved)
+ * splits on the current device: 0 = one split, nothing to merge; 1 = inside the attention
+ * kernel (thread-block clusters, one launch); 2 = a second kernel over partials in the
+ * workspace.  -1 on invalid sizes or without a usable device.
+ */
+QSA_API int qsa_decode_split_merge(int B, int Hq, int Hkv, int D, int num_splits);
 
 /*
  * Synchronises `stream`, then reads and clears the current device's status word:

@@ -145,3 +145,11 @@ def test_rope_params_checks(lib):
     rp = Q.RopeParams(0.0, 1.0, 0.0, 1.0, 32.0, 0.0)          # the query rotation needs a base
     assert lib.qsa_rope_index_queries_rope(1, 1, 1, 4, 4, 64, 0, None, ctypes.byref(rp), None) == Q.QSA_ERR_INVALID_ARGUMENT
     assert lib.qsa_rope_index_queries_rope(1, 1, 1, 4, 4, 64, 0, None, None, None) == Q.QSA_ERR_INVALID_ARGUMENT
+
+
+def test_decode_split_merge_host_rules(lib):
+    # one split never merges; invalid sizes are refused before any device query
+    assert lib.qsa_decode_split_merge(32, 16, 2, 128, 1) == 0
+    assert lib.qsa_decode_split_merge(0, 16, 2, 128, 4) == -1
+    assert lib.qsa_decode_split_merge(4, 16, 3, 128, 4) == -1   # Hq not a multiple of Hkv
+    assert lib.qsa_decode_split_merge(4, 16, 2, 128, 0) == -1

@@ -123,3 +123,39 @@ def test_coarse_scores_with_ties_at_the_kth():
     one = _select(qi, kp, seqlens, k, cluster=False)
     two = _select(qi, kp, seqlens, k, cluster=True)
     assert np.array_equal(one, two)
+
+
+# ------------------------------------------------------------------ split-KV merge inside a cluster
+@pytest.mark.parametrize("B,L,k", [(32, 65536, 512), (3, 20000, 512), (12, 9001, 100)])
+def test_cluster_split_merge_matches_the_merge_kernel_and_the_oracle(B, L, k):
+    """With B * splits <= SMs the splits of a sequence run as a cluster and merge through
+    distributed shared memory; with more items they write partials that a second kernel merges.
+    Both (and one split) against each other and against the oracle's attention over the same
+    index lists, with ragged lengths (the split holding the own block, empty splits)."""
+    from tests import harness as H
+    w = I.WORKLOADS["decode_256k"].with_(B=B, T=L, seed=B + L)
+    lens = [L, L - 1, 4 * k + 3, 17, L - 100, 1]
+    seqlens = [lens[b % len(lens)] for b in range(B)]
+    x = I.make_decode(w, DEV, seqlens=seqlens)
+    kp = Q.qsa_pool_block_keys(x["ki"])
+    idx = Q.qsa_select_topk(k, qi=x["qi"], kp=kp, seqlens=x["seqlens"])
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    many = sms // B + 1   # B * many > SMs: partials + merge kernel
+    assert Q.lib().qsa_decode_split_merge(B, 16, 2, 128, 2) == 1
+    assert Q.lib().qsa_decode_split_merge(B, 16, 2, 128, many) == 2
+    outs = {}
+    for sp in (1, 2, max(2, min(8, sms // B)), many):
+        o, l = Q.qsa_sparse_attn_decode(x["q"], x["k"], x["v"], x["seqlens"], idx, num_splits=sp)
+        torch.cuda.synchronize()
+        assert Q.qsa_get_device_status() == Q.QSA_OK
+        outs[sp] = (I.bits(o), l.cpu().numpy())
+    ref = outs[1]
+    for sp, (o, l) in outs.items():
+        P.assert_outputs_close(o, ref[0])
+        assert np.allclose(l, ref[1], atol=1e-4), sp
+    h = {n: I.bits(x[n]) for n in ("q", "k", "v", "qi")}
+    seqs = list(range(min(B, 6)))
+    sp = max(2, min(8, sms // B))
+    st = H.compare_decode(idx.cpu().numpy()[seqs], outs[sp][0][seqs], outs[sp][1][seqs], h["q"], h["k"], h["v"],
+                          h["qi"], I.bits(kp), np.array(seqlens), seqs, topk=k)
+    print("cluster decode:", st)
