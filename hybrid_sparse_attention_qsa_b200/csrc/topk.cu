@@ -809,6 +809,10 @@ __device__ __forceinline__ uint2 ld_cluster_v2(uint32_t a) {
   return v;
 }
 
+__device__ __forceinline__ float key_to_float(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
 // Block-wide min and max (ws: 2 * kCWarps words).  Ends synchronised.
 __device__ __forceinline__ void block_minmax512(uint32_t& kmin, uint32_t& kmax, uint32_t* ws) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -823,6 +827,39 @@ __device__ __forceinline__ void block_minmax512(uint32_t& kmin, uint32_t& kmax, 
   for (int w = 0; w < kCWarps; ++w) {
     kmin = min(kmin, ws[2 * w]);
     kmax = max(kmax, ws[2 * w + 1]);
+  }
+  __syncthreads();
+}
+
+// The bin of 2048 (4 per thread, thread t holding bins 4t .. 4t + 3) that holds the rank-th
+// largest hit, with two barriers: sel[0] = bin, sel[1] = hits in the bins above it.  ws: kCWarps
+// words.  Ends synchronised.
+__device__ __forceinline__ void find_bin2(const uint32_t* hist, uint32_t rank, uint32_t* ws, uint32_t* sel) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint4 h4 = *reinterpret_cast<const uint4*>(hist + 4 * tid);
+  const uint32_t local = h4.x + h4.y + h4.z + h4.w;
+  uint32_t incl = local;   // this lane's bins and those of the higher lanes of the warp
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_down_sync(0xffffffffu, incl, o);
+    if (lane + o < 32) incl += y;
+  }
+  if (lane == 0) ws[warp] = incl;   // the warp's total
+  __syncthreads();
+  uint32_t above = incl - local;     // hits in the bins above this thread's four
+#pragma unroll
+  for (int w = 0; w < kCWarps; ++w) above += w > warp ? ws[w] : 0u;
+  if (above < rank && above + local >= rank) {
+    const uint32_t hb[4] = {h4.x, h4.y, h4.z, h4.w};
+    uint32_t acc = above;
+#pragma unroll
+    for (int q = 3; q >= 0; --q) {
+      if (acc < rank && acc + hb[q] >= rank) {
+        sel[0] = static_cast<uint32_t>(4 * tid + q);
+        sel[1] = acc;
+      }
+      acc += hb[q];
+    }
   }
   __syncthreads();
 }
@@ -873,17 +910,12 @@ __global__ void __launch_bounds__(kCT, 1) topk_cluster_kernel(const float* __res
   const int chunk = ((n + P - 1) / P + 3) & ~3;
   const int lo = min(n, static_cast<int>(part) * chunk), hi = min(n, lo + chunk);
 
-  // ---- 1. the slice's first round and the samples in flight together
-  float4 v[kCLoads];
-  load_round(v, s, lo, hi, vec);
-  for (int i = tid * 4; i < kBins; i += kCT * 4) *reinterpret_cast<uint4*>(hist + i) = make_uint4(0u, 0u, 0u, 0u);
-
-  // ---- 2. threshold key
-  uint32_t tkey = 0u;   // every key is >= 0
+  // ---- 1. the samples, then the slice's first round, in flight together (the samples first: the
+  // threshold needs only them and is found while the slice is still arriving)
+  float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
   if (!keep_every) {
     const int run = tid >> 5, off = (tid & 31) * 4;
     const int i0 = (static_cast<int>((static_cast<long long>(run) * n) / (kSamples / 128)) & ~3) + off;  // i0 + 3 < n
-    float4 f;
     if (vec) {
       f = __ldcs(reinterpret_cast<const float4*>(s + i0));
     } else {
@@ -892,6 +924,18 @@ __global__ void __launch_bounds__(kCT, 1) topk_cluster_kernel(const float* __res
       f.z = s[i0 + 2];
       f.w = s[i0 + 3];
     }
+  }
+  float4 v[kCLoads];
+  load_round(v, s, lo, hi, vec);
+  for (int i = tid * 4; i < kBins; i += kCT * 4) *reinterpret_cast<uint4*>(hist + i) = make_uint4(0u, 0u, 0u, 0u);
+  if (tid == 0) {
+    misc[2] = 0xFFFFFFFFu;   // this slice's smallest and largest candidate key
+    misc[3] = 0u;
+  }
+
+  // ---- 2. threshold key
+  uint32_t tkey = 0u;   // every key is >= 0
+  if (!keep_every) {
     const uint32_t sk[4] = {key_of(f.x), key_of(f.y), key_of(f.z), key_of(f.w)};
     uint32_t kmin = min(min(sk[0], sk[1]), min(sk[2], sk[3]));
     uint32_t kmax = max(max(sk[0], sk[1]), max(sk[2], sk[3]));
@@ -906,27 +950,28 @@ __global__ void __launch_bounds__(kCT, 1) topk_cluster_kernel(const float* __res
       __syncthreads();
       const long long target = min(static_cast<long long>(k) * 5 / 2 + 128, static_cast<long long>(k + kCCap) / 2);
       const long long rank = max(1ll, min(static_cast<long long>(kSamples), (kSamples * target + n - 1) / n));
-      find_bin(hist, kBins, static_cast<uint32_t>(rank), ws, sel);   // ends synchronised
+      find_bin2(hist, static_cast<uint32_t>(rank), ws, sel);   // ends synchronised
       const uint32_t hi_mask = (sh + 11 >= 32) ? 0u : (0xFFFFFFFFu << (sh + 11));
       tkey = (kmax & hi_mask) | (sel[0] << sh);
     }
   }
+  __syncthreads();   // misc[2..3] initialised (keep_every reaches no barrier above)
 
   // ---- 3. the slice's candidates, in block order, into this CTA's list
+  const float tau_f = keep_every ? -INFINITY : key_to_float(tkey);   // key_of(x) >= tkey <=> x >= tau_f
   uint32_t count = 0;   // entries of the earlier rounds
   for (int r0 = lo; r0 < hi; r0 += 4 * kCT * kCLoads) {
     if (r0 != lo) load_round(v, s, r0, hi, vec);
     uint32_t hm[kCLoads], lp[kCLoads];
 #pragma unroll
     for (int u = 0; u < kCLoads; ++u) {
-      const float e4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
       const int i0 = r0 + 4 * (u * kCT + tid);
-      uint32_t m = 0, before = 0, wc = 0;
+      const uint32_t m = (v[u].x >= tau_f && i0 < hi ? 1u : 0u) | (v[u].y >= tau_f && i0 + 1 < hi ? 2u : 0u) |
+                         (v[u].z >= tau_f && i0 + 2 < hi ? 4u : 0u) | (v[u].w >= tau_f && i0 + 3 < hi ? 8u : 0u);
+      uint32_t before = 0, wc = 0;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const bool hit = i0 + e < hi && key_of(e4[e]) >= tkey;
-        m |= (hit ? 1u : 0u) << e;
-        const uint32_t bal = __ballot_sync(0xffffffffu, hit);
+        const uint32_t bal = __ballot_sync(0xffffffffu, (m >> e) & 1u);
         before += static_cast<uint32_t>(__popc(bal & lt));
         wc += static_cast<uint32_t>(__popc(bal));
       }
@@ -958,18 +1003,29 @@ __global__ void __launch_bounds__(kCT, 1) topk_cluster_kernel(const float* __res
       if (lane == 31) misc[1] = incl;   // the round's total
     }
     __syncthreads();
+    uint32_t cmin = 0xFFFFFFFFu, cmax = 0u;   // this thread's candidate keys
 #pragma unroll
     for (int u = 0; u < kCLoads; ++u) {
-      const float e4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+      uint32_t mm = hm[u];
+      if (mm == 0u) continue;   // most loads hold no candidate
       const int i0 = r0 + 4 * (u * kCT + tid);
       uint32_t p = count + wcnt[u * kCWarps + warp] + lp[u];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        if (hm[u] & (1u << e)) {
-          if (p < static_cast<uint32_t>(kCCap)) list[p] = make_uint2(key_of(e4[e]), static_cast<uint32_t>(i0 + e));
-          ++p;
-        }
+      while (mm) {
+        const int e = __ffs(mm) - 1;
+        mm &= mm - 1;
+        const float x = e == 0 ? v[u].x : e == 1 ? v[u].y : e == 2 ? v[u].z : v[u].w;
+        const uint32_t key = key_of(x);
+        cmin = min(cmin, key);
+        cmax = max(cmax, key);
+        if (p < static_cast<uint32_t>(kCCap)) list[p] = make_uint2(key, static_cast<uint32_t>(i0 + e));
+        ++p;
       }
+    }
+    cmin = __reduce_min_sync(0xffffffffu, cmin);
+    cmax = __reduce_max_sync(0xffffffffu, cmax);
+    if (lane == 0 && cmax >= cmin) {
+      atomicMin(&misc[2], cmin);
+      atomicMax(&misc[3], cmax);
     }
     count += misc[1];
     __syncthreads();   // wcnt and misc[1] are rewritten by the next round
@@ -982,24 +1038,31 @@ __global__ void __launch_bounds__(kCT, 1) topk_cluster_kernel(const float* __res
     cluster_barrier();   // CTA 0 has read this CTA's list
     return;
   }
-  uint32_t cnt[8], base[8], total = 0;
+  uint32_t base[8], total = 0, kmin = 0xFFFFFFFFu, kmax = 0u;
   bool fits = true;
 #pragma unroll
   for (int p = 0; p < 8; ++p) {
-    cnt[p] = p < P ? ld_cluster_u32(cluster_addr(misc, p)) : 0u;
-    fits = fits && cnt[p] <= static_cast<uint32_t>(kCCap);
+    uint32_t cp = 0u;
+    if (p < P) {
+      const uint32_t a = cluster_addr(misc, p);
+      cp = ld_cluster_u32(a);
+      kmin = min(kmin, ld_cluster_u32(a + 8));
+      kmax = max(kmax, ld_cluster_u32(a + 12));
+    }
+    fits = fits && cp <= static_cast<uint32_t>(kCCap);
     base[p] = total;
-    total += cnt[p];
+    total += cp;
   }
   const bool ok = fits && total >= static_cast<uint32_t>(k) && total <= static_cast<uint32_t>(kCCap);
-  // thread t holds merged entries [kCU t, kCU t + kCU): (key, block)
+  // merged entry j = tid + kCT u (round u of R): (key, block), in block order over (u, tid)
+  const int c = ok ? static_cast<int>(total) : 0;
+  const int R = (c + kCT - 1) / kCT;   // uniform
   uint2 ent[kCU];
-  const int j0 = tid * kCU;
 #pragma unroll
   for (int u = 0; u < kCU; ++u) {
-    const uint32_t j = static_cast<uint32_t>(j0 + u);
     ent[u] = make_uint2(0u, 0u);
-    if (ok && j < total) {
+    const uint32_t j = static_cast<uint32_t>(tid + u * kCT);
+    if (u < R && j < static_cast<uint32_t>(c)) {
       uint32_t p = 0, rel = j;   // the slice holding merged entry j, and j's place in it
 #pragma unroll
       for (int q = 1; q < 8; ++q) {
@@ -1016,23 +1079,13 @@ __global__ void __launch_bounds__(kCT, 1) topk_cluster_kernel(const float* __res
     topk_global(s, n, k, out, hist, ws, sel);
     return;
   }
-  const int c = static_cast<int>(total);
-  const int mine = max(0, min(kCU, c - j0));   // entries this thread holds
+  auto valid = [&](int u) { return u < R && tid + u * kCT < c; };
   bool keep_all = false;
   uint32_t kth = 0, need_eq = 0;
   if (c == k) {
     keep_all = true;
   } else {
-    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
-#pragma unroll
-    for (int u = 0; u < kCU; ++u) {
-      if (u < mine) {
-        kmin = min(kmin, ent[u].x);
-        kmax = max(kmax, ent[u].x);
-      }
-    }
-    block_minmax512(kmin, kmax, ws);
-    if (kmin == kmax) {
+    if (kmin == kmax) {   // the listed keys' range, from the slices' own minima and maxima
       kth = kmin;
       need_eq = static_cast<uint32_t>(k);
     } else {
@@ -1042,9 +1095,9 @@ __global__ void __launch_bounds__(kCT, 1) topk_cluster_kernel(const float* __res
       __syncthreads();
 #pragma unroll
       for (int u = 0; u < kCU; ++u)
-        if (u < mine) atomicAdd(&hist[(ent[u].x >> sh) & (kBins - 1)], 1u);
+        if (valid(u)) atomicAdd(&hist[(ent[u].x >> sh) & (kBins - 1)], 1u);
       __syncthreads();
-      find_bin(hist, kBins, static_cast<uint32_t>(k), ws, sel);
+      find_bin2(hist, static_cast<uint32_t>(k), ws, sel);
       const uint32_t B = sel[0];
       uint32_t krem = static_cast<uint32_t>(k) - sel[1];
       const uint32_t hi_mask = (sh + 11 >= 32) ? 0u : (0xFFFFFFFFu << (sh + 11));
@@ -1056,21 +1109,34 @@ __global__ void __launch_bounds__(kCT, 1) topk_cluster_kernel(const float* __res
         uint32_t* buf = hist;   // kBins + 2 kCCap words (the histogram and this CTA's list) >= kCCap
 #pragma unroll
         for (int u = 0; u < kCU; ++u)
-          if (u < mine && ((ent[u].x >> sh) & (kBins - 1)) == B) buf[atomicAdd(&sel[2], 1u)] = ent[u].x;
+          if (valid(u) && ((ent[u].x >> sh) & (kBins - 1)) == B) buf[atomicAdd(&sel[2], 1u)] = ent[u].x;
         __syncthreads();
         if (warp == 0) {
           const int mb = static_cast<int>(inbin);
-          for (int bit = sh - 1; bit >= 0; --bit) {
-            const uint32_t want = (prefix >> bit) | 1u;
-            uint32_t cntb = 0;
-            for (int i0 = 0; i0 < mb; i0 += 32) {
-              const int i = i0 + lane;
-              cntb += __popc(__ballot_sync(0xffffffffu, i < mb && (buf[i] >> bit) == want));
+          if (mb <= 32) {   // the usual case: the bin's keys in registers, one ballot per bit
+            const bool have = lane < mb;
+            const uint32_t key = have ? buf[lane] : 0u;
+            for (int bit = sh - 1; bit >= 0; --bit) {
+              const uint32_t want = (prefix >> bit) | 1u;
+              const uint32_t cntb = __popc(__ballot_sync(0xffffffffu, have && (key >> bit) == want));
+              if (cntb >= krem)
+                prefix |= 1u << bit;
+              else
+                krem -= cntb;
             }
-            if (cntb >= krem)
-              prefix |= 1u << bit;
-            else
-              krem -= cntb;
+          } else {
+            for (int bit = sh - 1; bit >= 0; --bit) {
+              const uint32_t want = (prefix >> bit) | 1u;
+              uint32_t cntb = 0;
+              for (int i0 = 0; i0 < mb; i0 += 32) {
+                const int i = i0 + lane;
+                cntb += __popc(__ballot_sync(0xffffffffu, i < mb && (buf[i] >> bit) == want));
+              }
+              if (cntb >= krem)
+                prefix |= 1u << bit;
+              else
+                krem -= cntb;
+            }
           }
           if (lane == 0) {
             sel[0] = prefix;
@@ -1085,31 +1151,49 @@ __global__ void __launch_bounds__(kCT, 1) topk_cluster_kernel(const float* __res
       need_eq = krem;
     }
   }
-  // ordered emission: one CTA-wide scan of (entries > K*, entries == K*) per thread
-  uint32_t gt_n = 0, eq_n = 0;
+  // ordered emission: per round a warp scan of (entries > K*, entries == K*), one exchange of the
+  // warps' round totals (in the list, no longer needed), then every kept entry's position
+  uint32_t* xs = reinterpret_cast<uint32_t*>(list);   // [kCU][kCWarps]
+  uint32_t pk[kCU], incl[kCU];
 #pragma unroll
   for (int u = 0; u < kCU; ++u) {
-    if (u < mine) {
-      gt_n += (keep_all || ent[u].x > kth) ? 1u : 0u;
-      eq_n += (!keep_all && ent[u].x == kth) ? 1u : 0u;
+    pk[u] = incl[u] = 0u;
+    if (u < R) {   // uniform
+      const bool val = valid(u);
+      const bool gt = val && (keep_all || ent[u].x > kth), eq = val && !keep_all && ent[u].x == kth;
+      pk[u] = (gt ? 0x10000u : 0u) | (eq ? 1u : 0u);
+      uint32_t x = pk[u];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      incl[u] = x;
+      if (lane == 31) xs[u * kCWarps + warp] = x;
     }
   }
-  uint32_t all;
-  const uint32_t ex = block_excl_scan((gt_n << 16) | eq_n, ws, &all);
-  uint32_t gt_run = ex >> 16, eq_run = ex & 0xFFFFu;
+  __syncthreads();
+  uint32_t gt_tot = 0, eq_tot = 0;   // entries of the earlier rounds
 #pragma unroll
   for (int u = 0; u < kCU; ++u) {
-    if (u < mine) {
-      const bool gt = keep_all || ent[u].x > kth, eq = !keep_all && ent[u].x == kth;
-      if (gt) {
-        const uint32_t p = gt_run + min(eq_run, need_eq);
-        if (p < static_cast<uint32_t>(k)) out[p] = static_cast<int32_t>(ent[u].y);
-        ++gt_run;
-      } else if (eq) {
-        if (eq_run < need_eq && gt_run + eq_run < static_cast<uint32_t>(k)) out[gt_run + eq_run] = static_cast<int32_t>(ent[u].y);
-        ++eq_run;
-      }
+    if (u >= R) break;   // uniform
+    uint32_t before = 0, all = 0;
+#pragma unroll
+    for (int w = 0; w < kCWarps; ++w) {
+      const uint32_t t = xs[u * kCWarps + w];
+      before += w < warp ? t : 0u;
+      all += t;
     }
+    const uint32_t ex = before + incl[u] - pk[u];
+    const uint32_t gt_run = gt_tot + (ex >> 16), eq_run = eq_tot + (ex & 0xFFFFu);
+    if (pk[u] >> 16) {
+      const uint32_t p = gt_run + min(eq_run, need_eq);
+      if (p < static_cast<uint32_t>(k)) out[p] = static_cast<int32_t>(ent[u].y);
+    } else if (pk[u] & 1u) {
+      if (eq_run < need_eq && gt_run + eq_run < static_cast<uint32_t>(k)) out[gt_run + eq_run] = static_cast<int32_t>(ent[u].y);
+    }
+    gt_tot += all >> 16;
+    eq_tot += all & 0xFFFFu;
   }
 }
 
