@@ -292,17 +292,30 @@ __device__ __forceinline__ void select_row(const uint2* __restrict__ cand, const
       __syncthreads();
       if (warp == 0) {
         const int mb = static_cast<int>(inbin);
-        for (int bit = sh - 1; bit >= 0; --bit) {
-          const uint32_t want = (prefix >> bit) | 1u;
-          uint32_t cntb = 0;
-          for (int base = 0; base < mb; base += 32) {
-            const int i = base + lane;
-            cntb += __popc(__ballot_sync(0xffffffffu, i < mb && (buf[i] >> bit) == want));
+        if (mb <= 32) {   // the usual case: the bin's keys in registers, one ballot per bit
+          const bool have = lane < mb;
+          const uint32_t key = have ? buf[lane] : 0u;
+          for (int bit = sh - 1; bit >= 0; --bit) {
+            const uint32_t want = (prefix >> bit) | 1u;
+            const uint32_t cntb = __popc(__ballot_sync(0xffffffffu, have && (key >> bit) == want));
+            if (cntb >= krem)
+              prefix |= 1u << bit;
+            else
+              krem -= cntb;
           }
-          if (cntb >= krem)
-            prefix |= 1u << bit;
-          else
-            krem -= cntb;
+        } else {
+          for (int bit = sh - 1; bit >= 0; --bit) {
+            const uint32_t want = (prefix >> bit) | 1u;
+            uint32_t cntb = 0;
+            for (int base = 0; base < mb; base += 32) {
+              const int i = base + lane;
+              cntb += __popc(__ballot_sync(0xffffffffu, i < mb && (buf[i] >> bit) == want));
+            }
+            if (cntb >= krem)
+              prefix |= 1u << bit;
+            else
+              krem -= cntb;
+          }
         }
         if (lane == 0) {
           sel[0] = prefix;
