@@ -367,14 +367,15 @@ def _copy_stream(device, which: str = "in") -> "torch.cuda.Stream":
 
 def prefill_host(q, k, v, qi, ki, *, topk: int, device="cuda", out=None, q_pos0: int = 0, rope_theta: float = 0.0,
                  head_w=None, mode: int = QSA_SCORE_RELU_SUM, scale: float | None = None, workspace=None,
-                 device_buffers: dict | None = None, chunks: int = 32, yarn=None):
+                 device_buffers: dict | None = None, chunks: int = 32, sel_chunks: int = 2, yarn=None):
     """The QSA layer for a prefill whose inputs live in (pinned) host memory; returns the output in
-    host memory.  Transfers overlap the kernels.  ki and qi are copied first and the pooling and
-    block selection of all rows run while q, k and v follow in ``chunks`` causal row chunks on a
-    copy stream: chunk c's attention needs only its own query rows and the keys and values of the
-    positions before its end, so it starts as soon as that chunk has arrived, and its output goes
-    back on a second copy stream while the next chunk is computed.  ``device_buffers`` (name ->
-    device tensor) lets a caller reuse device memory.
+    host memory.  Transfers overlap the kernels.  ki and qi are copied first, in ``sel_chunks``
+    causal row chunks: the pooling and block selection of a chunk's rows need only the indexer keys
+    and queries up to the chunk's end, so they start as soon as those have arrived.  q, k and v
+    follow in ``chunks`` causal row chunks on the same copy stream: chunk c's attention needs only
+    its own query rows and the keys and values of the positions before its end, so it starts as
+    soon as that chunk has arrived, and its output goes back on a second copy stream while the next
+    chunk is computed.  ``device_buffers`` (name -> device tensor) lets a caller reuse device memory.
     Returns dict(out=host tensor, lse=device tensor, idx=device tensor)."""
     dev = torch.device(device)
     main = torch.cuda.current_stream(dev)
@@ -396,12 +397,21 @@ def prefill_host(q, k, v, qi, ki, *, topk: int, device="cuda", out=None, q_pos0:
     # row chunks (one sequence only: the rows of a chunk are then contiguous in every tensor)
     n = max(1, min(chunks, Tq)) if B == 1 else 1
     bounds = [(Tq * c) // n for c in range(n + 1)]
+    # selection chunks: query rows [slo, shi), whose blocks lie below key position q_pos0 + shi; the
+    # pooled keys of a chunk start on a whole block (row bounds in multiples of 4 when q_pos0 is)
+    ns = max(1, min(sel_chunks, Tq // 4)) if (B == 1 and q_pos0 % 4 == 0 and Tk == q_pos0 + Tq) else 1
+    sbounds = [0] + [(Tq * c // ns) // 4 * 4 for c in range(1, ns)] + [Tq]
     cin.wait_stream(main)   # the device buffers may still be read by earlier work on `main`
     with torch.cuda.stream(cin):
-        bufs["ki"].copy_(ki, non_blocking=True)
-        bufs["qi"].copy_(qi, non_blocking=True)
-        sel_ready = torch.cuda.Event()
-        sel_ready.record(cin)
+        sel_ready = []
+        for c in range(ns):
+            slo, shi = sbounds[c], sbounds[c + 1]
+            klo, khi = (q_pos0 + slo if c else 0), (q_pos0 + shi if c < ns - 1 else Tk)
+            bufs["ki"][:, klo:khi].copy_(ki[:, klo:khi], non_blocking=True)
+            bufs["qi"][:, slo:shi].copy_(qi[:, slo:shi], non_blocking=True)
+            ev = torch.cuda.Event()
+            ev.record(cin)
+            sel_ready.append(ev)
         arrived = []
         kv_done = 0   # key/value positions already sent
         for c in range(n):
@@ -415,13 +425,32 @@ def prefill_host(q, k, v, qi, ki, *, topk: int, device="cuda", out=None, q_pos0:
             ev = torch.cuda.Event()
             ev.record(cin)
             arrived.append(ev)
-    main.wait_event(sel_ready)
-    kp = qsa_pool_block_keys(bufs["ki"], bufs["kp"], rope_theta=rope_theta, yarn=yarn)
-    qr = (qsa_rope_index_queries(bufs["qi"], rope_theta=rope_theta, q_pos0=q_pos0, yarn=yarn) if rope_theta > 0
-          else bufs["qi"])
-    idx = qsa_select_topk(topk, qi=qr, kp=kp, head_w=head_w, q_pos0=q_pos0, mode=mode, workspace=workspace,
-                          idx=bufs.get("idx"))
-    bufs["idx"] = idx
+    kp = bufs["kp"]
+    if "idx" not in bufs:
+        bufs["idx"] = torch.empty(B, Tq, topk, dtype=torch.int32, device=dev)
+    idx = bufs["idx"]
+    for c in range(ns):
+        slo, shi = sbounds[c], sbounds[c + 1]
+        main.wait_event(sel_ready[c])
+        if ns == 1:
+            qsa_pool_block_keys(bufs["ki"], kp, rope_theta=rope_theta, yarn=yarn)
+            qr = (qsa_rope_index_queries(bufs["qi"], rope_theta=rope_theta, q_pos0=q_pos0, yarn=yarn)
+                  if rope_theta > 0 else bufs["qi"])
+            qsa_select_topk(topk, qi=qr, kp=kp, head_w=head_w, q_pos0=q_pos0, mode=mode, workspace=workspace,
+                            idx=idx)
+            break
+        # keys of positions [klo, khi) pooled into blocks [klo/4, khi/4); the chunk's rows select
+        # among blocks below (q_pos0 + shi - 1) / 4
+        klo, khi = (q_pos0 + slo if c else 0), (q_pos0 + shi if c < ns - 1 else Tk)
+        if khi // 4 > klo // 4:
+            qsa_pool_block_keys(bufs["ki"][:, klo:khi // 4 * 4], kp[:, klo // 4:khi // 4], pos0=klo,
+                                rope_theta=rope_theta, yarn=yarn)
+        qc = bufs["qi"][:, slo:shi]
+        qr = (qsa_rope_index_queries(qc, rope_theta=rope_theta, q_pos0=q_pos0 + slo, yarn=yarn) if rope_theta > 0
+              else qc)
+        nbk = max(1, (q_pos0 + shi - 1) // 4)
+        qsa_select_topk(topk, qi=qr, kp=kp[:, :nbk], head_w=head_w, q_pos0=q_pos0 + slo, mode=mode,
+                        workspace=workspace, idx=idx[:, slo:shi])
     for c in range(n):
         lo, hi = bounds[c], bounds[c + 1]
         if hi <= lo:

@@ -159,3 +159,49 @@ def test_cluster_split_merge_matches_the_merge_kernel_and_the_oracle(B, L, k):
     st = H.compare_decode(idx.cpu().numpy()[seqs], outs[sp][0][seqs], outs[sp][1][seqs], h["q"], h["k"], h["v"],
                           h["qi"], I.bits(kp), np.array(seqlens), seqs, topk=k)
     print("cluster decode:", st)
+
+
+def test_cluster_split_merge_one_kv_head_and_clusters_of_eight():
+    """Hkv = 1 (8 query heads on one KV head) with 8 splits per sequence (clusters of 8 CTAs) and
+    Hkv = 2 with 3 splits, against one split and the oracle."""
+    from tests import harness as H
+    for Hq, Hkv, B, splits in [(8, 1, 5, 8), (16, 2, 7, 3)]:
+        w = I.WORKLOADS["decode_256k"].with_(B=B, T=12000, Hq=Hq, Hkv=Hkv, seed=Hq * 100 + B)
+        seqlens = [12000, 9001, 4 * 300 + 2, 12000 - 3, 33, 6000, 7777][:B]
+        x = I.make_decode(w, DEV, seqlens=seqlens)
+        kp = Q.qsa_pool_block_keys(x["ki"])
+        idx = Q.qsa_select_topk(256, qi=x["qi"], kp=kp, seqlens=x["seqlens"])
+        assert Q.lib().qsa_decode_split_merge(B, Hq, Hkv, 128, splits) == 1
+        o1, l1 = Q.qsa_sparse_attn_decode(x["q"], x["k"], x["v"], x["seqlens"], idx, num_splits=1)
+        oc, lc = Q.qsa_sparse_attn_decode(x["q"], x["k"], x["v"], x["seqlens"], idx, num_splits=splits)
+        torch.cuda.synchronize()
+        assert Q.qsa_get_device_status() == Q.QSA_OK
+        P.assert_outputs_close(I.bits(oc), I.bits(o1))
+        assert torch.allclose(lc, l1, atol=1e-4)
+        h = {n: I.bits(x[n]) for n in ("q", "k", "v", "qi")}
+        H.compare_decode(idx.cpu().numpy(), I.bits(oc), lc.cpu().numpy(), h["q"], h["k"], h["v"], h["qi"], I.bits(kp),
+                         np.array(seqlens), list(range(B)), topk=256)
+
+
+def test_cluster_split_merge_reports_a_bad_length_and_finishes():
+    """A sequence length of 0 (no query position) in a cluster launch: its items record
+    INVALID_ARGUMENT and attend to nothing, every CTA still passes both cluster barriers, the
+    other sequences are unaffected."""
+    B, L, k = 6, 8000, 128
+    w = I.WORKLOADS["decode_256k"].with_(B=B, T=L, seed=3)
+    seqlens = [L, 5000, 0, L, 1, 7000]
+    x = I.make_decode(w, DEV, seqlens=seqlens)
+    kp = Q.qsa_pool_block_keys(x["ki"])
+    good = torch.tensor([L, 5000, 1, L, 1, 7000], dtype=torch.int32, device=DEV)
+    idx = Q.qsa_select_topk(k, qi=x["qi"], kp=kp, seqlens=good)
+    torch.cuda.synchronize()
+    assert Q.qsa_get_device_status() == Q.QSA_OK
+    assert Q.lib().qsa_decode_split_merge(B, 16, 2, 128, 4) == 1
+    ref, _ = Q.qsa_sparse_attn_decode(x["q"], x["k"], x["v"], good, idx, num_splits=4)
+    out, _ = Q.qsa_sparse_attn_decode(x["q"], x["k"], x["v"], x["seqlens"], idx, num_splits=4)
+    torch.cuda.synchronize()
+    assert Q.qsa_get_device_status() == Q.QSA_ERR_INVALID_ARGUMENT
+    keep = [0, 1, 3, 4, 5]
+    assert torch.equal(out[keep], ref[keep])
+    assert torch.isfinite(out.float()).all()
+    assert Q.qsa_get_device_status() == Q.QSA_OK

@@ -16,13 +16,15 @@ def _pinned(x):
     return {n: t.cpu().pin_memory() for n, t in x.items()}
 
 
-@pytest.mark.parametrize("chunks", [1, 3, 8])
-def test_prefill_host_matches_device_path(chunks):
-    w = I.WORKLOADS["prefill_32k"].with_(T=12000)
+@pytest.mark.parametrize("chunks,sel_chunks", [(1, 1), (3, 4), (8, 3), (8, 7)])
+def test_prefill_host_matches_device_path(chunks, sel_chunks):
+    """Attention in `chunks` row chunks, pooling and selection in `sel_chunks` (ragged ones too)."""
+    w = I.WORKLOADS["prefill_32k"].with_(T=12002)
     x = I.make_prefill(w, DEV)
     ref = Q.prefill(x["q"], x["k"], x["v"], x["qi"], x["ki"], topk=w.k)
     h = _pinned(x)
-    got = Q.prefill_host(h["q"], h["k"], h["v"], h["qi"], h["ki"], topk=w.k, device=DEV, chunks=chunks)
+    got = Q.prefill_host(h["q"], h["k"], h["v"], h["qi"], h["ki"], topk=w.k, device=DEV, chunks=chunks,
+                         sel_chunks=sel_chunks)
     torch.cuda.synchronize()
     assert Q.qsa_get_device_status() == Q.QSA_OK
     assert torch.equal(got["idx"], ref["idx"])
@@ -51,4 +53,21 @@ def test_prefill_host_two_sequences_single_chunk():
     h = _pinned(x)
     got = Q.prefill_host(h["q"], h["k"], h["v"], h["qi"], h["ki"], topk=w.k, device=DEV)
     torch.cuda.synchronize()
+    assert torch.equal(got["out"], ref["out"].cpu())
+
+
+@pytest.mark.parametrize("q0", [3000, 3001])
+def test_prefill_host_window_with_rope_and_selection_chunks(q0):
+    """Rotated indexer keys and queries, a window starting on a block boundary (selection in chunks)
+    or inside a block (one selection call), against the device path."""
+    w = I.WORKLOADS["prefill_32k"].with_(T=10000)
+    x = I.make_prefill(w, DEV)
+    xq = {n: (t[:, q0:].contiguous() if n in ("q", "qi") else t) for n, t in x.items()}
+    ref = Q.prefill(xq["q"], xq["k"], xq["v"], xq["qi"], xq["ki"], topk=w.k, q_pos0=q0, rope_theta=10000.0)
+    h = _pinned(xq)
+    got = Q.prefill_host(h["q"], h["k"], h["v"], h["qi"], h["ki"], topk=w.k, device=DEV, q_pos0=q0, chunks=4,
+                         sel_chunks=3, rope_theta=10000.0)
+    torch.cuda.synchronize()
+    assert Q.qsa_get_device_status() == Q.QSA_OK
+    assert torch.equal(got["idx"], ref["idx"])
     assert torch.equal(got["out"], ref["out"].cpu())
