@@ -28,6 +28,7 @@
 // Entries -1 and the own block in an index list are skipped; other entries outside [0, own) are
 // skipped and recorded in the device status word.  Every mbarrier wait is bounded.
 #include <algorithm>
+#include <atomic>
 #include <cfloat>
 #include <mutex>
 
@@ -1035,14 +1036,15 @@ cudaError_t launch_attn_prefill(const DeviceInfo* di, const void* q, const void*
 bool decode_cluster_ok(const DeviceInfo* di, int B, int Hq, int Hkv, int D, int splits) {
   if (splits < 2 || splits > 8 || D != kD || Hq / Hkv > 8 || (Hkv != 1 && Hkv != 2)) return false;
   if (static_cast<long long>(B) * splits > di->num_sms) return false;
-  static int max_clusters[64][2][9];
+  static std::atomic<int> max_clusters[64][2][9];   // 0: not asked yet; -1: the query failed
   static std::once_flag once[64];
   std::call_once(once[di->device & 63], [] {
     cudaFuncSetAttribute(sparse_attn_kernel<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<1>::kSmem);
     cudaFuncSetAttribute(sparse_attn_kernel<2, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<2>::kSmem);
   });
-  int& mc = max_clusters[di->device & 63][Hkv - 1][splits];
-  if (mc == 0) {   // cached per device, KV head count and cluster size (-1: query failed)
+  std::atomic<int>& slot = max_clusters[di->device & 63][Hkv - 1][splits];
+  int mc = slot.load(std::memory_order_relaxed);
+  if (mc == 0) {   // cached per device, KV head count and cluster size (two first callers may both ask)
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(splits * B));
     cfg.blockDim = dim3(Hkv == 1 ? Cfg<1>::kThreads : Cfg<2>::kThreads);
@@ -1059,6 +1061,7 @@ bool decode_cluster_ok(const DeviceInfo* di, int B, int Hq, int Hkv, int D, int 
                                    : cudaOccupancyMaxActiveClusters(&n, sparse_attn_kernel<2, true>, &cfg);
     mc = (e == cudaSuccess && n > 0) ? n : -1;
     if (e != cudaSuccess) cudaGetLastError();
+    slot.store(mc, std::memory_order_relaxed);
   }
   return mc >= B;
 }
