@@ -392,14 +392,12 @@ def run_qsa(args):
         idxd = torch.empty(wd.B, wd.k, dtype=torch.int32, device=dev)
         outd = torch.empty_like(xd["q"])
         lsed = torch.empty(wd.B, wd.Hq, dtype=torch.float32, device=dev)
-        j = (wd.T - 1) // wd.blk          # the block holding the newest token
-        ki_last = xd["ki"][:, j * wd.blk:(j + 1) * wd.blk]
-        kp_last = kpd[:, j:j + 1]
 
         def dsel():
-            if (wd.T % wd.blk) == 0:       # the new token completed block j: pool that row of every sequence
-                Q.qsa_pool_block_keys(ki_last, kp_last, pos0=j * wd.blk)
-            Q.qsa_select_topk(wd.k, qi=xd["qi"], kp=kpd, seqlens=xd["seqlens"], idx=idxd, workspace=wsd)
+            # pool the block the new token completes (when it completes one) inside the score
+            # kernel, then score and select
+            Q.qsa_decode_select(wd.k, qi=xd["qi"], kp=kpd, ki=xd["ki"], seqlens=xd["seqlens"], idx=idxd,
+                                workspace=wsd)
 
         def datt():
             Q.qsa_sparse_attn_decode(xd["q"], xd["k"], xd["v"], xd["seqlens"], idxd, num_splits=splits, out=outd,
@@ -453,7 +451,7 @@ def run_qsa(args):
                   "ms_per_step": dms, "launch": "CUDA graph of one step, replayed",
                   "steps": dsteps, "num_splits": splits,
                   "step_breakdown_ms": {"score_topk": d_sel, "attention_and_merge": d_att},
-                  "gpu_launches_per_step": 1 + 2 + 1 + (1 if Q.qsa.lib().qsa_decode_split_merge(
+                  "gpu_launches_per_step": 2 + 1 + (1 if Q.qsa.lib().qsa_decode_split_merge(
                       wd.B, wd.Hq, wd.Hkv, wd.D, splits) == 2 else 0),
                   "roofline": {"bound": "hbm", "achieved": dgbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                                "frac": dgbs / pk["hbm_gbs"], "bytes_per_step": dw["bytes"],

@@ -370,6 +370,38 @@ static qsa_status_t check_attn_shape(int Hq, int Hkv, int D, int blk, int k_bloc
   return QSA_OK;
 }
 
+qsa_status_t qsa_decode_select(const void* qi, void* kp, const void* ki, int64_t ki_batch_stride,
+                               const float* head_w, const int32_t* seqlens, int B, int NBk, int Hi, int Di, int blk,
+                               qsa_score_mode_t mode, const qsa_rope_params_t* rope, int k, int32_t* idx,
+                               void* workspace, size_t ws_bytes, void* stream) {
+  if (k < 1 || B < 0 || NBk < 0 || ki_batch_stride < 0) return QSA_ERR_INVALID_ARGUMENT;
+  if (blk != 4) return QSA_ERR_UNSUPPORTED;
+  if (B == 0) return QSA_OK;
+  if (seqlens == nullptr || idx == nullptr || !ok_ptr(ki)) return QSA_ERR_INVALID_ARGUMENT;
+  RopeParams rp;
+  if (resolve_rope(rope, &rp) != QSA_OK) return QSA_ERR_INVALID_ARGUMENT;
+  const long long kis = ki_batch_stride ? ki_batch_stride : static_cast<long long>(NBk) * blk * Di;
+  if (kis < static_cast<long long>(NBk) * blk * Di) return QSA_ERR_INVALID_ARGUMENT;
+  qsa_status_t st = check_score_args(qi, kp, seqlens, B, 1, NBk, Hi, Di, blk, 0, mode);
+  if (st != QSA_OK) return st;
+  if (NBk == 0) return qsa_select_topk(nullptr, 0, qi, kp, head_w, seqlens, B, 1, NBk, Hi, Di, blk, 0, mode, k, idx,
+                                       workspace, ws_bytes, stream);
+  float* ws = static_cast<float*>(workspace);
+  const long long row_bytes = static_cast<long long>(NBk) * 4;
+  if (ws == nullptr || static_cast<long long>(ws_bytes) < row_bytes * B) return QSA_ERR_WORKSPACE_TOO_SMALL;
+  const DeviceInfo* di = device_info();
+  if (!di) return QSA_ERR_CUDA;
+  cudaStream_t s = S(stream);
+  const NewBlockPool np{static_cast<const uint16_t*>(ki), static_cast<uint16_t*>(kp), kis,
+                        static_cast<long long>(NBk) * Di, rp};
+  const int parts = topk_cluster_parts(di, B, NBk, k);
+  cudaError_t e = launch_score_decode(di, qi, kp, head_w, seqlens, B, NBk, Hi, Di, blk, mode, ws, NBk, s, &np);
+  if (e == cudaSuccess)
+    e = parts > 0 ? launch_topk_cluster(di, ws, NBk, seqlens, B, NBk, blk, k, idx, parts, s)
+                  : launch_topk(di, ws, NBk, NBk, seqlens, 1, NBk, blk, 0, 0, B, 0, 1, k, idx, s);
+  return cuda_status(e);
+}
+
 qsa_status_t qsa_sparse_attn_prefill(const void* q, const void* k, const void* v, const int32_t* idx, int B, int Tq,
                                      int Tk, int Hq, int Hkv, int D, int k_blocks, int blk, int64_t q_pos0,
                                      float scale, void* out, float* lse, void* stream) {

@@ -22,7 +22,7 @@
 #include <mutex>
 #include <type_traits>
 
-#include "launch.h"
+#include "pool_math.cuh"
 
 namespace qsa {
 namespace {
@@ -489,19 +489,31 @@ constexpr int kDecStages = QSA_DEC_STAGES;
 constexpr int kDecThreads = 160;
 constexpr int kDecSmem = 1024 + kDecStages * kKpBytes + 128;
 
+// With np.ki set, the last warp of each sequence's first CTA first pools that sequence's newest
+// block when the new token has just completed it (L a multiple of blk): kp[b][L/blk - 1] from the
+// key cache rows (L/blk - 1) * blk .. L - 1, rotated at their first position.  That block is the
+// query's own block, never scored here (candidates are the blocks below it), so the pooling needs
+// no ordering with this kernel's reads of kp (a tile may read the row only inside its masked tail).
 template <int HI>
 __global__ void __launch_bounds__(kDecThreads) score_decode_kernel(const __grid_constant__ CUtensorMap kp_map,
                                                                    const uint16_t* __restrict__ qi,
                                                                    const float* __restrict__ head_w,
                                                                    const int32_t* __restrict__ seqlens, int NBk,
                                                                    int blk, int mode, float* __restrict__ scores,
-                                                                   long long ld, int part_len, KernelCtl ctl) {
+                                                                   long long ld, int part_len, KernelCtl ctl,
+                                                                   NewBlockPool np) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(ring + kDecStages * kKpBytes);
   uint64_t* empty = full + kDecStages;
   const int b = blockIdx.y;
   const int L = seqlens[b];
+  if (np.ki != nullptr && blockIdx.x == 0 && (threadIdx.x >> 5) == kDecThreads / 32 - 1 && L >= blk &&
+      L % blk == 0 && L / blk <= NBk) {
+    const long long j = L / blk - 1;
+    pool_row_warp(np.ki + b * np.ki_bs + j * blk * kDi, np.kp + b * np.kp_bs + j * kDi, kDi, blk, np.rp,
+                  static_cast<double>(j * blk));
+  }
   int nb = L >= 1 ? (L - 1) / blk : 0;
   if (L < 1 || nb > NBk) {
     if (blockIdx.x == 0 && threadIdx.x == 0) record_status(ctl, kStBadArg);
@@ -734,7 +746,7 @@ cudaError_t launch_score_filter(const DeviceInfo* di, const void* qi, const void
 
 cudaError_t launch_score_decode(const DeviceInfo* di, const void* qi, const void* kp, const float* head_w,
                                 const int32_t* seqlens, int B, int NBk, int Hi, int Di, int blk, int mode,
-                                float* scores, long long ld, cudaStream_t s) {
+                                float* scores, long long ld, cudaStream_t s, const NewBlockPool* np) {
   (void)Di;
   if (B <= 0 || NBk <= 0) return cudaSuccess;
   const KernelCtl ctl = kernel_ctl(di);
@@ -767,11 +779,12 @@ cudaError_t launch_score_decode(const DeviceInfo* di, const void* qi, const void
   const int part_len = part_tiles * kM;
   dim3 grid((NBk + part_len - 1) / part_len, B);
   const uint16_t* q = static_cast<const uint16_t*>(qi);
+  const NewBlockPool pool = np ? *np : NewBlockPool{};
   switch (Hi) {
-    case 1: score_decode_kernel<1><<<grid, kDecThreads, kDecSmem, s>>>(kmap, q, head_w, seqlens, NBk, blk, mode, scores, ld, part_len, ctl); break;
-    case 2: score_decode_kernel<2><<<grid, kDecThreads, kDecSmem, s>>>(kmap, q, head_w, seqlens, NBk, blk, mode, scores, ld, part_len, ctl); break;
-    case 4: score_decode_kernel<4><<<grid, kDecThreads, kDecSmem, s>>>(kmap, q, head_w, seqlens, NBk, blk, mode, scores, ld, part_len, ctl); break;
-    case 8: score_decode_kernel<8><<<grid, kDecThreads, kDecSmem, s>>>(kmap, q, head_w, seqlens, NBk, blk, mode, scores, ld, part_len, ctl); break;
+    case 1: score_decode_kernel<1><<<grid, kDecThreads, kDecSmem, s>>>(kmap, q, head_w, seqlens, NBk, blk, mode, scores, ld, part_len, ctl, pool); break;
+    case 2: score_decode_kernel<2><<<grid, kDecThreads, kDecSmem, s>>>(kmap, q, head_w, seqlens, NBk, blk, mode, scores, ld, part_len, ctl, pool); break;
+    case 4: score_decode_kernel<4><<<grid, kDecThreads, kDecSmem, s>>>(kmap, q, head_w, seqlens, NBk, blk, mode, scores, ld, part_len, ctl, pool); break;
+    case 8: score_decode_kernel<8><<<grid, kDecThreads, kDecSmem, s>>>(kmap, q, head_w, seqlens, NBk, blk, mode, scores, ld, part_len, ctl, pool); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaPeekAtLastError();

@@ -44,9 +44,17 @@ cudaError_t launch_score_prefill(const DeviceInfo* di, const void* qi, const voi
 cudaError_t launch_score_filter(const DeviceInfo* di, const void* qi, const void* kp, const float* head_w, int Tq,
                                 int NBk, int Hi, long long q_pos0, int mode, int b0, int nb, int row0, int rows,
                                 const float* tau, uint2* cand, int* cnt, int cap, cudaStream_t s);
+// Optional pooling of each sequence's newest completed block by the decode score kernel (ki
+// nullptr: none).  ki/kp batch strides in elements; kp rows of Di = 64 keys.
+struct NewBlockPool {
+  const uint16_t* ki;
+  uint16_t* kp;
+  long long ki_bs, kp_bs;
+  RopeParams rp;
+};
 cudaError_t launch_score_decode(const DeviceInfo* di, const void* qi, const void* kp, const float* head_w,
                                 const int32_t* seqlens, int B, int NBk, int Hi, int Di, int blk, int mode,
-                                float* scores, long long ld, cudaStream_t s);
+                                float* scores, long long ld, cudaStream_t s, const NewBlockPool* np = nullptr);
 
 // Top-k over score rows: row r of batch b (b0 <= b < b0 + nb, row0 <= r < row0 + rows) reads
 // scores + (b - b0) * batch_stride + (r - row0) * ld and writes idx + (b * Tq + r) * k.

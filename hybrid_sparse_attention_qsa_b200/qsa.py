@@ -40,6 +40,7 @@ SIGNATURES = {
     "qsa_rope_index_queries_rope": (_I, [_P, _P, _I, _I, _I, _I, _I64, _P, _P, _P]),
     "qsa_index_score": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I64, _I, _P, _I64, _P]),
     "qsa_select_topk": (_I, [_P, _I64, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I64, _I, _I, _P, _P, _SZ, _P]),
+    "qsa_decode_select": (_I, [_P, _P, _P, _I64, _P, _P, _I, _I, _I, _I, _I, _I, _P, _I, _P, _P, _SZ, _P]),
     "qsa_sparse_attn_prefill": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I64, _F, _P, _P, _P]),
     "qsa_sparse_attn_decode": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P, _P, _P, _SZ, _P]),
     "qsa_sparse_attn_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P, _P, _P]),
@@ -236,6 +237,36 @@ def qsa_select_topk(k: int, *, scores: torch.Tensor | None = None, qi: torch.Ten
     _check(lib().qsa_select_topk(_ptr(scores), ld, _ptr(qi), _ptr(kp), _ptr(head_w), _ptr(seqlens), B, Tq, NBk, Hi,
                                  Di, blk, q_pos0, mode, k, _ptr(idx), _ptr(workspace), ws_bytes, _stream(dev)),
            "qsa_select_topk")
+    return idx
+
+
+def qsa_decode_select(k: int, *, qi: torch.Tensor, kp: torch.Tensor, ki: torch.Tensor, seqlens: torch.Tensor,
+                      head_w: torch.Tensor | None = None, mode: int = QSA_SCORE_RELU_SUM, rope_theta: float = 0.0,
+                      yarn: dict | None = None, idx: torch.Tensor | None = None,
+                      workspace: torch.Tensor | None = None, blk: int = 4) -> torch.Tensor:
+    """One decode step's selection with the pooling of the newest block folded in: for every
+    sequence whose new token completes a block, kp[b, seqlens[b] // blk - 1] is pooled from the
+    key cache ki [B, Lmax, Di] first (as qsa_pool_block_keys would), then idx [B, k] is selected as
+    qsa_select_topk(k, qi=qi, kp=kp, seqlens=seqlens).  kp is updated in place."""
+    _need(qi, torch.bfloat16, "qi")
+    _need(kp, torch.bfloat16, "kp")
+    _need(seqlens, torch.int32, "seqlens")
+    if not ki.is_cuda or ki.dtype != torch.bfloat16 or not _batch_view_ok(ki):
+        raise ValueError("ki must be a CUDA bf16 [B, Lmax, Di] tensor with packed rows")
+    B, Hi, Di = qi.shape
+    NBk = kp.shape[1]
+    if workspace is None:
+        workspace = torch.empty(qsa_workspace_size(QSA_OP_SELECT_TOPK, B, 1, NBk, k, 0, 0), dtype=torch.uint8,
+                                device=qi.device)
+    if idx is None:
+        idx = torch.empty((B, k), dtype=torch.int32, device=qi.device)
+    _need(idx, torch.int32, "idx")
+    # without YaRN the rotary base goes through fp32, as in qsa_pool_block_keys(rope_theta=...)
+    rp = _rope_params(rope_theta if yarn else ctypes.c_float(rope_theta).value, yarn)
+    _check(lib().qsa_decode_select(_ptr(qi), _ptr(kp), _ptr(ki), ki.stride(0), _ptr(head_w), _ptr(seqlens), B, NBk,
+                                   Hi, Di, blk, mode, ctypes.byref(rp), k, _ptr(idx), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream(qi.device)),
+           "qsa_decode_select")
     return idx
 
 

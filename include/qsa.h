@@ -200,6 +200,25 @@ QSA_API qsa_status_t qsa_select_topk(const float* scores, int64_t ld_scores, con
                              size_t ws_bytes, void* stream);
 
 /*
+ * Decode selection with the pooling of the newest block folded in (one decode step's steps 1-3).
+ *   qi [B][Hi][Di] bf16 (rotated if RoPE is used), kp [B][NBk][Di] bf16 (read and written),
+ *   ki [B][Lmax][Di] bf16 key cache, row b at ki + b * ki_batch_stride (elements; 0 = NBk * blk *
+ *   Di), seqlens [B] -> idx [B][k] as qsa_select_topk with seqlens.
+ * For every sequence whose new token completes a block (seqlens[b] a multiple of blk and
+ * seqlens[b] / blk <= NBk), kp[b][seqlens[b]/blk - 1] is first set to the pooled (and, with rope,
+ * rotated) key of cache rows seqlens[b] - blk .. seqlens[b] - 1, exactly as qsa_pool_block_keys
+ * would write it.  That block is the query's own block, so the selection does not depend on it;
+ * the pooling runs inside the score kernel and saves a launch per step.  rope may be NULL (no
+ * rotation).  Workspace: at least B * NBk * 4 bytes (the score rows).
+ * Errors: as for qsa_select_topk.
+ */
+QSA_API qsa_status_t qsa_decode_select(const void* qi, void* kp, const void* ki, int64_t ki_batch_stride,
+                                       const float* head_w, const int32_t* seqlens, int B, int NBk, int Hi,
+                                       int Di, int blk, qsa_score_mode_t mode,
+                                       const qsa_rope_params_t* rope, int k, int32_t* idx, void* workspace,
+                                       size_t ws_bytes, void* stream);
+
+/*
  * Gather-sparse attention, prefill (step 4: exact attention over the selected tokens, GQA).
  *   q [B][Tq][Hq][D] bf16 for positions q_pos0 .. q_pos0+Tq-1 (q_pos0 + Tq <= Tk),
  *   k, v [B][Tk][Hkv][D] bf16, idx [B][Tq][k_blocks] int32 (from qsa_select_topk; entries -1

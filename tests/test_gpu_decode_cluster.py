@@ -205,3 +205,30 @@ def test_cluster_split_merge_reports_a_bad_length_and_finishes():
     assert torch.equal(out[keep], ref[keep])
     assert torch.isfinite(out.float()).all()
     assert Q.qsa_get_device_status() == Q.QSA_OK
+
+
+
+# ------------------------------------------------------------------ pooling folded into the selection
+@pytest.mark.parametrize("rope", [None, dict(theta=10000.0), dict(theta=10000.0, yarn=dict(factor=4.0, orig_ctx=4096))])
+def test_decode_select_pools_the_newest_block(rope):
+    """qsa_decode_select = pooling of the block the new token completes (bit-exact with
+    qsa_pool_block_keys) + the decode selection over the updated pooled keys (identical lists)."""
+    B, L, k = 6, 30000, 512
+    w = I.WORKLOADS["decode_256k"].with_(B=B, T=L, seed=55)
+    seqlens = [L, L - 1, 4 * 5000, 4 * 5000 + 3, 8, 4 * 7000]   # multiples of 4 complete a block
+    x = I.make_decode(w, DEV, seqlens=seqlens)
+    theta = rope["theta"] if rope else 0.0
+    yarn = rope.get("yarn") if rope else None
+    kp_full = Q.qsa_pool_block_keys(x["ki"], rope_theta=theta, yarn=yarn)
+    kp = kp_full.clone()
+    done = [b for b, n in enumerate(seqlens) if n % 4 == 0]
+    for b in done:
+        kp[b, seqlens[b] // 4 - 1] = 0       # the block each completing token finishes: not yet pooled
+    qi = x["qi"] if theta == 0 else Q.qsa_rope_index_queries(x["qi"], rope_theta=theta, seqlens=x["seqlens"],
+                                                             yarn=yarn)
+    ref = Q.qsa_select_topk(k, qi=qi, kp=kp_full, seqlens=x["seqlens"])
+    got = Q.qsa_decode_select(k, qi=qi, kp=kp, ki=x["ki"], seqlens=x["seqlens"], rope_theta=theta, yarn=yarn)
+    torch.cuda.synchronize()
+    assert Q.qsa_get_device_status() == Q.QSA_OK
+    assert torch.equal(kp, kp_full)          # every completed block pooled, nothing else touched
+    assert torch.equal(got, ref)
