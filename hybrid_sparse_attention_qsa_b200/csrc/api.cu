@@ -311,7 +311,7 @@ qsa_status_t qsa_select_topk(const float* scores, int64_t ld_scores, const void*
             e = launch_score_filter(di, qib, kpb, head_w, Tq, NBk, Hi, q_pos0, mode, 0, 1, r0, rows, tau, cand, cnt,
                                     fp.cap, s);
           if (e == cudaSuccess)
-            e = launch_select_candidates(di, cand, cnt, fp.cap, Tq, NBk, q_pos0, b, r0, rows, k, idx, fail, 0, s);
+            e = launch_select_candidates(di, cand, cnt, fp.cap, Tq, NBk, q_pos0, b, r0, rows, k, idx, fail, s);
           if (e == cudaSuccess)
             e = launch_topk_fallback(di, qi, kp, head_w, Hi, mode, Tq, NBk, q_pos0, b, fail, scratch, kFallbackCtas, k,
                                      idx, s);

@@ -73,10 +73,9 @@ cudaError_t launch_topk_cluster(const DeviceInfo* di, const float* scores, long 
 cudaError_t launch_select_tau(const DeviceInfo* di, const float* samp, long long ld, int NBk, long long q_pos0,
                               int row0, int rows, int cap, int rank, int kshift, int koff, float* tau, int* fail,
                               cudaStream_t s);
-// max_ctas > 0: a persistent grid of at most max_ctas CTAs walks the rows.
 cudaError_t launch_select_candidates(const DeviceInfo* di, const uint2* cand, const int* cnt, int cap, int Tq, int NBk,
                                      long long q_pos0, int b, int row0, int rows, int k, int32_t* idx, int* fail,
-                                     int max_ctas, cudaStream_t s);
+                                     cudaStream_t s);
 cudaError_t launch_topk_fallback(const DeviceInfo* di, const void* qi, const void* kp, const float* head_w, int Hi,
                                  int mode, int Tq, int NBk, long long q_pos0, int b, const int* fail, float* scratch,
                                  int nctas, int k, int32_t* idx, cudaStream_t s);

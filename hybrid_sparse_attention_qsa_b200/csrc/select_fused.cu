@@ -401,20 +401,17 @@ __device__ __forceinline__ void select_row(const uint2* __restrict__ cand, const
   }
 }
 
-// One CTA per row, or a persistent grid of fewer CTAs that walks the rows (so that it can run beside
-// the next chunk's score + filter kernel, one CTA per SM).
+// One CTA per row (a grid-strided loop over rows held ~40 more registers per thread live and cut
+// the resident CTAs per SM from 6 to 4).
 template <int U>
 __global__ void __launch_bounds__(kSelThreads) cand_select_kernel(const uint2* __restrict__ cand,
                                                                   const int* __restrict__ cnt, int cap, int Tq, int NBk,
-                                                                  long long q_pos0, int b, int row0, int rows, int k,
+                                                                  long long q_pos0, int b, int row0, int k,
                                                                   int32_t* __restrict__ idx, int* __restrict__ fail) {
   __shared__ __align__(16) uint32_t hist[kSelBins];   // histogram, then the k-th bin's keys
   __shared__ uint32_t ws[2 * kSelWarpsPerRow];
   __shared__ uint32_t sel[4];
-  for (int L = static_cast<int>(blockIdx.x); L < rows; L += static_cast<int>(gridDim.x)) {
-    select_row<U>(cand, cnt, cap, Tq, NBk, q_pos0, b, row0, k, idx, fail, L, hist, ws, sel);
-    __syncthreads();   // the next row reuses the shared memory
-  }
+  select_row<U>(cand, cnt, cap, Tq, NBk, q_pos0, b, row0, k, idx, fail, static_cast<int>(blockIdx.x), hist, ws, sel);
 }
 
 }  // namespace
@@ -430,16 +427,15 @@ cudaError_t launch_select_tau(const DeviceInfo* di, const float* samp, long long
 
 cudaError_t launch_select_candidates(const DeviceInfo* di, const uint2* cand, const int* cnt, int cap, int Tq, int NBk,
                                      long long q_pos0, int b, int row0, int rows, int k, int32_t* idx, int* fail,
-                                     int max_ctas, cudaStream_t s) {
+                                     cudaStream_t s) {
   (void)di;
   if (rows <= 0) return cudaSuccess;
   // lists of up to 2 * U * kSelThreads entries fit the registers; longer ones are refused (the
   // caller only plans caps that fit)
-  const int grid = max_ctas > 0 ? std::min(rows, max_ctas) : rows;
   if (cap <= 2 * 10 * kSelThreads)
-    cand_select_kernel<10><<<grid, kSelThreads, 0, s>>>(cand, cnt, cap, Tq, NBk, q_pos0, b, row0, rows, k, idx, fail);
+    cand_select_kernel<10><<<rows, kSelThreads, 0, s>>>(cand, cnt, cap, Tq, NBk, q_pos0, b, row0, k, idx, fail);
   else if (cap <= 2 * 20 * kSelThreads)
-    cand_select_kernel<20><<<grid, kSelThreads, 0, s>>>(cand, cnt, cap, Tq, NBk, q_pos0, b, row0, rows, k, idx, fail);
+    cand_select_kernel<20><<<rows, kSelThreads, 0, s>>>(cand, cnt, cap, Tq, NBk, q_pos0, b, row0, k, idx, fail);
   else
     return cudaErrorInvalidValue;
   return cudaPeekAtLastError();
