@@ -153,3 +153,23 @@ def test_decode_split_merge_host_rules(lib):
     assert lib.qsa_decode_split_merge(0, 16, 2, 128, 4) == -1
     assert lib.qsa_decode_split_merge(4, 16, 3, 128, 4) == -1   # Hq not a multiple of Hkv
     assert lib.qsa_decode_split_merge(4, 16, 2, 128, 0) == -1
+
+
+def test_decode_select_argument_checks(lib):
+    """Host-side checks run before any device work (no GPU needed)."""
+    def call(qi=FAKE, kp=FAKE, ki=FAKE, kis=0, sl=FAKE, B=2, NBk=64, Hi=4, Di=64, blk=4, mode=0, rope=None, k=8,
+             idx=FAKE, ws=FAKE, wsb=1 << 20):
+        return lib.qsa_decode_select(qi, kp, ki, kis, None, sl, B, NBk, Hi, Di, blk, mode, rope, k, idx, ws, wsb, None)
+    assert call(k=0) == Q.QSA_ERR_INVALID_ARGUMENT
+    assert call(blk=8) == Q.QSA_ERR_UNSUPPORTED
+    assert call(B=0) == Q.QSA_OK                                  # nothing to do
+    assert call(sl=None) == Q.QSA_ERR_INVALID_ARGUMENT            # decode needs the lengths
+    assert call(idx=None) == Q.QSA_ERR_INVALID_ARGUMENT
+    assert call(ki=None) == Q.QSA_ERR_INVALID_ARGUMENT            # the key cache to pool from
+    assert call(ki=P(8)) == Q.QSA_ERR_INVALID_ARGUMENT            # misaligned
+    assert call(kis=100) == Q.QSA_ERR_INVALID_ARGUMENT            # a row shorter than NBk * blk keys
+    assert call(Di=32) == Q.QSA_ERR_UNSUPPORTED
+    assert call(mode=2) == Q.QSA_ERR_INVALID_ARGUMENT
+    assert call(wsb=16) == Q.QSA_ERR_WORKSPACE_TOO_SMALL          # less than the B score rows
+    rp = Q.RopeParams(10000.0, 4.0, 0.0, 1.0, 32.0, 0.0)         # YaRN without an original context
+    assert call(rope=ctypes.byref(rp)) == Q.QSA_ERR_INVALID_ARGUMENT
