@@ -18,6 +18,11 @@
 // than kCap candidates (heavy ties), it is moved and the pass retried; after that, or when the row
 // is too long for the bitmap, an exact three-pass radix select over the row in memory is used.
 // Lanes of a warp that hit the same histogram bin are merged with match.any (one atomic per bin).
+//
+// Also in this file: a warp-per-row variant for launches with many short rows, the decode kernel
+// that spreads each of a few long rows over a thread-block cluster (slices merged through
+// distributed shared memory), and the exact redo of rows the filtered prefill selection could not
+// settle.
 #include <algorithm>
 #include <mutex>
 
