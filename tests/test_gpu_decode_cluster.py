@@ -232,3 +232,33 @@ def test_decode_select_pools_the_newest_block(rope):
     assert Q.qsa_get_device_status() == Q.QSA_OK
     assert torch.equal(kp, kp_full)          # every completed block pooled, nothing else touched
     assert torch.equal(got, ref)
+
+
+def test_many_sequences_take_one_cta_each():
+    """80 sequences on 148 SMs: fewer than 2 SMs per sequence, so the decode selection runs one CTA
+    per sequence (no cluster) and the split merge a merge kernel or one split; the pooling-folded
+    entry point gives the same lists; the oracle agrees on sampled sequences."""
+    B, L, k = 80, 24000, 256
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert sms // B < 2
+    w = I.WORKLOADS["decode_256k"].with_(B=B, T=L, seed=80)
+    seqlens = [L - (b * 37) % 5000 for b in range(B)]
+    x = I.make_decode(w, DEV, seqlens=seqlens)
+    kp_full = Q.qsa_pool_block_keys(x["ki"])
+    one = _select(x["qi"], kp_full, x["seqlens"], k, cluster=False)
+    two = _select(x["qi"], kp_full, x["seqlens"], k, cluster=True)
+    assert np.array_equal(one, two)
+    kp = kp_full.clone()
+    for b, n in enumerate(seqlens):
+        if n % 4 == 0:
+            kp[b, n // 4 - 1] = 0
+    got = Q.qsa_decode_select(k, qi=x["qi"], kp=kp, ki=x["ki"], seqlens=x["seqlens"])
+    torch.cuda.synchronize()
+    assert Q.qsa_get_device_status() == Q.QSA_OK
+    assert torch.equal(kp, kp_full)
+    assert np.array_equal(got.cpu().numpy(), two)
+    _oracle_rows(two, x["qi"], kp_full, np.array(seqlens), k, [0, 17, 40, 79])
+    out, lse = Q.qsa_sparse_attn_decode(x["q"], x["k"], x["v"], x["seqlens"], got)
+    ref, _ = Q.qsa_sparse_attn_decode(x["q"], x["k"], x["v"], x["seqlens"], got, num_splits=1)
+    torch.cuda.synchronize()
+    P.assert_outputs_close(I.bits(out), I.bits(ref))
