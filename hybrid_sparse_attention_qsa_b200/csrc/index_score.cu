@@ -427,11 +427,12 @@ __global__ void __launch_bounds__(kFiltThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive_relaxed(&tm_empty[acc]);   // the tile's TMEM loads are complete
       // counts of this tile per (quadrant, query) -> the offset of each query's entries
-      uint32_t mine = 0;   // lane q: this warp's count for query q
-#pragma unroll
-      for (int q = 0; q < QW; ++q) mine = lane == q ? static_cast<uint32_t>(__popc(m[q])) : mine;
       uint32_t* xc = xcnt + ((i & 1) * kFiltGroups + grp) * 4 * 32;
-      if (lane < QW) xc[quad * 32 + lane] = mine;
+      if (lane == 0) {   // this warp's count of each query (the masks are warp-uniform)
+#pragma unroll
+        for (int q = 0; q < QW; ++q) xc[quad * 32 + q] = static_cast<uint32_t>(__popc(m[q]));
+      }
+      __syncwarp();
       named_bar_sync(1 + grp, 128);
       if (lane < QW) {
         uint32_t pre = 0, tot = 0;

@@ -402,9 +402,10 @@ __device__ __forceinline__ void select_row(const uint2* __restrict__ cand, const
 }
 
 // One CTA per row (a grid-strided loop over rows held ~40 more registers per thread live and cut
-// the resident CTAs per SM from 6 to 4).
+// the resident CTAs per SM from 6 to 4).  At most 64 registers, for 8 resident rows per SM: the few
+// spills that costs are cheaper than the rows it adds in flight.
 template <int U>
-__global__ void __launch_bounds__(kSelThreads) cand_select_kernel(const uint2* __restrict__ cand,
+__global__ void __launch_bounds__(kSelThreads, 8) cand_select_kernel(const uint2* __restrict__ cand,
                                                                   const int* __restrict__ cnt, int cap, int Tq, int NBk,
                                                                   long long q_pos0, int b, int row0, int k,
                                                                   int32_t* __restrict__ idx, int* __restrict__ fail) {
