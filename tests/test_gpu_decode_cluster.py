@@ -262,3 +262,38 @@ def test_many_sequences_take_one_cta_each():
     ref, _ = Q.qsa_sparse_attn_decode(x["q"], x["k"], x["v"], x["seqlens"], got, num_splits=1)
     torch.cuda.synchronize()
     P.assert_outputs_close(I.bits(out), I.bits(ref))
+
+
+def test_cluster_with_unaligned_score_rows():
+    """NBk not a multiple of 4: every other sequence's score row starts off a 16-byte boundary, so
+    the cluster kernel's sample and slice loads take their scalar form; lists still equal the
+    one-CTA selection's and the oracle's."""
+    B, nbk, k = 7, 65537, 512
+    qi, kp = _case(B, nbk, 71)
+    seqlens = torch.tensor([4 * nbk, 4 * nbk - 2, 4 * 40001 + 1, 4 * nbk, 30001, 4 * 6145, 4 * nbk - 5],
+                           dtype=torch.int32, device=DEV)
+    one = _select(qi, kp, seqlens, k, cluster=False)
+    two = _select(qi, kp, seqlens, k, cluster=True)
+    assert np.array_equal(one, two)
+    _oracle_rows(two, qi, kp, seqlens.cpu().numpy(), k, [0, 1, 6])
+
+
+def test_decode_select_cache_too_short_is_reported():
+    """A length past the pooled-key cache (seqlens[b] / 4 > NBk) is an invalid argument recorded on
+    the device; nothing is pooled for it and the other sequences are unaffected."""
+    B, L, k = 3, 8000, 128
+    w = I.WORKLOADS["decode_256k"].with_(B=B, T=L, seed=12)
+    x = I.make_decode(w, DEV)
+    kp_full = Q.qsa_pool_block_keys(x["ki"])
+    good = torch.tensor([L, L, L - 4], dtype=torch.int32, device=DEV)
+    ref = Q.qsa_select_topk(k, qi=x["qi"], kp=kp_full, seqlens=good)
+    torch.cuda.synchronize()
+    assert Q.qsa_get_device_status() == Q.QSA_OK
+    bad = torch.tensor([L, L + 400, L - 4], dtype=torch.int32, device=DEV)
+    kp = kp_full.clone()
+    got = Q.qsa_decode_select(k, qi=x["qi"], kp=kp, ki=x["ki"], seqlens=bad)
+    torch.cuda.synchronize()
+    assert Q.qsa_get_device_status() == Q.QSA_ERR_INVALID_ARGUMENT
+    assert torch.equal(kp, kp_full)
+    assert torch.equal(got[[0, 2]], ref[[0, 2]])
+    assert Q.qsa_get_device_status() == Q.QSA_OK
