@@ -26,10 +26,6 @@ namespace {
 
 constexpr int kSelBins = 2048;    // bins of the first select pass (11 bits)
 
-__device__ __forceinline__ float key_to_float(uint32_t k) {
-  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
-}
-
 constexpr int kSelThreads = 128;
 constexpr int kSelWarpsPerRow = kSelThreads / 32;
 

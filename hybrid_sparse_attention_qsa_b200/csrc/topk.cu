@@ -787,37 +787,6 @@ constexpr int kCU = kCCap / kCT;           // merged entries per thread of CTA 0
 constexpr int kCLoads = 8;                 // 16-byte loads per thread per round (16384 scores)
 constexpr int kCSmem = kBins * 4 + kCCap * 8 + (kCLoads * kCWarps + 2 * kCWarps + 2 + 4 + 4) * 4;
 
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-// Every thread of every CTA of the cluster: shared-memory writes before it are visible to the
-// cluster's reads after it.
-__device__ __forceinline__ void cluster_barrier() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-// The address of `p` (this CTA's shared memory) in the shared memory of cluster CTA `rank`.
-__device__ __forceinline__ uint32_t cluster_addr(const void* p, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(p))), "r"(rank));
-  return r;
-}
-__device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t a) {
-  uint32_t v;
-  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
-  return v;
-}
-__device__ __forceinline__ uint2 ld_cluster_v2(uint32_t a) {
-  uint2 v;
-  asm volatile("ld.shared::cluster.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a) : "memory");
-  return v;
-}
-
-__device__ __forceinline__ float key_to_float(uint32_t k) {
-  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
-}
-
 // Block-wide min and max (ws: 2 * kCWarps words).  Ends synchronised.
 __device__ __forceinline__ void block_minmax512(uint32_t& kmin, uint32_t& kmax, uint32_t* ws) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -1038,9 +1007,9 @@ __global__ void __launch_bounds__(kCT, 1) topk_cluster_kernel(const float* __res
   if (tid == 0) misc[0] = count;
 
   // ---- 4. merge in CTA 0
-  cluster_barrier();
+  cluster_sync_all();
   if (part != 0) {
-    cluster_barrier();   // CTA 0 has read this CTA's list
+    cluster_sync_all();   // CTA 0 has read this CTA's list
     return;
   }
   uint32_t base[8], total = 0, kmin = 0xFFFFFFFFu, kmax = 0u;
@@ -1079,7 +1048,7 @@ __global__ void __launch_bounds__(kCT, 1) topk_cluster_kernel(const float* __res
       ent[u] = ld_cluster_v2(cluster_addr(list + rel, p));
     }
   }
-  cluster_barrier();
+  cluster_sync_all();
   if (!ok) {
     topk_global(s, n, k, out, hist, ws, sel);
     return;
