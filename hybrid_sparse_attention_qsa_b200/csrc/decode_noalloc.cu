@@ -49,12 +49,13 @@ extern "C" qsa_status_t qsa_sparse_attn_decode_noalloc(const void* q, const void
     return QSA_ERR_INVALID_ARGUMENT;
   const size_t per_split = static_cast<size_t>(B) * Hq * (D + 2) * sizeof(float);
   const int fit = static_cast<int>(std::min<size_t>(QSA_NOALLOC_DECODE_SCRATCH_BYTES / per_split, 1 << 20));
-  if (num_splits > 1 && num_splits > fit) return QSA_ERR_WORKSPACE_TOO_SMALL;
   const DeviceInfo* di = device_info();
   if (!di) return QSA_ERR_CUDA;
+  // The split count the launch really uses (never more splits than listed blocks) is what must fit.
   int splits = num_splits == 0 ? std::min(decode_default_splits(di, B, std::max(k_blocks, 1)), std::max(fit, 1))
                                : num_splits;
   splits = std::max(1, std::min(splits, std::max(k_blocks, 1)));
+  if (splits > 1 && splits > fit) return QSA_ERR_WORKSPACE_TOO_SMALL;
   float* part = nullptr;
   if (splits > 1) {
     cudaError_t e;

@@ -51,6 +51,7 @@ SIGNATURES = {
     "qsa_set_select_options": (_I, [_I, _I]),
     "qsa_set_wait_timeout_ns": (None, [_U64]),
     "qsa_wait_timeout_selftest": (_I, [_U64, _P]),
+    "qsa_probe_gather": (_I, [_P, _SZ, _I, _I, _I, _I, _I, _I, _I, _U64, _P]),
 }
 
 _lib = None
@@ -362,6 +363,20 @@ def qsa_wait_timeout_selftest(timeout_ns: int, device=None) -> None:
 
 
 # ---------------------------------------------------------------------------------------- whole path
+def qsa_probe_gather(src: torch.Tensor, *, chunk_bytes: int = 2048, method: int = 0, issuer_warps: int = 4,
+                     stages: int = 3, slots_per_warp: int = 8, iterations: int = 1000, ctas: int = 0,
+                     seed: int = 1) -> int:
+    """Gather-rate probe over the bytes of ``src`` (a contiguous CUDA tensor); returns the bytes the
+    launch delivers to shared memory.  Time it with CUDA events on the current stream."""
+    if not src.is_cuda or not src.is_contiguous():
+        raise ValueError("src must be a contiguous CUDA tensor")
+    nbytes = src.numel() * src.element_size()
+    _check(lib().qsa_probe_gather(_ptr(src), nbytes, chunk_bytes, method, issuer_warps, stages, slots_per_warp,
+                                  iterations, ctas, seed, _stream(src.device)), "qsa_probe_gather")
+    n_ctas = ctas or torch.cuda.get_device_properties(src.device).multi_processor_count
+    return n_ctas * issuer_warps * iterations * slots_per_warp * chunk_bytes
+
+
 def prefill(q, k, v, qi, ki, *, topk: int, q_pos0: int = 0, rope_theta: float = 0.0, head_w=None,
             mode: int = QSA_SCORE_RELU_SUM, scale: float | None = None, workspace=None, kp=None, yarn=None):
     """The QSA layer for a prefill: pool (+RoPE) -> [RoPE queries] -> score + top-k -> sparse attention.

@@ -35,8 +35,9 @@
  *     sequence length outside the cache, a wait that ran out of time) are skipped by the kernel
  *     and recorded in a per-device status word that qsa_get_device_status reads and clears.
  *   - Supported shapes: blk = 4; Di = 64 for scoring (any even Di <= 256 for pooling/RoPE);
- *     Hi in {1, 2, 4, 8}; attention D = 128, Hkv in {1, 2}, Hq/Hkv <= 8.  Other shapes return
- *     QSA_ERR_UNSUPPORTED.
+ *     Hi in {1, 2, 4, 8}; attention D in {128, 256}, Hkv in {1, 2}, Hq/Hkv <= 16 (the decode
+ *     split merge inside thread-block clusters needs D = 128 and Hq/Hkv <= 8; other decode shapes
+ *     merge through the workspace).  Other shapes return QSA_ERR_UNSUPPORTED.
  *   - Calls are thread-safe.  The library keeps only per-device caches (device attributes, the
  *     status word) and no other mutable global state.
  */
@@ -153,7 +154,8 @@ QSA_API qsa_status_t qsa_rope_index_queries_rope(const void* qi, void* qi_out, i
  *   scores[b][t][j] = s(t, j) for j < NB(p) = floor(p/blk), p = q_pos0 + t (or seqlens[b]-1 with
  *   seqlens != NULL, Tq == 1).  Entries j >= NB(p) are not written.
  * Prefill runs on tcgen05 tensor cores (TMEM accumulators, TMA-fed); decode (seqlens != NULL)
- * is a bandwidth-bound CUDA-core pass over the pooled-key cache.
+ * is a bandwidth-bound pass over the pooled-key cache on warp-level tensor-core MMAs (mma.sync,
+ * fp32 accumulate): its fp32 sums may differ from the prefill kernel's in the last bit.
  * Requires floor((q_pos0 + Tq - 1)/blk) <= NBk (prefill) and ld_scores >= NBk.
  * Errors: INVALID_ARGUMENT, UNSUPPORTED (Di != 64, Hi not in {1,2,4,8}, blk != 4).
  */
@@ -170,7 +172,9 @@ QSA_API qsa_status_t qsa_index_score(const void* qi, const void* kp, const float
  * scores != NULL: select from scores [B][Tq][ld_scores] (as written by qsa_index_score); qi, kp,
  *   head_w, mode and workspace are ignored.
  * scores == NULL: the scores are computed here.  Arguments as for qsa_index_score.  Two ways,
- *   both giving the same index lists; qsa_set_select_options can force one:
+ *   both selecting the top k of the same tensor-core fp32 scores (rows redone exactly, see below,
+ *   use CUDA-core fp32 scores, which may differ in the last bit, so such a row can differ from the
+ *   other way only by blocks tied within that rounding); qsa_set_select_options can force one:
  *   - materialised (decode; Hi of 1 or 2; short prefills): the scores are computed chunk by chunk
  *     into `workspace` (at least one score row of NBk floats; decode: B rows).  In decode, with
  *     few sequences (2 or more SMs per sequence), k <= 1024 and more than 6144 blocks, each
@@ -186,7 +190,8 @@ QSA_API qsa_status_t qsa_index_score(const void* qi, const void* kp, const float
  *     row's scores expected above it is read off these samples; the tensor-core score kernel then
  *     keeps only the scores at or above the threshold, in block order, and the top-k is selected
  *     from that list.  A row whose list is shorter than k or longer than its capacity is redone
- *     exactly over all its scores, so the result never depends on the thresholds.  Workspace per
+ *     exactly over all its scores (CUDA-core fp32 scores), so a threshold decides only which rows
+ *     are redone, never which blocks a row keeps beyond last-bit ties.  Workspace per
  *     row of a chunk: about 4 * NBk / 16 + 256 * max(64, ceil(5 k / 32)) bytes, plus
  *     128 * NBk * 4 bytes for the redo.
  *   qsa_workspace_size(QSA_OP_SELECT_TOPK, ...) gives a size that fits either way in few chunks
@@ -271,8 +276,11 @@ QSA_API qsa_status_t qsa_sparse_attn_decode(const void* q, const void* kcache, c
  * (QSA_NOALLOC_DECODE_SCRATCH_BYTES per GPU, held by every GPU that loads the library until the
  * process exits).  It calls no allocator.
  *   - num_splits == 0 picks the largest split count up to qsa_decode_default_splits that fits the
- *     array; an explicit num_splits > 1 whose partials, B * num_splits * Hq * (D + 2) * 4 bytes,
- *     exceed QSA_NOALLOC_DECODE_SCRATCH_BYTES returns QSA_ERR_WORKSPACE_TOO_SMALL.
+ *     array.  An explicit num_splits is first capped at max(k_blocks, 1), as in
+ *     qsa_sparse_attn_decode; if the capped count s > 1 needs partials, B * s * Hq * (D + 2) * 4
+ *     bytes, beyond QSA_NOALLOC_DECODE_SCRATCH_BYTES, the call returns QSA_ERR_WORKSPACE_TOO_SMALL.
+ *   - The array is read only when the splits merge through partials (qsa_decode_split_merge
+ *     returns 2); when they merge inside thread-block clusters it is not touched.
  *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
  *     that device current; make that first call before any stream capture that should contain it.
  *   - Every call, on every stream, shares the one array per device: calls whose kernels overlap on
@@ -338,6 +346,25 @@ QSA_API void qsa_set_wait_timeout_ns(uint64_t ns);
  * QSA_ERR_TIMEOUT and the context stays usable.
  */
 QSA_API qsa_status_t qsa_wait_timeout_selftest(uint64_t timeout_ns, void* stream);
+
+/*
+ * Gather-rate probe (measurement only; not a step of the method).  The sparse attention fetches
+ * every selected 4-token block of K and of V as one scattered chunk (2 KB at 2 KV heads x D 128)
+ * into a shared-memory ring; this call measures how fast the SMs can do that alone, which is the
+ * ceiling the attention's gather is compared with.  `ctas` CTAs (0 = one per SM) of `issuer_warps`
+ * warps each keep `stages` x `slots_per_warp` chunks in flight per warp and refill them
+ * `iterations` times from pseudo-random chunk-aligned offsets of src [src_bytes] (device memory,
+ * 16-byte aligned; a buffer that fits in L2 gives the L2 -> SM ceiling).  method 0: 1-D bulk copies
+ * (TMA engine, one per chunk); 1: 16-byte cp.async by every lane; 2: the two alternating by warp.
+ * Bytes delivered = CTAs * issuer_warps * iterations * slots_per_warp * chunk_bytes; time the
+ * launch with events on `stream`.  The landed data are not read.
+ * Errors: INVALID_ARGUMENT (null or misaligned src, chunk_bytes not a multiple of 16 in 16 .. 16384
+ * or above src_bytes, method outside 0..2, issuer_warps outside 1..16, slots_per_warp outside
+ * 1..32), UNSUPPORTED (stages outside 2..4, ring above 227 KB of shared memory).
+ */
+QSA_API qsa_status_t qsa_probe_gather(const void* src, size_t src_bytes, int chunk_bytes, int method,
+                                      int issuer_warps, int stages, int slots_per_warp, int iterations,
+                                      int ctas, uint64_t seed, void* stream);
 
 #ifdef __cplusplus
 }

@@ -173,3 +173,32 @@ def test_decode_select_argument_checks(lib):
     assert call(wsb=16) == Q.QSA_ERR_WORKSPACE_TOO_SMALL          # less than the B score rows
     rp = Q.RopeParams(10000.0, 4.0, 0.0, 1.0, 32.0, 0.0)         # YaRN without an original context
     assert call(rope=ctypes.byref(rp)) == Q.QSA_ERR_INVALID_ARGUMENT
+
+
+def test_declared_attention_shape_limits(lib):
+    """The supported-shape line of include/qsa.h and the host checks of the attention calls agree."""
+    src = open(os.path.join(ROOT, "include", "qsa.h")).read()
+    m = re.search(r"attention D in \{([0-9, ]+)\}, Hkv in \{([0-9, ]+)\}, Hq/Hkv <= (\d+)", src)
+    assert m, "the header states the attention shapes"
+    dims = [int(x) for x in m.group(1).split(",")]
+    hkvs = [int(x) for x in m.group(2).split(",")]
+    gmax = int(m.group(3))
+    assert dims == [128, 256] and hkvs == [1, 2] and gmax == 16
+
+    def pre(D, Hq, Hkv):
+        return lib.qsa_sparse_attn_prefill(FAKE, FAKE, FAKE, FAKE, 1, 8, 8, Hq, Hkv, D, 8, 4, 0, ctypes.c_float(0.1),
+                                           FAKE, None, P(0), )
+
+    def dec(D, Hq, Hkv):
+        return lib.qsa_sparse_attn_decode(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 100, Hq, Hkv, D, 64, 4, ctypes.c_float(0.1),
+                                          -1, FAKE, None, None, 0, None)
+
+    for D in (64, 96, 192, 512):
+        assert pre(D, 16, 2) == Q.QSA_ERR_UNSUPPORTED
+    for Hkv in hkvs:
+        for D in dims:
+            # the largest declared group passes the shape checks (it then fails only on num_splits = -1)
+            assert dec(D, gmax * Hkv, Hkv) == Q.QSA_ERR_INVALID_ARGUMENT
+            assert dec(D, (gmax + 1) * Hkv, Hkv) == Q.QSA_ERR_UNSUPPORTED
+            assert pre(D, (gmax + 1) * Hkv, Hkv) == Q.QSA_ERR_UNSUPPORTED
+    assert pre(128, 12, 3) == Q.QSA_ERR_UNSUPPORTED
