@@ -109,8 +109,9 @@ def gather_ceiling(dev, stream, w, sweep: bool = False) -> dict:
     import hybrid_sparse_attention_qsa_b200 as Q
     chunk = w.blk * w.Hkv * w.D * 2
     res = {"chunk_bytes": chunk, "config": dict(GATHER_PROBE)}
-    cases = [("l2_bulk", 32 << 20, 0, GATHER_PROBE), ("hbm_bulk", 4 << 30, 0, GATHER_PROBE),
-             ("l2_lsu", 32 << 20, 1, GATHER_PROBE), ("l2_mixed", 32 << 20, 2, GATHER_PROBE)]
+    wide = dict(issuer_warps=8, stages=3, slots_per_warp=4)   # the same ring, issued by 8 warps
+    cases = [("l2_bulk", 32 << 20, 0, GATHER_PROBE), ("l2_bulk_w8", 32 << 20, 0, wide),
+             ("hbm_bulk", 4 << 30, 0, GATHER_PROBE), ("l2_lsu", 32 << 20, 1, GATHER_PROBE)]
     if sweep:
         for iw, sl in ((1, 32), (2, 16), (8, 4), (8, 3), (12, 2), (16, 2)):
             cfg = dict(issuer_warps=iw, stages=3, slots_per_warp=sl)
@@ -133,6 +134,7 @@ def gather_ceiling(dev, stream, w, sweep: bool = False) -> dict:
             gbs = nb / (e0.elapsed_time(e1) / 1000) / 1e9
             best = gbs if best is None else max(best, gbs)
         res[name + "_gbs"] = best
+    res["ceiling_gbs"] = max(v for k, v in res.items() if k.startswith("l2_bulk") and k.endswith("_gbs"))
     assert Q.qsa_get_device_status() == 0
     del bufs
     torch.cuda.empty_cache()
@@ -323,38 +325,60 @@ def run_qsa(args):
     stream = torch.cuda.current_stream(dev)
 
     # ---------------------------------------------------------------- prefill (headline)
-    w = I.WORKLOADS[args.workload].with_(seed=I.WORKLOADS[args.workload].seed + 1000 * rank)
+    # One job: every rank draws the same seeded inputs.  With N > 1 the query rows are sharded in
+    # zig-zag chunks (shard.py): each rank keeps its rows' inputs, pools its indexer keys, takes part
+    # in one all-gather of K, V and the pooled keys per step, then selects and attends for its rows.
+    w = I.WORKLOADS[args.workload]
     x = I.make_prefill(w, dev)
     nbk = w.T // w.blk
-    ws_bytes = Q.qsa_workspace_size(Q.qsa.QSA_OP_SELECT_TOPK, w.B, w.T, nbk, w.k, w.Hq, w.D)
-    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
-    kp = torch.empty(w.B, nbk, w.Di, dtype=torch.bfloat16, device=dev)
-    idx = torch.empty(w.B, w.T, w.k, dtype=torch.int32, device=dev)
-    out = torch.empty_like(x["q"])
-    lse = torch.empty(w.B, w.T, w.Hq, dtype=torch.float32, device=dev)
+    sp = None
+    if world > 1:
+        from hybrid_sparse_attention_qsa_b200 import shard as SH
+        sp = SH.ShardedPrefill(w.B, w.T, w.Hq, w.Hkv, w.D, w.Hi, w.Di, w.k, world, rank, dev)
+        x = {n: [x[n][:, a:b].contiguous() for a, b in sp.ranges] for n in x}
+        ws = sp.ws
+        ws_bytes = ws.numel()
+        my_ranges = sp.ranges
+    else:
+        ws_bytes = Q.qsa_workspace_size(Q.qsa.QSA_OP_SELECT_TOPK, w.B, w.T, nbk, w.k, w.Hq, w.D)
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+        kp = torch.empty(w.B, nbk, w.Di, dtype=torch.bfloat16, device=dev)
+        idx = torch.empty(w.B, w.T, w.k, dtype=torch.int32, device=dev)
+        out = torch.empty_like(x["q"])
+        lse = torch.empty(w.B, w.T, w.Hq, dtype=torch.float32, device=dev)
+        my_ranges = [(0, w.T)]
 
     def step(ev=None):
-        Q.qsa_pool_block_keys(x["ki"], kp)
-        if ev:
-            ev[0].record(stream)
-        Q.qsa_select_topk(w.k, qi=x["qi"], kp=kp, idx=idx, workspace=ws)
-        if ev:
-            ev[1].record(stream)
-        Q.qsa_sparse_attn_prefill(x["q"], x["k"], x["v"], idx, out=out, lse=lse)
-        if ev:
-            ev[2].record(stream)
+        """One step; with `ev` = [(label, event), ...] the events mark where each part ends."""
+        mark = (lambda i: ev[i][1].record(stream)) if ev else (lambda i: None)
+        if sp is None:
+            Q.qsa_pool_block_keys(x["ki"], kp)
+            mark(0)
+            Q.qsa_select_topk(w.k, qi=x["qi"], kp=kp, idx=idx, workspace=ws)
+            mark(1)
+            Q.qsa_sparse_attn_prefill(x["q"], x["k"], x["v"], idx, out=out, lse=lse)
+            mark(2)
+        else:
+            sp.pool_local(x["ki"])
+            sp.exchange(x["k"], x["v"])
+            mark(0)
+            sp.compute(x["q"], x["qi"], events=[e for _, e in ev[1:]] if ev else None)
 
+    labels = ["pool", "score_topk", "attention"] if sp is None else \
+        ["pool_allgather"] + ["score_topk", "attention"] * len(my_ranges)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
     assert Q.qsa_get_device_status() == 0
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    evs = [[(lab, torch.cuda.Event(enable_timing=True)) for lab in labels] for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     barrier(world)
     torch.cuda.synchronize()
     with Clocks(local) as clk:
         t0.record(stream)
         for s in range(args.steps):
+            starts[s].record(stream)
             step(evs[s])
         t1.record(stream)
         torch.cuda.synchronize()
@@ -362,21 +386,37 @@ def run_qsa(args):
     clocks = clk.summary()
     ms_total = max_over_ranks(t0.elapsed_time(t1), world, dev)
     ms_step = ms_total / args.steps
-    ms_select = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
-    ms_attn = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
-    value = world * w.B * w.T / (ms_step / 1000)
+    parts = {lab: 0.0 for lab in labels}
+    for s in range(args.steps):
+        prev = starts[s]
+        for lab, e in evs[s]:
+            parts[lab] += prev.elapsed_time(e) / args.steps
+            prev = e
+    ms_select = parts["score_topk"]
+    ms_attn = parts["attention"]
+    value = w.B * w.T / (ms_step / 1000)    # the whole job's tokens (every rank's rows)
     work = prefill_work(w)
+    if sp is not None:   # this rank's share of the work
+        from hybrid_sparse_attention_qsa_b200 import shard as SH
+        mine = SH.causal_cost(my_ranges, w.k, w.blk)
+        work = dict(attn_bytes=mine["attended_tokens"] * w.Hkv * w.D * 4 * w.B
+                    + sum(b - a for a, b in my_ranges) * w.Hq * w.D * 4 * w.B,
+                    attn_flops=mine["attended_tokens"] * w.Hq * 4 * w.D * w.B,
+                    index_flops=mine["index_pairs"] * 2 * w.Hi * w.Di * w.B, pairs=mine["index_pairs"] * w.B)
     attn_gbs = work["attn_bytes"] / (ms_attn / 1000) / 1e9
     attn_tflops = work["attn_flops"] / (ms_attn / 1000) / 1e12
     compulsory = unique_kv_bytes(w)
     traffic, traffic_src = profile_traffic(args.workload)
     ceiling = gather_ceiling(dev, stream, w)
-    launches = (1 + select_launches(w, ws_bytes) + 1) * args.steps
+    if sp is None:
+        launches = (1 + select_launches(w, ws_bytes) + 1) * args.steps
+    else:   # per chunk: pooling, the selection's kernels, attention (NCCL's own kernels not counted)
+        launches = sum(2 + select_launches(w.with_(T=b - a), ws_bytes) for a, b in my_ranges) * args.steps
 
     # indexer alone (scores for all rows materialised once; untimed in the step above)
     idx_ms = None
     try:
-        if args.no_indexer:
+        if args.no_indexer or sp is not None:
             raise torch.OutOfMemoryError("skipped")
         scores = torch.empty(w.B, w.T, nbk, dtype=torch.float32, device=dev)
         Q.qsa_index_score(x["qi"], kp, scores=scores)
@@ -395,7 +435,7 @@ def run_qsa(args):
     # dense causal attention on the same q/k/v (library SDPA, GQA), the comparison the vendor's
     # kernel-level speedups are stated against; QSA's step (selection included) over it
     dense = None
-    if not args.no_dense:
+    if not args.no_dense and sp is None:
         try:
             g = w.Hq // w.Hkv   # K/V expanded to every query head so the flash backend takes the call
             qd = x["q"].transpose(1, 2)
@@ -420,7 +460,36 @@ def run_qsa(args):
 
     # end to end through the public API from pinned host buffers
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and sp is not None:
+        # each rank's own rows from pinned host buffers: H2D of its input chunks, the sharded step,
+        # D2H of its output rows
+        hin = {n: [t.cpu().pin_memory() for t in x[n]] for n in x}
+        hout = [torch.empty_like(o, device="cpu").pin_memory() for o in sp.out]
+        h2d = sum(t.numel() * t.element_size() for ts in hin.values() for t in ts)
+        d2h = sum(t.numel() * t.element_size() for t in hout)
+
+        def e2e_step():
+            for n in x:
+                for dst, src in zip(x[n], hin[n]):
+                    dst.copy_(src, non_blocking=True)
+            step()
+            for dst, src in zip(hout, sp.out):
+                dst.copy_(src, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        a0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        a1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(a0.elapsed_time(a1), world, dev) / args.e2e_steps
+        e2e = {"value": w.B * w.T / (e2e_ms / 1000), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "per_rank": True}
+        del hin, hout
+    elif not args.no_e2e:
         host = {n: torch.empty_like(x[n], device="cpu").pin_memory() for n in ("q", "k", "v", "qi", "ki")}
         for n in host:
             host[n].copy_(x[n])
@@ -443,17 +512,26 @@ def run_qsa(args):
         a1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = max_over_ranks(a0.elapsed_time(a1), world, dev) / args.e2e_steps
-        e2e = {"value": world * w.B * w.T / (e2e_ms / 1000), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+        e2e = {"value": w.B * w.T / (e2e_ms / 1000), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
         del host, hout, dbufs
-    del x, ws, idx, out, lse, kp
+    if sp is None:
+        del idx, out, lse, kp
+    del x, ws, sp
     torch.cuda.empty_cache()
 
     # ---------------------------------------------------------------- decode leg
     decode = None
     if not args.no_decode:
-        wd = I.WORKLOADS[args.decode_workload].with_(seed=I.WORKLOADS[args.decode_workload].seed + 1000 * rank)
+        # the decode batch is split across the ranks (no collective): each keeps its sequences
+        wd = I.WORKLOADS[args.decode_workload]
         xd = I.make_decode(wd, dev)
+        if world > 1:
+            from hybrid_sparse_attention_qsa_b200 import shard as SH
+            b0, b1 = SH.batch_range(wd.B, world, rank)
+            xd = {n: t[b0:b1].contiguous() for n, t in xd.items()}
+            wd = wd.with_(B=b1 - b0)
+            torch.cuda.empty_cache()
         nbd = wd.T // wd.blk
         kpd = Q.qsa_pool_block_keys(xd["ki"])
         wsd = torch.empty(Q.qsa_workspace_size(Q.qsa.QSA_OP_SELECT_TOPK, wd.B, 1, nbd, wd.k, wd.Hq, wd.D),
@@ -519,7 +597,8 @@ def run_qsa(args):
         del g_step, g_sel, g_att
         dw = decode_work(wd)
         dgbs = dw["bytes"] / (dms / 1000) / 1e9
-        decode = {"workload": args.decode_workload, "value": world * wd.B / (dms / 1000), "unit": "tokens/s",
+        decode = {"workload": args.decode_workload, "value": I.WORKLOADS[args.decode_workload].B / (dms / 1000),
+                  "unit": "tokens/s",
                   "ms_per_step": dms, "launch": "CUDA graph of one step, replayed",
                   "steps": dsteps, "num_splits": splits,
                   "step_breakdown_ms": {"score_topk": d_sel, "attention_and_merge": d_att},
@@ -555,11 +634,13 @@ def run_qsa(args):
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "strong",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": args.workload, "B": w.B, "T": w.T, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "Hi": w.Hi,
                        "Di": w.Di, "blk": w.blk, "k": w.k, "boost": f"{w.boost_frac:g} of keys x{w.boost:g}",
-                       "l2": "inputs larger than L2, no flush", "parallelism": f"independent replicas x{world}"},
+                       "l2": "inputs larger than L2, no flush",
+                       "parallelism": "single GPU" if world == 1 else
+                       f"zig-zag query-row shards x{world}, one all-gather of K/V/kp per step; decode batch split"},
             # The attention's compulsory work is its tensor-core flops (the unique K/V bytes take a
             # tenth of that time at HBM peak), so the roofline is stated on the tensor basis; the
             # gathered-bytes rate is compared with the measured gather ceiling, not with HBM.
@@ -575,13 +656,14 @@ def run_qsa(args):
                                             "basis": "every K/V row once + q read + o write"},
                          "gathered_bytes_rate": {
                              "bytes_per_launch": work["attn_bytes"], "achieved_gbs": attn_gbs,
-                             "ceiling_gbs": ceiling["l2_bulk_gbs"],
-                             "frac_of_ceiling": attn_gbs / ceiling["l2_bulk_gbs"],
+                             "ceiling_gbs": ceiling["ceiling_gbs"],
+                             "frac_of_ceiling": attn_gbs / ceiling["ceiling_gbs"],
                              "basis": "K/V rows of every selected token as gathered (a block once per query "
-                                      "that selects it) + q read + o write; ceiling = bulk-copy gather of "
-                                      "the same chunks from an L2-resident buffer (measured in this run)"},
+                                      "that selects it) + q read + o write; ceiling = the best bulk-copy "
+                                      "gather of the same chunks from an L2-resident buffer, measured in "
+                                      "this run (gather_probe)"},
                          "gather_probe": ceiling},
-            "step_breakdown_ms": {"pool": None, "score_topk": ms_select, "attention": ms_attn},
+            "step_breakdown_ms": parts,
             "indexer": {
                 "flops": work["index_flops"],
                 "selection": {"ms": ms_select, "tflops": work["index_flops"] / ms_select / 1e9,

@@ -66,7 +66,7 @@ constexpr int kSampleShift = 4;       // every 16th pooled block is sampled ...
 constexpr int kSampleOff = 8;         // ... starting at block 8
 constexpr int kFallbackCtas = 128;    // CTAs (and scratch rows) of the exact redo of failed rows
 constexpr long long kFusedTarget = 4ll << 30;   // workspace the size query plans the filtered path in
-constexpr int kFusedMinRows = 16384;  // automatic choice: rows per sequence from which it pays
+constexpr int kFusedMinRows = 16384;  // automatic choice: row length (last position) from which it pays
 constexpr int kFusedMaxCap = 5120;    // longest candidate list the select kernel holds (k <= 1024)
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -279,7 +279,9 @@ qsa_status_t qsa_select_topk(const float* scores, int64_t ld_scores, const void*
     const bool able = (Hi == 4 || Hi == 8) && fp.cap <= kFusedMaxCap;
     if (path == 2 && !able) return QSA_ERR_UNSUPPORTED;
     if (path == 2 && fit < 1) return QSA_ERR_WORKSPACE_TOO_SMALL;
-    if (path == 2 || (path == 0 && able && Tq >= kFusedMinRows && fit >= std::min(Tq, 4096))) {
+    // automatic: rows long enough (the chunk's last row sees 16384 positions or more), and a
+    // workspace holding 4096 rows or all of them
+    if (path == 2 || (path == 0 && able && q_pos0 + Tq >= kFusedMinRows && fit >= std::min(Tq, 4096))) {
       long long R = std::min<long long>(Tq, fit);
       if (R < Tq && R >= 64) R &= ~63ll;
       uint8_t* w8 = static_cast<uint8_t*>(workspace);

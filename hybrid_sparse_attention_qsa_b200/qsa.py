@@ -341,6 +341,17 @@ def qsa_sparse_attn_decode_noalloc(q: torch.Tensor, kcache: torch.Tensor, vcache
     return out, lse
 
 
+def qsa_decode_default_splits(B: int, k_blocks: int) -> int:
+    """Split count qsa_sparse_attn_decode picks for num_splits == 0 on the current device."""
+    return lib().qsa_decode_default_splits(B, k_blocks)
+
+
+def qsa_decode_split_merge(B: int, Hq: int, Hkv: int, D: int, num_splits: int) -> int:
+    """0: one split; 1: splits merged inside thread-block clusters; 2: through workspace partials and
+    the merge kernel; -1: invalid sizes or no usable device."""
+    return lib().qsa_decode_split_merge(B, Hq, Hkv, D, num_splits)
+
+
 def qsa_get_device_status(device=None) -> int:
     """Synchronise the current stream and read + clear the device status word."""
     return int(lib().qsa_get_device_status(_stream(device)))

@@ -184,8 +184,9 @@ QSA_API qsa_status_t qsa_index_score(const void* qi, const void* kp, const float
  *     workspace is split in two halves and the top-k of one chunk runs on a per-device internal
  *     stream while the next chunk is scored on `stream`; the internal stream is joined back into
  *     `stream` before the call returns, so the call keeps the usual stream-ordered semantics.
- *   - filtered (prefill with Hi of 4 or 8 and k <= 1024, chosen automatically from 16384 rows per
- *     sequence when the workspace holds 4096 rows or all of them): the scores are never stored.  Every 16th
+ *   - filtered (prefill with Hi of 4 or 8 and k <= 1024, chosen automatically when the call's last
+ *     row sits at position 16384 or later, q_pos0 + Tq >= 16384, and the workspace holds 4096 rows
+ *     or all of them): the scores are never stored.  Every 16th
  *     pooled block is scored first; per row, a threshold with about 2.5 k (at least 1024) of the
  *     row's scores expected above it is read off these samples; the tensor-core score kernel then
  *     keeps only the scores at or above the threshold, in block order, and the top-k is selected
