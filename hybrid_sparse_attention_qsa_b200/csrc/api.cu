@@ -61,6 +61,7 @@ bool hi_supported(int Hi) { return Hi == 1 || Hi == 2 || Hi == 4 || Hi == 8; }
 
 // ---- filtered selection (prefill without materialised scores)
 std::atomic<int> g_select_path{0};    // 0 automatic, 1 materialised scores, 2 filtered
+std::atomic<int> g_attn_path{0};      // prefill attention: 0 automatic, 1 row by row, 2 query tiles
 std::atomic<int> g_sample_rank{0};    // 0: the default rank of the threshold among the samples
 constexpr int kSampleShift = 4;       // every 16th pooled block is sampled ...
 constexpr int kSampleOff = 8;         // ... starting at block 8
@@ -420,6 +421,37 @@ qsa_status_t qsa_sparse_attn_prefill(const void* q, const void* k, const void* v
       launch_attn_prefill(di, q, k, v, idx, B, Tq, Tk, Hq, Hkv, D, k_blocks, q_pos0, scale, out, lse, S(stream)));
 }
 
+qsa_status_t qsa_sparse_attn_prefill_ws(const void* q, const void* k, const void* v, const int32_t* idx, int B,
+                                        int Tq, int Tk, int Hq, int Hkv, int D, int k_blocks, int blk,
+                                        int64_t q_pos0, float scale, void* out, float* lse, void* workspace,
+                                        size_t ws_bytes, void* stream) {
+  qsa_status_t st = check_attn_shape(Hq, Hkv, D, blk, k_blocks);
+  if (st != QSA_OK) return st;
+  if (B < 0 || Tq < 0 || Tk < 0 || q_pos0 < 0 || q_pos0 + Tq > Tk) return QSA_ERR_INVALID_ARGUMENT;
+  if (static_cast<long long>(B) * Tq == 0) return QSA_OK;
+  if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(out) || (k_blocks > 0 && idx == nullptr))
+    return QSA_ERR_INVALID_ARGUMENT;
+  if (static_cast<long long>(B) * Tq > 0x7fffffffLL) return QSA_ERR_UNSUPPORTED;
+  const DeviceInfo* di = device_info();
+  if (!di) return QSA_ERR_CUDA;
+  const int path = g_attn_path.load();
+  const bool tiles_ok = attn_tc_supported(Hq, Hkv, D, k_blocks) && path != 1 && workspace != nullptr &&
+                        ok_ptr(workspace) && ws_bytes >= 256 + attn_tc_tile_bytes(k_blocks);
+  if (path == 2 && !tiles_ok)
+    return attn_tc_supported(Hq, Hkv, D, k_blocks) ? QSA_ERR_WORKSPACE_TOO_SMALL : QSA_ERR_UNSUPPORTED;
+  if (!tiles_ok)
+    return cuda_status(
+        launch_attn_prefill(di, q, k, v, idx, B, Tq, Tk, Hq, Hkv, D, k_blocks, q_pos0, scale, out, lse, S(stream)));
+  return cuda_status(launch_attn_prefill_tc(di, q, k, v, idx, B, Tq, Tk, Hq, Hkv, k_blocks, q_pos0, scale, out, lse,
+                                            workspace, ws_bytes, S(stream)));
+}
+
+qsa_status_t qsa_set_attn_options(int path) {
+  if (path < 0 || path > 2) return QSA_ERR_INVALID_ARGUMENT;
+  g_attn_path.store(path);
+  return QSA_OK;
+}
+
 int qsa_decode_default_splits(int B, int k_blocks) {
   const DeviceInfo* di = device_info();
   if (!di || B < 1) return 1;
@@ -473,6 +505,13 @@ size_t qsa_workspace_size(qsa_op_t op, int B, int Tq, int NBk, int k, int Hq, in
       bytes = std::max(bytes, fp.fixed + frows * fp.per_row);
     }
     return static_cast<size_t>(bytes);
+  }
+  if (op == QSA_OP_SPARSE_ATTN_PREFILL) {
+    // the tile unions of up to 4096 tiles of 16 rows (all tiles when fewer)
+    if (B < 0 || Tq < 0 || k < 1) return 0;
+    const long long tiles = static_cast<long long>(B) * ((Tq + 15) / 16);
+    const long long n = std::max(1ll, std::min(tiles, 4096ll));
+    return static_cast<size_t>(256 + ((n * 4 + 255) & ~255ll) + n * static_cast<long long>(attn_tc_tile_bytes(k)));
   }
   if (op == QSA_OP_SPARSE_ATTN_DECODE) {
     if (B < 1 || Hq < 1 || D < 1) return 0;

@@ -83,6 +83,15 @@ cudaError_t launch_topk_fallback(const DeviceInfo* di, const void* qi, const voi
 cudaError_t launch_attn_prefill(const DeviceInfo* di, const void* q, const void* k, const void* v, const int32_t* idx,
                                 int B, int Tq, int Tk, int Hq, int Hkv, int D, int k_blocks, long long q_pos0,
                                 float scale, void* out, float* lse, cudaStream_t s);
+// Query-tile prefill attention on tcgen05 (sparse_attn_tc.cu): D = 128, groups of 8 query heads,
+// k_blocks <= 1024.  The workspace holds the tile unions of as many 16-row tiles as fit (at least
+// one: 256 + attn_tc_tile_bytes(k_blocks) bytes); the call walks the tiles in ranges of that many.
+bool attn_tc_supported(int Hq, int Hkv, int D, int k_blocks);
+size_t attn_tc_tile_bytes(int k_blocks);
+cudaError_t launch_attn_prefill_tc(const DeviceInfo* di, const void* q, const void* k, const void* v,
+                                   const int32_t* idx, int B, int Tq, int Tk, int Hq, int Hkv, int k_blocks,
+                                   long long q_pos0, float scale, void* out, float* lse, void* ws, size_t ws_bytes,
+                                   cudaStream_t s);
 cudaError_t launch_attn_decode(const DeviceInfo* di, const void* q, const void* kc, const void* vc,
                                const int32_t* seqlens, const int32_t* idx, int B, int Lmax, int Hq, int Hkv, int D,
                                int k_blocks, float scale, int num_splits, void* out, float* lse, float* part,

@@ -1,0 +1,649 @@
+// Query-tile sparse attention on the 5th-generation tensor cores (prefill; D = 128, GQA groups of 8).
+//
+// "Qwen3.8-Flash-Next architecture" (flozi.net), "Der Weg eines Tokens durch das Modell", item 2:
+// after the selection, exact attention runs over only the selected tokens of each query (its top-k
+// micro-blocks plus its own block), with 16 query heads over 2 KV heads.
+//
+// Consecutive queries select overlapping block sets, so a tile of 16 consecutive query rows is
+// processed together: the tile attends over the UNION of its rows' blocks, each union block is
+// gathered once per tile instead of once per row, and every row masks out the union blocks it did
+// not select.  16 rows x the 8 query heads of one KV head are the 128 rows (M) of one tcgen05 MMA.
+// On the 128K workload the union of 16 rows is about 0.37 of the sum of their lists, so the gather
+// (the cost of the row-by-row kernel) shrinks ~2.7x while the contraction grows to about 6x the
+// selected pairs -- cheap on tcgen05.  The result is the same exact attention: a masked entry
+// contributes exp(-inf) = 0, and the softmax runs in fp32 over exactly the selected tokens.
+//
+// tile_union_kernel (one CTA per tile): keys (block << 4 | row) of the 16 index lists are sorted
+// (bitonic; ascending lists enter as sorted runs so only the merge stages run), the tile's own
+// blocks (one per row, always attended) are merged in, and equal blocks are folded into one entry
+// (block, 16-bit mask of the rows that attend it), ascending by block.  Entries outside a row's
+// causal range are skipped and recorded in the device status (-1 and the own block are skipped
+// silently).
+//
+// sparse_attn_tc_kernel (persistent, one CTA per SM), per (tile, KV head):
+//   warp 0   producer: the Q tile (two 128-byte-swizzled TMA boxes of [16 rows][8 heads][64 d]),
+//            then per chunk of 32 union entries one TMA box of [4 tokens][64 d] per block, half and
+//            tensor (K and V) into a 2-stage ring; the chunk's block ids and per-row member words
+//            go to shared memory;
+//   warp 1   TMEM owner and MMA issuer (one thread): S = Q K^T (M 128, N 128 tokens, K 128) into
+//            one of three S buffers, then O += P V with P read from TMEM (A operand) and V as an
+//            MN-major B operand;
+//   warps 2-5 softmax (one thread per row): mask, fp32 online softmax in exp2 form with a lazy
+//            rescale of O (only when the running max grows by more than 2^8), P packed to bf16
+//            into the S buffer's columns, and the epilogue (O / l -> bf16 rows, log-sum-exp).
+// TMEM: S0 S1 S2 at columns 0, 128, 256, O at 384 (fp32, lane = row).  Every wait is bounded; a
+// role whose wait runs out stops, and every role reaches the final barrier and TMEM release.
+#include <algorithm>
+#include <mutex>
+
+#include "launch.h"
+
+namespace qsa {
+namespace {
+
+constexpr int kTQ = 16;          // query rows per tile
+constexpr int kGrp = 8;          // query heads per KV head (the M of a tile is kTQ * kGrp = 128)
+constexpr int kD = 128;
+constexpr int kCB = 32;          // union blocks per chunk
+constexpr int kCT = kCB * 4;     // tokens per chunk (the N of S)
+constexpr int kHalf = 128 * 128; // bytes of one 64-column half of a 128-row operand (16 KB)
+constexpr int kQBytes = 2 * kHalf;
+constexpr int kKVBytes = 2 * kHalf;   // K (or V) of one chunk
+constexpr int kStages = 2;
+constexpr int kSoftWarps = 4;
+constexpr int kThreads = (2 + kSoftWarps) * 32;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleLog2 = 8.0f;  // O is rescaled only when the row max grows by more than this
+
+struct ChunkInfo {
+  int blocks[kCB];
+  uint32_t words[kTQ];   // bit j: the row attends union slot j of the chunk
+};
+
+constexpr int kInfoOff = kQBytes + kStages * 2 * kKVBytes;
+constexpr int kBarOff = kInfoOff + kStages * static_cast<int>(sizeof(ChunkInfo));
+constexpr int kSmem = 1024 + kBarOff + 256;
+
+struct TcArgs {
+  const uint2* ent;      // [tiles][cap] (block, row mask) per tile of this launch
+  const int* cnt;        // [tiles]
+  uint16_t* out;
+  float* lse;
+  long long q_pos0;
+  int B, Tq, Hq, Hkv, cap, tile0, ntiles, tpb;
+  float scale_log2;
+  KernelCtl ctl;
+};
+
+__device__ __forceinline__ int tile_chunks(int nu) { return max(1, (nu + kCB - 1) / kCB); }
+
+// ---------------------------------------------------------------------------- tile unions
+__global__ void __launch_bounds__(512) tile_union_kernel(const int32_t* __restrict__ idx, int Tq, int kb,
+                                                         long long q_pos0, int tile0, int tpb, int n2,
+                                                         uint2* __restrict__ ent, int* __restrict__ cnt, int cap,
+                                                         KernelCtl ctl) {
+  extern __shared__ uint32_t ukeys[];
+  uint32_t* keys = ukeys;                 // [n2]
+  uint32_t* merged = keys + n2;           // [16 * kb + 16]
+  __shared__ int s_flags[2];
+  __shared__ int s_scan[17];
+  const int tid = threadIdx.x;
+  const int tl = blockIdx.x;
+  const int tile = tile0 + tl;
+  const int b = tile / tpb, t0 = (tile % tpb) * kTQ;
+  const int nlist = kTQ * kb;
+  const bool pow2 = (kb & (kb - 1)) == 0;
+  if (tid < 2) s_flags[tid] = 0;
+  __syncthreads();
+  bool bad = false, unsorted = false;
+  for (int e = tid; e < n2; e += blockDim.x) {
+    uint32_t key = 0xFFFFFFFFu;
+    if (e < nlist) {
+      const int r = e / kb;
+      int j = e - r * kb;
+      // with power-of-two lists the odd lists enter reversed, so the runs alternate direction
+      if (pow2 && (r & 1)) j = kb - 1 - j;
+      const int row = t0 + r;
+      if (row < Tq) {
+        const long long rowg = static_cast<long long>(b) * Tq + row;
+        const int x = idx[rowg * kb + j];
+        const long long own = (q_pos0 + row) >> 2;
+        if (x >= 0 && x < own) {
+          key = (static_cast<uint32_t>(x) << 4) | static_cast<uint32_t>(r);
+        } else if (x != -1 && x != own) {
+          bad = true;
+        }
+        // the source list must be ascending with skipped entries last: check the pair (j, j + 1)
+        if (j + 1 < kb) {
+          const int xn = idx[rowg * kb + j + 1];
+          const bool vn = xn >= 0 && xn < own;
+          const uint32_t kn = vn ? ((static_cast<uint32_t>(xn) << 4) | static_cast<uint32_t>(r)) : 0xFFFFFFFFu;
+          if (kn < key) unsorted = true;
+        }
+      }
+    }
+    keys[e] = key;
+  }
+  if (bad) s_flags[0] = 1;
+  if (unsorted) s_flags[1] = 1;
+  __syncthreads();
+  if (tid == 0 && s_flags[0]) record_status(ctl, kStBadArg);
+  // bitonic sort of keys[0 .. n2) ascending; sorted runs of kb (alternating) skip the first stages
+  const int kstart = (pow2 && !s_flags[1] && kb >= 2) ? 2 * kb : 2;
+  for (int k2 = kstart; k2 <= n2; k2 <<= 1) {
+    for (int j2 = k2 >> 1; j2 > 0; j2 >>= 1) {
+      for (int i = tid; i < n2; i += blockDim.x) {
+        const int p = i ^ j2;
+        if (p > i) {
+          const uint32_t a = keys[i], c = keys[p];
+          const bool asc = (i & k2) == 0;
+          if ((a > c) == asc) {
+            keys[i] = c;
+            keys[p] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  // valid keys: those below 0xFFFFFFFF (a prefix of the sorted array)
+  int lo = 0, hi = n2;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (keys[mid] == 0xFFFFFFFFu) hi = mid; else lo = mid + 1;
+  }
+  const int nv = lo;
+  // the own block of every row of the tile, keys ascending in the row
+  const int nown = min(kTQ, Tq - t0);
+  uint32_t okey[kTQ];
+#pragma unroll
+  for (int r = 0; r < kTQ; ++r)
+    okey[r] = r < nown ? (static_cast<uint32_t>((q_pos0 + t0 + r) >> 2) << 4) | static_cast<uint32_t>(r) : 0xFFFFFFFFu;
+  for (int i = tid; i < nv; i += blockDim.x) {
+    const uint32_t key = keys[i];
+    int c = 0;
+#pragma unroll
+    for (int r = 0; r < kTQ; ++r) c += okey[r] < key ? 1 : 0;
+    merged[i + c] = key;
+  }
+  if (tid < nown) {
+    const uint32_t key = okey[tid];
+    int a = 0, z = nv;
+    while (a < z) {
+      const int mid = (a + z) >> 1;
+      if (keys[mid] < key) a = mid + 1; else z = mid;
+    }
+    merged[tid + a] = key;
+  }
+  __syncthreads();
+  // fold equal blocks: one entry per run, the rows of the run OR-ed into its mask
+  const int N = nv + nown;
+  const int per = (N + blockDim.x - 1) / blockDim.x;
+  const int i0 = min(N, tid * per), i1 = min(N, i0 + per);
+  int heads = 0;
+  for (int i = i0; i < i1; ++i)
+    if (i == 0 || (merged[i] >> 4) != (merged[i - 1] >> 4)) ++heads;
+  // block-wide exclusive scan of the head counts
+  const int lane = tid & 31, w = tid >> 5;
+  int incl = heads;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) s_scan[w] = incl;
+  __syncthreads();
+  if (tid == 0) {
+    int run = 0;
+    for (int q = 0; q < static_cast<int>(blockDim.x >> 5); ++q) {
+      const int v = s_scan[q];
+      s_scan[q] = run;
+      run += v;
+    }
+    s_scan[16] = run;
+  }
+  __syncthreads();
+  int u = s_scan[w] + incl - heads;
+  uint2* te = ent + static_cast<long long>(tl) * cap;
+  for (int i = i0; i < i1; ++i) {
+    const uint32_t blk = merged[i] >> 4;
+    if (i == 0 || blk != (merged[i - 1] >> 4)) {
+      uint32_t mask = 0;
+      for (int j = i; j < N && (merged[j] >> 4) == blk; ++j) mask |= 1u << (merged[j] & 15u);
+      te[u++] = make_uint2(blk, mask);
+    }
+  }
+  if (tid == 0) cnt[tl] = s_scan[16];
+}
+
+// ---------------------------------------------------------------------------- attention
+struct Bars {
+  uint64_t kv_full[kStages], kv_empty[kStages];
+  uint64_t s_full[3], p_full[3], s_free[3];
+  uint64_t q_full, q_empty, pv_done, o_free;
+  uint32_t tmem;
+};
+
+template <int HKV>
+__global__ void __launch_bounds__(kThreads, 1)
+    sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
+                          const __grid_constant__ CUtensorMap vmap, TcArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* qs = smem;                                   // [2 halves][128 rows][128 B]
+  uint8_t* kvs = smem + kQBytes;                        // per stage: K [2][128 tokens][128 B], V likewise
+  ChunkInfo* info = reinterpret_cast<ChunkInfo*>(smem + kInfoOff);
+  Bars* bar = reinterpret_cast<Bars*>(smem + kBarOff);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&bar->kv_full[s], 1);
+      mbar_init(&bar->kv_empty[s], 1);
+    }
+    for (int i = 0; i < 3; ++i) {
+      mbar_init(&bar->s_full[i], 1);
+      mbar_init(&bar->p_full[i], kSoftWarps);
+      mbar_init(&bar->s_free[i], 1);
+    }
+    mbar_init(&bar->q_full, 1);
+    mbar_init(&bar->q_empty, 1);
+    mbar_init(&bar->pv_done, 1);
+    mbar_init(&bar->o_free, kSoftWarps);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bar->tmem, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bar->tmem;
+  const int ntl = a.ntiles;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ producer
+    prefetch_tensormap(&qmap);
+    prefetch_tensormap(&kmap);
+    prefetch_tensormap(&vmap);
+    int n = 0, hp = 0;
+    bool alive = true;
+    for (int it = blockIdx.x; alive && it < ntl; it += gridDim.x) {
+      const int tl = ntl - 1 - it;
+      const int tile = a.tile0 + tl;
+      const int b = tile / a.tpb, t0 = (tile % a.tpb) * kTQ;
+      const int nu = a.cnt[tl];
+      const int nch = tile_chunks(nu);
+      const uint2* te = a.ent + static_cast<long long>(tl) * a.cap;
+      for (int g = 0; alive && g < HKV; ++g, ++hp) {
+        bool ok = true;
+        if (lane == 0) {
+          ok = mbar_wait(&bar->q_empty, (hp & 1) ^ 1u, a.ctl);
+          if (ok) {
+            mbar_arrive_expect_tx(&bar->q_full, kQBytes);
+            tma_load_4d(qs, &qmap, &bar->q_full, 0, g * kGrp, t0, b);
+            tma_load_4d(qs + kHalf, &qmap, &bar->q_full, 64, g * kGrp, t0, b);
+          }
+        }
+        alive = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        for (int c = 0; alive && c < nch; ++c, ++n) {
+          const int s = n & 1;
+          const unsigned f = static_cast<unsigned>(n >> 1);
+          ok = true;
+          if (lane == 0) ok = mbar_wait(&bar->kv_empty[s], (f & 1u) ^ 1u, a.ctl);
+          alive = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+          if (!alive) break;
+          const int u = c * kCB + lane;
+          const uint2 e = nu > 0 ? te[min(u, nu - 1)] : make_uint2(0u, 0u);   // past the end: a repeat, masked
+          const uint32_t mask = u < nu ? e.y : 0u;
+          uint32_t myw = 0;
+#pragma unroll
+          for (int q = 0; q < kTQ; ++q) {
+            const uint32_t bq = __ballot_sync(0xffffffffu, (mask >> q) & 1u);
+            if (lane == q) myw = bq;
+          }
+          info[s].blocks[lane] = static_cast<int>(e.x);
+          if (lane < kTQ) info[s].words[lane] = myw;
+          __syncwarp();
+          if (lane == 0) mbar_arrive_expect_tx(&bar->kv_full[s], 2 * kKVBytes);
+          __syncwarp();
+          uint8_t* ks = kvs + s * 2 * kKVBytes;
+          uint8_t* vs = ks + kKVBytes;
+          const int tok = static_cast<int>(e.x) * 4;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            tma_load_4d(ks + h * kHalf + lane * 512, &kmap, &bar->kv_full[s], h * 64, g, tok, b);
+            tma_load_4d(vs + h * kHalf + lane * 512, &vmap, &bar->kv_full[s], h * 64, g, tok, b);
+          }
+        }
+      }
+    }
+    // never leave with a copy in flight: the last fill of each stage and the last Q tile
+    if (lane == 0) {
+      for (int s = 0; s < kStages && s < n; ++s) {
+        const int last = s + ((n - 1 - s) / kStages) * kStages;
+        mbar_wait(&bar->kv_full[s], static_cast<unsigned>(last >> 1) & 1u, a.ctl);
+      }
+      if (hp > 0) mbar_wait(&bar->q_full, static_cast<unsigned>(hp - 1) & 1u, a.ctl);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_s = umma_idesc_bf16_f32(128, kCT);
+      const uint32_t idesc_pv = umma_idesc_bf16_f32_bmn(128, kD);
+      const uint32_t o_col = tmem + 384;
+      int n = 0, hp = 0;
+      bool alive = true;
+      auto issue_pv = [&](int m, bool first) -> bool {
+        const int sb = m % 3, s = m & 1;
+        if (!mbar_wait(&bar->p_full[sb], static_cast<unsigned>(m / 3) & 1u, a.ctl)) return false;
+        if (first && hp > 0 && !mbar_wait(&bar->o_free, static_cast<unsigned>(hp - 1) & 1u, a.ctl)) return false;
+        tc_fence_after();
+        const uint32_t vbase = smem_u32(kvs + s * 2 * kKVBytes + kKVBytes);
+#pragma unroll
+        for (int kk = 0; kk < kCT / 16; ++kk) {
+          const uint64_t bd = sw128_mnmajor_desc(vbase + kk * 2048, kHalf, 1024);
+          umma_bf16_ta(o_col, tmem + sb * 128 + kk * 8, bd, idesc_pv, (first && kk == 0) ? 0u : 1u);
+        }
+        umma_commit(&bar->kv_empty[s]);
+        umma_commit(&bar->s_free[sb]);
+        umma_commit(&bar->pv_done);
+        return true;
+      };
+      for (int it = blockIdx.x; alive && it < ntl; it += gridDim.x) {
+        const int tl = ntl - 1 - it;
+        const int nch = tile_chunks(a.cnt[tl]);
+        for (int g = 0; alive && g < HKV; ++g, ++hp) {
+          if (!mbar_wait(&bar->q_full, static_cast<unsigned>(hp) & 1u, a.ctl)) {
+            alive = false;
+            break;
+          }
+          const uint32_t qbase = smem_u32(qs);
+          for (int c = 0; c < nch; ++c, ++n) {
+            const int s = n & 1, sb = n % 3;
+            if (!mbar_wait(&bar->kv_full[s], static_cast<unsigned>(n >> 1) & 1u, a.ctl) ||
+                !mbar_wait(&bar->s_free[sb], (static_cast<unsigned>(n / 3) & 1u) ^ 1u, a.ctl)) {
+              alive = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t kbase = smem_u32(kvs + s * 2 * kKVBytes);
+#pragma unroll
+            for (int kk = 0; kk < kD / 16; ++kk) {
+              const int h = kk >> 2;
+              const uint64_t ad = sw128_kmajor_desc(qbase + h * kHalf) + 2 * (kk & 3);
+              const uint64_t bd = sw128_kmajor_desc(kbase + h * kHalf) + 2 * (kk & 3);
+              umma_bf16(tmem + sb * 128, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+            }
+            umma_commit(&bar->s_full[sb]);
+            if (c == nch - 1) umma_commit(&bar->q_empty);
+            if (c > 0 && !issue_pv(n - 1, c == 1)) {
+              alive = false;
+              break;
+            }
+          }
+          if (alive && !issue_pv(n - 1, nch == 1)) alive = false;
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------------ softmax + epilogue
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const int t = row >> 3, hh = row & 7;
+    const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t o_addr = tmem + lane_addr + 384;
+    int n = 0, hp = 0;
+    bool alive = true;
+    for (int it = blockIdx.x; alive && it < ntl; it += gridDim.x) {
+      const int tl = ntl - 1 - it;
+      const int tile = a.tile0 + tl;
+      const int b = tile / a.tpb, t0 = (tile % a.tpb) * kTQ;
+      const int nch = tile_chunks(a.cnt[tl]);
+      const bool vrow = t0 + t < a.Tq;
+      const long long pos = a.q_pos0 + t0 + t;
+      const int own = static_cast<int>(pos >> 2);
+      const int lim = static_cast<int>(pos & 3);
+      for (int g = 0; alive && g < HKV; ++g, ++hp) {
+        float m_ref = -INFINITY, l = 0.f;
+        for (int c = 0; c < nch; ++c, ++n) {
+          const int s = n & 1, sb = n % 3;
+          if (!mbar_wait(&bar->s_full[sb], static_cast<unsigned>(n / 3) & 1u, a.ctl) ||
+              !mbar_wait(&bar->kv_full[s], static_cast<unsigned>(n >> 1) & 1u, a.ctl)) {
+            alive = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t word = vrow ? info[s].words[t] : 0u;
+          const uint32_t s_addr = tmem + lane_addr + sb * 128;
+          float x[kCT];
+#pragma unroll
+          for (int p4 = 0; p4 < 4; ++p4) {
+            uint32_t r[32];
+            tmem_ld_32x32(s_addr + p4 * 32, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) x[p4 * 32 + i] = __uint_as_float(r[i]);
+          }
+          float mx = -INFINITY;
+#pragma unroll
+          for (int j = 0; j < kCB; ++j) {
+            const bool mem = (word >> j) & 1u;
+            const int tl_lim = info[s].blocks[j] == own ? lim : 3;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const bool ok = mem && i <= tl_lim;
+              const float v = ok ? x[4 * j + i] * a.scale_log2 : -INFINITY;
+              x[4 * j + i] = v;
+              mx = fmaxf(mx, v);
+            }
+          }
+          bool resc = false;
+          float factor = 1.f;
+          if (mx > m_ref + kRescaleLog2) {
+            if (c > 0) {
+              factor = exp2f(m_ref - mx);
+              l *= factor;
+              resc = true;
+            }
+            m_ref = mx;
+          }
+          if (__any_sync(0xffffffffu, resc)) {
+            // O holds PV of chunks 0 .. c-1 once the last of them is complete
+            if (!mbar_wait(&bar->pv_done, static_cast<unsigned>(n - 1) & 1u, a.ctl)) {
+              alive = false;
+              break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int p4 = 0; p4 < 4; ++p4) {
+              uint32_t r[32];
+              tmem_ld_32x32(o_addr + p4 * 32, r);
+              tmem_ld_wait();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * factor);
+              tmem_st_32x32(o_addr + p4 * 32, r);
+            }
+            tmem_st_wait();
+          }
+          const float ref = m_ref == -INFINITY ? 0.f : m_ref;
+          float sum = 0.f;
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            uint32_t pk[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float p0 = exp2f(x[h2 * 64 + 2 * i] - ref);
+              const float p1 = exp2f(x[h2 * 64 + 2 * i + 1] - ref);
+              sum += p0 + p1;
+              pk[i] = pack_bf16x2(p0, p1);
+            }
+            tmem_st_32x32(s_addr + h2 * 32, pk);
+          }
+          l += sum;
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar->p_full[sb]);
+        }
+        if (!alive) break;
+        // ---- epilogue of (tile, head): O / l -> bf16 row, log-sum-exp
+        if (!mbar_wait(&bar->pv_done, static_cast<unsigned>(n - 1) & 1u, a.ctl)) {
+          alive = false;
+          break;
+        }
+        tc_fence_after();
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        const long long orow = (static_cast<long long>(b) * a.Tq + t0 + t) * a.Hq + g * kGrp + hh;
+        uint4* op = reinterpret_cast<uint4*>(a.out + orow * kD);
+#pragma unroll
+        for (int p4 = 0; p4 < 4; ++p4) {
+          uint32_t r[32];
+          tmem_ld_32x32(o_addr + p4 * 32, r);
+          tmem_ld_wait();
+          if (vrow) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              uint4 v;
+              v.x = pack_bf16x2(__uint_as_float(r[8 * i + 0]) * inv, __uint_as_float(r[8 * i + 1]) * inv);
+              v.y = pack_bf16x2(__uint_as_float(r[8 * i + 2]) * inv, __uint_as_float(r[8 * i + 3]) * inv);
+              v.z = pack_bf16x2(__uint_as_float(r[8 * i + 4]) * inv, __uint_as_float(r[8 * i + 5]) * inv);
+              v.w = pack_bf16x2(__uint_as_float(r[8 * i + 6]) * inv, __uint_as_float(r[8 * i + 7]) * inv);
+              op[p4 * 4 + i] = v;
+            }
+          }
+        }
+        if (vrow && a.lse) a.lse[orow] = l > 0.f ? (m_ref + __log2f(l)) * kLn2 : -INFINITY;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar->o_free);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------- host side
+using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                              const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                              CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeFn encode_fn() {
+  static EncodeFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeFn>(p);
+  });
+  return fn;
+}
+
+// 4-D bf16 map over [d3][d2][d1][128] (innermost 128 elements = one head's row of D) with a
+// 128-byte-swizzled box of {64, box1, box2, 1}.  The batch stride spans d2_stride rows of d2 (the
+// map may cover only the first d2 of them).
+bool make_map4(CUtensorMap* m, const void* base, unsigned long long d1, unsigned long long d2,
+               unsigned long long d3, unsigned box1, unsigned box2, unsigned long long d2_stride = 0) {
+  EncodeFn fn = encode_fn();
+  if (!fn) return false;
+  if (d2_stride == 0) d2_stride = d2;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(kD), d1, d2, d3};
+  cuuint64_t strides[3] = {kD * 2ull, d1 * kD * 2ull, d2_stride * d1 * kD * 2ull};
+  cuuint32_t box[4] = {64, box1, box2, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int next_pow2(int x) {
+  int p = 1;
+  while (p < x) p <<= 1;
+  return p;
+}
+
+}  // namespace
+
+bool attn_tc_supported(int Hq, int Hkv, int D, int k_blocks) {
+  return D == kD && (Hkv == 1 || Hkv == 2) && Hq == kGrp * Hkv && k_blocks >= 1 && k_blocks <= 1024;
+}
+
+size_t attn_tc_tile_bytes(int k_blocks) {
+  return static_cast<size_t>(kTQ * k_blocks + kTQ) * sizeof(uint2) + sizeof(int);
+}
+
+cudaError_t launch_attn_prefill_tc(const DeviceInfo* di, const void* q, const void* k, const void* v,
+                                   const int32_t* idx, int B, int Tq, int Tk, int Hq, int Hkv, int k_blocks,
+                                   long long q_pos0, float scale, void* out, float* lse, void* ws, size_t ws_bytes,
+                                   cudaStream_t s) {
+  const int tpb = (Tq + kTQ - 1) / kTQ;
+  const long long ntiles = static_cast<long long>(B) * tpb;
+  const int cap = kTQ * k_blocks + kTQ;
+  const size_t per_tile = attn_tc_tile_bytes(k_blocks);
+  const long long fit = static_cast<long long>((ws_bytes > 256 ? ws_bytes - 256 : 0) / per_tile);
+  if (fit < 1 || ntiles > 0x7fffffffLL) return cudaErrorInvalidValue;
+  const int R = static_cast<int>(std::min<long long>(ntiles, fit));
+  // layout: cnt[R] (256-byte aligned), then ent[R][cap]
+  int* cnt = static_cast<int*>(ws);
+  uint2* ent = reinterpret_cast<uint2*>(static_cast<uint8_t*>(ws) + ((static_cast<size_t>(R) * 4 + 255) & ~size_t(255)));
+  // K and V are mapped only up to the call's last query position: a tile's last own block can
+  // reach past it, and those rows then read as zeros (masked for every row; a zero times a zero
+  // probability keeps the product finite whatever the buffer holds there).
+  CUtensorMap qm, km, vm;
+  const unsigned long long tk_used = static_cast<unsigned long long>(q_pos0 + Tq);
+  if (!make_map4(&qm, q, Hq, Tq, B, kGrp, kTQ) || !make_map4(&km, k, Hkv, tk_used, B, 1, 4, static_cast<unsigned long long>(Tk)) ||
+      !make_map4(&vm, v, Hkv, tk_used, B, 1, 4, static_cast<unsigned long long>(Tk)))
+    return cudaErrorInvalidValue;
+  const int n2 = next_pow2(std::max(kTQ * k_blocks, 32));
+  const size_t usmem = static_cast<size_t>(n2) * 4 + static_cast<size_t>(cap) * 4;
+  static std::once_flag once[64];
+  std::call_once(once[di->device & 63], [] {
+    cudaFuncSetAttribute(tile_union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024);
+    cudaFuncSetAttribute(sparse_attn_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    cudaFuncSetAttribute(sparse_attn_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+  });
+  if (usmem > 160 * 1024) return cudaErrorInvalidValue;
+  TcArgs ta{};
+  ta.ent = ent;
+  ta.cnt = cnt;
+  ta.out = static_cast<uint16_t*>(out);
+  ta.lse = lse;
+  ta.q_pos0 = q_pos0;
+  ta.B = B;
+  ta.Tq = Tq;
+  ta.Hq = Hq;
+  ta.Hkv = Hkv;
+  ta.cap = cap;
+  ta.tpb = tpb;
+  ta.scale_log2 = scale * 1.4426950408889634f;
+  ta.ctl = kernel_ctl(di);
+  for (long long t0 = 0; t0 < ntiles; t0 += R) {
+    const int nt = static_cast<int>(std::min<long long>(R, ntiles - t0));
+    tile_union_kernel<<<nt, 512, usmem, s>>>(idx, Tq, k_blocks, q_pos0, static_cast<int>(t0), tpb, n2, ent, cnt, cap,
+                                             ta.ctl);
+    cudaError_t e = cudaPeekAtLastError();
+    if (e != cudaSuccess) return e;
+    ta.tile0 = static_cast<int>(t0);
+    ta.ntiles = nt;
+    const int grid = std::min(nt, di->num_sms);
+    if (Hkv == 1)
+      sparse_attn_tc_kernel<1><<<grid, kThreads, kSmem, s>>>(qm, km, vm, ta);
+    else
+      sparse_attn_tc_kernel<2><<<grid, kThreads, kSmem, s>>>(qm, km, vm, ta);
+    e = cudaPeekAtLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace qsa

@@ -27,6 +27,11 @@ QSA_SCORE_LINEAR = 1
 
 QSA_OP_SELECT_TOPK = 1
 QSA_OP_SPARSE_ATTN_DECODE = 2
+QSA_OP_SPARSE_ATTN_PREFILL = 3
+
+QSA_ATTN_AUTO = 0
+QSA_ATTN_ROWS = 1
+QSA_ATTN_TILES = 2
 
 # name -> (restype, argtypes), in the order of include/qsa.h
 _P, _I, _I64, _F, _SZ, _U64 = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t,
@@ -42,6 +47,9 @@ SIGNATURES = {
     "qsa_select_topk": (_I, [_P, _I64, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I64, _I, _I, _P, _P, _SZ, _P]),
     "qsa_decode_select": (_I, [_P, _P, _P, _I64, _P, _P, _I, _I, _I, _I, _I, _I, _P, _I, _P, _P, _SZ, _P]),
     "qsa_sparse_attn_prefill": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I64, _F, _P, _P, _P]),
+    "qsa_sparse_attn_prefill_ws": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I64, _F, _P, _P, _P, _SZ,
+                                        _P]),
+    "qsa_set_attn_options": (_I, [_I]),
     "qsa_sparse_attn_decode": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P, _P, _P, _SZ, _P]),
     "qsa_sparse_attn_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P, _P, _P]),
     "qsa_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I, _I]),
@@ -273,8 +281,13 @@ def qsa_decode_select(k: int, *, qi: torch.Tensor, kp: torch.Tensor, ki: torch.T
 
 def qsa_sparse_attn_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, idx: torch.Tensor, *, q_pos0: int = 0,
                             scale: float | None = None, out: torch.Tensor | None = None,
-                            lse: torch.Tensor | None = None, want_lse: bool = True, blk: int = 4):
-    """q [B, Tq, Hq, D], k/v [B, Tk, Hkv, D], idx [B, Tq, kb] -> (out [B, Tq, Hq, D], lse [B, Tq, Hq])."""
+                            lse: torch.Tensor | None = None, want_lse: bool = True, blk: int = 4,
+                            workspace: torch.Tensor | None = None, tiles: bool = True):
+    """q [B, Tq, Hq, D], k/v [B, Tk, Hkv, D], idx [B, Tq, kb] -> (out [B, Tq, Hq, D], lse [B, Tq, Hq]).
+
+    With ``tiles`` (default) the call goes through qsa_sparse_attn_prefill_ws with ``workspace``
+    (allocated here when omitted): query tiles on tcgen05 where the shape allows, else row by row.
+    ``tiles=False`` calls qsa_sparse_attn_prefill (row by row, no workspace)."""
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _need(t, torch.bfloat16, n)
     _need(idx, torch.int32, "idx")
@@ -286,9 +299,25 @@ def qsa_sparse_attn_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, i
         out = torch.empty_like(q)
     if lse is None and want_lse:
         lse = torch.empty(B, Tq, Hq, dtype=torch.float32, device=q.device)
-    _check(lib().qsa_sparse_attn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(idx), B, Tq, Tk, Hq, Hkv, D, kb, blk, q_pos0,
-                                         scale, _ptr(out), _ptr(lse), _stream(q.device)), "qsa_sparse_attn_prefill")
+    if not tiles:
+        _check(lib().qsa_sparse_attn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(idx), B, Tq, Tk, Hq, Hkv, D, kb, blk,
+                                             q_pos0, scale, _ptr(out), _ptr(lse), _stream(q.device)),
+               "qsa_sparse_attn_prefill")
+        return out, lse
+    if workspace is None:
+        nbytes = qsa_workspace_size(QSA_OP_SPARSE_ATTN_PREFILL, B, Tq, 0, kb, Hq, D)
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib().qsa_sparse_attn_prefill_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(idx), B, Tq, Tk, Hq, Hkv, D, kb, blk,
+                                            q_pos0, scale, _ptr(out), _ptr(lse), _ptr(workspace), ws_bytes,
+                                            _stream(q.device)), "qsa_sparse_attn_prefill_ws")
     return out, lse
+
+
+def qsa_set_attn_options(path: int = QSA_ATTN_AUTO) -> None:
+    """Prefill attention of qsa_sparse_attn_prefill_ws for later calls: QSA_ATTN_AUTO (query tiles
+    where supported), QSA_ATTN_ROWS or QSA_ATTN_TILES."""
+    _check(lib().qsa_set_attn_options(path), "qsa_set_attn_options")
 
 
 def qsa_sparse_attn_decode(q: torch.Tensor, kcache: torch.Tensor, vcache: torch.Tensor, seqlens: torch.Tensor,
@@ -508,6 +537,10 @@ def prefill_host(q, k, v, qi, ki, *, topk: int, device="cuda", out=None, q_pos0:
         nbk = max(1, (q_pos0 + shi - 1) // 4)
         qsa_select_topk(topk, qi=qr, kp=kp[:, :nbk], head_w=head_w, q_pos0=q_pos0 + slo, mode=mode,
                         workspace=workspace, idx=idx[:, slo:shi])
+    if "attn_ws" not in bufs:
+        rows = max(bounds[c + 1] - bounds[c] for c in range(n))
+        bufs["attn_ws"] = torch.empty(max(16, qsa_workspace_size(QSA_OP_SPARSE_ATTN_PREFILL, B, rows, 0, topk, Hq, D)),
+                                      dtype=torch.uint8, device=dev)
     for c in range(n):
         lo, hi = bounds[c], bounds[c + 1]
         if hi <= lo:
@@ -515,7 +548,7 @@ def prefill_host(q, k, v, qi, ki, *, topk: int, device="cuda", out=None, q_pos0:
         main.wait_event(arrived[c])
         opart = bufs["out"][:, lo:hi]
         qsa_sparse_attn_prefill(bufs["q"][:, lo:hi], bufs["k"], bufs["v"], idx[:, lo:hi], q_pos0=q_pos0 + lo,
-                                scale=scale, out=opart, lse=bufs["lse"][:, lo:hi])
+                                scale=scale, out=opart, lse=bufs["lse"][:, lo:hi], workspace=bufs["attn_ws"])
         cout.wait_stream(main)
         with torch.cuda.stream(cout):
             out[:, lo:hi].copy_(opart, non_blocking=True)

@@ -75,7 +75,8 @@ typedef enum {
 
 typedef enum {
   QSA_OP_SELECT_TOPK = 1,       /* qsa_select_topk with scores == NULL */
-  QSA_OP_SPARSE_ATTN_DECODE = 2 /* qsa_sparse_attn_decode with num_splits > 1 */
+  QSA_OP_SPARSE_ATTN_DECODE = 2, /* qsa_sparse_attn_decode with num_splits > 1 */
+  QSA_OP_SPARSE_ATTN_PREFILL = 3 /* qsa_sparse_attn_prefill_ws (query tiles) */
 } qsa_op_t;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -244,6 +245,38 @@ QSA_API qsa_status_t qsa_sparse_attn_prefill(const void* q, const void* k, const
                                      const int32_t* idx, int B, int Tq, int Tk, int Hq, int Hkv,
                                      int D, int k_blocks, int blk, int64_t q_pos0, float scale,
                                      void* out, float* lse, void* stream);
+
+/*
+ * qsa_sparse_attn_prefill with a workspace: the same arguments, result and errors, plus `workspace`
+ * (caller-owned device memory, 16-byte aligned) of ws_bytes.
+ * When D = 128, Hq = 8 * Hkv (groups of 8 query heads), k_blocks <= 1024 and the workspace holds at
+ * least one tile (256 + 8 * (16 * k_blocks + 16) + 4 bytes; qsa_workspace_size(
+ * QSA_OP_SPARSE_ATTN_PREFILL, B, Tq, 0, k_blocks, Hq, D, 0) gives room for up to 4096 tiles), the
+ * rows are processed in tiles of 16 consecutive query rows on tcgen05 tensor cores: a tile attends
+ * over the union of its rows' listed blocks and own blocks, gathered once per tile, and each row
+ * masks out the union blocks it did not list ("Qwen3.8-Flash-Next architecture" (flozi.net), "Der
+ * Weg eines Tokens durch das Modell", item 2: exact attention over the selected tokens;
+ * consecutive queries select overlapping blocks).  The result is the same exact attention up to
+ * fp32 summation order.  Index lists must be ascending with -1 padding last (as qsa_select_topk
+ * writes them); other orders are accepted and cost a full sort per tile.  A non-finite K/V value in
+ * a block that one row of a tile lists reaches the other rows of the tile (0 * inf); positions
+ * past the call's last query are never read.  Other shapes, or no workspace, run the row-by-row
+ * kernel of qsa_sparse_attn_prefill.  Calls with more tiles than the workspace holds are processed
+ * in ranges of tiles.
+ */
+QSA_API qsa_status_t qsa_sparse_attn_prefill_ws(const void* q, const void* k, const void* v,
+                                        const int32_t* idx, int B, int Tq, int Tk, int Hq, int Hkv,
+                                        int D, int k_blocks, int blk, int64_t q_pos0, float scale,
+                                        void* out, float* lse, void* workspace, size_t ws_bytes,
+                                        void* stream);
+
+/*
+ * Chooses the prefill attention of qsa_sparse_attn_prefill_ws for all later calls from this
+ * process: 0 = automatic (query tiles where supported), 1 = row by row, 2 = query tiles
+ * (UNSUPPORTED for other shapes, WORKSPACE_TOO_SMALL without room for one tile).  A testing and
+ * tuning knob.  Errors: INVALID_ARGUMENT (path outside 0..2).
+ */
+QSA_API qsa_status_t qsa_set_attn_options(int path);
 
 /*
  * Gather-sparse attention, decode (split-KV).  One new token per sequence.
