@@ -116,25 +116,34 @@ def gather_ceiling(dev, stream, w, sweep: bool = False) -> dict:
         for iw, sl in ((1, 32), (2, 16), (8, 4), (8, 3), (12, 2), (16, 2)):
             cfg = dict(issuer_warps=iw, stages=3, slots_per_warp=sl)
             cases.append((f"l2_bulk_w{iw}_s{sl}", 32 << 20, 0, cfg))
-            cases.append((f"l2_lsu_w{iw}_s{sl}", 32 << 20, 1, cfg))
+        # smaller pieces: bulk copies of 512 B and tiled tensor boxes of 512 B / 1 KB
+        for iw, sl in ((1, 32), (4, 32), (8, 16), (16, 8)):   # 192 KB rings at most
+            cfg = dict(issuer_warps=iw, stages=3, slots_per_warp=sl)
+            cases.append((f"l2_bulk512_w{iw}_s{sl}", 32 << 20, 0, dict(cfg, chunk_bytes=512)))
+            cases.append((f"l2_tma512_w{iw}_s{sl}", 32 << 20, 3, dict(cfg, chunk_bytes=512)))
+            cfg = dict(issuer_warps=iw, stages=3, slots_per_warp=max(1, sl // 2))
+            cases.append((f"l2_tma1k_w{iw}_s{sl // 2}", 32 << 20, 4, dict(cfg, chunk_bytes=1024)))
     bufs = {}
     for name, nbytes, method, cfg in cases:
         if nbytes not in bufs:
             bufs[nbytes] = torch.ones(nbytes // 2, dtype=torch.bfloat16, device=dev)
         src = bufs[nbytes]
-        iters = max(1, int(2e9 // (148 * cfg["issuer_warps"] * cfg["slots_per_warp"] * chunk)))
-        Q.qsa.qsa_probe_gather(src, chunk_bytes=chunk, method=method, iterations=max(1, iters // 10), **cfg)
+        cfg = dict(cfg)
+        cb = cfg.pop("chunk_bytes", chunk)
+        iters = max(1, int(2e9 // (148 * cfg["issuer_warps"] * cfg["slots_per_warp"] * cb)))
+        Q.qsa.qsa_probe_gather(src, chunk_bytes=cb, method=method, iterations=max(1, iters // 10), **cfg)
         best = None
         for _ in range(3):
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-            nb = Q.qsa.qsa_probe_gather(src, chunk_bytes=chunk, method=method, iterations=iters, **cfg)
+            nb = Q.qsa.qsa_probe_gather(src, chunk_bytes=cb, method=method, iterations=iters, **cfg)
             e1.record(stream)
             torch.cuda.synchronize()
             gbs = nb / (e0.elapsed_time(e1) / 1000) / 1e9
             best = gbs if best is None else max(best, gbs)
         res[name + "_gbs"] = best
-    res["ceiling_gbs"] = max(v for k, v in res.items() if k.startswith("l2_bulk") and k.endswith("_gbs"))
+    res["ceiling_gbs"] = max(v for k, v in res.items()
+                             if k.startswith("l2_bulk") and "512" not in k and k.endswith("_gbs"))
     assert Q.qsa_get_device_status() == 0
     del bufs
     torch.cuda.empty_cache()

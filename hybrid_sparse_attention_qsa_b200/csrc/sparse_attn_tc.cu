@@ -21,16 +21,20 @@
 // silently).
 //
 // sparse_attn_tc_kernel (persistent, one CTA per SM), per (tile, KV head):
-//   warp 0   producer: the Q tile (two 128-byte-swizzled TMA boxes of [16 rows][8 heads][64 d]),
-//            then per chunk of 32 union entries one TMA box of [4 tokens][64 d] per block, half and
-//            tensor (K and V) into a 2-stage ring; the chunk's block ids and per-row member words
-//            go to shared memory;
-//   warp 1   TMEM owner and MMA issuer (one thread): S = Q K^T (M 128, N 128 tokens, K 128) into
+//   warps 0-7 producers: warp 0 loads the Q tile (two 128-byte-swizzled TMA boxes of [16 rows]
+//            [8 heads][64 d]) and, per chunk of 32 union entries, publishes the chunk's blocks and,
+//            per row, its member slots and the slot of its own block (the next chunk's entries are
+//            fetched ahead); then all 8 warps issue the chunk's 128 TMA boxes of [4 tokens][64 d]
+//            (block x half x K/V) into a 3-stage ring.  A single issuing warp caps these 512-byte
+//            gathers near 2 TB/s; eight reach ~10 TB/s (the gather probe);
+//   warp 8   TMEM owner and MMA issuer (one thread): S = Q K^T (M 128, N 128 tokens, K 128) into
 //            one of three S buffers, then O += P V with P read from TMEM (A operand) and V as an
 //            MN-major B operand;
-//   warps 2-5 softmax (one thread per row): mask, fp32 online softmax in exp2 form with a lazy
+//   warps 12-15 softmax (one thread per row): mask, fp32 online softmax in exp2 form with a lazy
 //            rescale of O (only when the running max grows by more than 2^8), P packed to bf16
 //            into the S buffer's columns, and the epilogue (O / l -> bf16 rows, log-sum-exp).
+//            Two passes over the row in TMEM (max, then exponentials), skipping groups of 8 union
+//            slots that no row of the warp attends.
 // TMEM: S0 S1 S2 at columns 0, 128, 256, O at 384 (fp32, lane = row).  Every wait is bounded; a
 // role whose wait runs out stops, and every role reaches the final barrier and TMEM release.
 #include <algorithm>
@@ -49,15 +53,19 @@ constexpr int kCT = kCB * 4;     // tokens per chunk (the N of S)
 constexpr int kHalf = 128 * 128; // bytes of one 64-column half of a 128-row operand (16 KB)
 constexpr int kQBytes = 2 * kHalf;
 constexpr int kKVBytes = 2 * kHalf;   // K (or V) of one chunk
-constexpr int kStages = 2;
+constexpr int kStages = 3;
 constexpr int kSoftWarps = 4;
-constexpr int kThreads = (2 + kSoftWarps) * 32;
+constexpr int kProdWarps = 8;         // warps issuing the TMA boxes (one issuing warp caps near 2 TB/s)
+constexpr int kMmaWarp = 8;
+constexpr int kSoftWarp0 = 12;        // softmax warps 12..15: TMEM lane quadrants 0..3
+constexpr int kThreads = 16 * 32;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleLog2 = 8.0f;  // O is rescaled only when the row max grows by more than this
 
 struct ChunkInfo {
   int blocks[kCB];
   uint32_t words[kTQ];   // bit j: the row attends union slot j of the chunk
+  uint32_t own[kTQ];     // bit j: union slot j holds the row's own block
 };
 
 constexpr int kInfoOff = kQBytes + kStages * 2 * kKVBytes;
@@ -76,6 +84,14 @@ struct TcArgs {
 };
 
 __device__ __forceinline__ int tile_chunks(int nu) { return max(1, (nu + kCB - 1) / kCB); }
+
+// 2^x on the special-function unit (flushes subnormal results to zero; 2^-inf = 0).  The
+// probabilities it produces are rounded to bf16 for the P.V product anyway.
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 // ---------------------------------------------------------------------------- tile unions
 __global__ void __launch_bounds__(512) tile_union_kernel(const int32_t* __restrict__ idx, int Tq, int kb,
@@ -218,9 +234,9 @@ __global__ void __launch_bounds__(512) tile_union_kernel(const int32_t* __restri
 
 // ---------------------------------------------------------------------------- attention
 struct Bars {
-  uint64_t kv_full[kStages], kv_empty[kStages];
+  uint64_t kv_full[kStages], kv_empty[kStages], ready[kStages];
   uint64_t s_full[3], p_full[3], s_free[3];
-  uint64_t q_full, q_empty, pv_done, o_free;
+  uint64_t q_full, q_empty, pv_done, o_full, o_free;
   uint32_t tmem;
 };
 
@@ -240,6 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bar->kv_full[s], 1);
       mbar_init(&bar->kv_empty[s], 1);
+      mbar_init(&bar->ready[s], 1);
     }
     for (int i = 0; i < 3; ++i) {
       mbar_init(&bar->s_full[i], 1);
@@ -249,10 +266,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bar->q_full, 1);
     mbar_init(&bar->q_empty, 1);
     mbar_init(&bar->pv_done, 1);
+    mbar_init(&bar->o_full, 1);
     mbar_init(&bar->o_free, kSoftWarps);
     fence_mbar_init();
   }
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tmem_alloc(&bar->tmem, 512);
     tmem_relinquish();
   }
@@ -262,11 +280,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = bar->tmem;
   const int ntl = a.ntiles;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------------ producer
-    prefetch_tensormap(&qmap);
-    prefetch_tensormap(&kmap);
-    prefetch_tensormap(&vmap);
+  if (warp < kProdWarps) {
+    // ------------------------------------------------------------------ producers
+    const bool lead = warp == 0;
+    if (lead) {
+      prefetch_tensormap(&qmap);
+      prefetch_tensormap(&kmap);
+      prefetch_tensormap(&vmap);
+    }
     int n = 0, hp = 0;
     bool alive = true;
     for (int it = blockIdx.x; alive && it < ntl; it += gridDim.x) {
@@ -278,7 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint2* te = a.ent + static_cast<long long>(tl) * a.cap;
       for (int g = 0; alive && g < HKV; ++g, ++hp) {
         bool ok = true;
-        if (lane == 0) {
+        if (lead && lane == 0) {
           ok = mbar_wait(&bar->q_empty, (hp & 1) ^ 1u, a.ctl);
           if (ok) {
             mbar_arrive_expect_tx(&bar->q_full, kQBytes);
@@ -287,48 +308,65 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         alive = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        uint2 e_next = (lead && nu > 0) ? te[min(lane, nu - 1)] : make_uint2(0u, 0u);   // first chunk's entries
         for (int c = 0; alive && c < nch; ++c, ++n) {
-          const int s = n & 1;
-          const unsigned f = static_cast<unsigned>(n >> 1);
+          const int s = n % kStages;
+          const unsigned f = static_cast<unsigned>(n / kStages);
+          if (lead) {
+            const int u = c * kCB + lane;
+            const uint2 e = e_next;
+            if (c + 1 < nch && nu > 0) e_next = te[min(u + kCB, nu - 1)];   // in flight while this chunk is set up
+            ok = true;
+            if (lane == 0) ok = mbar_wait(&bar->kv_empty[s], (f & 1u) ^ 1u, a.ctl);
+            alive = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (!alive) break;
+            const uint32_t mask = u < nu ? e.y : 0u;   // past the end: a repeat of the last entry, masked
+            uint32_t myw = 0, myo = 0;
+#pragma unroll
+            for (int q = 0; q < kTQ; ++q) {
+              const uint32_t bq = __ballot_sync(0xffffffffu, (mask >> q) & 1u);
+              const uint32_t oq = __ballot_sync(0xffffffffu, ((mask >> q) & 1u) &&
+                                                                 static_cast<long long>(e.x) == ((a.q_pos0 + t0 + q) >> 2));
+              if (lane == q) {
+                myw = bq;
+                myo = oq;
+              }
+            }
+            info[s].blocks[lane] = static_cast<int>(e.x);
+            if (lane < kTQ) {
+              info[s].words[lane] = myw;
+              info[s].own[lane] = myo;
+            }
+            __syncwarp();
+            if (lane == 0) {
+              mbar_arrive_expect_tx(&bar->kv_full[s], 2 * kKVBytes);   // before any box of the chunk is issued
+              mbar_arrive(&bar->ready[s]);
+            }
+          }
+          // every producer warp: its share of the 32 blocks x (K, V) x 2 halves = 128 boxes
           ok = true;
-          if (lane == 0) ok = mbar_wait(&bar->kv_empty[s], (f & 1u) ^ 1u, a.ctl);
+          if (lane == 0) ok = mbar_wait(&bar->ready[s], f & 1u, a.ctl);
           alive = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
           if (!alive) break;
-          const int u = c * kCB + lane;
-          const uint2 e = nu > 0 ? te[min(u, nu - 1)] : make_uint2(0u, 0u);   // past the end: a repeat, masked
-          const uint32_t mask = u < nu ? e.y : 0u;
-          uint32_t myw = 0;
-#pragma unroll
-          for (int q = 0; q < kTQ; ++q) {
-            const uint32_t bq = __ballot_sync(0xffffffffu, (mask >> q) & 1u);
-            if (lane == q) myw = bq;
-          }
-          info[s].blocks[lane] = static_cast<int>(e.x);
-          if (lane < kTQ) info[s].words[lane] = myw;
-          __syncwarp();
-          if (lane == 0) mbar_arrive_expect_tx(&bar->kv_full[s], 2 * kKVBytes);
-          __syncwarp();
-          uint8_t* ks = kvs + s * 2 * kKVBytes;
-          uint8_t* vs = ks + kKVBytes;
-          const int tok = static_cast<int>(e.x) * 4;
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            tma_load_4d(ks + h * kHalf + lane * 512, &kmap, &bar->kv_full[s], h * 64, g, tok, b);
-            tma_load_4d(vs + h * kHalf + lane * 512, &vmap, &bar->kv_full[s], h * 64, g, tok, b);
+          for (int bx = lane * kProdWarps + warp; bx < 4 * kCB; bx += 32 * kProdWarps) {
+            const int j = bx >> 2;
+            const int tv = (bx >> 1) & 1, half = bx & 1;
+            uint8_t* dst = kvs + s * 2 * kKVBytes + tv * kKVBytes + half * kHalf + j * 512;
+            tma_load_4d(dst, tv ? &vmap : &kmap, &bar->kv_full[s], half * 64, g, info[s].blocks[j] * 4, b);
           }
         }
       }
     }
     // never leave with a copy in flight: the last fill of each stage and the last Q tile
-    if (lane == 0) {
+    if (lead && lane == 0) {
       for (int s = 0; s < kStages && s < n; ++s) {
         const int last = s + ((n - 1 - s) / kStages) * kStages;
-        mbar_wait(&bar->kv_full[s], static_cast<unsigned>(last >> 1) & 1u, a.ctl);
+        mbar_wait(&bar->kv_full[s], static_cast<unsigned>(last / kStages) & 1u, a.ctl);
       }
       if (hp > 0) mbar_wait(&bar->q_full, static_cast<unsigned>(hp - 1) & 1u, a.ctl);
     }
     __syncwarp();
-  } else if (warp == 1) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc_s = umma_idesc_bf16_f32(128, kCT);
@@ -337,7 +375,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int n = 0, hp = 0;
       bool alive = true;
       auto issue_pv = [&](int m, bool first) -> bool {
-        const int sb = m % 3, s = m & 1;
+        const int sb = m % 3, s = m % kStages;
         if (!mbar_wait(&bar->p_full[sb], static_cast<unsigned>(m / 3) & 1u, a.ctl)) return false;
         if (first && hp > 0 && !mbar_wait(&bar->o_free, static_cast<unsigned>(hp - 1) & 1u, a.ctl)) return false;
         tc_fence_after();
@@ -362,8 +400,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const uint32_t qbase = smem_u32(qs);
           for (int c = 0; c < nch; ++c, ++n) {
-            const int s = n & 1, sb = n % 3;
-            if (!mbar_wait(&bar->kv_full[s], static_cast<unsigned>(n >> 1) & 1u, a.ctl) ||
+            const int s = n % kStages, sb = n % 3;
+            if (!mbar_wait(&bar->kv_full[s], static_cast<unsigned>(n / kStages) & 1u, a.ctl) ||
                 !mbar_wait(&bar->s_free[sb], (static_cast<unsigned>(n / 3) & 1u) ^ 1u, a.ctl)) {
               alive = false;
               break;
@@ -385,11 +423,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           if (alive && !issue_pv(n - 1, nch == 1)) alive = false;
+          // O of this (tile, head) is final once every MMA issued so far is complete.  (The epilogue
+          // cannot wait on pv_done: the last two PVs of a pass may both be pending then, and a
+          // parity wait cannot tell two phases apart.)
+          if (alive) umma_commit(&bar->o_full);
         }
       }
     }
     __syncwarp();
-  } else {
+  } else if (warp >= kSoftWarp0) {
     // ------------------------------------------------------------------ softmax + epilogue
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
@@ -405,54 +447,59 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int nch = tile_chunks(a.cnt[tl]);
       const bool vrow = t0 + t < a.Tq;
       const long long pos = a.q_pos0 + t0 + t;
-      const int own = static_cast<int>(pos >> 2);
       const int lim = static_cast<int>(pos & 3);
       for (int g = 0; alive && g < HKV; ++g, ++hp) {
         float m_ref = -INFINITY, l = 0.f;
         for (int c = 0; c < nch; ++c, ++n) {
-          const int s = n & 1, sb = n % 3;
+          const int s = n % kStages, sb = n % 3;
           if (!mbar_wait(&bar->s_full[sb], static_cast<unsigned>(n / 3) & 1u, a.ctl) ||
-              !mbar_wait(&bar->kv_full[s], static_cast<unsigned>(n >> 1) & 1u, a.ctl)) {
+              !mbar_wait(&bar->kv_full[s], static_cast<unsigned>(n / kStages) & 1u, a.ctl)) {
             alive = false;
             break;
           }
           tc_fence_after();
           const uint32_t word = vrow ? info[s].words[t] : 0u;
+          const uint32_t ownb = vrow ? info[s].own[t] : 0u;
+          const int oslot = ownb ? __ffs(ownb) - 1 : -1;
+          // slots some row of this warp (4 query rows) attends; the others need no exponentials
+          const uint32_t wor = __reduce_or_sync(0xffffffffu, word);
           const uint32_t s_addr = tmem + lane_addr + sb * 128;
-          float x[kCT];
+          // pass 1: the maximum of the attended raw scores (groups of 8 slots = 32 TMEM columns that
+          // no row of the warp attends are not even loaded)
+          float mraw = -INFINITY;
 #pragma unroll
           for (int p4 = 0; p4 < 4; ++p4) {
+            if (((wor >> (8 * p4)) & 0xFFu) == 0u) continue;   // warp-uniform
             uint32_t r[32];
             tmem_ld_32x32(s_addr + p4 * 32, r);
             tmem_ld_wait();
+            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-            for (int i = 0; i < 32; ++i) x[p4 * 32 + i] = __uint_as_float(r[i]);
-          }
-          float mx = -INFINITY;
+            for (int jj = 0; jj < 8; ++jj) {
+              const int j = 8 * p4 + jj;
+              const bool mem = (word >> j) & 1u;
+              const int lj = j == oslot ? lim : 3;
 #pragma unroll
-          for (int j = 0; j < kCB; ++j) {
-            const bool mem = (word >> j) & 1u;
-            const int tl_lim = info[s].blocks[j] == own ? lim : 3;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const bool ok = mem && i <= tl_lim;
-              const float v = ok ? x[4 * j + i] * a.scale_log2 : -INFINITY;
-              x[4 * j + i] = v;
-              mx = fmaxf(mx, v);
+              for (int i = 0; i < 4; ++i)
+                if (mem && i <= lj) m4[i] = fmaxf(m4[i], __uint_as_float(r[4 * jj + i]));
             }
+            mraw = fmaxf(mraw, fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])));
           }
+          const float mx = mraw * a.scale_log2;   // scale > 0: the max of the scaled logits
           bool resc = false;
           float factor = 1.f;
           if (mx > m_ref + kRescaleLog2) {
             if (c > 0) {
-              factor = exp2f(m_ref - mx);
+              factor = fast_exp2(m_ref - mx);
               l *= factor;
               resc = true;
             }
             m_ref = mx;
           }
           if (__any_sync(0xffffffffu, resc)) {
-            // O holds PV of chunks 0 .. c-1 once the last of them is complete
+            // O holds PV of chunks 0 .. c-1 once the last of them is complete.  S(n) was issued after
+            // PV(n-2) and is complete, so pv_done has completed n-1 or n phases here: the parity of
+            // phase n-1 is unambiguous.
             if (!mbar_wait(&bar->pv_done, static_cast<unsigned>(n - 1) & 1u, a.ctl)) {
               alive = false;
               break;
@@ -460,29 +507,50 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
 #pragma unroll
             for (int p4 = 0; p4 < 4; ++p4) {
-              uint32_t r[32];
-              tmem_ld_32x32(o_addr + p4 * 32, r);
+              uint32_t o[32];
+              tmem_ld_32x32(o_addr + p4 * 32, o);
               tmem_ld_wait();
 #pragma unroll
-              for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * factor);
-              tmem_st_32x32(o_addr + p4 * 32, r);
+              for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * factor);
+              tmem_st_32x32(o_addr + p4 * 32, o);
             }
             tmem_st_wait();
           }
-          const float ref = m_ref == -INFINITY ? 0.f : m_ref;
-          float sum = 0.f;
+          const float nref = m_ref == -INFINITY ? 0.f : -m_ref;
+          // pass 2: probabilities, packed to bf16 pairs into the S buffer's first 64 columns
+          float sum4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int h2 = 0; h2 < 2; ++h2) {
             uint32_t pk[32];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const float p0 = exp2f(x[h2 * 64 + 2 * i] - ref);
-              const float p1 = exp2f(x[h2 * 64 + 2 * i + 1] - ref);
-              sum += p0 + p1;
-              pk[i] = pack_bf16x2(p0, p1);
+            for (int q2 = 0; q2 < 2; ++q2) {
+              const int p4 = 2 * h2 + q2;
+              if (((wor >> (8 * p4)) & 0xFFu) == 0u) {   // warp-uniform
+#pragma unroll
+                for (int i = 0; i < 16; ++i) pk[16 * q2 + i] = 0u;
+                continue;
+              }
+              uint32_t r[32];
+              tmem_ld_32x32(s_addr + p4 * 32, r);
+              tmem_ld_wait();
+#pragma unroll
+              for (int jj = 0; jj < 8; ++jj) {
+                const int j = 8 * p4 + jj;
+                const bool mem = (word >> j) & 1u;
+                const int lj = j == oslot ? lim : 3;
+                float p[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  p[i] = (mem && i <= lj) ? fast_exp2(fmaf(__uint_as_float(r[4 * jj + i]), a.scale_log2, nref)) : 0.f;
+                  sum4[i] += p[i];
+                }
+                pk[16 * q2 + 2 * jj] = pack_bf16x2(p[0], p[1]);
+                pk[16 * q2 + 2 * jj + 1] = pack_bf16x2(p[2], p[3]);
+              }
             }
             tmem_st_32x32(s_addr + h2 * 32, pk);
           }
+          const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
           l += sum;
           tmem_st_wait();
           tc_fence_before();
@@ -491,7 +559,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!alive) break;
         // ---- epilogue of (tile, head): O / l -> bf16 row, log-sum-exp
-        if (!mbar_wait(&bar->pv_done, static_cast<unsigned>(n - 1) & 1u, a.ctl)) {
+        if (!mbar_wait(&bar->o_full, static_cast<unsigned>(hp) & 1u, a.ctl)) {
           alive = false;
           break;
         }
@@ -525,7 +593,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

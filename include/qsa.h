@@ -389,11 +389,13 @@ QSA_API qsa_status_t qsa_wait_timeout_selftest(uint64_t timeout_ns, void* stream
  * warps each keep `stages` x `slots_per_warp` chunks in flight per warp and refill them
  * `iterations` times from pseudo-random chunk-aligned offsets of src [src_bytes] (device memory,
  * 16-byte aligned; a buffer that fits in L2 gives the L2 -> SM ceiling).  method 0: 1-D bulk copies
- * (TMA engine, one per chunk); 1: 16-byte cp.async by every lane; 2: the two alternating by warp.
+ * (TMA engine, one per chunk); 1: 16-byte cp.async by every lane; 2: the two alternating by warp;
+ * 3 and 4: tiled tensor copies with the 128-byte swizzle from src viewed as [tokens][2][128] bf16,
+ * one box of [4 tokens][1 head][64] (chunk_bytes must be 512) or [4 tokens][2 heads][64] (1024).
  * Bytes delivered = CTAs * issuer_warps * iterations * slots_per_warp * chunk_bytes; time the
  * launch with events on `stream`.  The landed data are not read.
  * Errors: INVALID_ARGUMENT (null or misaligned src, chunk_bytes not a multiple of 16 in 16 .. 16384
- * or above src_bytes, method outside 0..2, issuer_warps outside 1..16, slots_per_warp outside
+ * or above src_bytes, method outside 0..4, issuer_warps outside 1..16, slots_per_warp outside
  * 1..32), UNSUPPORTED (stages outside 2..4, ring above 227 KB of shared memory).
  */
 QSA_API qsa_status_t qsa_probe_gather(const void* src, size_t src_bytes, int chunk_bytes, int method,
