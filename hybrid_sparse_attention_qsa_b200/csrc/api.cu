@@ -436,7 +436,7 @@ qsa_status_t qsa_sparse_attn_prefill_ws(const void* q, const void* k, const void
   if (!di) return QSA_ERR_CUDA;
   const int path = g_attn_path.load();
   const bool tiles_ok = attn_tc_supported(Hq, Hkv, D, k_blocks) && path != 1 && workspace != nullptr &&
-                        ok_ptr(workspace) && ws_bytes >= 256 + attn_tc_tile_bytes(k_blocks);
+                        ok_ptr(workspace) && ws_bytes >= 512 + attn_tc_tile_bytes(k_blocks);
   if (path == 2 && !tiles_ok)
     return attn_tc_supported(Hq, Hkv, D, k_blocks) ? QSA_ERR_WORKSPACE_TOO_SMALL : QSA_ERR_UNSUPPORTED;
   if (!tiles_ok)
@@ -511,7 +511,7 @@ size_t qsa_workspace_size(qsa_op_t op, int B, int Tq, int NBk, int k, int Hq, in
     if (B < 0 || Tq < 0 || k < 1) return 0;
     const long long tiles = static_cast<long long>(B) * ((Tq + 15) / 16);
     const long long n = std::max(1ll, std::min(tiles, 4096ll));
-    return static_cast<size_t>(256 + ((n * 4 + 255) & ~255ll) + n * static_cast<long long>(attn_tc_tile_bytes(k)));
+    return static_cast<size_t>(1024 + n * static_cast<long long>(attn_tc_tile_bytes(k)));
   }
   if (op == QSA_OP_SPARSE_ATTN_DECODE) {
     if (B < 1 || Hq < 1 || D < 1) return 0;

@@ -35,8 +35,10 @@
 //            into the S buffer's columns, and the epilogue (O / l -> bf16 rows, log-sum-exp).
 //            Two passes over the row in TMEM (max, then exponentials), skipping groups of 8 union
 //            slots that no row of the warp attends.
-// TMEM: S0 S1 S2 at columns 0, 128, 256, O at 384 (fp32, lane = row).  Every wait is bounded; a
-// role whose wait runs out stops, and every role reaches the final barrier and TMEM release.
+// TMEM: S0 S1 S2 at columns 0, 128, 256, O at 384 (fp32, lane = row).  Every wait is bounded and
+// suspends the waiting warp (spinning producer and MMA warps would take issue slots from the softmax
+// warps on their schedulers); a role whose wait runs out stops, and every role reaches the final
+// barrier and TMEM release.
 #include <algorithm>
 #include <mutex>
 
@@ -48,37 +50,56 @@ namespace {
 constexpr int kTQ = 16;          // query rows per tile
 constexpr int kGrp = 8;          // query heads per KV head (the M of a tile is kTQ * kGrp = 128)
 constexpr int kD = 128;
-constexpr int kCB = 32;          // union blocks per chunk
-constexpr int kCT = kCB * 4;     // tokens per chunk (the N of S)
-constexpr int kHalf = 128 * 128; // bytes of one 64-column half of a 128-row operand (16 KB)
-constexpr int kQBytes = 2 * kHalf;
-constexpr int kKVBytes = 2 * kHalf;   // K (or V) of one chunk
-constexpr int kStages = 3;
-constexpr int kSoftWarps = 4;
-constexpr int kProdWarps = 8;         // warps issuing the TMA boxes (one issuing warp caps near 2 TB/s)
-constexpr int kMmaWarp = 8;
-constexpr int kSoftWarp0 = 12;        // softmax warps 12..15: TMEM lane quadrants 0..3
-constexpr int kThreads = 16 * 32;
+constexpr int kCB = 16;          // union blocks per chunk
+constexpr int kCT = kCB * 4;     // tokens per chunk (the N of S; S columns per buffer)
+constexpr int kQHalf = 128 * 128;         // one 64-column half of the Q tile (128 rows x 128 B)
+constexpr int kQBytes = 2 * kQHalf;
+constexpr int kKVHalf = kCT * 128;        // one 64-column half of a chunk's K (or V): kCT rows x 128 B
+constexpr int kKVBytes = 2 * kKVHalf;     // K (or V) of one chunk
+constexpr int kStages = 5;                // K/V ring depth (shared memory)
+constexpr int kSBuf = 4;                  // S buffers in TMEM (kCT columns each), then two O accumulators
+constexpr int kProdWarps = 7;             // warps issuing the TMA boxes (each box costs its warp ~80 cycles)
+constexpr int kMmaWarp = 7;
+constexpr int kSoftWarp0 = 8;             // softmax warps 8..15: group (w - 8) / 4 takes every other chunk
+constexpr int kSoftWarps = 8;             // of a pass; warp w reads TMEM lane quadrant w % 4
+constexpr int kThreads = (kSoftWarp0 + kSoftWarps) * 32;
+// Register split (setmaxnreg): the block launches with kLaunchRegs per thread; warpgroups 0-1
+// (producers, MMA) drop to kLowRegs and warpgroups 2-3 (softmax) rise to kHighRegs.  The sum must
+// not exceed the launch's total, or the increase would wait for ever; the host refuses the launch
+// unless the compiled kernel has exactly kLaunchRegs registers per thread.
+constexpr int kLaunchRegs = 65536 / kThreads;
+constexpr int kLowRegs = 64;
+constexpr int kHighRegs = 192;
+static_assert(kThreads == 512 && kSoftWarp0 == 8, "two warpgroups per side of the split");
+static_assert(256 * kLowRegs + 256 * kHighRegs <= kThreads * kLaunchRegs, "register split");
+constexpr int kOCol = kSBuf * kCT;        // TMEM columns of the two O accumulators (128 columns each)
+static_assert(kOCol + 2 * kD <= 512, "TMEM columns");
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleLog2 = 8.0f;  // O is rescaled only when the row max grows by more than this
 
+// One chunk of a tile's union, as the union kernel writes it and one bulk copy brings it to shared
+// memory beside the chunk's K/V.
 struct ChunkInfo {
-  int blocks[kCB];
-  uint32_t words[kTQ];   // bit j: the row attends union slot j of the chunk
-  uint32_t own[kTQ];     // bit j: union slot j holds the row's own block
+  int blocks[kCB];        // union block of each slot (past the end of the union: a repeat, masked)
+  uint16_t words[kTQ];    // per row: bit j = the row attends slot j
+  int8_t oslot[kTQ];      // per row: the slot holding its own block, or -1
+  uint8_t pad[16];
 };
+static_assert(sizeof(ChunkInfo) == 128, "one 128-byte bulk copy per chunk");
 
 constexpr int kInfoOff = kQBytes + kStages * 2 * kKVBytes;
 constexpr int kBarOff = kInfoOff + kStages * static_cast<int>(sizeof(ChunkInfo));
-constexpr int kSmem = 1024 + kBarOff + 256;
+constexpr int kXchgOff = kBarOff + 512;   // [4 quadrants][2 groups][2 values][32 lanes] floats
+constexpr int kSmem = 1024 + kXchgOff + 4 * 2 * 2 * 32 * 4;
+static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
 
 struct TcArgs {
-  const uint2* ent;      // [tiles][cap] (block, row mask) per tile of this launch
+  const ChunkInfo* recs; // [tiles][capc] chunk records per tile of this launch
   const int* cnt;        // [tiles]
   uint16_t* out;
   float* lse;
   long long q_pos0;
-  int B, Tq, Hq, Hkv, cap, tile0, ntiles, tpb;
+  int B, Tq, Hq, Hkv, capc, tile0, ntiles, tpb;
   float scale_log2;
   KernelCtl ctl;
 };
@@ -97,7 +118,7 @@ __device__ __forceinline__ float fast_exp2(float x) {
 __global__ void __launch_bounds__(512) tile_union_kernel(const int32_t* __restrict__ idx, int Tq, int kb,
                                                          long long q_pos0, int tile0, int tpb, int n2,
                                                          uint2* __restrict__ ent, int* __restrict__ cnt, int cap,
-                                                         KernelCtl ctl) {
+                                                         ChunkInfo* __restrict__ recs, int capc, KernelCtl ctl) {
   extern __shared__ uint32_t ukeys[];
   uint32_t* keys = ukeys;                 // [n2]
   uint32_t* merged = keys + n2;           // [16 * kb + 16]
@@ -230,15 +251,46 @@ __global__ void __launch_bounds__(512) tile_union_kernel(const int32_t* __restri
     }
   }
   if (tid == 0) cnt[tl] = s_scan[16];
+  // the chunk records: one warp per chunk of 16 entries (the entries written above are visible to
+  // the whole block after the barrier)
+  __syncthreads();
+  const int nu = s_scan[16];
+  const int nch = max(1, (nu + kCB - 1) / kCB);
+  ChunkInfo* tr = recs + static_cast<long long>(tl) * capc;
+  for (int c = w; c < nch; c += blockDim.x >> 5) {
+    const int uu = c * kCB + lane;
+    const uint2 e = te[min(uu, max(nu - 1, 0))];
+    const uint32_t mask = (lane < kCB && uu < nu) ? e.y : 0u;
+    uint32_t myw = 0;
+    int myo = -1;
+#pragma unroll
+    for (int q = 0; q < kTQ; ++q) {
+      const uint32_t bq = __ballot_sync(0xffffffffu, (mask >> q) & 1u);
+      const uint32_t oq = __ballot_sync(0xffffffffu, ((mask >> q) & 1u) &&
+                                                         static_cast<long long>(e.x) == ((q_pos0 + t0 + q) >> 2));
+      if (lane == q) {
+        myw = bq;
+        myo = oq ? __ffs(oq) - 1 : -1;
+      }
+    }
+    ChunkInfo* r = tr + c;
+    if (lane < kCB) r->blocks[lane] = static_cast<int>(e.x);
+    if (lane < kTQ) {
+      r->words[lane] = static_cast<uint16_t>(myw);
+      r->oslot[lane] = static_cast<int8_t>(myo);
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------- attention
 struct Bars {
-  uint64_t kv_full[kStages], kv_empty[kStages], ready[kStages];
-  uint64_t s_full[3], p_full[3], s_free[3];
-  uint64_t q_full, q_empty, pv_done, o_full, o_free;
+  uint64_t kv_full[kStages], kv_empty[kStages];
+  uint64_t s_full[kSBuf], p_full[kSBuf], s_free[kSBuf];
+  uint64_t q_full, q_empty, o_full, o_free;
+  uint64_t pair[4];      // per TMEM lane quadrant: both groups have posted their (m, l) of the pass
   uint32_t tmem;
 };
+static_assert(sizeof(Bars) <= 512, "barrier area");
 
 template <int HKV>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -247,27 +299,26 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* qs = smem;                                   // [2 halves][128 rows][128 B]
-  uint8_t* kvs = smem + kQBytes;                        // per stage: K [2][128 tokens][128 B], V likewise
+  uint8_t* kvs = smem + kQBytes;                        // per stage: K [2 halves][kCT tokens][128 B], V likewise
   ChunkInfo* info = reinterpret_cast<ChunkInfo*>(smem + kInfoOff);
   Bars* bar = reinterpret_cast<Bars*>(smem + kBarOff);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&bar->kv_full[s], 1);
+      mbar_init(&bar->kv_full[s], kProdWarps);   // every producer warp registers its own bytes
       mbar_init(&bar->kv_empty[s], 1);
-      mbar_init(&bar->ready[s], 1);
     }
-    for (int i = 0; i < 3; ++i) {
+    for (int i = 0; i < kSBuf; ++i) {
       mbar_init(&bar->s_full[i], 1);
-      mbar_init(&bar->p_full[i], kSoftWarps);
+      mbar_init(&bar->p_full[i], kSoftWarps / 2);   // one group writes a chunk's P
       mbar_init(&bar->s_free[i], 1);
     }
     mbar_init(&bar->q_full, 1);
     mbar_init(&bar->q_empty, 1);
-    mbar_init(&bar->pv_done, 1);
     mbar_init(&bar->o_full, 1);
     mbar_init(&bar->o_free, kSoftWarps);
+    for (int i = 0; i < 4; ++i) mbar_init(&bar->pair[i], 2);
     fence_mbar_init();
   }
   if (warp == kMmaWarp) {
@@ -279,166 +330,170 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = bar->tmem;
   const int ntl = a.ntiles;
-
+  if (warp < kSoftWarp0) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kLowRegs));
   if (warp < kProdWarps) {
     // ------------------------------------------------------------------ producers
+    // Every producer warp takes a fixed share of a chunk's 4 * kCB boxes (block x K/V x half), with
+    // the block ids fetched one chunk ahead from the chunk records; it registers its own bytes on
+    // the stage's full barrier and issues its boxes.  Warp 0 also brings the chunk's record.
     const bool lead = warp == 0;
     if (lead) {
       prefetch_tensormap(&qmap);
       prefetch_tensormap(&kmap);
       prefetch_tensormap(&vmap);
     }
+    const int bx = lane * kProdWarps + warp;      // this lane's box of a chunk (none past 4 * kCB)
+    const bool has_box = bx < 4 * kCB;
+    const int bj = bx >> 2, btv = (bx >> 1) & 1, bhalf = bx & 1;
+    const uint32_t nbox = __popc(__ballot_sync(0xffffffffu, has_box));
+    const uint32_t my_bytes = nbox * 512 + (lead ? static_cast<uint32_t>(sizeof(ChunkInfo)) : 0u);
     int n = 0, hp = 0;
     bool alive = true;
     for (int it = blockIdx.x; alive && it < ntl; it += gridDim.x) {
       const int tl = ntl - 1 - it;
       const int tile = a.tile0 + tl;
       const int b = tile / a.tpb, t0 = (tile % a.tpb) * kTQ;
-      const int nu = a.cnt[tl];
-      const int nch = tile_chunks(nu);
-      const uint2* te = a.ent + static_cast<long long>(tl) * a.cap;
+      const int nch = tile_chunks(a.cnt[tl]);
+      const ChunkInfo* tr = a.recs + static_cast<long long>(tl) * a.capc;
       for (int g = 0; alive && g < HKV; ++g, ++hp) {
         bool ok = true;
         if (lead && lane == 0) {
-          ok = mbar_wait(&bar->q_empty, (hp & 1) ^ 1u, a.ctl);
+          ok = mbar_wait_suspend(&bar->q_empty, (hp & 1) ^ 1u, a.ctl);
           if (ok) {
             mbar_arrive_expect_tx(&bar->q_full, kQBytes);
             tma_load_4d(qs, &qmap, &bar->q_full, 0, g * kGrp, t0, b);
-            tma_load_4d(qs + kHalf, &qmap, &bar->q_full, 64, g * kGrp, t0, b);
+            tma_load_4d(qs + kQHalf, &qmap, &bar->q_full, 64, g * kGrp, t0, b);
           }
         }
         alive = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-        uint2 e_next = (lead && nu > 0) ? te[min(lane, nu - 1)] : make_uint2(0u, 0u);   // first chunk's entries
+        int blk_next = has_box ? tr[0].blocks[bj] : 0;   // the first chunk's block of this lane's box
         for (int c = 0; alive && c < nch; ++c, ++n) {
           const int s = n % kStages;
           const unsigned f = static_cast<unsigned>(n / kStages);
-          if (lead) {
-            const int u = c * kCB + lane;
-            const uint2 e = e_next;
-            if (c + 1 < nch && nu > 0) e_next = te[min(u + kCB, nu - 1)];   // in flight while this chunk is set up
-            ok = true;
-            if (lane == 0) ok = mbar_wait(&bar->kv_empty[s], (f & 1u) ^ 1u, a.ctl);
-            alive = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-            if (!alive) break;
-            const uint32_t mask = u < nu ? e.y : 0u;   // past the end: a repeat of the last entry, masked
-            uint32_t myw = 0, myo = 0;
-#pragma unroll
-            for (int q = 0; q < kTQ; ++q) {
-              const uint32_t bq = __ballot_sync(0xffffffffu, (mask >> q) & 1u);
-              const uint32_t oq = __ballot_sync(0xffffffffu, ((mask >> q) & 1u) &&
-                                                                 static_cast<long long>(e.x) == ((a.q_pos0 + t0 + q) >> 2));
-              if (lane == q) {
-                myw = bq;
-                myo = oq;
-              }
-            }
-            info[s].blocks[lane] = static_cast<int>(e.x);
-            if (lane < kTQ) {
-              info[s].words[lane] = myw;
-              info[s].own[lane] = myo;
-            }
-            __syncwarp();
-            if (lane == 0) {
-              mbar_arrive_expect_tx(&bar->kv_full[s], 2 * kKVBytes);   // before any box of the chunk is issued
-              mbar_arrive(&bar->ready[s]);
-            }
-          }
-          // every producer warp: its share of the 32 blocks x (K, V) x 2 halves = 128 boxes
+          const int blk = blk_next;
+          if (c + 1 < nch && has_box) blk_next = tr[c + 1].blocks[bj];   // in flight while this chunk is issued
           ok = true;
-          if (lane == 0) ok = mbar_wait(&bar->ready[s], f & 1u, a.ctl);
+          if (lane == 0) {
+            ok = mbar_wait_suspend(&bar->kv_empty[s], (f & 1u) ^ 1u, a.ctl);
+            if (ok) mbar_arrive_expect_tx(&bar->kv_full[s], my_bytes);   // before this warp's copies
+          }
           alive = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
           if (!alive) break;
-          for (int bx = lane * kProdWarps + warp; bx < 4 * kCB; bx += 32 * kProdWarps) {
-            const int j = bx >> 2;
-            const int tv = (bx >> 1) & 1, half = bx & 1;
-            uint8_t* dst = kvs + s * 2 * kKVBytes + tv * kKVBytes + half * kHalf + j * 512;
-            tma_load_4d(dst, tv ? &vmap : &kmap, &bar->kv_full[s], half * 64, g, info[s].blocks[j] * 4, b);
+          if (lead && lane == 0)
+            bulk_g2s(&info[s], tr + c, static_cast<unsigned>(sizeof(ChunkInfo)), &bar->kv_full[s]);
+          if (has_box) {
+            uint8_t* dst = kvs + s * 2 * kKVBytes + btv * kKVBytes + bhalf * kKVHalf + bj * 512;
+            tma_load_4d(dst, btv ? &vmap : &kmap, &bar->kv_full[s], bhalf * 64, g, blk * 4, b);
           }
         }
       }
     }
-    // never leave with a copy in flight: the last fill of each stage and the last Q tile
-    if (lead && lane == 0) {
+    // never leave with a copy in flight: the last fill of each stage (all warps' copies) and the
+    // last Q tile
+    if (lane == 0) {
       for (int s = 0; s < kStages && s < n; ++s) {
         const int last = s + ((n - 1 - s) / kStages) * kStages;
-        mbar_wait(&bar->kv_full[s], static_cast<unsigned>(last / kStages) & 1u, a.ctl);
+        mbar_wait_suspend(&bar->kv_full[s], static_cast<unsigned>(last / kStages) & 1u, a.ctl);
       }
-      if (hp > 0) mbar_wait(&bar->q_full, static_cast<unsigned>(hp - 1) & 1u, a.ctl);
+      if (lead && hp > 0) mbar_wait_suspend(&bar->q_full, static_cast<unsigned>(hp - 1) & 1u, a.ctl);
     }
     __syncwarp();
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer
+    // Within a (tile, head) pass, S(i) and PV(j) are issued as soon as each is ready (S(i): the
+    // chunk's K/V and a free S buffer; PV(j): the softmax's P and, for each accumulator's first PV
+    // of the pass, both accumulators read out by the previous epilogue), so a PV whose P is ready
+    // never waits behind the next chunk's data.  Chunk j of a pass accumulates into O[j & 1].
     if (lane == 0) {
       const uint32_t idesc_s = umma_idesc_bf16_f32(128, kCT);
       const uint32_t idesc_pv = umma_idesc_bf16_f32_bmn(128, kD);
-      const uint32_t o_col = tmem + 384;
-      int n = 0, hp = 0;
+      int n0 = 0, hp = 0;   // n0: global index of the pass's first chunk
       bool alive = true;
-      auto issue_pv = [&](int m, bool first) -> bool {
-        const int sb = m % 3, s = m % kStages;
-        if (!mbar_wait(&bar->p_full[sb], static_cast<unsigned>(m / 3) & 1u, a.ctl)) return false;
-        if (first && hp > 0 && !mbar_wait(&bar->o_free, static_cast<unsigned>(hp - 1) & 1u, a.ctl)) return false;
-        tc_fence_after();
-        const uint32_t vbase = smem_u32(kvs + s * 2 * kKVBytes + kKVBytes);
-#pragma unroll
-        for (int kk = 0; kk < kCT / 16; ++kk) {
-          const uint64_t bd = sw128_mnmajor_desc(vbase + kk * 2048, kHalf, 1024);
-          umma_bf16_ta(o_col, tmem + sb * 128 + kk * 8, bd, idesc_pv, (first && kk == 0) ? 0u : 1u);
-        }
-        umma_commit(&bar->kv_empty[s]);
-        umma_commit(&bar->s_free[sb]);
-        umma_commit(&bar->pv_done);
-        return true;
-      };
       for (int it = blockIdx.x; alive && it < ntl; it += gridDim.x) {
         const int tl = ntl - 1 - it;
         const int nch = tile_chunks(a.cnt[tl]);
-        for (int g = 0; alive && g < HKV; ++g, ++hp) {
-          if (!mbar_wait(&bar->q_full, static_cast<unsigned>(hp) & 1u, a.ctl)) {
+        for (int g = 0; alive && g < HKV; ++g, ++hp, n0 += nch) {
+          if (!mbar_wait_suspend(&bar->q_full, static_cast<unsigned>(hp) & 1u, a.ctl)) {
             alive = false;
             break;
           }
           const uint32_t qbase = smem_u32(qs);
-          for (int c = 0; c < nch; ++c, ++n) {
-            const int s = n % kStages, sb = n % 3;
-            if (!mbar_wait(&bar->kv_full[s], static_cast<unsigned>(n / kStages) & 1u, a.ctl) ||
-                !mbar_wait(&bar->s_free[sb], (static_cast<unsigned>(n / 3) & 1u) ^ 1u, a.ctl)) {
-              alive = false;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t kbase = smem_u32(kvs + s * 2 * kKVBytes);
+          int si = 0, pj = 0;   // next S and next PV of the pass
+          unsigned long long t_last = globaltimer_ns();
+          while (pj < nch) {
+            bool progress = false;
+            if (si < nch) {
+              const int n = n0 + si, s = n % kStages, sb = n % kSBuf;
+              if (mbar_try_wait(&bar->kv_full[s], static_cast<unsigned>(n / kStages) & 1u) &&
+                  mbar_try_wait(&bar->s_free[sb], (static_cast<unsigned>(n / kSBuf) & 1u) ^ 1u)) {
+                tc_fence_after();
+                const uint32_t kbase = smem_u32(kvs + s * 2 * kKVBytes);
 #pragma unroll
-            for (int kk = 0; kk < kD / 16; ++kk) {
-              const int h = kk >> 2;
-              const uint64_t ad = sw128_kmajor_desc(qbase + h * kHalf) + 2 * (kk & 3);
-              const uint64_t bd = sw128_kmajor_desc(kbase + h * kHalf) + 2 * (kk & 3);
-              umma_bf16(tmem + sb * 128, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+                for (int kk = 0; kk < kD / 16; ++kk) {
+                  const int h = kk >> 2;
+                  const uint64_t ad = sw128_kmajor_desc(qbase + h * kQHalf) + 2 * (kk & 3);
+                  const uint64_t bd = sw128_kmajor_desc(kbase + h * kKVHalf) + 2 * (kk & 3);
+                  umma_bf16(tmem + sb * kCT, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(&bar->s_full[sb]);
+                if (si == nch - 1) umma_commit(&bar->q_empty);   // Q is free once the pass's S are done
+                ++si;
+                progress = true;
+              }
             }
-            umma_commit(&bar->s_full[sb]);
-            if (c == nch - 1) umma_commit(&bar->q_empty);
-            if (c > 0 && !issue_pv(n - 1, c == 1)) {
+            if (pj < si) {
+              const int m = n0 + pj, s = m % kStages, sb = m % kSBuf;
+              const bool first = pj < 2;   // the accumulator's first PV of the pass
+              if (mbar_try_wait(&bar->p_full[sb], static_cast<unsigned>(m / kSBuf) & 1u) &&
+                  (!first || hp == 0 || mbar_try_wait(&bar->o_free, static_cast<unsigned>(hp - 1) & 1u))) {
+                tc_fence_after();
+                const uint32_t vbase = smem_u32(kvs + s * 2 * kKVBytes + kKVBytes);
+                const uint32_t o_col = tmem + kOCol + (pj & 1) * kD;
+#pragma unroll
+                for (int kk = 0; kk < kCT / 16; ++kk) {
+                  const uint64_t bd = sw128_mnmajor_desc(vbase + kk * 2048, kKVHalf, 1024);
+                  umma_bf16_ta(o_col, tmem + sb * kCT + kk * 8, bd, idesc_pv, (first && kk == 0) ? 0u : 1u);
+                }
+                umma_commit(&bar->kv_empty[s]);
+                umma_commit(&bar->s_free[sb]);
+                ++pj;
+                progress = true;
+              }
+            }
+            if (progress) {
+              t_last = globaltimer_ns();
+            } else if (globaltimer_ns() - t_last > a.ctl.wait_ns) {
+              record_status(a.ctl, kStTimeout);
               alive = false;
               break;
             }
           }
-          if (alive && !issue_pv(n - 1, nch == 1)) alive = false;
           // O of this (tile, head) is final once every MMA issued so far is complete.  (The epilogue
-          // cannot wait on pv_done: the last two PVs of a pass may both be pending then, and a
+          // cannot wait on a per-chunk barrier: the last PVs of a pass may be pending then, and a
           // parity wait cannot tell two phases apart.)
           if (alive) umma_commit(&bar->o_full);
         }
       }
     }
     __syncwarp();
-  } else if (warp >= kSoftWarp0) {
+  }
+  } else {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kHighRegs));
+  {
     // ------------------------------------------------------------------ softmax + epilogue
+    // Two groups of four warps (one per TMEM lane quadrant) take alternate chunks of a pass, each
+    // with its own running (m, l) and its own O accumulator, so two chunks are in the softmax at
+    // once.  At the end of the pass the two states merge by log-sum-exp: each warp of a quadrant
+    // pair writes 64 of the 128 output columns.
     const int quad = warp & 3;
+    const int grp = (warp - kSoftWarp0) >> 2;
     const int row = quad * 32 + lane;
     const int t = row >> 3, hh = row & 7;
     const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
-    const uint32_t o_addr = tmem + lane_addr + 384;
-    int n = 0, hp = 0;
+    const uint32_t o_mine = tmem + lane_addr + kOCol + grp * kD;
+    float* xchg = reinterpret_cast<float*>(smem + kXchgOff) + quad * 2 * 2 * 32;   // [grp][m, l][lane]
+    int n0 = 0, hp = 0;
     bool alive = true;
     for (int it = blockIdx.x; alive && it < ntl; it += gridDim.x) {
       const int tl = ntl - 1 - it;
@@ -448,48 +503,45 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool vrow = t0 + t < a.Tq;
       const long long pos = a.q_pos0 + t0 + t;
       const int lim = static_cast<int>(pos & 3);
-      for (int g = 0; alive && g < HKV; ++g, ++hp) {
+      for (int g = 0; alive && g < HKV; ++g, ++hp, n0 += nch) {
         float m_ref = -INFINITY, l = 0.f;
-        for (int c = 0; c < nch; ++c, ++n) {
-          const int s = n % kStages, sb = n % 3;
-          if (!mbar_wait(&bar->s_full[sb], static_cast<unsigned>(n / 3) & 1u, a.ctl) ||
-              !mbar_wait(&bar->kv_full[s], static_cast<unsigned>(n / kStages) & 1u, a.ctl)) {
+        for (int c = grp; c < nch; c += 2) {
+          const int n = n0 + c, s = n % kStages, sb = n % kSBuf;
+          if (!mbar_wait_suspend(&bar->s_full[sb], static_cast<unsigned>(n / kSBuf) & 1u, a.ctl) ||
+              !mbar_wait_suspend(&bar->kv_full[s], static_cast<unsigned>(n / kStages) & 1u, a.ctl)) {
             alive = false;
             break;
           }
           tc_fence_after();
+          // the row's member slots of the chunk and the slot of its own block
           const uint32_t word = vrow ? info[s].words[t] : 0u;
-          const uint32_t ownb = vrow ? info[s].own[t] : 0u;
-          const int oslot = ownb ? __ffs(ownb) - 1 : -1;
-          // slots some row of this warp (4 query rows) attends; the others need no exponentials
-          const uint32_t wor = __reduce_or_sync(0xffffffffu, word);
-          const uint32_t s_addr = tmem + lane_addr + sb * 128;
-          // pass 1: the maximum of the attended raw scores (groups of 8 slots = 32 TMEM columns that
-          // no row of the warp attends are not even loaded)
-          float mraw = -INFINITY;
+          const int oslot = vrow ? info[s].oslot[t] : -1;
+          const uint32_t wor = __reduce_or_sync(0xffffffffu, word);   // slots some row of the warp attends
+          const uint32_t s_addr = tmem + lane_addr + sb * kCT;
+          uint32_t r[2][32];
+          if (wor & 0xFFu) tmem_ld_32x32(s_addr, r[0]);
+          if (wor & 0xFF00u) tmem_ld_32x32(s_addr + 32, r[1]);
+          tmem_ld_wait();
+          // masked raw scores (-inf where the row does not attend) and their maximum; straight-line
+          // selects (per-slot branches cost more than the arithmetic they skip)
+          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-          for (int p4 = 0; p4 < 4; ++p4) {
-            if (((wor >> (8 * p4)) & 0xFFu) == 0u) continue;   // warp-uniform
-            uint32_t r[32];
-            tmem_ld_32x32(s_addr + p4 * 32, r);
-            tmem_ld_wait();
-            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+          for (int j = 0; j < kCB; ++j) {
+            const bool mem = (word >> j) & 1u;
+            const int lj = j == oslot ? lim : 3;
 #pragma unroll
-            for (int jj = 0; jj < 8; ++jj) {
-              const int j = 8 * p4 + jj;
-              const bool mem = (word >> j) & 1u;
-              const int lj = j == oslot ? lim : 3;
-#pragma unroll
-              for (int i = 0; i < 4; ++i)
-                if (mem && i <= lj) m4[i] = fmaxf(m4[i], __uint_as_float(r[4 * jj + i]));
+            for (int i = 0; i < 4; ++i) {
+              const float v = (mem && i <= lj) ? __uint_as_float(r[j >> 3][(j & 7) * 4 + i]) : -INFINITY;
+              r[j >> 3][(j & 7) * 4 + i] = __float_as_uint(v);
+              m4[i] = fmaxf(m4[i], v);
             }
-            mraw = fmaxf(mraw, fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])));
           }
+          const float mraw = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
           const float mx = mraw * a.scale_log2;   // scale > 0: the max of the scaled logits
           bool resc = false;
           float factor = 1.f;
           if (mx > m_ref + kRescaleLog2) {
-            if (c > 0) {
+            if (c >= 2) {   // the group's accumulator holds earlier chunks
               factor = fast_exp2(m_ref - mx);
               l *= factor;
               resc = true;
@@ -497,10 +549,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             m_ref = mx;
           }
           if (__any_sync(0xffffffffu, resc)) {
-            // O holds PV of chunks 0 .. c-1 once the last of them is complete.  S(n) was issued after
-            // PV(n-2) and is complete, so pv_done has completed n-1 or n phases here: the parity of
-            // phase n-1 is unambiguous.
-            if (!mbar_wait(&bar->pv_done, static_cast<unsigned>(n - 1) & 1u, a.ctl)) {
+            // The group's O holds its chunks before c once PV(n-2), its previous chunk, is complete
+            // (its commit covers every earlier MMA): s_free of that S buffer.  That barrier's
+            // previous phase, PV(n-2-kSBuf), is complete (S(n-2) waited for it), so the parity of
+            // PV(n-2)'s phase is unambiguous.
+            const int pm = n - 2;
+            if (!mbar_wait_suspend(&bar->s_free[pm % kSBuf], static_cast<unsigned>(pm / kSBuf) & 1u, a.ctl)) {
               alive = false;
               break;
             }
@@ -508,88 +562,92 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int p4 = 0; p4 < 4; ++p4) {
               uint32_t o[32];
-              tmem_ld_32x32(o_addr + p4 * 32, o);
+              tmem_ld_32x32(o_mine + p4 * 32, o);
               tmem_ld_wait();
 #pragma unroll
               for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * factor);
-              tmem_st_32x32(o_addr + p4 * 32, o);
+              tmem_st_32x32(o_mine + p4 * 32, o);
             }
             tmem_st_wait();
           }
           const float nref = m_ref == -INFINITY ? 0.f : -m_ref;
-          // pass 2: probabilities, packed to bf16 pairs into the S buffer's first 64 columns
           float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+          // P of the chunk's kCB slots = bf16 pairs in the S buffer's first kCT / 2 columns
 #pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
-            uint32_t pk[32];
+          for (int q8 = 0; q8 < 2; ++q8) {
+            uint32_t pk[16];
 #pragma unroll
-            for (int q2 = 0; q2 < 2; ++q2) {
-              const int p4 = 2 * h2 + q2;
-              if (((wor >> (8 * p4)) & 0xFFu) == 0u) {   // warp-uniform
+            for (int jj = 0; jj < 8; ++jj) {
+              float p[4];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) pk[16 * q2 + i] = 0u;
-                continue;
+              for (int i = 0; i < 4; ++i) {   // masked entries hold -inf: 2^-inf = 0
+                p[i] = fast_exp2(fmaf(__uint_as_float(r[q8][jj * 4 + i]), a.scale_log2, nref));
+                sum4[i] += p[i];
               }
-              uint32_t r[32];
-              tmem_ld_32x32(s_addr + p4 * 32, r);
-              tmem_ld_wait();
-#pragma unroll
-              for (int jj = 0; jj < 8; ++jj) {
-                const int j = 8 * p4 + jj;
-                const bool mem = (word >> j) & 1u;
-                const int lj = j == oslot ? lim : 3;
-                float p[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                  p[i] = (mem && i <= lj) ? fast_exp2(fmaf(__uint_as_float(r[4 * jj + i]), a.scale_log2, nref)) : 0.f;
-                  sum4[i] += p[i];
-                }
-                pk[16 * q2 + 2 * jj] = pack_bf16x2(p[0], p[1]);
-                pk[16 * q2 + 2 * jj + 1] = pack_bf16x2(p[2], p[3]);
-              }
+              pk[2 * jj] = pack_bf16x2(p[0], p[1]);
+              pk[2 * jj + 1] = pack_bf16x2(p[2], p[3]);
             }
-            tmem_st_32x32(s_addr + h2 * 32, pk);
+            tmem_st_32x16(s_addr + q8 * 16, pk);
           }
-          const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
-          l += sum;
+          l += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
           tmem_st_wait();
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&bar->p_full[sb]);
         }
         if (!alive) break;
-        // ---- epilogue of (tile, head): O / l -> bf16 row, log-sum-exp
-        if (!mbar_wait(&bar->o_full, static_cast<unsigned>(hp) & 1u, a.ctl)) {
+        // ---- epilogue of (tile, head): merge the two groups' (m, l, O), O / l -> bf16, lse.
+        // The exchange buffer is written once per pass: a warp posts again only after its partner
+        // has arrived on o_free below, which it does after reading.
+        xchg[(grp * 2 + 0) * 32 + lane] = m_ref;
+        xchg[(grp * 2 + 1) * 32 + lane] = l;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar->pair[quad]);
+        if (!mbar_wait_suspend(&bar->pair[quad], static_cast<unsigned>(hp) & 1u, a.ctl) ||
+            !mbar_wait_suspend(&bar->o_full, static_cast<unsigned>(hp) & 1u, a.ctl)) {
           alive = false;
           break;
         }
+        const float m0 = xchg[0 * 32 + lane], l0 = xchg[1 * 32 + lane];
+        const float m1 = xchg[2 * 32 + lane], l1 = xchg[3 * 32 + lane];
         tc_fence_after();
-        const float inv = l > 0.f ? 1.f / l : 0.f;
+        const float M = fmaxf(m0, m1);
+        const float f0 = m0 == -INFINITY ? 0.f : fast_exp2(m0 - M);
+        const float f1 = m1 == -INFINITY ? 0.f : fast_exp2(m1 - M);
+        const float lt = l0 * f0 + l1 * f1;
+        const float inv = lt > 0.f ? 1.f / lt : 0.f;
+        const float w0 = f0 * inv, w1 = f1 * inv;
+        // an accumulator with no chunk in this pass (nch == 1: group 1) holds stale values: not read
+        const bool use1 = nch > 1;
         const long long orow = (static_cast<long long>(b) * a.Tq + t0 + t) * a.Hq + g * kGrp + hh;
-        uint4* op = reinterpret_cast<uint4*>(a.out + orow * kD);
+        uint4* op = reinterpret_cast<uint4*>(a.out + orow * kD + grp * 64);
+        const uint32_t oc0 = tmem + lane_addr + kOCol + grp * 64;      // this warp's 64 columns of O[0]
+        const uint32_t oc1 = oc0 + kD;                                 // ... and of O[1]
 #pragma unroll
-        for (int p4 = 0; p4 < 4; ++p4) {
-          uint32_t r[32];
-          tmem_ld_32x32(o_addr + p4 * 32, r);
+        for (int p2 = 0; p2 < 2; ++p2) {
+          uint32_t x0[32], x1[32];
+          tmem_ld_32x32(oc0 + p2 * 32, x0);
+          if (use1) tmem_ld_32x32(oc1 + p2 * 32, x1);
           tmem_ld_wait();
           if (vrow) {
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-              uint4 v;
-              v.x = pack_bf16x2(__uint_as_float(r[8 * i + 0]) * inv, __uint_as_float(r[8 * i + 1]) * inv);
-              v.y = pack_bf16x2(__uint_as_float(r[8 * i + 2]) * inv, __uint_as_float(r[8 * i + 3]) * inv);
-              v.z = pack_bf16x2(__uint_as_float(r[8 * i + 4]) * inv, __uint_as_float(r[8 * i + 5]) * inv);
-              v.w = pack_bf16x2(__uint_as_float(r[8 * i + 6]) * inv, __uint_as_float(r[8 * i + 7]) * inv);
-              op[p4 * 4 + i] = v;
+              float v[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                v[e] = __uint_as_float(x0[8 * i + e]) * w0 + (use1 ? __uint_as_float(x1[8 * i + e]) * w1 : 0.f);
+              op[p2 * 4 + i] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                                          pack_bf16x2(v[6], v[7]));
             }
           }
         }
-        if (vrow && a.lse) a.lse[orow] = l > 0.f ? (m_ref + __log2f(l)) * kLn2 : -INFINITY;
+        if (grp == 0 && vrow && a.lse) a.lse[orow] = lt > 0.f ? (M + __log2f(lt)) * kLn2 : -INFINITY;
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar->o_free);
       }
     }
+  }
   }
   tc_fence_before();
   __syncthreads();
@@ -646,8 +704,10 @@ bool attn_tc_supported(int Hq, int Hkv, int D, int k_blocks) {
   return D == kD && (Hkv == 1 || Hkv == 2) && Hq == kGrp * Hkv && k_blocks >= 1 && k_blocks <= 1024;
 }
 
+// Per tile: the count, the union entries (16 k + 16 at most) and one record per chunk of 16 entries.
 size_t attn_tc_tile_bytes(int k_blocks) {
-  return static_cast<size_t>(kTQ * k_blocks + kTQ) * sizeof(uint2) + sizeof(int);
+  return static_cast<size_t>(kTQ * k_blocks + kTQ) * sizeof(uint2) + static_cast<size_t>(k_blocks + 1) * sizeof(ChunkInfo) +
+         sizeof(int);
 }
 
 cudaError_t launch_attn_prefill_tc(const DeviceInfo* di, const void* q, const void* k, const void* v,
@@ -657,13 +717,17 @@ cudaError_t launch_attn_prefill_tc(const DeviceInfo* di, const void* q, const vo
   const int tpb = (Tq + kTQ - 1) / kTQ;
   const long long ntiles = static_cast<long long>(B) * tpb;
   const int cap = kTQ * k_blocks + kTQ;
+  const int capc = k_blocks + 1;   // chunks of 16 entries
   const size_t per_tile = attn_tc_tile_bytes(k_blocks);
-  const long long fit = static_cast<long long>((ws_bytes > 256 ? ws_bytes - 256 : 0) / per_tile);
+  const long long fit = static_cast<long long>((ws_bytes > 512 ? ws_bytes - 512 : 0) / per_tile);
   if (fit < 1 || ntiles > 0x7fffffffLL) return cudaErrorInvalidValue;
   const int R = static_cast<int>(std::min<long long>(ntiles, fit));
-  // layout: cnt[R] (256-byte aligned), then ent[R][cap]
+  // layout: cnt[R] (256-byte aligned), ent[R][cap], rec[R][capc] (256-byte aligned)
   int* cnt = static_cast<int*>(ws);
-  uint2* ent = reinterpret_cast<uint2*>(static_cast<uint8_t*>(ws) + ((static_cast<size_t>(R) * 4 + 255) & ~size_t(255)));
+  const size_t ent_off = (static_cast<size_t>(R) * 4 + 255) & ~size_t(255);
+  uint2* ent = reinterpret_cast<uint2*>(static_cast<uint8_t*>(ws) + ent_off);
+  const size_t rec_off = (ent_off + static_cast<size_t>(R) * cap * sizeof(uint2) + 255) & ~size_t(255);
+  ChunkInfo* recs = reinterpret_cast<ChunkInfo*>(static_cast<uint8_t*>(ws) + rec_off);
   // K and V are mapped only up to the call's last query position: a tile's last own block can
   // reach past it, and those rows then read as zeros (masked for every row; a zero times a zero
   // probability keeps the product finite whatever the buffer holds there).
@@ -681,8 +745,18 @@ cudaError_t launch_attn_prefill_tc(const DeviceInfo* di, const void* q, const vo
     cudaFuncSetAttribute(sparse_attn_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   });
   if (usmem > 160 * 1024) return cudaErrorInvalidValue;
+  // the register split inside the kernel needs exactly kLaunchRegs registers per thread at launch
+  static int regs_ok[64][2];   // 0 unknown, 1 ok, -1 refused
+  int& rk = regs_ok[di->device & 63][Hkv - 1];
+  if (rk == 0) {
+    cudaFuncAttributes fa{};
+    const cudaError_t e = Hkv == 1 ? cudaFuncGetAttributes(&fa, sparse_attn_tc_kernel<1>)
+                                   : cudaFuncGetAttributes(&fa, sparse_attn_tc_kernel<2>);
+    rk = (e == cudaSuccess && fa.numRegs == kLaunchRegs && fa.maxThreadsPerBlock >= kThreads) ? 1 : -1;
+  }
+  if (rk != 1) return cudaErrorInvalidConfiguration;
   TcArgs ta{};
-  ta.ent = ent;
+  ta.recs = recs;
   ta.cnt = cnt;
   ta.out = static_cast<uint16_t*>(out);
   ta.lse = lse;
@@ -691,14 +765,14 @@ cudaError_t launch_attn_prefill_tc(const DeviceInfo* di, const void* q, const vo
   ta.Tq = Tq;
   ta.Hq = Hq;
   ta.Hkv = Hkv;
-  ta.cap = cap;
+  ta.capc = capc;
   ta.tpb = tpb;
   ta.scale_log2 = scale * 1.4426950408889634f;
   ta.ctl = kernel_ctl(di);
   for (long long t0 = 0; t0 < ntiles; t0 += R) {
     const int nt = static_cast<int>(std::min<long long>(R, ntiles - t0));
     tile_union_kernel<<<nt, 512, usmem, s>>>(idx, Tq, k_blocks, q_pos0, static_cast<int>(t0), tpb, n2, ent, cnt, cap,
-                                             ta.ctl);
+                                             recs, capc, ta.ctl);
     cudaError_t e = cudaPeekAtLastError();
     if (e != cudaSuccess) return e;
     ta.tile0 = static_cast<int>(t0);

@@ -482,7 +482,9 @@ def prefill_host(q, k, v, qi, ki, *, topk: int, device="cuda", out=None, q_pos0:
         bufs["kp"] = torch.empty(ki.shape[0], ki.shape[1] // 4, ki.shape[2], dtype=ki.dtype, device=dev)
     # row chunks (one sequence only: the rows of a chunk are then contiguous in every tensor)
     n = max(1, min(chunks, Tq)) if B == 1 else 1
-    bounds = [(Tq * c) // n for c in range(n + 1)]
+    # chunk bounds on multiples of 16 rows: the query-tile attention groups rows 16 at a time from a
+    # call's first row, so aligned chunks make the same tiles (and the same bits) as one call
+    bounds = [0] + [((Tq * c) // n) // 16 * 16 for c in range(1, n)] + [Tq]
     # selection chunks: query rows [slo, shi), whose blocks lie below key position q_pos0 + shi; the
     # pooled keys of a chunk start on a whole block (row bounds in multiples of 4 when q_pos0 is)
     ns = max(1, min(sel_chunks, Tq // 4)) if (B == 1 and q_pos0 % 4 == 0 and Tk == q_pos0 + Tq) else 1

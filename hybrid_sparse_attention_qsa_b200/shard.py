@@ -108,6 +108,8 @@ class ShardedPrefill:
         rows = max(b - a for a, b in self.ranges)
         ws = Q.qsa_workspace_size(Q.QSA_OP_SELECT_TOPK, B, rows, T // blk, topk, Hq, D)
         self.ws = torch.empty(ws, dtype=torch.uint8, device=dev)
+        aws = Q.qsa_workspace_size(Q.QSA_OP_SPARSE_ATTN_PREFILL, B, rows, 0, topk, Hq, D)
+        self.attn_ws = torch.empty(max(aws, 16), dtype=torch.uint8, device=dev)
         self.idx = [torch.empty(B, b - a, topk, dtype=torch.int32, device=dev) for a, b in self.ranges]
         self.out = [torch.empty(B, b - a, Hq, D, dtype=torch.bfloat16, device=dev) for a, b in self.ranges]
         self.lse = [torch.empty(B, b - a, Hq, dtype=torch.float32, device=dev) for a, b in self.ranges]
@@ -132,7 +134,7 @@ class ShardedPrefill:
             if events:
                 events[2 * i].record()
             Q.qsa_sparse_attn_prefill(q[i], self.kfull, self.vfull, self.idx[i], q_pos0=a, out=self.out[i],
-                                      lse=self.lse[i])
+                                      lse=self.lse[i], workspace=self.attn_ws)
             if events:
                 events[2 * i + 1].record()
         return self.out, self.lse, self.idx

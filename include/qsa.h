@@ -250,7 +250,7 @@ QSA_API qsa_status_t qsa_sparse_attn_prefill(const void* q, const void* k, const
  * qsa_sparse_attn_prefill with a workspace: the same arguments, result and errors, plus `workspace`
  * (caller-owned device memory, 16-byte aligned) of ws_bytes.
  * When D = 128, Hq = 8 * Hkv (groups of 8 query heads), k_blocks <= 1024 and the workspace holds at
- * least one tile (256 + 8 * (16 * k_blocks + 16) + 4 bytes; qsa_workspace_size(
+ * least one tile (512 + 8 * (16 * k_blocks + 16) + 128 * (k_blocks + 1) + 4 bytes; qsa_workspace_size(
  * QSA_OP_SPARSE_ATTN_PREFILL, B, Tq, 0, k_blocks, Hq, D, 0) gives room for up to 4096 tiles), the
  * rows are processed in tiles of 16 consecutive query rows on tcgen05 tensor cores: a tile attends
  * over the union of its rows' listed blocks and own blocks, gathered once per tile, and each row

@@ -270,14 +270,21 @@ def test_whole_layer_with_yarn_rope():
     print("yarn", st)
 
 
-def test_chunked_prefill_matches_full_prefill():
-    T, k, q0 = 2500, 64, 1234
+@pytest.mark.parametrize("q0", [1234, 1232])
+def test_chunked_prefill_matches_full_prefill(q0):
+    # The lists are the same bit for bit.  The query-tile attention groups rows 16 at a time from the
+    # call's first row: with q0 a multiple of 16 the chunk's tiles are the full call's tiles and the
+    # outputs are bit-identical; otherwise only the fp32 summation order differs.
+    T, k = 2500, 64
     x = _small_prefill(T, 16, 2, 4, 55)
     full = Q.prefill(x["q"], x["k"], x["v"], x["qi"], x["ki"], topk=k)
     part = Q.prefill(x["q"][:, q0:].contiguous(), x["k"], x["v"], x["qi"][:, q0:].contiguous(), x["ki"], topk=k,
                      q_pos0=q0)
     assert torch.equal(full["idx"][:, q0:], part["idx"])
-    assert torch.equal(full["out"][:, q0:], part["out"])
+    if q0 % 16 == 0:
+        assert torch.equal(full["out"][:, q0:], part["out"])
+    else:
+        P.assert_outputs_close(I.bits(full["out"][:, q0:]), I.bits(part["out"]))
 
 
 def test_unselected_tokens_poisoned_with_nan_do_not_matter():
