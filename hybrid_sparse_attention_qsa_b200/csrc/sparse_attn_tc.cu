@@ -13,12 +13,12 @@
 // selected pairs -- cheap on tcgen05.  The result is the same exact attention: a masked entry
 // contributes exp(-inf) = 0, and the softmax runs in fp32 over exactly the selected tokens.
 //
-// tile_union_kernel (one CTA per tile): keys (block << 4 | row) of the 16 index lists are sorted
-// (bitonic; ascending lists enter as sorted runs so only the merge stages run), the tile's own
-// blocks (one per row, always attended) are merged in, and equal blocks are folded into one entry
-// (block, 16-bit mask of the rows that attend it), ascending by block.  Entries outside a row's
-// causal range are skipped and recorded in the device status (-1 and the own block are skipped
-// silently).
+// tile_union_kernel (one CTA per tile): every listed block of the 16 rows, and each row's own block,
+// sets the row's bit in the block's 16-bit mask in a shared-memory bitmap (windows of 16384 blocks);
+// the blocks with a non-zero mask, ascending, are the union, written as (block, row mask) entries
+// and as one 128-byte record per chunk of 16 entries (block ids, per-row member bits, per-row own
+// slot) for the attention kernel.  Entries outside a row's causal range are skipped and recorded in
+// the device status (-1 and the own block are skipped silently); list order does not matter.
 //
 // sparse_attn_tc_kernel (persistent, one CTA per SM), per (tile, KV head):
 //   warps 0-7 producers: warp 0 loads the Q tile (two 128-byte-swizzled TMA boxes of [16 rows]
@@ -115,151 +115,119 @@ __device__ __forceinline__ float fast_exp2(float x) {
 }
 
 // ---------------------------------------------------------------------------- tile unions
-__global__ void __launch_bounds__(512) tile_union_kernel(const int32_t* __restrict__ idx, int Tq, int kb,
-                                                         long long q_pos0, int tile0, int tpb, int n2,
-                                                         uint2* __restrict__ ent, int* __restrict__ cnt, int cap,
-                                                         ChunkInfo* __restrict__ recs, int capc, KernelCtl ctl) {
-  extern __shared__ uint32_t ukeys[];
-  uint32_t* keys = ukeys;                 // [n2]
-  uint32_t* merged = keys + n2;           // [16 * kb + 16]
-  __shared__ int s_flags[2];
-  __shared__ int s_scan[17];
-  const int tid = threadIdx.x;
+constexpr int kUnionThreads = 512;
+constexpr int kWin = 16384;                 // blocks per window of the union bitmap
+constexpr int kMaxListPerThread = 32;       // 16 rows x k_blocks <= 16384 entries -> 32 per thread
+
+// One CTA per tile.  Every listed block of the tile's rows (and each row's own block) ORs the row's
+// bit into the block's 16-bit mask in a shared-memory bitmap; the blocks whose mask is non-zero,
+// ascending, are the union.  The block range is walked in windows of kWin blocks.
+__global__ void __launch_bounds__(kUnionThreads) tile_union_kernel(const int32_t* __restrict__ idx, int Tq, int kb,
+                                                                  long long q_pos0, int tile0, int tpb,
+                                                                  uint2* __restrict__ ent, int* __restrict__ cnt,
+                                                                  int cap, ChunkInfo* __restrict__ recs, int capc,
+                                                                  KernelCtl ctl) {
+  extern __shared__ uint32_t umask[];       // [kWin] row masks of the window's blocks, then the union
+  uint2* sent = reinterpret_cast<uint2*>(umask + kWin);   // [cap] the union, for the chunk records
+  __shared__ int s_scan[kUnionThreads / 32 + 1];
+  __shared__ int s_bad;
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const int tl = blockIdx.x;
   const int tile = tile0 + tl;
   const int b = tile / tpb, t0 = (tile % tpb) * kTQ;
+  const int nrows = min(kTQ, Tq - t0);
   const int nlist = kTQ * kb;
-  const bool pow2 = (kb & (kb - 1)) == 0;
-  if (tid < 2) s_flags[tid] = 0;
-  __syncthreads();
-  bool bad = false, unsorted = false;
-  for (int e = tid; e < n2; e += blockDim.x) {
-    uint32_t key = 0xFFFFFFFFu;
+  if (tid == 0) s_bad = 0;
+  // this thread's entries, as (block << 4 | row), or ~0 when skipped
+  uint32_t key[kMaxListPerThread];
+  bool bad = false;
+#pragma unroll
+  for (int i = 0; i < kMaxListPerThread; ++i) {
+    const int e = tid + i * kUnionThreads;
+    key[i] = 0xFFFFFFFFu;
     if (e < nlist) {
       const int r = e / kb;
-      int j = e - r * kb;
-      // with power-of-two lists the odd lists enter reversed, so the runs alternate direction
-      if (pow2 && (r & 1)) j = kb - 1 - j;
       const int row = t0 + r;
       if (row < Tq) {
-        const long long rowg = static_cast<long long>(b) * Tq + row;
-        const int x = idx[rowg * kb + j];
+        const int x = idx[(static_cast<long long>(b) * Tq + row) * kb + (e - r * kb)];
         const long long own = (q_pos0 + row) >> 2;
-        if (x >= 0 && x < own) {
-          key = (static_cast<uint32_t>(x) << 4) | static_cast<uint32_t>(r);
-        } else if (x != -1 && x != own) {
+        if (x >= 0 && x < own)
+          key[i] = (static_cast<uint32_t>(x) << 4) | static_cast<uint32_t>(r);
+        else if (x != -1 && x != own)
           bad = true;
-        }
-        // the source list must be ascending with skipped entries last: check the pair (j, j + 1)
-        if (j + 1 < kb) {
-          const int xn = idx[rowg * kb + j + 1];
-          const bool vn = xn >= 0 && xn < own;
-          const uint32_t kn = vn ? ((static_cast<uint32_t>(xn) << 4) | static_cast<uint32_t>(r)) : 0xFFFFFFFFu;
-          if (kn < key) unsorted = true;
-        }
       }
     }
-    keys[e] = key;
   }
-  if (bad) s_flags[0] = 1;
-  if (unsorted) s_flags[1] = 1;
+  const long long own_first = (q_pos0 + t0) >> 2;
+  const long long own_last = (q_pos0 + t0 + nrows - 1) >> 2;
+  const int nblk = static_cast<int>(own_last + 1);   // every attended block lies below this
   __syncthreads();
-  if (tid == 0 && s_flags[0]) record_status(ctl, kStBadArg);
-  // bitonic sort of keys[0 .. n2) ascending; sorted runs of kb (alternating) skip the first stages
-  const int kstart = (pow2 && !s_flags[1] && kb >= 2) ? 2 * kb : 2;
-  for (int k2 = kstart; k2 <= n2; k2 <<= 1) {
-    for (int j2 = k2 >> 1; j2 > 0; j2 >>= 1) {
-      for (int i = tid; i < n2; i += blockDim.x) {
-        const int p = i ^ j2;
-        if (p > i) {
-          const uint32_t a = keys[i], c = keys[p];
-          const bool asc = (i & k2) == 0;
-          if ((a > c) == asc) {
-            keys[i] = c;
-            keys[p] = a;
-          }
-        }
-      }
-      __syncthreads();
-    }
-  }
-  // valid keys: those below 0xFFFFFFFF (a prefix of the sorted array)
-  int lo = 0, hi = n2;
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if (keys[mid] == 0xFFFFFFFFu) hi = mid; else lo = mid + 1;
-  }
-  const int nv = lo;
-  // the own block of every row of the tile, keys ascending in the row
-  const int nown = min(kTQ, Tq - t0);
-  uint32_t okey[kTQ];
-#pragma unroll
-  for (int r = 0; r < kTQ; ++r)
-    okey[r] = r < nown ? (static_cast<uint32_t>((q_pos0 + t0 + r) >> 2) << 4) | static_cast<uint32_t>(r) : 0xFFFFFFFFu;
-  for (int i = tid; i < nv; i += blockDim.x) {
-    const uint32_t key = keys[i];
-    int c = 0;
-#pragma unroll
-    for (int r = 0; r < kTQ; ++r) c += okey[r] < key ? 1 : 0;
-    merged[i + c] = key;
-  }
-  if (tid < nown) {
-    const uint32_t key = okey[tid];
-    int a = 0, z = nv;
-    while (a < z) {
-      const int mid = (a + z) >> 1;
-      if (keys[mid] < key) a = mid + 1; else z = mid;
-    }
-    merged[tid + a] = key;
-  }
-  __syncthreads();
-  // fold equal blocks: one entry per run, the rows of the run OR-ed into its mask
-  const int N = nv + nown;
-  const int per = (N + blockDim.x - 1) / blockDim.x;
-  const int i0 = min(N, tid * per), i1 = min(N, i0 + per);
-  int heads = 0;
-  for (int i = i0; i < i1; ++i)
-    if (i == 0 || (merged[i] >> 4) != (merged[i - 1] >> 4)) ++heads;
-  // block-wide exclusive scan of the head counts
-  const int lane = tid & 31, w = tid >> 5;
-  int incl = heads;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int v = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += v;
-  }
-  if (lane == 31) s_scan[w] = incl;
-  __syncthreads();
-  if (tid == 0) {
-    int run = 0;
-    for (int q = 0; q < static_cast<int>(blockDim.x >> 5); ++q) {
-      const int v = s_scan[q];
-      s_scan[q] = run;
-      run += v;
-    }
-    s_scan[16] = run;
-  }
-  __syncthreads();
-  int u = s_scan[w] + incl - heads;
+  if (bad) s_bad = 1;
   uint2* te = ent + static_cast<long long>(tl) * cap;
-  for (int i = i0; i < i1; ++i) {
-    const uint32_t blk = merged[i] >> 4;
-    if (i == 0 || blk != (merged[i - 1] >> 4)) {
-      uint32_t mask = 0;
-      for (int j = i; j < N && (merged[j] >> 4) == blk; ++j) mask |= 1u << (merged[j] & 15u);
-      te[u++] = make_uint2(blk, mask);
+  int total = 0;
+  for (int w0 = 0; w0 < nblk; w0 += kWin) {
+    const int wn = min(kWin, nblk - w0);
+    for (int i = tid; i < wn; i += kUnionThreads) umask[i] = 0u;
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < kMaxListPerThread; ++i) {
+      const uint32_t x = key[i] >> 4;
+      if (key[i] != 0xFFFFFFFFu && x >= static_cast<uint32_t>(w0) && x < static_cast<uint32_t>(w0 + wn))
+        atomicOr(&umask[x - w0], 1u << (key[i] & 15u));
     }
+    if (tid < nrows) {   // the rows' own blocks
+      const long long o = (q_pos0 + t0 + tid) >> 2;
+      if (o >= w0 && o < w0 + wn) atomicOr(&umask[o - w0], 1u << tid);
+    }
+    __syncthreads();
+    // ascending compaction: thread tid scans its contiguous slice of the window
+    const int per = (wn + kUnionThreads - 1) / kUnionThreads;
+    const int i0 = min(wn, tid * per), i1 = min(wn, i0 + per);
+    int mine = 0;
+    for (int i = i0; i < i1; ++i) mine += umask[i] != 0u;
+    int incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) s_scan[w] = incl;
+    __syncthreads();
+    if (tid == 0) {
+      int run = 0;
+      for (int q = 0; q < kUnionThreads / 32; ++q) {
+        const int v = s_scan[q];
+        s_scan[q] = run;
+        run += v;
+      }
+      s_scan[kUnionThreads / 32] = run;
+    }
+    __syncthreads();
+    int u = total + s_scan[w] + incl - mine;
+    for (int i = i0; i < i1; ++i) {
+      const uint32_t m = umask[i];
+      if (m) {
+        const uint2 e = make_uint2(static_cast<uint32_t>(w0 + i), m);
+        te[u] = e;
+        sent[u++] = e;
+      }
+    }
+    total += s_scan[kUnionThreads / 32];
+    __syncthreads();   // the window is reused
   }
-  if (tid == 0) cnt[tl] = s_scan[16];
-  // the chunk records: one warp per chunk of 16 entries (the entries written above are visible to
-  // the whole block after the barrier)
+  (void)own_first;
+  if (tid == 0) {
+    cnt[tl] = total;
+    if (s_bad) record_status(ctl, kStBadArg);
+  }
+  // the chunk records: one warp per chunk of 16 entries (from the shared-memory copy of the union)
   __syncthreads();
-  const int nu = s_scan[16];
+  const int nu = total;
   const int nch = max(1, (nu + kCB - 1) / kCB);
   ChunkInfo* tr = recs + static_cast<long long>(tl) * capc;
-  for (int c = w; c < nch; c += blockDim.x >> 5) {
+  for (int c = w; c < nch; c += kUnionThreads >> 5) {
     const int uu = c * kCB + lane;
-    const uint2 e = te[min(uu, max(nu - 1, 0))];
+    const uint2 e = sent[min(uu, max(nu - 1, 0))];
     const uint32_t mask = (lane < kCB && uu < nu) ? e.y : 0u;
     uint32_t myw = 0;
     int myo = -1;
@@ -692,12 +660,6 @@ bool make_map4(CUtensorMap* m, const void* base, unsigned long long d1, unsigned
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int next_pow2(int x) {
-  int p = 1;
-  while (p < x) p <<= 1;
-  return p;
-}
-
 }  // namespace
 
 bool attn_tc_supported(int Hq, int Hkv, int D, int k_blocks) {
@@ -736,15 +698,16 @@ cudaError_t launch_attn_prefill_tc(const DeviceInfo* di, const void* q, const vo
   if (!make_map4(&qm, q, Hq, Tq, B, kGrp, kTQ) || !make_map4(&km, k, Hkv, tk_used, B, 1, 4, static_cast<unsigned long long>(Tk)) ||
       !make_map4(&vm, v, Hkv, tk_used, B, 1, 4, static_cast<unsigned long long>(Tk)))
     return cudaErrorInvalidValue;
-  const int n2 = next_pow2(std::max(kTQ * k_blocks, 32));
-  const size_t usmem = static_cast<size_t>(n2) * 4 + static_cast<size_t>(cap) * 4;
+  const size_t usmem = static_cast<size_t>(kWin) * 4 + static_cast<size_t>(cap) * sizeof(uint2);
+  if (kTQ * k_blocks > kMaxListPerThread * kUnionThreads) return cudaErrorInvalidValue;
   static std::once_flag once[64];
   std::call_once(once[di->device & 63], [] {
-    cudaFuncSetAttribute(tile_union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024);
+    cudaFuncSetAttribute(tile_union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         kWin * 4 + (kTQ * 1024 + kTQ) * static_cast<int>(sizeof(uint2)));
     cudaFuncSetAttribute(sparse_attn_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     cudaFuncSetAttribute(sparse_attn_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   });
-  if (usmem > 160 * 1024) return cudaErrorInvalidValue;
+
   // the register split inside the kernel needs exactly kLaunchRegs registers per thread at launch
   static int regs_ok[64][2];   // 0 unknown, 1 ok, -1 refused
   int& rk = regs_ok[di->device & 63][Hkv - 1];
@@ -771,8 +734,8 @@ cudaError_t launch_attn_prefill_tc(const DeviceInfo* di, const void* q, const vo
   ta.ctl = kernel_ctl(di);
   for (long long t0 = 0; t0 < ntiles; t0 += R) {
     const int nt = static_cast<int>(std::min<long long>(R, ntiles - t0));
-    tile_union_kernel<<<nt, 512, usmem, s>>>(idx, Tq, k_blocks, q_pos0, static_cast<int>(t0), tpb, n2, ent, cnt, cap,
-                                             recs, capc, ta.ctl);
+    tile_union_kernel<<<nt, kUnionThreads, usmem, s>>>(idx, Tq, k_blocks, q_pos0, static_cast<int>(t0), tpb, ent, cnt,
+                                                       cap, recs, capc, ta.ctl);
     cudaError_t e = cudaPeekAtLastError();
     if (e != cudaSuccess) return e;
     ta.tile0 = static_cast<int>(t0);

@@ -286,8 +286,9 @@ def qsa_sparse_attn_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, i
     """q [B, Tq, Hq, D], k/v [B, Tk, Hkv, D], idx [B, Tq, kb] -> (out [B, Tq, Hq, D], lse [B, Tq, Hq]).
 
     With ``tiles`` (default) the call goes through qsa_sparse_attn_prefill_ws with ``workspace``
-    (allocated here when omitted): query tiles on tcgen05 where the shape allows, else row by row.
-    ``tiles=False`` calls qsa_sparse_attn_prefill (row by row, no workspace)."""
+    (allocated here when omitted), which runs the path qsa_set_attn_options chose (automatic: row by
+    row; QSA_ATTN_TILES: query tiles on tcgen05 where the shape allows).  ``tiles=False`` calls
+    qsa_sparse_attn_prefill (row by row, no workspace)."""
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _need(t, torch.bfloat16, n)
     _need(idx, torch.int32, "idx")
@@ -315,8 +316,8 @@ def qsa_sparse_attn_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, i
 
 
 def qsa_set_attn_options(path: int = QSA_ATTN_AUTO) -> None:
-    """Prefill attention of qsa_sparse_attn_prefill_ws for later calls: QSA_ATTN_AUTO (query tiles
-    where supported), QSA_ATTN_ROWS or QSA_ATTN_TILES."""
+    """Prefill attention of qsa_sparse_attn_prefill_ws for later calls: QSA_ATTN_AUTO (row by row),
+    QSA_ATTN_ROWS or QSA_ATTN_TILES."""
     _check(lib().qsa_set_attn_options(path), "qsa_set_attn_options")
 
 

@@ -249,7 +249,9 @@ QSA_API qsa_status_t qsa_sparse_attn_prefill(const void* q, const void* k, const
 /*
  * qsa_sparse_attn_prefill with a workspace: the same arguments, result and errors, plus `workspace`
  * (caller-owned device memory, 16-byte aligned) of ws_bytes.
- * When D = 128, Hq = 8 * Hkv (groups of 8 query heads), k_blocks <= 1024 and the workspace holds at
+ * With the query-tile path chosen (qsa_set_attn_options(2); the automatic choice is row by row,
+ * the faster of the two on workloads whose consecutive rows share little of their selections), and
+ * when D = 128, Hq = 8 * Hkv (groups of 8 query heads), k_blocks <= 1024 and the workspace holds at
  * least one tile (512 + 8 * (16 * k_blocks + 16) + 128 * (k_blocks + 1) + 4 bytes; qsa_workspace_size(
  * QSA_OP_SPARSE_ATTN_PREFILL, B, Tq, 0, k_blocks, Hq, D, 0) gives room for up to 4096 tiles), the
  * rows are processed in tiles of 16 consecutive query rows on tcgen05 tensor cores: a tile attends
@@ -272,9 +274,9 @@ QSA_API qsa_status_t qsa_sparse_attn_prefill_ws(const void* q, const void* k, co
 
 /*
  * Chooses the prefill attention of qsa_sparse_attn_prefill_ws for all later calls from this
- * process: 0 = automatic (query tiles where supported), 1 = row by row, 2 = query tiles
- * (UNSUPPORTED for other shapes, WORKSPACE_TOO_SMALL without room for one tile).  A testing and
- * tuning knob.  Errors: INVALID_ARGUMENT (path outside 0..2).
+ * process: 0 = automatic (row by row), 1 = row by row, 2 = query tiles (UNSUPPORTED for other
+ * shapes, WORKSPACE_TOO_SMALL without room for one tile).  Errors: INVALID_ARGUMENT (path outside
+ * 0..2).
  */
 QSA_API qsa_status_t qsa_set_attn_options(int path);
 
