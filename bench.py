@@ -422,6 +422,46 @@ def run_qsa(args):
     else:   # per chunk: pooling, the selection's kernels, attention (NCCL's own kernels not counted)
         launches = sum(2 + select_launches(w.with_(T=b - a), ws_bytes) for a, b in my_ranges) * args.steps
 
+    # the query-tile attention (tcgen05 over the union of 16 rows' blocks) on the same lists, beside
+    # the row-by-row kernel the step uses (both are the library's own kernels)
+    tiles = None
+    if sp is None and not args.no_tiles:
+        try:
+            aws = torch.empty(Q.qsa_workspace_size(Q.qsa.QSA_OP_SPARSE_ATTN_PREFILL, w.B, w.T, 0, w.k, w.Hq, w.D),
+                              dtype=torch.uint8, device=dev)
+            Q.qsa.qsa_set_attn_options(Q.qsa.QSA_ATTN_TILES)
+            otile = torch.empty_like(out)
+            ltile = torch.empty_like(lse)
+            Q.qsa_sparse_attn_prefill(x["q"], x["k"], x["v"], idx, out=otile, lse=ltile, workspace=aws)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(3):
+                Q.qsa_sparse_attn_prefill(x["q"], x["k"], x["v"], idx, out=otile, lse=ltile, workspace=aws)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            Q.qsa.qsa_set_attn_options(Q.qsa.QSA_ATTN_AUTO)
+            assert Q.qsa_get_device_status() == 0
+            t_ms = e0.elapsed_time(e1) / 3
+            ntiles = w.B * ((w.T + 15) // 16)
+            held = min(ntiles, 4096)
+            cnt = aws[:held * 4].view(torch.int32).double()   # union sizes of the last range of tiles
+            ublk = float(cnt.mean())
+            gath = ublk * ntiles * w.Hkv * w.blk * w.D * 2 * 2          # K/V of every union block, per tile
+            # dense over the union: 128 rows x blk tokens x D, times 2 flop, for S and for PV
+            tflop = ublk * ntiles * w.Hkv * (128 * w.blk * w.D * 2 * 2) / 1e12
+            diff = (otile.float() - out.float()).abs()
+            tiles = {"kernel": "tile_union_kernel + sparse_attn_tc_kernel<%d>" % w.Hkv, "ms": t_ms,
+                     "rows_kernel_ms": ms_attn, "speedup_vs_rows": ms_attn / t_ms,
+                     "union_blocks_per_tile_mean": ublk, "union_over_sum_of_lists": ublk / (16 * (w.k + 1)),
+                     "gathered_bytes": gath, "gathered_bytes_rows_kernel": work["attn_bytes"],
+                     "tensor_tflops_dense_union": tflop / (t_ms / 1000),
+                     "frac_of_bf16_peak": tflop / (t_ms / 1000) / pk["bf16_tflops"],
+                     "max_abs_diff_vs_rows": float(diff.max()), "mean_abs_diff_vs_rows": float(diff.mean())}
+            del aws, otile, ltile
+        except Exception as exc:
+            Q.qsa.qsa_set_attn_options(Q.qsa.QSA_ATTN_AUTO)
+            tiles = {"unavailable": f"{type(exc).__name__}: {exc}"[:200]}
+
     # indexer alone (scores for all rows materialised once; untimed in the step above)
     idx_ms = None
     try:
@@ -688,6 +728,7 @@ def run_qsa(args):
             "e2e": e2e,
             "decode": decode,
             "dense_compare": dense,
+            "attention_query_tiles": tiles,
         }
         if not args.no_cpu_baseline and world == 1:
             dt, rows, cores = oracle_sample(I.WORKLOADS[args.workload], args.ref_rows)
@@ -714,6 +755,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-indexer", action="store_true", help="skip the stand-alone indexer timing (17 GB of scores)")
     ap.add_argument("--no-dense", action="store_true", help="skip timing dense causal attention on the same inputs")
+    ap.add_argument("--no-tiles", action="store_true", help="skip timing the query-tile attention beside the rows")
     ap.add_argument("--probe-l2-gather", action="store_true",
                     help="only measure the gather ceiling (bulk-copy and cp.async gathers of the attention's "
                          "chunks from L2 and HBM, with a sweep of issuing warps) and print it as one JSON line")
