@@ -161,6 +161,7 @@ static qsa_status_t resolve_rope(const qsa_rope_params_t* in, RopeParams* out) {
 qsa_status_t qsa_pool_block_keys_rope(const void* ki, void* kp, int B, int L, int Di, int blk,
                                       const qsa_rope_params_t* rope, int64_t pos0, int64_t ki_batch_stride,
                                       int64_t kp_batch_stride, void* stream) {
+  QSA_NVTX();
   if (B < 0 || L < 0 || Di < 2 || Di > 256 || (Di & 1) || pos0 < 0) return QSA_ERR_INVALID_ARGUMENT;
   if (ki_batch_stride < 0 || kp_batch_stride < 0) return QSA_ERR_INVALID_ARGUMENT;
   RopeParams rp;
@@ -177,12 +178,14 @@ qsa_status_t qsa_pool_block_keys_rope(const void* ki, void* kp, int B, int L, in
 
 qsa_status_t qsa_pool_block_keys(const void* ki, void* kp, int B, int L, int Di, int blk, float rope_theta,
                                  int64_t pos0, int64_t ki_batch_stride, int64_t kp_batch_stride, void* stream) {
+  QSA_NVTX();
   const qsa_rope_params_t rope{rope_theta > 0.f ? static_cast<double>(rope_theta) : 0.0, 1.0, 0.0, 1.0, 32.0, 0.0};
   return qsa_pool_block_keys_rope(ki, kp, B, L, Di, blk, &rope, pos0, ki_batch_stride, kp_batch_stride, stream);
 }
 
 qsa_status_t qsa_rope_index_queries_rope(const void* qi, void* qi_out, int B, int Tq, int Hi, int Di, int64_t q_pos0,
                                          const int32_t* seqlens, const qsa_rope_params_t* rope, void* stream) {
+  QSA_NVTX();
   RopeParams rp;
   if (B < 0 || Tq < 0 || Hi < 1 || Di < 2 || Di > 256 || (Di & 1) || q_pos0 < 0) return QSA_ERR_INVALID_ARGUMENT;
   if (resolve_rope(rope, &rp) != QSA_OK || !(rp.theta > 0.0)) return QSA_ERR_INVALID_ARGUMENT;
@@ -195,6 +198,7 @@ qsa_status_t qsa_rope_index_queries_rope(const void* qi, void* qi_out, int B, in
 
 qsa_status_t qsa_rope_index_queries(const void* qi, void* qi_out, int B, int Tq, int Hi, int Di, int64_t q_pos0,
                                     const int32_t* seqlens, float rope_theta, void* stream) {
+  QSA_NVTX();
   if (!(rope_theta > 0.f)) return QSA_ERR_INVALID_ARGUMENT;
   const qsa_rope_params_t rope{static_cast<double>(rope_theta), 1.0, 0.0, 1.0, 32.0, 0.0};
   return qsa_rope_index_queries_rope(qi, qi_out, B, Tq, Hi, Di, q_pos0, seqlens, &rope, stream);
@@ -216,6 +220,7 @@ static qsa_status_t check_score_args(const void* qi, const void* kp, const int32
 qsa_status_t qsa_index_score(const void* qi, const void* kp, const float* head_w, const int32_t* seqlens, int B,
                              int Tq, int NBk, int Hi, int Di, int blk, int64_t q_pos0, qsa_score_mode_t mode,
                              float* scores, int64_t ld_scores, void* stream) {
+  QSA_NVTX();
   qsa_status_t st = check_score_args(qi, kp, seqlens, B, Tq, NBk, Hi, Di, blk, q_pos0, mode);
   if (st != QSA_OK) return st;
   if (ld_scores < std::max(NBk, 1)) return QSA_ERR_INVALID_ARGUMENT;
@@ -234,6 +239,7 @@ qsa_status_t qsa_select_topk(const float* scores, int64_t ld_scores, const void*
                              const float* head_w, const int32_t* seqlens, int B, int Tq, int NBk, int Hi, int Di,
                              int blk, int64_t q_pos0, qsa_score_mode_t mode, int k, int32_t* idx, void* workspace,
                              size_t ws_bytes, void* stream) {
+  QSA_NVTX();
   if (k < 1 || B < 0 || Tq < 0 || NBk < 0 || q_pos0 < 0) return QSA_ERR_INVALID_ARGUMENT;
   if (blk != 4) return QSA_ERR_UNSUPPORTED;
   if (seqlens && Tq != 1) return QSA_ERR_INVALID_ARGUMENT;
@@ -377,6 +383,7 @@ qsa_status_t qsa_decode_select(const void* qi, void* kp, const void* ki, int64_t
                                const float* head_w, const int32_t* seqlens, int B, int NBk, int Hi, int Di, int blk,
                                qsa_score_mode_t mode, const qsa_rope_params_t* rope, int k, int32_t* idx,
                                void* workspace, size_t ws_bytes, void* stream) {
+  QSA_NVTX();
   if (k < 1 || B < 0 || NBk < 0 || ki_batch_stride < 0) return QSA_ERR_INVALID_ARGUMENT;
   if (blk != 4) return QSA_ERR_UNSUPPORTED;
   if (B == 0) return QSA_OK;
@@ -408,6 +415,7 @@ qsa_status_t qsa_decode_select(const void* qi, void* kp, const void* ki, int64_t
 qsa_status_t qsa_sparse_attn_prefill(const void* q, const void* k, const void* v, const int32_t* idx, int B, int Tq,
                                      int Tk, int Hq, int Hkv, int D, int k_blocks, int blk, int64_t q_pos0,
                                      float scale, void* out, float* lse, void* stream) {
+  QSA_NVTX();
   qsa_status_t st = check_attn_shape(Hq, Hkv, D, blk, k_blocks);
   if (st != QSA_OK) return st;
   if (B < 0 || Tq < 0 || Tk < 0 || q_pos0 < 0 || q_pos0 + Tq > Tk) return QSA_ERR_INVALID_ARGUMENT;
@@ -425,6 +433,7 @@ qsa_status_t qsa_sparse_attn_prefill_ws(const void* q, const void* k, const void
                                         int Tq, int Tk, int Hq, int Hkv, int D, int k_blocks, int blk,
                                         int64_t q_pos0, float scale, void* out, float* lse, void* workspace,
                                         size_t ws_bytes, void* stream) {
+  QSA_NVTX();
   qsa_status_t st = check_attn_shape(Hq, Hkv, D, blk, k_blocks);
   if (st != QSA_OK) return st;
   if (B < 0 || Tq < 0 || Tk < 0 || q_pos0 < 0 || q_pos0 + Tq > Tk) return QSA_ERR_INVALID_ARGUMENT;
@@ -473,6 +482,7 @@ qsa_status_t qsa_sparse_attn_decode(const void* q, const void* kcache, const voi
                                     const int32_t* idx, int B, int Lmax, int Hq, int Hkv, int D, int k_blocks, int blk,
                                     float scale, int num_splits, void* out, float* lse, void* workspace,
                                     size_t ws_bytes, void* stream) {
+  QSA_NVTX();
   qsa_status_t st = check_attn_shape(Hq, Hkv, D, blk, k_blocks);
   if (st != QSA_OK) return st;
   if (B < 0 || Lmax < 1 || num_splits < 0) return QSA_ERR_INVALID_ARGUMENT;

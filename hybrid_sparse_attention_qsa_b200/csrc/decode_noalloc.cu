@@ -40,6 +40,7 @@ extern "C" qsa_status_t qsa_sparse_attn_decode_noalloc(const void* q, const void
                                                        const int32_t* seqlens, const int32_t* idx, int B, int Lmax,
                                                        int Hq, int Hkv, int D, int k_blocks, int blk, float scale,
                                                        int num_splits, void* out, float* lse, void* stream) {
+  QSA_NVTX();
   if (Hq < 1 || Hkv < 1 || k_blocks < 0 || Hq % Hkv) return QSA_ERR_INVALID_ARGUMENT;
   if ((D != 128 && D != 256) || blk != 4 || Hkv > 2 || Hq / Hkv > 16) return QSA_ERR_UNSUPPORTED;
   if (B < 0 || Lmax < 1 || num_splits < 0) return QSA_ERR_INVALID_ARGUMENT;

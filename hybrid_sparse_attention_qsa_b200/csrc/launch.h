@@ -6,9 +6,20 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "common.cuh"
 
 namespace qsa {
+
+// An NVTX range around a C-ABI call (header-only NVTX v3: one pointer test when no tool listens).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+#define QSA_NVTX() ::qsa::NvtxRange qsa_nvtx_range_(__func__)
 
 struct DeviceInfo {
   int device;

@@ -204,6 +204,7 @@ using namespace qsa;
 extern "C" qsa_status_t qsa_probe_gather(const void* src, size_t src_bytes, int chunk_bytes, int method,
                                          int issuer_warps, int stages, int slots_per_warp, int iterations, int ctas,
                                          uint64_t seed, void* stream) {
+  QSA_NVTX();
   if (src == nullptr || (reinterpret_cast<uintptr_t>(src) & 15u) != 0) return QSA_ERR_INVALID_ARGUMENT;
   if (chunk_bytes < 16 || chunk_bytes > 16384 || chunk_bytes % 16 != 0) return QSA_ERR_INVALID_ARGUMENT;
   if (src_bytes < static_cast<size_t>(chunk_bytes)) return QSA_ERR_INVALID_ARGUMENT;

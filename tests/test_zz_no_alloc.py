@@ -63,7 +63,7 @@ def test_noalloc_decode_cluster_merge_twice():
 def test_noalloc_decode_partials_in_scratch_twice(B, splits):
     # 12 splits (more than a cluster merges) or 24 x 7 = 168 items (more than one per SM): the
     # partials go through the scratch array and the merge kernel
-    lens = [12000 - 997 * i for i in range(B)]
+    lens = [12000 - 11000 * i // B for i in range(B)]
     lens[-1] = 5
     x, kp, idx = _case(B, 12000, lens, 256, 72 + B)
     _twice_against_workspace_and_oracle(x, kp, idx, splits, 256, merge=2)
