@@ -11,4 +11,4 @@ from .qsa import (QSA_SELECT_AUTO, QSA_SELECT_FILTERED, QSA_SELECT_MATERIALISED,
                   qsa_pool_block_keys, qsa_rope_index_queries, qsa_select_topk, qsa_set_select_options,
                   qsa_set_wait_timeout_ns, qsa_sparse_attn_decode, qsa_sparse_attn_prefill,
                   qsa_sparse_attn_decode_noalloc, qsa_wait_timeout_selftest, qsa_workspace_size,
-                  qsa_set_attn_options, QSA_ATTN_AUTO, QSA_ATTN_ROWS, QSA_ATTN_TILES)
+                  qsa_set_attn_options, QSA_ATTN_AUTO, QSA_ATTN_ROWS, QSA_ATTN_TILES, qsa_check_canaries)

@@ -125,6 +125,7 @@ const char* qsa_status_string(qsa_status_t status) {
     case QSA_ERR_WORKSPACE_TOO_SMALL: return "QSA_ERR_WORKSPACE_TOO_SMALL";
     case QSA_ERR_CUDA: return "QSA_ERR_CUDA";
     case QSA_ERR_TIMEOUT: return "QSA_ERR_TIMEOUT";
+    case QSA_ERR_DEVICE_CHECK: return "QSA_ERR_DEVICE_CHECK";
   }
   return "QSA_ERR_UNKNOWN";
 }

@@ -11,7 +11,7 @@
 namespace qsa {
 
 // Status codes recorded on the device (same values as qsa_status_t).
-enum : unsigned { kStOk = 0, kStBadArg = 1, kStTimeout = 5 };
+enum : unsigned { kStOk = 0, kStBadArg = 1, kStTimeout = 5, kStDeviceCheck = 6 };
 
 // Passed by value to every kernel that waits or can see a bad input.
 struct KernelCtl {
@@ -22,6 +22,21 @@ struct KernelCtl {
 __device__ __forceinline__ void record_status(const KernelCtl& c, unsigned code) {
   atomicCAS(c.status, 0u, code);
 }
+
+// Device-side bounds checks of the debug build (compiled with -DQSA_DEBUG).  QSA_DCHECK(ctl, cond)
+// is true when cond holds; when it does not, the check records kStDeviceCheck in the status word
+// and is false, and the caller skips the access (a skipped copy still settles its bytes on the
+// barrier, so no wait is left hanging).  In the release build the macro is the constant true and
+// cond is not evaluated.
+#ifdef QSA_DEBUG
+__device__ __forceinline__ bool dcheck(const KernelCtl& c, bool ok) {
+  if (!ok) record_status(c, kStDeviceCheck);
+  return ok;
+}
+#define QSA_DCHECK(ctl, cond) (::qsa::dcheck((ctl), static_cast<bool>(cond)))
+#else
+#define QSA_DCHECK(ctl, cond) true
+#endif
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -42,6 +57,12 @@ __device__ __forceinline__ void fence_mbar_init() {
 }
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, unsigned bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+// Settles `bytes` of the barrier's expected transaction count without a copy (a copy the debug
+// build's bounds check skipped).
+__device__ __forceinline__ void mbar_complete_tx(uint64_t* bar, unsigned bytes) {
+  asm volatile("mbarrier.complete_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                : "memory");
 }
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {

@@ -105,6 +105,14 @@ struct AttnArgs {
   KernelCtl ctl;
 };
 
+#ifdef QSA_DEBUG
+// Rows of out / lse the launch writes (prefill: B * Tq; decode: B); the decode partials have one
+// row per item.
+__device__ __forceinline__ long long out_rows(const AttnArgs& a) {
+  return a.seqlens ? static_cast<long long>(a.B) : static_cast<long long>(a.B) * a.Tq;
+}
+#endif
+
 struct Item {
   const uint16_t* kbase;
   const uint16_t* vbase;
@@ -177,8 +185,12 @@ __device__ __forceinline__ void attn_helper(const AttnArgs& a, int h, uint8_t* r
       const long long tok0 = inf->tok0[slot];
       uint8_t* kd = ring + st * R::kStageBytes + slot * R::kPitch;
       uint8_t* vd = kd + R::kSlots * R::kPitch;
-      bulk_g2s(kd, inf->kbase + tok0 * HKV * D, ntok * tok_bytes, &full[st]);
-      bulk_g2s(vd, inf->vbase + tok0 * HKV * D, ntok * tok_bytes, &full[st]);
+      if (QSA_DCHECK(a.ctl, tok0 >= 0 && ntok <= kBlk && tok0 + ntok <= a.Tk)) {
+        bulk_g2s(kd, inf->kbase + tok0 * HKV * D, ntok * tok_bytes, &full[st]);
+        bulk_g2s(vd, inf->vbase + tok0 * HKV * D, ntok * tok_bytes, &full[st]);
+      } else {
+        mbar_complete_tx(&full[st], 2u * ntok * tok_bytes);
+      }
     }
     __syncwarp();
     if (++st == kStages) {
@@ -246,8 +258,12 @@ __device__ __forceinline__ void attn_producer(const AttnArgs& a, uint8_t* ring, 
     if (lane < n && lane % kIssuers_ == 0) {
       uint8_t* kd = ring + st * R::kStageBytes + lane * R::kPitch;
       uint8_t* vd = kd + R::kSlots * R::kPitch;
-      bulk_g2s(kd, it.kbase + tok0 * HKV * D, ntok * tok_bytes, &full[st]);
-      bulk_g2s(vd, it.vbase + tok0 * HKV * D, ntok * tok_bytes, &full[st]);
+      if (QSA_DCHECK(a.ctl, tok0 >= 0 && ntok <= kBlk && tok0 + ntok <= a.Tk)) {
+        bulk_g2s(kd, it.kbase + tok0 * HKV * D, ntok * tok_bytes, &full[st]);
+        bulk_g2s(vd, it.vbase + tok0 * HKV * D, ntok * tok_bytes, &full[st]);
+      } else {
+        mbar_complete_tx(&full[st], 2u * ntok * tok_bytes);
+      }
     }
     // drop the flushed entries from the pending list
     int rest0 = n + lane < 64 ? pend[n + lane] : 0;
@@ -617,16 +633,17 @@ __global__ void __launch_bounds__(Cfg<HKV>::kThreads, 1) sparse_attn_kernel(Attn
         const long long frow = it.partial ? it.qrow : it.orow;   // cluster mode: the sequence's row
         uint16_t* orow = a.out + (frow * a.Hq + g * group) * kD;
         const int chunks = group * kD / 8;   // 16-byte chunks of this KV head's output heads
-        for (int c = lane; c < chunks; c += 32)
+        const bool row_ok = QSA_DCHECK(a.ctl, frow >= 0 && frow < out_rows(a));
+        for (int c = lane; row_ok && c < chunks; c += 32)
           reinterpret_cast<uint4*>(orow)[c] = reinterpret_cast<const uint4*>(stg)[c];
-        if (a.lse && lane < 4) {
+        if (row_ok && a.lse && lane < 4) {
           if (cpair < group)
             a.lse[frow * a.Hq + g * group + cpair] = l0 > 0.f ? (m0 + __log2f(l0)) * kLn2 : -INFINITY;
           if (cpair + 1 < group)
             a.lse[frow * a.Hq + g * group + cpair + 1] = l1 > 0.f ? (m1 + __log2f(l1)) * kLn2 : -INFINITY;
         }
         __syncwarp();
-      } else if (!CL) {
+      } else if (!CL && QSA_DCHECK(a.ctl, it.orow >= 0 && it.orow < a.num_items)) {
         // unnormalised partial: part[item][h][0..D) = o, part[item][h][D] = m (log2 units), [D+1] = l
         float* prow = a.part + it.orow * a.Hq * (kD + 2);
 #pragma unroll
@@ -884,15 +901,16 @@ __global__ void __launch_bounds__(WideCfg<HKV, D, NSUB>::kThreads, 1) sparse_att
       __syncwarp();
       uint16_t* orow = a.out + (it.orow * a.Hq + hbase) * D;
       const int chunks = nvalid * D / 8;   // 16-byte chunks of this warp's output heads
-      for (int c = lane; c < chunks; c += 32)
+      const bool row_ok = QSA_DCHECK(a.ctl, it.orow >= 0 && it.orow < out_rows(a));
+      for (int c = lane; row_ok && c < chunks; c += 32)
         reinterpret_cast<uint4*>(orow)[c] = reinterpret_cast<const uint4*>(stg)[c];
-      if (a.lse && lane < 4) {
+      if (row_ok && a.lse && lane < 4) {
         if (cpair < nvalid) a.lse[it.orow * a.Hq + hbase + cpair] = l0 > 0.f ? (m0 + __log2f(l0)) * kLn2 : -INFINITY;
         if (cpair + 1 < nvalid)
           a.lse[it.orow * a.Hq + hbase + cpair + 1] = l1 > 0.f ? (m1 + __log2f(l1)) * kLn2 : -INFINITY;
       }
       __syncwarp();
-    } else {
+    } else if (QSA_DCHECK(a.ctl, it.orow >= 0 && it.orow < a.num_items)) {
       // unnormalised partial: part[item][h][0..D) = o, part[item][h][D] = m (log2 units), [D+1] = l
       float* prow = a.part + it.orow * a.Hq * (D + 2);
 #pragma unroll

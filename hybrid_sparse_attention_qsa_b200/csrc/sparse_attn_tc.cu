@@ -105,6 +105,11 @@ struct TcArgs {
 };
 
 __device__ __forceinline__ int tile_chunks(int nu) { return max(1, (nu + kCB - 1) / kCB); }
+// The chunks of tile tl (the debug build checks them against the record capacity).
+__device__ __forceinline__ int tile_chunks(const TcArgs& a, int tl) {
+  const int n = tile_chunks(a.cnt[tl]);
+  return QSA_DCHECK(a.ctl, n <= a.capc) ? n : a.capc;
+}
 
 // 2^x on the special-function unit (flushes subnormal results to zero; 2^-inf = 0).  The
 // probabilities it produces are rounded to bf16 for the P.V product anyway.
@@ -208,8 +213,11 @@ __global__ void __launch_bounds__(kUnionThreads) tile_union_kernel(const int32_t
       const uint32_t m = umask[i];
       if (m) {
         const uint2 e = make_uint2(static_cast<uint32_t>(w0 + i), m);
-        te[u] = e;
-        sent[u++] = e;
+        if (QSA_DCHECK(ctl, u < cap)) {
+          te[u] = e;
+          sent[u] = e;
+        }
+        ++u;
       }
     }
     total += s_scan[kUnionThreads / 32];
@@ -242,6 +250,7 @@ __global__ void __launch_bounds__(kUnionThreads) tile_union_kernel(const int32_t
       }
     }
     ChunkInfo* r = tr + c;
+    if (!QSA_DCHECK(ctl, c < capc)) continue;
     if (lane < kCB) r->blocks[lane] = static_cast<int>(e.x);
     if (lane < kTQ) {
       r->words[lane] = static_cast<uint16_t>(myw);
@@ -322,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int tl = ntl - 1 - it;
       const int tile = a.tile0 + tl;
       const int b = tile / a.tpb, t0 = (tile % a.tpb) * kTQ;
-      const int nch = tile_chunks(a.cnt[tl]);
+      const int nch = tile_chunks(a, tl);
       const ChunkInfo* tr = a.recs + static_cast<long long>(tl) * a.capc;
       for (int g = 0; alive && g < HKV; ++g, ++hp) {
         bool ok = true;
@@ -351,8 +360,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lead && lane == 0)
             bulk_g2s(&info[s], tr + c, static_cast<unsigned>(sizeof(ChunkInfo)), &bar->kv_full[s]);
           if (has_box) {
+            const int blk_ok = QSA_DCHECK(a.ctl, blk >= 0 && 4ll * blk < a.q_pos0 + a.Tq) ? blk : 0;
             uint8_t* dst = kvs + s * 2 * kKVBytes + btv * kKVBytes + bhalf * kKVHalf + bj * 512;
-            tma_load_4d(dst, btv ? &vmap : &kmap, &bar->kv_full[s], bhalf * 64, g, blk * 4, b);
+            tma_load_4d(dst, btv ? &vmap : &kmap, &bar->kv_full[s], bhalf * 64, g, blk_ok * 4, b);
           }
         }
       }
@@ -380,7 +390,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool alive = true;
       for (int it = blockIdx.x; alive && it < ntl; it += gridDim.x) {
         const int tl = ntl - 1 - it;
-        const int nch = tile_chunks(a.cnt[tl]);
+        const int nch = tile_chunks(a, tl);
         for (int g = 0; alive && g < HKV; ++g, ++hp, n0 += nch) {
           if (!mbar_wait_suspend(&bar->q_full, static_cast<unsigned>(hp) & 1u, a.ctl)) {
             alive = false;
@@ -467,7 +477,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int tl = ntl - 1 - it;
       const int tile = a.tile0 + tl;
       const int b = tile / a.tpb, t0 = (tile % a.tpb) * kTQ;
-      const int nch = tile_chunks(a.cnt[tl]);
+      const int nch = tile_chunks(a, tl);
       const bool vrow = t0 + t < a.Tq;
       const long long pos = a.q_pos0 + t0 + t;
       const int lim = static_cast<int>(pos & 3);
@@ -589,6 +599,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool use1 = nch > 1;
         const long long orow = (static_cast<long long>(b) * a.Tq + t0 + t) * a.Hq + g * kGrp + hh;
         uint4* op = reinterpret_cast<uint4*>(a.out + orow * kD + grp * 64);
+        const bool row_ok = vrow && QSA_DCHECK(a.ctl, orow < static_cast<long long>(a.B) * a.Tq * a.Hq);
         const uint32_t oc0 = tmem + lane_addr + kOCol + grp * 64;      // this warp's 64 columns of O[0]
         const uint32_t oc1 = oc0 + kD;                                 // ... and of O[1]
 #pragma unroll
@@ -597,7 +608,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld_32x32(oc0 + p2 * 32, x0);
           if (use1) tmem_ld_32x32(oc1 + p2 * 32, x1);
           tmem_ld_wait();
-          if (vrow) {
+          if (row_ok) {
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               float v[8];
@@ -609,7 +620,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        if (grp == 0 && vrow && a.lse) a.lse[orow] = lt > 0.f ? (M + __log2f(lt)) * kLn2 : -INFINITY;
+        if (grp == 0 && row_ok && a.lse) a.lse[orow] = lt > 0.f ? (M + __log2f(lt)) * kLn2 : -INFINITY;
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar->o_free);

@@ -9,11 +9,16 @@ from __future__ import annotations
 import ctypes
 import math
 import os
+import weakref
 
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libqsa_b200.so")
+# QSA_DEBUG=1 in the environment (read at import) selects the debug build of the library, whose
+# device-side bounds checks record QSA_ERR_DEVICE_CHECK instead of touching memory out of range,
+# and puts a canary guard after every buffer this binding allocates (checked by qsa_check_canaries).
+DEBUG = os.environ.get("QSA_DEBUG", "0") not in ("", "0")
+LIB_PATH = os.path.join(_PKG, "libqsa_b200_debug.so" if DEBUG else "libqsa_b200.so")
 
 QSA_OK = 0
 QSA_ERR_INVALID_ARGUMENT = 1
@@ -21,6 +26,7 @@ QSA_ERR_UNSUPPORTED = 2
 QSA_ERR_WORKSPACE_TOO_SMALL = 3
 QSA_ERR_CUDA = 4
 QSA_ERR_TIMEOUT = 5
+QSA_ERR_DEVICE_CHECK = 6
 
 QSA_SCORE_RELU_SUM = 0
 QSA_SCORE_LINEAR = 1
@@ -113,6 +119,58 @@ def _need(t: torch.Tensor, dtype, name: str):
         raise ValueError(f"{name} must be contiguous")
 
 
+# ------------------------------------------------------------------------------- canary guards
+# In debug mode every device buffer this binding allocates (outputs, workspaces, staged inputs) is
+# followed by CANARY_BYTES bytes of CANARY_BYTE.  A kernel that writes past the end of its buffer
+# changes them; qsa_check_canaries() finds it.
+CANARY_BYTES = 256
+CANARY_BYTE = 0xA5
+_guards: list = []   # (weak reference to the returned tensor, bytes in use, what it holds)
+
+
+def _empty(*shape, dtype, device, what: str = "buffer") -> torch.Tensor:
+    """torch.empty; in debug mode the allocation carries a canary guard after its last byte."""
+    if len(shape) == 1 and isinstance(shape[0], (tuple, list, torch.Size)):
+        shape = tuple(shape[0])
+    if not DEBUG:
+        return torch.empty(shape, dtype=dtype, device=device)
+    numel = math.prod(shape)
+    esz = torch.empty((), dtype=dtype).element_size()
+    raw = torch.empty(numel + CANARY_BYTES // esz, dtype=dtype, device=device)
+    raw[numel:].view(torch.uint8).fill_(CANARY_BYTE)
+    t = raw[:numel].view(shape)   # t._base is raw
+    n = numel * esz
+    if len(_guards) > 4096:
+        _guards[:] = [g for g in _guards if g[0]() is not None]
+    _guards.append((weakref.ref(t), n, what))
+    return t
+
+
+def _empty_like(t: torch.Tensor, what: str = "buffer") -> torch.Tensor:
+    return _empty(t.shape, dtype=t.dtype, device=t.device, what=what)
+
+
+def qsa_check_canaries() -> int:
+    """Debug mode: synchronise and check the guard after every live buffer the binding allocated.
+    Returns how many were checked; raises RuntimeError naming the buffers whose guard changed."""
+    if not DEBUG:
+        return 0
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
+    bad, checked = [], 0
+    for ref, n, what in _guards:
+        t = ref()
+        if t is None:     # freed: no longer checked
+            continue
+        guard = t._base[t.numel():].view(torch.uint8)
+        checked += 1
+        if bool((guard != CANARY_BYTE).any()):
+            bad.append(f"{what} ({n} bytes)")
+    if bad:
+        raise RuntimeError("canary guard overwritten after: " + ", ".join(bad))
+    return checked
+
+
 # ---------------------------------------------------------------------------------------- ABI calls
 def qsa_abi_version() -> int:
     return lib().qsa_abi_version()
@@ -145,7 +203,7 @@ def qsa_pool_block_keys(ki: torch.Tensor, kp: torch.Tensor | None = None, *, blk
         raise ValueError("ki must be a CUDA bf16 [B, L, Di] tensor with packed rows")
     B, L, Di = ki.shape
     if kp is None:
-        kp = torch.empty(B, L // blk, Di, dtype=torch.bfloat16, device=ki.device)
+        kp = _empty(B, L // blk, Di, dtype=torch.bfloat16, device=ki.device, what="kp")
     if kp.dtype != torch.bfloat16 or not _batch_view_ok(kp) or tuple(kp.shape) != (B, L // blk, Di):
         raise ValueError("kp must be a bf16 [B, L // blk, Di] tensor with packed rows")
     if yarn:
@@ -169,7 +227,7 @@ def qsa_rope_index_queries(qi: torch.Tensor, qi_out: torch.Tensor | None = None,
     else:
         B, Tq, Hi, Di = qi.shape
     if qi_out is None:
-        qi_out = torch.empty_like(qi)
+        qi_out = _empty_like(qi, what="rotated qi")
     if yarn:
         rp = _rope_params(rope_theta, yarn)
         _check(lib().qsa_rope_index_queries_rope(_ptr(qi), _ptr(qi_out), B, Tq, Hi, Di, q_pos0, _ptr(seqlens),
@@ -195,7 +253,7 @@ def qsa_index_score(qi: torch.Tensor, kp: torch.Tensor, *, head_w: torch.Tensor 
         B, Tq, Hi, Di = qi.shape
     NBk = kp.shape[1]
     if scores is None:
-        scores = torch.full((B, Tq, max(NBk, 1)), float("nan"), dtype=torch.float32, device=qi.device)
+        scores = _empty((B, Tq, max(NBk, 1)), dtype=torch.float32, device=qi.device, what="scores").fill_(float("nan"))
     _need(scores, torch.float32, "scores")
     if head_w is not None:
         _need(head_w, torch.float32, "head_w")
@@ -236,11 +294,11 @@ def qsa_select_topk(k: int, *, scores: torch.Tensor | None = None, qi: torch.Ten
         ld = 0
         if workspace is None:
             nbytes = qsa_workspace_size(QSA_OP_SELECT_TOPK, B, Tq, NBk, k, 0, 0)
-            workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+            workspace = _empty(nbytes, dtype=torch.uint8, device=dev, what="select workspace")
     if seqlens is not None:
         _need(seqlens, torch.int32, "seqlens")
     if idx is None:
-        idx = torch.empty((B, k) if seqlens is not None else (B, Tq, k), dtype=torch.int32, device=dev)
+        idx = _empty((B, k) if seqlens is not None else (B, Tq, k), dtype=torch.int32, device=dev, what="idx")
     _need(idx, torch.int32, "idx")
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().qsa_select_topk(_ptr(scores), ld, _ptr(qi), _ptr(kp), _ptr(head_w), _ptr(seqlens), B, Tq, NBk, Hi,
@@ -265,10 +323,10 @@ def qsa_decode_select(k: int, *, qi: torch.Tensor, kp: torch.Tensor, ki: torch.T
     B, Hi, Di = qi.shape
     NBk = kp.shape[1]
     if workspace is None:
-        workspace = torch.empty(qsa_workspace_size(QSA_OP_SELECT_TOPK, B, 1, NBk, k, 0, 0), dtype=torch.uint8,
-                                device=qi.device)
+        workspace = _empty(qsa_workspace_size(QSA_OP_SELECT_TOPK, B, 1, NBk, k, 0, 0), dtype=torch.uint8,
+                           device=qi.device, what="select workspace")
     if idx is None:
-        idx = torch.empty((B, k), dtype=torch.int32, device=qi.device)
+        idx = _empty((B, k), dtype=torch.int32, device=qi.device, what="idx")
     _need(idx, torch.int32, "idx")
     # without YaRN the rotary base goes through fp32, as in qsa_pool_block_keys(rope_theta=...)
     rp = _rope_params(rope_theta if yarn else ctypes.c_float(rope_theta).value, yarn)
@@ -297,9 +355,9 @@ def qsa_sparse_attn_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, i
     kb = idx.shape[-1]
     scale = 1.0 / math.sqrt(D) if scale is None else scale
     if out is None:
-        out = torch.empty_like(q)
+        out = _empty_like(q, what="out")
     if lse is None and want_lse:
-        lse = torch.empty(B, Tq, Hq, dtype=torch.float32, device=q.device)
+        lse = _empty(B, Tq, Hq, dtype=torch.float32, device=q.device, what="lse")
     if not tiles:
         _check(lib().qsa_sparse_attn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(idx), B, Tq, Tk, Hq, Hkv, D, kb, blk,
                                              q_pos0, scale, _ptr(out), _ptr(lse), _stream(q.device)),
@@ -307,7 +365,7 @@ def qsa_sparse_attn_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, i
         return out, lse
     if workspace is None:
         nbytes = qsa_workspace_size(QSA_OP_SPARSE_ATTN_PREFILL, B, Tq, 0, kb, Hq, D)
-        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+        workspace = _empty(max(nbytes, 16), dtype=torch.uint8, device=q.device, what="attention workspace")
     ws_bytes = workspace.numel() * workspace.element_size()
     _check(lib().qsa_sparse_attn_prefill_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(idx), B, Tq, Tk, Hq, Hkv, D, kb, blk,
                                             q_pos0, scale, _ptr(out), _ptr(lse), _ptr(workspace), ws_bytes,
@@ -335,12 +393,12 @@ def qsa_sparse_attn_decode(q: torch.Tensor, kcache: torch.Tensor, vcache: torch.
     kb = idx.shape[-1]
     scale = 1.0 / math.sqrt(D) if scale is None else scale
     if out is None:
-        out = torch.empty_like(q)
+        out = _empty_like(q, what="out")
     if lse is None and want_lse:
-        lse = torch.empty(B, Hq, dtype=torch.float32, device=q.device)
+        lse = _empty(B, Hq, dtype=torch.float32, device=q.device, what="lse")
     if workspace is None:
         nbytes = qsa_workspace_size(QSA_OP_SPARSE_ATTN_DECODE, B, 1, 0, kb, Hq, D, num_splits)
-        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+        workspace = _empty(max(nbytes, 16), dtype=torch.uint8, device=q.device, what="attention workspace")
     ws_bytes = workspace.numel() * workspace.element_size()
     _check(lib().qsa_sparse_attn_decode(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(seqlens), _ptr(idx), B, Lmax, Hq, Hkv,
                                         D, kb, blk, scale, num_splits, _ptr(out), _ptr(lse), _ptr(workspace), ws_bytes,
@@ -364,7 +422,7 @@ def qsa_sparse_attn_decode_noalloc(q: torch.Tensor, kcache: torch.Tensor, vcache
     kb = idx.shape[-1]
     scale = 1.0 / math.sqrt(D) if scale is None else scale
     if out is None:
-        out = torch.empty_like(q)
+        out = _empty_like(q, what="out")
     _check(lib().qsa_sparse_attn_decode_noalloc(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(seqlens), _ptr(idx), B,
                                                 Lmax, Hq, Hkv, D, kb, blk, scale, num_splits, _ptr(out), _ptr(lse),
                                                 _stream(q.device)), "qsa_sparse_attn_decode_noalloc")
@@ -470,17 +528,17 @@ def prefill_host(q, k, v, qi, ki, *, topk: int, device="cuda", out=None, q_pos0:
     bufs = device_buffers if device_buffers is not None else {}
     for name, t in (("q", q), ("k", k), ("v", v), ("qi", qi), ("ki", ki)):
         if name not in bufs:
-            bufs[name] = torch.empty(t.shape, dtype=t.dtype, device=dev)
+            bufs[name] = _empty(t.shape, dtype=t.dtype, device=dev, what=name)
     B, Tq, Hq, D = q.shape
     Tk = k.shape[1]
     if out is None:
         out = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
     if "out" not in bufs:
-        bufs["out"] = torch.empty(q.shape, dtype=q.dtype, device=dev)
+        bufs["out"] = _empty(q.shape, dtype=q.dtype, device=dev, what="out")
     if "lse" not in bufs:
-        bufs["lse"] = torch.empty(B, Tq, Hq, dtype=torch.float32, device=dev)
+        bufs["lse"] = _empty(B, Tq, Hq, dtype=torch.float32, device=dev, what="lse")
     if "kp" not in bufs:
-        bufs["kp"] = torch.empty(ki.shape[0], ki.shape[1] // 4, ki.shape[2], dtype=ki.dtype, device=dev)
+        bufs["kp"] = _empty(ki.shape[0], ki.shape[1] // 4, ki.shape[2], dtype=ki.dtype, device=dev, what="kp")
     # row chunks (one sequence only: the rows of a chunk are then contiguous in every tensor)
     n = max(1, min(chunks, Tq)) if B == 1 else 1
     # chunk bounds on multiples of 16 rows: the query-tile attention groups rows 16 at a time from a
@@ -516,7 +574,7 @@ def prefill_host(q, k, v, qi, ki, *, topk: int, device="cuda", out=None, q_pos0:
             arrived.append(ev)
     kp = bufs["kp"]
     if "idx" not in bufs:
-        bufs["idx"] = torch.empty(B, Tq, topk, dtype=torch.int32, device=dev)
+        bufs["idx"] = _empty(B, Tq, topk, dtype=torch.int32, device=dev, what="idx")
     idx = bufs["idx"]
     for c in range(ns):
         slo, shi = sbounds[c], sbounds[c + 1]
@@ -542,8 +600,8 @@ def prefill_host(q, k, v, qi, ki, *, topk: int, device="cuda", out=None, q_pos0:
                         workspace=workspace, idx=idx[:, slo:shi])
     if "attn_ws" not in bufs:
         rows = max(bounds[c + 1] - bounds[c] for c in range(n))
-        bufs["attn_ws"] = torch.empty(max(16, qsa_workspace_size(QSA_OP_SPARSE_ATTN_PREFILL, B, rows, 0, topk, Hq, D)),
-                                      dtype=torch.uint8, device=dev)
+        bufs["attn_ws"] = _empty(max(16, qsa_workspace_size(QSA_OP_SPARSE_ATTN_PREFILL, B, rows, 0, topk, Hq, D)),
+                                 dtype=torch.uint8, device=dev, what="attention workspace")
     for c in range(n):
         lo, hi = bounds[c], bounds[c + 1]
         if hi <= lo:

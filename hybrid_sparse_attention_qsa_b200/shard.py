@@ -101,18 +101,20 @@ class ShardedPrefill:
         self.k, self.blk, self.world, self.rank, self.group = topk, blk, world, rank, group
         self.ranges = rank_chunks(T, world, rank, blk)
         dev = torch.device(device)
-        self.kfull = torch.empty(B, T, Hkv, D, dtype=torch.bfloat16, device=dev)
-        self.vfull = torch.empty_like(self.kfull)
-        self.kpfull = torch.empty(B, T // blk, Di, dtype=torch.bfloat16, device=dev)
-        self.kp_local = [torch.empty(B, (b - a) // blk, Di, dtype=torch.bfloat16, device=dev) for a, b in self.ranges]
+        E = Q._empty   # torch.empty, with canary guards in debug mode
+        self.kfull = E(B, T, Hkv, D, dtype=torch.bfloat16, device=dev, what="gathered k")
+        self.vfull = E(B, T, Hkv, D, dtype=torch.bfloat16, device=dev, what="gathered v")
+        self.kpfull = E(B, T // blk, Di, dtype=torch.bfloat16, device=dev, what="gathered kp")
+        self.kp_local = [E(B, (b - a) // blk, Di, dtype=torch.bfloat16, device=dev, what="local kp")
+                         for a, b in self.ranges]
         rows = max(b - a for a, b in self.ranges)
         ws = Q.qsa_workspace_size(Q.QSA_OP_SELECT_TOPK, B, rows, T // blk, topk, Hq, D)
-        self.ws = torch.empty(ws, dtype=torch.uint8, device=dev)
+        self.ws = E(ws, dtype=torch.uint8, device=dev, what="select workspace")
         aws = Q.qsa_workspace_size(Q.QSA_OP_SPARSE_ATTN_PREFILL, B, rows, 0, topk, Hq, D)
-        self.attn_ws = torch.empty(max(aws, 16), dtype=torch.uint8, device=dev)
-        self.idx = [torch.empty(B, b - a, topk, dtype=torch.int32, device=dev) for a, b in self.ranges]
-        self.out = [torch.empty(B, b - a, Hq, D, dtype=torch.bfloat16, device=dev) for a, b in self.ranges]
-        self.lse = [torch.empty(B, b - a, Hq, dtype=torch.float32, device=dev) for a, b in self.ranges]
+        self.attn_ws = E(max(aws, 16), dtype=torch.uint8, device=dev, what="attention workspace")
+        self.idx = [E(B, b - a, topk, dtype=torch.int32, device=dev, what="idx") for a, b in self.ranges]
+        self.out = [E(B, b - a, Hq, D, dtype=torch.bfloat16, device=dev, what="out") for a, b in self.ranges]
+        self.lse = [E(B, b - a, Hq, dtype=torch.float32, device=dev, what="lse") for a, b in self.ranges]
 
     def pool_local(self, ki: list):
         """Pool this rank's indexer keys, each chunk at its own positions."""

@@ -40,6 +40,13 @@
  *     merge through the workspace).  Other shapes return QSA_ERR_UNSUPPORTED.
  *   - Calls are thread-safe.  The library keeps only per-device caches (device attributes, the
  *     status word) and no other mutable global state.
+ *   - Every call opens an NVTX range named after the function (visible in Nsight Systems and
+ *     Nsight Compute; costs one pointer test when no tool is attached).
+ *   - The debug build of the library (libqsa_b200_debug.so, compiled with -DQSA_DEBUG) has the
+ *     same ABI.  Its kernels check the data-dependent addresses they form (gathered K/V rows,
+ *     output and partial rows, tile-union entries and chunk records) against the sizes of the
+ *     call; a failed check skips the access and records QSA_ERR_DEVICE_CHECK.  In a correct
+ *     library no check fails; the release build compiles them out.
  */
 #ifndef QSA_H
 #define QSA_H
@@ -65,7 +72,9 @@ typedef enum {
   QSA_ERR_UNSUPPORTED = 2,         /* a shape outside the supported set above */
   QSA_ERR_WORKSPACE_TOO_SMALL = 3, /* ws_bytes below what the call needs */
   QSA_ERR_CUDA = 4,                /* the CUDA runtime rejected a launch or query */
-  QSA_ERR_TIMEOUT = 5              /* a device-side wait ran out of time (device status only) */
+  QSA_ERR_TIMEOUT = 5,             /* a device-side wait ran out of time (device status only) */
+  QSA_ERR_DEVICE_CHECK = 6         /* debug build only: a device-side bounds check failed and the
+                                      access was skipped (device status only) */
 } qsa_status_t;
 
 typedef enum {
@@ -354,7 +363,8 @@ QSA_API int qsa_decode_split_merge(int B, int Hq, int Hkv, int D, int num_splits
 /*
  * Synchronises `stream`, then reads and clears the current device's status word:
  * QSA_OK, QSA_ERR_INVALID_ARGUMENT (an index or sequence length was out of range and skipped),
- * QSA_ERR_TIMEOUT (a device-side wait ran out of time and the kernel returned early), or
+ * QSA_ERR_TIMEOUT (a device-side wait ran out of time and the kernel returned early),
+ * QSA_ERR_DEVICE_CHECK (debug build: a device-side bounds check failed), or
  * QSA_ERR_CUDA (the synchronisation itself failed).
  */
 QSA_API qsa_status_t qsa_get_device_status(void* stream);

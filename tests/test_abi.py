@@ -38,6 +38,17 @@ def test_library_exports_every_declared_symbol(lib):
     assert set(names) == set(Q.SIGNATURES), "binding and header disagree"
 
 
+def test_debug_library_exports_the_same_symbols():
+    # the debug build (-DQSA_DEBUG): same ABI, device-side bounds checks compiled in
+    path = B.build(debug=True)
+    assert path == B.LIB_DEBUG
+    dl = ctypes.CDLL(path)
+    for n in declared_symbols():
+        assert hasattr(dl, n), n
+    dl.qsa_status_string.restype = ctypes.c_char_p
+    assert dl.qsa_status_string(Q.QSA_ERR_DEVICE_CHECK) == b"QSA_ERR_DEVICE_CHECK"
+
+
 def test_abi_version_and_status_strings(lib):
     assert Q.qsa_abi_version() == 1
     assert Q.status_string(Q.QSA_ERR_WORKSPACE_TOO_SMALL) == "QSA_ERR_WORKSPACE_TOO_SMALL"
