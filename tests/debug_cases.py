@@ -17,13 +17,21 @@ from hybrid_sparse_attention_qsa_b200 import inputs as I
 from hybrid_sparse_attention_qsa_b200 import qsa as Q
 
 
+_checked = [0]   # canary guards checked so far (debug library only)
+
+
 def _ok(name: str):
+    """No device-side check or argument fault recorded, and (debug mode) the guard after every live
+    buffer the binding allocated is intact, while this case's workspaces are still alive."""
     st = Q.qsa_get_device_status()
     if st != Q.QSA_OK:
         raise RuntimeError(f"{name}: device status {Q.status_string(st)}")
+    _checked[0] += Q.qsa_check_canaries()
 
 
 def run_cases(dev="cuda:0") -> dict:
+    """Results of every case on the host.  With the debug library, canaries_checked() then counts
+    the guard checks made along the way."""
     res = {}
     # prefill through the whole path: pooling, scores, materialised top-k, row attention
     w = I.WORKLOADS["prefill_32k"].with_(T=3000, k=64, seed=501)
@@ -75,11 +83,15 @@ def run_cases(dev="cuda:0") -> dict:
     return {n: t.detach().cpu() for n, t in res.items()}
 
 
+def canaries_checked() -> int:
+    return _checked[0]
+
+
 if __name__ == "__main__":
     if not Q.DEBUG:
         raise SystemExit("set QSA_DEBUG=1: this run is meant for the debug library")
     out = run_cases()
-    n = Q.qsa_check_canaries()
+    n = canaries_checked()
     if n == 0:
         raise SystemExit("no canary guard was checked")
     torch.save({"results": out, "canaries_checked": n, "lib": Q.LIB_PATH}, sys.argv[1])
