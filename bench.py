@@ -9,8 +9,10 @@ One step = the whole hot path over one batch of synthetic input:
     score + top-k over the pooled-key cache -> split-KV sparse attention + merge.
 Inputs are resident in HBM when the timed region starts and are larger than L2 (126 MB), so no L2
 flush is done between steps.  Times are CUDA events on the launching stream, max over ranks.
-With N > 1 every rank runs its own workload (different seed; no data-path collective), so the
-scaling is weak.  ``--impl reference`` times the CPU oracle on a bounded sample of the same workload.
+With N > 1 the ranks share one job (strong scaling): the prefill's query rows are sharded in
+zig-zag chunks with one all-gather of K, V and the pooled keys per step (shard.py), and the decode
+batch is split by sequence.  ``--impl reference`` times the CPU oracle on a bounded sample of the
+same workload.
 """
 from __future__ import annotations
 
@@ -285,7 +287,7 @@ def run_reference(args):
     sample = f"{rows} query rows spread evenly over the {w.T}-token prefill (pooling of all keys included)"
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * total / args.steps,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": {"workload": PREFILL, "B": w.B, "T": w.T, "Hq": w.Hq, "Hkv": w.Hkv,
                                               "D": w.D, "Hi": w.Hi, "Di": w.Di, "blk": w.blk, "k": w.k},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},

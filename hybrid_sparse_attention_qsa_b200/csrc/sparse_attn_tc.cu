@@ -8,9 +8,9 @@
 // processed together: the tile attends over the UNION of its rows' blocks, each union block is
 // gathered once per tile instead of once per row, and every row masks out the union blocks it did
 // not select.  16 rows x the 8 query heads of one KV head are the 128 rows (M) of one tcgen05 MMA.
-// On the 128K workload the union of 16 rows is about 0.37 of the sum of their lists, so the gather
-// (the cost of the row-by-row kernel) shrinks ~2.7x while the contraction grows to about 6x the
-// selected pairs -- cheap on tcgen05.  The result is the same exact attention: a masked entry
+// The union of 16 rows is 0.38 (32K workload) to 0.46 (128K) of the sum of their lists, so the
+// gathered bytes shrink 2.2-2.6x, while the contraction grows to the whole union for every row
+// (about 7x the selected pairs at 128K).  The result is the same exact attention: a masked entry
 // contributes exp(-inf) = 0, and the softmax runs in fp32 over exactly the selected tokens.
 //
 // tile_union_kernel (one CTA per tile): every listed block of the 16 rows, and each row's own block,
@@ -20,25 +20,29 @@
 // slot) for the attention kernel.  Entries outside a row's causal range are skipped and recorded in
 // the device status (-1 and the own block are skipped silently); list order does not matter.
 //
-// sparse_attn_tc_kernel (persistent, one CTA per SM), per (tile, KV head):
-//   warps 0-7 producers: warp 0 loads the Q tile (two 128-byte-swizzled TMA boxes of [16 rows]
-//            [8 heads][64 d]) and, per chunk of 32 union entries, publishes the chunk's blocks and,
-//            per row, its member slots and the slot of its own block (the next chunk's entries are
-//            fetched ahead); then all 8 warps issue the chunk's 128 TMA boxes of [4 tokens][64 d]
-//            (block x half x K/V) into a 3-stage ring.  A single issuing warp caps these 512-byte
-//            gathers near 2 TB/s; eight reach ~10 TB/s (the gather probe);
-//   warp 8   TMEM owner and MMA issuer (one thread): S = Q K^T (M 128, N 128 tokens, K 128) into
-//            one of three S buffers, then O += P V with P read from TMEM (A operand) and V as an
-//            MN-major B operand;
-//   warps 12-15 softmax (one thread per row): mask, fp32 online softmax in exp2 form with a lazy
-//            rescale of O (only when the running max grows by more than 2^8), P packed to bf16
-//            into the S buffer's columns, and the epilogue (O / l -> bf16 rows, log-sum-exp).
-//            Two passes over the row in TMEM (max, then exponentials), skipping groups of 8 union
-//            slots that no row of the warp attends.
-// TMEM: S0 S1 S2 at columns 0, 128, 256, O at 384 (fp32, lane = row).  Every wait is bounded and
-// suspends the waiting warp (spinning producer and MMA warps would take issue slots from the softmax
-// warps on their schedulers); a role whose wait runs out stops, and every role reaches the final
-// barrier and TMEM release.
+// sparse_attn_tc_kernel (persistent, one CTA per SM, 512 threads), per (tile, KV head):
+//   warps 0-6 producers: warp 0 loads the Q tile (two 128-byte-swizzled TMA boxes of [16 rows]
+//            [8 heads][64 d]) and brings each chunk's record into shared memory beside its K/V
+//            (one bulk copy); all seven issue the chunk's 64 TMA boxes of [4 tokens][64 d]
+//            (block x K/V x half) into a 5-stage ring, each warp a fixed share, with the block ids
+//            of the next chunk fetched ahead.  Each box costs its issuing warp ~80 cycles, so one
+//            warp caps these 512-byte gathers near 2 TB/s device-wide; seven to eight reach
+//            ~10 TB/s (the gather probe);
+//   warp 7   MMA issuer (one thread), event-driven: S = Q K^T (M 128, N 64 tokens, K 128) into one
+//            of four S buffers as soon as a chunk and a buffer are ready, and O += P V (P read from
+//            TMEM as the A operand, V as an MN-major B operand) as soon as a chunk's P is written;
+//            chunks alternate between two O accumulators;
+//   warps 8-15 softmax, two groups of four warps (one TMEM lane quadrant each, one thread per row):
+//            group g takes every other chunk of a pass and owns O[g]: mask, fp32 online softmax in
+//            exp2 form with a lazy rescale of its O (only when the running max grows by more than
+//            2^8), P packed to bf16 into the S buffer's columns.  The epilogue merges the two
+//            groups' (m, l) through shared memory and their O accumulators from TMEM, then writes
+//            the bf16 rows and the log-sum-exp.
+// Register split (setmaxnreg): producers and MMA drop to 64 registers, softmax rises to 192.
+// TMEM: S0..S3 at columns 0, 64, 128, 192, O[0] at 256, O[1] at 384 (fp32, lane = row).  Every wait
+// is bounded and suspends the waiting warp (spinning producer and MMA warps would take issue slots
+// from the softmax warps on their schedulers); a role whose wait runs out stops, and every role
+// reaches the final barrier and TMEM release.
 #include <algorithm>
 #include <mutex>
 
