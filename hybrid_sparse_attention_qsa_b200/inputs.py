@@ -58,6 +58,9 @@ WORKLOADS = {
                            k=1024, seed=4),
     "decode_1m": Workload("decode_1m", "decode", B=8, T=1048576, Hq=16, Hkv=2, D=128, Hi=4, Di=64, blk=4,
                           k=1024, seed=6),
+    # a small decode batch (4 sequences x 64K, caches of 268 MB: larger than L2) for profiling runs
+    "decode_64k_b4": Workload("decode_64k_b4", "decode", B=4, T=65536, Hq=16, Hkv=2, D=128, Hi=4, Di=64, blk=4,
+                              k=512, seed=8),
     # the attention shape of the model on the pages (24 query heads over 2 KV heads at head
     # dimension 256) with the 128K recipe otherwise
     "prefill_128k_model": Workload("prefill_128k_model", "prefill", B=1, T=131072, Hq=24, Hkv=2, D=256, Hi=4, Di=64,
