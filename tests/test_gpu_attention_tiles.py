@@ -10,6 +10,7 @@ import torch
 import oracle as O
 from hybrid_sparse_attention_qsa_b200 import inputs as I
 from hybrid_sparse_attention_qsa_b200 import qsa as Q
+from tests import harness as H
 from tests import parity as P
 
 pytestmark = pytest.mark.gpu
@@ -169,3 +170,47 @@ def test_forced_tiles_refuse_other_shapes_and_missing_workspace():
         Q.qsa_sparse_attn_prefill(x["q"], x["k"], x["v"], idx, workspace=torch.empty(64, dtype=torch.uint8,
                                                                                       device=DEV))
     assert e.value.status == Q.QSA_ERR_WORKSPACE_TOO_SMALL
+
+
+# ------------------------------------------------------------------------------------------ full sizes
+def _full_prefill_tiles(name, n_random):
+    # the whole layer at the benchmark sizes with the query-tile attention forced: sampled rows
+    # against the oracle (lists and outputs), every row against the row-by-row kernel
+    w = I.WORKLOADS[name]
+    x = I.make_prefill(w, DEV)
+    res = Q.prefill(x["q"], x["k"], x["v"], x["qi"], x["ki"], topk=w.k)
+    torch.cuda.synchronize()
+    _status_ok()
+    rows = H.sample_rows(w.T, w.k, n_random=n_random, seed=w.seed + 1)
+    ri = torch.tensor(rows, device=DEV)
+    kp = O.pool_block_keys(I.bits(x["ki"]))
+    st = H.compare_prefill(res["idx"][0, ri].cpu().numpy(), I.bits(res["out"][0, ri]), res["lse"][0, ri].cpu().numpy(),
+                           I.bits(x["q"][0, ri]), I.bits(x["qi"][0, ri]), I.bits(x["k"][0]), I.bits(x["v"][0]), kp[0],
+                           rows, topk=w.k)
+    Q.qsa_set_attn_options(Q.QSA_ATTN_ROWS)
+    o_rows, l_rows = Q.qsa_sparse_attn_prefill(x["q"], x["k"], x["v"], res["idx"])
+    torch.cuda.synchronize()
+    _status_ok()
+    # tiles against rows on every row, on the device in chunks (the 1M outputs are 4.3 GB each)
+    mx, tot = 0.0, 0.0
+    a, b = res["out"].view(-1, 128), o_rows.view(-1, 128)
+    for s in range(0, a.shape[0], 1 << 20):
+        d = (a[s:s + (1 << 20)].float() - b[s:s + (1 << 20)].float()).abs()
+        mx = max(mx, d.max().item())
+        tot += d.sum().item()
+    mean = tot / a.numel()
+    assert mx <= P.MAX_ABS and mean <= P.MEAN_ABS, (mx, mean)
+    assert (res["lse"] - l_rows).abs().max().item() <= 1e-4
+    print(name, "tiles", st, "vs rows max", mx, "mean", mean)
+
+
+def test_tiles_full_size_32k_sampled_rows():
+    _full_prefill_tiles("prefill_32k", 40)
+
+
+def test_tiles_full_size_128k_sampled_rows():
+    _full_prefill_tiles("prefill_128k", 40)
+
+
+def test_tiles_full_size_1m_sampled_rows():
+    _full_prefill_tiles("prefill_1m", 12)
