@@ -551,7 +551,7 @@ def run_qsa(args):
 
         def e2e_step():
             Q.qsa.prefill_host(host["q"], host["k"], host["v"], host["qi"], host["ki"], topk=w.k, device=dev, out=hout,
-                               workspace=ws, device_buffers=dbufs)
+                               device_buffers=dbufs)
 
         e2e_step()
         torch.cuda.synchronize()

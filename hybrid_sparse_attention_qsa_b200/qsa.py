@@ -66,6 +66,9 @@ SIGNATURES = {
     "qsa_set_wait_timeout_ns": (None, [_U64]),
     "qsa_wait_timeout_selftest": (_I, [_U64, _P]),
     "qsa_probe_gather": (_I, [_P, _SZ, _I, _I, _I, _I, _I, _I, _I, _U64, _P]),
+    "qsa_prefill_host": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _I, _I64, _F, _I, _P, _P,
+                              _I, _I, _P, _SZ, _P, _P, _P]),
+    "qsa_prefill_host_device_bytes": (_SZ, [_I, _I, _I, _I, _I, _I, _I, _I, _I, _I, _I64, _I, _I, _I]),
 }
 
 _lib = None
@@ -499,119 +502,53 @@ def decode(q, kcache, vcache, qi, kp, seqlens, *, topk: int, rope_theta: float =
     return dict(out=out, lse=lse, idx=idx)
 
 
-_copy_streams = {}
 
-
-def _copy_stream(device, which: str = "in") -> "torch.cuda.Stream":
-    """Per-device copy streams: one for host->device, one for device->host (PCIe is full duplex)."""
-    d = (torch.device(device).index, which)
-    if d not in _copy_streams:
-        _copy_streams[d] = torch.cuda.Stream(device=device)
-    return _copy_streams[d]
+def qsa_prefill_host_device_bytes(B: int, Tq: int, Tk: int, Hq: int, Hkv: int, D: int, Hi: int, Di: int, k: int, *,
+                                  q_pos0: int = 0, rope: bool = False, chunks: int = 32, sel_chunks: int = 2,
+                                  blk: int = 4) -> int:
+    return int(lib().qsa_prefill_host_device_bytes(B, Tq, Tk, Hq, Hkv, D, Hi, Di, k, blk, q_pos0, 1 if rope else 0,
+                                                   chunks, sel_chunks))
 
 
 def prefill_host(q, k, v, qi, ki, *, topk: int, device="cuda", out=None, q_pos0: int = 0, rope_theta: float = 0.0,
-                 head_w=None, mode: int = QSA_SCORE_RELU_SUM, scale: float | None = None, workspace=None,
+                 head_w=None, mode: int = QSA_SCORE_RELU_SUM, scale: float | None = None,
                  device_buffers: dict | None = None, chunks: int = 32, sel_chunks: int = 2, yarn=None):
-    """The QSA layer for a prefill whose inputs live in (pinned) host memory; returns the output in
-    host memory.  Transfers overlap the kernels.  ki and qi are copied first, in ``sel_chunks``
-    causal row chunks: the pooling and block selection of a chunk's rows need only the indexer keys
-    and queries up to the chunk's end, so they start as soon as those have arrived.  q, k and v
-    follow in ``chunks`` causal row chunks on the same copy stream: chunk c's attention needs only
-    its own query rows and the keys and values of the positions before its end, so it starts as
-    soon as that chunk has arrived, and its output goes back on a second copy stream while the next
-    chunk is computed.  ``device_buffers`` (name -> device tensor) lets a caller reuse device memory.
-    Returns dict(out=host tensor, lse=device tensor, idx=device tensor)."""
+    """The QSA layer for a prefill whose inputs live in (pinned) host memory, through
+    qsa_prefill_host: the library copies the inputs in causal row chunks on its own copy streams,
+    starts each chunk's pooling + selection and attention as soon as its data has arrived, and sends
+    each chunk's output rows back while the next is computed.  ``device_buffers`` (a dict) keeps the
+    device scratch ("scratch"), the index lists ("idx") and the log-sum-exps ("lse") for reuse.
+    Returns dict(out=host tensor, lse=device tensor, idx=device tensor); the output is complete once
+    the current stream of ``device`` has reached this call."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (qi, "qi"), (ki, "ki")):
+        if t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError(f"{n} must be a contiguous bf16 host tensor")
     dev = torch.device(device)
-    main = torch.cuda.current_stream(dev)
-    cin, cout = _copy_stream(dev, "in"), _copy_stream(dev, "out")
-    bufs = device_buffers if device_buffers is not None else {}
-    for name, t in (("q", q), ("k", k), ("v", v), ("qi", qi), ("ki", ki)):
-        if name not in bufs:
-            bufs[name] = _empty(t.shape, dtype=t.dtype, device=dev, what=name)
     B, Tq, Hq, D = q.shape
-    Tk = k.shape[1]
-    if out is None:
-        out = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
-    if "out" not in bufs:
-        bufs["out"] = _empty(q.shape, dtype=q.dtype, device=dev, what="out")
-    if "lse" not in bufs:
-        bufs["lse"] = _empty(B, Tq, Hq, dtype=torch.float32, device=dev, what="lse")
-    if "kp" not in bufs:
-        bufs["kp"] = _empty(ki.shape[0], ki.shape[1] // 4, ki.shape[2], dtype=ki.dtype, device=dev, what="kp")
-    # row chunks (one sequence only: the rows of a chunk are then contiguous in every tensor)
-    n = max(1, min(chunks, Tq)) if B == 1 else 1
-    # chunk bounds on multiples of 16 rows: the query-tile attention groups rows 16 at a time from a
-    # call's first row, so aligned chunks make the same tiles (and the same bits) as one call
-    bounds = [0] + [((Tq * c) // n) // 16 * 16 for c in range(1, n)] + [Tq]
-    # selection chunks: query rows [slo, shi), whose blocks lie below key position q_pos0 + shi; the
-    # pooled keys of a chunk start on a whole block (row bounds in multiples of 4 when q_pos0 is)
-    ns = max(1, min(sel_chunks, Tq // 4)) if (B == 1 and q_pos0 % 4 == 0 and Tk == q_pos0 + Tq) else 1
-    sbounds = [0] + [(Tq * c // ns) // 4 * 4 for c in range(1, ns)] + [Tq]
-    cin.wait_stream(main)   # the device buffers may still be read by earlier work on `main`
-    with torch.cuda.stream(cin):
-        sel_ready = []
-        for c in range(ns):
-            slo, shi = sbounds[c], sbounds[c + 1]
-            klo, khi = (q_pos0 + slo if c else 0), (q_pos0 + shi if c < ns - 1 else Tk)
-            bufs["ki"][:, klo:khi].copy_(ki[:, klo:khi], non_blocking=True)
-            bufs["qi"][:, slo:shi].copy_(qi[:, slo:shi], non_blocking=True)
-            ev = torch.cuda.Event()
-            ev.record(cin)
-            sel_ready.append(ev)
-        arrived = []
-        kv_done = 0   # key/value positions already sent
-        for c in range(n):
-            lo, hi = bounds[c], bounds[c + 1]
-            kv_end = Tk if c == n - 1 else min(Tk, q_pos0 + hi)   # keys a query of the chunk can see
-            if kv_end > kv_done:
-                bufs["k"][:, kv_done:kv_end].copy_(k[:, kv_done:kv_end], non_blocking=True)
-                bufs["v"][:, kv_done:kv_end].copy_(v[:, kv_done:kv_end], non_blocking=True)
-                kv_done = kv_end
-            bufs["q"][:, lo:hi].copy_(q[:, lo:hi], non_blocking=True)
-            ev = torch.cuda.Event()
-            ev.record(cin)
-            arrived.append(ev)
-    kp = bufs["kp"]
+    Tk, Hkv = k.shape[1], k.shape[2]
+    Hi, Di = qi.shape[2], qi.shape[3]
+    rope = _rope_params(rope_theta, yarn) if rope_theta > 0 else None
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    nbytes = qsa_prefill_host_device_bytes(B, Tq, Tk, Hq, Hkv, D, Hi, Di, topk, q_pos0=q_pos0, rope=rope is not None,
+                                           chunks=chunks, sel_chunks=sel_chunks)
+    if nbytes == 0:
+        raise ValueError("invalid sizes for qsa_prefill_host")
+    bufs = device_buffers if device_buffers is not None else {}
+    if "scratch" not in bufs or bufs["scratch"].numel() < nbytes:
+        bufs["scratch"] = _empty(nbytes, dtype=torch.uint8, device=dev, what="host pipeline scratch")
     if "idx" not in bufs:
         bufs["idx"] = _empty(B, Tq, topk, dtype=torch.int32, device=dev, what="idx")
-    idx = bufs["idx"]
-    for c in range(ns):
-        slo, shi = sbounds[c], sbounds[c + 1]
-        main.wait_event(sel_ready[c])
-        if ns == 1:
-            qsa_pool_block_keys(bufs["ki"], kp, rope_theta=rope_theta, yarn=yarn)
-            qr = (qsa_rope_index_queries(bufs["qi"], rope_theta=rope_theta, q_pos0=q_pos0, yarn=yarn)
-                  if rope_theta > 0 else bufs["qi"])
-            qsa_select_topk(topk, qi=qr, kp=kp, head_w=head_w, q_pos0=q_pos0, mode=mode, workspace=workspace,
-                            idx=idx)
-            break
-        # keys of positions [klo, khi) pooled into blocks [klo/4, khi/4); the chunk's rows select
-        # among blocks below (q_pos0 + shi - 1) / 4
-        klo, khi = (q_pos0 + slo if c else 0), (q_pos0 + shi if c < ns - 1 else Tk)
-        if khi // 4 > klo // 4:
-            qsa_pool_block_keys(bufs["ki"][:, klo:khi // 4 * 4], kp[:, klo // 4:khi // 4], pos0=klo,
-                                rope_theta=rope_theta, yarn=yarn)
-        qc = bufs["qi"][:, slo:shi]
-        qr = (qsa_rope_index_queries(qc, rope_theta=rope_theta, q_pos0=q_pos0 + slo, yarn=yarn) if rope_theta > 0
-              else qc)
-        nbk = max(1, (q_pos0 + shi - 1) // 4)
-        qsa_select_topk(topk, qi=qr, kp=kp[:, :nbk], head_w=head_w, q_pos0=q_pos0 + slo, mode=mode,
-                        workspace=workspace, idx=idx[:, slo:shi])
-    if "attn_ws" not in bufs:
-        rows = max(bounds[c + 1] - bounds[c] for c in range(n))
-        bufs["attn_ws"] = _empty(max(16, qsa_workspace_size(QSA_OP_SPARSE_ATTN_PREFILL, B, rows, 0, topk, Hq, D)),
-                                 dtype=torch.uint8, device=dev, what="attention workspace")
-    for c in range(n):
-        lo, hi = bounds[c], bounds[c + 1]
-        if hi <= lo:
-            continue
-        main.wait_event(arrived[c])
-        opart = bufs["out"][:, lo:hi]
-        qsa_sparse_attn_prefill(bufs["q"][:, lo:hi], bufs["k"], bufs["v"], idx[:, lo:hi], q_pos0=q_pos0 + lo,
-                                scale=scale, out=opart, lse=bufs["lse"][:, lo:hi], workspace=bufs["attn_ws"])
-        cout.wait_stream(main)
-        with torch.cuda.stream(cout):
-            out[:, lo:hi].copy_(opart, non_blocking=True)
-    main.wait_stream(cout)
-    return dict(out=out, lse=bufs["lse"], idx=idx)
+    if "lse" not in bufs:
+        bufs["lse"] = _empty(B, Tq, Hq, dtype=torch.float32, device=dev, what="lse")
+    if out is None:
+        out = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+    if head_w is not None:
+        _need(head_w, torch.float32, "head_w")
+    scratch, idx, lse = bufs["scratch"], bufs["idx"], bufs["lse"]
+    with torch.cuda.device(dev):
+        _check(lib().qsa_prefill_host(_ptr(q), _ptr(k), _ptr(v), _ptr(qi), _ptr(ki), _ptr(out), B, Tq, Tk, Hq, Hkv, D,
+                                      Hi, Di, topk, 4, q_pos0, scale, mode, _ptr(head_w),
+                                      ctypes.byref(rope) if rope is not None else None, chunks, sel_chunks,
+                                      _ptr(scratch), scratch.numel(), _ptr(idx), _ptr(lse), _stream(dev)),
+               "qsa_prefill_host")
+    return dict(out=out, lse=lse, idx=idx)

@@ -290,6 +290,55 @@ QSA_API qsa_status_t qsa_sparse_attn_prefill_ws(const void* q, const void* k, co
 QSA_API qsa_status_t qsa_set_attn_options(int path);
 
 /*
+ * The whole QSA layer for one prefill whose inputs and output live in HOST memory
+ * ("Qwen3.8-Flash-Next architecture" (flozi.net), "Der Weg eines Tokens durch das Modell", item 2:
+ * pooling, block selection and attention over the selected tokens), with the transfers overlapped
+ * with the kernels.  (The pages have no host-side counterpart: this is the library's own schedule
+ * of the three calls above around the copies.)
+ *   host, read:    q [B][Tq][Hq][D], k, v [B][Tk][Hkv][D], qi [B][Tq][Hi][Di], ki [B][Tk][Di] (bf16)
+ *   host, written: out [B][Tq][Hq][D] bf16
+ *   Host buffers should be page-locked (cudaHostAlloc / cudaHostRegister) for the copies to
+ *   overlap; pageable memory gives the same result without the overlap.
+ *   Query row t sits at position q_pos0 + t; Tk >= q_pos0 + Tq.  mode, head_w (device, or NULL) and
+ *   rope (NULL or theta <= 0: no rotation) as for qsa_select_topk / qsa_pool_block_keys_rope;
+ *   scale > 0 as for qsa_sparse_attn_prefill.
+ * Schedule (B = 1): ki and qi are sent first in `sel_chunks` causal row chunks and each chunk's
+ * pooling and selection starts as soon as it has arrived (only when Tk = q_pos0 + Tq and
+ * q_pos0 % 4 == 0; else one chunk); q, k, v follow in `chunks` causal row chunks (K/V only up to
+ * each chunk's last position, each row sent once), each chunk's attention starts when it has
+ * arrived and its output rows go back while the next chunk is computed.  B > 1: one chunk of each.
+ * The kernels run on `stream`; the copies on two streams of the library's own (one per direction
+ * and device), ordered against `stream` with events.  The call returns once everything is
+ * enqueued; `out` is complete when `stream` reaches the point of the call (synchronise it, or
+ * record an event after the call).
+ * Device memory: `dev` (256-byte aligned, dev_bytes >= qsa_prefill_host_device_bytes(...)) holds
+ * the device copies of the inputs, the pooled keys, the rotated queries, the output rows and both
+ * workspaces; it must not be used by other work until the call's work on `stream` is done.
+ * idx_out [B][Tq][k_blocks] int32 and lse_out [B][Tq][Hq] fp32 (device, may be NULL: then kept in
+ * `dev`) receive the index lists and log-sum-exps.
+ * Calls on one device enqueue one at a time (a lock); their work may overlap on the GPU only if
+ * they use different `dev` buffers.
+ * Errors: INVALID_ARGUMENT (null pointer, dev misaligned, sizes, Tk < q_pos0 + Tq, blk != 4,
+ * chunks or sel_chunks < 1, scale <= 0), WORKSPACE_TOO_SMALL (dev_bytes), both before anything is
+ * enqueued; a failing step (for example UNSUPPORTED for a shape the kernels do not take) returns
+ * its own status with the work before it already enqueued; CUDA on a runtime error.
+ */
+QSA_API qsa_status_t qsa_prefill_host(const void* q, const void* k, const void* v, const void* qi, const void* ki,
+                                      void* out, int B, int Tq, int Tk, int Hq, int Hkv, int D, int Hi, int Di,
+                                      int k_blocks, int blk, int64_t q_pos0, float scale, qsa_score_mode_t mode,
+                                      const float* head_w, const qsa_rope_params_t* rope, int chunks,
+                                      int sel_chunks, void* dev, size_t dev_bytes, int32_t* idx_out,
+                                      float* lse_out, void* stream);
+
+/*
+ * Bytes of the `dev` buffer qsa_prefill_host needs for these sizes (rope: 1 if the indexer RoPE
+ * is on).  0 for invalid sizes.  Host arithmetic only.
+ */
+QSA_API size_t qsa_prefill_host_device_bytes(int B, int Tq, int Tk, int Hq, int Hkv, int D, int Hi, int Di,
+                                             int k_blocks, int blk, int64_t q_pos0, int rope, int chunks,
+                                             int sel_chunks);
+
+/*
  * Gather-sparse attention, decode (split-KV).  One new token per sequence.
  *   q [B][Hq][D] bf16; caches k, v [B][Lmax][Hkv][D] bf16 holding seqlens[b] tokens (the new
  *   token included, so the query sits at position seqlens[b] - 1); idx [B][k_blocks] int32

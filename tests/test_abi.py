@@ -213,3 +213,33 @@ def test_declared_attention_shape_limits(lib):
             assert dec(D, (gmax + 1) * Hkv, Hkv) == Q.QSA_ERR_UNSUPPORTED
             assert pre(D, (gmax + 1) * Hkv, Hkv) == Q.QSA_ERR_UNSUPPORTED
     assert pre(128, 12, 3) == Q.QSA_ERR_UNSUPPORTED
+
+
+def test_prefill_host_sizes_and_argument_checks(lib):
+    # host arithmetic only: the device bytes grow with the inputs, shrink with more row chunks
+    # (smaller per-chunk workspaces), and are 0 for invalid sizes
+    full = Q.qsa_prefill_host_device_bytes(1, 131072, 131072, 16, 2, 128, 4, 64, 512, chunks=1, sel_chunks=1)
+    chunked = Q.qsa_prefill_host_device_bytes(1, 131072, 131072, 16, 2, 128, 4, 64, 512)
+    inputs = 131072 * (2 * 16 * 128 * 2 + 2 * 2 * 128 * 2 + 4 * 64 * 2 + 64 * 2)   # q, out, k, v, qi, ki
+    assert full > chunked > inputs
+    assert Q.qsa_prefill_host_device_bytes(1, 131072, 131072, 16, 2, 128, 4, 64, 512, rope=True) > chunked
+    assert Q.qsa_prefill_host_device_bytes(1, 100, 50, 16, 2, 128, 4, 64, 512) == 0        # Tk < q_pos0 + Tq
+    assert Q.qsa_prefill_host_device_bytes(1, 100, 100, 16, 2, 128, 4, 64, 512, chunks=0) == 0
+    args = [FAKE] * 6 + [1, 64, 64, 16, 2, 128, 4, 64, 8, 4, 0, 0.1, 0, None, None, 1, 1, FAKE, 1 << 30, None, None,
+                         None]
+
+    def call(**kw):
+        a = list(args)
+        names = {"q": 0, "dev": 23, "dev_bytes": 24, "Tk": 8, "blk": 15, "scale": 17, "chunks": 21}
+        for n, val in kw.items():
+            a[names[n]] = val
+        return lib.qsa_prefill_host(*a)
+
+    assert call(q=None) == Q.QSA_ERR_INVALID_ARGUMENT
+    assert call(dev=None) == Q.QSA_ERR_INVALID_ARGUMENT
+    assert call(dev=P((1 << 20) + 16)) == Q.QSA_ERR_INVALID_ARGUMENT      # not 256-byte aligned
+    assert call(Tk=60) == Q.QSA_ERR_INVALID_ARGUMENT
+    assert call(blk=8) == Q.QSA_ERR_INVALID_ARGUMENT
+    assert call(scale=0.0) == Q.QSA_ERR_INVALID_ARGUMENT
+    assert call(chunks=0) == Q.QSA_ERR_INVALID_ARGUMENT
+    assert call(dev_bytes=100) == Q.QSA_ERR_WORKSPACE_TOO_SMALL
