@@ -45,8 +45,8 @@ DECODE = "decode_256k"
 TRAFFIC_PROFILES = {"prefill_128k": ("profiles/sparse_attn_prefill_128k.md",
                                      "hybrid_sparse_attention_qsa_b200/csrc/sparse_attn.cu")}
 # The attention's gather: every selected 4-token block of K and of V is one chunk of
-# blk * Hkv * D * 2 bytes, fetched by 4 issuing warps into a 3-stage ring of 16 slots (K and V).
-GATHER_PROBE = dict(issuer_warps=4, stages=3, slots_per_warp=8)
+# blk * Hkv * D * 2 bytes, fetched by 8 issuing warps into a 3-stage ring of 16 slots (K and V).
+GATHER_PROBE = dict(issuer_warps=8, stages=3, slots_per_warp=4)
 
 
 # ------------------------------------------------------------------------------------------- helpers
@@ -111,8 +111,8 @@ def gather_ceiling(dev, stream, w, sweep: bool = False) -> dict:
     import hybrid_sparse_attention_qsa_b200 as Q
     chunk = w.blk * w.Hkv * w.D * 2
     res = {"chunk_bytes": chunk, "config": dict(GATHER_PROBE)}
-    wide = dict(issuer_warps=8, stages=3, slots_per_warp=4)   # the same ring, issued by 8 warps
-    cases = [("l2_bulk", 32 << 20, 0, GATHER_PROBE), ("l2_bulk_w8", 32 << 20, 0, wide),
+    narrow = dict(issuer_warps=4, stages=3, slots_per_warp=8)   # the same ring, issued by 4 warps
+    cases = [("l2_bulk", 32 << 20, 0, GATHER_PROBE), ("l2_bulk_w4", 32 << 20, 0, narrow),
              ("hbm_bulk", 4 << 30, 0, GATHER_PROBE), ("l2_lsu", 32 << 20, 1, GATHER_PROBE)]
     if sweep:
         for iw, sl in ((1, 32), (2, 16), (8, 4), (8, 3), (12, 2), (16, 2)):

@@ -59,9 +59,9 @@ struct StageInfo {
 
 // Shared-memory ring of the copy pipeline: per stage SLOTS block slots of K, then SLOTS of V.  A
 // block of 4 tokens of all KV heads is one contiguous run of kBlockBytes in the [T][Hkv][D] layout.
-template <int HKV, int D, int SLOTS>
+template <int HKV, int D, int SLOTS, int ISS = kIssuers_>
 struct Ring {
-  static_assert(SLOTS % kIssuers_ == 0 && SLOTS <= 16, "slots per issuer warp");
+  static_assert(SLOTS % ISS == 0 && SLOTS <= 16, "slots per issuer warp");
   static constexpr int kSlots = SLOTS;
   static constexpr int kTokBytes = HKV * D * 2;               // one token of K (or V), all KV heads
   static constexpr int kBlockBytes = kBlk * kTokBytes;        // one block of K (or of V)
@@ -76,8 +76,15 @@ struct Cfg {
   static constexpr int kPitch = kBlockBytes + 16;
   static constexpr int kStageBytes = 2 * kSlots * kPitch;     // K slots, then V slots
   static constexpr int kConsumerWarps = kBlk * HKV;
-  static constexpr int kIssuers = kIssuers_;
+  // 8 issuing warps: the per-SM rate of 1-D bulk copies grows with the warps issuing them (the
+  // gather probe: 12.5 TB/s from L2 with 4 warps, 13.9 with 8, same ring)
+  static constexpr int kIssuers = 8;
   static constexpr int kThreads = (kConsumerWarps + kIssuers) * 32;
+  // With 512 threads a thread launches with 128 registers; the issuer warpgroups give registers to
+  // the consumer warpgroups (setmaxnreg): 256 x kLowRegs + 256 x kHighRegs = 512 x 128.
+  static constexpr bool kRegSplit = kThreads == 512;
+  static constexpr int kLowRegs = 64, kHighRegs = 192;
+  static_assert(!kRegSplit || kConsumerWarps * 32 * kHighRegs + kIssuers * 32 * kLowRegs <= 65536, "register split");
   static constexpr int kMergeSlot = 32 * 32 * 4 + 32 * 4 * 4; // o fragments + (m0, m1, l0, l1) per lane
   static constexpr int kMergeBytes = 3 * HKV * kMergeSlot;
   static constexpr int kInfoBytes = kStages * ((sizeof(StageInfo) + 15) / 16 * 16);
@@ -162,10 +169,10 @@ __device__ __forceinline__ Item make_item(const AttnArgs& a, int i) {
 
 // Helper issuer warp h (1 .. kIssuers_ - 1): issues slots h, h + kIssuers_, ... of every stage the
 // leading producer publishes, until it publishes nslots == -1.
-template <int HKV, int D, int SLOTS>
+template <int HKV, int D, int SLOTS, int ISS = kIssuers_>
 __device__ __forceinline__ void attn_helper(const AttnArgs& a, int h, uint8_t* ring, uint8_t* info, uint64_t* full,
                                             uint64_t* ready) {
-  using R = Ring<HKV, D, SLOTS>;
+  using R = Ring<HKV, D, SLOTS, ISS>;
   const int lane = threadIdx.x & 31;
   auto info_at = [&](int s) { return reinterpret_cast<const StageInfo*>(info + s * R::kInfoStride); };
   // ------------------------------------------------------------------ helper issuer warps
@@ -179,8 +186,8 @@ __device__ __forceinline__ void attn_helper(const AttnArgs& a, int h, uint8_t* r
     const StageInfo* inf = info_at(st);
     const int n = inf->nslots;
     if (n < 0) break;
-    const int slot = h + kIssuers_ * lane;
-    if (lane < R::kSlots / kIssuers_ && slot < n) {
+    const int slot = h + ISS * lane;
+    if (lane < R::kSlots / ISS && slot < n) {
       const int ntok = inf->ntok[slot];
       const long long tok0 = inf->tok0[slot];
       uint8_t* kd = ring + st * R::kStageBytes + slot * R::kPitch;
@@ -218,11 +225,11 @@ __device__ __forceinline__ void attn_fetch_list(const AttnArgs& a, int item, int
 // query's own block last), publishes each stage's slot list for the helpers and issues its own
 // share of the copies.  Returns only when no copy it registered is still in flight.  With
 // `prefetched` the first segment of the CTA's first item is already on its way (attn_fetch_list).
-template <int HKV, int D, int SLOTS>
+template <int HKV, int D, int SLOTS, int ISS = kIssuers_>
 __device__ __forceinline__ void attn_producer(const AttnArgs& a, uint8_t* ring, uint8_t* info, uint64_t* full,
                                               uint64_t* empty, uint64_t* ready, int* pend, int* idxbuf,
                                               bool prefetched = false) {
-  using R = Ring<HKV, D, SLOTS>;
+  using R = Ring<HKV, D, SLOTS, ISS>;
   const int lane = threadIdx.x & 31;
   auto info_at = [&](int s) { return reinterpret_cast<StageInfo*>(info + s * R::kInfoStride); };
   // ------------------------------------------------------------------ leading producer warp
@@ -255,7 +262,7 @@ __device__ __forceinline__ void attn_producer(const AttnArgs& a, uint8_t* ring, 
       mbar_arrive(&ready[st]);
     }
     __syncwarp();
-    if (lane < n && lane % kIssuers_ == 0) {
+    if (lane < n && lane % ISS == 0) {
       uint8_t* kd = ring + st * R::kStageBytes + lane * R::kPitch;
       uint8_t* vd = kd + R::kSlots * R::kPitch;
       if (QSA_DCHECK(a.ctl, tok0 >= 0 && ntok <= kBlk && tok0 + ntok <= a.Tk)) {
@@ -399,22 +406,20 @@ __global__ void __launch_bounds__(Cfg<HKV>::kThreads, 1) sparse_attn_kernel(Attn
 
   // In cluster mode every warp of every CTA passes the two cluster barriers of the split merge
   // exactly once (the consumer warps that merge inside their epilogue, the others here).
-  if (warp > C::kConsumerWarps) {
-    attn_helper<HKV, kD, kSlots>(a, warp - C::kConsumerWarps, ring, reinterpret_cast<uint8_t*>(info), full, ready);
+  if (warp >= C::kConsumerWarps) {
+    if constexpr (C::kRegSplit) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::kLowRegs));
+    if (warp > C::kConsumerWarps)
+      attn_helper<HKV, kD, kSlots, C::kIssuers>(a, warp - C::kConsumerWarps, ring, reinterpret_cast<uint8_t*>(info),
+                                                full, ready);
+    else
+      attn_producer<HKV, kD, kSlots, C::kIssuers>(a, ring, reinterpret_cast<uint8_t*>(info), full, empty, ready, pend,
+                                                  idxbuf, true);
     if constexpr (CL) {
       cluster_sync_all();
       cluster_sync_all();
     }
-    return;
-  }
-  if (warp == C::kConsumerWarps) {
-    attn_producer<HKV, kD, kSlots>(a, ring, reinterpret_cast<uint8_t*>(info), full, empty, ready, pend, idxbuf, true);
-    if constexpr (CL) {
-      cluster_sync_all();
-      cluster_sync_all();
-    }
-    return;
-  }
+  } else {
+  if constexpr (C::kRegSplit) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::kHighRegs));
 
   // -------------------------------------------------------------------- consumer warps
   const int g = warp / kBlk;       // KV head
@@ -686,6 +691,7 @@ consumer_tail:
       cluster_sync_all();
     }
   }
+  }   // consumer warps
 }
 #pragma nv_diag_default 177
 
@@ -959,6 +965,21 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
   if (lse && d == 0) lse[static_cast<long long>(b) * Hq + h] = l > 0.f ? (M + __log2f(l)) * kLn2 : -INFINITY;
 }
 
+// With the register split the block must launch with exactly 128 registers a thread: the
+// consumers' setmaxnreg.inc draws on what the launch reserved, and would wait for ever if the
+// issuers' release could not cover it.  A build where ptxas chose fewer is refused, not launched.
+template <int HKV, bool CL>
+cudaError_t check_reg_split() {
+  using C = Cfg<HKV>;
+  if constexpr (C::kRegSplit) {
+    cudaFuncAttributes fa{};
+    const cudaError_t e = cudaFuncGetAttributes(&fa, sparse_attn_kernel<HKV, CL>);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs * C::kThreads != 65536) return cudaErrorInvalidConfiguration;
+  }
+  return cudaSuccess;
+}
+
 template <int HKV>
 cudaError_t launch_attn(const DeviceInfo* di, AttnArgs a, cudaStream_t s) {
   using C = Cfg<HKV>;
@@ -966,6 +987,7 @@ cudaError_t launch_attn(const DeviceInfo* di, AttnArgs a, cudaStream_t s) {
   std::call_once(once[di->device & 63], [] {
     cudaFuncSetAttribute(sparse_attn_kernel<HKV>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   });
+  if (const cudaError_t e = check_reg_split<HKV, false>(); e != cudaSuccess) return e;
   const int grid = std::min(a.num_items, di->num_sms);
   if (grid <= 0) return cudaSuccess;
   sparse_attn_kernel<HKV><<<grid, C::kThreads, C::kSmem, s>>>(a);
@@ -1078,6 +1100,7 @@ cudaError_t launch_attn_cluster(const DeviceInfo* di, AttnArgs a, cudaStream_t s
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if (const cudaError_t e = check_reg_split<HKV, true>(); e != cudaSuccess) return e;
   return cudaLaunchKernelEx(&cfg, sparse_attn_kernel<HKV, true>, a);
 }
 
