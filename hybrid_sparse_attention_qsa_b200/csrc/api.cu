@@ -111,6 +111,8 @@ const DeviceInfo* device_info() {
 
 KernelCtl kernel_ctl(const DeviceInfo* di) { return KernelCtl{di->status, g_wait_ns.load()}; }
 
+int attn_path() { return g_attn_path.load(); }
+
 }  // namespace qsa
 
 using namespace qsa;
@@ -446,17 +448,65 @@ qsa_status_t qsa_sparse_attn_prefill_ws(const void* q, const void* k, const void
   if (!di) return QSA_ERR_CUDA;
   // Automatic choice: row by row.  On the measured workloads (random queries, whose consecutive
   // rows share little of their selections: the union of 16 rows is 0.38-0.46 of their lists) the
-  // row kernel is the faster one; the query tiles are chosen with qsa_set_attn_options.
+  // row kernel is the faster one; the query tiles are chosen with qsa_set_attn_options.  When the
+  // workspace holds K and V interleaved by block (and the shape is the 16-slot kernel's), the
+  // automatic choice first interleaves the positions the rows can see and gathers each block's K
+  // and V with one copy: 4 KB copies instead of two of 2 KB, a higher per-SM gather rate.
   const int path = g_attn_path.load();
   const bool tiles_ok = attn_tc_supported(Hq, Hkv, D, k_blocks) && path == 2 && workspace != nullptr &&
                         ok_ptr(workspace) && ws_bytes >= 512 + attn_tc_tile_bytes(k_blocks);
   if (path == 2 && !tiles_ok)
     return attn_tc_supported(Hq, Hkv, D, k_blocks) ? QSA_ERR_WORKSPACE_TOO_SMALL : QSA_ERR_UNSUPPORTED;
+  if (path == 0 && attn_kv_supported(Hq, Hkv, D) && workspace != nullptr && ok_ptr(workspace) &&
+      ws_bytes >= attn_kv_bytes(B, Tk, Hkv, D)) {
+    const long long j1 = (q_pos0 + Tq + 3) / 4;
+    cudaError_t e = launch_interleave_kv(di, k, v, workspace, B, Tk, Hkv, D, 0, j1, S(stream));
+    if (e == cudaSuccess)
+      e = launch_attn_prefill_kv(di, q, workspace, idx, B, Tq, Tk, Hq, Hkv, k_blocks, q_pos0, scale, out, lse,
+                                 S(stream));
+    return cuda_status(e);
+  }
   if (!tiles_ok)
     return cuda_status(
         launch_attn_prefill(di, q, k, v, idx, B, Tq, Tk, Hq, Hkv, D, k_blocks, q_pos0, scale, out, lse, S(stream)));
   return cuda_status(launch_attn_prefill_tc(di, q, k, v, idx, B, Tq, Tk, Hq, Hkv, k_blocks, q_pos0, scale, out, lse,
                                             workspace, ws_bytes, S(stream)));
+}
+
+qsa_status_t qsa_interleave_kv(const void* k, const void* v, void* kv, int B, int Tk, int Hkv, int D, int blk,
+                               int64_t pos_lo, int64_t pos_hi, void* stream) {
+  QSA_NVTX();
+  if (blk != 4 || B < 0 || Tk < 0 || pos_lo < 0 || pos_lo > pos_hi || pos_hi > Tk) return QSA_ERR_INVALID_ARGUMENT;
+  if (D != 128 || (Hkv != 1 && Hkv != 2)) return QSA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * (pos_hi - pos_lo) == 0) return QSA_OK;
+  if (!ok_ptr(k) || !ok_ptr(v) || !ok_ptr(kv) || B > 65535) return QSA_ERR_INVALID_ARGUMENT;
+  const DeviceInfo* di = device_info();
+  if (!di) return QSA_ERR_CUDA;
+  return cuda_status(launch_interleave_kv(di, k, v, kv, B, Tk, Hkv, D, pos_lo / 4, (pos_hi + 3) / 4, S(stream)));
+}
+
+qsa_status_t qsa_sparse_attn_prefill_kv(const void* q, const void* kv, const int32_t* idx, int B, int Tq, int Tk,
+                                        int Hq, int Hkv, int D, int k_blocks, int blk, int64_t q_pos0, float scale,
+                                        void* out, float* lse, void* stream) {
+  QSA_NVTX();
+  qsa_status_t st = check_attn_shape(Hq, Hkv, D, blk, k_blocks);
+  if (st != QSA_OK) return st;
+  if (!attn_kv_supported(Hq, Hkv, D)) return QSA_ERR_UNSUPPORTED;
+  if (B < 0 || Tq < 0 || Tk < 0 || q_pos0 < 0 || q_pos0 + Tq > Tk) return QSA_ERR_INVALID_ARGUMENT;
+  if (static_cast<long long>(B) * Tq == 0) return QSA_OK;
+  if (!ok_ptr(q) || !ok_ptr(kv) || !ok_ptr(out) || (k_blocks > 0 && idx == nullptr)) return QSA_ERR_INVALID_ARGUMENT;
+  if (static_cast<long long>(B) * Tq > 0x7fffffffLL) return QSA_ERR_UNSUPPORTED;
+  const DeviceInfo* di = device_info();
+  if (!di) return QSA_ERR_CUDA;
+  return cuda_status(
+      launch_attn_prefill_kv(di, q, kv, idx, B, Tq, Tk, Hq, Hkv, k_blocks, q_pos0, scale, out, lse, S(stream)));
+}
+
+size_t qsa_attn_prefill_workspace_size(int B, int Tq, int Tk, int Hq, int Hkv, int D, int k_blocks) {
+  if (B < 0 || Tq < 0 || Tk < 0 || Hq < 1 || Hkv < 1 || D < 1 || k_blocks < 1) return 0;
+  size_t n = qsa_workspace_size(QSA_OP_SPARSE_ATTN_PREFILL, B, Tq, 0, k_blocks, Hq, D, 0);
+  if (attn_kv_supported(Hq, Hkv, D)) n = std::max(n, attn_kv_bytes(B, Tk, Hkv, D));
+  return n;
 }
 
 qsa_status_t qsa_set_attn_options(int path) {

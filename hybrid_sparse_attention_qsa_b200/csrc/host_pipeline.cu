@@ -20,8 +20,11 @@
 // one call), selection chunks on multiples of 4.
 //
 // The steps are the library's own entry points (qsa_pool_block_keys_rope, qsa_rope_index_queries_rope,
-// qsa_select_topk, qsa_sparse_attn_prefill_ws); this file only moves data and orders streams.
-// Copies are one cudaMemcpyAsync per contiguous range.
+// qsa_select_topk, and qsa_interleave_kv + qsa_sparse_attn_prefill_kv, or qsa_sparse_attn_prefill_ws);
+// this file only moves data and orders streams.  With the automatic attention path and a shape the
+// interleaved-K/V attention takes, each chunk interleaves only the K/V positions that arrived with
+// it (the block that straddles the previous chunk's end is rewritten whole), so K and V are
+// interleaved once per call, not once per chunk.  Copies are one cudaMemcpyAsync per contiguous range.
 #include <algorithm>
 #include <cmath>
 #include <mutex>
@@ -60,7 +63,7 @@ void chunk_bounds(const Shape& s, std::vector<int>& att, std::vector<int>& sel) 
 
 // Byte offsets of the regions of the device scratch buffer (each 256-byte aligned).
 struct Layout {
-  size_t q, k, v, qi, ki, kp, qr, out, idx, lse, sel_ws, att_ws, total;
+  size_t q, k, v, qi, ki, kp, qr, out, idx, lse, sel_ws, att_ws, kv, total;
   size_t sel_ws_bytes, att_ws_bytes;
 };
 
@@ -100,6 +103,7 @@ Layout layout(const Shape& s) {
   L.att_ws_bytes = aws;
   L.sel_ws = take(L.sel_ws_bytes);
   L.att_ws = take(L.att_ws_bytes);
+  L.kv = attn_kv_supported(s.Hq, s.Hkv, s.D) ? take(attn_kv_bytes(s.B, s.Tk, s.Hkv, s.D)) : 0;
   L.total = off;
   return L;
 }
@@ -194,6 +198,9 @@ qsa_status_t qsa_prefill_host(const void* q_h, const void* k_h, const void* v_h,
   float* lse_d = lse_out ? lse_out : reinterpret_cast<float*>(base + L.lse);
   void* sel_ws = base + L.sel_ws;
   void* att_ws = base + L.att_ws;
+  const bool use_kv = attn_path() == 0 && attn_kv_supported(Hq, Hkv, D);
+  void* kv_d = base + L.kv;
+  long long kv_done_i = 0;   // positions interleaved so far (the block holding it is rewritten next)
   const char* qh = static_cast<const char*>(q_h);
   const char* kh = static_cast<const char*>(k_h);
   const char* vh = static_cast<const char*>(v_h);
@@ -278,9 +285,20 @@ qsa_status_t qsa_prefill_host(const void* q_h, const void* k_h, const void* v_h,
     if (cudaError_t e = cudaStreamWaitEvent(main, ev_arr[c], 0); e != cudaSuccess) return cuda_st(e);
     // B > 1: one chunk covering every row of every sequence
     const size_t r0 = static_cast<size_t>(lo);
-    qsa_status_t r = qsa_sparse_attn_prefill_ws(q_d + r0 * Hq * D, k_d, v_d, idx_d + r0 * k_blocks, B, hi - lo, Tk,
-                                                Hq, Hkv, D, k_blocks, blk, q_pos0 + lo, scale, out_d + r0 * Hq * D,
-                                                lse_d + r0 * Hq, att_ws, L.att_ws_bytes, stream);
+    qsa_status_t r;
+    if (use_kv) {
+      const long long kv_end = c == n - 1 ? Tk : std::min<long long>(Tk, q_pos0 + hi);
+      r = qsa_interleave_kv(k_d, v_d, kv_d, B, Tk, Hkv, D, blk, kv_done_i, kv_end, stream);
+      kv_done_i = kv_end;
+      if (r == QSA_OK)
+        r = qsa_sparse_attn_prefill_kv(q_d + r0 * Hq * D, kv_d, idx_d + r0 * k_blocks, B, hi - lo, Tk, Hq, Hkv, D,
+                                       k_blocks, blk, q_pos0 + lo, scale, out_d + r0 * Hq * D, lse_d + r0 * Hq,
+                                       stream);
+    } else {
+      r = qsa_sparse_attn_prefill_ws(q_d + r0 * Hq * D, k_d, v_d, idx_d + r0 * k_blocks, B, hi - lo, Tk, Hq, Hkv, D,
+                                     k_blocks, blk, q_pos0 + lo, scale, out_d + r0 * Hq * D, lse_d + r0 * Hq, att_ws,
+                                     L.att_ws_bytes, stream);
+    }
     if (r != QSA_OK) return r;
     cudaError_t e = cudaEventRecord(ev_out[c], main);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(st.cout, ev_out[c], 0);

@@ -29,6 +29,8 @@ struct DeviceInfo {
 // Per-device cached attributes of the current device (nullptr on a runtime error).
 const DeviceInfo* device_info();
 KernelCtl kernel_ctl(const DeviceInfo* di);
+// The prefill attention path chosen with qsa_set_attn_options (0 automatic, 1 rows, 2 tiles).
+int attn_path();
 
 // Rotary parameters of the indexer (theta <= 0: no rotation); factor > 1 turns on YaRN scaling
 // with the given original context, ramp bounds and magnitude factor (already resolved).
@@ -94,6 +96,16 @@ cudaError_t launch_topk_fallback(const DeviceInfo* di, const void* qi, const voi
 cudaError_t launch_attn_prefill(const DeviceInfo* di, const void* q, const void* k, const void* v, const int32_t* idx,
                                 int B, int Tq, int Tk, int Hq, int Hkv, int D, int k_blocks, long long q_pos0,
                                 float scale, void* out, float* lse, cudaStream_t s);
+// Row-by-row prefill attention over K and V interleaved by block (kv [B][ceil(Tk/4)][2][4][Hkv][D]:
+// one copy fetches a block's K and V): D = 128, Hkv in {1, 2}, groups of up to 8 query heads.
+bool attn_kv_supported(int Hq, int Hkv, int D);
+size_t attn_kv_bytes(int B, int Tk, int Hkv, int D);
+// Writes the interleaved blocks [j0, j1) of every sequence from k and v ([B][Tk][Hkv][D]).
+cudaError_t launch_interleave_kv(const DeviceInfo* di, const void* k, const void* v, void* kv, int B, int Tk, int Hkv,
+                                 int D, long long j0, long long j1, cudaStream_t s);
+cudaError_t launch_attn_prefill_kv(const DeviceInfo* di, const void* q, const void* kv, const int32_t* idx, int B,
+                                   int Tq, int Tk, int Hq, int Hkv, int k_blocks, long long q_pos0, float scale,
+                                   void* out, float* lse, cudaStream_t s);
 // Query-tile prefill attention on tcgen05 (sparse_attn_tc.cu): D = 128, groups of 8 query heads,
 // k_blocks <= 1024.  The workspace holds the tile unions of as many 16-row tiles as fit (at least
 // one: 256 + attn_tc_tile_bytes(k_blocks) bytes); the call walks the tiles in ranges of that many.

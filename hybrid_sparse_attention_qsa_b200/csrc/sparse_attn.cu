@@ -59,22 +59,29 @@ struct StageInfo {
 
 // Shared-memory ring of the copy pipeline: per stage SLOTS block slots of K, then SLOTS of V.  A
 // block of 4 tokens of all KV heads is one contiguous run of kBlockBytes in the [T][Hkv][D] layout.
-template <int HKV, int D, int SLOTS, int ISS = kIssuers_>
+// KVI: K and V interleaved by block in memory ([B][ceil(T/4)][K, V][4][Hkv][D]), so a block's K
+// and V are one contiguous run of 2 * kBlockBytes, fetched by one copy into a slot that holds the
+// block's K followed by its V.
+template <int HKV, int D, int SLOTS, int ISS = kIssuers_, bool KVI = false>
 struct Ring {
   static_assert(SLOTS % ISS == 0 && SLOTS <= 16, "slots per issuer warp");
+  static constexpr bool kKVI = KVI;
   static constexpr int kSlots = SLOTS;
   static constexpr int kTokBytes = HKV * D * 2;               // one token of K (or V), all KV heads
   static constexpr int kBlockBytes = kBlk * kTokBytes;        // one block of K (or of V)
-  static constexpr int kPitch = kBlockBytes + 16;             // +16: conflict-free ldmatrix across slots
-  static constexpr int kStageBytes = 2 * SLOTS * kPitch;      // K slots, then V slots
+  // +16: the same token row of consecutive slots falls in different 16-byte bank groups
+  static constexpr int kPitch = (KVI ? 2 * kBlockBytes : kBlockBytes) + 16;
+  static constexpr int kVOff = KVI ? kBlockBytes : SLOTS * kPitch;   // from a slot's K to its V
+  static constexpr int kStageBytes = KVI ? SLOTS * kPitch : 2 * SLOTS * kPitch;
   static constexpr int kInfoStride = (sizeof(StageInfo) + 15) / 16 * 16;
 };
 
-template <int HKV>
+template <int HKV, bool KVI = false>
 struct Cfg {
   static constexpr int kBlockBytes = kBlk * HKV * kD * 2;     // one block of K (or of V)
-  static constexpr int kPitch = kBlockBytes + 16;
-  static constexpr int kStageBytes = 2 * kSlots * kPitch;     // K slots, then V slots
+  static constexpr int kPitch = (KVI ? 2 * kBlockBytes : kBlockBytes) + 16;
+  static constexpr int kVOff = KVI ? kBlockBytes : kSlots * kPitch;
+  static constexpr int kStageBytes = KVI ? kSlots * kPitch : 2 * kSlots * kPitch;
   static constexpr int kConsumerWarps = kBlk * HKV;
   // 8 issuing warps: the per-SM rate of 1-D bulk copies grows with the warps issuing them (the
   // gather probe: 12.5 TB/s from L2 with 4 warps, 13.9 with 8, same ring)
@@ -101,6 +108,7 @@ struct AttnArgs {
   const uint16_t* k;
   const uint16_t* v;
   const int32_t* idx;
+  const uint16_t* kv;       // K and V interleaved by block (KVI kernels), else unused
   const int32_t* seqlens;   // decode when non-null
   uint16_t* out;
   float* lse;
@@ -140,8 +148,14 @@ __device__ __forceinline__ Item make_item(const AttnArgs& a, int i) {
     it.qrow = static_cast<long long>(b) * a.Tq + t;
     it.orow = it.qrow;
     it.pos = a.q_pos0 + t;
-    it.kbase = a.k + static_cast<long long>(b) * a.Tk * HKV * D;
-    it.vbase = a.v + static_cast<long long>(b) * a.Tk * HKV * D;
+    if (a.kv) {   // interleaved: blocks of [K 4 tokens][V 4 tokens]
+      const long long nblk = (a.Tk + kBlk - 1) / kBlk;
+      it.kbase = a.kv + static_cast<long long>(b) * nblk * 2 * kBlk * HKV * D;
+      it.vbase = it.kbase + kBlk * HKV * D;
+    } else {
+      it.kbase = a.k + static_cast<long long>(b) * a.Tk * HKV * D;
+      it.vbase = a.v + static_cast<long long>(b) * a.Tk * HKV * D;
+    }
     it.idx_row = a.idx + it.qrow * a.kblocks;
     it.lo = 0;
     it.hi = a.kblocks;
@@ -169,10 +183,30 @@ __device__ __forceinline__ Item make_item(const AttnArgs& a, int i) {
 
 // Helper issuer warp h (1 .. kIssuers_ - 1): issues slots h, h + kIssuers_, ... of every stage the
 // leading producer publishes, until it publishes nslots == -1.
-template <int HKV, int D, int SLOTS, int ISS = kIssuers_>
+// Copies of one slot: the block's K and V rows [tok0, tok0 + ntok) into kd and vd.  KVI: kbase is the
+// interleaved block array (vbase = kbase + one block of K); a whole block is one copy of its K and V.
+template <class R, int HKV, int D>
+__device__ __forceinline__ void copy_slot(uint8_t* kd, uint8_t* vd, const uint16_t* kbase, const uint16_t* vbase,
+                                          long long tok0, int ntok, uint64_t* bar) {
+  const uint32_t bytes = static_cast<uint32_t>(ntok) * R::kTokBytes;
+  if constexpr (R::kKVI) {
+    const uint16_t* src = kbase + (tok0 / kBlk) * (2 * kBlk * HKV * D);
+    if (ntok == kBlk) {
+      bulk_g2s(kd, src, 2 * bytes, bar);
+    } else {
+      bulk_g2s(kd, src, bytes, bar);
+      bulk_g2s(vd, src + kBlk * HKV * D, bytes, bar);
+    }
+  } else {
+    bulk_g2s(kd, kbase + tok0 * HKV * D, bytes, bar);
+    bulk_g2s(vd, vbase + tok0 * HKV * D, bytes, bar);
+  }
+}
+
+template <int HKV, int D, int SLOTS, int ISS = kIssuers_, bool KVI = false>
 __device__ __forceinline__ void attn_helper(const AttnArgs& a, int h, uint8_t* ring, uint8_t* info, uint64_t* full,
                                             uint64_t* ready) {
-  using R = Ring<HKV, D, SLOTS, ISS>;
+  using R = Ring<HKV, D, SLOTS, ISS, KVI>;
   const int lane = threadIdx.x & 31;
   auto info_at = [&](int s) { return reinterpret_cast<const StageInfo*>(info + s * R::kInfoStride); };
   // ------------------------------------------------------------------ helper issuer warps
@@ -191,10 +225,9 @@ __device__ __forceinline__ void attn_helper(const AttnArgs& a, int h, uint8_t* r
       const int ntok = inf->ntok[slot];
       const long long tok0 = inf->tok0[slot];
       uint8_t* kd = ring + st * R::kStageBytes + slot * R::kPitch;
-      uint8_t* vd = kd + R::kSlots * R::kPitch;
+      uint8_t* vd = kd + R::kVOff;
       if (QSA_DCHECK(a.ctl, tok0 >= 0 && ntok <= kBlk && tok0 + ntok <= a.Tk)) {
-        bulk_g2s(kd, inf->kbase + tok0 * HKV * D, ntok * tok_bytes, &full[st]);
-        bulk_g2s(vd, inf->vbase + tok0 * HKV * D, ntok * tok_bytes, &full[st]);
+        copy_slot<R, HKV, D>(kd, vd, inf->kbase, inf->vbase, tok0, ntok, &full[st]);
       } else {
         mbar_complete_tx(&full[st], 2u * ntok * tok_bytes);
       }
@@ -225,11 +258,11 @@ __device__ __forceinline__ void attn_fetch_list(const AttnArgs& a, int item, int
 // query's own block last), publishes each stage's slot list for the helpers and issues its own
 // share of the copies.  Returns only when no copy it registered is still in flight.  With
 // `prefetched` the first segment of the CTA's first item is already on its way (attn_fetch_list).
-template <int HKV, int D, int SLOTS, int ISS = kIssuers_>
+template <int HKV, int D, int SLOTS, int ISS = kIssuers_, bool KVI = false>
 __device__ __forceinline__ void attn_producer(const AttnArgs& a, uint8_t* ring, uint8_t* info, uint64_t* full,
                                               uint64_t* empty, uint64_t* ready, int* pend, int* idxbuf,
                                               bool prefetched = false) {
-  using R = Ring<HKV, D, SLOTS, ISS>;
+  using R = Ring<HKV, D, SLOTS, ISS, KVI>;
   const int lane = threadIdx.x & 31;
   auto info_at = [&](int s) { return reinterpret_cast<StageInfo*>(info + s * R::kInfoStride); };
   // ------------------------------------------------------------------ leading producer warp
@@ -264,10 +297,9 @@ __device__ __forceinline__ void attn_producer(const AttnArgs& a, uint8_t* ring, 
     __syncwarp();
     if (lane < n && lane % ISS == 0) {
       uint8_t* kd = ring + st * R::kStageBytes + lane * R::kPitch;
-      uint8_t* vd = kd + R::kSlots * R::kPitch;
+      uint8_t* vd = kd + R::kVOff;
       if (QSA_DCHECK(a.ctl, tok0 >= 0 && ntok <= kBlk && tok0 + ntok <= a.Tk)) {
-        bulk_g2s(kd, it.kbase + tok0 * HKV * D, ntok * tok_bytes, &full[st]);
-        bulk_g2s(vd, it.vbase + tok0 * HKV * D, ntok * tok_bytes, &full[st]);
+        copy_slot<R, HKV, D>(kd, vd, it.kbase, it.vbase, tok0, ntok, &full[st]);
       } else {
         mbar_complete_tx(&full[st], 2u * ntok * tok_bytes);
       }
@@ -358,9 +390,9 @@ __device__ __forceinline__ void attn_producer(const AttnArgs& a, uint8_t* ring, 
 // instantiation, so that the prefill and split-partials code is compiled without it; there the
 // label of the cluster tail has no jump to it).
 #pragma nv_diag_suppress 177
-template <int HKV, bool CL = false>
-__global__ void __launch_bounds__(Cfg<HKV>::kThreads, 1) sparse_attn_kernel(AttnArgs a) {
-  using C = Cfg<HKV>;
+template <int HKV, bool CL = false, bool KVI = false>
+__global__ void __launch_bounds__(Cfg<HKV, KVI>::kThreads, 1) sparse_attn_kernel(AttnArgs a) {
+  using C = Cfg<HKV, KVI>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
   uint8_t* ring = smem;
@@ -396,10 +428,11 @@ __global__ void __launch_bounds__(Cfg<HKV>::kThreads, 1) sparse_attn_kernel(Attn
   // Zero the V slots once so that unused slot rows are finite (their probabilities are 0, but
   // 0 * NaN = NaN).  Unused K rows need no zeroing: their scores are replaced by -inf (a select,
   // no arithmetic on them).
-  constexpr int kVChunks = kSlots * C::kPitch / 16;   // 16-byte chunks of one stage's V slots
-  for (int i = threadIdx.x; i < kStages * kVChunks; i += blockDim.x) {
-    const int s = i / kVChunks, c = i - s * kVChunks;
-    reinterpret_cast<uint4*>(ring + s * C::kStageBytes + kSlots * C::kPitch)[c] = make_uint4(0, 0, 0, 0);
+  constexpr int kVChunks = C::kBlockBytes / 16;   // 16-byte chunks of one slot's V block
+  for (int i = threadIdx.x; i < kStages * kSlots * kVChunks; i += blockDim.x) {
+    const int s = i / (kSlots * kVChunks), r = i - s * (kSlots * kVChunks), slot = r / kVChunks;
+    reinterpret_cast<uint4*>(ring + s * C::kStageBytes + slot * C::kPitch + C::kVOff)[r - slot * kVChunks] =
+        make_uint4(0, 0, 0, 0);
   }
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // order these writes before the bulk copies
   __syncthreads();
@@ -409,11 +442,11 @@ __global__ void __launch_bounds__(Cfg<HKV>::kThreads, 1) sparse_attn_kernel(Attn
   if (warp >= C::kConsumerWarps) {
     if constexpr (C::kRegSplit) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::kLowRegs));
     if (warp > C::kConsumerWarps)
-      attn_helper<HKV, kD, kSlots, C::kIssuers>(a, warp - C::kConsumerWarps, ring, reinterpret_cast<uint8_t*>(info),
-                                                full, ready);
+      attn_helper<HKV, kD, kSlots, C::kIssuers, KVI>(a, warp - C::kConsumerWarps, ring,
+                                                     reinterpret_cast<uint8_t*>(info), full, ready);
     else
-      attn_producer<HKV, kD, kSlots, C::kIssuers>(a, ring, reinterpret_cast<uint8_t*>(info), full, empty, ready, pend,
-                                                  idxbuf, true);
+      attn_producer<HKV, kD, kSlots, C::kIssuers, KVI>(a, ring, reinterpret_cast<uint8_t*>(info), full, empty, ready,
+                                                       pend, idxbuf, true);
     if constexpr (CL) {
       cluster_sync_all();
       cluster_sync_all();
@@ -474,7 +507,7 @@ __global__ void __launch_bounds__(Cfg<HKV>::kThreads, 1) sparse_attn_kernel(Attn
       const bool last = info_at(st)->last != 0;
       if (ns > 0) {
         const uint32_t kst = ring_u32 + st * C::kStageBytes;
-        const uint32_t vst = kst + kSlots * C::kPitch;
+        const uint32_t vst = kst + C::kVOff;
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
@@ -968,30 +1001,48 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
 // With the register split the block must launch with exactly 128 registers a thread: the
 // consumers' setmaxnreg.inc draws on what the launch reserved, and would wait for ever if the
 // issuers' release could not cover it.  A build where ptxas chose fewer is refused, not launched.
-template <int HKV, bool CL>
+template <int HKV, bool CL, bool KVI = false>
 cudaError_t check_reg_split() {
-  using C = Cfg<HKV>;
+  using C = Cfg<HKV, KVI>;
   if constexpr (C::kRegSplit) {
     cudaFuncAttributes fa{};
-    const cudaError_t e = cudaFuncGetAttributes(&fa, sparse_attn_kernel<HKV, CL>);
+    const cudaError_t e = cudaFuncGetAttributes(&fa, sparse_attn_kernel<HKV, CL, KVI>);
     if (e != cudaSuccess) return e;
     if (fa.numRegs * C::kThreads != 65536) return cudaErrorInvalidConfiguration;
   }
   return cudaSuccess;
 }
 
-template <int HKV>
+template <int HKV, bool KVI = false>
 cudaError_t launch_attn(const DeviceInfo* di, AttnArgs a, cudaStream_t s) {
-  using C = Cfg<HKV>;
+  using C = Cfg<HKV, KVI>;
   static std::once_flag once[64];
   std::call_once(once[di->device & 63], [] {
-    cudaFuncSetAttribute(sparse_attn_kernel<HKV>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    cudaFuncSetAttribute(sparse_attn_kernel<HKV, false, KVI>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   });
-  if (const cudaError_t e = check_reg_split<HKV, false>(); e != cudaSuccess) return e;
+  if (const cudaError_t e = check_reg_split<HKV, false, KVI>(); e != cudaSuccess) return e;
   const int grid = std::min(a.num_items, di->num_sms);
   if (grid <= 0) return cudaSuccess;
-  sparse_attn_kernel<HKV><<<grid, C::kThreads, C::kSmem, s>>>(a);
+  sparse_attn_kernel<HKV, false, KVI><<<grid, C::kThreads, C::kSmem, s>>>(a);
   return cudaPeekAtLastError();
+}
+
+// K and V interleaved by block: kv[b][j][0] = k[b][4j .. 4j+3], kv[b][j][1] = v[b][4j .. 4j+3]
+// ([4][Hkv][D] each), positions >= Tk zero.  One CTA per (block, sequence), one 16-byte chunk per
+// thread: thread w copies chunk w of the block, i.e. part w >> (2 + lg) (K or V), token
+// (w >> lg) & 3, chunk w & (2^lg - 1) of the token (2^lg chunks per token of all KV heads).
+__global__ void __launch_bounds__(256) interleave_kv_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
+                                                            uint4* __restrict__ kv, int Tk, int lg, long long j0) {
+  const long long j = j0 + blockIdx.x;
+  const long long b = blockIdx.y;
+  const long long nblk = (Tk + kBlk - 1) / kBlk;
+  const int w = threadIdx.x;
+  const int which = w >> (2 + lg);
+  const long long t = j * kBlk + ((w >> lg) & 3);
+  const int c = w & ((1 << lg) - 1);
+  uint4 val = make_uint4(0u, 0u, 0u, 0u);
+  if (t < Tk) val = (which ? v : k)[((b * Tk + t) << lg) + c];
+  kv[((b * nblk + j) << (3 + lg)) + w] = val;
 }
 
 template <int HKV, int D, int NSUB>
@@ -1012,6 +1063,7 @@ cudaError_t launch_attn_wide_cfg(const DeviceInfo* di, AttnArgs a, cudaStream_t 
 // the wide one.
 cudaError_t launch_attn_any(const DeviceInfo* di, AttnArgs a, int Hkv, int D, cudaStream_t s) {
   const int group = a.Hq / Hkv;
+  if (a.kv) return Hkv == 1 ? launch_attn<1, true>(di, a, s) : launch_attn<2, true>(di, a, s);
   if (D == kD && group <= 8) return Hkv == 1 ? launch_attn<1>(di, a, s) : launch_attn<2>(di, a, s);
   const int nsub = group <= 8 ? 1 : 2;
   if (D == 128) {
@@ -1047,6 +1099,48 @@ cudaError_t launch_attn_prefill(const DeviceInfo* di, const void* q, const void*
   a.scale_log2 = scale * kLog2e;
   a.ctl = kernel_ctl(di);
   return launch_attn_any(di, a, Hkv, D, s);
+}
+
+bool attn_kv_supported(int Hq, int Hkv, int D) { return D == kD && (Hkv == 1 || Hkv == 2) && Hq / Hkv <= 8; }
+
+size_t attn_kv_bytes(int B, int Tk, int Hkv, int D) {
+  return static_cast<size_t>(B) * ((Tk + kBlk - 1) / kBlk) * 2 * kBlk * Hkv * D * 2;
+}
+
+cudaError_t launch_interleave_kv(const DeviceInfo* di, const void* k, const void* v, void* kv, int B, int Tk, int Hkv,
+                                 int D, long long j0, long long j1, cudaStream_t s) {
+  (void)di;
+  if (j1 <= j0 || B <= 0) return cudaSuccess;
+  const int tok16 = Hkv * D * 2 / 16;   // 16-byte chunks of one token of all KV heads: 16 or 32
+  const int lg = tok16 == 32 ? 5 : 4;
+  if ((1 << lg) != tok16 || j1 - j0 > 0x7fffffffLL || B > 65535) return cudaErrorInvalidValue;
+  interleave_kv_kernel<<<dim3(static_cast<unsigned>(j1 - j0), static_cast<unsigned>(B)), 8 * tok16, 0, s>>>(
+      static_cast<const uint4*>(k), static_cast<const uint4*>(v), static_cast<uint4*>(kv), Tk, lg, j0);
+  return cudaPeekAtLastError();
+}
+
+cudaError_t launch_attn_prefill_kv(const DeviceInfo* di, const void* q, const void* kv, const int32_t* idx, int B,
+                                   int Tq, int Tk, int Hq, int Hkv, int k_blocks, long long q_pos0, float scale,
+                                   void* out, float* lse, cudaStream_t s) {
+  AttnArgs a{};
+  a.q = static_cast<const uint16_t*>(q);
+  a.kv = static_cast<const uint16_t*>(kv);
+  a.idx = idx;
+  a.seqlens = nullptr;
+  a.out = static_cast<uint16_t*>(out);
+  a.lse = lse;
+  a.part = nullptr;
+  a.q_pos0 = q_pos0;
+  a.B = B;
+  a.Tq = Tq;
+  a.Tk = Tk;
+  a.Hq = Hq;
+  a.kblocks = k_blocks;
+  a.splits = 1;
+  a.num_items = B * Tq;
+  a.scale_log2 = scale * kLog2e;
+  a.ctl = kernel_ctl(di);
+  return launch_attn_any(di, a, Hkv, kD, s);
 }
 
 // Split-KV decode as clusters: one CTA per item (B * splits <= SMs), a cluster of `splits` CTAs per

@@ -56,6 +56,9 @@ SIGNATURES = {
     "qsa_sparse_attn_prefill_ws": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I64, _F, _P, _P, _P, _SZ,
                                         _P]),
     "qsa_set_attn_options": (_I, [_I]),
+    "qsa_attn_prefill_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I]),
+    "qsa_interleave_kv": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I64, _I64, _P]),
+    "qsa_sparse_attn_prefill_kv": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I64, _F, _P, _P, _P]),
     "qsa_sparse_attn_decode": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P, _P, _P, _SZ, _P]),
     "qsa_sparse_attn_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P, _P, _P]),
     "qsa_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I, _I]),
@@ -347,9 +350,11 @@ def qsa_sparse_attn_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, i
     """q [B, Tq, Hq, D], k/v [B, Tk, Hkv, D], idx [B, Tq, kb] -> (out [B, Tq, Hq, D], lse [B, Tq, Hq]).
 
     With ``tiles`` (default) the call goes through qsa_sparse_attn_prefill_ws with ``workspace``
-    (allocated here when omitted), which runs the path qsa_set_attn_options chose (automatic: row by
-    row; QSA_ATTN_TILES: query tiles on tcgen05 where the shape allows).  ``tiles=False`` calls
-    qsa_sparse_attn_prefill (row by row, no workspace)."""
+    (allocated here when omitted, qsa_attn_prefill_workspace_size bytes), which runs the path
+    qsa_set_attn_options chose (automatic: row by row over K/V interleaved by block in the
+    workspace where the shape allows; QSA_ATTN_ROWS: row by row over k and v; QSA_ATTN_TILES: query
+    tiles on tcgen05 where the shape allows).  ``tiles=False`` calls qsa_sparse_attn_prefill (row by
+    row, no workspace)."""
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _need(t, torch.bfloat16, n)
     _need(idx, torch.int32, "idx")
@@ -367,12 +372,54 @@ def qsa_sparse_attn_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, i
                "qsa_sparse_attn_prefill")
         return out, lse
     if workspace is None:
-        nbytes = qsa_workspace_size(QSA_OP_SPARSE_ATTN_PREFILL, B, Tq, 0, kb, Hq, D)
+        nbytes = qsa_attn_prefill_workspace_size(B, Tq, Tk, Hq, Hkv, D, kb)
         workspace = _empty(max(nbytes, 16), dtype=torch.uint8, device=q.device, what="attention workspace")
     ws_bytes = workspace.numel() * workspace.element_size()
     _check(lib().qsa_sparse_attn_prefill_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(idx), B, Tq, Tk, Hq, Hkv, D, kb, blk,
                                             q_pos0, scale, _ptr(out), _ptr(lse), _ptr(workspace), ws_bytes,
                                             _stream(q.device)), "qsa_sparse_attn_prefill_ws")
+    return out, lse
+
+
+def qsa_attn_prefill_workspace_size(B: int, Tq: int, Tk: int, Hq: int, Hkv: int, D: int, k_blocks: int) -> int:
+    return int(lib().qsa_attn_prefill_workspace_size(B, Tq, Tk, Hq, Hkv, D, k_blocks))
+
+
+def qsa_interleave_kv(k: torch.Tensor, v: torch.Tensor, kv: torch.Tensor | None = None, *, pos_lo: int = 0,
+                      pos_hi: int | None = None, blk: int = 4) -> torch.Tensor:
+    """k, v [B, Tk, Hkv, D] -> kv [B, ceil(Tk / blk), 2, blk, Hkv, D]: K and V interleaved by block
+    (positions >= Tk zero); writes the blocks holding positions [pos_lo, pos_hi)."""
+    _need(k, torch.bfloat16, "k")
+    _need(v, torch.bfloat16, "v")
+    B, Tk, Hkv, D = k.shape
+    if kv is None:
+        kv = _empty(B, (Tk + blk - 1) // blk, 2, blk, Hkv, D, dtype=torch.bfloat16, device=k.device,
+                    what="interleaved kv")
+    _need(kv, torch.bfloat16, "kv")
+    pos_hi = Tk if pos_hi is None else pos_hi
+    _check(lib().qsa_interleave_kv(_ptr(k), _ptr(v), _ptr(kv), B, Tk, Hkv, D, blk, pos_lo, pos_hi,
+                                   _stream(k.device)), "qsa_interleave_kv")
+    return kv
+
+
+def qsa_sparse_attn_prefill_kv(q: torch.Tensor, kv: torch.Tensor, idx: torch.Tensor, *, Tk: int, q_pos0: int = 0,
+                               scale: float | None = None, out: torch.Tensor | None = None,
+                               lse: torch.Tensor | None = None, blk: int = 4):
+    """qsa_sparse_attn_prefill over kv from qsa_interleave_kv (Tk: the positions of k and v)."""
+    _need(q, torch.bfloat16, "q")
+    _need(kv, torch.bfloat16, "kv")
+    _need(idx, torch.int32, "idx")
+    B, Tq, Hq, D = q.shape
+    Hkv = kv.shape[4]
+    kb = idx.shape[-1]
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    if out is None:
+        out = _empty_like(q, what="out")
+    if lse is None:
+        lse = _empty(B, Tq, Hq, dtype=torch.float32, device=q.device, what="lse")
+    _check(lib().qsa_sparse_attn_prefill_kv(_ptr(q), _ptr(kv), _ptr(idx), B, Tq, Tk, Hq, Hkv, D, kb, blk, q_pos0,
+                                            scale, _ptr(out), _ptr(lse), _stream(q.device)),
+           "qsa_sparse_attn_prefill_kv")
     return out, lse
 
 

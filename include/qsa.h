@@ -268,12 +268,17 @@ QSA_API qsa_status_t qsa_sparse_attn_prefill(const void* q, const void* k, const
  * masks out the union blocks it did not list ("Qwen3.8-Flash-Next architecture" (flozi.net), "Der
  * Weg eines Tokens durch das Modell", item 2: exact attention over the selected tokens;
  * consecutive queries select overlapping blocks).  The result is the same exact attention up to
- * fp32 summation order.  Index lists must be ascending with -1 padding last (as qsa_select_topk
- * writes them); other orders are accepted and cost a full sort per tile.  A non-finite K/V value in
+ * fp32 summation order.  The order of the entries in a list does not matter.  A non-finite K/V value in
  * a block that one row of a tile lists reaches the other rows of the tile (0 * inf); positions
- * past the call's last query are never read.  Other shapes, or no workspace, run the row-by-row
- * kernel of qsa_sparse_attn_prefill.  Calls with more tiles than the workspace holds are processed
- * in ranges of tiles.
+ * past the call's last query are never read.  Calls with more tiles than the workspace holds are
+ * processed in ranges of tiles.
+ * The automatic choice (qsa_set_attn_options(0)) runs row by row; when the shape is one that
+ * qsa_sparse_attn_prefill_kv takes and the workspace holds K and V interleaved by block
+ * (ws_bytes >= B * ceil(Tk / 4) * 2 * 4 * Hkv * D * 2; qsa_attn_prefill_workspace_size covers it),
+ * it first writes the interleaved blocks of the positions the rows can see (qsa_interleave_kv)
+ * into the workspace and then runs qsa_sparse_attn_prefill_kv: the same result bit for bit, with
+ * each block's K and V fetched by one copy.  Otherwise, and with qsa_set_attn_options(1), it runs
+ * the row-by-row kernel of qsa_sparse_attn_prefill.
  */
 QSA_API qsa_status_t qsa_sparse_attn_prefill_ws(const void* q, const void* k, const void* v,
                                         const int32_t* idx, int B, int Tq, int Tk, int Hq, int Hkv,
@@ -282,8 +287,41 @@ QSA_API qsa_status_t qsa_sparse_attn_prefill_ws(const void* q, const void* k, co
                                         void* stream);
 
 /*
+ * Bytes of workspace with which qsa_sparse_attn_prefill_ws can take every path it has for these
+ * sizes: the query-tile unions (up to 4096 tiles) and, for the shapes of
+ * qsa_sparse_attn_prefill_kv, K and V interleaved by block.  0 for invalid sizes.
+ */
+QSA_API size_t qsa_attn_prefill_workspace_size(int B, int Tq, int Tk, int Hq, int Hkv, int D, int k_blocks);
+
+/*
+ * K and V interleaved by micro-block, the layout qsa_sparse_attn_prefill_kv reads.  (The pages have
+ * no counterpart: a layout for the attention's gather, "Qwen3.8-Flash-Next architecture"
+ * (flozi.net), "Der Weg eines Tokens durch das Modell", item 2.)
+ *   k, v [B][Tk][Hkv][D] bf16  ->  kv [B][ceil(Tk/blk)][2][blk][Hkv][D] bf16
+ *   kv[b][j][0][i] = k[b][blk*j + i], kv[b][j][1][i] = v[b][blk*j + i]; positions >= Tk are zero.
+ * Writes the blocks that hold positions [pos_lo, pos_hi) (0 <= pos_lo <= pos_hi <= Tk; a block is
+ * rewritten whole, so a block that straddles pos_hi also receives the positions after pos_hi that
+ * it holds, read from k and v as they are).  D = 128, Hkv in {1, 2}, blk = 4.
+ * Errors: INVALID_ARGUMENT (null or misaligned pointer, sizes, blk), UNSUPPORTED (D, Hkv).
+ */
+QSA_API qsa_status_t qsa_interleave_kv(const void* k, const void* v, void* kv, int B, int Tk, int Hkv, int D,
+                                       int blk, int64_t pos_lo, int64_t pos_hi, void* stream);
+
+/*
+ * qsa_sparse_attn_prefill over K and V interleaved by block (kv as qsa_interleave_kv writes it, for
+ * at least the positions < q_pos0 + Tq): the same arguments otherwise, the same result bit for bit.
+ * A block's K and V are one contiguous run, fetched with one copy.  D = 128, Hkv in {1, 2}, groups
+ * of up to 8 query heads; other shapes return UNSUPPORTED.
+ */
+QSA_API qsa_status_t qsa_sparse_attn_prefill_kv(const void* q, const void* kv, const int32_t* idx, int B, int Tq,
+                                                int Tk, int Hq, int Hkv, int D, int k_blocks, int blk,
+                                                int64_t q_pos0, float scale, void* out, float* lse,
+                                                void* stream);
+
+/*
  * Chooses the prefill attention of qsa_sparse_attn_prefill_ws for all later calls from this
- * process: 0 = automatic (row by row), 1 = row by row, 2 = query tiles (UNSUPPORTED for other
+ * process: 0 = automatic (row by row, over interleaved K/V when the workspace holds them), 1 = row by
+ * row over k and v as given, 2 = query tiles (UNSUPPORTED for other
  * shapes, WORKSPACE_TOO_SMALL without room for one tile).  Errors: INVALID_ARGUMENT (path outside
  * 0..2).
  */
