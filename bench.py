@@ -44,9 +44,10 @@ DECODE = "decode_256k"
 # line reports traffic as null until the kernel is captured again.
 TRAFFIC_PROFILES = {"prefill_128k": ("profiles/sparse_attn_prefill_128k.md",
                                      "hybrid_sparse_attention_qsa_b200/csrc/sparse_attn.cu")}
-# The attention's gather: every selected 4-token block of K and of V is one chunk of
-# blk * Hkv * D * 2 bytes, fetched by 8 issuing warps into a 3-stage ring of 16 slots (K and V).
-GATHER_PROBE = dict(issuer_warps=8, stages=3, slots_per_warp=4)
+# The attention's gather: K and V interleaved by block, every selected 4-token block is one chunk of
+# 2 * blk * Hkv * D * 2 bytes (its K then its V), fetched by 8 issuing warps into a 3-stage ring of
+# 16 slots: 48 chunks of 4 KB in flight.
+GATHER_PROBE = dict(issuer_warps=8, stages=3, slots_per_warp=2)
 
 
 # ------------------------------------------------------------------------------------------- helpers
@@ -105,15 +106,23 @@ def unique_kv_bytes(w) -> int:
 
 
 def gather_ceiling(dev, stream, w, sweep: bool = False) -> dict:
-    """The measured ceiling of the attention's gather: 1-D bulk copies of one block of K (or V) from
-    random offsets of an L2-resident 32 MiB buffer into the same ring the attention kernel keeps in
-    flight, and of a 4 GiB buffer (HBM).  GB/s of delivered bytes, best of 3 timed launches."""
+    """The measured ceiling of the attention's gather: 1-D bulk copies of one block of K and V (4 KB,
+    the interleaved layout the kernel reads) from random offsets of an L2-resident 32 MiB buffer into
+    the same ring the attention kernel keeps in flight, and of a 4 GiB buffer (HBM); for comparison
+    the same ring in 2 KB chunks (K and V of a block fetched separately, 8 and 4 warps) and with
+    plain loads.  GB/s of delivered bytes, best of 3 timed launches."""
     import hybrid_sparse_attention_qsa_b200 as Q
-    chunk = w.blk * w.Hkv * w.D * 2
-    res = {"chunk_bytes": chunk, "config": dict(GATHER_PROBE)}
-    narrow = dict(issuer_warps=4, stages=3, slots_per_warp=8)   # the same ring, issued by 4 warps
-    cases = [("l2_bulk", 32 << 20, 0, GATHER_PROBE), ("l2_bulk_w4", 32 << 20, 0, narrow),
-             ("hbm_bulk", 4 << 30, 0, GATHER_PROBE), ("l2_lsu", 32 << 20, 1, GATHER_PROBE)]
+    if kv_interleaved(w):
+        chunk, cfg0 = 2 * w.blk * w.Hkv * w.D * 2, dict(GATHER_PROBE)
+        half = dict(issuer_warps=8, stages=3, slots_per_warp=4, chunk_bytes=chunk // 2)
+        half4 = dict(issuer_warps=4, stages=3, slots_per_warp=8, chunk_bytes=chunk // 2)
+        extra = [("l2_bulk_half", 32 << 20, 0, half), ("l2_bulk_half_w4", 32 << 20, 0, half4)]
+    else:   # the wide kernel: K and V blocks fetched separately by 4 warps, 8 slots a stage
+        chunk, cfg0 = w.blk * w.Hkv * w.D * 2, dict(issuer_warps=4, stages=3, slots_per_warp=4)
+        extra = []
+    res = {"chunk_bytes": chunk, "config": dict(cfg0)}
+    cases = [("l2_bulk", 32 << 20, 0, cfg0)] + extra + [("hbm_bulk", 4 << 30, 0, cfg0),
+                                                        ("l2_lsu", 32 << 20, 1, cfg0)]
     if sweep:
         for iw, sl in ((1, 32), (2, 16), (8, 4), (8, 3), (12, 2), (16, 2)):
             cfg = dict(issuer_warps=iw, stages=3, slots_per_warp=sl)
@@ -152,9 +161,16 @@ def gather_ceiling(dev, stream, w, sweep: bool = False) -> dict:
     return res
 
 
+def kv_interleaved(w) -> bool:
+    """Whether the automatic attention path reads K and V interleaved by block for this shape."""
+    return w.D == 128 and w.Hkv in (1, 2) and w.Hq // w.Hkv <= 8
+
+
 def attn_kernel_name(w) -> str:
     """The attention kernel the library launches for this shape."""
     group = w.Hq // w.Hkv
+    if kv_interleaved(w):
+        return f"interleave_kv_kernel + sparse_attn_kernel<{w.Hkv}, false, true>"
     if w.D == 128 and group <= 8:
         return f"sparse_attn_kernel<{w.Hkv}>"
     return f"sparse_attn_wide_kernel<{w.Hkv},{w.D},{1 if group <= 8 else 2}>"
@@ -710,9 +726,10 @@ def run_qsa(args):
                              "ceiling_gbs": ceiling["ceiling_gbs"],
                              "frac_of_ceiling": attn_gbs / ceiling["ceiling_gbs"],
                              "basis": "K/V rows of every selected token as gathered (a block once per query "
-                                      "that selects it) + q read + o write; ceiling = the best bulk-copy "
-                                      "gather of the same chunks from an L2-resident buffer, measured in "
-                                      "this run (gather_probe)"},
+                                      "that selects it) + q read + o write, over the attention call (the "
+                                      "K/V interleave pass and the kernel); ceiling = the best bulk-copy "
+                                      "gather of the same 4 KB blocks (K then V) from an L2-resident "
+                                      "buffer into the kernel's ring, measured in this run (gather_probe)"},
                          "gather_probe": ceiling},
             "step_breakdown_ms": parts,
             "indexer": {
