@@ -436,9 +436,12 @@ def run_qsa(args):
     traffic, traffic_src = profile_traffic(args.workload)
     ceiling = gather_ceiling(dev, stream, w)
     if sp is None:
-        launches = (1 + select_launches(w, ws_bytes) + 1) * args.steps
+        attn_launches = 2 if kv_interleaved(w) else 1   # the K/V interleave pass and the kernel
+        launches = (1 + select_launches(w, ws_bytes) + attn_launches) * args.steps
     else:   # per chunk: pooling, the selection's kernels, attention (NCCL's own kernels not counted)
-        launches = sum(2 + select_launches(w.with_(T=b - a), ws_bytes) for a, b in my_ranges) * args.steps
+        attn_launches = 2 if kv_interleaved(w) else 1
+        launches = sum(1 + attn_launches + select_launches(w.with_(T=b - a), ws_bytes) for a, b in my_ranges) * \
+            args.steps
 
     # the query-tile attention (tcgen05 over the union of 16 rows' blocks) on the same lists, beside
     # the row-by-row kernel the step uses (both are the library's own kernels)

@@ -110,7 +110,7 @@ class ShardedPrefill:
         rows = max(b - a for a, b in self.ranges)
         ws = Q.qsa_workspace_size(Q.QSA_OP_SELECT_TOPK, B, rows, T // blk, topk, Hq, D)
         self.ws = E(ws, dtype=torch.uint8, device=dev, what="select workspace")
-        aws = Q.qsa_workspace_size(Q.QSA_OP_SPARSE_ATTN_PREFILL, B, rows, 0, topk, Hq, D)
+        aws = Q.qsa_attn_prefill_workspace_size(B, rows, T, Hq, Hkv, D, topk)
         self.attn_ws = E(max(aws, 16), dtype=torch.uint8, device=dev, what="attention workspace")
         self.idx = [E(B, b - a, topk, dtype=torch.int32, device=dev, what="idx") for a, b in self.ranges]
         self.out = [E(B, b - a, Hq, D, dtype=torch.bfloat16, device=dev, what="out") for a, b in self.ranges]
