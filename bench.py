@@ -161,6 +161,15 @@ def gather_ceiling(dev, stream, w, sweep: bool = False) -> dict:
     return res
 
 
+def workload_config(name: str, w, world: int) -> dict:
+    """The `config` object of both arms' JSON lines (the same workload, the same keys)."""
+    return {"workload": name, "B": w.B, "T": w.T, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "Hi": w.Hi, "Di": w.Di,
+            "blk": w.blk, "k": w.k, "boost": f"{w.boost_frac:g} of keys x{w.boost:g}",
+            "l2": "inputs larger than L2, no flush",
+            "parallelism": "single GPU" if world == 1 else
+            f"zig-zag query-row shards x{world}, one all-gather of K/V/kp per step; decode batch split"}
+
+
 def kv_interleaved(w) -> bool:
     """Whether the automatic attention path reads K and V interleaved by block for this shape."""
     return w.D == 128 and w.Hkv in (1, 2) and w.Hq // w.Hkv <= 8
@@ -304,8 +313,7 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * total / args.steps,
             "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": PREFILL, "B": w.B, "T": w.T, "Hq": w.Hq, "Hkv": w.Hkv,
-                                              "D": w.D, "Hi": w.Hi, "Di": w.Di, "blk": w.blk, "k": w.k},
+            "data": "synthetic", "config": workload_config(PREFILL, w, world),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -706,11 +714,7 @@ def run_qsa(args):
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "strong",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": args.workload, "B": w.B, "T": w.T, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "Hi": w.Hi,
-                       "Di": w.Di, "blk": w.blk, "k": w.k, "boost": f"{w.boost_frac:g} of keys x{w.boost:g}",
-                       "l2": "inputs larger than L2, no flush",
-                       "parallelism": "single GPU" if world == 1 else
-                       f"zig-zag query-row shards x{world}, one all-gather of K/V/kp per step; decode batch split"},
+            "config": workload_config(args.workload, w, world),
             # The attention's compulsory work is its tensor-core flops (the unique K/V bytes take a
             # tenth of that time at HBM peak), so the roofline is stated on the tensor basis; the
             # gathered-bytes rate is compared with the measured gather ceiling, not with HBM.
