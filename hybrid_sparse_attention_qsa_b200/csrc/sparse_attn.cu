@@ -12,9 +12,15 @@
 //     successive items through a 3-stage shared-memory ring without draining between items.
 //   * A block of 4 tokens is one contiguous 4*Hkv*D*2-byte run of K (and of V) in the [T][Hkv][D]
 //     layout, so each block is one 1-D bulk copy (cp.async.bulk, TMA engine) for K and one for V.
-//     A stage holds 16 blocks.  The smem pitch of a block slot is its size + 16 bytes, so the same
-//     token row of 8 consecutive slots falls in 8 different 16-byte bank groups: ldmatrix on
-//     "token j of slots 0..7" is conflict-free.
+//     With K and V interleaved by block (KVI: [B][ceil(T/4)][K, V][4][Hkv][D], written by
+//     interleave_kv_kernel) a block's K and V are one copy of twice the size, which the TMA engine
+//     delivers at a higher rate.  A stage holds 16 blocks.  The smem pitch of a block slot is its
+//     size + 16 bytes, so the same token row of 8 consecutive slots falls in 8 different 16-byte
+//     bank groups: ldmatrix on "token j of slots 0..7" is conflict-free.
+//   * Eight warps issue the copies (a leader that walks the index lists and publishes each stage's
+//     slot map, and seven helpers): the per-SM bulk-copy rate grows with the issuing warps.  With
+//     two KV heads the block has 512 threads and a setmaxnreg split (issuers 64 registers,
+//     consumers 192).
 //   * Consumer warp (g, j) owns KV head g and token j of every block: its 16 rows per stage are
 //     token j of the 16 slots.  Scores are computed transposed, S^T[token][head] = K_g Q_g^T, with
 //     mma.m16n8k16 (M = 16 tokens, N = 8 query heads of the group, K = D), so the 8 heads of a GQA
