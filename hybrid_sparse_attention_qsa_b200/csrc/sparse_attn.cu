@@ -46,7 +46,7 @@ namespace {
 constexpr int kSlots = 16;
 constexpr int kStages = 3;
 constexpr int kSeg = 512;          // index-list entries staged in shared memory per buffer
-constexpr int kIssuers_ = 4;       // warps that issue the bulk copies of a stage
+constexpr int kIssuers_ = 4;       // warps that issue a stage's bulk copies in the wide kernel (the D = 128 kernel: 8)
 constexpr int kD = 128;
 constexpr int kBlk = 4;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -187,8 +187,6 @@ __device__ __forceinline__ Item make_item(const AttnArgs& a, int i) {
   return it;
 }
 
-// Helper issuer warp h (1 .. kIssuers_ - 1): issues slots h, h + kIssuers_, ... of every stage the
-// leading producer publishes, until it publishes nslots == -1.
 // Copies of one slot: the block's K and V rows [tok0, tok0 + ntok) into kd and vd.  KVI: kbase is the
 // interleaved block array (vbase = kbase + one block of K); a whole block is one copy of its K and V.
 template <class R, int HKV, int D>
@@ -209,6 +207,8 @@ __device__ __forceinline__ void copy_slot(uint8_t* kd, uint8_t* vd, const uint16
   }
 }
 
+// Helper issuer warp h (1 .. ISS - 1): issues slots h, h + ISS, ... of every stage the
+// leading producer publishes, until it publishes nslots == -1.
 template <int HKV, int D, int SLOTS, int ISS = kIssuers_, bool KVI = false>
 __device__ __forceinline__ void attn_helper(const AttnArgs& a, int h, uint8_t* ring, uint8_t* info, uint64_t* full,
                                             uint64_t* ready) {
