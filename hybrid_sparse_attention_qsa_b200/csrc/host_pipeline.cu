@@ -48,11 +48,30 @@ struct Shape {
   int chunks, sel_chunks;
 };
 
-// Row bounds of the attention chunks and of the selection chunks.
+// Row bounds of the attention chunks and of the selection chunks.  chunks == 0 (automatic, B = 1):
+// three chunks of a quarter of the rows, then chunks that halve what is left down to about 2048
+// rows.  The selection runs first, so the early chunks' inputs have arrived before they start
+// even when they are large; large chunks leave fewer partial last waves of the attention's
+// persistent CTAs, and the small last ones leave little output to copy back after the last kernel.
 void chunk_bounds(const Shape& s, std::vector<int>& att, std::vector<int>& sel) {
-  const int n = s.B == 1 ? std::max(1, std::min(s.chunks, s.Tq)) : 1;
   att.assign(1, 0);
-  for (int c = 1; c < n; ++c) att.push_back(static_cast<int>((static_cast<long long>(s.Tq) * c / n) / 16 * 16));
+  if (s.chunks == 0 && s.B == 1) {
+    const long long T = s.Tq;
+    auto push = [&](long long e) {
+      e = e / 16 * 16;
+      if (e > att.back() && e < T) att.push_back(static_cast<int>(e));
+    };
+    push(T / 4);
+    push(T / 2);
+    push(3 * T / 4);
+    for (long long rem = T - 3 * T / 4; rem > 2048;) {
+      rem /= 2;
+      push(T - rem);
+    }
+  } else {
+    const int n = s.B == 1 ? std::max(1, std::min(s.chunks, s.Tq)) : 1;
+    for (int c = 1; c < n; ++c) att.push_back(static_cast<int>((static_cast<long long>(s.Tq) * c / n) / 16 * 16));
+  }
   att.push_back(s.Tq);
   const bool can = s.B == 1 && s.q_pos0 % 4 == 0 && static_cast<long long>(s.Tk) == s.q_pos0 + s.Tq;
   const int ns = can ? std::max(1, std::min(s.sel_chunks, s.Tq / 4)) : 1;
@@ -102,8 +121,10 @@ Layout layout(const Shape& s) {
   L.sel_ws_bytes = std::max<size_t>(sws, 16);
   L.att_ws_bytes = aws;
   L.sel_ws = take(L.sel_ws_bytes);
-  L.att_ws = take(L.att_ws_bytes);
-  L.kv = attn_kv_supported(s.Hq, s.Hkv, s.D) ? take(attn_kv_bytes(s.B, s.Tk, s.Hkv, s.D)) : 0;
+  // the attention workspace (query tiles) and the interleaved K/V are never used by one call both
+  const size_t kvb = attn_kv_supported(s.Hq, s.Hkv, s.D) ? attn_kv_bytes(s.B, s.Tk, s.Hkv, s.D) : 0;
+  L.att_ws = take(std::max(L.att_ws_bytes, kvb));
+  L.kv = L.att_ws;
   L.total = off;
   return L;
 }
@@ -111,7 +132,7 @@ Layout layout(const Shape& s) {
 bool valid_shape(const Shape& s) {
   if (s.B < 1 || s.Tq < 1 || s.Tk < 1 || s.Hq < 1 || s.Hkv < 1 || s.D < 1 || s.Hi < 1 || s.Di < 1 || s.k < 1)
     return false;
-  if (s.blk != 4 || s.q_pos0 < 0 || s.q_pos0 + s.Tq > s.Tk || s.chunks < 1 || s.sel_chunks < 1) return false;
+  if (s.blk != 4 || s.q_pos0 < 0 || s.q_pos0 + s.Tq > s.Tk || s.chunks < 0 || s.sel_chunks < 1) return false;
   return true;
 }
 

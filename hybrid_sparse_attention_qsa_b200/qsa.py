@@ -551,7 +551,7 @@ def decode(q, kcache, vcache, qi, kp, seqlens, *, topk: int, rope_theta: float =
 
 
 def qsa_prefill_host_device_bytes(B: int, Tq: int, Tk: int, Hq: int, Hkv: int, D: int, Hi: int, Di: int, k: int, *,
-                                  q_pos0: int = 0, rope: bool = False, chunks: int = 32, sel_chunks: int = 2,
+                                  q_pos0: int = 0, rope: bool = False, chunks: int = 0, sel_chunks: int = 2,
                                   blk: int = 4) -> int:
     return int(lib().qsa_prefill_host_device_bytes(B, Tq, Tk, Hq, Hkv, D, Hi, Di, k, blk, q_pos0, 1 if rope else 0,
                                                    chunks, sel_chunks))
@@ -559,11 +559,12 @@ def qsa_prefill_host_device_bytes(B: int, Tq: int, Tk: int, Hq: int, Hkv: int, D
 
 def prefill_host(q, k, v, qi, ki, *, topk: int, device="cuda", out=None, q_pos0: int = 0, rope_theta: float = 0.0,
                  head_w=None, mode: int = QSA_SCORE_RELU_SUM, scale: float | None = None,
-                 device_buffers: dict | None = None, chunks: int = 32, sel_chunks: int = 2, yarn=None):
+                 device_buffers: dict | None = None, chunks: int = 0, sel_chunks: int = 2, yarn=None):
     """The QSA layer for a prefill whose inputs live in (pinned) host memory, through
     qsa_prefill_host: the library copies the inputs in causal row chunks on its own copy streams,
     starts each chunk's pooling + selection and attention as soon as its data has arrived, and sends
-    each chunk's output rows back while the next is computed.  ``device_buffers`` (a dict) keeps the
+    each chunk's output rows back while the next is computed (``chunks`` equal attention chunks, or
+    0: quarters, then halving chunks).  ``device_buffers`` (a dict) keeps the
     device scratch ("scratch"), the index lists ("idx") and the log-sum-exps ("lse") for reuse.
     Returns dict(out=host tensor, lse=device tensor, idx=device tensor); the output is complete once
     the current stream of ``device`` has reached this call."""

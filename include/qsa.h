@@ -342,9 +342,11 @@ QSA_API qsa_status_t qsa_set_attn_options(int path);
  *   scale > 0 as for qsa_sparse_attn_prefill.
  * Schedule (B = 1): ki and qi are sent first in `sel_chunks` causal row chunks and each chunk's
  * pooling and selection starts as soon as it has arrived (only when Tk = q_pos0 + Tq and
- * q_pos0 % 4 == 0; else one chunk); q, k, v follow in `chunks` causal row chunks (K/V only up to
- * each chunk's last position, each row sent once), each chunk's attention starts when it has
- * arrived and its output rows go back while the next chunk is computed.  B > 1: one chunk of each.
+ * q_pos0 % 4 == 0; else one chunk); q, k, v follow in causal row chunks (K/V only up to each
+ * chunk's last position, each row sent once), each chunk's attention starts when it has arrived
+ * and its output rows go back while the next chunk is computed: `chunks` equal chunks, or with
+ * chunks == 0 three chunks of a quarter of the rows and then chunks that halve the rest down to
+ * about 2048 rows (fewer partial last waves, a small last output copy).  B > 1: one chunk of each.
  * The kernels run on `stream`; the copies on two streams of the library's own (one per direction
  * and device), ordered against `stream` with events.  The call returns once everything is
  * enqueued; `out` is complete when `stream` reaches the point of the call (synchronise it, or
@@ -357,7 +359,7 @@ QSA_API qsa_status_t qsa_set_attn_options(int path);
  * Calls on one device enqueue one at a time (a lock); their work may overlap on the GPU only if
  * they use different `dev` buffers.
  * Errors: INVALID_ARGUMENT (null pointer, dev misaligned, sizes, Tk < q_pos0 + Tq, blk != 4,
- * chunks or sel_chunks < 1, scale <= 0), WORKSPACE_TOO_SMALL (dev_bytes), both before anything is
+ * chunks < 0, sel_chunks < 1, scale <= 0), WORKSPACE_TOO_SMALL (dev_bytes), both before anything is
  * enqueued; a failing step (for example UNSUPPORTED for a shape the kernels do not take) returns
  * its own status with the work before it already enqueued; CUDA on a runtime error.
  */

@@ -219,12 +219,13 @@ def test_prefill_host_sizes_and_argument_checks(lib):
     # host arithmetic only: the device bytes grow with the inputs, shrink with more row chunks
     # (smaller per-chunk workspaces), and are 0 for invalid sizes
     full = Q.qsa_prefill_host_device_bytes(1, 131072, 131072, 16, 2, 128, 4, 64, 512, chunks=1, sel_chunks=1)
-    chunked = Q.qsa_prefill_host_device_bytes(1, 131072, 131072, 16, 2, 128, 4, 64, 512)
+    chunked = Q.qsa_prefill_host_device_bytes(1, 131072, 131072, 16, 2, 128, 4, 64, 512, chunks=32)
     inputs = 131072 * (2 * 16 * 128 * 2 + 2 * 2 * 128 * 2 + 4 * 64 * 2 + 64 * 2)   # q, out, k, v, qi, ki
     assert full > chunked > inputs
-    assert Q.qsa_prefill_host_device_bytes(1, 131072, 131072, 16, 2, 128, 4, 64, 512, rope=True) > chunked
+    assert Q.qsa_prefill_host_device_bytes(1, 131072, 131072, 16, 2, 128, 4, 64, 512, chunks=32, rope=True) > chunked
+    assert Q.qsa_prefill_host_device_bytes(1, 131072, 131072, 16, 2, 128, 4, 64, 512, chunks=0) > 0
     assert Q.qsa_prefill_host_device_bytes(1, 100, 50, 16, 2, 128, 4, 64, 512) == 0        # Tk < q_pos0 + Tq
-    assert Q.qsa_prefill_host_device_bytes(1, 100, 100, 16, 2, 128, 4, 64, 512, chunks=0) == 0
+    assert Q.qsa_prefill_host_device_bytes(1, 100, 100, 16, 2, 128, 4, 64, 512, chunks=-1) == 0
     args = [FAKE] * 6 + [1, 64, 64, 16, 2, 128, 4, 64, 8, 4, 0, 0.1, 0, None, None, 1, 1, FAKE, 1 << 30, None, None,
                          None]
 
@@ -241,5 +242,5 @@ def test_prefill_host_sizes_and_argument_checks(lib):
     assert call(Tk=60) == Q.QSA_ERR_INVALID_ARGUMENT
     assert call(blk=8) == Q.QSA_ERR_INVALID_ARGUMENT
     assert call(scale=0.0) == Q.QSA_ERR_INVALID_ARGUMENT
-    assert call(chunks=0) == Q.QSA_ERR_INVALID_ARGUMENT
+    assert call(chunks=-1) == Q.QSA_ERR_INVALID_ARGUMENT
     assert call(dev_bytes=100) == Q.QSA_ERR_WORKSPACE_TOO_SMALL

@@ -16,9 +16,10 @@ def _pinned(x):
     return {n: t.cpu().pin_memory() for n, t in x.items()}
 
 
-@pytest.mark.parametrize("chunks,sel_chunks", [(1, 1), (3, 4), (8, 3), (8, 7)])
+@pytest.mark.parametrize("chunks,sel_chunks", [(1, 1), (3, 4), (8, 3), (8, 7), (0, 2)])
 def test_prefill_host_matches_device_path(chunks, sel_chunks):
-    """Attention in `chunks` row chunks, pooling and selection in `sel_chunks` (ragged ones too)."""
+    """Attention in `chunks` row chunks (0: quarters, then halving), pooling and selection in
+    `sel_chunks` (ragged ones too)."""
     w = I.WORKLOADS["prefill_32k"].with_(T=12002)
     x = I.make_prefill(w, DEV)
     ref = Q.prefill(x["q"], x["k"], x["v"], x["qi"], x["ki"], topk=w.k)
