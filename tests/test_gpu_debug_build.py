@@ -22,7 +22,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def test_debug_build_runs_clean_with_intact_canaries_and_equals_release(tmp_path):
-    assert not Q.DEBUG, "the parent process runs the release library"
+    if Q.DEBUG:
+        pytest.skip("compares the debug library with the release one: run without QSA_DEBUG")
     B.build(debug=True)
     out = tmp_path / "debug.pt"
     env = dict(os.environ, QSA_DEBUG="1")
