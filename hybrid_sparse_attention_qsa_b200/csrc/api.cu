@@ -457,7 +457,7 @@ qsa_status_t qsa_sparse_attn_prefill_ws(const void* q, const void* k, const void
                         ok_ptr(workspace) && ws_bytes >= 512 + attn_tc_tile_bytes(k_blocks);
   if (path == 2 && !tiles_ok)
     return attn_tc_supported(Hq, Hkv, D, k_blocks) ? QSA_ERR_WORKSPACE_TOO_SMALL : QSA_ERR_UNSUPPORTED;
-  if (path == 0 && attn_kv_supported(Hq, Hkv, D) && workspace != nullptr && ok_ptr(workspace) &&
+  if (path == 0 && attn_kv_supported(Hq, Hkv, D) && B <= 65535 && workspace != nullptr && ok_ptr(workspace) &&
       ws_bytes >= attn_kv_bytes(B, Tk, Hkv, D)) {
     const long long j1 = (q_pos0 + Tq + 3) / 4;
     cudaError_t e = launch_interleave_kv(di, k, v, workspace, B, Tk, Hkv, D, 0, j1, S(stream));

@@ -137,6 +137,7 @@ bool valid_shape(const Shape& s) {
 }
 
 // Per-device copy streams and a reusable pool of events; one call enqueues at a time per device.
+// They live until the process exits (like the library's other per-device caches).
 struct DevState {
   std::mutex mu;
   bool ready = false;
@@ -219,7 +220,7 @@ qsa_status_t qsa_prefill_host(const void* q_h, const void* k_h, const void* v_h,
   float* lse_d = lse_out ? lse_out : reinterpret_cast<float*>(base + L.lse);
   void* sel_ws = base + L.sel_ws;
   void* att_ws = base + L.att_ws;
-  const bool use_kv = attn_path() == 0 && attn_kv_supported(Hq, Hkv, D);
+  const bool use_kv = attn_path() == 0 && attn_kv_supported(Hq, Hkv, D) && B <= 65535;
   void* kv_d = base + L.kv;
   long long kv_done_i = 0;   // positions interleaved so far (the block holding it is rewritten next)
   const char* qh = static_cast<const char*>(q_h);
