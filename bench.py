@@ -325,12 +325,12 @@ def select_launches(w, ws_bytes: int) -> int:
     """Kernels qsa_select_topk launches for a prefill with a workspace of ws_bytes (the library's
     own choice between the filtered and the materialised selection, restated)."""
     nbk = w.T // w.blk
-    rank = max(64, (5 * w.k + 31) // 32)
+    rank = max(64, (2 * w.k + 15) // 16)
     ns = (nbk - 9) // 16 + 1 if nbk > 8 else 0
     per_row = ((max(ns, 1) + 3) // 4 * 4) * 4 + 12 + 32 * rank * 8
     fit = max(0, (ws_bytes - (12 * 256 + 4 + 128 * max(nbk, 1) * 4)) // per_row)
     n = 0
-    if w.Hi in (4, 8) and 32 * rank <= 5120 and w.T >= 16384 and fit >= min(w.T, 4096):
+    if w.Hi in (4, 8) and w.k <= 1024 and 32 * rank <= 5120 and w.T >= 16384 and fit >= min(w.T, 4096):
         R = min(w.T, fit)
         if R < w.T and R >= 64:
             R -= R % 64

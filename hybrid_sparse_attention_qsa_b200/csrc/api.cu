@@ -77,10 +77,12 @@ struct FusedPlan {
   long long per_row, fixed;
 };
 // rank r of the threshold among the row's samples (about 16 r scores expected above it, at least
-// 2.5 k so a short list is a many-sigma event) and the list capacity 32 r.
+// 2 k: the sample rank's relative spread is about 1 / sqrt(r), so a list shorter than k is a
+// four-sigma event or rarer) and the list capacity 32 r.  (2.5 k took 3 % longer at 128K, 1.5 k
+// sent enough rows to the exact redo to cost more.)
 FusedPlan fused_plan(int NBk, int k) {
   FusedPlan p;
-  p.rank = std::max(64, (5 * k + 31) / 32);
+  p.rank = std::max(64, (2 * k + 15) / 16);
   p.cap = 32 * p.rank;
   p.ns = NBk > kSampleOff ? ((NBk - kSampleOff - 1) >> kSampleShift) + 1 : 0;
   p.ld_s = (std::max(p.ns, 1) + 3) & ~3;
@@ -286,7 +288,7 @@ qsa_status_t qsa_select_topk(const float* scores, int64_t ld_scores, const void*
     const FusedPlan fp = fused_plan(NBk, k);
     const long long fit = fused_rows_fit(fp, ws_bytes);
     const int path = g_select_path.load();
-    const bool able = (Hi == 4 || Hi == 8) && fp.cap <= kFusedMaxCap;
+    const bool able = (Hi == 4 || Hi == 8) && k <= 1024 && fp.cap <= kFusedMaxCap;
     if (path == 2 && !able) return QSA_ERR_UNSUPPORTED;
     if (path == 2 && fit < 1) return QSA_ERR_WORKSPACE_TOO_SMALL;
     // automatic: rows long enough (the chunk's last row sees 16384 positions or more), and a

@@ -197,13 +197,13 @@ QSA_API qsa_status_t qsa_index_score(const void* qi, const void* kp, const float
  *   - filtered (prefill with Hi of 4 or 8 and k <= 1024, chosen automatically when the call's last
  *     row sits at position 16384 or later, q_pos0 + Tq >= 16384, and the workspace holds 4096 rows
  *     or all of them): the scores are never stored.  Every 16th
- *     pooled block is scored first; per row, a threshold with about 2.5 k (at least 1024) of the
+ *     pooled block is scored first; per row, a threshold with about 2 k (at least 1024) of the
  *     row's scores expected above it is read off these samples; the tensor-core score kernel then
  *     keeps only the scores at or above the threshold, in block order, and the top-k is selected
  *     from that list.  A row whose list is shorter than k or longer than its capacity is redone
  *     exactly over all its scores (CUDA-core fp32 scores), so a threshold decides only which rows
  *     are redone, never which blocks a row keeps beyond last-bit ties.  Workspace per
- *     row of a chunk: about 4 * NBk / 16 + 256 * max(64, ceil(5 k / 32)) bytes, plus
+ *     row of a chunk: about 4 * NBk / 16 + 256 * max(64, ceil(2 k / 16)) bytes, plus
  *     128 * NBk * 4 bytes for the redo.
  *   qsa_workspace_size(QSA_OP_SELECT_TOPK, ...) gives a size that fits either way in few chunks
  *   (up to about 4 GiB).

@@ -118,8 +118,8 @@ def test_select_and_attention_argument_checks(lib):
 def filtered_bytes(rows, nbk, k):
     # the filtered selection's workspace as include/qsa.h states it: per row the sampled scores
     # (every 16th block, padded to 4), threshold, count and failure slot, and the candidate list
-    # of 32 * max(64, ceil(5k/32)) (key, block) pairs; plus 128 scratch rows and alignment
-    rank = max(64, (5 * k + 31) // 32)
+    # of 32 * max(64, ceil(2k/16)) (key, block) pairs; plus 128 scratch rows and alignment
+    rank = max(64, (2 * k + 15) // 16)
     ns = (nbk - 9) // 16 + 1 if nbk > 8 else 0
     per_row = ((max(ns, 1) + 3) // 4 * 4) * 4 + 12 + 32 * rank * 8
     return 12 * 256 + 4 + 128 * max(nbk, 1) * 4 + rows * per_row

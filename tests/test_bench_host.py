@@ -43,9 +43,9 @@ def test_decode_work():
 def test_select_launch_count():
     w = I.WORKLOADS["prefill_128k"]
     nbk = w.T // 4
-    # a workspace too small for the filtered path (under 4096 rows of lists): 132 chunks of 1000
-    # score rows -> 132 score + 132 top-k launches
-    assert bench.select_launches(w, nbk * 4 * 1000) == 264
+    # a workspace too small for the filtered path (under 4096 rows of lists): 164 chunks of 800
+    # score rows -> 164 score + 164 top-k launches
+    assert bench.select_launches(w, nbk * 4 * 800) == 328
     # the first chunk of a 1-row workspace holds rows 0..0: no candidate, no score launch
     tiny = w.with_(T=12)
     assert bench.select_launches(tiny, 3 * 4) == 12 + 12 - 4
