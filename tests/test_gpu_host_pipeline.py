@@ -72,3 +72,23 @@ def test_prefill_host_window_with_rope_and_selection_chunks(q0):
     assert Q.qsa_get_device_status() == Q.QSA_OK
     assert torch.equal(got["idx"], ref["idx"])
     assert torch.equal(got["out"], ref["out"].cpu())
+
+
+@pytest.mark.parametrize("path", [Q.QSA_ATTN_ROWS, Q.QSA_ATTN_TILES])
+def test_prefill_host_with_each_attention_path(path):
+    """The host pipeline with the row kernel over k and v, or the query tiles, forced: the same
+    result as the device path under the same choice."""
+    w = I.WORKLOADS["prefill_32k"].with_(T=9000)
+    x = I.make_prefill(w, DEV)
+    Q.qsa_set_attn_options(path)
+    try:
+        ref = Q.prefill(x["q"], x["k"], x["v"], x["qi"], x["ki"], topk=w.k)
+        h = _pinned(x)
+        got = Q.prefill_host(h["q"], h["k"], h["v"], h["qi"], h["ki"], topk=w.k, device=DEV)
+        torch.cuda.synchronize()
+    finally:
+        Q.qsa_set_attn_options(Q.QSA_ATTN_AUTO)
+    assert Q.qsa_get_device_status() == Q.QSA_OK
+    assert torch.equal(got["idx"], ref["idx"])
+    assert torch.equal(got["out"], ref["out"].cpu())
+    assert torch.equal(got["lse"], ref["lse"])
