@@ -482,6 +482,9 @@ def run_qsa(args):
             tiles = {"kernel": "tile_union_kernel + sparse_attn_tc_kernel<%d>" % w.Hkv, "ms": t_ms,
                      "rows_kernel_ms": ms_attn, "speedup_vs_rows": ms_attn / t_ms,
                      "union_blocks_per_tile_mean": ublk, "union_over_sum_of_lists": ublk / (16 * (w.k + 1)),
+                     "union_blocks_per_tile_quantiles": {f"p{int(100 * qq)}": float(torch.quantile(cnt, qq))
+                                                          for qq in (0.0, 0.1, 0.5, 0.9, 1.0)},
+                     "union_tiles_sampled": f"the last {held} tiles of the call (the ones the workspace held last)",
                      "gathered_bytes": gath, "gathered_bytes_rows_kernel": work["attn_bytes"],
                      "tensor_tflops_dense_union": tflop / (t_ms / 1000),
                      "frac_of_bf16_peak": tflop / (t_ms / 1000) / pk["bf16_tflops"],
