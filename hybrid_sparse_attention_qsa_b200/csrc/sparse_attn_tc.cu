@@ -125,19 +125,18 @@ __device__ __forceinline__ float fast_exp2(float x) {
 
 // ---------------------------------------------------------------------------- tile unions
 constexpr int kUnionThreads = 512;
-constexpr int kWin = 16384;                 // blocks per window of the union bitmap
+constexpr int kWin = 8192;                  // blocks per window of the union bitmap (32 KB: two CTAs a SM)
 constexpr int kMaxListPerThread = 32;       // 16 rows x k_blocks <= 16384 entries -> 32 per thread
 
 // One CTA per tile.  Every listed block of the tile's rows (and each row's own block) ORs the row's
 // bit into the block's 16-bit mask in a shared-memory bitmap; the blocks whose mask is non-zero,
 // ascending, are the union.  The block range is walked in windows of kWin blocks.
-__global__ void __launch_bounds__(kUnionThreads) tile_union_kernel(const int32_t* __restrict__ idx, int Tq, int kb,
+__global__ void __launch_bounds__(kUnionThreads, 2) tile_union_kernel(const int32_t* __restrict__ idx, int Tq, int kb,
                                                                   long long q_pos0, int tile0, int tpb,
                                                                   uint2* __restrict__ ent, int* __restrict__ cnt,
                                                                   int cap, ChunkInfo* __restrict__ recs, int capc,
                                                                   KernelCtl ctl) {
-  extern __shared__ uint32_t umask[];       // [kWin] row masks of the window's blocks, then the union
-  uint2* sent = reinterpret_cast<uint2*>(umask + kWin);   // [cap] the union, for the chunk records
+  extern __shared__ uint32_t umask[];       // [kWin] row masks of the window's blocks
   __shared__ int s_scan[kUnionThreads / 32 + 1];
   __shared__ int s_bad;
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
@@ -217,10 +216,7 @@ __global__ void __launch_bounds__(kUnionThreads) tile_union_kernel(const int32_t
       const uint32_t m = umask[i];
       if (m) {
         const uint2 e = make_uint2(static_cast<uint32_t>(w0 + i), m);
-        if (QSA_DCHECK(ctl, u < cap)) {
-          te[u] = e;
-          sent[u] = e;
-        }
+        if (QSA_DCHECK(ctl, u < cap)) te[u] = e;
         ++u;
       }
     }
@@ -232,14 +228,15 @@ __global__ void __launch_bounds__(kUnionThreads) tile_union_kernel(const int32_t
     cnt[tl] = total;
     if (s_bad) record_status(ctl, kStBadArg);
   }
-  // the chunk records: one warp per chunk of 16 entries (from the shared-memory copy of the union)
+  // the chunk records: one warp per chunk of 16 entries, read back from the union this CTA has just
+  // written (L2; visible to the CTA's threads after the barrier)
   __syncthreads();
   const int nu = total;
   const int nch = max(1, (nu + kCB - 1) / kCB);
   ChunkInfo* tr = recs + static_cast<long long>(tl) * capc;
   for (int c = w; c < nch; c += kUnionThreads >> 5) {
     const int uu = c * kCB + lane;
-    const uint2 e = sent[min(uu, max(nu - 1, 0))];
+    const uint2 e = __ldcg(te + min(uu, max(min(nu, cap) - 1, 0)));
     const uint32_t mask = (lane < kCB && uu < nu) ? e.y : 0u;
     uint32_t myw = 0;
     int myo = -1;
@@ -713,12 +710,11 @@ cudaError_t launch_attn_prefill_tc(const DeviceInfo* di, const void* q, const vo
   if (!make_map4(&qm, q, Hq, Tq, B, kGrp, kTQ) || !make_map4(&km, k, Hkv, tk_used, B, 1, 4, static_cast<unsigned long long>(Tk)) ||
       !make_map4(&vm, v, Hkv, tk_used, B, 1, 4, static_cast<unsigned long long>(Tk)))
     return cudaErrorInvalidValue;
-  const size_t usmem = static_cast<size_t>(kWin) * 4 + static_cast<size_t>(cap) * sizeof(uint2);
+  const size_t usmem = static_cast<size_t>(kWin) * 4;
   if (kTQ * k_blocks > kMaxListPerThread * kUnionThreads) return cudaErrorInvalidValue;
   static std::once_flag once[64];
   std::call_once(once[di->device & 63], [] {
-    cudaFuncSetAttribute(tile_union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         kWin * 4 + (kTQ * 1024 + kTQ) * static_cast<int>(sizeof(uint2)));
+    cudaFuncSetAttribute(tile_union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kWin * 4);
     cudaFuncSetAttribute(sparse_attn_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     cudaFuncSetAttribute(sparse_attn_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   });
