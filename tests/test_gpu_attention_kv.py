@@ -60,7 +60,7 @@ def test_interleave_in_pieces_equals_whole():
 
 
 @pytest.mark.parametrize("B,T,q0,Hq,Hkv,k", [(1, 3000, 0, 16, 2, 64), (2, 1500, 0, 8, 1, 37), (1, 2000, 1233, 16, 2, 128),
-                                             (1, 800, 0, 8, 2, 512)])
+                                             (1, 800, 0, 8, 2, 512), (2, 600, 4101, 8, 1, 1024)])
 def test_attention_over_interleaved_kv_is_bit_identical(B, T, q0, Hq, Hkv, k):
     Tk = q0 + T
     q = _rand((B, T, Hq, 128), 5)
