@@ -85,6 +85,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
       : "memory");
   return ok != 0;
 }
+// Non-blocking test: true when the phase with the given parity has completed.  Unlike try_wait it
+// never suspends the thread, so a loop that polls several barriers is not held on one of them.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, unsigned parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 // As mbar_try_wait, but a thread whose phase is still open may be suspended for up to `hint_ns`
 // (it resumes as soon as the phase completes), so waiting warps take fewer issue slots.
 __device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, unsigned parity, unsigned hint_ns) {

@@ -383,7 +383,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Within a (tile, head) pass, S(i) and PV(j) are issued as soon as each is ready (S(i): the
     // chunk's K/V and a free S buffer; PV(j): the softmax's P and, for each accumulator's first PV
     // of the pass, both accumulators read out by the previous epilogue), so a PV whose P is ready
-    // never waits behind the next chunk's data.  Chunk j of a pass accumulates into O[j & 1].
+    // never waits behind the next chunk's data.  The barriers are polled with test_wait, which
+    // never suspends the thread (try_wait may hold it on a barrier that is not about to complete),
+    // PV before S: a PV frees an S buffer and its chunk's K/V stage.  Chunk j of a pass accumulates
+    // into O[j & 1].
     if (lane == 0) {
       const uint32_t idesc_s = umma_idesc_bf16_f32(128, kCT);
       const uint32_t idesc_pv = umma_idesc_bf16_f32_bmn(128, kD);
@@ -402,10 +405,29 @@ __global__ void __launch_bounds__(kThreads, 1)
           unsigned long long t_last = globaltimer_ns();
           while (pj < nch) {
             bool progress = false;
+            if (pj < si) {
+              const int m = n0 + pj, s = m % kStages, sb = m % kSBuf;
+              const bool first = pj < 2;   // the accumulator's first PV of the pass
+              if (mbar_test_wait(&bar->p_full[sb], static_cast<unsigned>(m / kSBuf) & 1u) &&
+                  (!first || hp == 0 || mbar_test_wait(&bar->o_free, static_cast<unsigned>(hp - 1) & 1u))) {
+                tc_fence_after();
+                const uint32_t vbase = smem_u32(kvs + s * 2 * kKVBytes + kKVBytes);
+                const uint32_t o_col = tmem + kOCol + (pj & 1) * kD;
+#pragma unroll
+                for (int kk = 0; kk < kCT / 16; ++kk) {
+                  const uint64_t bd = sw128_mnmajor_desc(vbase + kk * 2048, kKVHalf, 1024);
+                  umma_bf16_ta(o_col, tmem + sb * kCT + kk * 8, bd, idesc_pv, (first && kk == 0) ? 0u : 1u);
+                }
+                umma_commit(&bar->kv_empty[s]);
+                umma_commit(&bar->s_free[sb]);
+                ++pj;
+                progress = true;
+              }
+            }
             if (si < nch) {
               const int n = n0 + si, s = n % kStages, sb = n % kSBuf;
-              if (mbar_try_wait(&bar->kv_full[s], static_cast<unsigned>(n / kStages) & 1u) &&
-                  mbar_try_wait(&bar->s_free[sb], (static_cast<unsigned>(n / kSBuf) & 1u) ^ 1u)) {
+              if (mbar_test_wait(&bar->kv_full[s], static_cast<unsigned>(n / kStages) & 1u) &&
+                  mbar_test_wait(&bar->s_free[sb], (static_cast<unsigned>(n / kSBuf) & 1u) ^ 1u)) {
                 tc_fence_after();
                 const uint32_t kbase = smem_u32(kvs + s * 2 * kKVBytes);
 #pragma unroll
@@ -418,25 +440,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 umma_commit(&bar->s_full[sb]);
                 if (si == nch - 1) umma_commit(&bar->q_empty);   // Q is free once the pass's S are done
                 ++si;
-                progress = true;
-              }
-            }
-            if (pj < si) {
-              const int m = n0 + pj, s = m % kStages, sb = m % kSBuf;
-              const bool first = pj < 2;   // the accumulator's first PV of the pass
-              if (mbar_try_wait(&bar->p_full[sb], static_cast<unsigned>(m / kSBuf) & 1u) &&
-                  (!first || hp == 0 || mbar_try_wait(&bar->o_free, static_cast<unsigned>(hp - 1) & 1u))) {
-                tc_fence_after();
-                const uint32_t vbase = smem_u32(kvs + s * 2 * kKVBytes + kKVBytes);
-                const uint32_t o_col = tmem + kOCol + (pj & 1) * kD;
-#pragma unroll
-                for (int kk = 0; kk < kCT / 16; ++kk) {
-                  const uint64_t bd = sw128_mnmajor_desc(vbase + kk * 2048, kKVHalf, 1024);
-                  umma_bf16_ta(o_col, tmem + sb * kCT + kk * 8, bd, idesc_pv, (first && kk == 0) ? 0u : 1u);
-                }
-                umma_commit(&bar->kv_empty[s]);
-                umma_commit(&bar->s_free[sb]);
-                ++pj;
                 progress = true;
               }
             }
@@ -501,11 +504,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (wor & 0xFFu) tmem_ld_32x32(s_addr, r[0]);
           if (wor & 0xFF00u) tmem_ld_32x32(s_addr + 32, r[1]);
           tmem_ld_wait();
-          // masked raw scores (-inf where the row does not attend) and their maximum; straight-line
-          // selects (per-slot branches cost more than the arithmetic they skip)
+          // masked raw scores (-inf where the row does not attend) and their maximum.  A slot that no
+          // row of the warp attends (its bit clear in wor, the same for all 32 lanes) is skipped here
+          // and below: its probabilities are exactly 0.  Within an attended slot, straight-line selects.
           float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
           for (int j = 0; j < kCB; ++j) {
+            if (!((wor >> j) & 1u)) continue;
             const bool mem = (word >> j) & 1u;
             const int lj = j == oslot ? lim : 3;
 #pragma unroll
@@ -557,6 +562,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t pk[16];
 #pragma unroll
             for (int jj = 0; jj < 8; ++jj) {
+              pk[2 * jj] = 0u;
+              pk[2 * jj + 1] = 0u;
+              if (!((wor >> (q8 * 8 + jj)) & 1u)) continue;
               float p[4];
 #pragma unroll
               for (int i = 0; i < 4; ++i) {   // masked entries hold -inf: 2^-inf = 0
