@@ -238,6 +238,14 @@ __device__ __forceinline__ void umma_bf16_ta(uint32_t d_tmem, uint32_t a_tmem, u
       : "memory");
 }
 
+// 128 lanes x 256 bits from a shared-memory matrix (described as for an MMA operand: 128 rows of
+// 32 bytes) into TMEM: lane i gets row i in 8 consecutive 32-bit columns, the layout of an A
+// operand read from TMEM for one K step of 16 bf16.  Ordered before the MMAs this thread issues
+// after it.
+__device__ __forceinline__ void tmem_cp_128x256b(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
 // 32 lanes x 32 consecutive 32-bit columns: thread i of the warp gets lane (base + i), columns
 // col .. col+31 of the address.
 __device__ __forceinline__ void tmem_ld_32x32(uint32_t taddr, uint32_t (&r)[32]) {

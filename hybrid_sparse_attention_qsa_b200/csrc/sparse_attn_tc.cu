@@ -28,8 +28,9 @@
 //            of the next chunk fetched ahead.  Each box costs its issuing warp ~80 cycles, so one
 //            warp caps these 512-byte gathers near 2 TB/s device-wide; seven to eight reach
 //            ~10 TB/s (the gather probe);
-//   warp 7   MMA issuer (one thread), event-driven: S = Q K^T (M 128, N 64 tokens, K 128) into one
-//            of four S buffers as soon as a chunk and a buffer are ready, and O += P V (P read from
+//   warp 7   MMA issuer (one thread), event-driven: copies the pass's Q tile into TMEM, then
+//            S = Q K^T (M 128, N 64 tokens, K 128; Q read from TMEM as the A operand) into one of
+//            three S buffers as soon as a chunk and a buffer are ready, and O += P V (P read from
 //            TMEM as the A operand, V as an MN-major B operand) as soon as a chunk's P is written;
 //            chunks alternate between two O accumulators;
 //   warps 8-15 softmax, two groups of four warps (one TMEM lane quadrant each, one thread per row):
@@ -39,7 +40,10 @@
 //            groups' (m, l) through shared memory and their O accumulators from TMEM, then writes
 //            the bf16 rows and the log-sum-exp.
 // Register split (setmaxnreg): producers and MMA drop to 64 registers, softmax rises to 192.
-// TMEM: S0..S3 at columns 0, 64, 128, 192, O[0] at 256, O[1] at 384 (fp32, lane = row).  Every wait
+// TMEM: S0..S2 at columns 0, 64, 128, the Q tile at 192 (bf16 pairs, copied from shared memory with
+// tcgen05.cp at the start of a pass: S reads its A operand from TMEM, which the pipe executes in 32
+// cycles per K step at N = 64 against 48 with A in shared memory, where the 6 KB of operands an MMA
+// reads bound it), O[0] at 256, O[1] at 384 (fp32, lane = row).  Every wait
 // is bounded and suspends the waiting warp (spinning producer and MMA warps would take issue slots
 // from the softmax warps on their schedulers); a role whose wait runs out stops, and every role
 // reaches the final barrier and TMEM release.
@@ -61,7 +65,7 @@ constexpr int kQBytes = 2 * kQHalf;
 constexpr int kKVHalf = kCT * 128;        // one 64-column half of a chunk's K (or V): kCT rows x 128 B
 constexpr int kKVBytes = 2 * kKVHalf;     // K (or V) of one chunk
 constexpr int kStages = 5;                // K/V ring depth (shared memory)
-constexpr int kSBuf = 4;                  // S buffers in TMEM (kCT columns each), then two O accumulators
+constexpr int kSBuf = 3;                  // S buffers in TMEM (kCT columns each), then Q and two O accumulators
 constexpr int kProdWarps = 7;             // warps issuing the TMA boxes (each box costs its warp ~80 cycles)
 constexpr int kMmaWarp = 7;
 constexpr int kSoftWarp0 = 8;             // softmax warps 8..15: group (w - 8) / 4 takes every other chunk
@@ -76,7 +80,8 @@ constexpr int kLowRegs = 64;
 constexpr int kHighRegs = 192;
 static_assert(kThreads == 512 && kSoftWarp0 == 8, "two warpgroups per side of the split");
 static_assert(256 * kLowRegs + 256 * kHighRegs <= kThreads * kLaunchRegs, "register split");
-constexpr int kOCol = kSBuf * kCT;        // TMEM columns of the two O accumulators (128 columns each)
+constexpr int kQCol = kSBuf * kCT;        // TMEM columns of the Q tile (kD / 2 columns of bf16 pairs)
+constexpr int kOCol = kQCol + kD / 2;     // TMEM columns of the two O accumulators (128 columns each)
 static_assert(kOCol + 2 * kD <= 512, "TMEM columns");
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleLog2 = 8.0f;  // O is rescaled only when the row max grows by more than this
@@ -400,7 +405,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             alive = false;
             break;
           }
+          // Q into TMEM, one K step (32 bytes of each row) per copy.  The previous pass's S MMAs, the
+          // only readers of these columns, are complete: the producer loaded this Q only after they
+          // had released the shared-memory copy (q_empty).
+          tc_fence_after();
           const uint32_t qbase = smem_u32(qs);
+#pragma unroll
+          for (int kk = 0; kk < kD / 16; ++kk)
+            tmem_cp_128x256b(tmem + kQCol + kk * 8, sw128_kmajor_desc(qbase + (kk >> 2) * kQHalf) + 2 * (kk & 3));
           int si = 0, pj = 0;   // next S and next PV of the pass
           unsigned long long t_last = globaltimer_ns();
           while (pj < nch) {
@@ -432,13 +444,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t kbase = smem_u32(kvs + s * 2 * kKVBytes);
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk) {
-                  const int h = kk >> 2;
-                  const uint64_t ad = sw128_kmajor_desc(qbase + h * kQHalf) + 2 * (kk & 3);
-                  const uint64_t bd = sw128_kmajor_desc(kbase + h * kKVHalf) + 2 * (kk & 3);
-                  umma_bf16(tmem + sb * kCT, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+                  const uint64_t bd = sw128_kmajor_desc(kbase + (kk >> 2) * kKVHalf) + 2 * (kk & 3);
+                  umma_bf16_ta(tmem + sb * kCT, tmem + kQCol + kk * 8, bd, idesc_s, kk > 0 ? 1u : 0u);
                 }
                 umma_commit(&bar->s_full[sb]);
-                if (si == nch - 1) umma_commit(&bar->q_empty);   // Q is free once the pass's S are done
+                // the Q tile (shared memory and its TMEM copy) is free once the pass's S are done
+                if (si == nch - 1) umma_commit(&bar->q_empty);
                 ++si;
                 progress = true;
               }
