@@ -57,6 +57,30 @@ def test_tiles_match_the_oracle_on_every_row(T, Hq, Hkv, k):
     assert np.abs(lse.cpu().numpy()[0] - ora["lse"]).max() <= 1e-2
 
 
+def test_tiles_across_sequences_of_a_batch():
+    # three sequences of a ragged length: tiles 0-69 belong to sequence 0, 70-139 to 1, 140-209 to 2,
+    # the last tile of each holding 7 rows
+    B, T, Hq, Hkv, k = 3, 1111, 16, 2, 64
+    g = torch.Generator(device=DEV)
+    g.manual_seed(11)
+    rb = lambda shape, d: (torch.randn(shape, generator=g, device=DEV) / math.sqrt(d)).to(torch.bfloat16)
+    x = dict(q=rb((B, T, Hq, 128), 128), k=rb((B, T, Hkv, 128), 128), v=rb((B, T, Hkv, 128), 128),
+             qi=rb((B, T, 4, 64), 64), ki=rb((B, T, 64), 64))
+    h = {n: I.bits(t) for n, t in x.items()}
+    kp = O.pool_block_keys(h["ki"])
+    ora = O.prefill_rows(h["q"], h["k"], h["v"], h["qi"], kp, [(b, t) for b in range(B) for t in range(T)], topk=k)
+    idx = torch.from_numpy(ora["idx"]).to(DEV).view(B, T, k)
+    out, lse = Q.qsa_sparse_attn_prefill(x["q"], x["k"], x["v"], idx)
+    Q.qsa_set_attn_options(Q.QSA_ATTN_ROWS)
+    o_rows, l_rows = Q.qsa_sparse_attn_prefill(x["q"], x["k"], x["v"], idx)
+    torch.cuda.synchronize()
+    _status_ok()
+    P.assert_outputs_close(I.bits(out).reshape(B * T, Hq, 128), ora["out"])
+    assert np.abs(lse.cpu().numpy().reshape(B * T, Hq) - ora["lse"]).max() <= 1e-2
+    P.assert_outputs_close(I.bits(out), I.bits(o_rows))
+    assert torch.allclose(lse, l_rows, atol=1e-4)
+
+
 def test_tiles_at_an_offset_with_garbage_past_the_last_query():
     # rows 1234 .. 2233 of a 2400-token cache whose positions past the last query hold NaN: a tile's
     # last own block reaches past the last query, and those positions must not be read
