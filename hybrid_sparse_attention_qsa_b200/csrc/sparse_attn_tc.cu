@@ -14,7 +14,7 @@
 // contributes exp(-inf) = 0, and the softmax runs in fp32 over exactly the selected tokens.
 //
 // tile_union_kernel (one CTA per tile): every listed block of the 16 rows, and each row's own block,
-// sets the row's bit in the block's 16-bit mask in a shared-memory bitmap (windows of 16384 blocks);
+// sets the row's bit in the block's 16-bit mask in a shared-memory bitmap (windows of 8192 blocks);
 // the blocks with a non-zero mask, ascending, are the union, written as (block, row mask) entries
 // and as one 128-byte record per chunk of 16 entries (block ids, per-row member bits, per-row own
 // slot) for the attention kernel.  Entries outside a row's causal range are skipped and recorded in
@@ -36,17 +36,18 @@
 //   warps 8-15 softmax, two groups of four warps (one TMEM lane quadrant each, one thread per row):
 //            group g takes every other chunk of a pass and owns O[g]: mask, fp32 online softmax in
 //            exp2 form with a lazy rescale of its O (only when the running max grows by more than
-//            2^8), P packed to bf16 into the S buffer's columns.  The epilogue merges the two
+//            2^8), P packed to bf16 into the S buffer's columns; the slots that none of a warp's
+//            4 query rows attends are skipped (their P is 0).  The epilogue merges the two
 //            groups' (m, l) through shared memory and their O accumulators from TMEM, then writes
 //            the bf16 rows and the log-sum-exp.
 // Register split (setmaxnreg): producers and MMA drop to 64 registers, softmax rises to 192.
 // TMEM: S0..S2 at columns 0, 64, 128, the Q tile at 192 (bf16 pairs, copied from shared memory with
 // tcgen05.cp at the start of a pass: S reads its A operand from TMEM, which the pipe executes in 32
 // cycles per K step at N = 64 against 48 with A in shared memory, where the 6 KB of operands an MMA
-// reads bound it), O[0] at 256, O[1] at 384 (fp32, lane = row).  Every wait
-// is bounded and suspends the waiting warp (spinning producer and MMA warps would take issue slots
-// from the softmax warps on their schedulers); a role whose wait runs out stops, and every role
-// reaches the final barrier and TMEM release.
+// reads bound it), O[0] at 256, O[1] at 384 (fp32, lane = row).  Every wait is bounded; the producer
+// and softmax warps suspend while they wait (spinning would take issue slots from the softmax warps
+// on their schedulers), the MMA thread polls its barriers with test_wait; a role whose wait runs out
+// stops, and every role reaches the final barrier and TMEM release.
 #include <algorithm>
 #include <mutex>
 
