@@ -141,7 +141,7 @@ void index_scores_row(const uint16_t* qi_row, const uint16_t* kp, const float* h
       double dot = 0.0;
       for (int64_t d = 0; d < Di; ++d) dot += (QO_MUTANT == 9 ? q[d * Hi + h] : q[h * Di + d]) * kb[d];
       double term = (mode == 0 && QO_MUTANT != 1) ? std::max(0.0, dot) : dot;
-      double w = head_w ? static_cast<double>(head_w[h]) : 1.0;
+      double w = (head_w && QO_MUTANT != 14) ? static_cast<double>(head_w[h]) : 1.0;
       acc += w * term;
     }
     s[b] = static_cast<float>(acc);
@@ -211,7 +211,7 @@ int attend_row(const uint16_t* q_row, const uint16_t* kb, const uint16_t* vb, in
       for (int64_t d = 0; d < D; ++d) o[d] += p * bf16_to_double(vr[d]);
     }
     for (int64_t d = 0; d < D; ++d) out[h * D + d] = bf16_from_double(o[d] / l);
-    if (lse) lse[h] = static_cast<float>(zmax + std::log(l));
+    if (lse) lse[h] = static_cast<float>(QO_MUTANT == 13 ? std::log(l) : zmax + std::log(l));
   }
   return 0;
 }
@@ -372,7 +372,7 @@ int qo_prefill_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v, con
       }
       const int64_t nb = std::min(pos / blk + (QO_MUTANT == 3 ? 1 : 0), NBk);
       std::vector<float> s(static_cast<size_t>(std::max<int64_t>(nb, 1)));
-      index_scores_row(qrow.data(), kp + b * NBk * Di, head_w, Hi, Di, nb, mode, s.data());
+      index_scores_row(qrow.data(), kp + (QO_MUTANT == 15 ? 0 : b) * NBk * Di, head_w, Hi, Di, nb, mode, s.data());
       sel.assign(static_cast<size_t>(topk), -1);
       select_topk_row(s.data(), nb, topk, sel.data(), kth ? kth + 2 * r : nullptr);
       if (idx_out) std::memcpy(idx_out + r * topk, sel.data(), sizeof(int32_t) * topk);
@@ -414,7 +414,7 @@ int qo_decode(const uint16_t* q, const uint16_t* kc, const uint16_t* vc, const u
       }
       const int64_t nb = std::min(pos / blk + (QO_MUTANT == 3 ? 1 : 0), NBk);
       std::vector<float> s(static_cast<size_t>(std::max<int64_t>(nb, 1)));
-      index_scores_row(qrow.data(), kp + b * NBk * Di, head_w, Hi, Di, nb, mode, s.data());
+      index_scores_row(qrow.data(), kp + (QO_MUTANT == 15 ? 0 : b) * NBk * Di, head_w, Hi, Di, nb, mode, s.data());
       sel.assign(static_cast<size_t>(topk), -1);
       select_topk_row(s.data(), nb, topk, sel.data(), kth ? kth + 2 * r : nullptr);
       if (idx_out) std::memcpy(idx_out + r * topk, sel.data(), sizeof(int32_t) * topk);

@@ -22,6 +22,9 @@ MUTANTS = {
     10: "pooled key rotated at the block end",
     11: "bf16 rounding truncates",
     12: "YaRN ramp reversed (fast pairs interpolated, slow pairs kept)",
+    13: "log-sum-exp without the running maximum",
+    14: "indexer head weights ignored",
+    15: "every sequence scored against the first sequence's pooled keys",
 }
 
 

@@ -330,6 +330,21 @@ def test_topk_brute_force(n, k, levels):
     assert sk1 == (srt[k] if n > k else -math.inf)
 
 
+def test_each_sequence_selects_with_its_own_pooled_keys():
+    """One selection per token from the single shared key head, over the token's own sequence: in a
+    batch of two, every row's list is the brute-force top-k of the scores of that row's indexer
+    query against its own sequence's pooled keys alone (the two sequences' lists differ)."""
+    x = small_prefill(23, B=2, T=64)
+    kp = O.pool_block_keys(x["ki"])
+    k = 3
+    rows = [(b, t) for b in range(2) for t in range(64)]
+    res = O.prefill_rows(x["q"], x["k"], x["v"], x["qi"], kp, rows, topk=k)
+    for r, (b, t) in enumerate(rows):
+        s = O.index_scores(x["qi"][b, t], kp[b], t // 4)
+        assert res["idx"][r].tolist() == brute_topk(s, k), (b, t)
+    assert not np.array_equal(res["idx"][:64], res["idx"][64:])
+
+
 # ----------------------------------------------------------------------------------- attention
 def small_prefill(seed, B=1, T=45, Hq=4, Hkv=2, D=32, Hi=2, Di=16, blk=4):
     rng = np.random.default_rng(seed)
