@@ -429,7 +429,9 @@ cudaError_t launch_select_candidates(const DeviceInfo* di, const uint2* cand, co
   if (rows <= 0) return cudaSuccess;
   // lists of up to 2 * U * kSelThreads entries fit the registers; longer ones are refused (the
   // caller only plans caps that fit)
-  if (cap <= 2 * 10 * kSelThreads)
+  if (cap <= 2 * 8 * kSelThreads)   // k <= 512: no spills within the 64 registers
+    cand_select_kernel<8><<<rows, kSelThreads, 0, s>>>(cand, cnt, cap, Tq, NBk, q_pos0, b, row0, k, idx, fail);
+  else if (cap <= 2 * 10 * kSelThreads)
     cand_select_kernel<10><<<rows, kSelThreads, 0, s>>>(cand, cnt, cap, Tq, NBk, q_pos0, b, row0, k, idx, fail);
   else if (cap <= 2 * 20 * kSelThreads)
     cand_select_kernel<20><<<rows, kSelThreads, 0, s>>>(cand, cnt, cap, Tq, NBk, q_pos0, b, row0, k, idx, fail);
